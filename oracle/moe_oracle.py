@@ -1,0 +1,441 @@
+"""CPU oracle for the fused Mixture-of-Experts layer forward.
+
+TEST INFRASTRUCTURE. This module is a plain, slow, obviously-correct NumPy
+restatement of what the layer computes, in float64. It exists only to check
+the CUDA library. Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline / reference leg of ``bench.py`` may import it; the library and
+its Python binding never do, and it imports nothing from them.
+
+The layer (one forward call) computes, for every token t with hidden row x_t:
+
+  1. route:   pick the top-k experts of the router logits, softmax weights,
+              optional renormalisation, optional fused shared-expert slot;
+  2. align:   stable sort of the (token, slot) pairs by expert, each expert's
+              segment padded to the GEMM row tile ``block_m``;
+  3. GEMM1:   z = W13[e] x_t, then SwiGLU silu(gate)*up or relu2 max(z,0)^2;
+  4. GEMM2:   y = w_tj * (W2[e] a);
+  5. combine: out_t = sum_j y_tj in slot order j = 0..k'-1.
+
+Citations name the source pages by title and section:
+  [TRTLLM]  "FlashInfer TRTLLM-Gen MoE kernel optimisation: NemotronH support"
+            (sglang PR 21321)
+  [GATED]   "FlashInfer gated MoE kernel optimisation for Blackwell"
+            (flashinfer PR 4329)
+  [SHARED]  "Qwen3-Next FP8 MoE optimisation: shared-expert fusion for H200"
+            (sglang PR 26204)
+  [SWIGLU]  "[MoE] SwiGLU fusion into the MoE up-GEMM epilogue"
+            (sglang PR 32944)
+  [W4A8]    "W4A8 grouped GEMM optimisation for GLM-5.2 MoE on H200"
+            (sglang PR 38220)
+
+Where the pages leave a step open, the reading taken is stated at the
+function. Every function here is pinned by tests in ``tests/`` against
+brute force, closed forms or library routines (none is "parity unpinned").
+"""
+from __future__ import annotations
+
+import math
+from typing import Dict, Optional, Sequence
+
+import numpy as np
+
+E4M3_MAX = 448.0
+
+# --------------------------------------------------------------------------
+# Number formats
+# --------------------------------------------------------------------------
+
+
+def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    """Decode bf16 bit patterns (uint16) to float64 exactly.
+
+    A bf16 value is the upper 16 bits of an IEEE binary32 value.
+    """
+    b = np.ascontiguousarray(bits).astype(np.uint32) << 16
+    return b.view(np.float32).astype(np.float64)
+
+
+def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
+    b = np.ascontiguousarray(bits).astype(np.uint32) << 16
+    return b.view(np.float32)
+
+
+def e4m3_encode(x: np.ndarray) -> np.ndarray:
+    """Encode float32 values as FP8 E4M3 (the OCP "fn" variant) codes.
+
+    Format: 1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits; no
+    infinities; the largest finite magnitude is 448 (exponent field 15,
+    mantissa 6); exponent field 0 holds subnormals m * 2^-9.
+    Rounding is to nearest, ties to even; magnitudes beyond 448 saturate to
+    448 ("satfinite"). Inputs must be finite. The sign of zero is kept.
+    Used for the FP8 W8A8 128x128 block-scale configuration of [SHARED],
+    section 1 (dtype=fp8_w8a8, block_shape=[128, 128]).
+    """
+    x = np.asarray(x, dtype=np.float32)
+    a = np.abs(x).astype(np.float64)
+    sign = (np.signbit(x)).astype(np.uint8) << 7
+    # quantum (spacing of representable values) at the magnitude of a
+    _, ex = np.frexp(a)                     # a = m * 2^ex, m in [0.5, 1)
+    e_unb = ex.astype(np.int64) - 1         # a in [2^e_unb, 2^(e_unb+1))
+    e_unb = np.maximum(e_unb, -6)           # below 2^-6: subnormal spacing 2^-9
+    quantum = np.ldexp(1.0, (e_unb - 3).astype(np.int32))
+    r = np.rint(a / quantum) * quantum      # exact in float64; rint is ties-to-even
+    r = np.minimum(r, E4M3_MAX)
+    # r -> bits
+    codes = np.zeros(x.shape, dtype=np.uint8)
+    nz = r > 0
+    _, ex2 = np.frexp(r)
+    e2 = ex2.astype(np.int64) - 1
+    normal = nz & (e2 >= -6)
+    sub = nz & (e2 < -6)
+    mant_n = np.where(normal, r / np.ldexp(1.0, e2.astype(np.int32)) - 1.0, 0.0) * 8.0
+    exp_field = np.where(normal, e2 + 7, 0)
+    codes = np.where(normal, (exp_field.astype(np.uint8) << 3) | mant_n.astype(np.uint8), codes)
+    codes = np.where(sub, (r / 2.0 ** -9).astype(np.uint8), codes)
+    return (codes | sign).astype(np.uint8)
+
+
+def e4m3_decode(codes: np.ndarray) -> np.ndarray:
+    """Decode FP8 E4M3 codes to float64 (code 0x7F/0xFF, NaN, never occurs here)."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    s = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = c & 0x7
+    val = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * np.ldexp(1.0, (e - 7).astype(np.int32)))
+    return s * val
+
+
+def quant_groups_1x128(x: np.ndarray):
+    """Dynamic per-row, per-128-column quantisation to E4M3.
+
+    For each row and each group of 128 consecutive columns:
+    scale = amax / 448 (IEEE fp32 division), q = e4m3(x / scale) with the
+    fp32 division rounded to nearest. An all-zero group takes scale 1 (the
+    pages do not say; with scale 1 every code is 0 and dequantisation is
+    exact). Both the division and the encoding run in fp32, the precision the
+    kernel uses, so the codes are a bit-exact reference.
+    Returns (codes uint8 [R, C], scales float32 [R, C/128]).
+    """
+    x = np.asarray(x, dtype=np.float32)
+    R, C = x.shape
+    assert C % 128 == 0
+    g = x.reshape(R, C // 128, 128)
+    amax = np.abs(g).max(axis=2)
+    scale = (amax / np.float32(E4M3_MAX)).astype(np.float32)
+    scale = np.where(amax == 0, np.float32(1.0), scale).astype(np.float32)
+    q = e4m3_encode((g / scale[:, :, None]).astype(np.float32))
+    return q.reshape(R, C), scale
+
+
+def quant_blocks_128x128(w: np.ndarray):
+    """Static per-128x128-block quantisation of a weight matrix to E4M3.
+
+    ``w`` is [R, C] (fp32 values of the bf16 masters), R and C multiples of
+    128. scale = amax(block) / 448 in fp32, q = e4m3(w / scale); an all-zero
+    block takes scale 1. Returns (codes uint8 [R, C], scales float32
+    [R/128, C/128]).
+    """
+    w = np.asarray(w, dtype=np.float32)
+    R, C = w.shape
+    assert R % 128 == 0 and C % 128 == 0
+    b = w.reshape(R // 128, 128, C // 128, 128)
+    amax = np.abs(b).max(axis=(1, 3))
+    scale = (amax / np.float32(E4M3_MAX)).astype(np.float32)
+    scale = np.where(amax == 0, np.float32(1.0), scale).astype(np.float32)
+    q = e4m3_encode((b / scale[:, None, :, None]).astype(np.float32))
+    return q.reshape(R, C), scale
+
+
+def dequant_groups_1x128(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    return e4m3_decode(codes) * np.repeat(scales.astype(np.float64), 128, axis=1)
+
+
+def dequant_blocks_128x128(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    s = np.repeat(np.repeat(scales.astype(np.float64), 128, axis=0), 128, axis=1)
+    return e4m3_decode(codes) * s
+
+
+# --------------------------------------------------------------------------
+# Step 1: routing
+# --------------------------------------------------------------------------
+
+
+def route(logits: np.ndarray, topk: int, renormalize: bool, num_shared: int = 0):
+    """Top-k expert selection with softmax routing weights.
+
+    [TRTLLM] section 1 gives the fused op's arguments ``topk: int`` and
+    ``renormalize: bool`` but not the formula. Reading taken (the plainest
+    one consistent with an optional renormalisation and no bias or expert
+    grouping on the page):
+      * the k experts with the largest raw fp32 logits are selected, ordered
+        by logit descending, ties broken towards the lower expert index;
+      * p_e = softmax over all routed experts, in float64;
+      * w_j = p_{id_j}, or p_{id_j} / sum_j' p_{id_j'} when renormalize.
+    [SHARED] section 2 fuses a shared expert as an extra expert slot that
+    every token selects: with ``num_shared`` = 1 the slot id is E (the
+    routed expert count) with weight exactly 1, placed after the k routed
+    slots and never renormalised.
+    Returns ids int32 [T, k + num_shared] and weights float32 (same shape).
+    """
+    logits = np.asarray(logits, dtype=np.float32)
+    T, E = logits.shape
+    kk = topk + num_shared
+    ids = np.empty((T, kk), dtype=np.int32)
+    w = np.empty((T, kk), dtype=np.float32)
+    if T == 0:
+        return ids, w
+    # a stable sort of the negated logits keeps equal logits in index order
+    order = np.argsort(-logits, axis=1, kind="stable")[:, :topk]
+    l64 = logits.astype(np.float64)
+    m = l64.max(axis=1, keepdims=True)
+    ex = np.exp(l64 - m)
+    p = ex / ex.sum(axis=1, keepdims=True)
+    sel = np.take_along_axis(p, order, axis=1)
+    if renormalize:
+        sel = sel / sel.sum(axis=1, keepdims=True)
+    ids[:, :topk] = order
+    w[:, :topk] = sel
+    if num_shared:
+        ids[:, topk:] = E
+        w[:, topk:] = 1.0
+    return ids, w
+
+
+# --------------------------------------------------------------------------
+# Step 2: align / permute
+# --------------------------------------------------------------------------
+
+
+def align(ids: np.ndarray, num_experts: int, block_m: int) -> Dict[str, np.ndarray]:
+    """Sort (token, slot) pairs by expert and pad each expert to ``block_m``.
+
+    Pair p = t * k' + j. The grouped GEMM contract of [W4A8] section 1
+    (``expert_offsets``, ``problem_sizes``) gives each expert a contiguous
+    row range. Reading taken: the expert's segment lists its pairs in
+    ascending pair order (stable), followed by the sentinel P (= number of
+    pairs) up to the next multiple of ``block_m``; an expert with no pairs
+    gets no rows.
+      expert_offsets[e+1] = expert_offsets[e] + round_up(count_e, block_m)
+      block_expert[b]     = expert owning rows [b*block_m, (b+1)*block_m)
+      pair_to_row[p]      = row of pair p in the sorted order
+    """
+    flat = np.asarray(ids, dtype=np.int64).reshape(-1)
+    P = flat.size
+    counts = np.bincount(flat, minlength=num_experts)[:num_experts]
+    padded = (counts + block_m - 1) // block_m * block_m
+    offsets = np.zeros(num_experts + 1, dtype=np.int64)
+    offsets[1:] = np.cumsum(padded)
+    P_pad = int(offsets[-1])
+    sorted_pair_ids = np.full(P_pad, P, dtype=np.int32)
+    pair_to_row = np.empty(P, dtype=np.int32)
+    block_expert = np.empty(P_pad // block_m, dtype=np.int32)
+    for e in range(num_experts):
+        pairs = np.nonzero(flat == e)[0]
+        rows = offsets[e] + np.arange(pairs.size)
+        sorted_pair_ids[rows] = pairs
+        pair_to_row[pairs] = rows
+        block_expert[offsets[e] // block_m: offsets[e + 1] // block_m] = e
+    return {
+        "sorted_pair_ids": sorted_pair_ids,
+        "expert_offsets": offsets.astype(np.int32),
+        "block_expert": block_expert,
+        "pair_to_row": pair_to_row,
+        "P_pad": np.int64(P_pad),
+    }
+
+
+# --------------------------------------------------------------------------
+# Load-time weight preparation
+# --------------------------------------------------------------------------
+
+
+def padded_intermediate(I: int, gated: bool) -> int:
+    """Intermediate size after alignment padding.
+
+    [TRTLLM] section 2 (``_align_fp8_moe_weights`` and its caller): the
+    intermediate size is rounded up to a multiple of 16 for gated
+    activations and 128 for non-gated ones, and left unchanged when it is
+    already aligned.
+    """
+    a = 16 if gated else 128
+    return (I + a - 1) // a * a
+
+
+def pad_weights(w13: np.ndarray, w2: np.ndarray, I: int, gated: bool):
+    """Zero-pad w13 [E, up_mult*I, H] and w2 [E, H, I] to the padded I.
+
+    [TRTLLM] section 2: the gate/up block becomes up_mult * I_pad rows (up_mult
+    2 gated, 1 non-gated) with the original rows copied to the front and
+    zeros after, and w2's last axis is zero-padded to I_pad. Note that the
+    page copies the whole original w13 block to the front, so for a gated
+    layer the up rows move only if I changes; this oracle keeps gate rows
+    [0, I) and up rows [I_pad, I_pad + I) so that the padded matrix still
+    reads as [Gate, Up] with the zero rows at the end of each half.
+    """
+    I_pad = padded_intermediate(I, gated)
+    E, R, H = w13.shape
+    if I_pad == I:
+        return w13, w2, I
+    if gated:
+        out13 = np.zeros((E, 2 * I_pad, H), dtype=w13.dtype)
+        out13[:, :I] = w13[:, :I]
+        out13[:, I_pad:I_pad + I] = w13[:, I:2 * I]
+    else:
+        out13 = np.zeros((E, I_pad, H), dtype=w13.dtype)
+        out13[:, :I] = w13
+    out2 = np.zeros((E, w2.shape[1], I_pad), dtype=w2.dtype)
+    out2[:, :, :I] = w2
+    return out13, out2, I_pad
+
+
+def interleave_gate_up(w13: np.ndarray, I: int) -> np.ndarray:
+    """Row-interleave gate and up: [gate0, up0, gate1, up1, ...].
+
+    [SWIGLU] section 3 (load-time interleave) so that the gate and up rows of
+    one intermediate index sit in the same GEMM tile; [TRTLLM] section 2
+    applies the same idea (``reorder_rows_for_gated_act_gemm``) to gated
+    layers only.
+    """
+    E, R, H = w13.shape
+    assert R == 2 * I
+    out = np.empty_like(w13)
+    out[:, 0::2] = w13[:, :I]
+    out[:, 1::2] = w13[:, I:]
+    return out
+
+
+# --------------------------------------------------------------------------
+# Step 3-5: expert FFNs and combine
+# --------------------------------------------------------------------------
+
+
+def silu(x: np.ndarray) -> np.ndarray:
+    """silu(x) = x / (1 + e^-x), the gate activation of SwiGLU ([SWIGLU] section 1)."""
+    with np.errstate(over="ignore"):
+        return x / (1.0 + np.exp(-x))
+
+
+def relu2(x: np.ndarray) -> np.ndarray:
+    """relu2(x) = max(x, 0)^2, the non-gated activation of [TRTLLM] section 1."""
+    r = np.maximum(x, 0.0)
+    return r * r
+
+
+def activation_fn(z: np.ndarray, activation: str, I: int) -> np.ndarray:
+    """Apply the layer activation to GEMM1 rows z [n, N1] (gate-first layout).
+
+    SwiGLU: a = silu(z[:, :I]) * z[:, I:2I] ([SWIGLU] section 1,
+    ``silu(gate) * up``; [GATED] section 1, activation(gate) * up).
+    relu2: a = relu2(z) over the I columns.
+    """
+    if activation == "swiglu":
+        return silu(z[:, :I]) * z[:, I:2 * I]
+    if activation == "relu2":
+        return relu2(z[:, :I])
+    raise ValueError(activation)
+
+
+def moe_forward(hidden_bits: np.ndarray, logits: np.ndarray, w13_bits, w2_bits, *,
+                topk: int, renormalize: bool, activation: str, num_shared: int = 0,
+                tokens: Optional[Sequence[int]] = None, return_parts: bool = False):
+    """bf16 layer forward in float64.
+
+    ``hidden_bits`` uint16 [T, H] (bf16), ``logits`` float32 [T, E_r],
+    ``w13_bits`` uint16 [E, N1, H] and ``w2_bits`` uint16 [E, H, I] in the
+    checkpoint layout (gate rows first). No intermediate rounding: GEMM
+    products and sums are float64, the activation is applied to the exact
+    GEMM1 result, the routing weight multiplies the exact GEMM2 result and
+    the k' slot contributions are summed in slot order j = 0..k'-1.
+    ``tokens`` restricts the computation to a subset of tokens (routing is
+    per token, so the subset's outputs equal the full call's rows).
+    Returns out float64 [len(tokens) or T, H].
+    """
+    logits = np.asarray(logits, dtype=np.float32)
+    if tokens is not None:
+        tokens = np.asarray(tokens, dtype=np.int64)
+        hidden_bits = np.asarray(hidden_bits)[tokens]
+        logits = logits[tokens]
+    x = bf16_bits_to_f64(hidden_bits)
+    ids, w = route(logits, topk, renormalize, num_shared)
+    T, kk = ids.shape
+    H = x.shape[1]
+    I = w2_bits.shape[2]
+    y = np.zeros((T, kk, H), dtype=np.float64)
+    for e in np.unique(ids):
+        t_idx, j_idx = np.nonzero(ids == e)
+        W13 = bf16_bits_to_f64(np.asarray(w13_bits[e]))
+        W2 = bf16_bits_to_f64(np.asarray(w2_bits[e]))
+        z = x[t_idx] @ W13.T
+        a = activation_fn(z, activation, I)
+        y[t_idx, j_idx] = w[t_idx, j_idx].astype(np.float64)[:, None] * (a @ W2.T)
+    out = np.zeros((T, H), dtype=np.float64)
+    for j in range(kk):
+        out += y[:, j]
+    if return_parts:
+        return out, {"ids": ids, "w": w}
+    return out
+
+
+def moe_forward_fp8(hidden_bits: np.ndarray, logits: np.ndarray, w13_q, w13_s, w2_q, w2_s, *,
+                    topk: int, renormalize: bool, activation: str, num_shared: int = 0,
+                    tokens: Optional[Sequence[int]] = None):
+    """FP8 E4M3 W8A8 layer forward with 128x128 weight blocks, in float64.
+
+    [SHARED] section 1 names the configuration (fp8_w8a8, block_shape
+    [128, 128]); [TRTLLM] section 1 the fused op that takes per-block weight
+    scales. Reading taken (the pages print no formula):
+      * weights: e4m3 codes with one fp32 scale per 128x128 block of the
+        checkpoint-layout matrices w13 [E, N1, H] and w2 [E, H, I];
+      * activations: the bf16 hidden rows are quantised per token per 128
+        columns (``quant_groups_1x128``) before GEMM1, and the GEMM1
+        activation output, held in fp32, is quantised the same way before
+        GEMM2 (W8A8 means both GEMM inputs are 8-bit);
+      * every product uses the exactly dequantised values q * s in float64.
+    ``w13_q``/``w2_q`` are uint8 codes, ``w13_s`` [E, N1/128, H/128] and
+    ``w2_s`` [E, H/128, I/128] float32 scales.
+    """
+    logits = np.asarray(logits, dtype=np.float32)
+    if tokens is not None:
+        tokens = np.asarray(tokens, dtype=np.int64)
+        hidden_bits = np.asarray(hidden_bits)[tokens]
+        logits = logits[tokens]
+    xq, xs = quant_groups_1x128(bf16_bits_to_f32(hidden_bits))
+    x = dequant_groups_1x128(xq, xs)
+    ids, w = route(logits, topk, renormalize, num_shared)
+    T, kk = ids.shape
+    H = x.shape[1]
+    I = w2_q.shape[2]
+    y = np.zeros((T, kk, H), dtype=np.float64)
+    for e in np.unique(ids):
+        t_idx, j_idx = np.nonzero(ids == e)
+        W13 = dequant_blocks_128x128(np.asarray(w13_q[e]), np.asarray(w13_s[e]))
+        W2 = dequant_blocks_128x128(np.asarray(w2_q[e]), np.asarray(w2_s[e]))
+        a = activation_fn(x[t_idx] @ W13.T, activation, I)
+        aq, as_ = quant_groups_1x128(a.astype(np.float32))
+        ad = dequant_groups_1x128(aq, as_)
+        y[t_idx, j_idx] = w[t_idx, j_idx].astype(np.float64)[:, None] * (ad @ W2.T)
+    out = np.zeros((T, H), dtype=np.float64)
+    for j in range(kk):
+        out += y[:, j]
+    return out
+
+
+def quantize_weights_fp8(w13_bits, w2_bits):
+    """Quantise bf16 master weights per 128x128 block (``quant_blocks_128x128``).
+
+    Returns (w13_q, w13_s, w2_q, w2_s) in the checkpoint layout.
+    """
+    E = w13_bits.shape[0]
+    w13_q = np.empty(w13_bits.shape, dtype=np.uint8)
+    w2_q = np.empty(w2_bits.shape, dtype=np.uint8)
+    w13_s = np.empty((E, w13_bits.shape[1] // 128, w13_bits.shape[2] // 128), dtype=np.float32)
+    w2_s = np.empty((E, w2_bits.shape[1] // 128, w2_bits.shape[2] // 128), dtype=np.float32)
+    for e in range(E):
+        w13_q[e], w13_s[e] = quant_blocks_128x128(bf16_bits_to_f32(np.asarray(w13_bits[e])))
+        w2_q[e], w2_s[e] = quant_blocks_128x128(bf16_bits_to_f32(np.asarray(w2_bits[e])))
+    return w13_q, w13_s, w2_q, w2_s
+
+
+def rms(x: np.ndarray) -> float:
+    x = np.asarray(x, dtype=np.float64)
+    return math.sqrt(float(np.mean(x * x))) if x.size else 0.0

@@ -1,0 +1,457 @@
+"""Pins for the CPU oracle: brute force, closed forms, library routines, invariants.
+
+Each test checks the oracle against something other than itself, chosen so
+that a plausible mistake (dropped term, wrong sign or index, transposed
+operand, wrong tie-break or padding) fails at least one of them. The last
+tests plant such mistakes in copies of oracle functions and check that the
+pins catch them.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import moe_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rows(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return [ln.split() for ln in f if ln.strip() and not ln.startswith("#")]
+
+
+def _bf16_bits(x: torch.Tensor) -> np.ndarray:
+    return x.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+# --------------------------------------------------------------------------
+# routing
+# --------------------------------------------------------------------------
+
+
+def _route_brute(logits, topk, renorm, num_shared=0):
+    """Per-token brute force: Python sort on (-logit, index), math.exp softmax."""
+    T, E = logits.shape
+    ids, ws = [], []
+    for t in range(T):
+        row = [float(v) for v in logits[t]]
+        sel = sorted(range(E), key=lambda e: (-row[e], e))[:topk]
+        m = max(row)
+        den = sum(math.exp(v - m) for v in row)
+        p = [math.exp(row[e] - m) / den for e in sel]
+        if renorm:
+            s = sum(p)
+            p = [v / s for v in p]
+        ids.append(sel + [E] * num_shared)
+        ws.append(p + [1.0] * num_shared)
+    return np.array(ids, dtype=np.int64).reshape(T, topk + num_shared), np.array(ws).reshape(T, -1)
+
+
+@pytest.mark.parametrize("E,topk,renorm,shared", [(8, 2, True, 0), (16, 5, False, 0),
+                                                  (33, 7, True, 1), (5, 5, False, 0)])
+def test_route_matches_brute_force(E, topk, renorm, shared):
+    rng = np.random.default_rng(E * 100 + topk)
+    logits = rng.standard_normal((40, E)).astype(np.float32)
+    # plant exact ties: copy some entries onto others
+    logits[3, 1] = logits[3, 0]
+    logits[7, :] = 0.25
+    ids, w = O.route(logits, topk, renorm, shared)
+    bi, bw = _route_brute(logits, topk, renorm, shared)
+    np.testing.assert_array_equal(ids, bi)
+    np.testing.assert_allclose(w, bw, rtol=2e-7, atol=0)
+
+
+def test_route_two_expert_closed_form():
+    # k = 1 of 2 experts, no renormalisation: w = sigmoid(l_sel - l_other)
+    l = np.array([[1.5, -0.25], [-2.0, 0.75]], dtype=np.float32)
+    ids, w = O.route(l, 1, False)
+    assert ids[:, 0].tolist() == [0, 1]
+    exp0 = 1.0 / (1.0 + math.exp(-(1.5 + 0.25)))
+    exp1 = 1.0 / (1.0 + math.exp(-(0.75 + 2.0)))
+    np.testing.assert_allclose(w[:, 0], [exp0, exp1], rtol=1e-7)
+    # renormalised single choice is exactly 1
+    _, wr = O.route(l, 1, True)
+    assert np.all(wr == 1.0)
+
+
+def test_route_ties_and_one_hot():
+    E, k = 12, 4
+    ids, w = O.route(np.zeros((3, E), np.float32), k, False)
+    assert ids.tolist() == [[0, 1, 2, 3]] * 3            # lower index wins ties
+    np.testing.assert_allclose(w, 1.0 / E, rtol=1e-7)
+    _, wr = O.route(np.zeros((3, E), np.float32), k, True)
+    np.testing.assert_allclose(wr, 1.0 / k, rtol=1e-7)
+    oh = np.full((2, E), -50.0, np.float32)
+    oh[0, 7] = 5.0
+    oh[1, 11] = 5.0
+    ids, _ = O.route(oh, 1, False)
+    assert ids[:, 0].tolist() == [7, 11]
+
+
+def test_route_renormalized_weights_sum_to_one_and_shared_slot():
+    rng = np.random.default_rng(3)
+    l = rng.standard_normal((50, 64)).astype(np.float32)
+    ids, w = O.route(l, 10, True, num_shared=1)
+    np.testing.assert_allclose(w[:, :10].astype(np.float64).sum(1), 1.0, atol=1e-6)
+    assert np.all(ids[:, 10] == 64) and np.all(w[:, 10] == 1.0)
+    # weights are non-increasing along the slots (ordered by logit)
+    assert np.all(np.diff(w[:, :10], axis=1) <= 0)
+
+
+# --------------------------------------------------------------------------
+# align
+# --------------------------------------------------------------------------
+
+
+def _align_brute(ids, E, bm):
+    flat = [int(v) for v in np.asarray(ids).reshape(-1)]
+    P = len(flat)
+    order = sorted(range(P), key=lambda p: (flat[p], p))
+    sorted_ids, offsets, block_expert = [], [0], []
+    pos = 0
+    for e in range(E):
+        seg = [p for p in order if flat[p] == e]
+        n = (len(seg) + bm - 1) // bm * bm
+        sorted_ids += seg + [P] * (n - len(seg))
+        block_expert += [e] * (n // bm)
+        pos += n
+        offsets.append(pos)
+    p2r = [0] * P
+    for r, p in enumerate(sorted_ids):
+        if p < P:
+            p2r[p] = r
+    return sorted_ids, offsets, block_expert, p2r
+
+
+@pytest.mark.parametrize("T,E,k,bm", [(16, 8, 2, 128), (37, 5, 3, 4), (1, 9, 9, 16), (64, 40, 6, 8)])
+def test_align_matches_brute_force(T, E, k, bm):
+    rng = np.random.default_rng(T + E)
+    l = rng.standard_normal((T, E)).astype(np.float32)
+    l[:, 0] += 2.0  # expert 0 overloaded, some experts empty
+    ids, _ = O.route(l, k, True)
+    a = O.align(ids, E, bm)
+    s, off, be, p2r = _align_brute(ids, E, bm)
+    assert a["sorted_pair_ids"].tolist() == s
+    assert a["expert_offsets"].tolist() == off
+    assert a["block_expert"].tolist() == be
+    assert a["pair_to_row"].tolist() == p2r
+    assert int(a["P_pad"]) == off[-1] and off[-1] % bm == 0
+
+
+def test_align_empty_and_single_expert():
+    a = O.align(np.zeros((0, 2), np.int32), 4, 16)
+    assert a["expert_offsets"].tolist() == [0, 0, 0, 0, 0] and a["sorted_pair_ids"].size == 0
+    ids = np.full((10, 1), 2, np.int32)
+    a = O.align(ids, 4, 8)
+    assert a["expert_offsets"].tolist() == [0, 0, 0, 16, 16]
+    assert a["sorted_pair_ids"].tolist() == list(range(10)) + [10] * 6
+    assert a["block_expert"].tolist() == [2, 2]
+
+
+# --------------------------------------------------------------------------
+# activations and weight preparation (golden fixtures from the pages / closed forms)
+# --------------------------------------------------------------------------
+
+
+def test_activation_closed_forms():
+    for fn, x, v in _rows("activation_points.txt"):
+        f = O.silu if fn == "silu" else O.relu2
+        got = float(f(np.array([float(x)]))[0])
+        assert got == pytest.approx(float(v), rel=1e-15, abs=1e-300), (fn, x)
+    # limits: silu(x) -> x for large x, -> 0 for very negative x, no NaN at overflow
+    assert float(O.silu(np.array([1000.0]))[0]) == 1000.0
+    assert float(O.silu(np.array([-1000.0]))[0]) == 0.0
+
+
+def test_padding_rules_from_page():
+    for i_in, gated, i_pad in _rows("padding_rules.txt"):
+        assert O.padded_intermediate(int(i_in), gated == "1") == int(i_pad)
+
+
+def test_interleave_order_from_page():
+    rows = _rows("interleave_order.txt")
+    I = int(rows[0][1])
+    want = rows[1]
+    labels = [f"g{j}" for j in range(I)] + [f"u{j}" for j in range(I)]
+    w = np.arange(2 * I, dtype=np.float64).reshape(1, 2 * I, 1)
+    got = O.interleave_gate_up(w, I)[0, :, 0].astype(int)
+    assert [labels[i] for i in got] == want
+
+
+def test_padding_leaves_layer_unchanged():
+    # zero-padding the intermediate size adds exact zeros: silu(0)*0 = relu2(0) = 0
+    rng = np.random.default_rng(5)
+    for act, I in (("swiglu", 40), ("relu2", 100)):
+        gated = act == "swiglu"
+        T, H, E, k = 6, 128, 3, 2
+        x = _bf16_bits(torch.from_numpy(rng.standard_normal((T, H)).astype(np.float32)))
+        l = rng.standard_normal((T, E)).astype(np.float32)
+        w13 = _bf16_bits(torch.from_numpy(0.1 * rng.standard_normal((E, (2 if gated else 1) * I, H)).astype(np.float32)))
+        w2 = _bf16_bits(torch.from_numpy(0.1 * rng.standard_normal((E, H, I)).astype(np.float32)))
+        p13, p2, I_pad = O.pad_weights(w13, w2, I, gated)
+        assert I_pad == O.padded_intermediate(I, gated) and I_pad > I
+        a = O.moe_forward(x, l, w13, w2, topk=k, renormalize=True, activation=act)
+        b = O.moe_forward(x, l, p13, p2, topk=k, renormalize=True, activation=act)
+        np.testing.assert_allclose(b, a, rtol=1e-12, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# whole layer: dense-FFN invariant and scalar brute force
+# --------------------------------------------------------------------------
+
+
+def _dense_layer(x, logits, w13, w2, topk, renorm, act, num_shared=0):
+    """out_t = sum_e g_te * FFN_e(x_t) with every expert evaluated densely.
+
+    The gate vector g is zero outside the brute-force top-k; FFN_e uses
+    einsum over all experts at once (a different route through the math
+    than the oracle's per-expert grouping).
+    """
+    ids, wts = _route_brute(logits, topk, renorm, num_shared)
+    wts = wts.astype(np.float32).astype(np.float64)   # routing weights are stored as fp32
+    T = x.shape[0]
+    E = w13.shape[0]
+    I = w2.shape[2]
+    g = np.zeros((T, E))
+    for t in range(T):
+        for j in range(ids.shape[1]):
+            g[t, ids[t, j]] += wts[t, j]
+    z = np.einsum("th,enh->ten", x, w13)
+    if act == "swiglu":
+        a = z[:, :, :I] / (1.0 + np.exp(-z[:, :, :I])) * z[:, :, I:]
+    else:
+        a = np.maximum(z, 0.0) ** 2
+    ffn = np.einsum("tei,ehi->teh", a, w2)
+    return np.einsum("te,teh->th", g, ffn)
+
+
+@pytest.mark.parametrize("act,renorm,shared", [("swiglu", True, 0), ("relu2", False, 0), ("swiglu", True, 1)])
+def test_layer_dense_ffn_invariant(act, renorm, shared):
+    rng = np.random.default_rng(11)
+    T, H, E, k, I = 9, 64, 6, 3, 24
+    N1 = 2 * I if act == "swiglu" else I
+    x = _bf16_bits(torch.from_numpy(rng.standard_normal((T, H)).astype(np.float32)))
+    l = rng.standard_normal((T, E)).astype(np.float32)
+    Et = E + shared
+    w13 = _bf16_bits(torch.from_numpy(0.2 * rng.standard_normal((Et, N1, H)).astype(np.float32)))
+    w2 = _bf16_bits(torch.from_numpy(0.2 * rng.standard_normal((Et, H, I)).astype(np.float32)))
+    got = O.moe_forward(x, l, w13, w2, topk=k, renormalize=renorm, activation=act, num_shared=shared)
+    want = _dense_layer(O.bf16_bits_to_f64(x), l, O.bf16_bits_to_f64(w13), O.bf16_bits_to_f64(w2),
+                        k, renorm, act, shared)
+    np.testing.assert_allclose(got, want, rtol=1e-10, atol=1e-12)
+
+
+def test_layer_scalar_brute_force_tiny():
+    # pure-Python scalar loops on a 2-token, 3-expert, H=4, I=2 layer
+    rng = np.random.default_rng(2)
+    T, H, E, k, I = 2, 4, 3, 2, 2
+    x = _bf16_bits(torch.from_numpy(rng.standard_normal((T, H)).astype(np.float32)))
+    l = rng.standard_normal((T, E)).astype(np.float32)
+    w13 = _bf16_bits(torch.from_numpy(rng.standard_normal((E, 2 * I, H)).astype(np.float32)))
+    w2 = _bf16_bits(torch.from_numpy(rng.standard_normal((E, H, I)).astype(np.float32)))
+    X, W13, W2 = O.bf16_bits_to_f64(x), O.bf16_bits_to_f64(w13), O.bf16_bits_to_f64(w2)
+    ids, wts = _route_brute(l, k, True)
+    wts = wts.astype(np.float32).astype(np.float64)   # routing weights are stored as fp32
+    want = [[0.0] * H for _ in range(T)]
+    for t in range(T):
+        for j in range(k):
+            e = ids[t, j]
+            a = []
+            for n in range(I):
+                g = sum(X[t, h] * W13[e, n, h] for h in range(H))
+                u = sum(X[t, h] * W13[e, I + n, h] for h in range(H))
+                a.append(g / (1.0 + math.exp(-g)) * u)
+            for h in range(H):
+                want[t][h] += wts[t, j] * sum(a[n] * W2[e, h, n] for n in range(I))
+    got = O.moe_forward(x, l, w13, w2, topk=k, renormalize=True, activation="swiglu")
+    np.testing.assert_allclose(got, np.array(want), rtol=1e-12, atol=1e-14)
+
+
+def test_layer_subset_of_tokens_equals_full_rows():
+    rng = np.random.default_rng(8)
+    T, H, E, k, I = 12, 128, 5, 2, 16
+    x = _bf16_bits(torch.from_numpy(rng.standard_normal((T, H)).astype(np.float32)))
+    l = rng.standard_normal((T, E)).astype(np.float32)
+    w13 = _bf16_bits(torch.from_numpy(0.1 * rng.standard_normal((E, 2 * I, H)).astype(np.float32)))
+    w2 = _bf16_bits(torch.from_numpy(0.1 * rng.standard_normal((E, H, I)).astype(np.float32)))
+    full = O.moe_forward(x, l, w13, w2, topk=k, renormalize=True, activation="swiglu")
+    sub = O.moe_forward(x, l, w13, w2, topk=k, renormalize=True, activation="swiglu", tokens=[3, 0, 11])
+    np.testing.assert_allclose(sub, full[[3, 0, 11]], rtol=1e-13, atol=0)
+
+
+# --------------------------------------------------------------------------
+# FP8 E4M3 codec and quantisers (library routine: torch.float8_e4m3fn casts)
+# --------------------------------------------------------------------------
+
+
+def test_e4m3_golden_points():
+    for v, code in _rows("e4m3_points.txt"):
+        x = np.array([float(v)], dtype=np.float32)
+        assert int(O.e4m3_encode(x)[0]) == int(code, 16), v
+
+
+def test_e4m3_encode_matches_torch_cast_on_all_bf16_values():
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    x = O.bf16_bits_to_f32(bits)
+    keep = np.isfinite(x) & (np.abs(x) <= 448.0)
+    x = x[keep]
+    want = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    np.testing.assert_array_equal(O.e4m3_encode(x), want)
+
+
+def test_e4m3_encode_matches_torch_cast_on_random_and_midpoints():
+    rng = np.random.default_rng(1)
+    x = (rng.standard_normal(200000) * rng.choice([1e-3, 0.1, 1.0, 30.0, 200.0], 200000)).astype(np.float32)
+    x = np.clip(x, -448, 448)
+    # exact midpoints between neighbouring codes (ties-to-even cases)
+    vals = O.e4m3_decode(np.arange(0, 0x7E, dtype=np.uint8))
+    mids = ((vals[1:] + vals[:-1]) / 2).astype(np.float32)
+    x = np.concatenate([x, mids, -mids])
+    want = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    np.testing.assert_array_equal(O.e4m3_encode(x), want)
+
+
+def test_e4m3_decode_roundtrip_and_monotone():
+    codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], dtype=np.uint8)
+    v = O.e4m3_decode(codes)
+    want = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    np.testing.assert_array_equal(v, want)
+    np.testing.assert_array_equal(O.e4m3_encode(v.astype(np.float32)), codes)
+    pos = O.e4m3_decode(np.arange(0, 0x7F, dtype=np.uint8))
+    assert np.all(np.diff(pos) > 0) and pos[-1] == 448.0
+
+
+def test_e4m3_saturates():
+    x = np.array([449.0, 463.9, 464.0, 500.0, 1e30, -1e30], dtype=np.float32)
+    assert O.e4m3_encode(x).tolist() == [0x7E] * 4 + [0x7E, 0xFE]
+
+
+def test_quant_groups_definition():
+    rng = np.random.default_rng(4)
+    x = rng.standard_normal((3, 256)).astype(np.float32)
+    x[1, 128:] = 0.0                      # all-zero group -> scale 1, codes 0
+    q, s = O.quant_groups_1x128(x)
+    assert s.dtype == np.float32 and s.shape == (3, 2)
+    assert s[1, 1] == 1.0 and np.all(q[1, 128:] == 0)
+    for r in range(3):
+        for g in range(2):
+            blk = x[r, g * 128:(g + 1) * 128]
+            amax = np.float32(np.abs(blk).max())
+            if amax == 0:
+                continue
+            sc = np.float32(amax / np.float32(448.0))
+            assert s[r, g] == sc
+            want = torch.from_numpy((blk / sc).astype(np.float32)).to(torch.float8_e4m3fn)
+            np.testing.assert_array_equal(q[r, g * 128:(g + 1) * 128], want.view(torch.uint8).numpy())
+    # the group's largest magnitude maps to +-448 (code 0x7E / 0xFE)
+    i = int(np.argmax(np.abs(x[0, :128])))
+    assert (q[0, i] & 0x7F) == 0x7E
+    # dequantisation error is within half an e4m3 step (relative 2^-4) per element
+    d = O.dequant_groups_1x128(q, s)
+    assert np.all(np.abs(d - x) <= np.abs(x) * 2.0 ** -4 + np.repeat(s, 128, 1) * 2.0 ** -10)
+
+
+def test_quant_blocks_definition():
+    rng = np.random.default_rng(6)
+    w = (0.02 * rng.standard_normal((256, 384))).astype(np.float32)
+    q, s = O.quant_blocks_128x128(w)
+    assert s.shape == (2, 3)
+    for bi in range(2):
+        for bj in range(3):
+            blk = w[bi * 128:(bi + 1) * 128, bj * 128:(bj + 1) * 128]
+            sc = np.float32(np.float32(np.abs(blk).max()) / np.float32(448.0))
+            assert s[bi, bj] == sc
+            want = torch.from_numpy((blk / sc).astype(np.float32)).to(torch.float8_e4m3fn)
+            np.testing.assert_array_equal(q[bi * 128:(bi + 1) * 128, bj * 128:(bj + 1) * 128],
+                                          want.view(torch.uint8).numpy())
+
+
+def test_fp8_layer_equals_bf16_layer_on_dequantised_inputs():
+    # moe_forward_fp8 == dense invariant evaluated on the dequantised operands
+    rng = np.random.default_rng(9)
+    T, H, E, k, I = 5, 256, 3, 2, 128
+    x = _bf16_bits(torch.from_numpy(rng.standard_normal((T, H)).astype(np.float32)))
+    l = rng.standard_normal((T, E)).astype(np.float32)
+    w13 = _bf16_bits(torch.from_numpy(0.02 * rng.standard_normal((E, 2 * I, H)).astype(np.float32)))
+    w2 = _bf16_bits(torch.from_numpy(0.02 * rng.standard_normal((E, H, I)).astype(np.float32)))
+    q13, s13, q2, s2 = O.quantize_weights_fp8(w13, w2)
+    got = O.moe_forward_fp8(x, l, q13, s13, q2, s2, topk=k, renormalize=True, activation="swiglu")
+    # independent restatement: dequantise with torch casts, dense evaluation
+    X = O.bf16_bits_to_f32(x)
+    xs = np.abs(X.reshape(T, 2, 128)).max(2) / np.float32(448)
+    Xq = torch.from_numpy((X.reshape(T, 2, 128) / xs[:, :, None]).astype(np.float32)).to(torch.float8_e4m3fn)
+    Xd = (Xq.to(torch.float64).numpy() * xs[:, :, None]).reshape(T, H)
+    W13d = np.stack([np.kron(s13[e].astype(np.float64), np.ones((128, 128))) *
+                     torch.from_numpy(q13[e]).view(torch.float8_e4m3fn).to(torch.float64).numpy() for e in range(E)])
+    W2d = np.stack([np.kron(s2[e].astype(np.float64), np.ones((128, 128))) *
+                    torch.from_numpy(q2[e]).view(torch.float8_e4m3fn).to(torch.float64).numpy() for e in range(E)])
+    ids, wts = _route_brute(l, k, True)
+    wts = wts.astype(np.float32).astype(np.float64)
+    want = np.zeros((T, H))
+    for t in range(T):
+        for j in range(k):
+            e = ids[t, j]
+            z = W13d[e] @ Xd[t]
+            a = (z[:I] / (1 + np.exp(-z[:I])) * z[I:]).astype(np.float32)
+            asc = np.float32(np.abs(a).max() / np.float32(448))
+            aq = torch.from_numpy((a / asc).astype(np.float32)).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+            want[t] += wts[t, j] * (W2d[e] @ (aq * asc))
+    np.testing.assert_allclose(got, want, rtol=1e-9, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# planted mistakes: each mutated oracle must fail a pin above
+# --------------------------------------------------------------------------
+
+
+def _tiny_layer_inputs(act):
+    rng = np.random.default_rng(21)
+    T, H, E, k, I = 7, 32, 5, 2, 8
+    N1 = 2 * I if act == "swiglu" else I
+    x = _bf16_bits(torch.from_numpy(rng.standard_normal((T, H)).astype(np.float32)))
+    l = rng.standard_normal((T, E)).astype(np.float32)
+    w13 = _bf16_bits(torch.from_numpy(0.3 * rng.standard_normal((E, N1, H)).astype(np.float32)))
+    w2 = _bf16_bits(torch.from_numpy(0.3 * rng.standard_normal((E, H, I)).astype(np.float32)))
+    return x, l, w13, w2, k
+
+
+@pytest.mark.parametrize("mutation", ["silu_sign", "swap_gate_up", "no_renorm", "tie_high_index",
+                                      "transpose_w2_slice", "drop_last_slot"])
+def test_planted_mistakes_are_caught(monkeypatch, mutation):
+    act = "swiglu"
+    x, l, w13, w2, k = _tiny_layer_inputs(act)
+    want = _dense_layer(O.bf16_bits_to_f64(x), l, O.bf16_bits_to_f64(w13), O.bf16_bits_to_f64(w2),
+                        k, True, act)
+    real_route = O.route
+    if mutation == "silu_sign":
+        monkeypatch.setattr(O, "silu", lambda z: z / (1.0 + np.exp(z)))
+    elif mutation == "swap_gate_up":
+        monkeypatch.setattr(O, "activation_fn", lambda z, a, I: O.silu(z[:, I:2 * I]) * z[:, :I])
+    elif mutation == "no_renorm":
+        monkeypatch.setattr(O, "route", lambda lg, kk, r, s=0: real_route(lg, kk, False, s))
+    elif mutation == "tie_high_index":
+        l = l.copy()
+        l[:, :3] = [1.0, 1.0, 2.0]   # experts 0 and 1 tie at the top-2 cut
+        l[:, 3:] = -1.0
+        want = _dense_layer(O.bf16_bits_to_f64(x), l, O.bf16_bits_to_f64(w13), O.bf16_bits_to_f64(w2),
+                            k, True, act)
+
+        def bad_route(lg, kk, r, s=0):
+            E = lg.shape[1]
+            ids, w = real_route(lg[:, ::-1].copy(), kk, r, s)
+            return (E - 1 - ids).astype(np.int32), w
+        monkeypatch.setattr(O, "route", bad_route)
+    elif mutation == "transpose_w2_slice":
+        w2 = w2.copy()
+        w2_t = w2.copy()
+        w2_t[:, :8, :] = np.swapaxes(w2[:, :8, :8], 1, 2)
+        got = O.moe_forward(x, l, w13, w2_t, topk=k, renormalize=True, activation=act)
+        assert np.max(np.abs(got - want)) > 1e-6
+        return
+    elif mutation == "drop_last_slot":
+        monkeypatch.setattr(O, "route", lambda lg, kk, r, s=0: real_route(lg, max(kk - 1, 1), r, s))
+    got = O.moe_forward(x, l, w13, w2, topk=k, renormalize=True, activation=act)
+    assert np.max(np.abs(got - want)) > 1e-6, mutation
