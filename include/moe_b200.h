@@ -1,0 +1,229 @@
+/*
+ * moe_b200.h -- C ABI of the B200 (sm_100a) fused Mixture-of-Experts layer forward.
+ *
+ * One call computes, for T tokens with hidden rows x_t (bf16, H wide):
+ *   1. route    top-k experts per token from fp32 router logits, softmax weights,
+ *               optional renormalisation, optional fused shared-expert slot;
+ *   2. align    stable sort of the T*k' (token, slot) pairs by expert, each expert's
+ *               segment padded to the GEMM row tile (block_m);
+ *   3. GEMM1    z = W13[e] x_t with the SwiGLU (silu(gate)*up) or relu2 (max(z,0)^2)
+ *               activation applied in the GEMM epilogue, so only the I-wide result
+ *               reaches memory;
+ *   4. GEMM2    y = w_tj * (W2[e] a);
+ *   5. combine  out_t = sum_j y_tj, in slot order j = 0..k'-1 (deterministic).
+ * k' = topk + num_shared. Pair p = t*k' + j.
+ *
+ * Sources, by page title and section:
+ *   "FlashInfer TRTLLM-Gen MoE kernel optimisation: NemotronH support" (sglang PR 21321):
+ *       section 1, the fused op trtllm_fp8_block_scale_moe(hidden_states, w13, w2, scales,
+ *       expert_weights, topk, renormalize, ..., activation_type) returning a bf16 tensor
+ *       of the hidden shape; section 2, intermediate padding (16 gated / 128 non-gated)
+ *       and the gated-only gate/up row reordering.
+ *   "[MoE] SwiGLU fusion into the MoE up-GEMM epilogue" (sglang PR 32944): section 1, the
+ *       activation in the GEMM1 epilogue writing N/2 columns; section 3, the load-time
+ *       [gate0, up0, gate1, up1, ...] interleave.
+ *   "Qwen3-Next FP8 MoE optimisation: shared-expert fusion for H200" (sglang PR 26204):
+ *       sections 1-2, FP8 W8A8 with 128x128 block scales and the shared expert fused as
+ *       an extra, always-selected expert slot.
+ *   "W4A8 grouped GEMM optimisation for GLM-5.2 MoE on H200" (sglang PR 38220): section 1,
+ *       the grouped-GEMM contract (expert_offsets, problem sizes).
+ *
+ * Conventions for every entry point:
+ *   - Pointers named d_* or documented as "device" are CUDA device pointers; "host"
+ *     pointers are CPU memory. All buffers are owned by the caller; the library
+ *     allocates no memory and keeps no per-call state outside the caller's workspace.
+ *   - Device pointers must be 16-byte aligned. Tensors are dense, row-major, with the
+ *     layouts stated at each argument.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = the legacy default stream)
+ *     and runs asynchronously unless stated otherwise. No entry point synchronises
+ *     except moe_forward_host and moe_get_device_status.
+ *   - All argument checks run on the host before any launch; a failing check returns an
+ *     error status and enqueues nothing. No C++ exception crosses this interface.
+ *   - A launch failure returns MOE_ERR_CUDA (the CUDA error is left for
+ *     cudaGetLastError). A device without sm_100 support returns MOE_ERR_UNSUPPORTED:
+ *     there is no fallback path.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* moe_stream_t; /* == cudaStream_t */
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,         /* null/misaligned pointer, inconsistent sizes */
+  MOE_ERR_UNSUPPORTED = 2,         /* valid but not implemented (shape, dtype, device) */
+  MOE_ERR_WORKSPACE_TOO_SMALL = 3, /* workspace_bytes < moe_workspace_size() */
+  MOE_ERR_CUDA = 4,                /* a CUDA runtime call or launch failed */
+  MOE_ERR_DEVICE_TIMEOUT = 5       /* a kernel gave up a bounded wait (see moe_get_device_status) */
+} moe_status_t;
+
+/* Activation of GEMM1 ("activation_type", sglang PR 21321 section 1). The numeric
+ * values are this library's own; the page does not print FlashInfer's enum values. */
+typedef enum {
+  MOE_ACT_SWIGLU = 0, /* gated: a_n = silu(gate_n) * up_n, silu(x) = x / (1 + e^-x) */
+  MOE_ACT_RELU2 = 1   /* non-gated: a_n = max(z_n, 0)^2 */
+} moe_activation_t;
+
+/* Weight / activation number format. */
+typedef enum {
+  MOE_DTYPE_BF16 = 0,         /* bf16 weights and activations, fp32 accumulation */
+  MOE_DTYPE_FP8_BLOCK128 = 1  /* e4m3 weights with one fp32 scale per 128x128 block and
+                                 e4m3 activations with one fp32 scale per 1x128 group
+                                 (FP8 W8A8, block_shape [128, 128]; sglang PR 26204
+                                 section 1) */
+} moe_wdtype_t;
+
+/* Bit flags of moe_problem_t.flags. */
+#define MOE_FLAG_PDL 1u /* launch with programmatic dependent launch between kernels */
+
+/* Problem description shared by all entry points. */
+typedef struct {
+  int32_t num_tokens;   /* T >= 0 */
+  int32_t hidden;       /* H > 0, multiple of 128 */
+  int32_t num_routed;   /* E_r >= 1: columns of router_logits */
+  int32_t num_shared;   /* 0 or 1: shared-expert slots; slot id E_r, weight 1, after the
+                           routed slots (sglang PR 26204 section 2). Experts in the
+                           weights: E = E_r + num_shared <= 1024. */
+  int32_t intermediate; /* I after padding (moe_padded_intermediate): multiple of 16 for
+                           SWIGLU, of 128 for RELU2 and for FP8 */
+  int32_t topk;         /* 1 <= topk <= E_r; topk + num_shared <= 16 */
+  int32_t renormalize;  /* 0/1: divide the selected softmax weights by their sum */
+  int32_t activation;   /* moe_activation_t */
+  int32_t wdtype;       /* moe_wdtype_t */
+  int32_t block_m;      /* GEMM row tile; 0 = default (128); only 128 is supported */
+  uint32_t flags;       /* MOE_FLAG_* */
+} moe_problem_t;
+
+/* Byte offsets of the intermediates inside the caller's workspace (for inspection by
+ * tests and tools; the contents are this library's private format otherwise). */
+typedef struct {
+  size_t total_bytes;
+  size_t status;          /* int32 device status word (0 = ok) */
+  size_t num_blocks;      /* int32: number of block_m row tiles after align (= P_pad/block_m) */
+  size_t topk_ids;        /* int32 [T, k'] selected expert ids, slot order */
+  size_t topk_w;          /* fp32  [T, k'] routing weights */
+  size_t sorted_pair_ids; /* int32 [max_rows]: pair ids sorted by expert, sentinel P in padding */
+  size_t expert_offsets;  /* int32 [E+1]: first row of each expert segment; [E] = P_pad */
+  size_t block_expert;    /* int32 [max_rows/block_m]: expert of each row tile */
+  size_t pair_to_row;     /* int32 [T*k']: sorted row of each pair */
+  size_t chunk_hist;      /* int32 [num_chunks, E]: align scratch */
+  size_t xq;              /* FP8: e4m3 [T, H] quantised hidden */
+  size_t xq_scale;        /* FP8: fp32 [T, H/128] */
+  size_t act;             /* GEMM1 output [max_rows, I]: bf16, or e4m3 for FP8 */
+  size_t act_scale;       /* FP8: fp32 [max_rows, I/128] */
+  size_t y;               /* bf16 [T*k', H]: weighted GEMM2 rows in pair order */
+  size_t io_hidden;       /* staging for moe_forward_host: bf16 [T, H] */
+  size_t io_logits;       /* staging for moe_forward_host: fp32 [T, E_r] */
+  size_t io_out;          /* staging for moe_forward_host: bf16 [T, H] */
+  int64_t max_rows;       /* upper bound of P_pad: round_up(P + min(E,P)*(block_m-1), block_m) */
+  int32_t num_chunks;     /* align chunks of 1024 pairs */
+  int32_t block_m;
+} moe_workspace_layout_t;
+
+/* Human-readable name of a status code (static string). */
+const char* moe_status_string(moe_status_t status);
+
+/* Host-only validation of a problem description. No CUDA call. */
+moe_status_t moe_check_problem(const moe_problem_t* problem);
+
+/* Intermediate size after alignment padding: round up to 16 (SWIGLU) or 128 (RELU2),
+ * as in sglang PR 21321 section 2 (_align_fp8_moe_weights); FP8 requires 128. Returns
+ * -1 for invalid arguments. Host only. */
+int32_t moe_padded_intermediate(int32_t intermediate, int32_t activation, int32_t wdtype);
+
+/* Workspace layout and size for `problem` (host only). On error `*layout` is zeroed. */
+moe_status_t moe_workspace_layout(const moe_problem_t* problem, moe_workspace_layout_t* layout);
+
+/* Workspace bytes for `problem`, or 0 if the problem is invalid. Host only. */
+size_t moe_workspace_size(const moe_problem_t* problem);
+
+/* Load-time weight preparation (sglang PR 21321 section 2; PR 32944 section 3).
+ *   w13_in  device [E, up_mult*intermediate_in, H], checkpoint order: gate rows [0, I_in)
+ *           then up rows [I_in, 2*I_in) for SWIGLU (up_mult 2), I_in rows for RELU2.
+ *   w2_in   device [E, H, intermediate_in].
+ *   w13_out device [E, N1, H] with N1 = 2*I (SWIGLU) or I (RELU2), I = problem->intermediate
+ *           = moe_padded_intermediate(intermediate_in, ...). SWIGLU rows are interleaved
+ *           [gate0, up0, gate1, up1, ...]; rows of padded indices are zero.
+ *   w2_out  device [E, H, I], columns >= intermediate_in zero.
+ * Elements are bf16 (2 bytes) or e4m3 codes (1 byte) per problem->wdtype. For FP8 the
+ * block scales need no change (FP8 requires intermediate_in == I, a multiple of 128);
+ * pass them to moe_forward in the checkpoint layout. Output buffers must not overlap
+ * the inputs. Asynchronous on `stream`. */
+moe_status_t moe_prepare_weights(const moe_problem_t* problem, int32_t intermediate_in,
+                                 const void* w13_in, const void* w2_in, void* w13_out,
+                                 void* w2_out, moe_stream_t stream);
+
+/* Block quantisation of bf16 weights to e4m3 (FP8 W8A8 block-128 weights):
+ *   w        device bf16 [num_mats, rows, cols], rows and cols multiples of 128;
+ *   codes    device e4m3 [num_mats, rows, cols];
+ *   scales   device fp32 [num_mats, rows/128, cols/128].
+ * Per 128x128 block: scale = amax/448 (fp32, IEEE division; 1 if amax == 0),
+ * code = e4m3(w/scale), round to nearest even, saturating at 448. */
+moe_status_t moe_quantize_weights_fp8(const void* w, int64_t num_mats, int32_t rows,
+                                      int32_t cols, void* codes, float* scales,
+                                      moe_stream_t stream);
+
+/* The layer forward (all five steps), asynchronous on `stream`.
+ *   hidden         device bf16 [T, H]
+ *   router_logits  device fp32 [T, E_r] (finite values; NaN/Inf are not supported)
+ *   w13            device, prepared by moe_prepare_weights: [E, N1, H] bf16 or e4m3
+ *   w2             device, prepared: [E, H, I] bf16 or e4m3
+ *   w13_scale      FP8 only (else NULL): device fp32 [E, N1/128, H/128], checkpoint
+ *                  (gate-first, un-interleaved) block order
+ *   w2_scale       FP8 only (else NULL): device fp32 [E, H/128, I/128]
+ *   out            device bf16 [T, H] (must not alias hidden)
+ *   workspace      device, >= moe_workspace_size(problem) bytes, 256-byte aligned; one
+ *                  workspace must not be used by two calls in flight at once.
+ * T == 0 returns MOE_OK and enqueues nothing. Routing ids, the permutation and
+ * expert_offsets are deterministic; the output is bitwise reproducible run to run. */
+moe_status_t moe_forward(const moe_problem_t* problem, const void* hidden,
+                         const float* router_logits, const void* w13, const void* w2,
+                         const float* w13_scale, const float* w2_scale, void* out,
+                         void* workspace, size_t workspace_bytes, moe_stream_t stream);
+
+/* moe_forward with HOST hidden [T,H] bf16, router_logits [T,E_r] fp32 and out [T,H] bf16
+ * (pinned memory gives asynchronous copies; pageable memory works too). The inputs are
+ * copied into the workspace staging areas, the forward runs, the output is copied back
+ * and the stream is synchronised before returning. Weights and workspace are device
+ * memory as in moe_forward. */
+moe_status_t moe_forward_host(const moe_problem_t* problem, const void* h_hidden,
+                              const float* h_router_logits, const void* w13, const void* w2,
+                              const float* w13_scale, const float* w2_scale, void* h_out,
+                              void* workspace, size_t workspace_bytes, moe_stream_t stream);
+
+/* The five steps as separate calls on the same workspace (moe_forward runs exactly
+ * these, in this order). They exist so tests can check each intermediate and tools can
+ * time each kernel; each requires the previous steps to have been enqueued. */
+moe_status_t moe_stage_route(const moe_problem_t* problem, const float* router_logits,
+                             void* workspace, size_t workspace_bytes, moe_stream_t stream);
+moe_status_t moe_stage_align(const moe_problem_t* problem, void* workspace,
+                             size_t workspace_bytes, moe_stream_t stream);
+/* FP8 only: quantise hidden per token per 128 columns into the workspace (xq, xq_scale). */
+moe_status_t moe_stage_quant_act(const moe_problem_t* problem, const void* hidden,
+                                 void* workspace, size_t workspace_bytes, moe_stream_t stream);
+moe_status_t moe_stage_gemm1(const moe_problem_t* problem, const void* hidden, const void* w13,
+                             const float* w13_scale, void* workspace, size_t workspace_bytes,
+                             moe_stream_t stream);
+moe_status_t moe_stage_gemm2(const moe_problem_t* problem, const void* w2, const float* w2_scale,
+                             void* workspace, size_t workspace_bytes, moe_stream_t stream);
+moe_status_t moe_stage_combine(const moe_problem_t* problem, void* out, void* workspace,
+                               size_t workspace_bytes, moe_stream_t stream);
+
+/* Synchronises `stream`, reads and clears the workspace status word. Returns MOE_OK,
+ * MOE_ERR_DEVICE_TIMEOUT if a kernel abandoned a bounded wait since the last query
+ * (its outputs are then undefined), or MOE_ERR_CUDA. `*detail` (may be NULL) receives
+ * the raw word: bits 0-15 name the wait site. */
+moe_status_t moe_get_device_status(void* workspace, moe_stream_t stream, int32_t* detail);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

@@ -1,0 +1,262 @@
+"""B200 (sm_100a) fused Mixture-of-Experts layer forward.
+
+Thin Python binding over the C ABI of ``libmoe_b200.so`` (``include/moe_b200.h``).
+Every step of the layer runs in the library's CUDA kernels; this module only
+marshals torch tensors into pointers and sizes, allocates outputs and workspaces
+with torch, and passes ``torch.cuda.current_stream()``.
+
+    import mixture_experts_expert_topk_b200 as moe
+    prob = moe.make_problem(T, H, E, topk, I, renormalize=True, activation="swiglu")
+    w13p, w2p = moe.prepare_weights(prob, w13, w2, I_in)
+    out = moe.moe_forward(hidden, router_logits, w13p, w2p, topk, True, "swiglu")
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Dict, Optional, Tuple
+
+import torch
+
+from . import _capi
+from ._capi import (MOE_ACT_RELU2, MOE_ACT_SWIGLU, MOE_DTYPE_BF16, MOE_DTYPE_FP8_BLOCK128,
+                    MOE_FLAG_PDL, MoeError, Problem, check, lib)
+
+__all__ = [
+    "MoeError", "Problem", "make_problem", "padded_intermediate", "workspace_layout",
+    "workspace_size", "new_workspace", "prepare_weights", "quantize_weights_fp8", "moe_forward",
+    "moe_forward_host", "stage_route", "stage_align", "stage_quant_act", "stage_gemm1",
+    "stage_gemm2", "stage_combine", "device_status", "read_workspace", "lib",
+]
+
+_ACT = {"swiglu": MOE_ACT_SWIGLU, "silu": MOE_ACT_SWIGLU, "relu2": MOE_ACT_RELU2,
+        MOE_ACT_SWIGLU: MOE_ACT_SWIGLU, MOE_ACT_RELU2: MOE_ACT_RELU2}
+
+
+def _act(a) -> int:
+    if a not in _ACT:
+        raise ValueError(f"unknown activation_type {a!r}")
+    return _ACT[a]
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream: Optional[torch.cuda.Stream] = None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dev(t: torch.Tensor, name: str, dtype=None) -> torch.Tensor:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    return t
+
+
+def make_problem(T: int, H: int, num_routed: int, topk: int, intermediate: int, *,
+                 renormalize: bool = True, activation="swiglu", num_shared: int = 0,
+                 fp8: bool = False, pdl: bool = True, block_m: int = 0) -> Problem:
+    """Problem description; ``intermediate`` must already be padded."""
+    return Problem(num_tokens=T, hidden=H, num_routed=num_routed, num_shared=num_shared,
+                   intermediate=intermediate, topk=topk, renormalize=int(bool(renormalize)),
+                   activation=_act(activation),
+                   wdtype=MOE_DTYPE_FP8_BLOCK128 if fp8 else MOE_DTYPE_BF16, block_m=block_m,
+                   flags=MOE_FLAG_PDL if pdl else 0)
+
+
+def padded_intermediate(intermediate: int, activation="swiglu", fp8: bool = False) -> int:
+    v = lib().moe_padded_intermediate(intermediate, _act(activation),
+                                      MOE_DTYPE_FP8_BLOCK128 if fp8 else MOE_DTYPE_BF16)
+    if v < 0:
+        raise ValueError("invalid intermediate size or activation")
+    return v
+
+
+def workspace_layout(prob: Problem) -> Dict[str, int]:
+    lay = _capi.Layout()
+    check(lib().moe_workspace_layout(ctypes.byref(prob), ctypes.byref(lay)), "moe_workspace_layout")
+    return {name: getattr(lay, name) for name, _ in _capi.Layout._fields_}
+
+
+def workspace_size(prob: Problem) -> int:
+    n = lib().moe_workspace_size(ctypes.byref(prob))
+    if n == 0:
+        check(lib().moe_check_problem(ctypes.byref(prob)), "moe_workspace_size")
+    return n
+
+
+def new_workspace(prob: Problem, device=None) -> torch.Tensor:
+    """A uint8 CUDA tensor of moe_workspace_size bytes (256-byte aligned by torch)."""
+    return torch.empty(workspace_size(prob), dtype=torch.uint8,
+                       device=device if device is not None else "cuda")
+
+
+def prepare_weights(prob: Problem, w13: torch.Tensor, w2: torch.Tensor, intermediate_in: int,
+                    stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Load-time padding + gate/up interleave (bf16, or e4m3 codes as uint8)."""
+    fp8 = prob.wdtype == MOE_DTYPE_FP8_BLOCK128
+    dt = torch.uint8 if fp8 else torch.bfloat16
+    _dev(w13, "w13", dt)
+    _dev(w2, "w2", dt)
+    E = prob.num_routed + prob.num_shared
+    I = prob.intermediate
+    N1 = 2 * I if prob.activation == MOE_ACT_SWIGLU else I
+    w13p = torch.empty((E, N1, prob.hidden), dtype=dt, device=w13.device)
+    w2p = torch.empty((E, prob.hidden, I), dtype=dt, device=w2.device)
+    check(lib().moe_prepare_weights(ctypes.byref(prob), intermediate_in, _ptr(w13), _ptr(w2),
+                                    _ptr(w13p), _ptr(w2p), _stream(stream)), "moe_prepare_weights")
+    return w13p, w2p
+
+
+def quantize_weights_fp8(w: torch.Tensor, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Per-128x128-block e4m3 quantisation of bf16 [..., rows, cols] weights."""
+    _dev(w, "w", torch.bfloat16)
+    rows, cols = w.shape[-2], w.shape[-1]
+    mats = w.numel() // (rows * cols)
+    codes = torch.empty(w.shape, dtype=torch.uint8, device=w.device)
+    scales = torch.empty(tuple(w.shape[:-2]) + (rows // 128, cols // 128), dtype=torch.float32,
+                         device=w.device)
+    check(lib().moe_quantize_weights_fp8(_ptr(w), mats, rows, cols, _ptr(codes), _ptr(scales),
+                                         _stream(stream)), "moe_quantize_weights_fp8")
+    return codes, scales
+
+
+def _problem_from(hidden, router_logits, w2, topk, renormalize, activation_type, num_shared,
+                  fp8, pdl) -> Problem:
+    T, H = hidden.shape
+    E_r = router_logits.shape[1]
+    return make_problem(T, H, E_r, topk, w2.shape[2], renormalize=renormalize,
+                        activation=activation_type, num_shared=num_shared, fp8=fp8, pdl=pdl)
+
+
+_WS_CACHE: Dict[tuple, torch.Tensor] = {}
+
+
+def _workspace_for(prob: Problem, device) -> torch.Tensor:
+    key = (device, prob.num_tokens, prob.hidden, prob.num_routed, prob.num_shared,
+           prob.intermediate, prob.topk, prob.activation, prob.wdtype, prob.block_m)
+    ws = _WS_CACHE.get(key)
+    if ws is None:
+        ws = new_workspace(prob, device)
+        _WS_CACHE[key] = ws
+    return ws
+
+
+def moe_forward(hidden: torch.Tensor, router_logits: torch.Tensor, w13: torch.Tensor,
+                w2: torch.Tensor, topk: int, renormalize: bool, activation_type,
+                w13_scale: Optional[torch.Tensor] = None, w2_scale: Optional[torch.Tensor] = None,
+                num_shared: int = 0, *, workspace: Optional[torch.Tensor] = None,
+                out: Optional[torch.Tensor] = None, pdl: bool = True, stream=None) -> torch.Tensor:
+    """Fused MoE layer forward on the current CUDA stream.
+
+    ``hidden`` bf16 [T,H]; ``router_logits`` fp32 [T,E_r]; ``w13``/``w2`` prepared by
+    :func:`prepare_weights` (bf16, or uint8 e4m3 codes with fp32 block scales
+    ``w13_scale`` [E, N1/128, H/128] and ``w2_scale`` [E, H/128, I/128]). Returns bf16 [T,H].
+    """
+    fp8 = w13_scale is not None
+    _dev(hidden, "hidden", torch.bfloat16)
+    _dev(router_logits, "router_logits", torch.float32)
+    _dev(w13, "w13")
+    _dev(w2, "w2")
+    prob = _problem_from(hidden, router_logits, w2, topk, renormalize, activation_type,
+                         num_shared, fp8, pdl)
+    if workspace is None:
+        workspace = _workspace_for(prob, hidden.device)
+    if out is None:
+        out = torch.empty_like(hidden)
+    check(lib().moe_forward(ctypes.byref(prob), _ptr(hidden), _ptr(router_logits), _ptr(w13),
+                            _ptr(w2), _ptr(w13_scale), _ptr(w2_scale), _ptr(out),
+                            _ptr(workspace), workspace.numel(), _stream(stream)), "moe_forward")
+    return out
+
+
+def moe_forward_host(prob: Problem, hidden_host: torch.Tensor, logits_host: torch.Tensor,
+                     w13: torch.Tensor, w2: torch.Tensor, out_host: torch.Tensor,
+                     workspace: torch.Tensor, w13_scale=None, w2_scale=None, stream=None) -> None:
+    """The forward on HOST tensors (pinned for asynchronous copies); blocks until done."""
+    for t, n in ((hidden_host, "hidden"), (logits_host, "logits"), (out_host, "out")):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{n} must be a contiguous CPU tensor")
+    check(lib().moe_forward_host(ctypes.byref(prob), _ptr(hidden_host), _ptr(logits_host),
+                                 _ptr(w13), _ptr(w2), _ptr(w13_scale), _ptr(w2_scale),
+                                 _ptr(out_host), _ptr(workspace), workspace.numel(),
+                                 _stream(stream)), "moe_forward_host")
+
+
+# ---- the five steps, for tests and per-kernel timing -----------------------------------
+
+def stage_route(prob, router_logits, workspace, stream=None):
+    check(lib().moe_stage_route(ctypes.byref(prob), _ptr(router_logits), _ptr(workspace),
+                                workspace.numel(), _stream(stream)), "moe_stage_route")
+
+
+def stage_align(prob, workspace, stream=None):
+    check(lib().moe_stage_align(ctypes.byref(prob), _ptr(workspace), workspace.numel(),
+                                _stream(stream)), "moe_stage_align")
+
+
+def stage_quant_act(prob, hidden, workspace, stream=None):
+    check(lib().moe_stage_quant_act(ctypes.byref(prob), _ptr(hidden), _ptr(workspace),
+                                    workspace.numel(), _stream(stream)), "moe_stage_quant_act")
+
+
+def stage_gemm1(prob, hidden, w13, workspace, w13_scale=None, stream=None):
+    check(lib().moe_stage_gemm1(ctypes.byref(prob), _ptr(hidden), _ptr(w13), _ptr(w13_scale),
+                                _ptr(workspace), workspace.numel(), _stream(stream)),
+          "moe_stage_gemm1")
+
+
+def stage_gemm2(prob, w2, workspace, w2_scale=None, stream=None):
+    check(lib().moe_stage_gemm2(ctypes.byref(prob), _ptr(w2), _ptr(w2_scale), _ptr(workspace),
+                                workspace.numel(), _stream(stream)), "moe_stage_gemm2")
+
+
+def stage_combine(prob, out, workspace, stream=None):
+    check(lib().moe_stage_combine(ctypes.byref(prob), _ptr(out), _ptr(workspace),
+                                  workspace.numel(), _stream(stream)), "moe_stage_combine")
+
+
+def device_status(workspace: torch.Tensor, stream=None) -> Tuple[int, int]:
+    """(status, raw word) of the workspace's device status; synchronises the stream."""
+    detail = ctypes.c_int32(0)
+    st = lib().moe_get_device_status(_ptr(workspace), _stream(stream), ctypes.byref(detail))
+    return st, detail.value
+
+
+def read_workspace(prob: Problem, workspace: torch.Tensor) -> Dict[str, torch.Tensor]:
+    """Views of the intermediates inside a workspace (device tensors, no copy)."""
+    L = workspace_layout(prob)
+    T, kk = prob.num_tokens, prob.topk + prob.num_shared
+    P = T * kk
+    E = prob.num_routed + prob.num_shared
+    rows = L["max_rows"]
+    fp8 = prob.wdtype == MOE_DTYPE_FP8_BLOCK128
+    I, H = prob.intermediate, prob.hidden
+
+    def view(off, n, dtype):
+        nbytes = n * torch.tensor([], dtype=dtype).element_size()
+        return workspace[off:off + nbytes].view(dtype)
+
+    out = {
+        "status": view(L["status"], 1, torch.int32),
+        "num_blocks": view(L["num_blocks"], 1, torch.int32),
+        "topk_ids": view(L["topk_ids"], P, torch.int32).view(T, kk),
+        "topk_w": view(L["topk_w"], P, torch.float32).view(T, kk),
+        "sorted_pair_ids": view(L["sorted_pair_ids"], rows, torch.int32),
+        "expert_offsets": view(L["expert_offsets"], E + 1, torch.int32),
+        "block_expert": view(L["block_expert"], rows // L["block_m"], torch.int32),
+        "pair_to_row": view(L["pair_to_row"], P, torch.int32),
+        "y": view(L["y"], P * H, torch.bfloat16).view(P, H),
+    }
+    if fp8:
+        out["xq"] = view(L["xq"], T * H, torch.uint8).view(T, H)
+        out["xq_scale"] = view(L["xq_scale"], T * (H // 128), torch.float32).view(T, H // 128)
+        out["act"] = view(L["act"], rows * I, torch.uint8).view(rows, I)
+        out["act_scale"] = view(L["act_scale"], rows * (I // 128), torch.float32).view(rows, I // 128)
+    else:
+        out["act"] = view(L["act"], rows * I, torch.bfloat16).view(rows, I)
+    return out

@@ -1,0 +1,558 @@
+// C ABI of the fused MoE layer forward: argument checks, workspace carving, tensor-map
+// encoding and the launch sequence route -> align -> [quant] -> GEMM1 -> GEMM2 -> combine
+// on the caller's stream. See include/moe_b200.h for the contract of each entry point.
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cstring>
+#include <mutex>
+
+#include "moe_b200.h"
+#include "moe_internal.h"
+
+#define MOE_API extern "C" __attribute__((visibility("default")))
+
+namespace moe {
+
+void make_launch_config(cudaLaunchConfig_t* cfg, cudaLaunchAttribute* attr, const Launch& l, dim3 grid,
+                        dim3 block, size_t smem) {
+  std::memset(cfg, 0, sizeof(*cfg));
+  cfg->gridDim = grid;
+  cfg->blockDim = block;
+  cfg->dynamicSmemBytes = smem;
+  cfg->stream = l.stream;
+  if (l.pdl) {
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg->attrs = attr;
+    cfg->numAttrs = 1;
+  } else {
+    cfg->attrs = nullptr;
+    cfg->numAttrs = 0;
+  }
+}
+
+}  // namespace moe
+
+namespace {
+
+using moe::GemmBuffers;
+using moe::GemmShape;
+using moe::Launch;
+
+constexpr size_t kAlign = 1024;
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+struct Plan {
+  int T, H, Er, Es, E, I, topk, kk, bm, N1, gated, fp8, renorm, act;
+  long long P;
+  int bn1, bn2;
+  moe_workspace_layout_t lay;
+};
+
+moe_status_t make_plan(const moe_problem_t* p, Plan* pl) {
+  if (p == nullptr || pl == nullptr) return MOE_ERR_INVALID_ARG;
+  Plan q;
+  std::memset(&q, 0, sizeof(q));
+  if (p->num_tokens < 0 || p->hidden <= 0 || p->num_routed < 1 || p->topk < 1 || p->intermediate <= 0)
+    return MOE_ERR_INVALID_ARG;
+  if (p->num_shared != 0 && p->num_shared != 1) return MOE_ERR_INVALID_ARG;
+  if (p->topk > p->num_routed) return MOE_ERR_INVALID_ARG;
+  if (p->renormalize != 0 && p->renormalize != 1) return MOE_ERR_INVALID_ARG;
+  if (p->activation != MOE_ACT_SWIGLU && p->activation != MOE_ACT_RELU2) return MOE_ERR_INVALID_ARG;
+  if (p->wdtype != MOE_DTYPE_BF16 && p->wdtype != MOE_DTYPE_FP8_BLOCK128) return MOE_ERR_INVALID_ARG;
+  if (p->flags & ~MOE_FLAG_PDL) return MOE_ERR_INVALID_ARG;
+  q.gated = p->activation == MOE_ACT_SWIGLU;
+  q.fp8 = p->wdtype == MOE_DTYPE_FP8_BLOCK128;
+  // the intermediate size must already be padded (moe_padded_intermediate)
+  const int ialign = (q.fp8 || !q.gated) ? 128 : 16;
+  if (p->intermediate % ialign != 0) return MOE_ERR_INVALID_ARG;
+  if (p->hidden % 128 != 0) return MOE_ERR_UNSUPPORTED;
+  if (p->num_routed + p->num_shared > moe::kMaxExperts) return MOE_ERR_UNSUPPORTED;
+  if (p->topk + p->num_shared > moe::kMaxSlots) return MOE_ERR_UNSUPPORTED;
+  if (p->block_m != 0 && p->block_m != 128) return MOE_ERR_UNSUPPORTED;
+  if (p->hidden > (1 << 20) || p->intermediate > (1 << 20)) return MOE_ERR_UNSUPPORTED;
+
+  q.T = p->num_tokens;
+  q.H = p->hidden;
+  q.Er = p->num_routed;
+  q.Es = p->num_shared;
+  q.E = q.Er + q.Es;
+  q.I = p->intermediate;
+  q.topk = p->topk;
+  q.kk = q.topk + q.Es;
+  q.bm = 128;
+  q.N1 = q.gated ? 2 * q.I : q.I;
+  q.renorm = p->renormalize;
+  q.act = p->activation;
+  q.P = static_cast<long long>(q.T) * q.kk;
+  if (q.P >= (1LL << 31) - (1LL << 20)) return MOE_ERR_UNSUPPORTED;
+  q.bn1 = moe::pick_bn(q.N1, q.gated);
+  q.bn2 = moe::pick_bn(q.H, false);
+  if (q.bn1 == 0 || q.bn2 == 0) return MOE_ERR_UNSUPPORTED;
+
+  moe_workspace_layout_t& L = q.lay;
+  const long long active = q.P < q.E ? q.P : q.E;
+  L.block_m = q.bm;
+  L.max_rows = static_cast<int64_t>(align_up(static_cast<size_t>(q.P + active * (q.bm - 1)), q.bm));
+  L.num_chunks = static_cast<int32_t>(q.P == 0 ? 1 : (q.P + moe::kAlignChunk - 1) / moe::kAlignChunk);
+  const size_t T = static_cast<size_t>(q.T), H = q.H, I = q.I, P = static_cast<size_t>(q.P);
+  const size_t rows = static_cast<size_t>(L.max_rows);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align_up(off + bytes, kAlign);
+    return at;
+  };
+  L.status = take(256);  // always offset 0 (moe_get_device_status relies on it)
+  L.num_blocks = take(256);
+  L.topk_ids = take(P * 4);
+  L.topk_w = take(P * 4);
+  L.sorted_pair_ids = take(rows * 4);
+  L.expert_offsets = take((static_cast<size_t>(q.E) + 1) * 4);
+  L.block_expert = take(rows / q.bm * 4 + 4);
+  L.pair_to_row = take(P * 4);
+  L.chunk_hist = take(static_cast<size_t>(L.num_chunks) * q.E * 4);
+  L.xq = take(q.fp8 ? T * H : 0);
+  L.xq_scale = take(q.fp8 ? T * (H / 128) * 4 : 0);
+  L.act = take(rows * I * (q.fp8 ? 1 : 2));
+  L.act_scale = take(q.fp8 ? rows * (I / 128) * 4 : 0);
+  L.y = take(P * H * 2);
+  L.io_hidden = take(T * H * 2);
+  L.io_logits = take(T * static_cast<size_t>(q.Er) * 4);
+  L.io_out = take(T * H * 2);
+  L.total_bytes = off;
+  *pl = q;
+  return MOE_OK;
+}
+
+// Device support: sm_100 (compute capability 10.0) only. Caches the SM count.
+std::atomic<int> g_dev_sms[64];
+
+moe_status_t device_sms(int* num_sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (dev >= 0 && dev < 64) {
+    const int c = g_dev_sms[dev].load(std::memory_order_relaxed);
+    if (c > 0) {
+      *num_sms = c;
+      return MOE_OK;
+    }
+    if (c < 0) return MOE_ERR_UNSUPPORTED;
+  }
+  int major = 0, minor = 0, sms = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  const bool ok = major == 10 && minor == 0;
+  if (dev >= 0 && dev < 64) g_dev_sms[dev].store(ok ? sms : -1, std::memory_order_relaxed);
+  if (!ok) return MOE_ERR_UNSUPPORTED;
+  *num_sms = sms;
+  return MOE_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult qres;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &qres) ==
+            cudaSuccess &&
+        qres == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode;
+}
+
+// 2-D tensor map over a row-major [outer, inner] matrix with a {box_inner, box_outer}
+// box, 128-byte swizzle, zero fill out of bounds.
+bool make_tmap_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elt_bytes, uint64_t inner,
+                  uint64_t outer, uint32_t box_inner, uint32_t box_outer) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = encode_fn();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * static_cast<uint64_t>(elt_bytes)};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename T>
+T* ws_ptr(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+moe_status_t cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return MOE_OK;
+  if (e == cudaErrorNotSupported) return MOE_ERR_UNSUPPORTED;
+  return MOE_ERR_CUDA;
+}
+
+moe_status_t check_ws(const Plan& pl, const void* ws, size_t ws_bytes) {
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < pl.lay.total_bytes) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  return MOE_OK;
+}
+
+// ---- the steps (arguments already checked) ----------------------------------------
+
+moe_status_t run_route(const Plan& pl, const float* logits, void* ws, const Launch& l) {
+  const auto& L = pl.lay;
+  // the route kernel also resets the device status word: it starts every forward
+  return cuda_status(moe::launch_route(l, logits, pl.T, pl.Er, pl.topk, pl.Es, pl.renorm,
+                                       ws_ptr<int>(ws, L.topk_ids), ws_ptr<float>(ws, L.topk_w),
+                                       ws_ptr<int>(ws, L.status)));
+}
+
+moe_status_t run_align(const Plan& pl, void* ws, const Launch& l) {
+  const auto& L = pl.lay;
+  return cuda_status(moe::launch_align(l, ws_ptr<int>(ws, L.topk_ids), static_cast<int>(pl.P), pl.E, pl.bm,
+                                       L.num_chunks, ws_ptr<int>(ws, L.chunk_hist),
+                                       ws_ptr<int>(ws, L.sorted_pair_ids), ws_ptr<int>(ws, L.expert_offsets),
+                                       ws_ptr<int>(ws, L.block_expert), ws_ptr<int>(ws, L.pair_to_row),
+                                       ws_ptr<int>(ws, L.num_blocks)));
+}
+
+moe_status_t run_quant_act(const Plan& pl, const void* hidden, void* ws, const Launch& l) {
+  const auto& L = pl.lay;
+  return cuda_status(moe::launch_quant_act(l, hidden, pl.T, pl.H, ws_ptr<void>(ws, L.xq),
+                                           ws_ptr<float>(ws, L.xq_scale)));
+}
+
+GemmBuffers common_buffers(const Plan& pl, void* ws) {
+  const auto& L = pl.lay;
+  GemmBuffers b;
+  std::memset(&b, 0, sizeof(b));
+  b.num_blocks = ws_ptr<int>(ws, L.num_blocks);
+  b.block_expert = ws_ptr<int>(ws, L.block_expert);
+  b.sorted_pair_ids = ws_ptr<int>(ws, L.sorted_pair_ids);
+  b.topk_w = ws_ptr<float>(ws, L.topk_w);
+  b.status = ws_ptr<int>(ws, L.status);
+  return b;
+}
+
+moe_status_t run_gemm1(const Plan& pl, const void* hidden, const void* w13, const float* w13_scale, void* ws,
+                       const Launch& l, int num_sms) {
+  const auto& L = pl.lay;
+  GemmShape s;
+  s.K = pl.H;
+  s.N = pl.N1;
+  s.BN = pl.bn1;
+  s.w_rows_per_expert = pl.N1;
+  s.k_total = pl.kk;
+  s.num_pairs = static_cast<int>(pl.P);
+  s.activation = pl.act;
+  s.out_cols = pl.I;
+  s.num_sms = num_sms;
+  GemmBuffers b = common_buffers(pl, ws);
+  b.out = ws_ptr<void>(ws, L.act);
+  CUtensorMap ta, tb;
+  if (!pl.fp8) {
+    if (!make_tmap_2d(&ta, hidden, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, pl.H, pl.T, 64, 1) ||
+        !make_tmap_2d(&tb, w13, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, pl.H,
+                      static_cast<uint64_t>(pl.E) * pl.N1, 64, pl.bn1))
+      return MOE_ERR_CUDA;
+    return cuda_status(moe::launch_gemm1_bf16(l, ta, tb, s, b));
+  }
+  if (!make_tmap_2d(&ta, ws_ptr<void>(ws, L.xq), CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, pl.H, pl.T, 128, 1) ||
+      !make_tmap_2d(&tb, w13, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, pl.H, static_cast<uint64_t>(pl.E) * pl.N1, 128,
+                    pl.bn1))
+    return MOE_ERR_CUDA;
+  b.out_scale = ws_ptr<float>(ws, L.act_scale);
+  b.a_scale = ws_ptr<float>(ws, L.xq_scale);
+  b.w_scale = w13_scale;
+  b.a_scale_cols = pl.H / 128;
+  b.w_scale_rows = pl.N1 / 128;
+  b.w_scale_cols = pl.H / 128;
+  b.up_block_offset = pl.I / 128;
+  return cuda_status(moe::launch_gemm1_fp8(l, ta, tb, s, b));
+}
+
+moe_status_t run_gemm2(const Plan& pl, const void* w2, const float* w2_scale, void* ws, const Launch& l,
+                       int num_sms) {
+  const auto& L = pl.lay;
+  GemmShape s;
+  s.K = pl.I;
+  s.N = pl.H;
+  s.BN = pl.bn2;
+  s.w_rows_per_expert = pl.H;
+  s.k_total = pl.kk;
+  s.num_pairs = static_cast<int>(pl.P);
+  s.activation = pl.act;
+  s.out_cols = pl.H;
+  s.num_sms = num_sms;
+  GemmBuffers b = common_buffers(pl, ws);
+  b.out = ws_ptr<void>(ws, L.y);
+  CUtensorMap ta, tb;
+  const uint64_t rows = static_cast<uint64_t>(L.max_rows);
+  if (!pl.fp8) {
+    if (!make_tmap_2d(&ta, ws_ptr<void>(ws, L.act), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, pl.I, rows, 64, 128) ||
+        !make_tmap_2d(&tb, w2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, pl.I, static_cast<uint64_t>(pl.E) * pl.H, 64,
+                      pl.bn2))
+      return MOE_ERR_CUDA;
+    return cuda_status(moe::launch_gemm2_bf16(l, ta, tb, s, b));
+  }
+  if (!make_tmap_2d(&ta, ws_ptr<void>(ws, L.act), CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, pl.I, rows, 128, 128) ||
+      !make_tmap_2d(&tb, w2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, pl.I, static_cast<uint64_t>(pl.E) * pl.H, 128,
+                    pl.bn2))
+    return MOE_ERR_CUDA;
+  b.a_scale = ws_ptr<float>(ws, L.act_scale);
+  b.w_scale = w2_scale;
+  b.a_scale_cols = pl.I / 128;
+  b.w_scale_rows = pl.H / 128;
+  b.w_scale_cols = pl.I / 128;
+  return cuda_status(moe::launch_gemm2_fp8(l, ta, tb, s, b));
+}
+
+moe_status_t run_combine(const Plan& pl, void* out, void* ws, const Launch& l) {
+  return cuda_status(moe::launch_combine(l, ws_ptr<void>(ws, pl.lay.y), pl.T, pl.kk, pl.H, out));
+}
+
+// Common preamble of the entry points that launch: plan, workspace, device.
+moe_status_t prologue(const moe_problem_t* p, const void* ws, size_t ws_bytes, Plan* pl, int* num_sms) {
+  moe_status_t st = make_plan(p, pl);
+  if (st != MOE_OK) return st;
+  st = check_ws(*pl, ws, ws_bytes);
+  if (st != MOE_OK) return st;
+  if (pl->T == 0) return MOE_OK;
+  return device_sms(num_sms);
+}
+
+Launch launch_of(const moe_problem_t* p, moe_stream_t stream) {
+  Launch l;
+  l.stream = reinterpret_cast<cudaStream_t>(stream);
+  l.pdl = (p->flags & MOE_FLAG_PDL) != 0;
+  return l;
+}
+
+moe_status_t forward_device(const Plan& pl, const moe_problem_t* p, const void* hidden, const float* logits,
+                            const void* w13, const void* w2, const float* s13, const float* s2, void* out,
+                            void* ws, moe_stream_t stream, int num_sms) {
+  const Launch l = launch_of(p, stream);
+  moe_status_t st = run_route(pl, logits, ws, l);
+  if (st == MOE_OK) st = run_align(pl, ws, l);
+  if (st == MOE_OK && pl.fp8) st = run_quant_act(pl, hidden, ws, l);
+  if (st == MOE_OK) st = run_gemm1(pl, hidden, w13, s13, ws, l, num_sms);
+  if (st == MOE_OK) st = run_gemm2(pl, w2, s2, ws, l, num_sms);
+  if (st == MOE_OK) st = run_combine(pl, out, ws, l);
+  return st;
+}
+
+moe_status_t check_weights(const Plan& pl, const void* w13, const void* w2, const float* s13, const float* s2) {
+  if (!aligned16(w13) || !aligned16(w2)) return MOE_ERR_INVALID_ARG;
+  if (pl.fp8 && (!aligned4(s13) || !aligned4(s2))) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+}  // namespace
+
+MOE_API const char* moe_status_string(moe_status_t s) {
+  switch (s) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+    case MOE_ERR_WORKSPACE_TOO_SMALL: return "MOE_ERR_WORKSPACE_TOO_SMALL";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_DEVICE_TIMEOUT: return "MOE_ERR_DEVICE_TIMEOUT";
+  }
+  return "MOE_ERR_UNKNOWN";
+}
+
+MOE_API moe_status_t moe_check_problem(const moe_problem_t* problem) {
+  Plan pl;
+  return make_plan(problem, &pl);
+}
+
+MOE_API int32_t moe_padded_intermediate(int32_t intermediate, int32_t activation, int32_t wdtype) {
+  if (intermediate <= 0 || intermediate > (1 << 20)) return -1;
+  if (activation != MOE_ACT_SWIGLU && activation != MOE_ACT_RELU2) return -1;
+  if (wdtype != MOE_DTYPE_BF16 && wdtype != MOE_DTYPE_FP8_BLOCK128) return -1;
+  const int a = (wdtype == MOE_DTYPE_FP8_BLOCK128 || activation == MOE_ACT_RELU2) ? 128 : 16;
+  return (intermediate + a - 1) / a * a;
+}
+
+MOE_API moe_status_t moe_workspace_layout(const moe_problem_t* problem, moe_workspace_layout_t* layout) {
+  if (layout == nullptr) return MOE_ERR_INVALID_ARG;
+  std::memset(layout, 0, sizeof(*layout));
+  Plan pl;
+  const moe_status_t st = make_plan(problem, &pl);
+  if (st == MOE_OK) *layout = pl.lay;
+  return st;
+}
+
+MOE_API size_t moe_workspace_size(const moe_problem_t* problem) {
+  Plan pl;
+  return make_plan(problem, &pl) == MOE_OK ? pl.lay.total_bytes : 0;
+}
+
+MOE_API moe_status_t moe_prepare_weights(const moe_problem_t* problem, int32_t intermediate_in, const void* w13_in,
+                                         const void* w2_in, void* w13_out, void* w2_out, moe_stream_t stream) {
+  Plan pl;
+  moe_status_t st = make_plan(problem, &pl);  // num_tokens plays no part in weight preparation
+  if (st != MOE_OK) return st;
+  if (moe_padded_intermediate(intermediate_in, pl.act, problem->wdtype) != pl.I) return MOE_ERR_INVALID_ARG;
+  if (pl.fp8 && intermediate_in != pl.I) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(w13_in) || !aligned16(w13_out) || w2_in == nullptr || w2_out == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  const int elt = pl.fp8 ? 1 : 2;
+  if ((reinterpret_cast<uintptr_t>(w2_in) | reinterpret_cast<uintptr_t>(w2_out)) & (elt - 1))
+    return MOE_ERR_INVALID_ARG;
+  int sms = 0;
+  st = device_sms(&sms);
+  if (st != MOE_OK) return st;
+  const Launch l = launch_of(problem, stream);
+  cudaError_t e = moe::launch_prepare_w13(l, w13_in, w13_out, pl.E, intermediate_in, pl.I, pl.H, pl.gated, elt);
+  if (e == cudaSuccess) e = moe::launch_prepare_w2(l, w2_in, w2_out, pl.E, pl.H, intermediate_in, pl.I, elt);
+  return cuda_status(e);
+}
+
+MOE_API moe_status_t moe_quantize_weights_fp8(const void* w, int64_t num_mats, int32_t rows, int32_t cols,
+                                              void* codes, float* scales, moe_stream_t stream) {
+  if (num_mats < 0 || rows <= 0 || cols <= 0 || rows % 128 != 0 || cols % 128 != 0) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(w) || !aligned16(codes) || !aligned4(scales)) return MOE_ERR_INVALID_ARG;
+  if (num_mats * static_cast<int64_t>(rows / 128) * (cols / 128) >= (1LL << 31)) return MOE_ERR_UNSUPPORTED;
+  if (num_mats == 0) return MOE_OK;
+  int sms = 0;
+  const moe_status_t st = device_sms(&sms);
+  if (st != MOE_OK) return st;
+  Launch l;
+  l.stream = reinterpret_cast<cudaStream_t>(stream);
+  l.pdl = false;
+  return cuda_status(moe::launch_quant_weights(l, w, num_mats, rows, cols, codes, scales));
+}
+
+MOE_API moe_status_t moe_forward(const moe_problem_t* problem, const void* hidden, const float* router_logits,
+                                 const void* w13, const void* w2, const float* w13_scale, const float* w2_scale,
+                                 void* out, void* workspace, size_t workspace_bytes, moe_stream_t stream) {
+  Plan pl;
+  int sms = 0;
+  moe_status_t st = make_plan(problem, &pl);
+  if (st != MOE_OK || pl.T == 0) return st;  // T == 0: nothing to do, pointers unused
+  if (!aligned16(hidden) || !aligned16(router_logits) || !aligned16(out) || hidden == out)
+    return MOE_ERR_INVALID_ARG;
+  st = check_weights(pl, w13, w2, w13_scale, w2_scale);
+  if (st != MOE_OK) return st;
+  st = prologue(problem, workspace, workspace_bytes, &pl, &sms);
+  if (st != MOE_OK || pl.T == 0) return st;
+  return forward_device(pl, problem, hidden, router_logits, w13, w2, w13_scale, w2_scale, out, workspace, stream,
+                        sms);
+}
+
+MOE_API moe_status_t moe_forward_host(const moe_problem_t* problem, const void* h_hidden,
+                                      const float* h_router_logits, const void* w13, const void* w2,
+                                      const float* w13_scale, const float* w2_scale, void* h_out, void* workspace,
+                                      size_t workspace_bytes, moe_stream_t stream) {
+  Plan pl;
+  int sms = 0;
+  moe_status_t st = make_plan(problem, &pl);
+  if (st != MOE_OK || pl.T == 0) return st;  // T == 0: nothing to do, pointers unused
+  if (h_hidden == nullptr || h_router_logits == nullptr || h_out == nullptr) return MOE_ERR_INVALID_ARG;
+  st = check_weights(pl, w13, w2, w13_scale, w2_scale);
+  if (st != MOE_OK) return st;
+  st = prologue(problem, workspace, workspace_bytes, &pl, &sms);
+  if (st != MOE_OK || pl.T == 0) return st;
+  const auto& L = pl.lay;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  void* d_hidden = ws_ptr<void>(workspace, L.io_hidden);
+  float* d_logits = ws_ptr<float>(workspace, L.io_logits);
+  void* d_out = ws_ptr<void>(workspace, L.io_out);
+  const size_t hbytes = static_cast<size_t>(pl.T) * pl.H * 2;
+  if (cudaMemcpyAsync(d_hidden, h_hidden, hbytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(d_logits, h_router_logits, static_cast<size_t>(pl.T) * pl.Er * 4, cudaMemcpyHostToDevice,
+                      s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  st = forward_device(pl, problem, d_hidden, d_logits, w13, w2, w13_scale, w2_scale, d_out, workspace, stream, sms);
+  if (st != MOE_OK) return st;
+  if (cudaMemcpyAsync(h_out, d_out, hbytes, cudaMemcpyDeviceToHost, s) != cudaSuccess) return MOE_ERR_CUDA;
+  return cudaStreamSynchronize(s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+MOE_API moe_status_t moe_stage_route(const moe_problem_t* problem, const float* router_logits, void* workspace,
+                                     size_t workspace_bytes, moe_stream_t stream) {
+  Plan pl;
+  int sms = 0;
+  moe_status_t st = make_plan(problem, &pl);
+  if (st != MOE_OK || pl.T == 0) return st;  // T == 0: nothing to do, pointers unused
+  if (!aligned16(router_logits)) return MOE_ERR_INVALID_ARG;
+  st = prologue(problem, workspace, workspace_bytes, &pl, &sms);
+  if (st != MOE_OK || pl.T == 0) return st;
+  return run_route(pl, router_logits, workspace, launch_of(problem, stream));
+}
+
+MOE_API moe_status_t moe_stage_align(const moe_problem_t* problem, void* workspace, size_t workspace_bytes,
+                                     moe_stream_t stream) {
+  Plan pl;
+  int sms = 0;
+  moe_status_t st = prologue(problem, workspace, workspace_bytes, &pl, &sms);
+  if (st != MOE_OK || pl.T == 0) return st;
+  return run_align(pl, workspace, launch_of(problem, stream));
+}
+
+MOE_API moe_status_t moe_stage_quant_act(const moe_problem_t* problem, const void* hidden, void* workspace,
+                                         size_t workspace_bytes, moe_stream_t stream) {
+  Plan pl;
+  int sms = 0;
+  moe_status_t st = make_plan(problem, &pl);
+  if (st != MOE_OK || pl.T == 0) return st;  // T == 0: nothing to do, pointers unused
+  if (!pl.fp8 || !aligned16(hidden)) return MOE_ERR_INVALID_ARG;
+  st = prologue(problem, workspace, workspace_bytes, &pl, &sms);
+  if (st != MOE_OK || pl.T == 0) return st;
+  return run_quant_act(pl, hidden, workspace, launch_of(problem, stream));
+}
+
+MOE_API moe_status_t moe_stage_gemm1(const moe_problem_t* problem, const void* hidden, const void* w13,
+                                     const float* w13_scale, void* workspace, size_t workspace_bytes,
+                                     moe_stream_t stream) {
+  Plan pl;
+  int sms = 0;
+  moe_status_t st = make_plan(problem, &pl);
+  if (st != MOE_OK || pl.T == 0) return st;  // T == 0: nothing to do, pointers unused
+  if (!aligned16(hidden) || !aligned16(w13) || (pl.fp8 && !aligned4(w13_scale))) return MOE_ERR_INVALID_ARG;
+  st = prologue(problem, workspace, workspace_bytes, &pl, &sms);
+  if (st != MOE_OK || pl.T == 0) return st;
+  return run_gemm1(pl, hidden, w13, w13_scale, workspace, launch_of(problem, stream), sms);
+}
+
+MOE_API moe_status_t moe_stage_gemm2(const moe_problem_t* problem, const void* w2, const float* w2_scale,
+                                     void* workspace, size_t workspace_bytes, moe_stream_t stream) {
+  Plan pl;
+  int sms = 0;
+  moe_status_t st = make_plan(problem, &pl);
+  if (st != MOE_OK || pl.T == 0) return st;  // T == 0: nothing to do, pointers unused
+  if (!aligned16(w2) || (pl.fp8 && !aligned4(w2_scale))) return MOE_ERR_INVALID_ARG;
+  st = prologue(problem, workspace, workspace_bytes, &pl, &sms);
+  if (st != MOE_OK || pl.T == 0) return st;
+  return run_gemm2(pl, w2, w2_scale, workspace, launch_of(problem, stream), sms);
+}
+
+MOE_API moe_status_t moe_stage_combine(const moe_problem_t* problem, void* out, void* workspace,
+                                       size_t workspace_bytes, moe_stream_t stream) {
+  Plan pl;
+  int sms = 0;
+  moe_status_t st = make_plan(problem, &pl);
+  if (st != MOE_OK || pl.T == 0) return st;  // T == 0: nothing to do, pointers unused
+  if (!aligned16(out)) return MOE_ERR_INVALID_ARG;
+  st = prologue(problem, workspace, workspace_bytes, &pl, &sms);
+  if (st != MOE_OK || pl.T == 0) return st;
+  return run_combine(pl, out, workspace, launch_of(problem, stream));
+}
+
+MOE_API moe_status_t moe_get_device_status(void* workspace, moe_stream_t stream, int32_t* detail) {
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MOE_ERR_INVALID_ARG;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int32_t word = 0;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  if (word != 0 && cudaMemset(workspace, 0, sizeof(word)) != cudaSuccess) return MOE_ERR_CUDA;
+  if (detail != nullptr) *detail = word;
+  return word == 0 ? MOE_OK : MOE_ERR_DEVICE_TIMEOUT;
+}

@@ -1,0 +1,85 @@
+// Host-side declarations shared by the kernel files and the C-ABI layer.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+constexpr int kMaxExperts = 1024;  // routed + shared
+constexpr int kMaxSlots = 16;      // k' = topk + num_shared
+constexpr int kAlignChunk = 1024;  // pairs per align chunk
+
+// Launch configuration shared by all launchers.
+struct Launch {
+  cudaStream_t stream;
+  bool pdl;
+};
+
+// Fill `cfg` (grid, block, smem, stream) and the PDL attribute in `attr`.
+void make_launch_config(cudaLaunchConfig_t* cfg, cudaLaunchAttribute* attr, const Launch& l,
+                        dim3 grid, dim3 block, size_t smem);
+
+// ---- route (route.cu) ----
+cudaError_t launch_route(const Launch& l, const float* logits, int T, int E_routed, int topk,
+                         int num_shared, int renormalize, int* topk_ids, float* topk_w,
+                         int* status);
+
+// ---- align (align.cu) ----
+cudaError_t launch_align(const Launch& l, const int* topk_ids, int P, int E, int block_m,
+                         int num_chunks, int* chunk_hist, int* sorted_pair_ids,
+                         int* expert_offsets, int* block_expert, int* pair_to_row,
+                         int* num_blocks);
+
+// ---- GEMMs (gemm_bf16.cu, gemm_fp8.cu) ----
+struct GemmShape {
+  int K;                  // reduction length
+  int N;                  // output columns of the GEMM (N1 or H)
+  int BN;                 // N tile
+  int w_rows_per_expert;  // rows per expert in the 2-D weight tensor map
+  int k_total;            // slots per token (k')
+  int num_pairs;          // P
+  int activation;         // moe_activation_t (GEMM1)
+  int out_cols;           // leading dimension of the output (I for act, H for y)
+  int num_sms;
+};
+struct GemmBuffers {
+  const int* num_blocks;
+  const int* block_expert;
+  const int* sorted_pair_ids;
+  const float* topk_w;
+  void* out;
+  float* out_scale;         // FP8 GEMM1: act scales [max_rows, I/128]
+  const float* a_scale;     // FP8: activation scales of the A operand
+  const float* w_scale;     // FP8: weight block scales
+  int a_scale_cols;         // FP8: columns of a_scale (K/128)
+  int w_scale_rows;         // FP8: rows of w_scale per expert
+  int w_scale_cols;         // FP8: columns of w_scale (K/128)
+  int up_block_offset;      // FP8 GEMM1: row-block offset of the up half (I/128)
+  int* status;
+};
+int pick_bn(int N, bool gated);
+size_t gemm_bf16_smem_bytes();
+cudaError_t launch_gemm1_bf16(const Launch& l, const CUtensorMap& tm_hidden,
+                              const CUtensorMap& tm_w13, const GemmShape& s,
+                              const GemmBuffers& b);
+cudaError_t launch_gemm2_bf16(const Launch& l, const CUtensorMap& tm_act, const CUtensorMap& tm_w2,
+                              const GemmShape& s, const GemmBuffers& b);
+size_t gemm_fp8_smem_bytes();
+cudaError_t launch_gemm1_fp8(const Launch& l, const CUtensorMap& tm_xq, const CUtensorMap& tm_w13,
+                             const GemmShape& s, const GemmBuffers& b);
+cudaError_t launch_gemm2_fp8(const Launch& l, const CUtensorMap& tm_actq, const CUtensorMap& tm_w2,
+                             const GemmShape& s, const GemmBuffers& b);
+
+// ---- elementwise (combine.cu, quant.cu, prepare.cu) ----
+cudaError_t launch_combine(const Launch& l, const void* y, int T, int k_total, int H, void* out);
+cudaError_t launch_quant_act(const Launch& l, const void* x, int T, int H, void* q, float* scale);
+cudaError_t launch_quant_weights(const Launch& l, const void* w, int64_t num_mats, int rows,
+                                 int cols, void* q, float* scale);
+cudaError_t launch_prepare_w13(const Launch& l, const void* in, void* out, int E, int I_in,
+                               int I_pad, int H, int gated, int elt_bytes);
+cudaError_t launch_prepare_w2(const Launch& l, const void* in, void* out, int E, int H, int I_in,
+                              int I_pad, int elt_bytes);
+
+}  // namespace moe

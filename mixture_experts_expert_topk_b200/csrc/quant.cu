@@ -1,0 +1,116 @@
+// FP8 E4M3 quantisers for the W8A8 block-128 configuration ("Qwen3-Next FP8 MoE
+// optimisation: shared-expert fusion for H200", sglang PR 26204, section 1:
+// dtype=fp8_w8a8, block_shape=[128, 128]).
+//
+//   activations: one fp32 scale per token per 128 consecutive columns (1x128 groups);
+//   weights:     one fp32 scale per 128x128 block.
+// In both, scale = amax / 448 (IEEE fp32 division), or 1 for an all-zero group, and
+// code = e4m3(x / scale) with IEEE fp32 division, round to nearest even, saturating at
+// +-448 (cvt ... .satfinite). The oracle takes the same decisions in the same
+// precision, so the codes and scales are compared bit for bit.
+#include <cuda_fp8.h>
+
+#include "moe_device.cuh"
+#include "moe_internal.h"
+
+namespace moe {
+namespace {
+
+__device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
+  const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+  const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(make_float2(c, d), __NV_SATFINITE, __NV_E4M3);
+  return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+}
+
+// One warp per (token, 128-column group): lane l quantises columns 4l..4l+3.
+__global__ void __launch_bounds__(256)
+    quant_act_kernel(const uint2* __restrict__ x, int T, int G, uint32_t* __restrict__ q,
+                     float* __restrict__ scale) {
+  griddep_wait();
+  const long long g = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (g >= static_cast<long long>(T) * G) return;
+  const int lane = threadIdx.x & 31;
+  const uint2 raw = x[g * 32 + lane];
+  const float2 f01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.x));
+  const float2 f23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.y));
+  float amax = fmaxf(fmaxf(fabsf(f01.x), fabsf(f01.y)), fmaxf(fabsf(f23.x), fabsf(f23.y)));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  const float s = amax == 0.f ? 1.f : __fdiv_rn(amax, 448.f);
+  q[g * 32 + lane] = e4m3x4(__fdiv_rn(f01.x, s), __fdiv_rn(f01.y, s), __fdiv_rn(f23.x, s),
+                            __fdiv_rn(f23.y, s));
+  if (lane == 0) scale[g] = s;
+}
+
+// One CTA of 256 threads per 128x128 block: thread t covers 64 columns of row t/2.
+__global__ void __launch_bounds__(256)
+    quant_weights_kernel(const uint4* __restrict__ w, int rows, int cols, uint2* __restrict__ q,
+                         float* __restrict__ scale) {
+  __shared__ float red[8];
+  griddep_wait();
+  const int rb = rows / 128, cb = cols / 128;
+  const long long blk = blockIdx.x;
+  const long long mat = blk / (static_cast<long long>(rb) * cb);
+  const int rem = static_cast<int>(blk - mat * rb * cb);
+  const int bi = rem / cb, bj = rem - (rem / cb) * cb;
+  const int r = bi * 128 + (threadIdx.x >> 1);
+  const int c0 = bj * 128 + (threadIdx.x & 1) * 64;
+  const long long base = (mat * rows + r) * static_cast<long long>(cols) + c0;  // element index
+  float v[64];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint4 u = w[base / 8 + i];
+    const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 f = __bfloat1622float2(b[k]);
+      v[8 * i + 2 * k] = f.x;
+      v[8 * i + 2 * k + 1] = f.y;
+    }
+  }
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 64; ++i) amax = fmaxf(amax, fabsf(v[i]));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+  __syncthreads();
+  amax = red[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) amax = fmaxf(amax, red[i]);
+  const float s = amax == 0.f ? 1.f : __fdiv_rn(amax, 448.f);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    uint2 o;
+    o.x = e4m3x4(__fdiv_rn(v[8 * i + 0], s), __fdiv_rn(v[8 * i + 1], s), __fdiv_rn(v[8 * i + 2], s),
+                 __fdiv_rn(v[8 * i + 3], s));
+    o.y = e4m3x4(__fdiv_rn(v[8 * i + 4], s), __fdiv_rn(v[8 * i + 5], s), __fdiv_rn(v[8 * i + 6], s),
+                 __fdiv_rn(v[8 * i + 7], s));
+    q[base / 8 + i] = o;
+  }
+  if (threadIdx.x == 0) scale[blk] = s;
+}
+
+}  // namespace
+
+cudaError_t launch_quant_act(const Launch& l, const void* x, int T, int H, void* q, float* scale) {
+  const int G = H / 128;
+  const long long groups = static_cast<long long>(T) * G;
+  cudaLaunchConfig_t cfg;
+  cudaLaunchAttribute attr[1];
+  make_launch_config(&cfg, attr, l, dim3(static_cast<unsigned>((groups + 7) / 8)), dim3(256), 0);
+  return cudaLaunchKernelEx(&cfg, quant_act_kernel, static_cast<const uint2*>(x), T, G,
+                            static_cast<uint32_t*>(q), scale);
+}
+
+cudaError_t launch_quant_weights(const Launch& l, const void* w, int64_t num_mats, int rows, int cols,
+                                 void* q, float* scale) {
+  const long long blocks = num_mats * static_cast<long long>(rows / 128) * (cols / 128);
+  cudaLaunchConfig_t cfg;
+  cudaLaunchAttribute attr[1];
+  make_launch_config(&cfg, attr, l, dim3(static_cast<unsigned>(blocks)), dim3(256), 0);
+  return cudaLaunchKernelEx(&cfg, quant_weights_kernel, static_cast<const uint4*>(w), rows, cols,
+                            static_cast<uint2*>(q), scale);
+}
+
+}  // namespace moe

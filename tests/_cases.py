@@ -1,0 +1,96 @@
+"""Shared helpers for the GPU parity tests: build a case, run the CUDA path through the
+Python binding (C ABI), and evaluate the CPU oracle on the same seeded inputs."""
+from __future__ import annotations
+
+import functools
+from typing import Dict, Optional
+
+import numpy as np
+import torch
+
+import mixture_experts_expert_topk_b200 as moe
+from mixture_experts_expert_topk_b200.synth import CONFIGS, MoeConfig, make_inputs
+from oracle import moe_oracle as O
+
+
+def bits(t: torch.Tensor) -> np.ndarray:
+    """bf16 tensor -> uint16 bit patterns (numpy, CPU)."""
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+@functools.lru_cache(maxsize=4)
+def cpu_inputs(cfg: MoeConfig, seed: int = 0) -> Dict[str, torch.Tensor]:
+    return make_inputs(cfg, seed)
+
+
+class GpuRun:
+    """One forward of ``cfg`` on cuda:0 with every intermediate kept in the workspace."""
+
+    def __init__(self, cfg: MoeConfig, seed: int = 0, inputs: Optional[dict] = None, pdl: bool = True):
+        self.cfg = cfg
+        inp = inputs if inputs is not None else cpu_inputs(cfg, seed)
+        self.inp = inp
+        self.I_pad = moe.padded_intermediate(cfg.I, cfg.activation, cfg.fp8)
+        self.prob = moe.make_problem(cfg.T, cfg.H, cfg.E, cfg.topk, self.I_pad,
+                                     renormalize=cfg.renormalize, activation=cfg.activation,
+                                     num_shared=cfg.num_shared, fp8=cfg.fp8, pdl=pdl)
+        dev = torch.device("cuda:0")
+        self.hidden = inp["hidden"].to(dev)
+        self.logits = inp["logits"].to(dev)
+        w13 = inp["w13"].to(dev)
+        w2 = inp["w2"].to(dev)
+        self.w13_scale = self.w2_scale = None
+        if cfg.fp8:
+            self.w13_q, self.w13_scale = moe.quantize_weights_fp8(w13)
+            self.w2_q, self.w2_scale = moe.quantize_weights_fp8(w2)
+            self.w13p, self.w2p = moe.prepare_weights(self.prob, self.w13_q, self.w2_q, cfg.I)
+        else:
+            self.w13p, self.w2p = moe.prepare_weights(self.prob, w13, w2, cfg.I)
+        del w13, w2
+        self.ws = moe.new_workspace(self.prob)
+        self.out = torch.empty_like(self.hidden)
+
+    def forward(self) -> torch.Tensor:
+        moe.moe_forward(self.hidden, self.logits, self.w13p, self.w2p, self.cfg.topk,
+                        self.cfg.renormalize, self.cfg.activation, self.w13_scale, self.w2_scale,
+                        num_shared=self.cfg.num_shared, workspace=self.ws, out=self.out,
+                        pdl=bool(self.prob.flags & 1))
+        torch.cuda.synchronize()
+        return self.out
+
+    def parts(self) -> Dict[str, np.ndarray]:
+        v = moe.read_workspace(self.prob, self.ws)
+        out = {}
+        for k, t in v.items():
+            if t.dtype == torch.bfloat16:
+                out[k] = bits(t)
+            else:
+                out[k] = t.cpu().numpy()
+        return out
+
+
+def oracle_out(cfg: MoeConfig, inp, tokens=None, fp8_weights=None) -> np.ndarray:
+    if cfg.fp8:
+        q13, s13, q2, s2 = fp8_weights
+        return O.moe_forward_fp8(bits(inp["hidden"]), inp["logits"].numpy(), q13, s13, q2, s2,
+                                 topk=cfg.topk, renormalize=cfg.renormalize,
+                                 activation=cfg.activation, num_shared=cfg.num_shared,
+                                 tokens=tokens)
+    # the oracle takes the checkpoint (unpadded, gate-first) weights
+    w13, w2 = bits(inp["w13"]), bits(inp["w2"])
+    return O.moe_forward(bits(inp["hidden"]), inp["logits"].numpy(), w13, w2, topk=cfg.topk,
+                         renormalize=cfg.renormalize, activation=cfg.activation,
+                         num_shared=cfg.num_shared, tokens=tokens)
+
+
+def bf16_to_f64(t_or_bits) -> np.ndarray:
+    b = bits(t_or_bits) if isinstance(t_or_bits, torch.Tensor) else t_or_bits
+    return O.bf16_bits_to_f64(b)
+
+
+def max_err_over_rms(got: np.ndarray, ref: np.ndarray) -> float:
+    r = O.rms(ref)
+    return float(np.max(np.abs(got - ref)) / r) if r > 0 else float(np.max(np.abs(got - ref)))
+
+
+__all__ = ["CONFIGS", "GpuRun", "bits", "cpu_inputs", "oracle_out", "bf16_to_f64", "max_err_over_rms"]

@@ -1,0 +1,162 @@
+"""Host-side checks of the C ABI: the library loads, exports every declared entry
+point, and validates arguments before touching the GPU (no kernel runs here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import mixture_experts_expert_topk_b200 as moe
+from mixture_experts_expert_topk_b200 import _capi
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe_b200.h")
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+@pytest.fixture(scope="module")
+def L():
+    if not os.path.exists(_capi.LIB_PATH):
+        from mixture_experts_expert_topk_b200 import build
+        build.build()
+    return moe.lib()
+
+
+def _declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_functions_exported_and_bound(L):
+    names = _declared_functions()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(L, n), n            # exported by the .so
+        assert n in _capi.SIGNATURES, n    # bound by the Python layer
+    assert set(_capi.SIGNATURES) == set(names)
+
+
+def _prob(**kw):
+    base = dict(T=16, H=256, num_routed=8, topk=2, intermediate=512, renormalize=True,
+                activation="swiglu")
+    base.update(kw)
+    T, H, E, k, I = base.pop("T"), base.pop("H"), base.pop("num_routed"), base.pop("topk"), base.pop("intermediate")
+    return moe.make_problem(T, H, E, k, I, **base)
+
+
+def test_check_problem_accepts_the_workloads(L):
+    from mixture_experts_expert_topk_b200.synth import CONFIGS
+    for cfg in CONFIGS.values():
+        p = moe.make_problem(cfg.T, cfg.H, cfg.E, cfg.topk, cfg.I, renormalize=cfg.renormalize,
+                             activation=cfg.activation, num_shared=cfg.num_shared, fp8=cfg.fp8)
+        assert L.moe_check_problem(ctypes.byref(p)) == 0, cfg.name
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(T=-1), 1), (dict(H=0), 1), (dict(H=200), 2), (dict(num_routed=0), 1),
+    (dict(topk=9), 1), (dict(topk=0), 1), (dict(intermediate=500), 1),
+    (dict(intermediate=512, activation="relu2"), 0), (dict(intermediate=528, activation="relu2"), 1),
+    (dict(num_routed=1100, topk=2), 2), (dict(num_routed=32, topk=17), 2),
+    (dict(block_m=64), 2), (dict(intermediate=528, fp8=True), 1),
+])
+def test_check_problem_rejects(L, kw, status):
+    p = _prob(**kw)
+    assert L.moe_check_problem(ctypes.byref(p)) == status
+
+
+def test_check_problem_flags_and_shared(L):
+    p = _prob()
+    p.flags = 0x10
+    assert L.moe_check_problem(ctypes.byref(p)) == 1
+    p = _prob(num_shared=2)
+    assert L.moe_check_problem(ctypes.byref(p)) == 1
+    p = _prob(num_shared=1, topk=8)   # E_r = 8, topk 8 + shared slot
+    assert L.moe_check_problem(ctypes.byref(p)) == 0
+    assert L.moe_check_problem(None) == 1
+
+
+def test_padded_intermediate_follows_page_rule(L):
+    with open(os.path.join(GOLDEN, "padding_rules.txt")) as f:
+        rows = [ln.split() for ln in f if ln.strip() and not ln.startswith("#")]
+    for i_in, gated, i_pad in rows:
+        act = _capi.MOE_ACT_SWIGLU if gated == "1" else _capi.MOE_ACT_RELU2
+        assert L.moe_padded_intermediate(int(i_in), act, 0) == int(i_pad)
+    assert L.moe_padded_intermediate(500, _capi.MOE_ACT_SWIGLU, 1) == 512   # FP8: 128
+    assert L.moe_padded_intermediate(0, 0, 0) == -1
+    assert L.moe_padded_intermediate(16, 7, 0) == -1
+
+
+def test_workspace_layout(L):
+    from mixture_experts_expert_topk_b200.synth import CONFIGS
+    for cfg in CONFIGS.values():
+        p = moe.make_problem(cfg.T, cfg.H, cfg.E, cfg.topk, cfg.I, renormalize=cfg.renormalize,
+                             activation=cfg.activation, num_shared=cfg.num_shared, fp8=cfg.fp8)
+        lay = moe.workspace_layout(p)
+        P = cfg.T * cfg.k_total
+        E = cfg.E_total
+        assert lay["status"] == 0
+        assert lay["max_rows"] == -(-(P + min(E, P) * 127) // 128) * 128
+        assert lay["num_chunks"] == -(-P // 1024)
+        offs = sorted(v for k, v in lay.items() if k not in ("total_bytes", "max_rows", "num_chunks", "block_m"))
+        assert all(o % 1024 == 0 for o in offs)
+        assert lay["y"] + P * cfg.H * 2 <= lay["total_bytes"]
+        assert moe.workspace_size(p) == lay["total_bytes"]
+    bad = _prob(H=0)
+    assert L.moe_workspace_size(ctypes.byref(bad)) == 0
+
+
+def test_entry_points_validate_before_any_cuda_call(L):
+    p = _prob()
+    n = moe.workspace_size(p)
+    fake = ctypes.c_void_p(1 << 20)      # aligned, never dereferenced
+    mis = ctypes.c_void_p((1 << 20) + 4)
+    s = ctypes.c_void_p(0)
+    f = L.moe_forward
+    # null / misaligned pointers
+    assert f(ctypes.byref(p), None, fake, fake, fake, None, None, fake, fake, n, s) == 1
+    assert f(ctypes.byref(p), mis, fake, fake, fake, None, None, fake, fake, n, s) == 1
+    # output aliasing the input
+    assert f(ctypes.byref(p), fake, fake, fake, fake, None, None, fake, ctypes.c_void_p(2 << 20), n, s) == 1
+    # workspace too small / misaligned
+    ws = ctypes.c_void_p(4 << 20)
+    assert f(ctypes.byref(p), fake, fake, fake, fake, None, None, ctypes.c_void_p(3 << 20), ws, n - 1, s) == 3
+    assert f(ctypes.byref(p), fake, fake, fake, fake, None, None, ctypes.c_void_p(3 << 20),
+             ctypes.c_void_p((4 << 20) + 16), n, s) == 1
+    # FP8 without scales
+    p8 = _prob(fp8=True)
+    n8 = moe.workspace_size(p8)
+    assert f(ctypes.byref(p8), fake, fake, fake, fake, None, None, ctypes.c_void_p(3 << 20), ws, n8, s) == 1
+    # T == 0: valid, nothing enqueued, no device needed
+    p0 = _prob(T=0)
+    n0 = moe.workspace_size(p0)
+    assert f(ctypes.byref(p0), fake, fake, fake, fake, None, None, ctypes.c_void_p(3 << 20), ws, n0, s) == 0
+    # invalid problem
+    pb = _prob(topk=0)
+    assert f(ctypes.byref(pb), fake, fake, fake, fake, None, None, ctypes.c_void_p(3 << 20), ws, n, s) == 1
+    # stages and helpers
+    assert L.moe_stage_route(ctypes.byref(p), None, ws, n, s) == 1
+    assert L.moe_stage_align(ctypes.byref(p), ws, n - 1, s) == 3
+    assert L.moe_stage_quant_act(ctypes.byref(p), fake, ws, n, s) == 1          # bf16 problem
+    assert L.moe_stage_gemm1(ctypes.byref(p), None, fake, None, ws, n, s) == 1
+    assert L.moe_stage_gemm2(ctypes.byref(p8), fake, None, ws, n8, s) == 1       # FP8 needs scales
+    assert L.moe_stage_combine(ctypes.byref(p), None, ws, n, s) == 1
+    assert L.moe_forward_host(ctypes.byref(p), None, fake, fake, fake, None, None, fake, ws, n, s) == 1
+    assert L.moe_prepare_weights(ctypes.byref(p), 300, fake, fake, fake, fake, s) == 1   # pads to 304 != 512
+    assert L.moe_quantize_weights_fp8(fake, 1, 100, 128, fake, fake, s) == 1
+    assert L.moe_quantize_weights_fp8(fake, 0, 128, 128, fake, fake, s) == 0
+    assert L.moe_get_device_status(None, s, None) == 1
+
+
+def test_status_strings(L):
+    for code, name in [(0, "MOE_OK"), (1, "MOE_ERR_INVALID_ARG"), (2, "MOE_ERR_UNSUPPORTED"),
+                       (3, "MOE_ERR_WORKSPACE_TOO_SMALL"), (4, "MOE_ERR_CUDA"),
+                       (5, "MOE_ERR_DEVICE_TIMEOUT")]:
+        assert L.moe_status_string(code).decode() == name
+
+
+def test_python_layer_fails_loudly_without_a_gpu_tensor():
+    import torch
+    with pytest.raises(ValueError):
+        moe.moe_forward(torch.zeros(4, 256, dtype=torch.bfloat16), torch.zeros(4, 8),
+                        torch.zeros(1), torch.zeros(1), 2, True, "swiglu")
