@@ -1,0 +1,387 @@
+"""Benchmark of the fused MoE layer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config NAME]
+
+One step = one full layer forward (route, align, GEMM1+activation, GEMM2+weight,
+combine) over one batch of the workload, inputs resident in HBM. The default workload
+is the prefill configuration: bf16 SwiGLU, T=4096 tokens, H=2048, 256 experts, top-8,
+I=512, renormalised routing with a per-expert logit bias (skewed expert load).
+Synthetic seeded data, random-init weights.
+
+Timing: W untimed warm-up steps, then exactly K steps bracketed by a barrier and
+cuda.synchronize; each step is timed with CUDA events on the launching stream, with L2
+flushed (a 512 MB write) before every step outside the events. For N > 1 each rank runs
+an independent replica (the layer needs no exchange between replicas) and the time is
+the max over ranks. Rank 0 prints one JSON line.
+
+``--impl reference`` times the CPU oracle (the plain float64 restatement of the method)
+on a bounded sample of the same workload on the host cores, as the reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from mixture_experts_expert_topk_b200.synth import CONFIGS, MoeConfig, make_inputs  # noqa: E402
+
+L2_FLUSH_BYTES = 512 << 20
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d.get("hbm_gbs", 6650.0), d.get("bf16_tflops", 1590.0), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+def _workload_name(cfg: MoeConfig) -> str:
+    act = "SwiGLU" if cfg.gated else "relu2"
+    dt = "FP8 e4m3 W8A8 block-128" if cfg.fp8 else "bf16"
+    sh = f"+{cfg.num_shared} shared" if cfg.num_shared else ""
+    return (f"{cfg.name}: {dt} {act} MoE layer forward, T={cfg.T} H={cfg.H} E={cfg.E}{sh} "
+            f"top-{cfg.topk}{sh} I={cfg.I}")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for ln in f:
+                parts = [p.strip() for p in ln.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax = float(parts[2])
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def _dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    """Max of a per-rank scalar over all ranks (identity for one rank)."""
+    if world <= 1:
+        return x
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def touched_expert_bytes(ids: np.ndarray, cfg: MoeConfig, elt: int):
+    touched = np.unique(ids)
+    w13 = len(touched) * cfg.N1 * cfg.H * elt
+    w2 = len(touched) * cfg.H * cfg.I * elt
+    return len(touched), w13, w2
+
+
+# ---------------------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------------------
+
+def run_ours(cfg: MoeConfig, steps: int, warmup: int, world: int, rank: int, local: int, args):
+    import mixture_experts_expert_topk_b200 as moe
+    dev = torch.device("cuda", local)
+    inp = make_inputs(cfg, seed=0)
+    I_pad = moe.padded_intermediate(cfg.I, cfg.activation, cfg.fp8)
+    prob = moe.make_problem(cfg.T, cfg.H, cfg.E, cfg.topk, I_pad, renormalize=cfg.renormalize,
+                            activation=cfg.activation, num_shared=cfg.num_shared, fp8=cfg.fp8)
+    hidden = inp["hidden"].to(dev)
+    logits = inp["logits"].to(dev)
+    s13 = s2 = None
+    w13 = inp["w13"].to(dev)
+    w2 = inp["w2"].to(dev)
+    if cfg.fp8:
+        w13, s13 = moe.quantize_weights_fp8(w13)
+        w2, s2 = moe.quantize_weights_fp8(w2)
+    w13p, w2p = moe.prepare_weights(prob, w13, w2, cfg.I)
+    del w13, w2
+    ws = moe.new_workspace(prob, dev)
+    out = torch.empty_like(hidden)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    torch.cuda.synchronize(dev)
+
+    def step():
+        moe.moe_forward(hidden, logits, w13p, w2p, cfg.topk, cfg.renormalize, cfg.activation,
+                        s13, s2, num_shared=cfg.num_shared, workspace=ws, out=out)
+
+    for _ in range(warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    st = moe.device_status(ws)
+    if st[0] != 0:
+        raise RuntimeError(f"device status after warm-up: {st}")
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        for i in range(steps):
+            flush.zero_()
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = max_over_ranks(sum(step_ms), world)
+    clocks = clk.summary()
+
+    # per-kernel breakdown: the same kernels through the per-step entry points, events
+    # between the steps on the launching stream
+    names = ["route", "align"] + (["quant_act"] if cfg.fp8 else []) + ["gemm1", "gemm2", "combine"]
+    per = {n: [] for n in names}
+    for _ in range(steps):
+        flush.zero_()
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
+        evs[0].record(stream)
+        k = 0
+        moe.stage_route(prob, logits, ws); k += 1; evs[k].record(stream)
+        moe.stage_align(prob, ws); k += 1; evs[k].record(stream)
+        if cfg.fp8:
+            moe.stage_quant_act(prob, hidden, ws); k += 1; evs[k].record(stream)
+        moe.stage_gemm1(prob, hidden, w13p, ws, s13); k += 1; evs[k].record(stream)
+        moe.stage_gemm2(prob, w2p, ws, s2); k += 1; evs[k].record(stream)
+        moe.stage_combine(prob, out, ws); k += 1; evs[k].record(stream)
+        torch.cuda.synchronize(dev)
+        for i, n in enumerate(names):
+            per[n].append(evs[i].elapsed_time(evs[i + 1]))
+    kernel_ms = {n: statistics.mean(v) for n, v in per.items()}
+
+    # e2e through the public API with host buffers (pinned), copies inside the timed region
+    h_hidden = inp["hidden"].pin_memory()
+    h_logits = inp["logits"].pin_memory()
+    h_out = torch.empty_like(inp["hidden"]).pin_memory()
+    for _ in range(max(1, warmup // 2)):
+        moe.moe_forward_host(prob, h_hidden, h_logits, w13p, w2p, h_out, ws, s13, s2)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    e2e_ms = []
+    for _ in range(steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        moe.moe_forward_host(prob, h_hidden, h_logits, w13p, w2p, h_out, ws, s13, s2)
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms.append(a.elapsed_time(b))
+    barrier(world)
+    e2e_total = max_over_ranks(sum(e2e_ms), world)
+
+    # routing statistics for the algorithmic byte counts
+    ids = moe.read_workspace(prob, ws)["topk_ids"].cpu().numpy()
+    return {
+        "total_ms": total_ms, "step_ms": step_ms, "kernel_ms": kernel_ms, "clocks": clocks,
+        "e2e_total_ms": e2e_total, "ids": ids, "inp": inp,
+        "h2d": h_hidden.numel() * 2 + h_logits.numel() * 4, "d2h": h_out.numel() * 2,
+        "launches_per_step": len(names) + 2,  # align is three kernels
+    }
+
+
+def cpu_baseline(cfg: MoeConfig, inp, budget_s: float, tokens_hint: int):
+    """Time the CPU oracle, as it stands, on the first tokens of the workload."""
+    from oracle import moe_oracle as O
+
+    def bits(t):
+        return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+    hb, lg = bits(inp["hidden"]), inp["logits"].numpy()
+    w13b, w2b = bits(inp["w13"]), bits(inp["w2"])
+    fp8w = O.quantize_weights_fp8(w13b, w2b) if cfg.fp8 else None
+    n = max(1, min(cfg.T, tokens_hint))
+    tok = np.arange(n)
+    t0 = time.perf_counter()
+    if cfg.fp8:
+        O.moe_forward_fp8(hb, lg, *fp8w, topk=cfg.topk, renormalize=cfg.renormalize,
+                          activation=cfg.activation, num_shared=cfg.num_shared, tokens=tok)
+    else:
+        O.moe_forward(hb, lg, w13b, w2b, topk=cfg.topk, renormalize=cfg.renormalize,
+                      activation=cfg.activation, num_shared=cfg.num_shared, tokens=tok)
+    dt = time.perf_counter() - t0
+    flops = cfg.flops() * n / cfg.T
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count() or 1
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"first {n} of {cfg.T} tokens (routing, both GEMMs, combine), float64 NumPy",
+            "seconds": dt}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default="prefill", choices=sorted(CONFIGS))
+    ap.add_argument("--cpu-tokens", type=int, default=256)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    cfg = CONFIGS[args.config]
+    if args.impl == "reference":
+        # the reference arm runs on rank 0's host cores only; other ranks exit at once
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank, local = int(os.environ.get("RANK", "0")), 0
+    else:
+        world, rank, local = _dist_setup(args.gpus)
+    flops = cfg.flops()
+    metric = "fused MoE layer forward throughput (TFLOP/s; us/call in ms_per_step)"
+    base = {"metric": metric, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "fp8_e4m3" if cfg.fp8 else "bf16", "data": "synthetic"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        inp = make_inputs(cfg, seed=0)
+        times, vals = [], []
+        per_step = max(8, args.cpu_tokens // 8)   # a few seconds of host work per step
+        for _ in range(args.warmup):
+            cpu_baseline(cfg, inp, 0, per_step)
+        for _ in range(args.steps):
+            r = cpu_baseline(cfg, inp, 0, per_step)
+            times.append(r["seconds"])
+            vals.append(r["value"])
+        v = sum(vals) / len(vals)
+        line = dict(base)
+        line.update({"impl": "reference", "value": v, "n_gpus": world,
+                     "ms_per_step": 1000.0 * sum(times) / len(times),
+                     "config": {"workload": _workload_name(cfg),
+                                "sample_tokens": per_step, "l2": "n/a (host)"},
+                     "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": r["cores"],
+                                      "kind": "oracle", "sample": r["sample"]},
+                     "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                             "d2h_bytes_per_step": 0},
+                     "gpu_launches": 0})
+        print(json.dumps(line))
+        return
+
+    r = run_ours(cfg, args.steps, args.warmup, world, rank, local, args)
+    ms_per_step = r["total_ms"] / args.steps
+    value = flops * world / (r["total_ms"] / args.steps / 1e3) / 1e12
+    e2e_value = flops * world / (r["e2e_total_ms"] / args.steps / 1e3) / 1e12
+    hbm_peak, tc_peak, peak_kind = _peaks()
+    elt = 1 if cfg.fp8 else 2
+    n_touched, w13_bytes, w2_bytes = touched_expert_bytes(r["ids"], cfg, elt)
+    P = cfg.T * cfg.k_total
+    # GEMM1 algorithmic bytes per launch: touched w13, hidden rows read once, act written
+    g1_bytes = w13_bytes + cfg.T * cfg.H * elt + P * cfg.I * elt
+    g1_ms = r["kernel_ms"]["gemm1"]
+    g1_gbs = g1_bytes / (g1_ms / 1e3) / 1e9
+    minimal_bytes = w13_bytes + w2_bytes + cfg.T * cfg.H * 2 * 2 + cfg.T * cfg.E * 4
+    layer_gbs = minimal_bytes / (ms_per_step / 1e3) / 1e9
+    line = dict(base)
+    line.update({
+        "value": value, "ms_per_step": ms_per_step,
+        "us_per_call": ms_per_step * 1e3,
+        "config": {"workload": _workload_name(cfg), "T": cfg.T, "H": cfg.H, "E": cfg.E_total,
+                   "topk": cfg.k_total, "I": cfg.I,
+                   "l2": "flushed before every step (512 MB write, outside the events)"},
+        "clocks": r["clocks"],
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": r["h2d"],
+                "d2h_bytes_per_step": r["d2h"]},
+        "gpu_launches": r["launches_per_step"] * args.steps,
+        "roofline": {"bound": "hbm", "kernel": "gemm1 (grouped up-GEMM + activation)",
+                     "achieved": g1_gbs, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": g1_gbs / hbm_peak, "traffic": None,
+                     "peak_source": f"{peak_kind} hbm_gbs",
+                     "algorithmic_bytes_per_launch": g1_bytes, "avg_launch_ms": g1_ms},
+        "layer_hbm": {"minimal_bytes": minimal_bytes, "achieved_gbs": layer_gbs,
+                      "frac": layer_gbs / hbm_peak, "touched_experts": n_touched},
+        "tensor_frac": value / tc_peak,
+        "kernel_ms": r["kernel_ms"],
+    })
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cb = cpu_baseline(cfg, r["inp"], 20.0, args.cpu_tokens)
+        cb.pop("seconds")
+        line["cpu_baseline"] = cb
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

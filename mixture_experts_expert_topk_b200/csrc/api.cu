@@ -121,7 +121,7 @@ moe_status_t make_plan(const moe_problem_t* p, Plan* pl) {
   L.xq_scale = take(q.fp8 ? T * (H / 128) * 4 : 0);
   L.act = take(rows * I * (q.fp8 ? 1 : 2));
   L.act_scale = take(q.fp8 ? rows * (I / 128) * 4 : 0);
-  L.y = take(P * H * 2);
+  L.y = take(P * H * 4);
   L.io_hidden = take(T * H * 2);
   L.io_logits = take(T * static_cast<size_t>(q.Er) * 4);
   L.io_out = take(T * H * 2);

@@ -11,7 +11,7 @@
 //
 // GEMM2 (down-GEMM with routing weight): A is the activation in sorted row order, B is
 // w2 of the row tile's expert; the epilogue multiplies row r by topk_w[p] and writes it
-// to row p of y (pair order), ready for the fixed-order combine.
+// in fp32 to row p of y (pair order), ready for the fixed-order combine.
 //
 // Kernel structure (one persistent CTA per SM, 6 warps):
 //   warp 0      TMA producer: B tile (weights, 2-D tiled load) + A tile (gather4 or 2-D)
@@ -55,7 +55,7 @@ struct Args {
   const int* block_expert;
   const int* sorted_pair_ids;
   const float* topk_w;
-  __nv_bfloat16* out;
+  void* out;  // GEMM1: bf16 act [rows, I]; GEMM2: fp32 y [P, H]
   int* status;
 };
 
@@ -221,7 +221,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (a.mode == 0) {
         const bool gated = a.activation == 0;
         const int ncol = gated ? a.BN / 2 : a.BN;
-        __nv_bfloat16* orow = a.out + static_cast<size_t>(grow) * a.out_cols + nt * ncol;
+        __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.out) + static_cast<size_t>(grow) * a.out_cols + nt * ncol;
         for (int c = 0; c < a.BN / 32; ++c) {
           uint32_t v[32];
           __syncwarp();  // tcgen05.ld is .sync.aligned
@@ -256,21 +256,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       } else {
+        // y is kept in fp32: rounding it to bf16 before the combine would cost about as
+        // much accuracy as the final bf16 output rounding itself
         const float w = valid ? a.topk_w[pid] : 0.f;
-        __nv_bfloat16* orow = a.out + static_cast<size_t>(valid ? pid : 0) * a.out_cols + nt * a.BN;
+        float* orow = reinterpret_cast<float*>(a.out) + static_cast<size_t>(valid ? pid : 0) * a.out_cols + nt * a.BN;
         for (int c = 0; c < a.BN / 32; ++c) {
           uint32_t v[32];
           __syncwarp();  // tcgen05.ld is .sync.aligned
           tmem_ld32(taddr + c * 32, v);
           tmem_wait_ld();
-          uint32_t o[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i)
-            o[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * w, __uint_as_float(v[2 * i + 1]) * w);
           if (valid) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+            float4* dst = reinterpret_cast<float4*>(orow + c * 32);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+            for (int i = 0; i < 8; ++i)
+              dst[i] = make_float4(__uint_as_float(v[4 * i]) * w, __uint_as_float(v[4 * i + 1]) * w,
+                                   __uint_as_float(v[4 * i + 2]) * w, __uint_as_float(v[4 * i + 3]) * w);
           }
         }
       }
@@ -322,7 +322,7 @@ Args make_args(int mode, const GemmShape& s, const GemmBuffers& b) {
   a.block_expert = b.block_expert;
   a.sorted_pair_ids = b.sorted_pair_ids;
   a.topk_w = b.topk_w;
-  a.out = static_cast<__nv_bfloat16*>(b.out);
+  a.out = b.out;
   a.status = b.status;
   return a;
 }
