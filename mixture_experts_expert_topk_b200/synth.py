@@ -83,6 +83,13 @@ CONFIGS: Dict[str, MoeConfig] = {
 }
 
 
+# A smaller case of the prefill workload for profiler captures: the same shapes per
+# expert (H, I, top-8, about 128 pairs per expert) with 64 experts, so the weights
+# (400 MB) still exceed L2 but a capture holds well under a gigabyte.
+CONFIGS["prefill_e64"] = MoeConfig("prefill_e64", T=1024, H=2048, E=64, topk=8, I=512,
+                                   renormalize=True, activation="swiglu", logit_bias_std=0.5)
+
+
 def decode_config(T: int) -> MoeConfig:
     """Decode-sweep workload: T in {1, 4, 16, 64} tokens, uniform logits."""
     return MoeConfig(f"decode_T{T}", T=T, H=2048, E=256, topk=8, I=512, renormalize=True,
