@@ -123,7 +123,7 @@ typedef struct {
   size_t io_logits;       /* staging for moe_forward_host: fp32 [T, E_r] */
   size_t io_out;          /* staging for moe_forward_host: bf16 [T, H] */
   int64_t max_rows;       /* upper bound of P_pad: round_up(P + min(E,P)*(block_m-1), block_m) */
-  int32_t num_chunks;     /* align chunks of 1024 pairs */
+  int32_t num_chunks;     /* align chunks of 2048 pairs */
   int32_t block_m;
 } moe_workspace_layout_t;
 

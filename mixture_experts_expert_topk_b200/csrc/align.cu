@@ -7,23 +7,109 @@
 // ascending order, then the sentinel P up to the next multiple of block_m; an expert
 // with no pairs has no rows.
 //
-// Deterministic three-pass counting sort, no atomics on positions:
-//   count   one CTA per chunk of 1024 pairs: per-expert histogram of the chunk;
-//   scan    one CTA: per-expert prefix over chunks, padded segment sizes, exclusive
-//           scan over experts -> expert_offsets, block_expert, sentinel padding;
-//   scatter one warp per chunk: walks its chunk in order, 32 pairs at a time; lanes with
-//           the same expert find each other with __match_any_sync and take consecutive
-//           ranks, so the in-chunk order is the pair order.
+// Deterministic counting sort (no atomics decide any position). Pairs are cut into
+// chunks of kAlignChunk; a chunk is handled by 8 warps of 256 consecutive pairs each:
+//   count   per chunk: per-expert histogram (shared-memory atomics; counts only);
+//   scan    one CTA: per-expert exclusive prefix over chunks (chunk histograms staged in
+//           shared memory batch by batch, so no thread walks global memory serially),
+//           padded segment sizes, exclusive scan over experts -> expert_offsets,
+//           block_expert, sentinel padding;
+//   scatter per chunk: each warp counts its 256 pairs per expert, the 8 warp counts are
+//           prefix-summed per expert, then each warp places its pairs 32 at a time; lanes
+//           with the same expert find each other with __match_any_sync and take
+//           consecutive ranks, so the order within an expert is the pair order.
+// With a single chunk (decode-sized batches) the three phases run in one CTA.
+#include <algorithm>
+
 #include "moe_device.cuh"
 #include "moe_internal.h"
 
 namespace moe {
 namespace {
 
-constexpr int kCountThreads = 256;
+constexpr int kWarps = 8;                        // warps per chunk
+constexpr int kPairsPerWarp = kAlignChunk / kWarps;  // 256
+constexpr int kIdsPerLane = kPairsPerWarp / 32;  // 8
 constexpr int kScanThreads = 1024;
+constexpr int kScanSmemInts = 40960;             // 160 KB of chunk-histogram staging
 
-__global__ void __launch_bounds__(kCountThreads)
+static_assert(kPairsPerWarp % 32 == 0, "warp slices are whole 32-pair steps");
+
+// Load this warp's pair ids (p = base + 32 i + lane); -1 marks pairs past the end.
+__device__ __forceinline__ void load_ids(const int* ids, int base, int end, int lane, int (&e)[kIdsPerLane]) {
+#pragma unroll
+  for (int i = 0; i < kIdsPerLane; ++i) {
+    const int p = base + 32 * i + lane;
+    e[i] = p < end ? ids[p] : -1;
+  }
+}
+
+// Per-expert counts of this warp's pairs into cnt[] (shared; one writer per expert per step).
+__device__ __forceinline__ void warp_count(const int (&e)[kIdsPerLane], int lane, int* cnt) {
+#pragma unroll
+  for (int i = 0; i < kIdsPerLane; ++i) {
+    const unsigned peers = __match_any_sync(0xffffffffu, e[i]);
+    if (e[i] >= 0 && lane == 31 - __clz(peers)) cnt[e[i]] += __popc(peers);
+    __syncwarp();
+  }
+}
+
+// Place this warp's pairs: next[] holds each expert's next free row for this warp.
+__device__ __forceinline__ void warp_place(const int (&e)[kIdsPerLane], int base, int lane, int* next,
+                                           int* sorted_pair_ids, int* pair_to_row) {
+  const unsigned lt = (1u << lane) - 1u;
+#pragma unroll
+  for (int i = 0; i < kIdsPerLane; ++i) {
+    const unsigned peers = __match_any_sync(0xffffffffu, e[i]);
+    if (e[i] >= 0) {
+      const int p = base + 32 * i + lane;
+      const int pos = next[e[i]] + __popc(peers & lt);
+      sorted_pair_ids[pos] = p;
+      pair_to_row[p] = pos;
+    }
+    __syncwarp();
+    if (e[i] >= 0 && lane == 31 - __clz(peers)) next[e[i]] += __popc(peers);
+    __syncwarp();
+  }
+}
+
+// Exclusive scan of one value per thread over a CTA of up to 1024 threads.
+__device__ __forceinline__ int block_exclusive_scan(int v, int* warp_sums, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int nw = (blockDim.x + 31) >> 5;
+    int w = lane < nw ? warp_sums[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    warp_sums[lane] = w;  // inclusive over warps
+  }
+  __syncthreads();
+  const int excl = incl - v + (warp > 0 ? warp_sums[warp - 1] : 0);
+  if (total) *total = warp_sums[((blockDim.x + 31) >> 5) - 1];
+  __syncthreads();
+  return excl;
+}
+
+// Padded segment of expert e starting at row `off` with `count` pairs: sentinel rows and
+// the expert id of its row tiles.
+__device__ __forceinline__ void write_segment(int e, int off, int count, int padded, int block_m, int P,
+                                              int* sorted_pair_ids, int* block_expert) {
+  for (int r = off + count; r < off + padded; ++r) sorted_pair_ids[r] = P;
+  for (int b = off / block_m; b < (off + padded) / block_m; ++b) block_expert[b] = e;
+}
+
+__global__ void __launch_bounds__(kWarps * 32)
     align_count_kernel(const int* __restrict__ ids, int P, int E, int* __restrict__ chunk_hist) {
   __shared__ int hist[kMaxExperts];
   griddep_wait();
@@ -41,101 +127,146 @@ __global__ void __launch_bounds__(kScanThreads)
     align_scan_kernel(int* __restrict__ chunk_hist, int num_chunks, int E, int P, int block_m,
                       int* __restrict__ sorted_pair_ids, int* __restrict__ expert_offsets,
                       int* __restrict__ block_expert, int* __restrict__ num_blocks) {
-  __shared__ int warp_sums[kScanThreads / 32];
+  extern __shared__ int stage[];  // [batch chunks][E]
+  __shared__ int warp_sums[32];
   griddep_wait();
   const int e = threadIdx.x;  // E <= 1024: one expert per thread
+  const int batch = max(1, kScanSmemInts / E);
   int count = 0;
-  if (e < E) {
-    for (int c = 0; c < num_chunks; ++c) {
-      int* h = chunk_hist + static_cast<size_t>(c) * E + e;
-      const int x = *h;
-      *h = count;  // exclusive prefix of expert e over chunks
-      count += x;
+  for (int c0 = 0; c0 < num_chunks; c0 += batch) {
+    const int nc = min(batch, num_chunks - c0);
+    int* g = chunk_hist + static_cast<size_t>(c0) * E;
+    for (int i = threadIdx.x; i < nc * E; i += blockDim.x) stage[i] = g[i];
+    __syncthreads();
+    if (e < E) {
+      for (int c = 0; c < nc; ++c) {
+        const int x = stage[c * E + e];
+        g[c * E + e] = count;  // exclusive prefix of expert e over chunks
+        count += x;
+      }
     }
+    __syncthreads();
   }
-  const int padded = (count + block_m - 1) / block_m * block_m;
-  // block-wide exclusive scan of `padded` over experts
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int incl = padded;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
-  }
-  if (lane == 31) warp_sums[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    int w = warp_sums[lane];
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, w, o);
-      if (lane >= o) w += y;
-    }
-    warp_sums[lane] = w;  // inclusive over warps
-  }
-  __syncthreads();
-  const int off = incl - padded + (warp > 0 ? warp_sums[warp - 1] : 0);
+  const int padded = e < E ? (count + block_m - 1) / block_m * block_m : 0;
+  int total = 0;
+  const int off = block_exclusive_scan(padded, warp_sums, &total);
   if (e < E) {
     expert_offsets[e] = off;
-    for (int r = off + count; r < off + padded; ++r) sorted_pair_ids[r] = P;
-    for (int b = off / block_m; b < (off + padded) / block_m; ++b) block_expert[b] = e;
-    if (e == E - 1) {
-      expert_offsets[E] = off + padded;
-      *num_blocks = (off + padded) / block_m;
-    }
+    write_segment(e, off, count, padded, block_m, P, sorted_pair_ids, block_expert);
+  }
+  if (threadIdx.x == 0) {
+    expert_offsets[E] = total;
+    *num_blocks = total / block_m;
   }
 }
 
-__global__ void __launch_bounds__(32)
-    align_scatter_kernel(const int* __restrict__ ids, int P, int E,
-                         const int* __restrict__ chunk_hist, const int* __restrict__ expert_offsets,
-                         int* __restrict__ sorted_pair_ids, int* __restrict__ pair_to_row) {
-  __shared__ int next[kMaxExperts];
+__global__ void __launch_bounds__(kWarps * 32)
+    align_scatter_kernel(const int* __restrict__ ids, int P, int E, const int* __restrict__ chunk_hist,
+                         const int* __restrict__ expert_offsets, int* __restrict__ sorted_pair_ids,
+                         int* __restrict__ pair_to_row) {
+  __shared__ int cnt[kWarps][kMaxExperts];
   griddep_wait();
-  const int lane = threadIdx.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int i = threadIdx.x; i < kWarps * E; i += blockDim.x) cnt[i / E][i % E] = 0;
+  const int base = blockIdx.x * kAlignChunk + warp * kPairsPerWarp;
+  int e[kIdsPerLane];
+  load_ids(ids, base, P, lane, e);
+  __syncthreads();
+  warp_count(e, lane, cnt[warp]);
+  __syncthreads();
   const int* h = chunk_hist + static_cast<size_t>(blockIdx.x) * E;
-  for (int e = lane; e < E; e += 32) next[e] = expert_offsets[e] + h[e];
-  __syncwarp();
-  const unsigned lt_mask = (1u << lane) - 1u;
-  const int base = blockIdx.x * kAlignChunk;
-  const int end = min(base + kAlignChunk, P);
-  for (int s = base; s < end; s += 32) {
-    const int p = s + lane;
-    const bool valid = p < end;
-    const int e = valid ? ids[p] : E;  // E never matches a real expert
-    const unsigned peers = __match_any_sync(0xffffffffu, e);
-    const int rank = __popc(peers & lt_mask);
-    int pos = 0;
-    if (valid) {
-      pos = next[e] + rank;
-      sorted_pair_ids[pos] = p;
-      pair_to_row[p] = pos;
+  for (int x = threadIdx.x; x < E; x += blockDim.x) {
+    int run = expert_offsets[x] + h[x];
+    for (int w = 0; w < kWarps; ++w) {
+      const int c = cnt[w][x];
+      cnt[w][x] = run;
+      run += c;
     }
-    __syncwarp();
-    if (valid && lane == 31 - __clz(peers)) next[e] += __popc(peers);
-    __syncwarp();
   }
+  __syncthreads();
+  warp_place(e, base, lane, cnt[warp], sorted_pair_ids, pair_to_row);
 }
+
+// All of align for P <= kAlignChunk in one CTA of kWarps warps.
+__global__ void __launch_bounds__(kWarps * 32)
+    align_single_kernel(const int* __restrict__ ids, int P, int E, int block_m, int* __restrict__ sorted_pair_ids,
+                        int* __restrict__ expert_offsets, int* __restrict__ block_expert,
+                        int* __restrict__ pair_to_row, int* __restrict__ num_blocks) {
+  __shared__ int cnt[kWarps][kMaxExperts];
+  __shared__ int warp_sums[32];
+  griddep_wait();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int i = threadIdx.x; i < kWarps * E; i += blockDim.x) cnt[i / E][i % E] = 0;
+  const int base = warp * kPairsPerWarp;
+  int e[kIdsPerLane];
+  load_ids(ids, base, P, lane, e);
+  __syncthreads();
+  warp_count(e, lane, cnt[warp]);
+  __syncthreads();
+  // experts in groups of blockDim.x: totals, padded sizes, exclusive scan, warp prefixes
+  int carry = 0;
+  for (int x0 = 0; x0 < E; x0 += blockDim.x) {
+    const int x = x0 + threadIdx.x;
+    int count = 0;
+    if (x < E)
+      for (int w = 0; w < kWarps; ++w) count += cnt[w][x];
+    const int padded = x < E ? (count + block_m - 1) / block_m * block_m : 0;
+    int total = 0;
+    const int off = carry + block_exclusive_scan(padded, warp_sums, &total);
+    if (x < E) {
+      expert_offsets[x] = off;
+      write_segment(x, off, count, padded, block_m, P, sorted_pair_ids, block_expert);
+      int run = off;
+      for (int w = 0; w < kWarps; ++w) {
+        const int c = cnt[w][x];
+        cnt[w][x] = run;
+        run += c;
+      }
+    }
+    carry += total;
+  }
+  if (threadIdx.x == 0) {
+    expert_offsets[E] = carry;
+    *num_blocks = carry / block_m;
+  }
+  __syncthreads();
+  warp_place(e, base, lane, cnt[warp], sorted_pair_ids, pair_to_row);
+}
+
+bool g_scan_attr[64] = {};
 
 }  // namespace
 
-cudaError_t launch_align(const Launch& l, const int* topk_ids, int P, int E, int block_m,
-                         int num_chunks, int* chunk_hist, int* sorted_pair_ids,
-                         int* expert_offsets, int* block_expert, int* pair_to_row,
-                         int* num_blocks) {
+cudaError_t launch_align(const Launch& l, const int* topk_ids, int P, int E, int block_m, int num_chunks,
+                         int* chunk_hist, int* sorted_pair_ids, int* expert_offsets, int* block_expert,
+                         int* pair_to_row, int* num_blocks) {
   cudaLaunchConfig_t cfg;
   cudaLaunchAttribute attr[1];
-  make_launch_config(&cfg, attr, l, dim3(num_chunks), dim3(kCountThreads), 0);
+  if (num_chunks == 1) {
+    make_launch_config(&cfg, attr, l, dim3(1), dim3(kWarps * 32), 0);
+    return cudaLaunchKernelEx(&cfg, align_single_kernel, topk_ids, P, E, block_m, sorted_pair_ids,
+                              expert_offsets, block_expert, pair_to_row, num_blocks);
+  }
+  make_launch_config(&cfg, attr, l, dim3(num_chunks), dim3(kWarps * 32), 0);
   cudaError_t err = cudaLaunchKernelEx(&cfg, align_count_kernel, topk_ids, P, E, chunk_hist);
   if (err != cudaSuccess) return err;
-  make_launch_config(&cfg, attr, l, dim3(1), dim3(kScanThreads), 0);
-  err = cudaLaunchKernelEx(&cfg, align_scan_kernel, chunk_hist, num_chunks, E, P, block_m,
-                           sorted_pair_ids, expert_offsets, block_expert, num_blocks);
+  const int batch = std::max(1, kScanSmemInts / E);
+  const size_t smem = static_cast<size_t>(std::min(batch, num_chunks)) * E * sizeof(int);
+  int dev = 0;
+  if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
+  if (dev < 64 && !g_scan_attr[dev]) {
+    err = cudaFuncSetAttribute(align_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kScanSmemInts * static_cast<int>(sizeof(int)));
+    if (err != cudaSuccess) return err;
+    g_scan_attr[dev] = true;
+  }
+  make_launch_config(&cfg, attr, l, dim3(1), dim3(kScanThreads), smem);
+  err = cudaLaunchKernelEx(&cfg, align_scan_kernel, chunk_hist, num_chunks, E, P, block_m, sorted_pair_ids,
+                           expert_offsets, block_expert, num_blocks);
   if (err != cudaSuccess) return err;
-  make_launch_config(&cfg, attr, l, dim3(num_chunks), dim3(32), 0);
-  return cudaLaunchKernelEx(&cfg, align_scatter_kernel, (const int*)topk_ids, P, E,
-                            (const int*)chunk_hist, (const int*)expert_offsets, sorted_pair_ids,
-                            pair_to_row);
+  make_launch_config(&cfg, attr, l, dim3(num_chunks), dim3(kWarps * 32), 0);
+  return cudaLaunchKernelEx(&cfg, align_scatter_kernel, (const int*)topk_ids, P, E, (const int*)chunk_hist,
+                            (const int*)expert_offsets, sorted_pair_ids, pair_to_row);
 }
 
 }  // namespace moe

@@ -257,11 +257,11 @@ moe_status_t run_gemm1(const Plan& pl, const void* hidden, const void* w13, cons
   b.out = ws_ptr<void>(ws, L.act);
   CUtensorMap ta, tb;
   if (!pl.fp8) {
-    if (!make_tmap_2d(&ta, hidden, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, pl.H, pl.T, 64, 1) ||
-        !make_tmap_2d(&tb, w13, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, pl.H,
-                      static_cast<uint64_t>(pl.E) * pl.N1, 64, pl.bn1))
+    // the token rows of hidden are gathered by the kernel itself (no tensor map)
+    if (!make_tmap_2d(&tb, w13, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, pl.H, static_cast<uint64_t>(pl.E) * pl.N1,
+                      64, pl.bn1))
       return MOE_ERR_CUDA;
-    return cuda_status(moe::launch_gemm1_bf16(l, ta, tb, s, b));
+    return cuda_status(moe::launch_gemm1_bf16(l, hidden, tb, s, b));
   }
   if (!make_tmap_2d(&ta, ws_ptr<void>(ws, L.xq), CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, pl.H, pl.T, 128, 1) ||
       !make_tmap_2d(&tb, w13, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, pl.H, static_cast<uint64_t>(pl.E) * pl.N1, 128,

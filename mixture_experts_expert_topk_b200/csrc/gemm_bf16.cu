@@ -3,25 +3,30 @@
 // GEMM1 (up-GEMM with fused activation; "[MoE] SwiGLU fusion into the MoE up-GEMM
 // epilogue", sglang PR 32944, sections 1 and 3): row r of the sorted order belongs to
 // pair p = sorted_pair_ids[r] and expert e = block_expert[r / 128]; its A row is
-// hidden[p / k'], gathered straight from the token-order hidden tensor with TMA
-// gather4. B is the prepared w13 of expert e, whose gate and up rows are interleaved
-// ([gate0, up0, gate1, up1, ...]), so accumulator columns (2j, 2j+1) of a tile hold
-// gate_j and up_j. The epilogue applies silu(gate)*up (or relu2) to the fp32
-// accumulators in registers and writes only the I-wide bf16 activation.
+// hidden[p / k'], gathered straight from the token-order hidden tensor. B is the
+// prepared w13 of expert e, whose gate and up rows are interleaved ([gate0, up0, gate1,
+// up1, ...]), so accumulator columns (2j, 2j+1) of a tile hold gate_j and up_j. The
+// epilogue applies silu(gate)*up (or relu2) to the fp32 accumulators in registers and
+// writes only the I-wide bf16 activation.
 //
 // GEMM2 (down-GEMM with routing weight): A is the activation in sorted row order, B is
 // w2 of the row tile's expert; the epilogue multiplies row r by topk_w[p] and writes it
 // in fp32 to row p of y (pair order), ready for the fixed-order combine.
 //
-// Kernel structure (one persistent CTA per SM, 6 warps):
-//   warp 0      TMA producer: B tile (weights, 2-D tiled load) + A tile (gather4 or 2-D)
-//               into a 4-stage shared-memory ring, 128-byte swizzle, 64 bf16 of K per
-//               stage;
-//   warp 1      TMEM allocator and MMA issuer: tcgen05.mma kind::f16, M=128, N=BN,
-//               K=16, fp32 accumulators in TMEM, double-buffered (2 x 256 columns) so
-//               the epilogue of tile i overlaps the main loop of tile i+1;
-//   warps 2-5   epilogue: tcgen05.ld 32 columns at a time, activation / weighting in
-//               registers, 16-byte global stores.
+// Kernel structure (one persistent CTA per SM, 10 warps):
+//   warps 0-3   GEMM1 A gather: 128 threads copy the tile's 128 token rows, 128 bytes of
+//               K each per stage, with 16-byte cp.async into the 128-byte-swizzled layout
+//               the MMA reads; each thread's copies arrive on the stage's barrier when they
+//               land (cp.async.mbarrier.arrive). A TMA gather4 per 4 rows was measured to
+//               cap the producer at one stage per ~1.3 us; cp.async keeps up with HBM.
+//   warp 4      TMA: B tile (weights, 2-D tiled load, 128-byte swizzle) and, for GEMM2,
+//               the contiguous A tile; 4-stage ring of 48 KB stages;
+//   warp 5      TMEM allocator and MMA issuer: tcgen05.mma kind::f16, M=128, N=BN, K=16,
+//               fp32 accumulators in TMEM, double-buffered (2 x 256 columns) so the
+//               epilogue of tile i overlaps the main loop of tile i+1;
+//   warps 6-9   epilogue: tcgen05.ld 32 columns at a time, activation / weighting in
+//               registers, rows staged through shared memory so global stores are
+//               coalesced whole-row segments.
 // Tiles are (row tile, N tile) pairs, row-tile-major, so the CTAs running at the same
 // time work on neighbouring row tiles of the same experts and share weight tiles in L2.
 #include "moe_device.cuh"
@@ -37,20 +42,29 @@ constexpr int kMaxBN = 256;
 constexpr int kStageA = kBM * kBKBytes;     // 16 KB
 constexpr int kStageB = kMaxBN * kBKBytes;  // 32 KB
 constexpr int kStageBytes = kStageA + kStageB;
-constexpr int kThreads = 192;
+constexpr int kNumAWarps = 4;
+constexpr int kWarpTma = 4;
+constexpr int kWarpMma = 5;
+constexpr int kWarpEpi = 6;
+constexpr int kThreads = 320;
 constexpr int kAccCols = 256;               // TMEM columns per accumulator buffer
 constexpr int kTmemCols = 512;
-constexpr int kBarOffset = kStages * kStageBytes;
+constexpr int kStagePitch = 144;            // epilogue staging row pitch: 128 B + 16 B pad
+constexpr int kStagingBytes = 32 * kStagePitch;
+constexpr int kStagingOffset = kStages * kStageBytes;
+constexpr int kBarOffset = kStagingOffset + 4 * kStagingBytes;
 constexpr int kSmemBytes = kBarOffset + 256 + 1024;  // barriers + 1024-byte alignment slack
 
 // wait sites (device status detail)
-enum : int { kSiteEmpty = 1, kSiteFull = 2, kSiteTmemEmpty = 3, kSiteTmemFull = 4, kSiteDrain = 5 };
+enum : int { kSiteEmpty = 1, kSiteFull = 2, kSiteTmemEmpty = 3, kSiteTmemFull = 4, kSiteEmptyA = 6 };
 
 struct Args {
   int mode;  // 0 = GEMM1 (gather + activation), 1 = GEMM2 (weighted scatter)
   int K, BN, n_tiles, k_blocks;
   int w_rows_per_expert;
   int k_total, num_pairs, activation, out_cols;
+  const uint8_t* a_rows;  // GEMM1: hidden [T, H] bf16
+  int a_row_bytes;        // GEMM1: H * 2
   const int* num_blocks;
   const int* block_expert;
   const int* sorted_pair_ids;
@@ -58,6 +72,11 @@ struct Args {
   void* out;  // GEMM1: bf16 act [rows, I]; GEMM2: fp32 y [P, H]
   int* status;
 };
+
+__device__ __forceinline__ int token_of(const Args& a, int row) {
+  const int pid = a.sorted_pair_ids[row];
+  return pid < a.num_pairs ? pid / a.k_total : 0;  // padding rows read token 0
+}
 
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -76,10 +95,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const bool gather_a = a.mode == 0;
 
   if (threadIdx.x == 0) {
+    // GEMM1: the B copy's expect-tx arrival plus one cp.async arrival per gather thread
+    const uint32_t full_count = gather_a ? 1 + 32 * kNumAWarps : 1;
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(full0 + 8 * s, 1);
+      mbar_init(full0 + 8 * s, full_count);
       mbar_init(empty0 + 8 * s, 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -90,11 +112,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) {
-    prefetch_tmap(&tmA);
+  if (warp == kWarpTma && lane == 0) {
     prefetch_tmap(&tmB);
+    if (!gather_a) prefetch_tmap(&tmA);
   }
-  if (warp == 1) {
+  if (warp == kWarpMma) {
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish();
   }
@@ -107,63 +129,102 @@ __global__ void __launch_bounds__(kThreads, 1)
   griddep_wait();
   const int num_tiles = *a.num_blocks * a.n_tiles;
 
-  if (warp == 0) {
-    // ---------------- TMA producer ----------------
-    const uint64_t pol_w = policy_evict_first();  // weights: streamed once
-    const uint64_t pol_a = policy_evict_last();   // activations: reused across N tiles
-    const uint32_t b_bytes = static_cast<uint32_t>(a.BN) * kBKBytes;
-    int stage = 0;
-    uint32_t phase = 0;
-    long long issued = 0;
-    bool ok = true;
-    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-      const int mb = tile / a.n_tiles;
-      const int nt = tile - mb * a.n_tiles;
-      const int e = a.block_expert[mb];
-      const int brow = e * a.w_rows_per_expert + nt * a.BN;
-      int r[4] = {0, 0, 0, 0};
-      if (a.mode == 0) {
+  if (warp < kNumAWarps) {
+    if (gather_a) {
+      // ---------------- A gather (cp.async) ----------------
+      const int t = threadIdx.x;  // 0..127
+      const int c = t & 7;        // 16-byte chunk of the 128-byte K slice
+      const int r0 = t >> 3;      // rows r0 + 16 i, i = 0..7
+      int stage = 0;
+      uint32_t phase = 0;
+      int tok_next[8];
+      if (static_cast<int>(blockIdx.x) < num_tiles) {
+        const int mb = blockIdx.x / a.n_tiles;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int pid = a.sorted_pair_ids[mb * kBM + lane * 4 + i];
-          r[i] = pid < a.num_pairs ? pid / a.k_total : 0;  // padding rows read token 0
+        for (int i = 0; i < 8; ++i) tok_next[i] = token_of(a, mb * kBM + r0 + 16 * i);
+      }
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        const uint8_t* src[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          src[i] = a.a_rows + static_cast<size_t>(tok_next[i]) * a.a_row_bytes + c * 16;
+        const int next = tile + gridDim.x;
+        if (next < num_tiles) {  // prefetch the next tile's token rows
+          const int mb = next / a.n_tiles;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) tok_next[i] = token_of(a, mb * kBM + r0 + 16 * i);
+        }
+        for (int kb = 0; kb < a.k_blocks; ++kb) {
+          int got = 0;
+          if (lane == 0) got = mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, a.status, kSiteEmptyA);
+          got = __shfl_sync(0xffffffffu, got, 0);
+          if (!got) {
+            ok = false;
+            break;
+          }
+          const uint32_t base = smem_u32(smem + stage * kStageBytes);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int r = r0 + 16 * i;
+            cp_async16(base + r * kBKBytes + ((c ^ (r & 7)) << 4), src[i] + kb * kBKBytes);
+          }
+          cp_async_mbar_arrive(full0 + 8 * stage);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
         }
       }
-      for (int kb = 0; kb < a.k_blocks; ++kb) {
-        int got = 0;
-        if (lane == 0) got = mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, a.status, kSiteEmpty);
-        got = __shfl_sync(0xffffffffu, got, 0);
-        if (!got) {
-          ok = false;
-          break;
+      cp_async_wait_all();  // no copy may land after the CTA exits
+    }
+  } else if (warp == kWarpTma) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      const uint64_t pol_w = policy_evict_first();  // weights: streamed once
+      const uint64_t pol_a = policy_evict_last();   // activations: reused across N tiles
+      const uint32_t bytes = static_cast<uint32_t>(a.BN) * kBKBytes + (gather_a ? 0u : kStageA);
+      int stage = 0;
+      uint32_t phase = 0;
+      long long issued = 0;
+      bool ok = true;
+      int e_next = static_cast<int>(blockIdx.x) < num_tiles ? a.block_expert[blockIdx.x / a.n_tiles] : 0;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        const int mb = tile / a.n_tiles;
+        const int nt = tile - mb * a.n_tiles;
+        const int e = e_next;
+        const int next = tile + gridDim.x;
+        if (next < num_tiles) e_next = a.block_expert[next / a.n_tiles];
+        const int brow = e * a.w_rows_per_expert + nt * a.BN;
+        for (int kb = 0; kb < a.k_blocks; ++kb) {
+          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, a.status, kSiteEmpty)) {
+            ok = false;
+            break;
+          }
+          const uint32_t full = full0 + 8 * stage;
+          const uint32_t a_dst = smem_u32(smem + stage * kStageBytes);
+          mbar_arrive_expect_tx(full, bytes);
+          // GEMM1 streams each weight tile once; GEMM2's weight tiles are short rows
+          // re-read at the next K step, so they keep the normal eviction priority
+          tma_load_2d(a_dst + kStageA, &tmB, full, kb * 64, brow, gather_a ? pol_w : pol_a);
+          if (!gather_a) tma_load_2d(a_dst, &tmA, full, kb * 64, mb * kBM, pol_a);
+          ++issued;
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
         }
-        const uint32_t full = full0 + 8 * stage;
-        const uint32_t a_dst = smem_u32(smem + stage * kStageBytes);
-        const uint32_t b_dst = a_dst + kStageA;
-        if (lane == 0) {
-          mbar_arrive_expect_tx(full, kStageA + b_bytes);
-          tma_load_2d(b_dst, &tmB, full, kb * 64, brow, pol_w);
-          if (a.mode != 0) tma_load_2d(a_dst, &tmA, full, kb * 64, mb * kBM, pol_a);
-        }
-        __syncwarp();
-        if (a.mode == 0)
-          tma_gather4(a_dst + lane * 4 * kBKBytes, &tmA, full, kb * 64, r[0], r[1], r[2], r[3], pol_a);
-        ++issued;
-        if (++stage == kStages) {
-          stage = 0;
-          phase ^= 1u;
+      }
+      if (!ok) {
+        // wait (bounded) for the last copy issued into each stage
+        for (int s = 0; s < kStages; ++s) {
+          if (issued <= s) break;
+          const long long last = issued - 1 - ((issued - 1 - s) % kStages);
+          mbar_wait_drain(full0 + 8 * s, static_cast<uint32_t>((last / kStages) & 1));
         }
       }
     }
-    if (!ok && lane == 0) {
-      // make sure no copy lands in shared memory after the CTA exits
-      for (int s = 0; s < kStages; ++s) {
-        if (issued <= s) break;
-        const long long last = issued - 1 - ((issued - 1 - s) % kStages);
-        mbar_wait_drain(full0 + 8 * s, static_cast<uint32_t>((last / kStages) & 1));
-      }
-    }
-  } else if (warp == 1) {
+  } else if (warp == kWarpMma) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16(kBM, a.BN);
@@ -202,9 +263,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait_drain(drain_bar, 0);
     }
   } else {
-    // ---------------- epilogue (warps 2..5) ----------------
+    // ---------------- epilogue (warps 6..9) ----------------
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
-    const int row = q * 32 + lane;
+    uint8_t* staging = smem + kStagingOffset + (warp - kWarpEpi) * kStagingBytes;
+    const uint32_t staging_u32 = smem_u32(staging);
+    const uint32_t stage_row = staging_u32 + lane * kStagePitch;
+    const bool gated = a.activation == 0;
+    // bytes one row contributes per 32 accumulator columns
+    const int row_bytes = a.mode == 0 ? (gated ? 32 : 64) : 128;
+    const int slots = row_bytes >> 4;  // 16-byte slots per row
+    const int rows_per_iter = 32 / slots;
+    const int my_slot = lane % slots;
     int it = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
       const int acc = it & 1;
@@ -214,64 +283,67 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const int mb = tile / a.n_tiles;
       const int nt = tile - mb * a.n_tiles;
-      const int grow = mb * kBM + row;
-      const int pid = a.sorted_pair_ids[grow];
+      const int grow0 = mb * kBM + q * 32;
+      const int pid = a.sorted_pair_ids[grow0 + lane];
       const bool valid = pid < a.num_pairs;
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * kAccCols;
+      const float w = (a.mode != 0 && valid) ? a.topk_w[pid] : 0.f;
+      // destination of this warp's row `lane` at the tile's first column
+      uint8_t* dst_row;
       if (a.mode == 0) {
-        const bool gated = a.activation == 0;
         const int ncol = gated ? a.BN / 2 : a.BN;
-        __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.out) + static_cast<size_t>(grow) * a.out_cols + nt * ncol;
-        for (int c = 0; c < a.BN / 32; ++c) {
-          uint32_t v[32];
-          __syncwarp();  // tcgen05.ld is .sync.aligned
-          tmem_ld32(taddr + c * 32, v);
-          tmem_wait_ld();
+        dst_row = static_cast<uint8_t*>(a.out) +
+                  (static_cast<size_t>(grow0 + lane) * a.out_cols + static_cast<size_t>(nt) * ncol) * 2;
+      } else {
+        dst_row = static_cast<uint8_t*>(a.out) +
+                  (static_cast<size_t>(valid ? pid : 0) * a.out_cols + static_cast<size_t>(nt) * a.BN) * 4;
+      }
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * kAccCols;
+      for (int c = 0; c < a.BN / 32; ++c) {
+        uint32_t v[32];
+        __syncwarp();  // tcgen05.ld is .sync.aligned; the previous chunk's staging is consumed
+        tmem_ld32(taddr + c * 32, v);
+        tmem_wait_ld();
+        uint32_t o[32];
+        if (a.mode == 0) {
           if (gated) {
-            uint32_t o[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
               const float g0 = __uint_as_float(v[4 * i + 0]), u0 = __uint_as_float(v[4 * i + 1]);
               const float g1 = __uint_as_float(v[4 * i + 2]), u1 = __uint_as_float(v[4 * i + 3]);
               o[i] = pack_bf16x2(silu_f32(g0) * u0, silu_f32(g1) * u1);
             }
-            if (valid) {
-              uint4* dst = reinterpret_cast<uint4*>(orow + c * 16);
-              dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
-              dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
-            }
           } else {
-            uint32_t o[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-              float z0 = fmaxf(__uint_as_float(v[2 * i + 0]), 0.f);
-              float z1 = fmaxf(__uint_as_float(v[2 * i + 1]), 0.f);
+              const float z0 = fmaxf(__uint_as_float(v[2 * i + 0]), 0.f);
+              const float z1 = fmaxf(__uint_as_float(v[2 * i + 1]), 0.f);
               o[i] = pack_bf16x2(z0 * z0, z1 * z1);
             }
-            if (valid) {
-              uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
-#pragma unroll
-              for (int i = 0; i < 4; ++i) dst[i] = make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
-            }
           }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(v[i]) * w);
         }
-      } else {
-        // y is kept in fp32: rounding it to bf16 before the combine would cost about as
-        // much accuracy as the final bf16 output rounding itself
-        const float w = valid ? a.topk_w[pid] : 0.f;
-        float* orow = reinterpret_cast<float*>(a.out) + static_cast<size_t>(valid ? pid : 0) * a.out_cols + nt * a.BN;
-        for (int c = 0; c < a.BN / 32; ++c) {
-          uint32_t v[32];
-          __syncwarp();  // tcgen05.ld is .sync.aligned
-          tmem_ld32(taddr + c * 32, v);
-          tmem_wait_ld();
-          if (valid) {
-            float4* dst = reinterpret_cast<float4*>(orow + c * 32);
+        // row `lane` -> staging (the 144-byte pitch keeps 16-byte stores conflict-free)
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-              dst[i] = make_float4(__uint_as_float(v[4 * i]) * w, __uint_as_float(v[4 * i + 1]) * w,
-                                   __uint_as_float(v[4 * i + 2]) * w, __uint_as_float(v[4 * i + 3]) * w);
-          }
+        for (int s = 0; s < 8; ++s)
+          if (s < slots)
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(stage_row + s * 16),
+                         "r"(o[4 * s]), "r"(o[4 * s + 1]), "r"(o[4 * s + 2]), "r"(o[4 * s + 3])
+                         : "memory");
+        __syncwarp();
+        // staging -> global in whole-row segments: `slots` consecutive lanes share a row
+        for (int r = lane / slots; r < 32; r += rows_per_iter) {
+          const bool rvalid = __shfl_sync(0xffffffffu, valid ? 1 : 0, r) != 0;
+          const unsigned long long rbase =
+              __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(dst_row), r);
+          uint4 x;
+          asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(x.x), "=r"(x.y), "=r"(x.z), "=r"(x.w)
+                       : "r"(staging_u32 + r * kStagePitch + my_slot * 16)
+                       : "memory");
+          if (rvalid)
+            *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(rbase) + c * row_bytes + my_slot * 16) = x;
         }
       }
       tc_fence_before();
@@ -281,7 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kWarpMma) {
     __syncwarp();  // tcgen05.dealloc is .sync.aligned: the whole warp, converged
     tc_fence_after();
     tmem_dealloc(tmem_base, kTmemCols);
@@ -306,7 +378,7 @@ cudaError_t launch(const Launch& l, const CUtensorMap& tmA, const CUtensorMap& t
   return cudaLaunchKernelEx(&cfg, gemm_bf16_kernel, tmA, tmB, args);
 }
 
-Args make_args(int mode, const GemmShape& s, const GemmBuffers& b) {
+Args make_args(int mode, const GemmShape& s, const GemmBuffers& b, const void* a_rows) {
   Args a;
   a.mode = mode;
   a.K = s.K;
@@ -318,6 +390,8 @@ Args make_args(int mode, const GemmShape& s, const GemmBuffers& b) {
   a.num_pairs = s.num_pairs;
   a.activation = s.activation;
   a.out_cols = s.out_cols;
+  a.a_rows = static_cast<const uint8_t*>(a_rows);
+  a.a_row_bytes = s.K * 2;
   a.num_blocks = b.num_blocks;
   a.block_expert = b.block_expert;
   a.sorted_pair_ids = b.sorted_pair_ids;
@@ -338,14 +412,15 @@ int pick_bn(int N, bool gated) {
 
 size_t gemm_bf16_smem_bytes() { return kSmemBytes; }
 
-cudaError_t launch_gemm1_bf16(const Launch& l, const CUtensorMap& tm_hidden, const CUtensorMap& tm_w13,
+cudaError_t launch_gemm1_bf16(const Launch& l, const void* hidden, const CUtensorMap& tm_w13,
                               const GemmShape& s, const GemmBuffers& b) {
-  return launch(l, tm_hidden, tm_w13, make_args(0, s, b), s.num_sms);
+  // the A operand is gathered with cp.async; tmA is not read in this mode
+  return launch(l, tm_w13, tm_w13, make_args(0, s, b, hidden), s.num_sms);
 }
 
 cudaError_t launch_gemm2_bf16(const Launch& l, const CUtensorMap& tm_act, const CUtensorMap& tm_w2,
                               const GemmShape& s, const GemmBuffers& b) {
-  return launch(l, tm_act, tm_w2, make_args(1, s, b), s.num_sms);
+  return launch(l, tm_act, tm_w2, make_args(1, s, b, nullptr), s.num_sms);
 }
 
 }  // namespace moe

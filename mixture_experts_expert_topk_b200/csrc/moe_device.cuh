@@ -122,6 +122,18 @@ __device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map
       "r"(r3), "l"(policy)
       : "memory");
 }
+// 16-byte asynchronous global -> shared copy (L2 only, bypassing L1).
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+// Arrive on `bar` once all cp.async copies issued so far by this thread have landed; the
+// arrival counts against the barrier's expected count (.noinc).
+__device__ __forceinline__ void cp_async_mbar_arrive(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
 __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
@@ -231,6 +243,9 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-__device__ __forceinline__ float silu_f32(float g) { return g / (1.0f + __expf(-g)); }
+// silu(g) = g / (1 + e^-g). The result is rounded to bf16 right after, so the fast
+// division (__fdividef, which returns 0 once the divisor exceeds 2^126, the right limit
+// for very negative g) costs no visible accuracy.
+__device__ __forceinline__ float silu_f32(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
 }  // namespace moe

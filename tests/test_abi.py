@@ -97,7 +97,7 @@ def test_workspace_layout(L):
         E = cfg.E_total
         assert lay["status"] == 0
         assert lay["max_rows"] == -(-(P + min(E, P) * 127) // 128) * 128
-        assert lay["num_chunks"] == -(-P // 1024)
+        assert lay["num_chunks"] == -(-P // 2048)
         offs = sorted(v for k, v in lay.items() if k not in ("total_bytes", "max_rows", "num_chunks", "block_m"))
         assert all(o % 1024 == 0 for o in offs)
         assert lay["y"] + P * cfg.H * 4 <= lay["total_bytes"]

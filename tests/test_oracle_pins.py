@@ -455,3 +455,17 @@ def test_planted_mistakes_are_caught(monkeypatch, mutation):
         monkeypatch.setattr(O, "route", lambda lg, kk, r, s=0: real_route(lg, max(kk - 1, 1), r, s))
     got = O.moe_forward(x, l, w13, w2, topk=k, renormalize=True, activation=act)
     assert np.max(np.abs(got - want)) > 1e-6, mutation
+
+
+def test_half_ulp_bf16_helper():
+    # the tolerance helper used by the parity tests: half the bf16 spacing at |x|
+    import sys
+    sys.path.insert(0, os.path.dirname(__file__))
+    from _cases import half_ulp_bf16
+    assert half_ulp_bf16(np.array([1.0]))[0] == 2.0 ** -8
+    assert half_ulp_bf16(np.array([1.99]))[0] == 2.0 ** -8
+    assert half_ulp_bf16(np.array([-2.0]))[0] == 2.0 ** -7
+    assert half_ulp_bf16(np.array([0.75]))[0] == 2.0 ** -9
+    x = np.random.default_rng(0).standard_normal(100000) * 10.0
+    r = torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.all(np.abs(r - x.astype(np.float32)) <= half_ulp_bf16(x) * (1 + 1e-7))
