@@ -118,7 +118,7 @@ typedef struct {
   size_t xq_scale;        /* FP8: fp32 [T, H/128] */
   size_t act;             /* GEMM1 output [max_rows, I]: bf16, or e4m3 for FP8 */
   size_t act_scale;       /* FP8: fp32 [max_rows, I/128] */
-  size_t y;               /* fp32 [T*k', H]: weighted GEMM2 rows in pair order */
+  size_t y;               /* fp32 [max_rows, H]: weighted GEMM2 rows in sorted order */
   size_t io_hidden;       /* staging for moe_forward_host: bf16 [T, H] */
   size_t io_logits;       /* staging for moe_forward_host: fp32 [T, E_r] */
   size_t io_out;          /* staging for moe_forward_host: bf16 [T, H] */

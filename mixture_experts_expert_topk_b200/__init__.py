@@ -250,7 +250,7 @@ def read_workspace(prob: Problem, workspace: torch.Tensor) -> Dict[str, torch.Te
         "expert_offsets": view(L["expert_offsets"], E + 1, torch.int32),
         "block_expert": view(L["block_expert"], rows // L["block_m"], torch.int32),
         "pair_to_row": view(L["pair_to_row"], P, torch.int32),
-        "y": view(L["y"], P * H, torch.float32).view(P, H),
+        "y": view(L["y"], rows * H, torch.float32).view(rows, H),
     }
     if fp8:
         out["xq"] = view(L["xq"], T * H, torch.uint8).view(T, H)

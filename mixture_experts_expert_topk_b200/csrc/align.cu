@@ -113,6 +113,7 @@ __global__ void __launch_bounds__(kWarps * 32)
     align_count_kernel(const int* __restrict__ ids, int P, int E, int* __restrict__ chunk_hist) {
   __shared__ int hist[kMaxExperts];
   griddep_wait();
+  griddep_launch_dependents();
   for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
   __syncthreads();
   const int base = blockIdx.x * kAlignChunk;
@@ -130,6 +131,7 @@ __global__ void __launch_bounds__(kScanThreads)
   extern __shared__ int stage[];  // [batch chunks][E]
   __shared__ int warp_sums[32];
   griddep_wait();
+  griddep_launch_dependents();
   const int e = threadIdx.x;  // E <= 1024: one expert per thread
   const int batch = max(1, kScanSmemInts / E);
   int count = 0;
@@ -166,6 +168,7 @@ __global__ void __launch_bounds__(kWarps * 32)
                          int* __restrict__ pair_to_row) {
   __shared__ int cnt[kWarps][kMaxExperts];
   griddep_wait();
+  griddep_launch_dependents();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int i = threadIdx.x; i < kWarps * E; i += blockDim.x) cnt[i / E][i % E] = 0;
   const int base = blockIdx.x * kAlignChunk + warp * kPairsPerWarp;
@@ -195,6 +198,7 @@ __global__ void __launch_bounds__(kWarps * 32)
   __shared__ int cnt[kWarps][kMaxExperts];
   __shared__ int warp_sums[32];
   griddep_wait();
+  griddep_launch_dependents();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int i = threadIdx.x; i < kWarps * E; i += blockDim.x) cnt[i / E][i % E] = 0;
   const int base = warp * kPairsPerWarp;

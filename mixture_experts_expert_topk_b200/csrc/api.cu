@@ -121,7 +121,7 @@ moe_status_t make_plan(const moe_problem_t* p, Plan* pl) {
   L.xq_scale = take(q.fp8 ? T * (H / 128) * 4 : 0);
   L.act = take(rows * I * (q.fp8 ? 1 : 2));
   L.act_scale = take(q.fp8 ? rows * (I / 128) * 4 : 0);
-  L.y = take(P * H * 4);
+  L.y = take(rows * H * 4);
   L.io_hidden = take(T * H * 2);
   L.io_logits = take(T * static_cast<size_t>(q.Er) * 4);
   L.io_out = take(T * H * 2);
@@ -172,18 +172,18 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // 2-D tensor map over a row-major [outer, inner] matrix with a {box_inner, box_outer}
-// box, 128-byte swizzle, zero fill out of bounds.
+// box (128-byte swizzle unless stated), zero fill out of bounds.
 bool make_tmap_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elt_bytes, uint64_t inner,
-                  uint64_t outer, uint32_t box_inner, uint32_t box_outer) {
+                  uint64_t outer, uint32_t box_inner, uint32_t box_outer,
+                  CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = encode_fn();
   if (enc == nullptr) return false;
   cuuint64_t dims[2] = {inner, outer};
   cuuint64_t strides[1] = {inner * static_cast<uint64_t>(elt_bytes)};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
-  return enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <typename T>
@@ -257,11 +257,15 @@ moe_status_t run_gemm1(const Plan& pl, const void* hidden, const void* w13, cons
   b.out = ws_ptr<void>(ws, L.act);
   CUtensorMap ta, tb;
   if (!pl.fp8) {
-    // the token rows of hidden are gathered by the kernel itself (no tensor map)
+    // the token rows of hidden are gathered by the kernel itself (no tensor map); the
+    // activation is written in boxes of 32 rows x 16 (SwiGLU) or 32 (relu2) columns
+    CUtensorMap tc;
     if (!make_tmap_2d(&tb, w13, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, pl.H, static_cast<uint64_t>(pl.E) * pl.N1,
-                      64, pl.bn1))
+                      64, pl.bn1) ||
+        !make_tmap_2d(&tc, ws_ptr<void>(ws, L.act), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, pl.I,
+                      static_cast<uint64_t>(L.max_rows), pl.gated ? 16 : 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE))
       return MOE_ERR_CUDA;
-    return cuda_status(moe::launch_gemm1_bf16(l, hidden, tb, s, b));
+    return cuda_status(moe::launch_gemm1_bf16(l, hidden, tb, tc, s, b));
   }
   if (!make_tmap_2d(&ta, ws_ptr<void>(ws, L.xq), CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, pl.H, pl.T, 128, 1) ||
       !make_tmap_2d(&tb, w13, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, pl.H, static_cast<uint64_t>(pl.E) * pl.N1, 128,
@@ -295,11 +299,13 @@ moe_status_t run_gemm2(const Plan& pl, const void* w2, const float* w2_scale, vo
   CUtensorMap ta, tb;
   const uint64_t rows = static_cast<uint64_t>(L.max_rows);
   if (!pl.fp8) {
+    CUtensorMap tc;  // y [max_rows, H] fp32 in sorted row order, boxes of 32 x 32
     if (!make_tmap_2d(&ta, ws_ptr<void>(ws, L.act), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, pl.I, rows, 64, 128) ||
         !make_tmap_2d(&tb, w2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, pl.I, static_cast<uint64_t>(pl.E) * pl.H, 64,
-                      pl.bn2))
+                      pl.bn2) ||
+        !make_tmap_2d(&tc, ws_ptr<void>(ws, L.y), CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, pl.H, rows, 32, 32))
       return MOE_ERR_CUDA;
-    return cuda_status(moe::launch_gemm2_bf16(l, ta, tb, s, b));
+    return cuda_status(moe::launch_gemm2_bf16(l, ta, tb, tc, s, b));
   }
   if (!make_tmap_2d(&ta, ws_ptr<void>(ws, L.act), CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, pl.I, rows, 128, 128) ||
       !make_tmap_2d(&tb, w2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, pl.I, static_cast<uint64_t>(pl.E) * pl.H, 128,
@@ -314,7 +320,8 @@ moe_status_t run_gemm2(const Plan& pl, const void* w2, const float* w2_scale, vo
 }
 
 moe_status_t run_combine(const Plan& pl, void* out, void* ws, const Launch& l) {
-  return cuda_status(moe::launch_combine(l, ws_ptr<void>(ws, pl.lay.y), pl.T, pl.kk, pl.H, out));
+  return cuda_status(moe::launch_combine(l, ws_ptr<void>(ws, pl.lay.y), ws_ptr<int>(ws, pl.lay.pair_to_row), pl.T,
+                                         pl.kk, pl.H, out));
 }
 
 // Common preamble of the entry points that launch: plan, workspace, device.

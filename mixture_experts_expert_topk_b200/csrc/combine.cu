@@ -1,8 +1,9 @@
 // Step 5 of the layer: deterministic combine back to token order.
 //
-// out[t, h] = sum_{j=0}^{k'-1} y[t*k' + j, h], where y (fp32) already carries the
-// routing weight (GEMM2 epilogue). The sum runs in slot order j = 0, 1, ..., k'-1 in fp32
-// and is rounded once to bf16, so the result does not depend on scheduling. The output is bf16
+// out[t, h] = sum_{j=0}^{k'-1} y[pair_to_row[t*k' + j], h], where y (fp32, sorted row
+// order) already carries the routing weight (GEMM2 epilogue). The sum runs in slot order
+// j = 0, 1, ..., k'-1 in fp32 and is rounded once to bf16, so the result does not depend
+// on scheduling. The output is bf16
 // of the hidden shape ("FlashInfer TRTLLM-Gen MoE kernel optimisation: NemotronH
 // support", sglang PR 21321, section 1: the fused op returns a bf16 tensor shaped like
 // hidden_states).
@@ -18,8 +19,10 @@ namespace {
 constexpr int kCombineThreads = 256;
 
 __global__ void __launch_bounds__(kCombineThreads)
-    combine_kernel(const float4* __restrict__ y, int T, int k_total, int H8, uint4* __restrict__ out) {
+    combine_kernel(const float4* __restrict__ y, const int* __restrict__ pair_to_row, int T, int k_total, int H8,
+                   uint4* __restrict__ out) {
   griddep_wait();
+  griddep_launch_dependents();
   const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (idx >= static_cast<long long>(T) * H8) return;
   const long long t = idx / H8;
@@ -27,11 +30,12 @@ __global__ void __launch_bounds__(kCombineThreads)
   float acc[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-  // row (t*k' + j) of y, columns 8c..8c+7 = float4 pair 2c, 2c+1 of that row
-  const float4* src = y + (t * k_total * H8 + c) * 2;
+  const int* rows = pair_to_row + t * k_total;
   for (int j = 0; j < k_total; ++j) {
-    const float4 a = __ldcs(src + static_cast<long long>(j) * H8 * 2);  // read once: streaming
-    const float4 b = __ldcs(src + static_cast<long long>(j) * H8 * 2 + 1);
+    // columns 8c..8c+7 of y row pair_to_row[t*k' + j] = float4 pair 2c, 2c+1 of that row
+    const float4* src = y + (static_cast<long long>(__ldg(rows + j)) * H8 + c) * 2;
+    const float4 a = __ldcs(src);  // read once: streaming
+    const float4 b = __ldcs(src + 1);
     acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
     acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
   }
@@ -45,14 +49,15 @@ __global__ void __launch_bounds__(kCombineThreads)
 
 }  // namespace
 
-cudaError_t launch_combine(const Launch& l, const void* y, int T, int k_total, int H, void* out) {
+cudaError_t launch_combine(const Launch& l, const void* y, const int* pair_to_row, int T, int k_total, int H,
+                           void* out) {
   const int H8 = H / 8;
   const long long n = static_cast<long long>(T) * H8;
   cudaLaunchConfig_t cfg;
   cudaLaunchAttribute attr[1];
   make_launch_config(&cfg, attr, l, dim3(static_cast<unsigned>((n + kCombineThreads - 1) / kCombineThreads)),
                      dim3(kCombineThreads), 0);
-  return cudaLaunchKernelEx(&cfg, combine_kernel, static_cast<const float4*>(y), T, k_total, H8,
+  return cudaLaunchKernelEx(&cfg, combine_kernel, static_cast<const float4*>(y), pair_to_row, T, k_total, H8,
                             static_cast<uint4*>(out));
 }
 

@@ -11,7 +11,8 @@
 //
 // GEMM2 (down-GEMM with routing weight): A is the activation in sorted row order, B is
 // w2 of the row tile's expert; the epilogue multiplies row r by topk_w[p] and writes it
-// in fp32 to row p of y (pair order), ready for the fixed-order combine.
+// in fp32 to row r of y (sorted order); the fixed-order combine gathers it back through
+// pair_to_row.
 //
 // Kernel structure (one persistent CTA per SM, 10 warps):
 //   warps 0-3   GEMM1 A gather: 128 threads copy the tile's 128 token rows, 128 bytes of
@@ -25,8 +26,8 @@
 //               fp32 accumulators in TMEM, double-buffered (2 x 256 columns) so the
 //               epilogue of tile i overlaps the main loop of tile i+1;
 //   warps 6-9   epilogue: tcgen05.ld 32 columns at a time, activation / weighting in
-//               registers, rows staged through shared memory so global stores are
-//               coalesced whole-row segments.
+//               registers, 32-row boxes staged in shared memory and written with TMA
+//               tensor stores (double-buffered per warp).
 // Tiles are (row tile, N tile) pairs, row-tile-major, so the CTAs running at the same
 // time work on neighbouring row tiles of the same experts and share weight tiles in L2.
 #include "moe_device.cuh"
@@ -49,8 +50,8 @@ constexpr int kWarpEpi = 6;
 constexpr int kThreads = 320;
 constexpr int kAccCols = 256;               // TMEM columns per accumulator buffer
 constexpr int kTmemCols = 512;
-constexpr int kStagePitch = 144;            // epilogue staging row pitch: 128 B + 16 B pad
-constexpr int kStagingBytes = 32 * kStagePitch;
+constexpr int kStagingBuf = 32 * 128;       // one 32-row epilogue box (<= 128 B per row)
+constexpr int kStagingBytes = 2 * kStagingBuf;  // double-buffered per epilogue warp
 constexpr int kStagingOffset = kStages * kStageBytes;
 constexpr int kBarOffset = kStagingOffset + 4 * kStagingBytes;
 constexpr int kSmemBytes = kBarOffset + 256 + 1024;  // barriers + 1024-byte alignment slack
@@ -69,7 +70,7 @@ struct Args {
   const int* block_expert;
   const int* sorted_pair_ids;
   const float* topk_w;
-  void* out;  // GEMM1: bf16 act [rows, I]; GEMM2: fp32 y [P, H]
+  void* out;  // unused by the kernel: outputs go through the store tensor map
   int* status;
 };
 
@@ -80,7 +81,7 @@ __device__ __forceinline__ int token_of(const Args& a, int row) {
 
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                     const Args a) {
+                     const __grid_constant__ CUtensorMap tmC, const Args a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -116,6 +117,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tmB);
     if (!gather_a) prefetch_tmap(&tmA);
   }
+  if (warp == kWarpEpi && lane == 0) prefetch_tmap(&tmC);
   if (warp == kWarpMma) {
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish();
@@ -127,6 +129,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // everything above overlaps the previous kernel; inputs are read only after this
   griddep_wait();
+  griddep_launch_dependents();
   const int num_tiles = *a.num_blocks * a.n_tiles;
 
   if (warp < kNumAWarps) {
@@ -264,16 +267,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ---------------- epilogue (warps 6..9) ----------------
+    // Each warp owns 32 accumulator rows (its TMEM lane quadrant). Per 32 accumulator
+    // columns it writes one box of 32 output rows to shared memory and stores it with a
+    // TMA tensor store; two staging buffers let the next box be written while the
+    // previous store drains.
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
-    uint8_t* staging = smem + kStagingOffset + (warp - kWarpEpi) * kStagingBytes;
-    const uint32_t staging_u32 = smem_u32(staging);
-    const uint32_t stage_row = staging_u32 + lane * kStagePitch;
+    const uint32_t staging = smem_u32(smem + kStagingOffset + (warp - kWarpEpi) * kStagingBytes);
     const bool gated = a.activation == 0;
-    // bytes one row contributes per 32 accumulator columns
-    const int row_bytes = a.mode == 0 ? (gated ? 32 : 64) : 128;
-    const int slots = row_bytes >> 4;  // 16-byte slots per row
-    const int rows_per_iter = 32 / slots;
-    const int my_slot = lane % slots;
+    // GEMM1: act bf16 rows of 16 (gated) or 32 (relu2) columns per box, no swizzle;
+    // GEMM2: y fp32 rows of 32 columns (128 B), 128-byte swizzle
+    const int box_cols = a.mode == 0 ? (gated ? 16 : 32) : 32;
+    int nst = 0;  // boxes this warp has staged (selects the staging buffer)
     int it = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
       const int acc = it & 1;
@@ -286,69 +290,68 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int grow0 = mb * kBM + q * 32;
       const int pid = a.sorted_pair_ids[grow0 + lane];
       const bool valid = pid < a.num_pairs;
+      const bool any_valid = __ballot_sync(0xffffffffu, valid) != 0u;  // skip all-padding boxes
       const float w = (a.mode != 0 && valid) ? a.topk_w[pid] : 0.f;
-      // destination of this warp's row `lane` at the tile's first column
-      uint8_t* dst_row;
-      if (a.mode == 0) {
-        const int ncol = gated ? a.BN / 2 : a.BN;
-        dst_row = static_cast<uint8_t*>(a.out) +
-                  (static_cast<size_t>(grow0 + lane) * a.out_cols + static_cast<size_t>(nt) * ncol) * 2;
-      } else {
-        dst_row = static_cast<uint8_t*>(a.out) +
-                  (static_cast<size_t>(valid ? pid : 0) * a.out_cols + static_cast<size_t>(nt) * a.BN) * 4;
-      }
+      const int col0 = nt * (a.mode == 0 && gated ? a.BN / 2 : a.BN);
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * kAccCols;
-      for (int c = 0; c < a.BN / 32; ++c) {
+      for (int c = 0; c < a.BN / 32; ++c, ++nst) {
+        const uint32_t buf = staging + (nst & 1) * kStagingBuf;
+        if (nst >= 2) {
+          if (lane == 0) bulk_wait_group_read<1>();  // the store that last used `buf` has read it
+        }
+        __syncwarp();  // also: tcgen05.ld below is .sync.aligned
         uint32_t v[32];
-        __syncwarp();  // tcgen05.ld is .sync.aligned; the previous chunk's staging is consumed
         tmem_ld32(taddr + c * 32, v);
         tmem_wait_ld();
-        uint32_t o[32];
         if (a.mode == 0) {
           if (gated) {
+            uint32_t o[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
               const float g0 = __uint_as_float(v[4 * i + 0]), u0 = __uint_as_float(v[4 * i + 1]);
               const float g1 = __uint_as_float(v[4 * i + 2]), u1 = __uint_as_float(v[4 * i + 3]);
               o[i] = pack_bf16x2(silu_f32(g0) * u0, silu_f32(g1) * u1);
             }
+            const uint32_t dst = buf + lane * 32;
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(o[0]), "r"(o[1]), "r"(o[2]),
+                         "r"(o[3]) : "memory");
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst + 16), "r"(o[4]), "r"(o[5]),
+                         "r"(o[6]), "r"(o[7]) : "memory");
           } else {
+            uint32_t o[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               const float z0 = fmaxf(__uint_as_float(v[2 * i + 0]), 0.f);
               const float z1 = fmaxf(__uint_as_float(v[2 * i + 1]), 0.f);
               o[i] = pack_bf16x2(z0 * z0, z1 * z1);
             }
+            const uint32_t dst = buf + lane * 64;
+#pragma unroll
+            for (int s4 = 0; s4 < 4; ++s4)
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst + 16 * s4), "r"(o[4 * s4]),
+                           "r"(o[4 * s4 + 1]), "r"(o[4 * s4 + 2]), "r"(o[4 * s4 + 3]) : "memory");
           }
         } else {
+          // 128-byte swizzle: 16-byte chunk s of row r lives at chunk (s ^ (r & 7))
+          const uint32_t dst = buf + lane * 128;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(v[i]) * w);
-        }
-        // row `lane` -> staging (the 144-byte pitch keeps 16-byte stores conflict-free)
-#pragma unroll
-        for (int s = 0; s < 8; ++s)
-          if (s < slots)
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(stage_row + s * 16),
-                         "r"(o[4 * s]), "r"(o[4 * s + 1]), "r"(o[4 * s + 2]), "r"(o[4 * s + 3])
+          for (int s8 = 0; s8 < 8; ++s8)
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst + ((s8 ^ (lane & 7)) << 4)),
+                         "f"(__uint_as_float(v[4 * s8]) * w), "f"(__uint_as_float(v[4 * s8 + 1]) * w),
+                         "f"(__uint_as_float(v[4 * s8 + 2]) * w), "f"(__uint_as_float(v[4 * s8 + 3]) * w)
                          : "memory");
+        }
+        fence_proxy_async_smem();  // the generic-proxy writes above feed an async-proxy store
         __syncwarp();
-        // staging -> global in whole-row segments: `slots` consecutive lanes share a row
-        for (int r = lane / slots; r < 32; r += rows_per_iter) {
-          const bool rvalid = __shfl_sync(0xffffffffu, valid ? 1 : 0, r) != 0;
-          const unsigned long long rbase =
-              __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(dst_row), r);
-          uint4 x;
-          asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                       : "=r"(x.x), "=r"(x.y), "=r"(x.z), "=r"(x.w)
-                       : "r"(staging_u32 + r * kStagePitch + my_slot * 16)
-                       : "memory");
-          if (rvalid)
-            *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(rbase) + c * row_bytes + my_slot * 16) = x;
+        if (lane == 0 && any_valid) {
+          tma_store_2d(&tmC, buf, col0 + c * box_cols, grow0);
+          bulk_commit_group();
         }
       }
       tc_fence_before();
       mbar_arrive(tempty0 + 8 * acc);
     }
+    if (lane == 0) bulk_wait_group<0>();  // stores complete before the CTA retires
   }
 
   tc_fence_before();
@@ -362,8 +365,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 bool g_attr_set[64] = {};
 
-cudaError_t launch(const Launch& l, const CUtensorMap& tmA, const CUtensorMap& tmB, const Args& args,
-                   int num_sms) {
+cudaError_t launch(const Launch& l, const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmC,
+                   const Args& args, int num_sms) {
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
@@ -375,7 +378,7 @@ cudaError_t launch(const Launch& l, const CUtensorMap& tmA, const CUtensorMap& t
   cudaLaunchConfig_t cfg;
   cudaLaunchAttribute attr[1];
   make_launch_config(&cfg, attr, l, dim3(num_sms), dim3(kThreads), kSmemBytes);
-  return cudaLaunchKernelEx(&cfg, gemm_bf16_kernel, tmA, tmB, args);
+  return cudaLaunchKernelEx(&cfg, gemm_bf16_kernel, tmA, tmB, tmC, args);
 }
 
 Args make_args(int mode, const GemmShape& s, const GemmBuffers& b, const void* a_rows) {
@@ -413,14 +416,14 @@ int pick_bn(int N, bool gated) {
 size_t gemm_bf16_smem_bytes() { return kSmemBytes; }
 
 cudaError_t launch_gemm1_bf16(const Launch& l, const void* hidden, const CUtensorMap& tm_w13,
-                              const GemmShape& s, const GemmBuffers& b) {
+                              const CUtensorMap& tm_act_store, const GemmShape& s, const GemmBuffers& b) {
   // the A operand is gathered with cp.async; tmA is not read in this mode
-  return launch(l, tm_w13, tm_w13, make_args(0, s, b, hidden), s.num_sms);
+  return launch(l, tm_w13, tm_w13, tm_act_store, make_args(0, s, b, hidden), s.num_sms);
 }
 
 cudaError_t launch_gemm2_bf16(const Launch& l, const CUtensorMap& tm_act, const CUtensorMap& tm_w2,
-                              const GemmShape& s, const GemmBuffers& b) {
-  return launch(l, tm_act, tm_w2, make_args(1, s, b, nullptr), s.num_sms);
+                              const CUtensorMap& tm_y_store, const GemmShape& s, const GemmBuffers& b) {
+  return launch(l, tm_act, tm_w2, tm_y_store, make_args(1, s, b, nullptr), s.num_sms);
 }
 
 }  // namespace moe

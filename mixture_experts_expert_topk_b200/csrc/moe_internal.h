@@ -62,9 +62,9 @@ struct GemmBuffers {
 int pick_bn(int N, bool gated);
 size_t gemm_bf16_smem_bytes();
 cudaError_t launch_gemm1_bf16(const Launch& l, const void* hidden, const CUtensorMap& tm_w13,
-                              const GemmShape& s, const GemmBuffers& b);
+                              const CUtensorMap& tm_act_store, const GemmShape& s, const GemmBuffers& b);
 cudaError_t launch_gemm2_bf16(const Launch& l, const CUtensorMap& tm_act, const CUtensorMap& tm_w2,
-                              const GemmShape& s, const GemmBuffers& b);
+                              const CUtensorMap& tm_y_store, const GemmShape& s, const GemmBuffers& b);
 size_t gemm_fp8_smem_bytes();
 cudaError_t launch_gemm1_fp8(const Launch& l, const CUtensorMap& tm_xq, const CUtensorMap& tm_w13,
                              const GemmShape& s, const GemmBuffers& b);
@@ -72,7 +72,8 @@ cudaError_t launch_gemm2_fp8(const Launch& l, const CUtensorMap& tm_actq, const 
                              const GemmShape& s, const GemmBuffers& b);
 
 // ---- elementwise (combine.cu, quant.cu, prepare.cu) ----
-cudaError_t launch_combine(const Launch& l, const void* y, int T, int k_total, int H, void* out);
+cudaError_t launch_combine(const Launch& l, const void* y, const int* pair_to_row, int T, int k_total, int H,
+                           void* out);
 cudaError_t launch_quant_act(const Launch& l, const void* x, int T, int H, void* q, float* scale);
 cudaError_t launch_quant_weights(const Launch& l, const void* w, int64_t num_mats, int rows,
                                  int cols, void* q, float* scale);

@@ -9,9 +9,11 @@
 // section 2: a fused shared expert is one more slot, id E_r, weight 1, after the routed
 // slots.
 //
-// One warp per token. A lane holds logits lane, lane+32, ... in registers; each of the
-// k selection rounds is a register scan plus a 5-step butterfly arg-max. Selection runs
-// on the raw logits, so the ids never depend on the exponential's rounding.
+// One warp per token. A lane holds logits lane, lane+32, ... as order-preserving integer
+// keys; each of the k selection rounds is a register scan plus two warp reductions
+// (redux.sync max of the key, then min of the expert index among the lanes holding it).
+// Selection runs on the raw logits, so the ids never depend on the exponential's
+// rounding.
 #include "moe_device.cuh"
 #include "moe_internal.h"
 
@@ -20,14 +22,15 @@ namespace {
 
 constexpr int kRouteWarps = 8;
 
-struct Cand {
-  float v;
-  int i;
-};
-
-// a beats b: larger logit, or equal logit and lower expert index.
-__device__ __forceinline__ bool beats(const Cand& a, const Cand& b) {
-  return a.v > b.v || (a.v == b.v && a.i < b.i);
+// Order-preserving map of finite floats to unsigned integers (larger float -> larger
+// key; -0 is folded onto +0 so the two compare equal, as floats do). Key 0 is below every
+// finite float's key and marks absent or already selected entries.
+__device__ __forceinline__ uint32_t order_key(float x) {
+  const uint32_t b = __float_as_uint(x == 0.f ? 0.f : x);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float key_value(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
 
 template <int VPL>
@@ -36,6 +39,7 @@ __global__ void __launch_bounds__(kRouteWarps * 32)
                  int renormalize, int* __restrict__ topk_ids, float* __restrict__ topk_w,
                  int* __restrict__ status) {
   griddep_wait();
+  griddep_launch_dependents();
   // routing starts every forward: clear the device status word of the workspace
   if (blockIdx.x == 0 && threadIdx.x == 0) *status = 0;
   const int lane = threadIdx.x & 31;
@@ -43,55 +47,53 @@ __global__ void __launch_bounds__(kRouteWarps * 32)
   if (t >= T) return;
   const float* row = logits + static_cast<size_t>(t) * E;
 
-  float v[VPL];
-  uint32_t taken = 0;  // bit i: value i of this lane selected or absent
+  // lane holds experts lane, lane + 32, ...; an expert's index is lane + 32 * i
+  uint32_t key[VPL];
+  uint32_t lmax = 0;
 #pragma unroll
   for (int i = 0; i < VPL; ++i) {
     const int e = lane + 32 * i;
-    if (e < E) {
-      v[i] = __ldg(row + e);
-    } else {
-      v[i] = -INFINITY;
-      taken |= 1u << i;
-    }
+    key[i] = e < E ? order_key(__ldg(row + e)) : 0u;
+    lmax = max(lmax, key[i]);
+  }
+  // softmax shift: the largest logit
+  const float m = key_value(__reduce_max_sync(0xffffffffu, lmax));
+  // with renormalisation the full softmax denominator cancels and is not needed
+  float s = 0.f;
+  if (!renormalize) {
+#pragma unroll
+    for (int i = 0; i < VPL; ++i)
+      if (key[i] != 0u) s += expf(key_value(key[i]) - m);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
   }
 
-  // softmax denominator over all routed experts (max subtracted)
-  float m = -INFINITY;
-#pragma unroll
-  for (int i = 0; i < VPL; ++i)
-    if (!(taken >> i & 1u)) m = fmaxf(m, v[i]);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  float s = 0.f;
-#pragma unroll
-  for (int i = 0; i < VPL; ++i)
-    if (!(taken >> i & 1u)) s += expf(v[i] - m);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-
-  // k rounds of arg-max; slot j's exp(l - m) is kept by lane j
+  // k rounds: the largest remaining key, ties to the lowest expert index. Lane j keeps
+  // slot j's expert and exp(l - m).
   float my_e = 0.f;
   int my_id = 0;
   float sel_sum = 0.f;
   for (int j = 0; j < topk; ++j) {
-    Cand best{-INFINITY, 0x7fffffff};
+    uint32_t bk = 0u;
+    int bi = 0;
 #pragma unroll
-    for (int i = 0; i < VPL; ++i) {
-      Cand c{v[i], lane + 32 * i};
-      if (!(taken >> i & 1u) && beats(c, best)) best = c;
-    }
+    for (int i = 0; i < VPL; ++i)
+      if (key[i] > bk) {  // strict: the lowest i among equal keys
+        bk = key[i];
+        bi = i;
+      }
+    const uint32_t wk = __reduce_max_sync(0xffffffffu, bk);
+    const uint32_t widx = __reduce_min_sync(0xffffffffu, bk == wk ? static_cast<uint32_t>(lane + 32 * bi) : 0xffffffffu);
+    if (static_cast<uint32_t>(lane) == (widx & 31u)) {
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      Cand other{__shfl_xor_sync(0xffffffffu, best.v, o), __shfl_xor_sync(0xffffffffu, best.i, o)};
-      if (beats(other, best)) best = other;
+      for (int i = 0; i < VPL; ++i)
+        if (i == bi) key[i] = 0u;
     }
-    if ((best.i & 31) == lane) taken |= 1u << (best.i >> 5);
-    const float ej = expf(best.v - m);
+    const float ej = expf(key_value(wk) - m);
     sel_sum += ej;
     if (lane == j) {
       my_e = ej;
-      my_id = best.i;
+      my_id = static_cast<int>(widx);
     }
   }
   const int kk = topk + num_shared;

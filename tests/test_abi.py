@@ -100,7 +100,7 @@ def test_workspace_layout(L):
         assert lay["num_chunks"] == -(-P // 2048)
         offs = sorted(v for k, v in lay.items() if k not in ("total_bytes", "max_rows", "num_chunks", "block_m"))
         assert all(o % 1024 == 0 for o in offs)
-        assert lay["y"] + P * cfg.H * 4 <= lay["total_bytes"]
+        assert lay["y"] + lay["max_rows"] * cfg.H * 4 <= lay["total_bytes"]
         assert moe.workspace_size(p) == lay["total_bytes"]
     bad = _prob(H=0)
     assert L.moe_workspace_size(ctypes.byref(bad)) == 0
