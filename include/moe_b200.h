@@ -216,6 +216,30 @@ moe_status_t moe_stage_gemm2(const moe_problem_t* problem, const void* w2, const
 moe_status_t moe_stage_combine(const moe_problem_t* problem, void* out, void* workspace,
                                size_t workspace_bytes, moe_stream_t stream);
 
+/* The align step without a workspace, for callers that cannot allocate device memory
+ * (an engine plugin that is handed only its input and output tensors, code running under
+ * stream capture, or a path where an allocation could synchronise the device). The pages
+ * have no counterpart of this entry point; it runs the same kernels as moe_stage_align.
+ *   topk_ids        device int32 [T, k'] expert ids (e.g. from moe_stage_route), each in
+ *                   [0, E); read only
+ *   sorted_pair_ids device int32 [max_rows]   } outputs, laid out exactly as the
+ *   expert_offsets  device int32 [E+1]        } workspace fields of the same names
+ *   block_expert    device int32 [max_rows/128] } (moe_workspace_layout gives max_rows)
+ *   pair_to_row     device int32 [T*k']       }
+ *   num_blocks      device int32 [1]          }
+ * Its scratch is a fixed array of 262144 int32 (1 MiB) in device memory owned by the
+ * library: every GPU that loads the library holds it until the process exits. A problem
+ * needing more (ceil(T*k'/2048) * E > 262144) returns MOE_ERR_UNSUPPORTED. The first call
+ * on a device looks the array up for that device (cudaGetSymbolAddress), so make that
+ * first call before any stream capture. All calls on a device share its one array, whose
+ * contents persist from call to call: calls that may overlap on the GPU (for example on
+ * two streams of one device) race, so the caller must order them. No memory is allocated
+ * and nothing is synchronised. */
+moe_status_t moe_align_noalloc(const moe_problem_t* problem, const int32_t* topk_ids,
+                               int32_t* sorted_pair_ids, int32_t* expert_offsets,
+                               int32_t* block_expert, int32_t* pair_to_row, int32_t* num_blocks,
+                               moe_stream_t stream);
+
 /* Synchronises `stream`, reads and clears the workspace status word. Returns MOE_OK,
  * MOE_ERR_DEVICE_TIMEOUT if a kernel abandoned a bounded wait since the last query
  * (its outputs are then undefined), or MOE_ERR_CUDA. `*detail` (may be NULL) receives

@@ -83,6 +83,7 @@ SIGNATURES = {
     "moe_stage_gemm2": (_I, [_P, _V, _V, _V, _S, _V]),
     "moe_stage_combine": (_I, [_P, _V, _V, _S, _V]),
     "moe_get_device_status": (_I, [_V, _V, ctypes.POINTER(_I)]),
+    "moe_align_noalloc": (_I, [_P, _V, _V, _V, _V, _V, _V, _V]),
 }
 
 _lib = None
