@@ -86,7 +86,7 @@ typedef enum {
 /* Problem description shared by all entry points. */
 typedef struct {
   int32_t num_tokens;   /* T >= 0 */
-  int32_t hidden;       /* H > 0, multiple of 128 */
+  int32_t hidden;       /* H > 0, multiple of 128 (FP8: H <= 4096 and I <= 4096) */
   int32_t num_routed;   /* E_r >= 1: columns of router_logits */
   int32_t num_shared;   /* 0 or 1: shared-expert slots; slot id E_r, weight 1, after the
                            routed slots (sglang PR 26204 section 2). Experts in the
@@ -105,7 +105,8 @@ typedef struct {
  * tests and tools; the contents are this library's private format otherwise). */
 typedef struct {
   size_t total_bytes;
-  size_t status;          /* int32 device status word (0 = ok) */
+  size_t status;          /* int32 device status word (0 = ok); the 256-byte region also
+                             holds the GEMM kernels' work counters */
   size_t num_blocks;      /* int32: number of block_m row tiles after align (= P_pad/block_m) */
   size_t topk_ids;        /* int32 [T, k'] selected expert ids, slot order */
   size_t topk_w;          /* fp32  [T, k'] routing weights */
@@ -116,7 +117,8 @@ typedef struct {
   size_t chunk_hist;      /* int32 [num_chunks, E]: align scratch */
   size_t xq;              /* FP8: e4m3 [T, H] quantised hidden */
   size_t xq_scale;        /* FP8: fp32 [T, H/128] */
-  size_t act;             /* GEMM1 output [max_rows, I]: bf16, or e4m3 for FP8 */
+  size_t act;             /* GEMM1 output: bf16 [max_rows, I] */
+  size_t actq;            /* FP8: the activation quantised per 1x128 group, e4m3 [max_rows, I] */
   size_t act_scale;       /* FP8: fp32 [max_rows, I/128] */
   size_t y;               /* fp32 [max_rows, H]: weighted GEMM2 rows in sorted order */
   size_t io_hidden;       /* staging for moe_forward_host: bf16 [T, H] */

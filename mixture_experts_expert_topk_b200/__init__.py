@@ -252,11 +252,10 @@ def read_workspace(prob: Problem, workspace: torch.Tensor) -> Dict[str, torch.Te
         "pair_to_row": view(L["pair_to_row"], P, torch.int32),
         "y": view(L["y"], rows * H, torch.float32).view(rows, H),
     }
+    out["act"] = view(L["act"], rows * I, torch.bfloat16).view(rows, I)
     if fp8:
         out["xq"] = view(L["xq"], T * H, torch.uint8).view(T, H)
         out["xq_scale"] = view(L["xq_scale"], T * (H // 128), torch.float32).view(T, H // 128)
-        out["act"] = view(L["act"], rows * I, torch.uint8).view(rows, I)
+        out["actq"] = view(L["actq"], rows * I, torch.uint8).view(rows, I)
         out["act_scale"] = view(L["act_scale"], rows * (I // 128), torch.float32).view(rows, I // 128)
-    else:
-        out["act"] = view(L["act"], rows * I, torch.bfloat16).view(rows, I)
     return out

@@ -47,7 +47,7 @@ class Layout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in (
         "total_bytes", "status", "num_blocks", "topk_ids", "topk_w", "sorted_pair_ids",
         "expert_offsets", "block_expert", "pair_to_row", "chunk_hist", "xq", "xq_scale", "act",
-        "act_scale", "y", "io_hidden", "io_logits", "io_out")] + [
+        "actq", "act_scale", "y", "io_hidden", "io_logits", "io_out")] + [
         ("max_rows", ctypes.c_int64),
         ("num_chunks", ctypes.c_int32),
         ("block_m", ctypes.c_int32),

@@ -101,12 +101,17 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_sums, int* 
   return excl;
 }
 
-// Padded segment of expert e starting at row `off` with `count` pairs: sentinel rows and
-// the expert id of its row tiles.
-__device__ __forceinline__ void write_segment(int e, int off, int count, int padded, int block_m, int P,
-                                              int* sorted_pair_ids, int* block_expert) {
-  for (int r = off + count; r < off + padded; ++r) sorted_pair_ids[r] = P;
-  for (int b = off / block_m; b < (off + padded) / block_m; ++b) block_expert[b] = e;
+// Padded segments of experts [0, E): sentinel rows after each expert's pairs and the
+// expert id of each row tile. One warp per expert, lanes striding over its rows, so the
+// stores are coalesced. seg_off/seg_cnt/seg_pad are shared-memory arrays.
+__device__ __forceinline__ void write_segments(int E, const int* seg_off, const int* seg_cnt, const int* seg_pad,
+                                               int block_m, int P, int* sorted_pair_ids, int* block_expert) {
+  const int lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+  for (int e = threadIdx.x >> 5; e < E; e += nwarps) {
+    const int off = seg_off[e], cnt = seg_cnt[e], pad = seg_pad[e];
+    for (int r = off + cnt + lane; r < off + pad; r += 32) sorted_pair_ids[r] = P;
+    for (int b = off / block_m + lane; b < (off + pad) / block_m; b += 32) block_expert[b] = e;
+  }
 }
 
 __global__ void __launch_bounds__(kWarps * 32)
@@ -130,6 +135,7 @@ __global__ void __launch_bounds__(kScanThreads)
                       int* __restrict__ block_expert, int* __restrict__ num_blocks) {
   extern __shared__ int stage[];  // [batch chunks][E]
   __shared__ int warp_sums[32];
+  __shared__ int seg_off[kMaxExperts], seg_cnt[kMaxExperts], seg_pad[kMaxExperts];
   griddep_wait();
   griddep_launch_dependents();
   const int e = threadIdx.x;  // E <= 1024: one expert per thread
@@ -154,12 +160,16 @@ __global__ void __launch_bounds__(kScanThreads)
   const int off = block_exclusive_scan(padded, warp_sums, &total);
   if (e < E) {
     expert_offsets[e] = off;
-    write_segment(e, off, count, padded, block_m, P, sorted_pair_ids, block_expert);
+    seg_off[e] = off;
+    seg_cnt[e] = count;
+    seg_pad[e] = padded;
   }
   if (threadIdx.x == 0) {
     expert_offsets[E] = total;
     *num_blocks = total / block_m;
   }
+  __syncthreads();
+  write_segments(E, seg_off, seg_cnt, seg_pad, block_m, P, sorted_pair_ids, block_expert);
 }
 
 __global__ void __launch_bounds__(kWarps * 32)
@@ -197,6 +207,7 @@ __global__ void __launch_bounds__(kWarps * 32)
                         int* __restrict__ pair_to_row, int* __restrict__ num_blocks) {
   __shared__ int cnt[kWarps][kMaxExperts];
   __shared__ int warp_sums[32];
+  __shared__ int seg_off[kMaxExperts], seg_cnt[kMaxExperts], seg_pad[kMaxExperts];
   griddep_wait();
   griddep_launch_dependents();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -219,7 +230,9 @@ __global__ void __launch_bounds__(kWarps * 32)
     const int off = carry + block_exclusive_scan(padded, warp_sums, &total);
     if (x < E) {
       expert_offsets[x] = off;
-      write_segment(x, off, count, padded, block_m, P, sorted_pair_ids, block_expert);
+      seg_off[x] = off;
+      seg_cnt[x] = count;
+      seg_pad[x] = padded;
       int run = off;
       for (int w = 0; w < kWarps; ++w) {
         const int c = cnt[w][x];
@@ -234,6 +247,7 @@ __global__ void __launch_bounds__(kWarps * 32)
     *num_blocks = carry / block_m;
   }
   __syncthreads();
+  write_segments(E, seg_off, seg_cnt, seg_pad, block_m, P, sorted_pair_ids, block_expert);
   warp_place(e, base, lane, cnt[warp], sorted_pair_ids, pair_to_row);
 }
 

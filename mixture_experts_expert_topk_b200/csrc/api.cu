@@ -76,6 +76,8 @@ moe_status_t make_plan(const moe_problem_t* p, Plan* pl) {
   if (p->topk + p->num_shared > moe::kMaxSlots) return MOE_ERR_UNSUPPORTED;
   if (p->block_m != 0 && p->block_m != 128) return MOE_ERR_UNSUPPORTED;
   if (p->hidden > (1 << 20) || p->intermediate > (1 << 20)) return MOE_ERR_UNSUPPORTED;
+  // FP8: a GEMM's K blocks (H/128 and I/128) are held one per lane of a warp
+  if (q.fp8 && (p->hidden > 4096 || p->intermediate > 4096)) return MOE_ERR_UNSUPPORTED;
 
   q.T = p->num_tokens;
   q.H = p->hidden;
@@ -91,8 +93,9 @@ moe_status_t make_plan(const moe_problem_t* p, Plan* pl) {
   q.act = p->activation;
   q.P = static_cast<long long>(q.T) * q.kk;
   if (q.P >= (1LL << 31) - (1LL << 20)) return MOE_ERR_UNSUPPORTED;
-  q.bn1 = moe::pick_bn(q.N1, q.gated);
-  q.bn2 = moe::pick_bn(q.H, false);
+  // N tiles for a full device; the launches refine them for the actual SM count
+  q.bn1 = moe::pick_bn(q.N1, 1, 1);
+  q.bn2 = moe::pick_bn(q.H, 1, 1);
   if (q.bn1 == 0 || q.bn2 == 0) return MOE_ERR_UNSUPPORTED;
 
   moe_workspace_layout_t& L = q.lay;
@@ -119,7 +122,8 @@ moe_status_t make_plan(const moe_problem_t* p, Plan* pl) {
   L.chunk_hist = take(static_cast<size_t>(L.num_chunks) * q.E * 4);
   L.xq = take(q.fp8 ? T * H : 0);
   L.xq_scale = take(q.fp8 ? T * (H / 128) * 4 : 0);
-  L.act = take(rows * I * (q.fp8 ? 1 : 2));
+  L.act = take(rows * I * 2);
+  L.actq = take(q.fp8 ? rows * I : 0);
   L.act_scale = take(q.fp8 ? rows * (I / 128) * 4 : 0);
   L.y = take(rows * H * 4);
   L.io_hidden = take(T * H * 2);
@@ -205,12 +209,13 @@ moe_status_t check_ws(const Plan& pl, const void* ws, size_t ws_bytes) {
 
 // ---- the steps (arguments already checked) ----------------------------------------
 
-moe_status_t run_route(const Plan& pl, const float* logits, void* ws, const Launch& l) {
+// `hidden` (may be NULL) is prefetched into L2 for GEMM1's row gather
+moe_status_t run_route(const Plan& pl, const float* logits, void* ws, const Launch& l, const void* hidden) {
   const auto& L = pl.lay;
   // the route kernel also resets the device status word: it starts every forward
   return cuda_status(moe::launch_route(l, logits, pl.T, pl.Er, pl.topk, pl.Es, pl.renorm,
                                        ws_ptr<int>(ws, L.topk_ids), ws_ptr<float>(ws, L.topk_w),
-                                       ws_ptr<int>(ws, L.status)));
+                                       ws_ptr<int>(ws, L.status), pl.fp8 ? nullptr : hidden, pl.H * 2));
 }
 
 moe_status_t run_align(const Plan& pl, void* ws, const Launch& l) {
@@ -240,8 +245,18 @@ GemmBuffers common_buffers(const Plan& pl, void* ws) {
   return b;
 }
 
-moe_status_t run_gemm1(const Plan& pl, const void* hidden, const void* w13, const float* w13_scale, void* ws,
+// Lower bound on the number of 128-row tiles align produces: every expert that receives
+// a pair gets at least one, and there are at least ceil(P / 128).
+long long est_row_tiles(const Plan& pl) {
+  const long long by_rows = (pl.P + 127) / 128;
+  const long long by_experts = pl.P < pl.E ? pl.P : pl.E;
+  return by_rows > by_experts ? by_rows : by_experts;
+}
+
+moe_status_t run_gemm1(const Plan& pl_in, const void* hidden, const void* w13, const float* w13_scale, void* ws,
                        const Launch& l, int num_sms) {
+  Plan pl = pl_in;
+  if (!pl.fp8) pl.bn1 = moe::pick_bn(pl.N1, est_row_tiles(pl), num_sms);
   const auto& L = pl.lay;
   GemmShape s;
   s.K = pl.H;
@@ -255,6 +270,7 @@ moe_status_t run_gemm1(const Plan& pl, const void* hidden, const void* w13, cons
   s.num_sms = num_sms;
   GemmBuffers b = common_buffers(pl, ws);
   b.out = ws_ptr<void>(ws, L.act);
+  b.tile_counter = ws_ptr<int>(ws, L.status) + 4;
   CUtensorMap ta, tb;
   if (!pl.fp8) {
     // the token rows of hidden are gathered by the kernel itself (no tensor map); the
@@ -267,22 +283,33 @@ moe_status_t run_gemm1(const Plan& pl, const void* hidden, const void* w13, cons
       return MOE_ERR_CUDA;
     return cuda_status(moe::launch_gemm1_bf16(l, hidden, tb, tc, s, b));
   }
-  if (!make_tmap_2d(&ta, ws_ptr<void>(ws, L.xq), CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, pl.H, pl.T, 128, 1) ||
-      !make_tmap_2d(&tb, w13, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, pl.H, static_cast<uint64_t>(pl.E) * pl.N1, 128,
-                    pl.bn1))
+  // FP8: quantised hidden rows gathered by the kernel; weight codes in 128 x 128 boxes;
+  // bf16 activation written in boxes of 32 rows x 64 columns, then quantised per 1x128
+  (void)ta;
+  CUtensorMap tc;
+  if (!make_tmap_2d(&tb, w13, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, pl.H, static_cast<uint64_t>(pl.E) * pl.N1, 128,
+                    128) ||
+      !make_tmap_2d(&tc, ws_ptr<void>(ws, L.act), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, pl.I,
+                    static_cast<uint64_t>(L.max_rows), 64, 32))
     return MOE_ERR_CUDA;
-  b.out_scale = ws_ptr<float>(ws, L.act_scale);
   b.a_scale = ws_ptr<float>(ws, L.xq_scale);
   b.w_scale = w13_scale;
   b.a_scale_cols = pl.H / 128;
   b.w_scale_rows = pl.N1 / 128;
   b.w_scale_cols = pl.H / 128;
   b.up_block_offset = pl.I / 128;
-  return cuda_status(moe::launch_gemm1_fp8(l, ta, tb, s, b));
+  s.BN = 128;
+  moe_status_t st = cuda_status(moe::launch_gemm1_fp8(l, ws_ptr<void>(ws, L.xq), tb, tc, s, b));
+  if (st != MOE_OK) return st;
+  return cuda_status(moe::launch_quant_rows(l, ws_ptr<void>(ws, L.act), static_cast<int>(L.max_rows), pl.I,
+                                            ws_ptr<int>(ws, L.num_blocks), pl.bm, ws_ptr<void>(ws, L.actq),
+                                            ws_ptr<float>(ws, L.act_scale)));
 }
 
-moe_status_t run_gemm2(const Plan& pl, const void* w2, const float* w2_scale, void* ws, const Launch& l,
+moe_status_t run_gemm2(const Plan& pl_in, const void* w2, const float* w2_scale, void* ws, const Launch& l,
                        int num_sms) {
+  Plan pl = pl_in;
+  if (!pl.fp8) pl.bn2 = moe::pick_bn(pl.H, est_row_tiles(pl), num_sms);
   const auto& L = pl.lay;
   GemmShape s;
   s.K = pl.I;
@@ -296,6 +323,7 @@ moe_status_t run_gemm2(const Plan& pl, const void* w2, const float* w2_scale, vo
   s.num_sms = num_sms;
   GemmBuffers b = common_buffers(pl, ws);
   b.out = ws_ptr<void>(ws, L.y);
+  b.tile_counter = ws_ptr<int>(ws, L.status) + 6;
   CUtensorMap ta, tb;
   const uint64_t rows = static_cast<uint64_t>(L.max_rows);
   if (!pl.fp8) {
@@ -307,16 +335,18 @@ moe_status_t run_gemm2(const Plan& pl, const void* w2, const float* w2_scale, vo
       return MOE_ERR_CUDA;
     return cuda_status(moe::launch_gemm2_bf16(l, ta, tb, tc, s, b));
   }
-  if (!make_tmap_2d(&ta, ws_ptr<void>(ws, L.act), CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, pl.I, rows, 128, 128) ||
-      !make_tmap_2d(&tb, w2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, pl.I, static_cast<uint64_t>(pl.E) * pl.H, 128,
-                    pl.bn2))
+  CUtensorMap tc;
+  if (!make_tmap_2d(&ta, ws_ptr<void>(ws, L.actq), CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, pl.I, rows, 128, 128) ||
+      !make_tmap_2d(&tb, w2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, pl.I, static_cast<uint64_t>(pl.E) * pl.H, 128, 128) ||
+      !make_tmap_2d(&tc, ws_ptr<void>(ws, L.y), CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, pl.H, rows, 32, 32))
     return MOE_ERR_CUDA;
   b.a_scale = ws_ptr<float>(ws, L.act_scale);
   b.w_scale = w2_scale;
   b.a_scale_cols = pl.I / 128;
   b.w_scale_rows = pl.H / 128;
   b.w_scale_cols = pl.I / 128;
-  return cuda_status(moe::launch_gemm2_fp8(l, ta, tb, s, b));
+  s.BN = 128;
+  return cuda_status(moe::launch_gemm2_fp8(l, ta, tb, tc, s, b));
 }
 
 moe_status_t run_combine(const Plan& pl, void* out, void* ws, const Launch& l) {
@@ -345,7 +375,7 @@ moe_status_t forward_device(const Plan& pl, const moe_problem_t* p, const void* 
                             const void* w13, const void* w2, const float* s13, const float* s2, void* out,
                             void* ws, moe_stream_t stream, int num_sms) {
   const Launch l = launch_of(p, stream);
-  moe_status_t st = run_route(pl, logits, ws, l);
+  moe_status_t st = run_route(pl, logits, ws, l, hidden);
   if (st == MOE_OK) st = run_align(pl, ws, l);
   if (st == MOE_OK && pl.fp8) st = run_quant_act(pl, hidden, ws, l);
   if (st == MOE_OK) st = run_gemm1(pl, hidden, w13, s13, ws, l, num_sms);
@@ -492,7 +522,7 @@ MOE_API moe_status_t moe_stage_route(const moe_problem_t* problem, const float* 
   if (!aligned16(router_logits)) return MOE_ERR_INVALID_ARG;
   st = prologue(problem, workspace, workspace_bytes, &pl, &sms);
   if (st != MOE_OK || pl.T == 0) return st;
-  return run_route(pl, router_logits, workspace, launch_of(problem, stream));
+  return run_route(pl, router_logits, workspace, launch_of(problem, stream), nullptr);
 }
 
 MOE_API moe_status_t moe_stage_align(const moe_problem_t* problem, void* workspace, size_t workspace_bytes,

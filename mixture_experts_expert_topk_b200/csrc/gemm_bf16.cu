@@ -15,21 +15,26 @@
 // pair_to_row.
 //
 // Kernel structure (one persistent CTA per SM, 10 warps):
-//   warps 0-3   GEMM1 A gather: 128 threads copy the tile's 128 token rows, 128 bytes of
-//               K each per stage, with 16-byte cp.async into the 128-byte-swizzled layout
-//               the MMA reads; each thread's copies arrive on the stage's barrier when they
-//               land (cp.async.mbarrier.arrive). A TMA gather4 per 4 rows was measured to
-//               cap the producer at one stage per ~1.3 us; cp.async keeps up with HBM.
-//   warp 4      TMA: B tile (weights, 2-D tiled load, 128-byte swizzle) and, for GEMM2,
-//               the contiguous A tile; 4-stage ring of 48 KB stages;
+//   warps 0-3   A producer. GEMM1: 128 threads gather the tile's 128 token rows, 128 bytes
+//               of K each per stage, with 16-byte cp.async into the 128-byte-swizzled
+//               layout the MMA reads; each thread's copies arrive on the stage barrier when
+//               they land (cp.async.mbarrier.arrive). (A TMA gather4 per 4 rows was measured
+//               to cap the producer at one stage per ~1.3 us.) GEMM2: warp 0 loads the
+//               contiguous A tile with TMA.
+//   warp 4      tile scheduler and B producer: takes tiles from a global atomic counter,
+//               publishes them to the other roles through a small shared-memory ring, and
+//               streams the weight tiles with TMA (2-D tiled loads, 128-byte swizzle).
 //   warp 5      TMEM allocator and MMA issuer: tcgen05.mma kind::f16, M=128, N=BN, K=16,
 //               fp32 accumulators in TMEM, double-buffered (2 x 256 columns) so the
-//               epilogue of tile i overlaps the main loop of tile i+1;
+//               epilogue of tile i overlaps the main loop of tile i+1.
 //   warps 6-9   epilogue: tcgen05.ld 32 columns at a time, activation / weighting in
 //               registers, 32-row boxes staged in shared memory and written with TMA
-//               tensor stores (double-buffered per warp).
-// Tiles are (row tile, N tile) pairs, row-tile-major, so the CTAs running at the same
-// time work on neighbouring row tiles of the same experts and share weight tiles in L2.
+//               tensor stores.
+// A and B have rings of their own: the weights (from HBM) keep more stages in flight
+// than the activation rows (mostly L2 hits). Tiles are (row tile, N tile) pairs handed out
+// in row-tile-major order, so CTAs running at the same time work on neighbouring row tiles
+// of the same experts and share weight tiles in L2; taking them from a counter rather
+// than a fixed stride lets CTAs whose tiles hit in L2 take more of them.
 #include "moe_device.cuh"
 #include "moe_internal.h"
 
@@ -37,46 +42,65 @@ namespace moe {
 namespace {
 
 constexpr int kBM = 128;
-constexpr int kBKBytes = 128;               // one 128-byte swizzle atom of K per stage
-constexpr int kStages = 4;
+constexpr int kBKBytes = 128;  // one 128-byte swizzle atom of K per stage
 constexpr int kMaxBN = 256;
 constexpr int kStageA = kBM * kBKBytes;     // 16 KB
 constexpr int kStageB = kMaxBN * kBKBytes;  // 32 KB
-constexpr int kStageBytes = kStageA + kStageB;
 constexpr int kNumAWarps = 4;
-constexpr int kWarpTma = 4;
+constexpr int kWarpSched = 4;
 constexpr int kWarpMma = 5;
 constexpr int kWarpEpi = 6;
 constexpr int kThreads = 320;
-constexpr int kAccCols = 256;               // TMEM columns per accumulator buffer
+constexpr int kAccCols = 256;  // TMEM columns per accumulator buffer
 constexpr int kTmemCols = 512;
-constexpr int kStagingBuf = 32 * 128;       // one 32-row epilogue box (<= 128 B per row)
-constexpr int kStagingBytes = 2 * kStagingBuf;  // double-buffered per epilogue warp
-constexpr int kStagingOffset = kStages * kStageBytes;
-constexpr int kBarOffset = kStagingOffset + 4 * kStagingBytes;
-constexpr int kSmemBytes = kBarOffset + 256 + 1024;  // barriers + 1024-byte alignment slack
+constexpr int kTileRing = 4;
+constexpr int kBarBytes = 512;
+constexpr int kSmemCap = 232448;  // opt-in shared memory per CTA on sm_100
 
 // wait sites (device status detail)
-enum : int { kSiteEmpty = 1, kSiteFull = 2, kSiteTmemEmpty = 3, kSiteTmemFull = 4, kSiteEmptyA = 6 };
+enum : int {
+  kSiteEmptyB = 1, kSiteFullA = 2, kSiteTmemEmpty = 3, kSiteTmemFull = 4, kSiteFullB = 5, kSiteEmptyA = 6,
+  kSiteTileFull = 7, kSiteTileEmpty = 8
+};
 
 struct Args {
-  int mode;  // 0 = GEMM1 (gather + activation), 1 = GEMM2 (weighted scatter)
-  int K, BN, n_tiles, k_blocks;
+  int mode;  // 0 = GEMM1 (gather + activation), 1 = GEMM2 (weighted rows)
+  int BN, n_tiles, k_blocks;
   int w_rows_per_expert;
-  int k_total, num_pairs, activation, out_cols;
+  int k_total, num_pairs, activation;
+  int stages_a, stages_b;            // ring depths
+  int staging_bufs, staging_bytes;   // per epilogue warp: buffers and bytes per buffer
   const uint8_t* a_rows;  // GEMM1: hidden [T, H] bf16
   int a_row_bytes;        // GEMM1: H * 2
   const int* num_blocks;
   const int* block_expert;
   const int* sorted_pair_ids;
   const float* topk_w;
-  void* out;  // unused by the kernel: outputs go through the store tensor map
+  int* tile_counter;  // [2]: next tile, CTAs finished; both 0 between launches
   int* status;
 };
+
+__host__ __device__ constexpr int smem_bytes(int sa, int sb, int bufs, int buf_bytes) {
+  return sa * kStageA + sb * kStageB + 4 * bufs * buf_bytes + kBarBytes + 1024;
+}
 
 __device__ __forceinline__ int token_of(const Args& a, int row) {
   const int pid = a.sorted_pair_ids[row];
   return pid < a.num_pairs ? pid / a.k_total : 0;  // padding rows read token 0
+}
+
+// Reader side of the tile ring: the next tile id (or -1 when done, -2 on abort). Called
+// by one thread; it releases the slot as soon as it has read it.
+__device__ __forceinline__ int ring_take(uint32_t tfull0, uint32_t tempty0, volatile int* ring, int& slot,
+                                         uint32_t& ph, volatile int* abort, int* status) {
+  int tile = -2;
+  if (mbar_wait(tfull0 + 8 * slot, ph, abort, status, kSiteTileFull)) tile = ring[slot];
+  mbar_arrive(tempty0 + 8 * slot);
+  if (++slot == kTileRing) {
+    slot = 0;
+    ph ^= 1u;
+  }
+  return tile;
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -85,13 +109,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBarOffset);
-  const uint32_t full0 = smem_u32(bars);
-  const uint32_t empty0 = smem_u32(bars + kStages);
-  const uint32_t tfull0 = smem_u32(bars + 2 * kStages);
-  const uint32_t tempty0 = smem_u32(bars + 2 * kStages + 2);
-  const uint32_t drain_bar = smem_u32(bars + 2 * kStages + 4);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 5);
+  const int SA = a.stages_a, SB = a.stages_b;
+  const uint32_t sA = smem_u32(smem);
+  const uint32_t sB = sA + SA * kStageA;
+  const uint32_t sStage = sB + SB * kStageB;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SA * kStageA + SB * kStageB + 4 * a.staging_bufs * a.staging_bytes);
+  const uint32_t fullA0 = smem_u32(bars);
+  const uint32_t emptyA0 = fullA0 + 8 * SA;
+  const uint32_t fullB0 = emptyA0 + 8 * SA;
+  const uint32_t emptyB0 = fullB0 + 8 * SB;
+  const uint32_t tfull0 = emptyB0 + 8 * SB;
+  const uint32_t tempty0 = tfull0 + 16;
+  const uint32_t ringfull0 = tempty0 + 16;
+  const uint32_t ringempty0 = ringfull0 + 8 * kTileRing;
+  const uint32_t drain_bar = ringempty0 + 8 * kTileRing;
+  volatile int* ring = reinterpret_cast<volatile int*>(bars + 2 * SA + 2 * SB + 4 + 2 * kTileRing + 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(const_cast<int*>(ring) + kTileRing);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -99,24 +132,31 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool gather_a = a.mode == 0;
 
   if (threadIdx.x == 0) {
-    // GEMM1: the B copy's expect-tx arrival plus one cp.async arrival per gather thread
-    const uint32_t full_count = gather_a ? 1 + 32 * kNumAWarps : 1;
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(full0 + 8 * s, full_count);
-      mbar_init(empty0 + 8 * s, 1);
+    for (int s = 0; s < SA; ++s) {
+      // GEMM1: one cp.async arrival per gather thread; GEMM2: the TMA expect-tx arrival
+      mbar_init(fullA0 + 8 * s, gather_a ? 32 * kNumAWarps : 1);
+      mbar_init(emptyA0 + 8 * s, 1);
+    }
+    for (int s = 0; s < SB; ++s) {
+      mbar_init(fullB0 + 8 * s, 1);
+      mbar_init(emptyB0 + 8 * s, 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull0 + 8 * b, 1);
       mbar_init(tempty0 + 8 * b, 128);
     }
+    // tile-ring readers: the A warps (4 gathering, or the one TMA warp), MMA, 4 epilogue warps
+    const uint32_t readers = (gather_a ? kNumAWarps : 1) + 1 + 4;
+    for (int s = 0; s < kTileRing; ++s) {
+      mbar_init(ringfull0 + 8 * s, 1);
+      mbar_init(ringempty0 + 8 * s, readers);
+    }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == kWarpTma && lane == 0) {
-    prefetch_tmap(&tmB);
-    if (!gather_a) prefetch_tmap(&tmA);
-  }
+  if (warp == kWarpSched && lane == 0) prefetch_tmap(&tmB);
+  if (warp == 0 && lane == 0 && !gather_a) prefetch_tmap(&tmA);
   if (warp == kWarpEpi && lane == 0) prefetch_tmap(&tmC);
   if (warp == kWarpMma) {
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
@@ -134,132 +174,151 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp < kNumAWarps) {
     if (gather_a) {
-      // ---------------- A gather (cp.async) ----------------
+      // ---------------- A gather (cp.async), all 4 warps ----------------
       const int t = threadIdx.x;  // 0..127
       const int c = t & 7;        // 16-byte chunk of the 128-byte K slice
       const int r0 = t >> 3;      // rows r0 + 16 i, i = 0..7
-      int stage = 0;
-      uint32_t phase = 0;
-      int tok_next[8];
-      if (static_cast<int>(blockIdx.x) < num_tiles) {
-        const int mb = blockIdx.x / a.n_tiles;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) tok_next[i] = token_of(a, mb * kBM + r0 + 16 * i);
-      }
-      bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      int rslot = 0, sa = 0;
+      uint32_t rph = 0, pha = 0;
+      while (true) {
+        int tile = 0;
+        if (lane == 0) tile = ring_take(ringfull0, ringempty0, ring, rslot, rph, abort_flag, a.status);
+        tile = __shfl_sync(0xffffffffu, tile, 0);
+        if (tile < 0) break;
+        const int mb = tile / a.n_tiles;
         const uint8_t* src[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i)
-          src[i] = a.a_rows + static_cast<size_t>(tok_next[i]) * a.a_row_bytes + c * 16;
-        const int next = tile + gridDim.x;
-        if (next < num_tiles) {  // prefetch the next tile's token rows
-          const int mb = next / a.n_tiles;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) tok_next[i] = token_of(a, mb * kBM + r0 + 16 * i);
-        }
+          src[i] = a.a_rows + static_cast<size_t>(token_of(a, mb * kBM + r0 + 16 * i)) * a.a_row_bytes + c * 16;
+        bool ok = true;
         for (int kb = 0; kb < a.k_blocks; ++kb) {
           int got = 0;
-          if (lane == 0) got = mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, a.status, kSiteEmptyA);
-          got = __shfl_sync(0xffffffffu, got, 0);
-          if (!got) {
+          if (lane == 0) got = mbar_wait(emptyA0 + 8 * sa, pha ^ 1u, abort_flag, a.status, kSiteEmptyA);
+          if (!__shfl_sync(0xffffffffu, got, 0)) {
             ok = false;
             break;
           }
-          const uint32_t base = smem_u32(smem + stage * kStageBytes);
+          const uint32_t base = sA + sa * kStageA;
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             const int r = r0 + 16 * i;
             cp_async16(base + r * kBKBytes + ((c ^ (r & 7)) << 4), src[i] + kb * kBKBytes);
           }
-          cp_async_mbar_arrive(full0 + 8 * stage);
-          if (++stage == kStages) {
-            stage = 0;
-            phase ^= 1u;
+          cp_async_mbar_arrive(fullA0 + 8 * sa);
+          if (++sa == SA) {
+            sa = 0;
+            pha ^= 1u;
           }
         }
+        if (!ok) break;
       }
       cp_async_wait_all();  // no copy may land after the CTA exits
-    }
-  } else if (warp == kWarpTma) {
-    // ---------------- TMA producer ----------------
-    if (lane == 0) {
-      const uint64_t pol_w = policy_evict_first();  // weights: streamed once
-      const uint64_t pol_a = policy_evict_last();   // activations: reused across N tiles
-      const uint32_t bytes = static_cast<uint32_t>(a.BN) * kBKBytes + (gather_a ? 0u : kStageA);
-      int stage = 0;
-      uint32_t phase = 0;
-      long long issued = 0;
+    } else if (warp == 0 && lane == 0) {
+      // ---------------- A tile (TMA), GEMM2 ----------------
+      const uint64_t pol_a = policy_evict_last();
+      int rslot = 0, sa = 0;
+      uint32_t rph = 0, pha = 0;
       bool ok = true;
-      int e_next = static_cast<int>(blockIdx.x) < num_tiles ? a.block_expert[blockIdx.x / a.n_tiles] : 0;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      while (ok) {
+        const int tile = ring_take(ringfull0, ringempty0, ring, rslot, rph, abort_flag, a.status);
+        if (tile < 0) break;
         const int mb = tile / a.n_tiles;
-        const int nt = tile - mb * a.n_tiles;
-        const int e = e_next;
-        const int next = tile + gridDim.x;
-        if (next < num_tiles) e_next = a.block_expert[next / a.n_tiles];
-        const int brow = e * a.w_rows_per_expert + nt * a.BN;
         for (int kb = 0; kb < a.k_blocks; ++kb) {
-          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, a.status, kSiteEmpty)) {
+          if (!mbar_wait(emptyA0 + 8 * sa, pha ^ 1u, abort_flag, a.status, kSiteEmptyA)) {
             ok = false;
             break;
           }
-          const uint32_t full = full0 + 8 * stage;
-          const uint32_t a_dst = smem_u32(smem + stage * kStageBytes);
-          mbar_arrive_expect_tx(full, bytes);
-          // GEMM1 streams each weight tile once; GEMM2's weight tiles are short rows
-          // re-read at the next K step, so they keep the normal eviction priority
-          tma_load_2d(a_dst + kStageA, &tmB, full, kb * 64, brow, gather_a ? pol_w : pol_a);
-          if (!gather_a) tma_load_2d(a_dst, &tmA, full, kb * 64, mb * kBM, pol_a);
-          ++issued;
-          if (++stage == kStages) {
-            stage = 0;
-            phase ^= 1u;
+          mbar_arrive_expect_tx(fullA0 + 8 * sa, kStageA);
+          tma_load_2d(sA + sa * kStageA, &tmA, fullA0 + 8 * sa, kb * 64, mb * kBM, pol_a);
+          if (++sa == SA) {
+            sa = 0;
+            pha ^= 1u;
           }
         }
       }
-      if (!ok) {
-        // wait (bounded) for the last copy issued into each stage
-        for (int s = 0; s < kStages; ++s) {
-          if (issued <= s) break;
-          const long long last = issued - 1 - ((issued - 1 - s) % kStages);
-          mbar_wait_drain(full0 + 8 * s, static_cast<uint32_t>((last / kStages) & 1));
+    }
+  } else if (warp == kWarpSched) {
+    // ---------------- tile scheduler + B producer ----------------
+    if (lane == 0) {
+      // GEMM1 streams each weight tile once; GEMM2's weight rows are short and re-read at
+      // the next K step, so they keep the normal eviction priority
+      const uint64_t pol_b = gather_a ? policy_evict_first() : policy_evict_last();
+      const uint32_t b_bytes = static_cast<uint32_t>(a.BN) * kBKBytes;
+      int wslot = 0, sb = 0;
+      uint32_t wph = 0, phb = 0;
+      int tile = atomicAdd(a.tile_counter, 1);
+      while (true) {
+        if (!mbar_wait(ringempty0 + 8 * wslot, wph ^ 1u, abort_flag, a.status, kSiteTileEmpty)) break;
+        const bool done = tile >= num_tiles;
+        ring[wslot] = done ? -1 : tile;
+        mbar_arrive(ringfull0 + 8 * wslot);  // release: the ring entry is visible to its readers
+        if (++wslot == kTileRing) {
+          wslot = 0;
+          wph ^= 1u;
         }
+        if (done) break;
+        const int next = atomicAdd(a.tile_counter, 1);  // its latency overlaps this tile's loads
+        const int mb = tile / a.n_tiles;
+        const int nt = tile - mb * a.n_tiles;
+        const int brow = a.block_expert[mb] * a.w_rows_per_expert + nt * a.BN;
+        bool ok = true;
+        for (int kb = 0; kb < a.k_blocks; ++kb) {
+          if (!mbar_wait(emptyB0 + 8 * sb, phb ^ 1u, abort_flag, a.status, kSiteEmptyB)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(fullB0 + 8 * sb, b_bytes);
+          tma_load_2d(sB + sb * kStageB, &tmB, fullB0 + 8 * sb, kb * 64, brow, pol_b);
+          if (++sb == SB) {
+            sb = 0;
+            phb ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tile = next;
       }
     }
   } else if (warp == kWarpMma) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16(kBM, a.BN);
-      int stage = 0;
-      uint32_t phase = 0;
+      int rslot = 0, sa = 0, sb = 0;
+      uint32_t rph = 0, pha = 0, phb = 0;
       int it = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
+      while (ok) {
+        const int tile = ring_take(ringfull0, ringempty0, ring, rslot, rph, abort_flag, a.status);
+        if (tile < 0) break;
         const int acc = it & 1;
         const uint32_t aphase = (it >> 1) & 1;
         if (!mbar_wait(tempty0 + 8 * acc, aphase ^ 1u, abort_flag, a.status, kSiteTmemEmpty)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * kAccCols;
         for (int kb = 0; kb < a.k_blocks; ++kb) {
-          if (!mbar_wait(full0 + 8 * stage, phase, abort_flag, a.status, kSiteFull)) {
+          if (!mbar_wait(fullA0 + 8 * sa, pha, abort_flag, a.status, kSiteFullA) ||
+              !mbar_wait(fullB0 + 8 * sb, phb, abort_flag, a.status, kSiteFullB)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(smem + stage * kStageBytes);
-          const uint64_t adesc = umma_desc_sw128(a_addr);
-          const uint64_t bdesc = umma_desc_sw128(a_addr + kStageA);
+          const uint64_t adesc = umma_desc_sw128(sA + sa * kStageA);
+          const uint64_t bdesc = umma_desc_sw128(sB + sb * kStageB);
 #pragma unroll
           for (int k = 0; k < 4; ++k)  // 4 x K=16 bf16 = 128 bytes; +32 bytes = +2 encoded
             umma_bf16(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb | k) != 0);
-          umma_commit(empty0 + 8 * stage);
-          if (++stage == kStages) {
-            stage = 0;
-            phase ^= 1u;
+          umma_commit(emptyA0 + 8 * sa);  // each arrives once these MMAs have read the stage
+          umma_commit(emptyB0 + 8 * sb);
+          if (++sa == SA) {
+            sa = 0;
+            pha ^= 1u;
+          }
+          if (++sb == SB) {
+            sb = 0;
+            phb ^= 1u;
           }
         }
         if (ok) umma_commit(tfull0 + 8 * acc);
+        ++it;
       }
       // all MMAs of this thread complete before TMEM is released
       umma_commit(drain_bar);
@@ -269,17 +328,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------- epilogue (warps 6..9) ----------------
     // Each warp owns 32 accumulator rows (its TMEM lane quadrant). Per 32 accumulator
     // columns it writes one box of 32 output rows to shared memory and stores it with a
-    // TMA tensor store; two staging buffers let the next box be written while the
+    // TMA tensor store; with two staging buffers the next box is written while the
     // previous store drains.
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
-    const uint32_t staging = smem_u32(smem + kStagingOffset + (warp - kWarpEpi) * kStagingBytes);
+    const uint32_t staging = sStage + (warp - kWarpEpi) * a.staging_bufs * a.staging_bytes;
     const bool gated = a.activation == 0;
     // GEMM1: act bf16 rows of 16 (gated) or 32 (relu2) columns per box, no swizzle;
     // GEMM2: y fp32 rows of 32 columns (128 B), 128-byte swizzle
     const int box_cols = a.mode == 0 ? (gated ? 16 : 32) : 32;
     int nst = 0;  // boxes this warp has staged (selects the staging buffer)
     int it = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+    int rslot = 0;
+    uint32_t rph = 0;
+    while (true) {
+      int tile = 0;
+      if (lane == 0) tile = ring_take(ringfull0, ringempty0, ring, rslot, rph, abort_flag, a.status);
+      tile = __shfl_sync(0xffffffffu, tile, 0);
+      if (tile < 0) break;
       const int acc = it & 1;
       const uint32_t aphase = (it >> 1) & 1;
       const bool got = mbar_wait(tfull0 + 8 * acc, aphase, abort_flag, a.status, kSiteTmemFull);
@@ -295,9 +360,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int col0 = nt * (a.mode == 0 && gated ? a.BN / 2 : a.BN);
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * kAccCols;
       for (int c = 0; c < a.BN / 32; ++c, ++nst) {
-        const uint32_t buf = staging + (nst & 1) * kStagingBuf;
-        if (nst >= 2) {
-          if (lane == 0) bulk_wait_group_read<1>();  // the store that last used `buf` has read it
+        const uint32_t buf = staging + (nst % a.staging_bufs) * a.staging_bytes;
+        if (nst >= a.staging_bufs && lane == 0) {
+          // the store that last used `buf` has finished reading it
+          if (a.staging_bufs == 2)
+            bulk_wait_group_read<1>();
+          else
+            bulk_wait_group_read<0>();
         }
         __syncwarp();  // also: tcgen05.ld below is .sync.aligned
         uint32_t v[32];
@@ -350,6 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
       mbar_arrive(tempty0 + 8 * acc);
+      ++it;
     }
     if (lane == 0) bulk_wait_group<0>();  // stores complete before the CTA retires
   }
@@ -361,6 +431,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, kTmemCols);
   }
+  if (threadIdx.x == 0) {
+    // the last CTA to finish resets the tile counter for the next launch (every CTA's
+    // scheduler has taken its last tile before its CTA gets here)
+    __threadfence();
+    if (atomicAdd(a.tile_counter + 1, 1) == static_cast<int>(gridDim.x) - 1) {
+      a.tile_counter[0] = 0;
+      a.tile_counter[1] = 0;
+    }
+  }
 }
 
 bool g_attr_set[64] = {};
@@ -371,20 +450,21 @@ cudaError_t launch(const Launch& l, const CUtensorMap& tmA, const CUtensorMap& t
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   if (dev < 64 && !g_attr_set[dev]) {
-    err = cudaFuncSetAttribute(gemm_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    err = cudaFuncSetAttribute(gemm_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemCap);
     if (err != cudaSuccess) return err;
     g_attr_set[dev] = true;
   }
+  const int smem = smem_bytes(args.stages_a, args.stages_b, args.staging_bufs, args.staging_bytes);
+  if (smem > kSmemCap) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg;
   cudaLaunchAttribute attr[1];
-  make_launch_config(&cfg, attr, l, dim3(num_sms), dim3(kThreads), kSmemBytes);
+  make_launch_config(&cfg, attr, l, dim3(num_sms), dim3(kThreads), smem);
   return cudaLaunchKernelEx(&cfg, gemm_bf16_kernel, tmA, tmB, tmC, args);
 }
 
 Args make_args(int mode, const GemmShape& s, const GemmBuffers& b, const void* a_rows) {
   Args a;
   a.mode = mode;
-  a.K = s.K;
   a.BN = s.BN;
   a.n_tiles = s.N / s.BN;
   a.k_blocks = (s.K + 63) / 64;
@@ -392,28 +472,38 @@ Args make_args(int mode, const GemmShape& s, const GemmBuffers& b, const void* a
   a.k_total = s.k_total;
   a.num_pairs = s.num_pairs;
   a.activation = s.activation;
-  a.out_cols = s.out_cols;
+  // 224 KB of rings and staging either way; GEMM1 boxes are at most 64 B x 32 rows
+  a.stages_a = 3;
+  a.stages_b = 5;
+  a.staging_bufs = mode == 0 ? 2 : 1;
+  a.staging_bytes = mode == 0 ? 2048 : 4096;
   a.a_rows = static_cast<const uint8_t*>(a_rows);
   a.a_row_bytes = s.K * 2;
   a.num_blocks = b.num_blocks;
   a.block_expert = b.block_expert;
   a.sorted_pair_ids = b.sorted_pair_ids;
   a.topk_w = b.topk_w;
-  a.out = b.out;
+  a.tile_counter = b.tile_counter;
   a.status = b.status;
   return a;
 }
 
 }  // namespace
 
-int pick_bn(int N, bool gated) {
-  (void)gated;
-  for (int bn = kMaxBN; bn >= 32; bn -= 32)
-    if (N % bn == 0) return bn;
-  return 0;
+int pick_bn(int N, long long est_row_tiles, int num_sms) {
+  // the widest N tile (multiple of 32 dividing N) that still gives every SM a tile;
+  // decode-sized batches have a handful of row tiles and need narrow N tiles to spread
+  // the weight stream over all SMs
+  int best = 0;
+  for (int bn = kMaxBN; bn >= 32; bn -= 32) {
+    if (N % bn != 0) continue;
+    best = bn;
+    if (est_row_tiles * (N / bn) >= num_sms) return bn;
+  }
+  return best;
 }
 
-size_t gemm_bf16_smem_bytes() { return kSmemBytes; }
+size_t gemm_bf16_smem_bytes() { return kSmemCap; }
 
 cudaError_t launch_gemm1_bf16(const Launch& l, const void* hidden, const CUtensorMap& tm_w13,
                               const CUtensorMap& tm_act_store, const GemmShape& s, const GemmBuffers& b) {

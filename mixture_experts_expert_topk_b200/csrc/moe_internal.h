@@ -24,7 +24,7 @@ void make_launch_config(cudaLaunchConfig_t* cfg, cudaLaunchAttribute* attr, cons
 // ---- route (route.cu) ----
 cudaError_t launch_route(const Launch& l, const float* logits, int T, int E_routed, int topk,
                          int num_shared, int renormalize, int* topk_ids, float* topk_w,
-                         int* status);
+                         int* status, const void* hidden, int hidden_row_bytes);
 
 // ---- align (align.cu) ----
 cudaError_t launch_align(const Launch& l, const int* topk_ids, int P, int E, int block_m,
@@ -57,24 +57,30 @@ struct GemmBuffers {
   int w_scale_rows;         // FP8: rows of w_scale per expert
   int w_scale_cols;         // FP8: columns of w_scale (K/128)
   int up_block_offset;      // FP8 GEMM1: row-block offset of the up half (I/128)
+  int* tile_counter;        // [2] work counter of the persistent kernel; 0 between launches
   int* status;
 };
-int pick_bn(int N, bool gated);
+// N tile for a GEMM with N output columns, given an estimate of the number of 128-row
+// tiles and the SM count (0 if no multiple of 32 divides N).
+int pick_bn(int N, long long est_row_tiles, int num_sms);
 size_t gemm_bf16_smem_bytes();
 cudaError_t launch_gemm1_bf16(const Launch& l, const void* hidden, const CUtensorMap& tm_w13,
                               const CUtensorMap& tm_act_store, const GemmShape& s, const GemmBuffers& b);
 cudaError_t launch_gemm2_bf16(const Launch& l, const CUtensorMap& tm_act, const CUtensorMap& tm_w2,
                               const CUtensorMap& tm_y_store, const GemmShape& s, const GemmBuffers& b);
 size_t gemm_fp8_smem_bytes();
-cudaError_t launch_gemm1_fp8(const Launch& l, const CUtensorMap& tm_xq, const CUtensorMap& tm_w13,
-                             const GemmShape& s, const GemmBuffers& b);
+cudaError_t launch_gemm1_fp8(const Launch& l, const void* xq, const CUtensorMap& tm_w13,
+                             const CUtensorMap& tm_act_store, const GemmShape& s, const GemmBuffers& b);
 cudaError_t launch_gemm2_fp8(const Launch& l, const CUtensorMap& tm_actq, const CUtensorMap& tm_w2,
-                             const GemmShape& s, const GemmBuffers& b);
+                             const CUtensorMap& tm_y_store, const GemmShape& s, const GemmBuffers& b);
 
 // ---- elementwise (combine.cu, quant.cu, prepare.cu) ----
 cudaError_t launch_combine(const Launch& l, const void* y, const int* pair_to_row, int T, int k_total, int H,
                            void* out);
 cudaError_t launch_quant_act(const Launch& l, const void* x, int T, int H, void* q, float* scale);
+// As launch_quant_act over the first num_blocks[0] * block_m of max_rows rows.
+cudaError_t launch_quant_rows(const Launch& l, const void* x, int max_rows, int cols, const int* num_blocks,
+                              int block_m, void* q, float* scale);
 cudaError_t launch_quant_weights(const Launch& l, const void* w, int64_t num_mats, int rows,
                                  int cols, void* q, float* scale);
 cudaError_t launch_prepare_w13(const Launch& l, const void* in, void* out, int E, int I_in,

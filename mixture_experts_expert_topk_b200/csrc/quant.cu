@@ -22,13 +22,16 @@ __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
   return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
 }
 
-// One warp per (token, 128-column group): lane l quantises columns 4l..4l+3.
+// One warp per (row, 128-column group): lane l quantises columns 4l..4l+3. When
+// `num_blocks` is given, only the first num_blocks[0] * block_m rows are processed.
 __global__ void __launch_bounds__(256)
     quant_act_kernel(const uint2* __restrict__ x, int T, int G, uint32_t* __restrict__ q,
-                     float* __restrict__ scale) {
+                     float* __restrict__ scale, const int* __restrict__ num_blocks, int block_m) {
   griddep_wait();
+  griddep_launch_dependents();
   const long long g = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
-  if (g >= static_cast<long long>(T) * G) return;
+  const long long rows = num_blocks != nullptr ? static_cast<long long>(*num_blocks) * block_m : T;
+  if (g >= rows * G) return;
   const int lane = threadIdx.x & 31;
   const uint2 raw = x[g * 32 + lane];
   const float2 f01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.x));
@@ -100,7 +103,18 @@ cudaError_t launch_quant_act(const Launch& l, const void* x, int T, int H, void*
   cudaLaunchAttribute attr[1];
   make_launch_config(&cfg, attr, l, dim3(static_cast<unsigned>((groups + 7) / 8)), dim3(256), 0);
   return cudaLaunchKernelEx(&cfg, quant_act_kernel, static_cast<const uint2*>(x), T, G,
-                            static_cast<uint32_t*>(q), scale);
+                            static_cast<uint32_t*>(q), scale, static_cast<const int*>(nullptr), 1);
+}
+
+cudaError_t launch_quant_rows(const Launch& l, const void* x, int max_rows, int cols, const int* num_blocks,
+                              int block_m, void* q, float* scale) {
+  const int G = cols / 128;
+  const long long groups = static_cast<long long>(max_rows) * G;
+  cudaLaunchConfig_t cfg;
+  cudaLaunchAttribute attr[1];
+  make_launch_config(&cfg, attr, l, dim3(static_cast<unsigned>((groups + 7) / 8)), dim3(256), 0);
+  return cudaLaunchKernelEx(&cfg, quant_act_kernel, static_cast<const uint2*>(x), max_rows, G,
+                            static_cast<uint32_t*>(q), scale, num_blocks, block_m);
 }
 
 cudaError_t launch_quant_weights(const Launch& l, const void* w, int64_t num_mats, int rows, int cols,

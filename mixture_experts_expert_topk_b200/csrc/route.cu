@@ -37,14 +37,18 @@ template <int VPL>
 __global__ void __launch_bounds__(kRouteWarps * 32)
     route_kernel(const float* __restrict__ logits, int T, int E, int topk, int num_shared,
                  int renormalize, int* __restrict__ topk_ids, float* __restrict__ topk_w,
-                 int* __restrict__ status) {
+                 int* __restrict__ status, const uint8_t* __restrict__ hidden, int hidden_row_bytes) {
   griddep_wait();
   griddep_launch_dependents();
-  // routing starts every forward: clear the device status word of the workspace
-  if (blockIdx.x == 0 && threadIdx.x == 0) *status = 0;
+  // routing starts every forward: clear the workspace's status word ([0]) and the GEMMs'
+  // work counters ([4..7])
+  if (blockIdx.x == 0 && threadIdx.x < 8) status[threadIdx.x] = 0;
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * kRouteWarps + (threadIdx.x >> 5);
   if (t >= T) return;
+  // start pulling this token's hidden row into L2: GEMM1 gathers it k times right after
+  if (hidden != nullptr && lane == 0)
+    prefetch_l2_bulk(hidden + static_cast<size_t>(t) * hidden_row_bytes, static_cast<uint32_t>(hidden_row_bytes));
   const float* row = logits + static_cast<size_t>(t) * E;
 
   // lane holds experts lane, lane + 32, ...; an expert's index is lane + 32 * i
@@ -109,27 +113,28 @@ __global__ void __launch_bounds__(kRouteWarps * 32)
 
 template <int VPL>
 cudaError_t launch_vpl(const Launch& l, const float* logits, int T, int E, int topk,
-                       int num_shared, int renormalize, int* ids, float* w, int* status) {
+                       int num_shared, int renormalize, int* ids, float* w, int* status,
+                       const void* hidden, int hidden_row_bytes) {
   cudaLaunchConfig_t cfg;
   cudaLaunchAttribute attr[1];
   make_launch_config(&cfg, attr, l, dim3((T + kRouteWarps - 1) / kRouteWarps),
                      dim3(kRouteWarps * 32), 0);
   return cudaLaunchKernelEx(&cfg, route_kernel<VPL>, logits, T, E, topk, num_shared, renormalize,
-                            ids, w, status);
+                            ids, w, status, static_cast<const uint8_t*>(hidden), hidden_row_bytes);
 }
 
 }  // namespace
 
 cudaError_t launch_route(const Launch& l, const float* logits, int T, int E_routed, int topk,
                          int num_shared, int renormalize, int* topk_ids, float* topk_w,
-                         int* status) {
+                         int* status, const void* hidden, int hidden_row_bytes) {
   const int vpl = (E_routed + 31) / 32;
-  if (vpl <= 1) return launch_vpl<1>(l, logits, T, E_routed, topk, num_shared, renormalize, topk_ids, topk_w, status);
-  if (vpl <= 2) return launch_vpl<2>(l, logits, T, E_routed, topk, num_shared, renormalize, topk_ids, topk_w, status);
-  if (vpl <= 4) return launch_vpl<4>(l, logits, T, E_routed, topk, num_shared, renormalize, topk_ids, topk_w, status);
-  if (vpl <= 8) return launch_vpl<8>(l, logits, T, E_routed, topk, num_shared, renormalize, topk_ids, topk_w, status);
-  if (vpl <= 16) return launch_vpl<16>(l, logits, T, E_routed, topk, num_shared, renormalize, topk_ids, topk_w, status);
-  return launch_vpl<32>(l, logits, T, E_routed, topk, num_shared, renormalize, topk_ids, topk_w, status);
+  if (vpl <= 1) return launch_vpl<1>(l, logits, T, E_routed, topk, num_shared, renormalize, topk_ids, topk_w, status, hidden, hidden_row_bytes);
+  if (vpl <= 2) return launch_vpl<2>(l, logits, T, E_routed, topk, num_shared, renormalize, topk_ids, topk_w, status, hidden, hidden_row_bytes);
+  if (vpl <= 4) return launch_vpl<4>(l, logits, T, E_routed, topk, num_shared, renormalize, topk_ids, topk_w, status, hidden, hidden_row_bytes);
+  if (vpl <= 8) return launch_vpl<8>(l, logits, T, E_routed, topk, num_shared, renormalize, topk_ids, topk_w, status, hidden, hidden_row_bytes);
+  if (vpl <= 16) return launch_vpl<16>(l, logits, T, E_routed, topk, num_shared, renormalize, topk_ids, topk_w, status, hidden, hidden_row_bytes);
+  return launch_vpl<32>(l, logits, T, E_routed, topk, num_shared, renormalize, topk_ids, topk_w, status, hidden, hidden_row_bytes);
 }
 
 }  // namespace moe

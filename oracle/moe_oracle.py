@@ -60,6 +60,18 @@ def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
     return b.view(np.float32)
 
 
+def round_to_bf16(x: np.ndarray) -> np.ndarray:
+    """Round to bf16 (8 significant bits, round to nearest even) via float32.
+
+    The value is first rounded to float32 (the precision the activation is computed
+    in) and then to bf16, returned as float32. Finite inputs only.
+    """
+    b = np.ascontiguousarray(np.asarray(x, dtype=np.float32)).view(np.uint32).astype(np.uint64)
+    lsb = (b >> 16) & 1
+    r = ((b + 0x7FFF + lsb) >> 16) << 16
+    return r.astype(np.uint32).view(np.float32)
+
+
 def e4m3_encode(x: np.ndarray) -> np.ndarray:
     """Encode float32 values as FP8 E4M3 (the OCP "fn" variant) codes.
 
@@ -388,8 +400,11 @@ def moe_forward_fp8(hidden_bits: np.ndarray, logits: np.ndarray, w13_q, w13_s, w
         checkpoint-layout matrices w13 [E, N1, H] and w2 [E, H, I];
       * activations: the bf16 hidden rows are quantised per token per 128
         columns (``quant_groups_1x128``) before GEMM1, and the GEMM1
-        activation output, held in fp32, is quantised the same way before
-        GEMM2 (W8A8 means both GEMM inputs are 8-bit);
+        activation output is quantised the same way before GEMM2 (W8A8 means
+        both GEMM inputs are 8-bit). The activation is first stored in the
+        compute dtype, bf16 ([SWIGLU] section 1: the fused epilogue casts
+        silu(gate)*up ``.to(compute_type)`` before the store), so its 1x128
+        codes are decided on the bf16 value;
       * every product uses the exactly dequantised values q * s in float64.
     ``w13_q``/``w2_q`` are uint8 codes, ``w13_s`` [E, N1/128, H/128] and
     ``w2_s`` [E, H/128, I/128] float32 scales.
@@ -411,7 +426,7 @@ def moe_forward_fp8(hidden_bits: np.ndarray, logits: np.ndarray, w13_q, w13_s, w
         W13 = dequant_blocks_128x128(np.asarray(w13_q[e]), np.asarray(w13_s[e]))
         W2 = dequant_blocks_128x128(np.asarray(w2_q[e]), np.asarray(w2_s[e]))
         a = activation_fn(x[t_idx] @ W13.T, activation, I)
-        aq, as_ = quant_groups_1x128(a.astype(np.float32))
+        aq, as_ = quant_groups_1x128(round_to_bf16(a))
         ad = dequant_groups_1x128(aq, as_)
         y[t_idx, j_idx] = w[t_idx, j_idx].astype(np.float64)[:, None] * (ad @ W2.T)
     out = np.zeros((T, H), dtype=np.float64)
@@ -420,17 +435,19 @@ def moe_forward_fp8(hidden_bits: np.ndarray, logits: np.ndarray, w13_q, w13_s, w
     return out
 
 
-def quantize_weights_fp8(w13_bits, w2_bits):
+def quantize_weights_fp8(w13_bits, w2_bits, experts=None):
     """Quantise bf16 master weights per 128x128 block (``quant_blocks_128x128``).
 
-    Returns (w13_q, w13_s, w2_q, w2_s) in the checkpoint layout.
+    Returns (w13_q, w13_s, w2_q, w2_s) in the checkpoint layout. ``experts`` limits the
+    work to the listed experts (the others are left zero), for evaluating a few tokens
+    of a large layer.
     """
     E = w13_bits.shape[0]
-    w13_q = np.empty(w13_bits.shape, dtype=np.uint8)
-    w2_q = np.empty(w2_bits.shape, dtype=np.uint8)
-    w13_s = np.empty((E, w13_bits.shape[1] // 128, w13_bits.shape[2] // 128), dtype=np.float32)
-    w2_s = np.empty((E, w2_bits.shape[1] // 128, w2_bits.shape[2] // 128), dtype=np.float32)
-    for e in range(E):
+    w13_q = np.zeros(w13_bits.shape, dtype=np.uint8)
+    w2_q = np.zeros(w2_bits.shape, dtype=np.uint8)
+    w13_s = np.zeros((E, w13_bits.shape[1] // 128, w13_bits.shape[2] // 128), dtype=np.float32)
+    w2_s = np.zeros((E, w2_bits.shape[1] // 128, w2_bits.shape[2] // 128), dtype=np.float32)
+    for e in (range(E) if experts is None else experts):
         w13_q[e], w13_s[e] = quant_blocks_128x128(bf16_bits_to_f32(np.asarray(w13_bits[e])))
         w2_q[e], w2_s[e] = quant_blocks_128x128(bf16_bits_to_f32(np.asarray(w2_bits[e])))
     return w13_q, w13_s, w2_q, w2_s

@@ -23,6 +23,7 @@ from _cases import GpuRun, bf16_to_f64, bits, cpu_inputs, err_beyond_rounding, m
 pytestmark = pytest.mark.gpu
 
 BF16_TOL = 2e-2
+FP8_TOL = 5e-2
 
 
 def _small(name, **kw) -> MoeConfig:
@@ -217,7 +218,9 @@ def _full_size(cfg, n_sample=48, seed=0):
     tokens = np.sort(rng.choice(cfg.T, size=min(n_sample, cfg.T), replace=False))
     fp8w = None
     if cfg.fp8:
-        fp8w = O.quantize_weights_fp8(bits(run.inp["w13"]), bits(run.inp["w2"]))
+        # the oracle quantises only the experts the sampled tokens use
+        fp8w = O.quantize_weights_fp8(bits(run.inp["w13"]), bits(run.inp["w2"]),
+                                      experts=np.unique(ids[tokens]))
     ref = oracle_out(cfg, run.inp, tokens=tokens, fp8_weights=fp8w)
     got = bf16_to_f64(out)[tokens]
     assert np.all(np.isfinite(bf16_to_f64(out)))
@@ -225,11 +228,13 @@ def _full_size(cfg, n_sample=48, seed=0):
     return err_beyond_rounding(got, ref), run
 
 
-@pytest.mark.parametrize("name,n_sample", [("prefill", 4096), ("relu2", 512)])
+@pytest.mark.parametrize("name,n_sample", [("prefill", 4096), ("relu2", 512), ("fp8_shared", 8)])
 def test_workload_full_size(name, n_sample):
-    # prefill: every token; relu2 (541 GFLOP in float64): a quarter of the tokens
-    e, run = _full_size(CONFIGS[name], n_sample=n_sample)
-    assert e <= BF16_TOL, e
+    # prefill: every token; relu2 (541 GFLOP in float64): a quarter of the tokens;
+    # FP8 with the shared slot: 8 tokens (the oracle quantises each expert they touch)
+    cfg = CONFIGS[name]
+    e, run = _full_size(cfg, n_sample=n_sample)
+    assert e <= (FP8_TOL if cfg.fp8 else BF16_TOL), e
     assert moe.device_status(run.ws)[0] == 0
 
 
@@ -242,3 +247,45 @@ def test_decode_full(T):
     _check_route_align(cfg, parts, run.inp["logits"])
     ref = oracle_out(cfg, run.inp)
     assert err_beyond_rounding(bf16_to_f64(out), ref) <= BF16_TOL
+
+
+# ---- FP8 E4M3 W8A8 block-128 ---------------------------------------------------------
+
+FP8_SMALL = {
+    "fp8_tiny": _small("fp8_tiny", T=64, H=256, E=8, topk=2, I=256, fp8=True),
+    # several row tiles per expert, shared slot, H and I not multiples of 256
+    "fp8_shared_small": _small("fp8_shared_small", T=300, H=384, E=16, topk=3, I=384, num_shared=1, fp8=True),
+    "fp8_relu2": _small("fp8_relu2", T=96, H=256, E=6, topk=2, I=256, activation="relu2", renormalize=False,
+                        fp8=True),
+}
+
+
+@pytest.mark.parametrize("name", list(FP8_SMALL))
+def test_fp8_layer_parity_small(name):
+    cfg = FP8_SMALL[name]
+    run = GpuRun(cfg)
+    out = run.forward()
+    parts = run.parts()
+    ids, a = _check_route_align(cfg, parts, run.inp["logits"])
+    # the GPU quantises its own bf16 activation per 1x128 group: codes and scales must be
+    # what the oracle's quantiser gives for those same bf16 values
+    P_pad = int(a["P_pad"])
+    rows = np.nonzero(a["sorted_pair_ids"] < cfg.T * cfg.k_total)[0]
+    act32 = O.bf16_bits_to_f32(parts["act"][rows])
+    q, sc = O.quant_groups_1x128(act32)
+    np.testing.assert_array_equal(parts["actq"][rows], q)
+    np.testing.assert_array_equal(parts["act_scale"][rows], sc)
+    # the hidden quantisation too
+    qx, sx = O.quant_groups_1x128(O.bf16_bits_to_f32(bits(run.inp["hidden"])))
+    np.testing.assert_array_equal(parts["xq"], qx)
+    np.testing.assert_array_equal(parts["xq_scale"], sx)
+    fp8w = O.quantize_weights_fp8(bits(run.inp["w13"]), bits(run.inp["w2"]))
+    np.testing.assert_array_equal(run.w13_q.cpu().numpy(), fp8w[0])
+    np.testing.assert_array_equal(run.w13_scale.cpu().numpy(), fp8w[1])
+    ref = oracle_out(cfg, run.inp, fp8_weights=fp8w)
+    got = bf16_to_f64(out)
+    assert np.all(np.isfinite(got))
+    e = err_beyond_rounding(got, ref)
+    print(f"{name}: beyond-rounding {e:.4f}, raw {max_err_over_rms(got, ref):.4f}")
+    assert e <= FP8_TOL, e
+    assert moe.device_status(run.ws)[0] == 0

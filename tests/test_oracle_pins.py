@@ -395,7 +395,9 @@ def test_fp8_layer_equals_bf16_layer_on_dequantised_inputs():
         for j in range(k):
             e = ids[t, j]
             z = W13d[e] @ Xd[t]
-            a = (z[:I] / (1 + np.exp(-z[:I])) * z[I:]).astype(np.float32)
+            # the activation is stored as bf16 before its 1x128 quantisation
+            a = torch.from_numpy((z[:I] / (1 + np.exp(-z[:I])) * z[I:]).astype(np.float32)).to(
+                torch.bfloat16).to(torch.float32).numpy()
             asc = np.float32(np.abs(a).max() / np.float32(448))
             aq = torch.from_numpy((a / asc).astype(np.float32)).to(torch.float8_e4m3fn).to(torch.float64).numpy()
             want[t] += wts[t, j] * (W2d[e] @ (aq * asc))
@@ -469,3 +471,14 @@ def test_half_ulp_bf16_helper():
     x = np.random.default_rng(0).standard_normal(100000) * 10.0
     r = torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).to(torch.float64).numpy()
     assert np.all(np.abs(r - x.astype(np.float32)) <= half_ulp_bf16(x) * (1 + 1e-7))
+
+
+def test_round_to_bf16_matches_torch_cast():
+    rng = np.random.default_rng(12)
+    x = np.concatenate([rng.standard_normal(200000) * 10.0 ** rng.integers(-6, 6, 200000),
+                        np.float64([0.0, -0.0, 1.0, 448.0, 3.0e38, -1e-30])])
+    want = torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).to(torch.float32).numpy()
+    np.testing.assert_array_equal(O.round_to_bf16(x), want)
+    # exact ties: halfway between neighbouring bf16 values round to the even one
+    a = np.float32([1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8])
+    assert O.round_to_bf16(a).tolist() == [1.0, 1.0 + 2 * 2.0 ** -7]
