@@ -25,7 +25,7 @@ __all__ = [
     "MoeError", "Problem", "make_problem", "padded_intermediate", "workspace_layout",
     "workspace_size", "new_workspace", "prepare_weights", "quantize_weights_fp8", "moe_forward",
     "moe_forward_host", "stage_route", "stage_align", "stage_quant_act", "stage_gemm1",
-    "stage_gemm2", "stage_combine", "device_status", "read_workspace", "lib",
+    "stage_gemm2", "stage_combine", "device_status", "read_workspace", "lib", "check",
 ]
 
 _ACT = {"swiglu": MOE_ACT_SWIGLU, "silu": MOE_ACT_SWIGLU, "relu2": MOE_ACT_RELU2,

@@ -41,6 +41,7 @@ using moe::GemmShape;
 using moe::Launch;
 
 constexpr size_t kAlign = 1024;
+constexpr long long kDecodeMaxPairs = 1024;  // auto block_m: 16-row blocks up to this many pairs
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -74,7 +75,7 @@ moe_status_t make_plan(const moe_problem_t* p, Plan* pl) {
   if (p->hidden % 128 != 0) return MOE_ERR_UNSUPPORTED;
   if (p->num_routed + p->num_shared > moe::kMaxExperts) return MOE_ERR_UNSUPPORTED;
   if (p->topk + p->num_shared > moe::kMaxSlots) return MOE_ERR_UNSUPPORTED;
-  if (p->block_m != 0 && p->block_m != 128) return MOE_ERR_UNSUPPORTED;
+  if (p->block_m != 0 && p->block_m != 16 && p->block_m != 128) return MOE_ERR_UNSUPPORTED;
   if (p->hidden > (1 << 20) || p->intermediate > (1 << 20)) return MOE_ERR_UNSUPPORTED;
   // FP8: a GEMM's K blocks (H/128 and I/128) are held one per lane of a warp
   if (q.fp8 && (p->hidden > 4096 || p->intermediate > 4096)) return MOE_ERR_UNSUPPORTED;
@@ -87,8 +88,15 @@ moe_status_t make_plan(const moe_problem_t* p, Plan* pl) {
   q.I = p->intermediate;
   q.topk = p->topk;
   q.kk = q.topk + q.Es;
-  q.bm = 128;
   q.N1 = q.gated ? 2 * q.I : q.I;
+  // Row tile: 128 rows, or 16-row token blocks with the weights as the MMA's M operand
+  // when the batch is decode-sized (bf16, N1 a multiple of 128).
+  {
+    const long long P = static_cast<long long>(p->num_tokens) * (p->topk + p->num_shared);
+    const bool small_ok = !q.fp8 && q.N1 % 128 == 0;
+    if (p->block_m == 16 && !small_ok) return MOE_ERR_UNSUPPORTED;
+    q.bm = p->block_m != 0 ? p->block_m : (small_ok && P <= kDecodeMaxPairs ? 16 : 128);
+  }
   q.renorm = p->renormalize;
   q.act = p->activation;
   q.P = static_cast<long long>(q.T) * q.kk;
@@ -272,6 +280,13 @@ moe_status_t run_gemm1(const Plan& pl_in, const void* hidden, const void* w13, c
   b.out = ws_ptr<void>(ws, L.act);
   b.tile_counter = ws_ptr<int>(ws, L.status) + 4;
   CUtensorMap ta, tb;
+  if (pl.bm == 16) {
+    // decode-sized: weight tiles of 128 rows as the MMA's M operand, token rows gathered
+    if (!make_tmap_2d(&tb, w13, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, pl.H, static_cast<uint64_t>(pl.E) * pl.N1,
+                      64, 128))
+      return MOE_ERR_CUDA;
+    return cuda_status(moe::launch_gemm_decode(l, 0, tb, tb, hidden, s, b));
+  }
   if (!pl.fp8) {
     // the token rows of hidden are gathered by the kernel itself (no tensor map); the
     // activation is written in boxes of 32 rows x 16 (SwiGLU) or 32 (relu2) columns
@@ -326,6 +341,14 @@ moe_status_t run_gemm2(const Plan& pl_in, const void* w2, const float* w2_scale,
   b.tile_counter = ws_ptr<int>(ws, L.status) + 6;
   CUtensorMap ta, tb;
   const uint64_t rows = static_cast<uint64_t>(L.max_rows);
+  if (pl.bm == 16) {
+    b.out = ws_ptr<void>(ws, L.y);
+    if (!make_tmap_2d(&tb, w2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, pl.I, static_cast<uint64_t>(pl.E) * pl.H, 64,
+                      128) ||
+        !make_tmap_2d(&ta, ws_ptr<void>(ws, L.act), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, pl.I, rows, 64, 16))
+      return MOE_ERR_CUDA;
+    return cuda_status(moe::launch_gemm_decode(l, 1, tb, ta, nullptr, s, b));
+  }
   if (!pl.fp8) {
     CUtensorMap tc;  // y [max_rows, H] fp32 in sorted row order, boxes of 32 x 32
     if (!make_tmap_2d(&ta, ws_ptr<void>(ws, L.act), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, pl.I, rows, 64, 128) ||

@@ -68,6 +68,10 @@ cudaError_t launch_gemm1_bf16(const Launch& l, const void* hidden, const CUtenso
                               const CUtensorMap& tm_act_store, const GemmShape& s, const GemmBuffers& b);
 cudaError_t launch_gemm2_bf16(const Launch& l, const CUtensorMap& tm_act, const CUtensorMap& tm_w2,
                               const CUtensorMap& tm_y_store, const GemmShape& s, const GemmBuffers& b);
+// Decode-sized batches (token blocks of 16): weights as the MMA's M operand. mode 0 =
+// GEMM1 (x_rows = hidden, gathered), mode 1 = GEMM2 (tm_x = activation rows).
+cudaError_t launch_gemm_decode(const Launch& l, int mode, const CUtensorMap& tm_w, const CUtensorMap& tm_x,
+                               const void* x_rows, const GemmShape& s, const GemmBuffers& b);
 size_t gemm_fp8_smem_bytes();
 cudaError_t launch_gemm1_fp8(const Launch& l, const void* xq, const CUtensorMap& tm_w13,
                              const CUtensorMap& tm_act_store, const GemmShape& s, const GemmBuffers& b);

@@ -26,14 +26,15 @@ def cpu_inputs(cfg: MoeConfig, seed: int = 0) -> Dict[str, torch.Tensor]:
 class GpuRun:
     """One forward of ``cfg`` on cuda:0 with every intermediate kept in the workspace."""
 
-    def __init__(self, cfg: MoeConfig, seed: int = 0, inputs: Optional[dict] = None, pdl: bool = True):
+    def __init__(self, cfg: MoeConfig, seed: int = 0, inputs: Optional[dict] = None, pdl: bool = True,
+                 block_m: int = 0):
         self.cfg = cfg
         inp = inputs if inputs is not None else cpu_inputs(cfg, seed)
         self.inp = inp
         self.I_pad = moe.padded_intermediate(cfg.I, cfg.activation, cfg.fp8)
         self.prob = moe.make_problem(cfg.T, cfg.H, cfg.E, cfg.topk, self.I_pad,
                                      renormalize=cfg.renormalize, activation=cfg.activation,
-                                     num_shared=cfg.num_shared, fp8=cfg.fp8, pdl=pdl)
+                                     num_shared=cfg.num_shared, fp8=cfg.fp8, pdl=pdl, block_m=block_m)
         dev = torch.device("cuda:0")
         self.hidden = inp["hidden"].to(dev)
         self.logits = inp["logits"].to(dev)
@@ -51,16 +52,23 @@ class GpuRun:
         self.out = torch.empty_like(self.hidden)
 
     def forward(self) -> torch.Tensor:
-        moe.moe_forward(self.hidden, self.logits, self.w13p, self.w2p, self.cfg.topk,
-                        self.cfg.renormalize, self.cfg.activation, self.w13_scale, self.w2_scale,
-                        num_shared=self.cfg.num_shared, workspace=self.ws, out=self.out,
-                        pdl=bool(self.prob.flags & 1))
+        # through the C ABI with this run's problem (block_m included)
+        import ctypes
+        L = moe.lib()
+        st = L.moe_forward(ctypes.byref(self.prob), ctypes.c_void_p(self.hidden.data_ptr()),
+                           ctypes.c_void_p(self.logits.data_ptr()), ctypes.c_void_p(self.w13p.data_ptr()),
+                           ctypes.c_void_p(self.w2p.data_ptr()),
+                           None if self.w13_scale is None else ctypes.c_void_p(self.w13_scale.data_ptr()),
+                           None if self.w2_scale is None else ctypes.c_void_p(self.w2_scale.data_ptr()),
+                           ctypes.c_void_p(self.out.data_ptr()), ctypes.c_void_p(self.ws.data_ptr()),
+                           self.ws.numel(), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+        moe.check(st, "moe_forward")
         torch.cuda.synchronize()
         return self.out
 
     def parts(self) -> Dict[str, np.ndarray]:
         v = moe.read_workspace(self.prob, self.ws)
-        out = {}
+        out = {"block_m": moe.workspace_layout(self.prob)["block_m"]}
         for k, t in v.items():
             if t.dtype == torch.bfloat16:
                 out[k] = bits(t)

@@ -58,7 +58,7 @@ def test_check_problem_accepts_the_workloads(L):
     (dict(topk=9), 1), (dict(topk=0), 1), (dict(intermediate=500), 1),
     (dict(intermediate=512, activation="relu2"), 0), (dict(intermediate=528, activation="relu2"), 1),
     (dict(num_routed=1100, topk=2), 2), (dict(num_routed=32, topk=17), 2),
-    (dict(block_m=64), 2), (dict(intermediate=528, fp8=True), 1),
+    (dict(block_m=64), 2), (dict(intermediate=528, fp8=True), 1), (dict(block_m=16, fp8=True), 2),
 ])
 def test_check_problem_rejects(L, kw, status):
     p = _prob(**kw)
@@ -96,7 +96,10 @@ def test_workspace_layout(L):
         P = cfg.T * cfg.k_total
         E = cfg.E_total
         assert lay["status"] == 0
-        assert lay["max_rows"] == -(-(P + min(E, P) * 127) // 128) * 128
+        bm = lay["block_m"]
+        # decode-sized bf16 batches use 16-row token blocks, everything else 128-row tiles
+        assert bm == (16 if (P <= 1024 and not cfg.fp8) else 128)
+        assert lay["max_rows"] == -(-(P + min(E, P) * (bm - 1)) // bm) * bm
         assert lay["num_chunks"] == -(-P // 2048)
         offs = sorted(v for k, v in lay.items() if k not in ("total_bytes", "max_rows", "num_chunks", "block_m"))
         assert all(o % 1024 == 0 for o in offs)

@@ -48,16 +48,17 @@ SMALL = {
 }
 
 
-def _check_route_align(cfg, parts, logits):
+def _check_route_align(cfg, parts, logits, bm=None):
     ids, w = O.route(logits.numpy(), cfg.topk, cfg.renormalize, cfg.num_shared)
     np.testing.assert_array_equal(parts["topk_ids"], ids)
     np.testing.assert_allclose(parts["topk_w"], w, rtol=1e-5, atol=1e-7)
-    a = O.align(ids, cfg.E_total, 128)
+    bm = bm or parts["block_m"]
+    a = O.align(ids, cfg.E_total, bm)
     P_pad = int(a["P_pad"])
-    assert int(parts["num_blocks"][0]) == P_pad // 128
+    assert int(parts["num_blocks"][0]) == P_pad // bm
     np.testing.assert_array_equal(parts["expert_offsets"], a["expert_offsets"])
     np.testing.assert_array_equal(parts["sorted_pair_ids"][:P_pad], a["sorted_pair_ids"])
-    np.testing.assert_array_equal(parts["block_expert"][:P_pad // 128], a["block_expert"])
+    np.testing.assert_array_equal(parts["block_expert"][:P_pad // bm], a["block_expert"])
     np.testing.assert_array_equal(parts["pair_to_row"], a["pair_to_row"])
     return ids, a
 
@@ -151,7 +152,9 @@ def test_all_tokens_one_expert_and_empty_experts():
     run.forward()
     parts = run.parts()
     ids, a = _check_route_align(cfg, parts, inp["logits"])
-    assert list(a["expert_offsets"]) == [0] * 6 + [768] * 3
+    bm = parts["block_m"]
+    seg = -(-700 // bm) * bm                      # 700 pairs padded to the row tile
+    assert list(a["expert_offsets"]) == [0] * 6 + [seg] * 3
     ref = oracle_out(cfg, inp)
     assert err_beyond_rounding(bf16_to_f64(run.out), ref) <= BF16_TOL
 
@@ -289,3 +292,17 @@ def test_fp8_layer_parity_small(name):
     print(f"{name}: beyond-rounding {e:.4f}, raw {max_err_over_rms(got, ref):.4f}")
     assert e <= FP8_TOL, e
     assert moe.device_status(run.ws)[0] == 0
+
+
+@pytest.mark.parametrize("T,bm", [(16, 128), (64, 128), (4, 16)])
+def test_decode_both_row_tilings(T, bm):
+    # the same decode batch through 16-row token blocks (weights as the MMA's M operand)
+    # and through 128-row tiles must both match the oracle
+    cfg = CONFIGS[f"decode_T{T}"]
+    run = GpuRun(cfg, block_m=bm)
+    out = run.forward()
+    parts = run.parts()
+    assert parts["block_m"] == bm
+    _check_route_align(cfg, parts, run.inp["logits"])
+    ref = oracle_out(cfg, run.inp)
+    assert err_beyond_rounding(bf16_to_f64(out), ref) <= BF16_TOL
