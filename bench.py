@@ -9,8 +9,9 @@ I=512, renormalised routing with a per-expert logit bias (skewed expert load).
 Synthetic seeded data, random-init weights.
 
 Timing: W untimed warm-up steps, then exactly K steps bracketed by a barrier and
-cuda.synchronize; each step is timed with CUDA events on the launching stream, with L2
-flushed (a 512 MB write) before every step outside the events. For N > 1 each rank runs
+cuda.synchronize; each step (the forward captured once as a CUDA graph and replayed,
+unless --no-graph) is timed with CUDA events on the launching stream, with L2 flushed (a
+512 MB write) before every step outside the events. For N > 1 each rank runs
 an independent replica (the layer needs no exchange between replicas) and the time is
 the max over ranks. Rank 0 prints one JSON line.
 
@@ -36,6 +37,11 @@ import torch  # noqa: E402
 from mixture_experts_expert_topk_b200.synth import CONFIGS, MoeConfig, make_inputs  # noqa: E402
 
 L2_FLUSH_BYTES = 512 << 20
+
+# DRAM traffic of GEMM1 relative to its algorithmic bytes, from one ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum, profiles/gemm_bf16_prefill_e64_ncu.md),
+# valid only for the kernel source it was taken on (sha256 prefix of gemm_bf16.cu).
+GEMM1_TRAFFIC = {"source_sha256": "92a46cf29e07", "ratio": 284.0 / 280.3}
 
 
 def _peaks():
@@ -189,17 +195,27 @@ def run_ours(cfg: MoeConfig, steps: int, warmup: int, world: int, rank: int, loc
     stream = torch.cuda.current_stream(dev)
     torch.cuda.synchronize(dev)
 
-    def step():
+    def forward():
         moe.moe_forward(hidden, logits, w13p, w2p, cfg.topk, cfg.renormalize, cfg.activation,
                         s13, s2, num_shared=cfg.num_shared, workspace=ws, out=out)
 
     for _ in range(warmup):
         flush.zero_()
-        step()
+        forward()
     torch.cuda.synchronize(dev)
     st = moe.device_status(ws)
     if st[0] != 0:
         raise RuntimeError(f"device status after warm-up: {st}")
+    step = forward
+    if args.graph:
+        # the whole forward (all kernels, programmatic dependent launches included) as one
+        # CUDA graph, replayed each step
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            forward()
+        graph.replay()
+        torch.cuda.synchronize(dev)
+        step = graph.replay
 
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     barrier(world)
@@ -267,6 +283,17 @@ def run_ours(cfg: MoeConfig, steps: int, warmup: int, world: int, rank: int, loc
     }
 
 
+def _gemm1_traffic(cfg: MoeConfig, g1_bytes: float):
+    """DRAM bytes per GEMM1 launch scaled from the ncu capture, or None if the kernel
+    source changed since (or the workload does not run that kernel)."""
+    import hashlib
+    src = os.path.join(ROOT, "mixture_experts_expert_topk_b200", "csrc", "gemm_bf16.cu")
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:12]
+    if cfg.fp8 or cfg.T * cfg.k_total <= 1024 or sha != GEMM1_TRAFFIC["source_sha256"]:
+        return None
+    return g1_bytes * GEMM1_TRAFFIC["ratio"]
+
+
 def cpu_baseline(cfg: MoeConfig, inp, budget_s: float, tokens_hint: int):
     """Time the CPU oracle, as it stands, on the first tokens of the workload."""
     from oracle import moe_oracle as O
@@ -307,6 +334,8 @@ def main():
     ap.add_argument("--config", default="prefill", choices=sorted(CONFIGS))
     ap.add_argument("--cpu-tokens", type=int, default=256)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", dest="graph", action="store_false",
+                    help="launch the kernels from the host each step instead of replaying a CUDA graph")
     args = ap.parse_args()
     cfg = CONFIGS[args.config]
     if args.impl == "reference":
@@ -367,14 +396,15 @@ def main():
         "us_per_call": ms_per_step * 1e3,
         "config": {"workload": _workload_name(cfg), "T": cfg.T, "H": cfg.H, "E": cfg.E_total,
                    "topk": cfg.k_total, "I": cfg.I,
-                   "l2": "flushed before every step (512 MB write, outside the events)"},
+                   "l2": "flushed before every step (512 MB write, outside the events)",
+                   "cuda_graph": bool(args.graph)},
         "clocks": r["clocks"],
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": r["h2d"],
                 "d2h_bytes_per_step": r["d2h"]},
         "gpu_launches": r["launches_per_step"] * args.steps,
         "roofline": {"bound": "hbm", "kernel": "gemm1 (grouped up-GEMM + activation)",
                      "achieved": g1_gbs, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": g1_gbs / hbm_peak, "traffic": None,
+                     "frac": g1_gbs / hbm_peak, "traffic": _gemm1_traffic(cfg, g1_bytes),
                      "peak_source": f"{peak_kind} hbm_gbs",
                      "algorithmic_bytes_per_launch": g1_bytes, "avg_launch_ms": g1_ms},
         "layer_hbm": {"minimal_bytes": minimal_bytes, "achieved_gbs": layer_gbs,
