@@ -97,7 +97,10 @@ typedef struct {
   int32_t renormalize;  /* 0/1: divide the selected softmax weights by their sum */
   int32_t activation;   /* moe_activation_t */
   int32_t wdtype;       /* moe_wdtype_t */
-  int32_t block_m;      /* GEMM row tile; 0 = default (128); only 128 is supported */
+  int32_t block_m;      /* row alignment of each expert's segment: 0 = default (16 for
+                           BF16, 128 for FP8), 16 (BF16 only: the expert's weight rows are
+                           the MMA's M operand and its token rows N) or 128 (128-row token
+                           tiles) */
   uint32_t flags;       /* MOE_FLAG_* */
 } moe_problem_t;
 
@@ -107,7 +110,8 @@ typedef struct {
   size_t total_bytes;
   size_t status;          /* int32 device status word (0 = ok); the 256-byte region also
                              holds the GEMM kernels' work counters */
-  size_t num_blocks;      /* int32: number of block_m row tiles after align (= P_pad/block_m) */
+  size_t num_blocks;      /* int32 [2]: block_m row blocks after align (= P_pad/block_m), row
+                             groups (block_m 16) */
   size_t topk_ids;        /* int32 [T, k'] selected expert ids, slot order */
   size_t topk_w;          /* fp32  [T, k'] routing weights */
   size_t sorted_pair_ids; /* int32 [max_rows]: pair ids sorted by expert, sentinel P in padding */
@@ -121,6 +125,11 @@ typedef struct {
   size_t actq;            /* FP8: the activation quantised per 1x128 group, e4m3 [max_rows, I] */
   size_t act_scale;       /* FP8: fp32 [max_rows, I/128] */
   size_t y;               /* fp32 [max_rows, H]: weighted GEMM2 rows in sorted order */
+  size_t xs;              /* bf16 [max_rows, H]: hidden rows in sorted order (block_m 16,
+                             more than 1024 pairs; size 0 otherwise) */
+  size_t group_info;      /* int32 pairs [max_rows/16 + 1]: row groups {first row, expert |
+                             rows << 16} of the GEMMs (block_m 16); the count is the second
+                             int32 of the num_blocks region */
   size_t io_hidden;       /* staging for moe_forward_host: bf16 [T, H] */
   size_t io_logits;       /* staging for moe_forward_host: fp32 [T, E_r] */
   size_t io_out;          /* staging for moe_forward_host: bf16 [T, H] */
@@ -150,17 +159,28 @@ size_t moe_workspace_size(const moe_problem_t* problem);
  *   w13_in  device [E, up_mult*intermediate_in, H], checkpoint order: gate rows [0, I_in)
  *           then up rows [I_in, 2*I_in) for SWIGLU (up_mult 2), I_in rows for RELU2.
  *   w2_in   device [E, H, intermediate_in].
- *   w13_out device [E, N1, H] with N1 = 2*I (SWIGLU) or I (RELU2), I = problem->intermediate
- *           = moe_padded_intermediate(intermediate_in, ...). SWIGLU rows are interleaved
- *           [gate0, up0, gate1, up1, ...]; rows of padded indices are zero.
- *   w2_out  device [E, H, I], columns >= intermediate_in zero.
+ * The prepared matrices are w13 [E, N1, H] with N1 = 2*I (SWIGLU) or I (RELU2), I =
+ * problem->intermediate = moe_padded_intermediate(intermediate_in, ...), SWIGLU rows
+ * interleaved [gate0, up0, gate1, up1, ...] and rows of padded indices zero; and w2
+ * [E, H, I] with columns >= intermediate_in zero. They are stored
+ *   - block_m 128 (FP8, or BF16 with block_m = 128): row-major as above;
+ *   - block_m 16 (the BF16 default): tiled for the GEMMs that take the weights as the
+ *     MMA's M operand: tile (e, m, c) of rows [128m, 128m+128) and columns [64c, 64c+64)
+ *     at byte ((e*MT + m)*KC + c) * 16384, MT = ceil(rows/128), KC = ceil(cols/64); each
+ *     tile row is 128 contiguous bytes whose 16-byte piece q sits at position q ^ (r % 8);
+ *     rows and columns past the matrix are zero.
+ *   w13_out, w2_out  device, moe_prepared_weights_bytes(problem, 0 / 1) bytes each,
+ *                    16-byte aligned, not overlapping the inputs.
  * Elements are bf16 (2 bytes) or e4m3 codes (1 byte) per problem->wdtype. For FP8 the
  * block scales need no change (FP8 requires intermediate_in == I, a multiple of 128);
- * pass them to moe_forward in the checkpoint layout. Output buffers must not overlap
- * the inputs. Asynchronous on `stream`. */
+ * pass them to moe_forward in the checkpoint layout. Asynchronous on `stream`. */
 moe_status_t moe_prepare_weights(const moe_problem_t* problem, int32_t intermediate_in,
                                  const void* w13_in, const void* w2_in, void* w13_out,
                                  void* w2_out, moe_stream_t stream);
+
+/* Bytes of the prepared w13 (which = 0) or w2 (which = 1) for `problem` (host only), or
+ * 0 for an invalid problem or `which`. */
+size_t moe_prepared_weights_bytes(const moe_problem_t* problem, int32_t which);
 
 /* Block quantisation of bf16 weights to e4m3 (FP8 W8A8 block-128 weights):
  *   w        device bf16 [num_mats, rows, cols], rows and cols multiples of 128;
@@ -175,8 +195,7 @@ moe_status_t moe_quantize_weights_fp8(const void* w, int64_t num_mats, int32_t r
 /* The layer forward (all five steps), asynchronous on `stream`.
  *   hidden         device bf16 [T, H]
  *   router_logits  device fp32 [T, E_r] (finite values; NaN/Inf are not supported)
- *   w13            device, prepared by moe_prepare_weights: [E, N1, H] bf16 or e4m3
- *   w2             device, prepared: [E, H, I] bf16 or e4m3
+ *   w13, w2        device, prepared by moe_prepare_weights for this problem's layout
  *   w13_scale      FP8 only (else NULL): device fp32 [E, N1/128, H/128], checkpoint
  *                  (gate-first, un-interleaved) block order
  *   w2_scale       FP8 only (else NULL): device fp32 [E, H/128, I/128]

@@ -97,7 +97,9 @@ def new_workspace(prob: Problem, device=None) -> torch.Tensor:
 
 def prepare_weights(prob: Problem, w13: torch.Tensor, w2: torch.Tensor, intermediate_in: int,
                     stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
-    """Load-time padding + gate/up interleave (bf16, or e4m3 codes as uint8)."""
+    """Load-time padding + gate/up interleave (bf16, or e4m3 codes as uint8), in the layout
+    the problem's GEMMs read: row-major [E, N1, H] / [E, H, I] for 128-row tiles, else the
+    tiled layout (1-D tensors; ``.moe_intermediate`` records I for :func:`moe_forward`)."""
     fp8 = prob.wdtype == MOE_DTYPE_FP8_BLOCK128
     dt = torch.uint8 if fp8 else torch.bfloat16
     _dev(w13, "w13", dt)
@@ -105,10 +107,21 @@ def prepare_weights(prob: Problem, w13: torch.Tensor, w2: torch.Tensor, intermed
     E = prob.num_routed + prob.num_shared
     I = prob.intermediate
     N1 = 2 * I if prob.activation == MOE_ACT_SWIGLU else I
-    w13p = torch.empty((E, N1, prob.hidden), dtype=dt, device=w13.device)
-    w2p = torch.empty((E, prob.hidden, I), dtype=dt, device=w2.device)
+    elt = 1 if fp8 else 2
+    n13 = lib().moe_prepared_weights_bytes(ctypes.byref(prob), 0)
+    n2 = lib().moe_prepared_weights_bytes(ctypes.byref(prob), 1)
+    if n13 == 0 or n2 == 0:
+        check(lib().moe_check_problem(ctypes.byref(prob)), "moe_prepared_weights_bytes")
+    if workspace_layout(prob)["block_m"] == 16:
+        w13p = torch.empty(n13 // elt, dtype=dt, device=w13.device)
+        w2p = torch.empty(n2 // elt, dtype=dt, device=w2.device)
+    else:
+        w13p = torch.empty((E, N1, prob.hidden), dtype=dt, device=w13.device)
+        w2p = torch.empty((E, prob.hidden, I), dtype=dt, device=w2.device)
     check(lib().moe_prepare_weights(ctypes.byref(prob), intermediate_in, _ptr(w13), _ptr(w2),
                                     _ptr(w13p), _ptr(w2p), _stream(stream)), "moe_prepare_weights")
+    w13p.moe_intermediate = I
+    w2p.moe_intermediate = I
     return w13p, w2p
 
 
@@ -129,7 +142,12 @@ def _problem_from(hidden, router_logits, w2, topk, renormalize, activation_type,
                   fp8, pdl) -> Problem:
     T, H = hidden.shape
     E_r = router_logits.shape[1]
-    return make_problem(T, H, E_r, topk, w2.shape[2], renormalize=renormalize,
+    I = getattr(w2, "moe_intermediate", None)
+    if I is None:
+        if w2.dim() != 3:
+            raise ValueError("w2 must come from prepare_weights (or be [E, H, I] row-major)")
+        I = w2.shape[2]
+    return make_problem(T, H, E_r, topk, I, renormalize=renormalize,
                         activation=activation_type, num_shared=num_shared, fp8=fp8, pdl=pdl)
 
 
@@ -243,7 +261,7 @@ def read_workspace(prob: Problem, workspace: torch.Tensor) -> Dict[str, torch.Te
 
     out = {
         "status": view(L["status"], 1, torch.int32),
-        "num_blocks": view(L["num_blocks"], 1, torch.int32),
+        "num_blocks": view(L["num_blocks"], 2, torch.int32),
         "topk_ids": view(L["topk_ids"], P, torch.int32).view(T, kk),
         "topk_w": view(L["topk_w"], P, torch.float32).view(T, kk),
         "sorted_pair_ids": view(L["sorted_pair_ids"], rows, torch.int32),
@@ -252,7 +270,15 @@ def read_workspace(prob: Problem, workspace: torch.Tensor) -> Dict[str, torch.Te
         "pair_to_row": view(L["pair_to_row"], P, torch.int32),
         "y": view(L["y"], rows * H, torch.float32).view(rows, H),
     }
-    out["act"] = view(L["act"], rows * I, torch.bfloat16).view(rows, I)
+    if L["block_m"] == 16:
+        # the swapped-operand GEMMs keep the activation and the permuted hidden rows in
+        # row-group order (64-column chunks per group, swizzled); flat views
+        act_cols = -(-I // 64) * 64
+        out["act"] = view(L["act"], rows * act_cols, torch.bfloat16)
+        out["xs"] = view(L["xs"], rows * H, torch.bfloat16)
+        out["group_info"] = view(L["group_info"], (rows // 16 + 1) * 2, torch.int32).view(-1, 2)
+    else:
+        out["act"] = view(L["act"], rows * I, torch.bfloat16).view(rows, I)
     if fp8:
         out["xq"] = view(L["xq"], T * H, torch.uint8).view(T, H)
         out["xq_scale"] = view(L["xq_scale"], T * (H // 128), torch.float32).view(T, H // 128)

@@ -47,7 +47,7 @@ class Layout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in (
         "total_bytes", "status", "num_blocks", "topk_ids", "topk_w", "sorted_pair_ids",
         "expert_offsets", "block_expert", "pair_to_row", "chunk_hist", "xq", "xq_scale", "act",
-        "actq", "act_scale", "y", "io_hidden", "io_logits", "io_out")] + [
+        "actq", "act_scale", "y", "xs", "group_info", "io_hidden", "io_logits", "io_out")] + [
         ("max_rows", ctypes.c_int64),
         ("num_chunks", ctypes.c_int32),
         ("block_m", ctypes.c_int32),
@@ -73,6 +73,7 @@ SIGNATURES = {
     "moe_workspace_layout": (_I, [_P, ctypes.POINTER(Layout)]),
     "moe_workspace_size": (_S, [_P]),
     "moe_prepare_weights": (_I, [_P, _I, _V, _V, _V, _V, _V]),
+    "moe_prepared_weights_bytes": (_S, [_P, _I]),
     "moe_quantize_weights_fp8": (_I, [_V, ctypes.c_int64, _I, _I, _V, _V, _V]),
     "moe_forward": (_I, [_P, _V, _V, _V, _V, _V, _V, _V, _V, _S, _V]),
     "moe_forward_host": (_I, [_P, _V, _V, _V, _V, _V, _V, _V, _V, _S, _V]),

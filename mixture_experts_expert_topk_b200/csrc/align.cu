@@ -19,6 +19,10 @@
 //           with the same expert find each other with __match_any_sync and take
 //           consecutive ranks, so the order within an expert is the pair order.
 // With a single chunk (decode-sized batches) the three phases run in one CTA.
+//
+// For the GEMMs that put the tokens on the MMA's N operand (block_m 16), the scan also
+// cuts every expert's padded segment into row groups of at most group_rows rows, in
+// multiples of 16 and as even in size as possible, and lists them in expert order.
 #include <algorithm>
 
 #include "moe_device.cuh"
@@ -114,6 +118,24 @@ __device__ __forceinline__ void write_segments(int E, const int* seg_off, const 
   }
 }
 
+__device__ __forceinline__ int num_groups_of(int padded, int group_rows) {
+  return group_rows > 0 && padded > 0 ? (padded + group_rows - 1) / group_rows : 0;
+}
+
+// Row groups of expert e's padded segment [off, off + padded), written from index g0.
+__device__ __forceinline__ void write_groups(int e, int off, int padded, int group_rows, int g0, int2* group_info) {
+  const int ng = num_groups_of(padded, group_rows);
+  if (ng == 0) return;
+  const int blocks = padded / 16;
+  const int base = blocks / ng, extra = blocks - base * ng;
+  int row = off;
+  for (int i = 0; i < ng; ++i) {
+    const int rows = 16 * (base + (i < extra ? 1 : 0));
+    group_info[g0 + i] = make_int2(row, e | (rows << 16));
+    row += rows;
+  }
+}
+
 __global__ void __launch_bounds__(kWarps * 32)
     align_count_kernel(const int* __restrict__ ids, int P, int E, int* __restrict__ chunk_hist) {
   __shared__ int hist[kMaxExperts];
@@ -132,7 +154,8 @@ __global__ void __launch_bounds__(kWarps * 32)
 __global__ void __launch_bounds__(kScanThreads)
     align_scan_kernel(int* __restrict__ chunk_hist, int num_chunks, int E, int P, int block_m,
                       int* __restrict__ sorted_pair_ids, int* __restrict__ expert_offsets,
-                      int* __restrict__ block_expert, int* __restrict__ num_blocks) {
+                      int* __restrict__ block_expert, int* __restrict__ num_blocks, int group_rows,
+                      int2* __restrict__ group_info) {
   extern __shared__ int stage[];  // [batch chunks][E]
   __shared__ int warp_sums[32];
   __shared__ int seg_off[kMaxExperts], seg_cnt[kMaxExperts], seg_pad[kMaxExperts];
@@ -164,9 +187,13 @@ __global__ void __launch_bounds__(kScanThreads)
     seg_cnt[e] = count;
     seg_pad[e] = padded;
   }
+  int gtotal = 0;
+  const int g0 = block_exclusive_scan(e < E ? num_groups_of(padded, group_rows) : 0, warp_sums, &gtotal);
+  if (e < E) write_groups(e, off, padded, group_rows, g0, group_info);
   if (threadIdx.x == 0) {
     expert_offsets[E] = total;
-    *num_blocks = total / block_m;
+    num_blocks[0] = total / block_m;
+    if (group_rows > 0) num_blocks[1] = gtotal;
   }
   __syncthreads();
   write_segments(E, seg_off, seg_cnt, seg_pad, block_m, P, sorted_pair_ids, block_expert);
@@ -204,7 +231,8 @@ __global__ void __launch_bounds__(kWarps * 32)
 __global__ void __launch_bounds__(kWarps * 32)
     align_single_kernel(const int* __restrict__ ids, int P, int E, int block_m, int* __restrict__ sorted_pair_ids,
                         int* __restrict__ expert_offsets, int* __restrict__ block_expert,
-                        int* __restrict__ pair_to_row, int* __restrict__ num_blocks) {
+                        int* __restrict__ pair_to_row, int* __restrict__ num_blocks, int group_rows,
+                        int2* __restrict__ group_info) {
   __shared__ int cnt[kWarps][kMaxExperts];
   __shared__ int warp_sums[32];
   __shared__ int seg_off[kMaxExperts], seg_cnt[kMaxExperts], seg_pad[kMaxExperts];
@@ -219,7 +247,7 @@ __global__ void __launch_bounds__(kWarps * 32)
   warp_count(e, lane, cnt[warp]);
   __syncthreads();
   // experts in groups of blockDim.x: totals, padded sizes, exclusive scan, warp prefixes
-  int carry = 0;
+  int carry = 0, gcarry = 0;
   for (int x0 = 0; x0 < E; x0 += blockDim.x) {
     const int x = x0 + threadIdx.x;
     int count = 0;
@@ -240,11 +268,16 @@ __global__ void __launch_bounds__(kWarps * 32)
         run += c;
       }
     }
+    int gtotal = 0;
+    const int g0 = gcarry + block_exclusive_scan(x < E ? num_groups_of(padded, group_rows) : 0, warp_sums, &gtotal);
+    if (x < E) write_groups(x, off, padded, group_rows, g0, group_info);
     carry += total;
+    gcarry += gtotal;
   }
   if (threadIdx.x == 0) {
     expert_offsets[E] = carry;
-    *num_blocks = carry / block_m;
+    num_blocks[0] = carry / block_m;
+    if (group_rows > 0) num_blocks[1] = gcarry;
   }
   __syncthreads();
   write_segments(E, seg_off, seg_cnt, seg_pad, block_m, P, sorted_pair_ids, block_expert);
@@ -257,13 +290,14 @@ bool g_scan_attr[64] = {};
 
 cudaError_t launch_align(const Launch& l, const int* topk_ids, int P, int E, int block_m, int num_chunks,
                          int* chunk_hist, int* sorted_pair_ids, int* expert_offsets, int* block_expert,
-                         int* pair_to_row, int* num_blocks) {
+                         int* pair_to_row, int* num_blocks, int group_rows, int2* group_info) {
+  if (group_rows != 0 && (block_m != 16 || group_rows % 16 != 0 || group_rows > 256)) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg;
   cudaLaunchAttribute attr[1];
   if (num_chunks == 1) {
     make_launch_config(&cfg, attr, l, dim3(1), dim3(kWarps * 32), 0);
     return cudaLaunchKernelEx(&cfg, align_single_kernel, topk_ids, P, E, block_m, sorted_pair_ids,
-                              expert_offsets, block_expert, pair_to_row, num_blocks);
+                              expert_offsets, block_expert, pair_to_row, num_blocks, group_rows, group_info);
   }
   make_launch_config(&cfg, attr, l, dim3(num_chunks), dim3(kWarps * 32), 0);
   cudaError_t err = cudaLaunchKernelEx(&cfg, align_count_kernel, topk_ids, P, E, chunk_hist);
@@ -280,7 +314,7 @@ cudaError_t launch_align(const Launch& l, const int* topk_ids, int P, int E, int
   }
   make_launch_config(&cfg, attr, l, dim3(1), dim3(kScanThreads), smem);
   err = cudaLaunchKernelEx(&cfg, align_scan_kernel, chunk_hist, num_chunks, E, P, block_m, sorted_pair_ids,
-                           expert_offsets, block_expert, num_blocks);
+                           expert_offsets, block_expert, num_blocks, group_rows, group_info);
   if (err != cudaSuccess) return err;
   make_launch_config(&cfg, attr, l, dim3(num_chunks), dim3(kWarps * 32), 0);
   return cudaLaunchKernelEx(&cfg, align_scatter_kernel, (const int*)topk_ids, P, E, (const int*)chunk_hist,

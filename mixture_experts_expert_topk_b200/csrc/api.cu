@@ -41,7 +41,7 @@ using moe::GemmShape;
 using moe::Launch;
 
 constexpr size_t kAlign = 1024;
-constexpr long long kDecodeMaxPairs = 1024;  // auto block_m: 16-row blocks up to this many pairs
+constexpr int kGroupRows = 256;  // row groups of the swapped-operand GEMMs: at most this many rows
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -49,7 +49,7 @@ bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr
 bool aligned4(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 struct Plan {
-  int T, H, Er, Es, E, I, topk, kk, bm, N1, gated, fp8, renorm, act;
+  int T, H, Er, Es, E, I, topk, kk, bm, grp, N1, gated, fp8, renorm, act;
   long long P;
   int bn1, bn2;
   moe_workspace_layout_t lay;
@@ -89,14 +89,12 @@ moe_status_t make_plan(const moe_problem_t* p, Plan* pl) {
   q.topk = p->topk;
   q.kk = q.topk + q.Es;
   q.N1 = q.gated ? 2 * q.I : q.I;
-  // Row tile: 128 rows, or 16-row token blocks with the weights as the MMA's M operand
-  // when the batch is decode-sized (bf16, N1 a multiple of 128).
-  {
-    const long long P = static_cast<long long>(p->num_tokens) * (p->topk + p->num_shared);
-    const bool small_ok = !q.fp8 && q.N1 % 128 == 0;
-    if (p->block_m == 16 && !small_ok) return MOE_ERR_UNSUPPORTED;
-    q.bm = p->block_m != 0 ? p->block_m : (small_ok && P <= kDecodeMaxPairs ? 16 : 128);
-  }
+  // Row alignment. bf16 (default): 16-row blocks, the expert's weights as the MMA's M
+  // operand and row groups of up to 256 token rows as N. FP8, or block_m = 128: 128-row
+  // token tiles.
+  if (p->block_m == 16 && q.fp8) return MOE_ERR_UNSUPPORTED;
+  q.bm = p->block_m != 0 ? p->block_m : (q.fp8 ? 128 : 16);
+  q.grp = q.bm == 16 ? kGroupRows : 0;
   q.renorm = p->renormalize;
   q.act = p->activation;
   q.P = static_cast<long long>(q.T) * q.kk;
@@ -130,10 +128,14 @@ moe_status_t make_plan(const moe_problem_t* p, Plan* pl) {
   L.chunk_hist = take(static_cast<size_t>(L.num_chunks) * q.E * 4);
   L.xq = take(q.fp8 ? T * H : 0);
   L.xq_scale = take(q.fp8 ? T * (H / 128) * 4 : 0);
-  L.act = take(rows * I * 2);
+  // the swapped-operand GEMMs keep the activation in row-group order, 64-column chunks
+  const size_t act_cols = q.bm == 16 ? align_up(I, 64) : I;
+  L.act = take(rows * act_cols * 2);
   L.actq = take(q.fp8 ? rows * I : 0);
   L.act_scale = take(q.fp8 ? rows * (I / 128) * 4 : 0);
   L.y = take(rows * H * 4);
+  L.xs = take(q.bm == 16 ? rows * H * 2 : 0);
+  L.group_info = take(q.bm == 16 ? (rows / 16 + 1) * 8 : 0);
   L.io_hidden = take(T * H * 2);
   L.io_logits = take(T * static_cast<size_t>(q.Er) * 4);
   L.io_out = take(T * H * 2);
@@ -232,7 +234,8 @@ moe_status_t run_align(const Plan& pl, void* ws, const Launch& l) {
                                        L.num_chunks, ws_ptr<int>(ws, L.chunk_hist),
                                        ws_ptr<int>(ws, L.sorted_pair_ids), ws_ptr<int>(ws, L.expert_offsets),
                                        ws_ptr<int>(ws, L.block_expert), ws_ptr<int>(ws, L.pair_to_row),
-                                       ws_ptr<int>(ws, L.num_blocks)));
+                                       ws_ptr<int>(ws, L.num_blocks), pl.grp,
+                                       pl.grp != 0 ? ws_ptr<int2>(ws, L.group_info) : nullptr));
 }
 
 moe_status_t run_quant_act(const Plan& pl, const void* hidden, void* ws, const Launch& l) {
@@ -250,8 +253,11 @@ GemmBuffers common_buffers(const Plan& pl, void* ws) {
   b.sorted_pair_ids = ws_ptr<int>(ws, L.sorted_pair_ids);
   b.topk_w = ws_ptr<float>(ws, L.topk_w);
   b.status = ws_ptr<int>(ws, L.status);
+  b.num_groups = ws_ptr<int>(ws, L.num_blocks) + 1;
+  b.group_info = ws_ptr<int2>(ws, L.group_info);
   return b;
 }
+
 
 // Lower bound on the number of 128-row tiles align produces: every expert that receives
 // a pair gets at least one, and there are at least ceil(P / 128).
@@ -281,11 +287,18 @@ moe_status_t run_gemm1(const Plan& pl_in, const void* hidden, const void* w13, c
   b.tile_counter = ws_ptr<int>(ws, L.status) + 4;
   CUtensorMap ta, tb;
   if (pl.bm == 16) {
-    // decode-sized: weight tiles of 128 rows as the MMA's M operand, token rows gathered
-    if (!make_tmap_2d(&tb, w13, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, pl.H, static_cast<uint64_t>(pl.E) * pl.N1,
-                      64, 128))
-      return MOE_ERR_CUDA;
-    return cuda_status(moe::launch_gemm_decode(l, 0, tb, tb, hidden, s, b));
+    // tiled weights as the MMA's M operand; the token rows of each row group are first
+    // copied into row-group order, then both operands load with bulk copies
+    void* xs = ws_ptr<void>(ws, L.xs);
+    const moe_status_t st = cuda_status(moe::launch_permute_rows(
+        l, hidden, pl.H, ws_ptr<int>(ws, L.sorted_pair_ids), b.num_groups, b.group_info, static_cast<int>(pl.P),
+        pl.kk, xs, num_sms));
+    if (st != MOE_OK) return st;
+    moe::SwapOperands o;
+    o.w = w13;
+    o.x = xs;
+    o.out_chunks = (pl.I + 63) / 64;
+    return cuda_status(moe::launch_gemm_swap(l, 0, o, s, b));
   }
   if (!pl.fp8) {
     // the token rows of hidden are gathered by the kernel itself (no tensor map); the
@@ -342,12 +355,11 @@ moe_status_t run_gemm2(const Plan& pl_in, const void* w2, const float* w2_scale,
   CUtensorMap ta, tb;
   const uint64_t rows = static_cast<uint64_t>(L.max_rows);
   if (pl.bm == 16) {
-    b.out = ws_ptr<void>(ws, L.y);
-    if (!make_tmap_2d(&tb, w2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, pl.I, static_cast<uint64_t>(pl.E) * pl.H, 64,
-                      128) ||
-        !make_tmap_2d(&ta, ws_ptr<void>(ws, L.act), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, pl.I, rows, 64, 16))
-      return MOE_ERR_CUDA;
-    return cuda_status(moe::launch_gemm_decode(l, 1, tb, ta, nullptr, s, b));
+    moe::SwapOperands o;
+    o.w = w2;
+    o.x = ws_ptr<void>(ws, L.act);
+    o.out_chunks = 0;
+    return cuda_status(moe::launch_gemm_swap(l, 1, o, s, b));
   }
   if (!pl.fp8) {
     CUtensorMap tc;  // y [max_rows, H] fp32 in sorted row order, boxes of 32 x 32
@@ -470,9 +482,25 @@ MOE_API moe_status_t moe_prepare_weights(const moe_problem_t* problem, int32_t i
   st = device_sms(&sms);
   if (st != MOE_OK) return st;
   const Launch l = launch_of(problem, stream);
-  cudaError_t e = moe::launch_prepare_w13(l, w13_in, w13_out, pl.E, intermediate_in, pl.I, pl.H, pl.gated, elt);
+  cudaError_t e;
+  if (pl.bm == 16) {
+    // the swapped-operand GEMMs read the weights tiled
+    e = moe::launch_tile_weights(l, 0, w13_in, w13_out, pl.E, pl.H, intermediate_in, pl.I, pl.gated);
+    if (e == cudaSuccess) e = moe::launch_tile_weights(l, 1, w2_in, w2_out, pl.E, pl.H, intermediate_in, pl.I, pl.gated);
+    return cuda_status(e);
+  }
+  e = moe::launch_prepare_w13(l, w13_in, w13_out, pl.E, intermediate_in, pl.I, pl.H, pl.gated, elt);
   if (e == cudaSuccess) e = moe::launch_prepare_w2(l, w2_in, w2_out, pl.E, pl.H, intermediate_in, pl.I, elt);
   return cuda_status(e);
+}
+
+MOE_API size_t moe_prepared_weights_bytes(const moe_problem_t* problem, int32_t which) {
+  Plan pl;
+  if (make_plan(problem, &pl) != MOE_OK || (which != 0 && which != 1)) return 0;
+  if (pl.bm == 16)
+    return which == 0 ? moe::tiled_weight_bytes(pl.E, pl.N1, pl.H) : moe::tiled_weight_bytes(pl.E, pl.H, pl.I);
+  const size_t elt = pl.fp8 ? 1 : 2;
+  return which == 0 ? static_cast<size_t>(pl.E) * pl.N1 * pl.H * elt : static_cast<size_t>(pl.E) * pl.H * pl.I * elt;
 }
 
 MOE_API moe_status_t moe_quantize_weights_fp8(const void* w, int64_t num_mats, int32_t rows, int32_t cols,

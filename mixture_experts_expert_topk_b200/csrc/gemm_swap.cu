@@ -1,0 +1,484 @@
+// Steps 3 and 4 of the layer in bf16: the grouped GEMMs with the expert's weight rows as
+// the MMA's M operand and its token rows as N.
+//
+// Each expert's rows in the sorted order are padded to a multiple of 16 only (not to a
+// 128-row tile) and cut into row groups of at most 256 rows (align writes the groups). A
+// tile is (row group, 128 weight rows): D^T[n, j] = sum_k W[e][n, k] * X[j, k] with
+// tcgen05.mma kind::f16, M = 128, N = the group's rows (16..256, a multiple of 16), K = 16,
+// fp32 accumulators in TMEM (double-buffered). Putting the tokens on N keeps the padding
+// per expert below 16 rows, where 128-row token tiles pad the skewed routing of a large
+// batch by about half.
+//
+// A TMEM lane is one weight row. GEMM1: the gate and up rows of an intermediate index sit
+// in adjacent lanes (the [gate0, up0, gate1, up1, ...] interleave prepared at load time,
+// "[MoE] SwiGLU fusion into the MoE up-GEMM epilogue", sglang PR 32944, section 3) and are
+// paired with one shuffle before silu(gate)*up (or relu2); the kernel writes only the
+// bf16 activation. GEMM2: the epilogue multiplies token column j by topk_w of its pair and
+// writes fp32 y rows (sorted order) for the fixed-order combine.
+//
+// Operand layout: both operands are stored in HBM already in the shared-memory layout the
+// MMA reads (K-major, 128-byte rows of 64 bf16, the 16-byte pieces of row r permuted by
+// r mod 8: the 128-byte swizzle), so every load is one plain bulk copy (cp.async.bulk)
+// rather than a tiled tensor copy. Measured on B200, one thread's copies are served one
+// after another, at roughly 600 cycles each for bulk copies and 1300 for tiled boxes,
+// nearly independent of their size up to 32 KB; so each step is a few large copies,
+// issued by two threads.
+//   W (prepared weights): tile (expert e, 128-row block m, K chunk c of 64) of 16 KB at
+//     ((e * MT + m) * KC + c) * 16 KB; rows and K past the matrix are zero.
+//   X (row-group order): the group of n rows starting at sorted row x_row occupies bytes
+//     [x_row * KC * 128, (x_row + n) * KC * 128); chunk c of the group is n rows of 128 B
+//     at offset c * n * 128 inside it. The token-row permutation writes GEMM1's X in this
+//     order, and GEMM1's epilogue writes the activation (GEMM2's X) in it.
+// One K step of a tile moves kc chunks of W (kc * 16 KB, one copy) and of X (kc * n * 128
+// bytes, one copy), kc = 1..4 chosen from n so that a step holds 48 to 72 KB.
+//
+// One persistent CTA per SM, 7 warps:
+//   warp 0      scheduler (tiles from a global atomic counter, published to the other
+//               roles through a shared-memory ring) and W copies;
+//   warp 6      X copies;
+//   warp 1      TMEM allocator and MMA issuer;
+//   warps 2-5   epilogue (TMEM lane quadrant = warp % 4).
+#include "moe_device.cuh"
+#include "moe_internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int kMW = 128;                   // weight rows per tile (MMA M)
+constexpr int kChunkBytes = 128;           // one K chunk of a row: 64 bf16
+constexpr int kTileW = kMW * kChunkBytes;  // 16 KB: one W chunk
+constexpr int kNMax = 256;                 // rows of a row group at most (MMA N)
+constexpr int kThreads = 224;
+constexpr int kWarpX = 6;
+constexpr int kTileRing = 4;
+constexpr int kRingReaders = 6;  // MMA, 4 epilogue warps, X producer
+constexpr int kSmemCap = 232448;
+constexpr uint32_t kTmemCols = 2 * kNMax;
+
+// Operand ring: a K step takes kc * (16 KB + n * 128) contiguous bytes (W chunks, then X
+// chunks); a step that would cross the end of the ring starts again at its beginning.
+// Offsets stay multiples of 1024 bytes, the period of the 128-byte swizzle.
+constexpr int kRingBytes = 225 * 1024;
+constexpr int kSlots = 16;  // barrier pairs: at most this many K steps in flight
+constexpr int kBarOff = kRingBytes;
+constexpr int kBarBytes = 1024;  // barriers, step ends, tile ring, TMEM address, abort flag
+constexpr int kSmemBytes = kBarOff + kBarBytes + 1024;
+static_assert(kSmemBytes <= kSmemCap, "shared memory");
+
+enum : int {
+  kSiteEmpty = 1, kSiteFull = 2, kSiteTmemEmpty = 3, kSiteTmemFull = 4, kSiteTileFull = 5, kSiteTileEmpty = 6,
+  kSiteEmptyX = 7
+};
+
+struct Args {
+  int mode;                // 0 = GEMM1 (activation), 1 = GEMM2 (routing weight)
+  int m_tiles;             // MT: 128-row weight blocks per expert
+  int k_chunks;            // KC: K chunks of 64 (weights and X)
+  int k_total, num_pairs, activation;
+  const uint8_t* w;        // tiled weights
+  const uint8_t* x;        // X in row-group order
+  void* out;               // GEMM1: activation in row-group order; GEMM2: y fp32 [rows, H]
+  int out_chunks;          // GEMM1: K chunks of the activation (GEMM2's KC)
+  int out_cols;            // GEMM2: H
+  const int* num_groups;
+  const int2* group_info;  // {first sorted row, expert | rows << 16}
+  const int* sorted_pair_ids;
+  const float* topk_w;
+  int* tile_counter;       // [2]: next tile, CTAs finished; both 0 between launches
+  int* status;
+};
+
+// K chunks per step for a group of n rows: steps of 48 to 72 KB.
+__host__ __device__ constexpr int chunks_per_step(int n) {
+  return n <= 32 ? 4 : (n <= 64 ? 3 : (n <= 128 ? 2 : 1));
+}
+static_assert(4 * (kTileW + 32 * kChunkBytes) <= kRingBytes / 2 && 2 * (kTileW + 128 * kChunkBytes) <= kRingBytes / 2 &&
+                  kTileW + kNMax * kChunkBytes <= kRingBytes / 2,
+              "at least two steps fit the ring");
+
+// Byte offset in the ring of the next step of `bytes`. pos: offset of the next free byte;
+// head: running count of the bytes used, skipped ring tails included.
+__device__ __forceinline__ uint32_t ring_alloc(uint32_t& pos, uint64_t& head, uint32_t bytes) {
+  if (pos + bytes > static_cast<uint32_t>(kRingBytes)) {
+    head += kRingBytes - pos;
+    pos = 0;
+  }
+  const uint32_t off = pos;
+  pos += bytes;
+  head += bytes;
+  return off;
+}
+
+// Waits, oldest step first, until the step just allocated (its end is `head`, its index
+// ks) fits the ring and has a free slot. Each producer keeps its own copy of this state;
+// both allocate the same sequence of steps.
+__device__ __forceinline__ bool ring_reserve(uint64_t head, uint64_t& freed, uint32_t ks, uint32_t& oldest,
+                                             uint64_t* step_end, uint32_t empty0, volatile int* abort, int* status,
+                                             int site) {
+  while (head - freed > static_cast<uint64_t>(kRingBytes) || ks - oldest >= static_cast<uint32_t>(kSlots)) {
+    if (!mbar_wait(empty0 + 8 * (oldest % kSlots), (oldest / kSlots) & 1u, abort, status, site)) return false;
+    freed = step_end[oldest % kSlots];
+    ++oldest;
+  }
+  step_end[ks % kSlots] = head;
+  return true;
+}
+
+// Reader side of the tile ring: {x_row, n (0 = no more tiles), expert, mt}.
+__device__ __forceinline__ bool ring_read(uint32_t rfull0, uint32_t rempty0, volatile int* ring, int& slot,
+                                          uint32_t& ph, volatile int* abort, int* status, int4& t) {
+  const bool ok = mbar_wait(rfull0 + 8 * slot, ph, abort, status, kSiteTileFull);
+  if (ok) t = make_int4(ring[4 * slot + 0], ring[4 * slot + 1], ring[4 * slot + 2], ring[4 * slot + 3]);
+  mbar_arrive(rempty0 + 8 * slot);
+  if (++slot == kTileRing) {
+    slot = 0;
+    ph ^= 1u;
+  }
+  return ok;
+}
+
+// One contiguous global -> shared copy completing on `bar` (16-byte aligned addresses,
+// size a multiple of 16).
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar,
+                                          uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
+          dst),
+      "l"(src), "r"(bytes), "r"(bar), "l"(policy)
+      : "memory");
+}
+
+__global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t s0 = smem_u32(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBarOff);
+  const uint32_t full0 = smem_u32(bars);
+  const uint32_t empty0 = full0 + 8 * kSlots;
+  const uint32_t tfull0 = empty0 + 8 * kSlots;
+  const uint32_t tempty0 = tfull0 + 16;
+  const uint32_t rfull0 = tempty0 + 16;
+  const uint32_t rempty0 = rfull0 + 8 * kTileRing;
+  const uint32_t drain_bar = rempty0 + 8 * kTileRing;
+  uint64_t* step_end_w = bars + 2 * kSlots + 4 + 2 * kTileRing + 1;           // [kSlots]
+  uint64_t* step_end_x = step_end_w + kSlots;                                 // [kSlots]
+  volatile int* ring = reinterpret_cast<volatile int*>(step_end_x + kSlots);  // [kTileRing][4]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(const_cast<int*>(ring) + 4 * kTileRing);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kSlots; ++s) {
+      mbar_init(full0 + 8 * s, 2);  // the W and the X expect-tx arrivals
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull0 + 8 * b, 1);
+      mbar_init(tempty0 + 8 * b, 128);
+    }
+    for (int s = 0; s < kTileRing; ++s) {
+      mbar_init(rfull0 + 8 * s, 1);
+      mbar_init(rempty0 + 8 * s, kRingReaders);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  // everything above overlaps the previous kernel; inputs are read only after this
+  griddep_wait();
+  griddep_launch_dependents();
+
+  const size_t x_row_bytes = static_cast<size_t>(a.k_chunks) * kChunkBytes;
+
+  if (warp == 0) {
+    // ---------------- scheduler + W producer ----------------
+    if (lane == 0) {
+      const int num_tiles = *a.num_groups * a.m_tiles;
+      const uint64_t pol = policy_evict_first();  // each weight tile is streamed by one group
+      int wslot = 0;
+      uint32_t wph = 0, pos = 0, ks = 0, oldest = 0;
+      uint64_t head = 0, freed = 0;
+      int tile = atomicAdd(a.tile_counter, 1);
+      bool ok = true;
+      while (ok) {
+        if (!mbar_wait(rempty0 + 8 * wslot, wph ^ 1u, abort_flag, a.status, kSiteTileEmpty)) break;
+        int x_row = 0, n = 0, e = 0, mt = 0;
+        if (tile < num_tiles) {
+          const int g = tile / a.m_tiles;
+          mt = tile - g * a.m_tiles;
+          const int2 gi = a.group_info[g];
+          x_row = gi.x;
+          n = gi.y >> 16;
+          e = gi.y & 0xffff;
+        }
+        ring[4 * wslot + 0] = x_row;
+        ring[4 * wslot + 1] = n;  // 0 tells the readers to stop
+        ring[4 * wslot + 2] = e;
+        ring[4 * wslot + 3] = mt;
+        mbar_arrive(rfull0 + 8 * wslot);  // release: the entry is visible to its readers
+        if (++wslot == kTileRing) {
+          wslot = 0;
+          wph ^= 1u;
+        }
+        if (n == 0) break;
+        const int next = atomicAdd(a.tile_counter, 1);  // its latency overlaps the loads
+        const int kc = chunks_per_step(n);
+        const uint8_t* wsrc = a.w + (static_cast<size_t>(e) * a.m_tiles + mt) * a.k_chunks * kTileW;
+        for (int c0 = 0; c0 < a.k_chunks; c0 += kc, ++ks) {
+          const int kcs = min(kc, a.k_chunks - c0);
+          const uint32_t off = ring_alloc(pos, head, static_cast<uint32_t>(kcs) * (kTileW + n * kChunkBytes));
+          if (!ring_reserve(head, freed, ks, oldest, step_end_w, empty0, abort_flag, a.status, kSiteEmpty)) {
+            ok = false;
+            break;
+          }
+          const uint32_t full = full0 + 8 * (ks % kSlots);
+          const uint32_t bytes = static_cast<uint32_t>(kcs) * kTileW;
+          mbar_arrive_expect_tx(full, bytes);
+          bulk_load(s0 + off, wsrc + static_cast<size_t>(c0) * kTileW, bytes, full, pol);
+        }
+        tile = next;
+      }
+    }
+  } else if (warp == kWarpX) {
+    // ---------------- X producer ----------------
+    if (lane == 0) {
+      const uint64_t pol = policy_evict_last();  // a group's rows are read by m_tiles tiles
+      int rslot = 0;
+      uint32_t rph = 0, pos = 0, ks = 0, oldest = 0;
+      uint64_t head = 0, freed = 0;
+      bool ok = true;
+      while (ok) {
+        int4 t;
+        if (!ring_read(rfull0, rempty0, ring, rslot, rph, abort_flag, a.status, t) || t.y == 0) break;
+        const int x_row = t.x, n = t.y;
+        const int kc = chunks_per_step(n);
+        const uint8_t* xsrc = a.x + static_cast<size_t>(x_row) * x_row_bytes;
+        for (int c0 = 0; c0 < a.k_chunks; c0 += kc, ++ks) {
+          const int kcs = min(kc, a.k_chunks - c0);
+          const uint32_t off = ring_alloc(pos, head, static_cast<uint32_t>(kcs) * (kTileW + n * kChunkBytes));
+          if (!ring_reserve(head, freed, ks, oldest, step_end_x, empty0, abort_flag, a.status, kSiteEmptyX)) {
+            ok = false;
+            break;
+          }
+          const uint32_t full = full0 + 8 * (ks % kSlots);
+          const uint32_t bytes = static_cast<uint32_t>(kcs * n) * kChunkBytes;
+          mbar_arrive_expect_tx(full, bytes);
+          bulk_load(s0 + off + kcs * kTileW, xsrc + static_cast<size_t>(c0) * n * kChunkBytes, bytes, full, pol);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      int rslot = 0, it = 0;
+      uint32_t rph = 0, ks = 0, pos = 0;
+      uint64_t head = 0;  // the producers' ring allocation, replayed
+      while (true) {
+        int4 t;
+        if (!ring_read(rfull0, rempty0, ring, rslot, rph, abort_flag, a.status, t) || t.y == 0) break;
+        const int n = t.y;
+        const int kc = chunks_per_step(n);
+        const int acc = it & 1;
+        if (!mbar_wait(tempty0 + 8 * acc, ((it >> 1) & 1) ^ 1u, abort_flag, a.status, kSiteTmemEmpty)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * kNMax;
+        const uint32_t idesc = idesc_bf16(kMW, n);
+        bool ok = true;
+        for (int c0 = 0; c0 < a.k_chunks; c0 += kc, ++ks) {
+          const int kcs = min(kc, a.k_chunks - c0);
+          const uint32_t base = s0 + ring_alloc(pos, head, static_cast<uint32_t>(kcs) * (kTileW + n * kChunkBytes));
+          if (!mbar_wait(full0 + 8 * (ks % kSlots), (ks / kSlots) & 1u, abort_flag, a.status, kSiteFull)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          for (int c = 0; c < kcs; ++c) {
+            const uint64_t adesc = umma_desc_sw128(base + c * kTileW);
+            const uint64_t bdesc = umma_desc_sw128(base + kcs * kTileW + c * n * kChunkBytes);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)  // 4 x K=16 bf16 = 128 bytes; +32 bytes = +2 encoded
+              umma_bf16(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (c0 | c | k) != 0);
+          }
+          umma_commit(empty0 + 8 * (ks % kSlots));  // arrives once these MMAs have read the step
+        }
+        if (!ok) break;
+        umma_commit(tfull0 + 8 * acc);
+        ++it;
+      }
+      // all MMAs of this thread complete before TMEM is released
+      umma_commit(drain_bar);
+      mbar_wait_drain(drain_bar, 0);
+    }
+  } else {
+    // ---------------- epilogue (warps 2..5): lane = weight row ----------------
+    // 32 token columns per TMEM load. For a given token the warp's 32 lanes hold
+    // neighbouring output columns, so each store writes one contiguous piece of an output
+    // row (GEMM2: 128 B of fp32; GEMM1: 64 or 32 B of a 128-byte activation chunk row).
+    const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    const bool gated = a.activation == 0;
+    const bool odd = (lane & 1) != 0;
+    int rslot = 0, it = 0;
+    uint32_t rph = 0;
+    while (true) {
+      int4 t = make_int4(0, 0, 0, 0);
+      int ok = 0;
+      if (lane == 0) ok = ring_read(rfull0, rempty0, ring, rslot, rph, abort_flag, a.status, t);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      const int n = __shfl_sync(0xffffffffu, t.y, 0);
+      if (!ok || n == 0) break;
+      const int x_row = __shfl_sync(0xffffffffu, t.x, 0);
+      const int mt = __shfl_sync(0xffffffffu, t.w, 0);
+      // GEMM2: routing weights of the group's tokens (token 32 b + lane in wreg[b]),
+      // loaded while the main loop still runs
+      float wreg[kNMax / 32];
+#pragma unroll
+      for (int b = 0; b < kNMax / 32; ++b) {
+        wreg[b] = 0.f;
+        if (a.mode != 0 && 32 * b + lane < n) {
+          const int pid = a.sorted_pair_ids[x_row + 32 * b + lane];
+          if (pid < a.num_pairs) wreg[b] = a.topk_w[pid];
+        }
+      }
+      const int acc = it & 1;
+      const bool got = mbar_wait(tfull0 + 8 * acc, (it >> 1) & 1, abort_flag, a.status, kSiteTmemFull);
+      if (!__all_sync(0xffffffffu, got)) break;  // leave warp-uniformly (tcgen05.ld is .aligned)
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * kNMax;
+      // GEMM1: this lane's activation feature f lies in K chunk f / 64 of the activation;
+      // byte (f % 64) * 2 of a 128-byte chunk row sits in 16-byte piece ((f % 64) / 8)
+      // ^ (row % 8)
+      const int f = gated ? mt * (kMW / 2) + q * 16 + (lane >> 1) : mt * kMW + q * 32 + lane;
+      const int fc = f >> 6, fo = f & 63;
+      uint8_t* act_grp = static_cast<uint8_t*>(a.out) + static_cast<size_t>(x_row) * a.out_chunks * kChunkBytes +
+                         static_cast<size_t>(fc) * n * kChunkBytes;
+      for (int c0 = 0; c0 < n; c0 += 32) {
+        const bool full = n - c0 >= 32;  // else 16 columns remain
+        float wl = wreg[0];              // GEMM2: routing weight of token column c0 + lane
+#pragma unroll
+        for (int b = 1; b < kNMax / 32; ++b)
+          if (c0 == 32 * b) wl = wreg[b];
+        uint32_t v[32];
+        if (full) {
+          tmem_ld32(taddr + c0, v);
+        } else {
+          uint32_t(&v16)[16] = *reinterpret_cast<uint32_t(*)[16]>(&v[0]);
+          tmem_ld16(taddr + c0, v16);
+#pragma unroll
+          for (int j = 16; j < 32; ++j) v[j] = 0u;
+        }
+        tmem_wait_ld();
+        if (c0 + 32 >= n) {
+          tc_fence_before();
+          mbar_arrive(tempty0 + 8 * acc);  // the accumulator is in registers now
+        }
+        if (a.mode != 0) {
+          const int col = mt * kMW + q * 32 + lane;
+          float* y = static_cast<float*>(a.out) + static_cast<size_t>(x_row + c0) * a.out_cols + col;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            if (j == 16 && !full) break;
+            const float w = __shfl_sync(0xffffffffu, wl, j);
+            y[static_cast<size_t>(j) * a.out_cols] = __uint_as_float(v[j]) * w;
+          }
+        } else if (!gated) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            if (j == 16 && !full) break;
+            const int row = c0 + j;
+            const float z = fmaxf(__uint_as_float(v[j]), 0.f);
+            *reinterpret_cast<__nv_bfloat16*>(act_grp + row * kChunkBytes + ((((fo >> 3) ^ row) & 7) << 4) +
+                                              (fo & 7) * 2) = __float2bfloat16_rn(z * z);
+          }
+        } else {
+          // lane pair (2m, 2m+1) = (gate, up) of feature m. The even lane finishes tokens
+          // 0..15 of the batch, the odd lane tokens 16..31: each passes the other the half
+          // it needs, so every lane evaluates silu on 16 tokens.
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float mine_lo = __uint_as_float(v[j]);       // even: gate_j; odd: up_j
+            const float mine_hi = __uint_as_float(v[16 + j]);  // even: gate_{16+j}; odd: up_{16+j}
+            const float other = __shfl_xor_sync(0xffffffffu, odd ? mine_lo : mine_hi, 1);
+            const float g = odd ? other : mine_lo;
+            const float u = odd ? mine_hi : other;
+            const int row = c0 + (odd ? 16 + j : j);
+            if (!odd || full)
+              *reinterpret_cast<__nv_bfloat16*>(act_grp + row * kChunkBytes + ((((fo >> 3) ^ row) & 7) << 4) +
+                                                (fo & 7) * 2) = __float2bfloat16_rn(silu_f32(g) * u);
+          }
+        }
+      }
+      ++it;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();  // tcgen05.dealloc is .sync.aligned: the whole warp, converged
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+  if (threadIdx.x == 0) {
+    // the last CTA to finish resets the tile counter for the next launch (every CTA's
+    // scheduler has taken its last tile before its CTA gets here)
+    __threadfence();
+    if (atomicAdd(a.tile_counter + 1, 1) == static_cast<int>(gridDim.x) - 1) {
+      a.tile_counter[0] = 0;
+      a.tile_counter[1] = 0;
+    }
+  }
+}
+
+bool g_attr_set[64] = {};
+
+}  // namespace
+
+cudaError_t launch_gemm_swap(const Launch& l, int mode, const SwapOperands& o, const GemmShape& s,
+                             const GemmBuffers& b) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!g_attr_set[dev]) {
+    err = cudaFuncSetAttribute(gemm_swap_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (err != cudaSuccess) return err;
+    g_attr_set[dev] = true;
+  }
+  if ((reinterpret_cast<uintptr_t>(o.w) | reinterpret_cast<uintptr_t>(o.x)) & 15u) return cudaErrorInvalidValue;
+  Args a;
+  a.mode = mode;
+  a.m_tiles = (s.N + kMW - 1) / kMW;
+  a.k_chunks = (s.K + 63) / 64;
+  a.k_total = s.k_total;
+  a.num_pairs = s.num_pairs;
+  a.activation = s.activation;
+  a.w = static_cast<const uint8_t*>(o.w);
+  a.x = static_cast<const uint8_t*>(o.x);
+  a.out = b.out;
+  a.out_chunks = o.out_chunks;
+  a.out_cols = s.out_cols;
+  a.num_groups = b.num_groups;
+  a.group_info = b.group_info;
+  a.sorted_pair_ids = b.sorted_pair_ids;
+  a.topk_w = b.topk_w;
+  a.tile_counter = b.tile_counter;
+  a.status = b.status;
+  cudaLaunchConfig_t cfg;
+  cudaLaunchAttribute attr[1];
+  make_launch_config(&cfg, attr, l, dim3(s.num_sms), dim3(kThreads), kSmemBytes);
+  return cudaLaunchKernelEx(&cfg, gemm_swap_kernel, a);
+}
+
+}  // namespace moe

@@ -27,10 +27,20 @@ cudaError_t launch_route(const Launch& l, const float* logits, int T, int E_rout
                          int* status, const void* hidden, int hidden_row_bytes);
 
 // ---- align (align.cu) ----
+// num_blocks[0] = P_pad / block_m. With group_rows > 0 (block_m 16), each expert's rows
+// are also cut into row groups of at most group_rows rows (multiples of 16, sizes as even
+// as possible): group_info[g] = {first row, expert | rows << 16}, num_blocks[1] = count
+// (num_blocks[1] is not touched when group_rows is 0).
 cudaError_t launch_align(const Launch& l, const int* topk_ids, int P, int E, int block_m,
                          int num_chunks, int* chunk_hist, int* sorted_pair_ids,
                          int* expert_offsets, int* block_expert, int* pair_to_row,
-                         int* num_blocks);
+                         int* num_blocks, int group_rows, int2* group_info);
+// The token rows of every row group in the row-group order of the swapped-operand GEMM
+// (gemm_swap.cu): row j of the group starting at x_row is hidden[sorted_pair_ids[x_row +
+// j] / k_total] (zero for padding), H / 64 chunks of 128 bytes, swizzled.
+cudaError_t launch_permute_rows(const Launch& l, const void* hidden, int H, const int* sorted_pair_ids,
+                                const int* num_groups, const int2* group_info, int P, int k_total, void* xs,
+                                int num_sms);
 
 // ---- GEMMs (gemm_bf16.cu, gemm_fp8.cu) ----
 struct GemmShape {
@@ -59,6 +69,15 @@ struct GemmBuffers {
   int up_block_offset;      // FP8 GEMM1: row-block offset of the up half (I/128)
   int* tile_counter;        // [2] work counter of the persistent kernel; 0 between launches
   int* status;
+  const int* num_groups;    // row groups (gemm_swap)
+  const int2* group_info;
+};
+// Operands of the swapped-operand GEMM: tiled weights, X in row-group order, and (GEMM1)
+// the number of 64-column chunks of the activation it writes in row-group order.
+struct SwapOperands {
+  const void* w;
+  const void* x;
+  int out_chunks;
 };
 // N tile for a GEMM with N output columns, given an estimate of the number of 128-row
 // tiles and the SM count (0 if no multiple of 32 divides N).
@@ -68,10 +87,10 @@ cudaError_t launch_gemm1_bf16(const Launch& l, const void* hidden, const CUtenso
                               const CUtensorMap& tm_act_store, const GemmShape& s, const GemmBuffers& b);
 cudaError_t launch_gemm2_bf16(const Launch& l, const CUtensorMap& tm_act, const CUtensorMap& tm_w2,
                               const CUtensorMap& tm_y_store, const GemmShape& s, const GemmBuffers& b);
-// Decode-sized batches (token blocks of 16): weights as the MMA's M operand. mode 0 =
-// GEMM1 (x_rows = hidden, gathered), mode 1 = GEMM2 (tm_x = activation rows).
-cudaError_t launch_gemm_decode(const Launch& l, int mode, const CUtensorMap& tm_w, const CUtensorMap& tm_x,
-                               const void* x_rows, const GemmShape& s, const GemmBuffers& b);
+// Row groups of at most 256 token rows as the MMA's N operand, 128 weight rows as M.
+// mode 0 = GEMM1 (b.out: activation in row-group order), mode 1 = GEMM2 (b.out: y fp32).
+cudaError_t launch_gemm_swap(const Launch& l, int mode, const SwapOperands& o, const GemmShape& s,
+                             const GemmBuffers& b);
 size_t gemm_fp8_smem_bytes();
 cudaError_t launch_gemm1_fp8(const Launch& l, const void* xq, const CUtensorMap& tm_w13,
                              const CUtensorMap& tm_act_store, const GemmShape& s, const GemmBuffers& b);
@@ -91,5 +110,10 @@ cudaError_t launch_prepare_w13(const Launch& l, const void* in, void* out, int E
                                int I_pad, int H, int gated, int elt_bytes);
 cudaError_t launch_prepare_w2(const Launch& l, const void* in, void* out, int E, int H, int I_in,
                               int I_pad, int elt_bytes);
+// bf16 weights in the tiled layout of gemm_swap.cu: which = 0 for w13 (rows N1, K = H),
+// 1 for w2 (rows H, K = I_pad), from the checkpoint layout (moe_prepare_weights).
+size_t tiled_weight_bytes(int E, int rows, int K);
+cudaError_t launch_tile_weights(const Launch& l, int which, const void* in, void* out, int E, int H, int I_in,
+                                int I_pad, int gated);
 
 }  // namespace moe

@@ -12,6 +12,13 @@
 //
 // Input w13 [E, up_mult*I_in, H] (gate rows first), output [E, N1, H]; input w2
 // [E, H, I_in], output [E, H, I_pad]. Elements are 1 (e4m3) or 2 (bf16) bytes.
+//
+// For the bf16 GEMMs that take the weights as the MMA's M operand (gemm_swap.cu) the same
+// padded, interleaved matrices are stored tiled instead: tile (expert e, 128-row block m,
+// 64-column chunk c) of 16 KB at ((e * MT + m) * KC + c) * 16 KB, MT = ceil(rows / 128),
+// KC = ceil(K / 64); row r of a tile is 128 contiguous bytes whose 16-byte piece q sits at
+// position q ^ (r % 8) (the 128-byte swizzle of the MMA's shared-memory operand); rows and
+// columns past the matrix are zero.
 #include "moe_device.cuh"
 #include "moe_internal.h"
 
@@ -49,7 +56,69 @@ __global__ void prepare_w2_kernel(const T* __restrict__ in, T* __restrict__ out,
   out[idx] = i < I_in ? in[r * I_in + i] : T(0);
 }
 
+// One thread per 16-byte piece of the tiled output. which = 0: w13 (rows N1, K = H; row n
+// from the checkpoint row of gate/up index n / 2 (gated) or n); which = 1: w2 (rows H,
+// K = I_pad; columns >= I_in zero).
+__global__ void tile_weights_kernel(const uint16_t* __restrict__ in, uint4* __restrict__ out, long long pieces,
+                                    int which, int rows, int MT, int KC, int H, int I_in, int gated) {
+  griddep_wait();
+  for (long long o = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; o < pieces;
+       o += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long t = o >> 10;  // 1024 pieces per 16 KB tile
+    const int rr = static_cast<int>((o >> 3) & 127);
+    const int q = static_cast<int>(o & 7) ^ (rr & 7);  // logical piece stored at this position
+    const int c = static_cast<int>(t % KC);
+    const long long tm = t / KC;
+    const int m = static_cast<int>(tm % MT);
+    const long long e = tm / MT;
+    const int r = m * 128 + rr;
+    const int k0 = c * 64 + q * 8;
+    long long src = -1;  // source row
+    int ld = H, kvalid = H;
+    if (r < rows) {
+      if (which == 0) {
+        if (gated) {
+          const int j = r >> 1, half = r & 1;
+          if (j < I_in) src = e * 2LL * I_in + static_cast<long long>(half) * I_in + j;
+        } else if (r < I_in) {
+          src = e * static_cast<long long>(I_in) + r;
+        }
+      } else {
+        src = e * static_cast<long long>(H) + r;
+        ld = I_in;
+        kvalid = I_in;
+      }
+    }
+    uint16_t v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = (src >= 0 && k0 + i < kvalid) ? in[src * ld + k0 + i] : uint16_t(0);
+    uint4 w;
+    w.x = v[0] | (static_cast<uint32_t>(v[1]) << 16);
+    w.y = v[2] | (static_cast<uint32_t>(v[3]) << 16);
+    w.z = v[4] | (static_cast<uint32_t>(v[5]) << 16);
+    w.w = v[6] | (static_cast<uint32_t>(v[7]) << 16);
+    out[o] = w;
+  }
+}
+
 }  // namespace
+
+size_t tiled_weight_bytes(int E, int rows, int K) {
+  return static_cast<size_t>(E) * ((rows + 127) / 128) * ((K + 63) / 64) * 16384;
+}
+
+cudaError_t launch_tile_weights(const Launch& l, int which, const void* in, void* out, int E, int H, int I_in,
+                                int I_pad, int gated) {
+  const int rows = which == 0 ? (gated ? 2 * I_pad : I_pad) : H;
+  const int K = which == 0 ? H : I_pad;
+  const int MT = (rows + 127) / 128, KC = (K + 63) / 64;
+  const long long pieces = static_cast<long long>(tiled_weight_bytes(E, rows, K) / 16);
+  cudaLaunchConfig_t cfg;
+  cudaLaunchAttribute attr[1];
+  make_launch_config(&cfg, attr, l, dim3(4096), dim3(256), 0);
+  return cudaLaunchKernelEx(&cfg, tile_weights_kernel, static_cast<const uint16_t*>(in), static_cast<uint4*>(out),
+                            pieces, which, rows, MT, KC, H, I_in, gated);
+}
 
 cudaError_t launch_prepare_w13(const Launch& l, const void* in, void* out, int E, int I_in, int I_pad,
                                int H, int gated, int elt_bytes) {

@@ -73,6 +73,7 @@ extern "C" __attribute__((visibility("default"))) moe_status_t moe_align_noalloc
   l.stream = reinterpret_cast<cudaStream_t>(stream);
   l.pdl = (problem->flags & MOE_FLAG_PDL) != 0;
   const cudaError_t e = moe::launch_align(l, topk_ids, static_cast<int>(P), E, lay.block_m, lay.num_chunks, scratch,
-                                          sorted_pair_ids, expert_offsets, block_expert, pair_to_row, num_blocks);
+                                          sorted_pair_ids, expert_offsets, block_expert, pair_to_row, num_blocks, 0,
+                                          nullptr);
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

@@ -68,7 +68,7 @@ class GpuRun:
 
     def parts(self) -> Dict[str, np.ndarray]:
         v = moe.read_workspace(self.prob, self.ws)
-        out = {"block_m": moe.workspace_layout(self.prob)["block_m"]}
+        out = {"block_m": moe.workspace_layout(self.prob)["block_m"], "hidden_bits": bits(self.inp["hidden"])}
         for k, t in v.items():
             if t.dtype == torch.bfloat16:
                 out[k] = bits(t)
@@ -121,3 +121,34 @@ def err_beyond_rounding(got: np.ndarray, ref: np.ndarray) -> float:
 
 __all__ = ["CONFIGS", "GpuRun", "bits", "cpu_inputs", "oracle_out", "bf16_to_f64", "max_err_over_rms",
            "half_ulp_bf16", "err_beyond_rounding"]
+
+
+def untile_groups(flat_bits: np.ndarray, group_info: np.ndarray, num_groups: int, rows: int,
+                  kchunks: int) -> np.ndarray:
+    """Row-major [rows, 64 * kchunks] from a buffer in the row-group order of the
+    swapped-operand GEMMs: the group of n rows at x_row starts at element x_row * 64 *
+    kchunks; its chunk c is n rows of 64 elements; row j's 16-byte piece q is stored at
+    position q ^ (j % 8). Rows outside every group stay zero."""
+    flat = np.asarray(flat_bits).reshape(-1)
+    out = np.zeros((rows, 64 * kchunks), dtype=flat.dtype)
+    for g in range(num_groups):
+        x_row, meta = int(group_info[g][0]), int(group_info[g][1])
+        n = meta >> 16
+        base = x_row * 64 * kchunks
+        grp = flat[base:base + n * 64 * kchunks].reshape(kchunks, n, 8, 8)
+        j = np.arange(n)
+        phys = np.arange(8)[None, :] ^ (j[:, None] & 7)       # where logical piece q is stored
+        logical = grp[:, j[:, None], phys, :]                  # [kchunks, n, 8, 8]
+        out[x_row:x_row + n] = logical.transpose(1, 0, 2, 3).reshape(n, 64 * kchunks)
+    return out
+
+
+def untile_weights(flat_bits: np.ndarray, E: int, rows: int, K: int) -> np.ndarray:
+    """[E, MT*128, KC*64] from the tiled weight layout: tile (e, m, c) of 128 x 64 at
+    ((e * MT + m) * KC + c) * 8192 elements, row r's 16-byte piece q at q ^ (r % 8)."""
+    MT, KC = -(-rows // 128), -(-K // 64)
+    t = np.asarray(flat_bits).reshape(E, MT, KC, 128, 8, 8)
+    r = np.arange(128)
+    phys = np.arange(8)[None, :] ^ (r[:, None] & 7)
+    u = t[:, :, :, r[:, None], phys, :]                          # [E, MT, KC, 128, 8, 8]
+    return u.transpose(0, 1, 3, 2, 4, 5).reshape(E, MT * 128, KC * 64)

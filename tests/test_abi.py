@@ -97,8 +97,11 @@ def test_workspace_layout(L):
         E = cfg.E_total
         assert lay["status"] == 0
         bm = lay["block_m"]
-        # decode-sized bf16 batches use 16-row token blocks, everything else 128-row tiles
-        assert bm == (16 if (P <= 1024 and not cfg.fp8) else 128)
+        # bf16 aligns each expert to 16 rows (token rows on the MMA's N), FP8 to 128-row tiles
+        assert bm == (128 if cfg.fp8 else 16)
+        # the permuted hidden rows (row-group order) exist for the 16-row alignment
+        xs_bytes = lay["group_info"] - lay["xs"]
+        assert xs_bytes == (-(-lay["max_rows"] * cfg.H * 2 // 1024) * 1024 if not cfg.fp8 else 0)
         assert lay["max_rows"] == -(-(P + min(E, P) * (bm - 1)) // bm) * bm
         assert lay["num_chunks"] == -(-P // 2048)
         offs = sorted(v for k, v in lay.items() if k not in ("total_bytes", "max_rows", "num_chunks", "block_m"))

@@ -18,7 +18,8 @@ import mixture_experts_expert_topk_b200 as moe
 from mixture_experts_expert_topk_b200.synth import CONFIGS, MoeConfig, make_inputs
 from oracle import moe_oracle as O
 
-from _cases import GpuRun, bf16_to_f64, bits, cpu_inputs, err_beyond_rounding, max_err_over_rms, oracle_out
+from _cases import (GpuRun, bf16_to_f64, bits, cpu_inputs, err_beyond_rounding, max_err_over_rms, oracle_out,
+                    untile_groups, untile_weights)
 
 pytestmark = pytest.mark.gpu
 
@@ -45,6 +46,11 @@ SMALL = {
     "shared_bf16": _small("shared_bf16", T=130, H=256, E=12, topk=3, I=256, num_shared=1),
     "k_equals_E": _small("k_equals_E", T=40, H=256, E=8, topk=8, I=128),
     "skewed": _small("skewed", T=512, H=256, E=32, topk=4, I=256, logit_bias_std=3.0),
+    # more than 1024 pairs (row groups of up to 256, permuted rows by TMA) with a partial
+    # last weight tile (N1 = 416) and a K tail in GEMM2 (K = 208)
+    "pad_gated_big": _small("pad_gated_big", T=600, H=256, E=6, topk=2, I=200),
+    "relu2_big": _small("relu2_big", T=600, H=384, E=8, topk=3, I=300, activation="relu2",
+                        renormalize=False),
 }
 
 
@@ -60,7 +66,42 @@ def _check_route_align(cfg, parts, logits, bm=None):
     np.testing.assert_array_equal(parts["sorted_pair_ids"][:P_pad], a["sorted_pair_ids"])
     np.testing.assert_array_equal(parts["block_expert"][:P_pad // bm], a["block_expert"])
     np.testing.assert_array_equal(parts["pair_to_row"], a["pair_to_row"])
+    if bm == 16:
+        _check_groups(cfg, parts, a)
     return ids, a
+
+
+def _check_groups(cfg, parts, a):
+    """Row groups of the swapped-operand GEMMs: each expert's padded segment cut into
+    ceil(rows / 256) groups of whole 16-row blocks, sizes as even as possible, larger
+    first; and the permuted hidden rows."""
+    P = cfg.T * cfg.k_total
+    G = 256
+    off = a["expert_offsets"]
+    expect = []
+    for e in range(cfg.E_total):
+        seg = int(off[e + 1] - off[e])
+        if seg == 0:
+            continue
+        ng = -(-seg // G)
+        base, extra = divmod(seg // 16, ng)
+        row = int(off[e])
+        for i in range(ng):
+            n = 16 * (base + (1 if i < extra else 0))
+            assert 16 <= n <= G
+            expect.append((row, e | (n << 16)))
+            row += n
+        assert row == off[e + 1]
+    assert int(parts["num_blocks"][1]) == len(expect)
+    np.testing.assert_array_equal(parts["group_info"][:len(expect)], np.array(expect, dtype=np.int32).reshape(-1, 2))
+    # the permuted hidden rows, in row-group order
+    rows = int(a["P_pad"])
+    xs = untile_groups(parts["xs"], parts["group_info"], len(expect), rows, cfg.H // 64)
+    pids = a["sorted_pair_ids"][:rows]
+    hb = parts["hidden_bits"]
+    real = pids < P
+    np.testing.assert_array_equal(xs[real], hb[pids[real] // cfg.k_total])
+    assert np.all(xs[~real] == 0)
 
 
 def _check_act(cfg, run, parts, ids, a):
@@ -68,8 +109,14 @@ def _check_act(cfg, run, parts, ids, a):
     x = bf16_to_f64(run.inp["hidden"])
     w13 = run.inp["w13"]
     kk = cfg.k_total
-    act_gpu = bf16_to_f64(parts["act"])
     P = cfg.T * kk
+    if parts["block_m"] == 16:   # row-group order: back to sorted rows
+        rows = parts["sorted_pair_ids"].shape[0]
+        act_bits = untile_groups(parts["act"], parts["group_info"], int(parts["num_blocks"][1]), rows,
+                                 -(-run.I_pad // 64))[:, :run.I_pad]
+    else:
+        act_bits = parts["act"]
+    act_gpu = bf16_to_f64(act_bits)
     worst = 0.0
     for e in np.unique(ids):
         rows = np.arange(a["expert_offsets"][e], a["expert_offsets"][e + 1])
@@ -87,10 +134,12 @@ def _check_act(cfg, run, parts, ids, a):
     assert worst <= 1.0, worst
 
 
-@pytest.mark.parametrize("name", list(SMALL))
-def test_layer_parity_small(name):
+@pytest.mark.parametrize("name,bm", [(n, 0) for n in SMALL] +
+                         [(n, 128) for n in ("ragged", "skewed", "pad_gated", "relu2_small")])
+def test_layer_parity_small(name, bm):
+    # bm 0: the default (bf16: 16-row alignment, weights on the MMA's M); 128: token tiles
     cfg = SMALL[name]
-    run = GpuRun(cfg)
+    run = GpuRun(cfg, block_m=bm)
     out = run.forward()
     parts = run.parts()
     ids, a = _check_route_align(cfg, parts, run.inp["logits"])
@@ -144,8 +193,9 @@ def test_tied_logits_pick_lowest_indices():
     assert err_beyond_rounding(bf16_to_f64(run.out), ref) <= BF16_TOL
 
 
-def test_all_tokens_one_expert_and_empty_experts():
-    cfg = _small("one_expert", T=700, H=256, E=8, topk=1, I=256)
+@pytest.mark.parametrize("T", [700, 1500])   # row groups of 16, and of up to 256 (uneven)
+def test_all_tokens_one_expert_and_empty_experts(T):
+    cfg = _small("one_expert", T=T, H=256, E=8, topk=1, I=256)
     inp = make_inputs(cfg, 4)
     inp["logits"][:, 5] += 100.0   # every token picks expert 5; 7 experts empty
     run = GpuRun(cfg, inputs=inp)
@@ -153,7 +203,7 @@ def test_all_tokens_one_expert_and_empty_experts():
     parts = run.parts()
     ids, a = _check_route_align(cfg, parts, inp["logits"])
     bm = parts["block_m"]
-    seg = -(-700 // bm) * bm                      # 700 pairs padded to the row tile
+    seg = -(-T // bm) * bm                        # T pairs padded to the row tile
     assert list(a["expert_offsets"]) == [0] * 6 + [seg] * 3
     ref = oracle_out(cfg, inp)
     assert err_beyond_rounding(bf16_to_f64(run.out), ref) <= BF16_TOL
@@ -171,20 +221,29 @@ def test_zero_tokens_is_a_no_op():
     assert out.shape == (0, 256)
 
 
-def test_prepare_weights_matches_oracle_layout():
+@pytest.mark.parametrize("bm", [16, 128])
+def test_prepare_weights_matches_oracle_layout(bm):
+    # bm 128: row-major; bm 16: tiled (128 x 64 tiles, swizzled, zero past the matrix)
     for act, I in (("swiglu", 200), ("swiglu", 512), ("relu2", 300)):
         cfg = _small("prep", T=4, H=256, E=3, topk=1, I=I, activation=act)
         inp = make_inputs(cfg, 1)
         I_pad = moe.padded_intermediate(I, act)
-        prob = moe.make_problem(4, 256, 3, 1, I_pad, activation=act)
+        prob = moe.make_problem(4, 256, 3, 1, I_pad, activation=act, block_m=bm)
         w13p, w2p = moe.prepare_weights(prob, inp["w13"].cuda(), inp["w2"].cuda(), I)
         torch.cuda.synchronize()
         p13, p2, ip = O.pad_weights(bits(inp["w13"]), bits(inp["w2"]), I, act == "swiglu")
         assert ip == I_pad
         if act == "swiglu":
             p13 = O.interleave_gate_up(p13, I_pad)
-        np.testing.assert_array_equal(bits(w13p), p13)
-        np.testing.assert_array_equal(bits(w2p), p2)
+        g13, g2 = bits(w13p), bits(w2p)
+        if bm == 16:
+            N1 = p13.shape[1]
+            t13 = untile_weights(g13, 3, N1, 256)
+            t2 = untile_weights(g2, 3, 256, I_pad)
+            assert np.all(t13[:, N1:] == 0) and np.all(t2[:, :, I_pad:] == 0)
+            g13, g2 = t13[:, :N1, :256], t2[:, :256, :I_pad]
+        np.testing.assert_array_equal(g13, p13)
+        np.testing.assert_array_equal(g2, p2)
 
 
 def test_fp8_quantizers_bit_exact():

@@ -50,7 +50,7 @@ def test_align_noalloc_matches_workspace_align_twice(T, E, topk, shared):
         rows = lay["max_rows"]
         Et = E + shared
         out = {"sorted_pair_ids": _i32(rows), "expert_offsets": _i32(Et + 1),
-               "block_expert": _i32(rows // 128), "pair_to_row": _i32(P), "num_blocks": _i32(1)}
+               "block_expert": _i32(rows // lay["block_m"]), "pair_to_row": _i32(P), "num_blocks": _i32(1)}
         ids = ref["topk_ids"].contiguous()
         st = L.moe_align_noalloc(ctypes.byref(prob), _ptr(ids), _ptr(out["sorted_pair_ids"]),
                                  _ptr(out["expert_offsets"]), _ptr(out["block_expert"]),
@@ -59,7 +59,7 @@ def test_align_noalloc_matches_workspace_align_twice(T, E, topk, shared):
         torch.cuda.synchronize()
         nb = int(ref["num_blocks"][0])
         assert int(out["num_blocks"][0]) == nb
-        p_pad = nb * 128
+        p_pad = nb * lay["block_m"]
         assert torch.equal(out["expert_offsets"], ref["expert_offsets"])
         assert torch.equal(out["sorted_pair_ids"][:p_pad], ref["sorted_pair_ids"][:p_pad])
         assert torch.equal(out["block_expert"][:nb], ref["block_expert"][:nb])
