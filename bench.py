@@ -39,9 +39,10 @@ from mixture_experts_expert_topk_b200.synth import CONFIGS, MoeConfig, make_inpu
 L2_FLUSH_BYTES = 512 << 20
 
 # DRAM traffic of GEMM1 relative to its algorithmic bytes, from one ncu capture
-# (dram__bytes_read.sum + dram__bytes_write.sum, profiles/gemm_bf16_prefill_e64_ncu.md),
-# valid only for the kernel source it was taken on (sha256 prefix of gemm_bf16.cu).
-GEMM1_TRAFFIC = {"source_sha256": "92a46cf29e07", "ratio": 284.0 / 280.3}
+# (dram__bytes_read.sum + dram__bytes_write.sum of the GEMM1 launch on the 64-expert
+# prefill case), valid only for the kernel source it was taken on (sha256 prefix of the
+# file below); None until such a capture exists for that source.
+GEMM1_TRAFFIC = {"source": "gemm_swap.cu", "source_sha256": None, "ratio": None}
 
 
 def _peaks():
@@ -234,7 +235,7 @@ def run_ours(cfg: MoeConfig, steps: int, warmup: int, world: int, rank: int, loc
 
     # per-kernel breakdown: the same kernels through the per-step entry points, events
     # between the steps on the launching stream
-    names = ["route", "align"] + (["quant_act"] if cfg.fp8 else []) + ["gemm1", "gemm2", "combine"]
+    names = ["route", "align"] + (["quant_act"] if cfg.fp8 else ["permute"]) + ["gemm1", "gemm2", "combine"]
     per = {n: [] for n in names}
     for _ in range(steps):
         flush.zero_()
@@ -245,6 +246,8 @@ def run_ours(cfg: MoeConfig, steps: int, warmup: int, world: int, rank: int, loc
         moe.stage_align(prob, ws); k += 1; evs[k].record(stream)
         if cfg.fp8:
             moe.stage_quant_act(prob, hidden, ws); k += 1; evs[k].record(stream)
+        else:
+            moe.stage_permute(prob, hidden, ws); k += 1; evs[k].record(stream)
         moe.stage_gemm1(prob, hidden, w13p, ws, s13); k += 1; evs[k].record(stream)
         moe.stage_gemm2(prob, w2p, ws, s2); k += 1; evs[k].record(stream)
         moe.stage_combine(prob, out, ws); k += 1; evs[k].record(stream)
@@ -279,7 +282,9 @@ def run_ours(cfg: MoeConfig, steps: int, warmup: int, world: int, rank: int, loc
         "total_ms": total_ms, "step_ms": step_ms, "kernel_ms": kernel_ms, "clocks": clocks,
         "e2e_total_ms": e2e_total, "ids": ids, "inp": inp,
         "h2d": h_hidden.numel() * 2 + h_logits.numel() * 4, "d2h": h_out.numel() * 2,
-        "launches_per_step": len(names) + 2,  # align is three kernels
+        # one kernel per stage, except align (three kernels above one 2048-pair chunk) and
+        # FP8 GEMM1 (the GEMM, then the per-row activation quantisation)
+        "launches_per_step": len(names) + (2 if cfg.T * cfg.k_total > 2048 else 0) + (1 if cfg.fp8 else 0),
     }
 
 
@@ -287,9 +292,9 @@ def _gemm1_traffic(cfg: MoeConfig, g1_bytes: float):
     """DRAM bytes per GEMM1 launch scaled from the ncu capture, or None if the kernel
     source changed since (or the workload does not run that kernel)."""
     import hashlib
-    src = os.path.join(ROOT, "mixture_experts_expert_topk_b200", "csrc", "gemm_bf16.cu")
+    src = os.path.join(ROOT, "mixture_experts_expert_topk_b200", "csrc", GEMM1_TRAFFIC["source"])
     sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:12]
-    if cfg.fp8 or cfg.T * cfg.k_total <= 1024 or sha != GEMM1_TRAFFIC["source_sha256"]:
+    if cfg.fp8 or GEMM1_TRAFFIC["ratio"] is None or sha != GEMM1_TRAFFIC["source_sha256"]:
         return None
     return g1_bytes * GEMM1_TRAFFIC["ratio"]
 

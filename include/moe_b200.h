@@ -219,9 +219,10 @@ moe_status_t moe_forward_host(const moe_problem_t* problem, const void* h_hidden
                               const float* w13_scale, const float* w2_scale, void* h_out,
                               void* workspace, size_t workspace_bytes, moe_stream_t stream);
 
-/* The five steps as separate calls on the same workspace (moe_forward runs exactly
- * these, in this order). They exist so tests can check each intermediate and tools can
- * time each kernel; each requires the previous steps to have been enqueued. */
+/* The steps as separate calls on the same workspace: route, align, quant_act (FP8),
+ * permute (block_m 16), gemm1, gemm2, combine; moe_forward runs exactly these, in this
+ * order. They exist so tests can check each intermediate and tools can time each kernel;
+ * each requires the previous steps to have been enqueued. */
 moe_status_t moe_stage_route(const moe_problem_t* problem, const float* router_logits,
                              void* workspace, size_t workspace_bytes, moe_stream_t stream);
 moe_status_t moe_stage_align(const moe_problem_t* problem, void* workspace,
@@ -229,6 +230,11 @@ moe_status_t moe_stage_align(const moe_problem_t* problem, void* workspace,
 /* FP8 only: quantise hidden per token per 128 columns into the workspace (xq, xq_scale). */
 moe_status_t moe_stage_quant_act(const moe_problem_t* problem, const void* hidden,
                                  void* workspace, size_t workspace_bytes, moe_stream_t stream);
+/* block_m 16 (the BF16 default): copy the token rows of every row group into the
+ * workspace in the order GEMM1 reads them (xs); hidden device bf16 [T, H]. Other
+ * problems: nothing to do, MOE_OK. */
+moe_status_t moe_stage_permute(const moe_problem_t* problem, const void* hidden, void* workspace,
+                               size_t workspace_bytes, moe_stream_t stream);
 moe_status_t moe_stage_gemm1(const moe_problem_t* problem, const void* hidden, const void* w13,
                              const float* w13_scale, void* workspace, size_t workspace_bytes,
                              moe_stream_t stream);

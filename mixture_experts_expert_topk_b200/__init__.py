@@ -222,6 +222,11 @@ def stage_quant_act(prob, hidden, workspace, stream=None):
                                     workspace.numel(), _stream(stream)), "moe_stage_quant_act")
 
 
+def stage_permute(prob, hidden, workspace, stream=None):
+    check(lib().moe_stage_permute(ctypes.byref(prob), _ptr(hidden), _ptr(workspace),
+                                  workspace.numel(), _stream(stream)), "moe_stage_permute")
+
+
 def stage_gemm1(prob, hidden, w13, workspace, w13_scale=None, stream=None):
     check(lib().moe_stage_gemm1(ctypes.byref(prob), _ptr(hidden), _ptr(w13), _ptr(w13_scale),
                                 _ptr(workspace), workspace.numel(), _stream(stream)),

@@ -80,6 +80,7 @@ SIGNATURES = {
     "moe_stage_route": (_I, [_P, _V, _V, _S, _V]),
     "moe_stage_align": (_I, [_P, _V, _S, _V]),
     "moe_stage_quant_act": (_I, [_P, _V, _V, _S, _V]),
+    "moe_stage_permute": (_I, [_P, _V, _V, _S, _V]),
     "moe_stage_gemm1": (_I, [_P, _V, _V, _V, _V, _S, _V]),
     "moe_stage_gemm2": (_I, [_P, _V, _V, _V, _S, _V]),
     "moe_stage_combine": (_I, [_P, _V, _V, _S, _V]),

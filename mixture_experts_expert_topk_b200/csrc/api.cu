@@ -287,16 +287,11 @@ moe_status_t run_gemm1(const Plan& pl_in, const void* hidden, const void* w13, c
   b.tile_counter = ws_ptr<int>(ws, L.status) + 4;
   CUtensorMap ta, tb;
   if (pl.bm == 16) {
-    // tiled weights as the MMA's M operand; the token rows of each row group are first
-    // copied into row-group order, then both operands load with bulk copies
-    void* xs = ws_ptr<void>(ws, L.xs);
-    const moe_status_t st = cuda_status(moe::launch_permute_rows(
-        l, hidden, pl.H, ws_ptr<int>(ws, L.sorted_pair_ids), b.num_groups, b.group_info, static_cast<int>(pl.P),
-        pl.kk, xs, num_sms));
-    if (st != MOE_OK) return st;
+    // tiled weights as the MMA's M operand, the token rows in row-group order (run_permute):
+    // both operands load with bulk copies
     moe::SwapOperands o;
     o.w = w13;
-    o.x = xs;
+    o.x = ws_ptr<void>(ws, L.xs);
     o.out_chunks = (pl.I + 63) / 64;
     return cuda_status(moe::launch_gemm_swap(l, 0, o, s, b));
   }
@@ -332,6 +327,15 @@ moe_status_t run_gemm1(const Plan& pl_in, const void* hidden, const void* w13, c
   return cuda_status(moe::launch_quant_rows(l, ws_ptr<void>(ws, L.act), static_cast<int>(L.max_rows), pl.I,
                                             ws_ptr<int>(ws, L.num_blocks), pl.bm, ws_ptr<void>(ws, L.actq),
                                             ws_ptr<float>(ws, L.act_scale)));
+}
+
+// The token rows of each row group in row-group order (block_m 16 only).
+moe_status_t run_permute(const Plan& pl, const void* hidden, void* ws, const Launch& l, int num_sms) {
+  if (pl.bm != 16) return MOE_OK;
+  const auto& L = pl.lay;
+  return cuda_status(moe::launch_permute_rows(l, hidden, pl.H, ws_ptr<int>(ws, L.sorted_pair_ids),
+                                              ws_ptr<int>(ws, L.num_blocks) + 1, ws_ptr<int2>(ws, L.group_info),
+                                              static_cast<int>(pl.P), pl.kk, ws_ptr<void>(ws, L.xs), num_sms));
 }
 
 moe_status_t run_gemm2(const Plan& pl_in, const void* w2, const float* w2_scale, void* ws, const Launch& l,
@@ -413,6 +417,7 @@ moe_status_t forward_device(const Plan& pl, const moe_problem_t* p, const void* 
   moe_status_t st = run_route(pl, logits, ws, l, hidden);
   if (st == MOE_OK) st = run_align(pl, ws, l);
   if (st == MOE_OK && pl.fp8) st = run_quant_act(pl, hidden, ws, l);
+  if (st == MOE_OK) st = run_permute(pl, hidden, ws, l, num_sms);
   if (st == MOE_OK) st = run_gemm1(pl, hidden, w13, s13, ws, l, num_sms);
   if (st == MOE_OK) st = run_gemm2(pl, w2, s2, ws, l, num_sms);
   if (st == MOE_OK) st = run_combine(pl, out, ws, l);
@@ -595,6 +600,18 @@ MOE_API moe_status_t moe_stage_quant_act(const moe_problem_t* problem, const voi
   st = prologue(problem, workspace, workspace_bytes, &pl, &sms);
   if (st != MOE_OK || pl.T == 0) return st;
   return run_quant_act(pl, hidden, workspace, launch_of(problem, stream));
+}
+
+MOE_API moe_status_t moe_stage_permute(const moe_problem_t* problem, const void* hidden, void* workspace,
+                                       size_t workspace_bytes, moe_stream_t stream) {
+  Plan pl;
+  int sms = 0;
+  moe_status_t st = make_plan(problem, &pl);
+  if (st != MOE_OK || pl.T == 0) return st;  // T == 0: nothing to do, pointers unused
+  if (pl.bm == 16 && !aligned16(hidden)) return MOE_ERR_INVALID_ARG;
+  st = prologue(problem, workspace, workspace_bytes, &pl, &sms);
+  if (st != MOE_OK || pl.T == 0) return st;
+  return run_permute(pl, hidden, workspace, launch_of(problem, stream), sms);
 }
 
 MOE_API moe_status_t moe_stage_gemm1(const moe_problem_t* problem, const void* hidden, const void* w13,

@@ -172,6 +172,7 @@ def test_stage_entry_points_match_forward():
     out = torch.empty_like(run.hidden)
     moe.stage_route(run.prob, run.logits, ws)
     moe.stage_align(run.prob, ws)
+    moe.stage_permute(run.prob, run.hidden, ws)
     moe.stage_gemm1(run.prob, run.hidden, run.w13p, ws)
     moe.stage_gemm2(run.prob, run.w2p, ws)
     moe.stage_combine(run.prob, out, ws)
