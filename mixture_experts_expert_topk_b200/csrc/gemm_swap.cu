@@ -304,13 +304,15 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
             break;
           }
           tc_fence_after();
-          for (int c = 0; c < kcs; ++c) {
-            const uint64_t adesc = umma_desc_sw128(base + c * kTileW);
-            const uint64_t bdesc = umma_desc_sw128(base + kcs * kTileW + c * n * kChunkBytes);
+          // descriptor low words: W chunk c at base + c * 16 KB, X chunk c at base + kcs * 16 KB
+          // + c * n * 128 (the encoded address counts 16-byte units)
+          const uint32_t a_lo = umma_desc_lo(base);
+          const uint32_t b_lo = a_lo + static_cast<uint32_t>(kcs) * (kTileW >> 4);
+          const uint32_t b_step = static_cast<uint32_t>(n) * (kChunkBytes >> 4);
+          umma_bf16_chunk(d_tmem, a_lo, b_lo, idesc, c0 != 0);
 #pragma unroll
-            for (int k = 0; k < 4; ++k)  // 4 x K=16 bf16 = 128 bytes; +32 bytes = +2 encoded
-              umma_bf16(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (c0 | c | k) != 0);
-          }
+          for (int c = 1; c < 4; ++c)
+            if (c < kcs) umma_bf16_chunk(d_tmem, a_lo + c * (kTileW >> 4), b_lo + c * b_step, idesc, 1u);
           umma_commit(empty0 + 8 * (ks % kSlots));  // arrives once these MMAs have read the step
         }
         if (!ok) break;
