@@ -51,6 +51,9 @@ SMALL = {
     "pad_gated_big": _small("pad_gated_big", T=600, H=256, E=6, topk=2, I=200),
     "relu2_big": _small("relu2_big", T=600, H=384, E=8, topk=3, I=300, activation="relu2",
                         renormalize=False),
+    # three align chunks (the single-launch align with its grid barrier) and more experts
+    # than the align CTA has threads
+    "many_experts": _small("many_experts", T=700, H=256, E=300, topk=8, I=128),
 }
 
 
