@@ -12,7 +12,8 @@ The layer (one forward call) computes, for every token t with hidden row x_t:
               optional renormalisation, optional fused shared-expert slot;
   2. align:   stable sort of the (token, slot) pairs by expert, each expert's
               segment padded to the GEMM row tile ``block_m``;
-  3. GEMM1:   z = W13[e] x_t, then SwiGLU silu(gate)*up or relu2 max(z,0)^2;
+  3. GEMM1:   z = W13[e] x_t, then a gated activation act(gate)*up (SwiGLU: silu;
+              gelu_tanh) or relu2 max(z,0)^2;
   4. GEMM2:   y = w_tj * (W2[e] a);
   5. combine: out_t = sum_j y_tj in slot order j = 0..k'-1.
 
@@ -333,23 +334,56 @@ def relu2(x: np.ndarray) -> np.ndarray:
     return r * r
 
 
+def gelu_tanh(x: np.ndarray) -> np.ndarray:
+    """GELU with the tanh approximation, one of the gated activations of [GATED]
+    section 2 (named there as the Gaussian error linear unit with the tanh
+    approximation; the pages print no formula, so the standard one is taken):
+    0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3)))."""
+    return 0.5 * x * (1.0 + np.tanh(math.sqrt(2.0 / math.pi) * (x + 0.044715 * x * x * x)))
+
+
+GATED_ACTIVATIONS = ("swiglu", "gelu_tanh")
+
+
+def is_gated(activation: str) -> bool:
+    return activation in GATED_ACTIVATIONS
+
+
 def activation_fn(z: np.ndarray, activation: str, I: int) -> np.ndarray:
     """Apply the layer activation to GEMM1 rows z [n, N1] (gate-first layout).
 
-    SwiGLU: a = silu(z[:, :I]) * z[:, I:2I] ([SWIGLU] section 1,
-    ``silu(gate) * up``; [GATED] section 1, activation(gate) * up).
+    Gated: a = act(z[:, :I]) * z[:, I:2I] with act = silu for SwiGLU ([SWIGLU]
+    section 1, ``silu(gate) * up``) or gelu_tanh ([GATED] section 2; [GATED]
+    section 1: activation(gate) * up).
     relu2: a = relu2(z) over the I columns.
     """
-    if activation == "swiglu":
-        return silu(z[:, :I]) * z[:, I:2 * I]
+    if is_gated(activation):
+        act = silu if activation == "swiglu" else gelu_tanh
+        return act(z[:, :I]) * z[:, I:2 * I]
     if activation == "relu2":
         return relu2(z[:, :I])
     raise ValueError(activation)
 
 
-def moe_forward(hidden_bits: np.ndarray, logits: np.ndarray, w13_bits, w2_bits, *,
+def append_shared_slot(ids: np.ndarray, w: np.ndarray, num_routed: int, num_shared: int):
+    """Caller-supplied routing ([TRTLLM] section 1 names a routed variant of the fused
+    op, ``trtllm_fp8_block_scale_routed_moe``, that takes the top-k choice instead of
+    router logits): routed ids [T, k] and weights [T, k] as given, then, with
+    num_shared = 1, the fused shared slot after them (id E_r, weight 1, the same rule
+    as ``route``)."""
+    ids = np.asarray(ids, dtype=np.int32)
+    w = np.asarray(w, dtype=np.float32)
+    if num_shared:
+        T = ids.shape[0]
+        ids = np.concatenate([ids, np.full((T, 1), num_routed, dtype=np.int32)], axis=1)
+        w = np.concatenate([w, np.ones((T, 1), dtype=np.float32)], axis=1)
+    return ids, w
+
+
+def moe_forward(hidden_bits: np.ndarray, logits: Optional[np.ndarray], w13_bits, w2_bits, *,
                 topk: int, renormalize: bool, activation: str, num_shared: int = 0,
-                tokens: Optional[Sequence[int]] = None, return_parts: bool = False):
+                tokens: Optional[Sequence[int]] = None, return_parts: bool = False,
+                routing=None):
     """bf16 layer forward in float64.
 
     ``hidden_bits`` uint16 [T, H] (bf16), ``logits`` float32 [T, E_r],
@@ -360,15 +394,24 @@ def moe_forward(hidden_bits: np.ndarray, logits: np.ndarray, w13_bits, w2_bits, 
     the k' slot contributions are summed in slot order j = 0..k'-1.
     ``tokens`` restricts the computation to a subset of tokens (routing is
     per token, so the subset's outputs equal the full call's rows).
+    ``routing`` = (ids [T, k'], weights [T, k']) replaces step 1 (the routed
+    variant, see ``append_shared_slot``); ``logits`` is then unused.
     Returns out float64 [len(tokens) or T, H].
     """
-    logits = np.asarray(logits, dtype=np.float32)
-    if tokens is not None:
-        tokens = np.asarray(tokens, dtype=np.int64)
-        hidden_bits = np.asarray(hidden_bits)[tokens]
-        logits = logits[tokens]
+    if routing is not None:
+        ids, w = (np.asarray(routing[0], dtype=np.int32), np.asarray(routing[1], dtype=np.float32))
+        if tokens is not None:
+            tokens = np.asarray(tokens, dtype=np.int64)
+            hidden_bits = np.asarray(hidden_bits)[tokens]
+            ids, w = ids[tokens], w[tokens]
+    else:
+        logits = np.asarray(logits, dtype=np.float32)
+        if tokens is not None:
+            tokens = np.asarray(tokens, dtype=np.int64)
+            hidden_bits = np.asarray(hidden_bits)[tokens]
+            logits = logits[tokens]
+        ids, w = route(logits, topk, renormalize, num_shared)
     x = bf16_bits_to_f64(hidden_bits)
-    ids, w = route(logits, topk, renormalize, num_shared)
     T, kk = ids.shape
     H = x.shape[1]
     I = w2_bits.shape[2]
@@ -388,9 +431,9 @@ def moe_forward(hidden_bits: np.ndarray, logits: np.ndarray, w13_bits, w2_bits, 
     return out
 
 
-def moe_forward_fp8(hidden_bits: np.ndarray, logits: np.ndarray, w13_q, w13_s, w2_q, w2_s, *,
+def moe_forward_fp8(hidden_bits: np.ndarray, logits: Optional[np.ndarray], w13_q, w13_s, w2_q, w2_s, *,
                     topk: int, renormalize: bool, activation: str, num_shared: int = 0,
-                    tokens: Optional[Sequence[int]] = None):
+                    tokens: Optional[Sequence[int]] = None, routing=None):
     """FP8 E4M3 W8A8 layer forward with 128x128 weight blocks, in float64.
 
     [SHARED] section 1 names the configuration (fp8_w8a8, block_shape
@@ -407,16 +450,23 @@ def moe_forward_fp8(hidden_bits: np.ndarray, logits: np.ndarray, w13_q, w13_s, w
         codes are decided on the bf16 value;
       * every product uses the exactly dequantised values q * s in float64.
     ``w13_q``/``w2_q`` are uint8 codes, ``w13_s`` [E, N1/128, H/128] and
-    ``w2_s`` [E, H/128, I/128] float32 scales.
+    ``w2_s`` [E, H/128, I/128] float32 scales. ``routing`` as in ``moe_forward``.
     """
-    logits = np.asarray(logits, dtype=np.float32)
-    if tokens is not None:
-        tokens = np.asarray(tokens, dtype=np.int64)
-        hidden_bits = np.asarray(hidden_bits)[tokens]
-        logits = logits[tokens]
+    if routing is not None:
+        ids, w = (np.asarray(routing[0], dtype=np.int32), np.asarray(routing[1], dtype=np.float32))
+        if tokens is not None:
+            tokens = np.asarray(tokens, dtype=np.int64)
+            hidden_bits = np.asarray(hidden_bits)[tokens]
+            ids, w = ids[tokens], w[tokens]
+    else:
+        logits = np.asarray(logits, dtype=np.float32)
+        if tokens is not None:
+            tokens = np.asarray(tokens, dtype=np.int64)
+            hidden_bits = np.asarray(hidden_bits)[tokens]
+            logits = logits[tokens]
+        ids, w = route(logits, topk, renormalize, num_shared)
     xq, xs = quant_groups_1x128(bf16_bits_to_f32(hidden_bits))
     x = dequant_groups_1x128(xq, xs)
-    ids, w = route(logits, topk, renormalize, num_shared)
     T, kk = ids.shape
     H = x.shape[1]
     I = w2_q.shape[2]

@@ -166,6 +166,58 @@ def test_activation_closed_forms():
     assert float(O.silu(np.array([-1000.0]))[0]) == 0.0
 
 
+def test_gelu_tanh_against_torch_and_limits():
+    # the library routine with the same (tanh) approximation, on a grid and random points
+    x = np.concatenate([np.linspace(-12.0, 12.0, 2001), np.random.default_rng(5).standard_normal(4000) * 3])
+    want = torch.nn.functional.gelu(torch.from_numpy(x), approximate="tanh").numpy()
+    np.testing.assert_allclose(O.gelu_tanh(x), want, rtol=1e-13, atol=1e-15)
+    # closed forms: odd part and limits; gelu_tanh(0) = 0, -> x for large x, -> 0 for very negative x
+    assert float(O.gelu_tanh(np.array([0.0]))[0]) == 0.0
+    assert float(O.gelu_tanh(np.array([30.0]))[0]) == 30.0
+    assert abs(float(O.gelu_tanh(np.array([-30.0]))[0])) < 1e-300 or float(O.gelu_tanh(np.array([-30.0]))[0]) == 0.0
+    y = np.linspace(0.1, 5.0, 50)
+    np.testing.assert_allclose(O.gelu_tanh(y) - O.gelu_tanh(-y), y, rtol=1e-12)   # gelu(x) - gelu(-x) = x
+    # the gated form is act(gate) * up on the gate-first halves
+    z = np.random.default_rng(6).standard_normal((5, 8))
+    np.testing.assert_array_equal(O.activation_fn(z, "gelu_tanh", 4), O.gelu_tanh(z[:, :4]) * z[:, 4:8])
+    assert O.is_gated("gelu_tanh") and O.is_gated("swiglu") and not O.is_gated("relu2")
+
+
+def test_routed_variant_equals_logit_routing():
+    # the forward with caller-supplied routing, given route()'s routed choice, is the
+    # logit-routed forward; append_shared_slot adds the shared slot exactly as route()
+    rng = np.random.default_rng(13)
+    T, H, E, k, I = 7, 32, 5, 2, 16
+    x = _bf16_bits(torch.from_numpy(rng.standard_normal((T, H)).astype(np.float32)))
+    l = rng.standard_normal((T, E)).astype(np.float32)
+    for shared in (0, 1):
+        Et = E + shared
+        w13 = _bf16_bits(torch.from_numpy(0.2 * rng.standard_normal((Et, 2 * I, H)).astype(np.float32)))
+        w2 = _bf16_bits(torch.from_numpy(0.2 * rng.standard_normal((Et, H, I)).astype(np.float32)))
+        ids, w = O.route(l, k, True, shared)
+        rid, rw = O.append_shared_slot(ids[:, :k], w[:, :k], E, shared)
+        np.testing.assert_array_equal(rid, ids)
+        np.testing.assert_array_equal(rw, w)
+        a = O.moe_forward(x, l, w13, w2, topk=k, renormalize=True, activation="swiglu", num_shared=shared)
+        b = O.moe_forward(x, None, w13, w2, topk=k, renormalize=True, activation="swiglu", num_shared=shared,
+                          routing=(rid, rw))
+        np.testing.assert_array_equal(a, b)
+        # arbitrary routing (repeated experts, unnormalised weights) against the dense form
+        rid2 = rng.integers(0, E, size=(T, k)).astype(np.int32)
+        rw2 = rng.uniform(0.1, 2.0, size=(T, k)).astype(np.float32)
+        rid2, rw2 = O.append_shared_slot(rid2, rw2, E, shared)
+        got = O.moe_forward(x, None, w13, w2, topk=k, renormalize=True, activation="swiglu", num_shared=shared,
+                            routing=(rid2, rw2))
+        X, W13, W2 = O.bf16_bits_to_f64(x), O.bf16_bits_to_f64(w13), O.bf16_bits_to_f64(w2)
+        want = np.zeros((T, H))
+        for t in range(T):
+            for j in range(rid2.shape[1]):
+                e = rid2[t, j]
+                z = W13[e] @ X[t]
+                want[t] += float(rw2[t, j]) * (W2[e] @ (z[:I] / (1 + np.exp(-z[:I])) * z[I:]))
+        np.testing.assert_allclose(got, want, rtol=1e-10, atol=1e-12)
+
+
 def test_padding_rules_from_page():
     for i_in, gated, i_pad in _rows("padding_rules.txt"):
         assert O.padded_intermediate(int(i_in), gated == "1") == int(i_pad)
@@ -222,17 +274,21 @@ def _dense_layer(x, logits, w13, w2, topk, renorm, act, num_shared=0):
     z = np.einsum("th,enh->ten", x, w13)
     if act == "swiglu":
         a = z[:, :, :I] / (1.0 + np.exp(-z[:, :, :I])) * z[:, :, I:]
+    elif act == "gelu_tanh":
+        g0 = z[:, :, :I]
+        a = 0.5 * g0 * (1.0 + np.tanh(np.sqrt(2.0 / np.pi) * (g0 + 0.044715 * g0 ** 3))) * z[:, :, I:]
     else:
         a = np.maximum(z, 0.0) ** 2
     ffn = np.einsum("tei,ehi->teh", a, w2)
     return np.einsum("te,teh->th", g, ffn)
 
 
-@pytest.mark.parametrize("act,renorm,shared", [("swiglu", True, 0), ("relu2", False, 0), ("swiglu", True, 1)])
+@pytest.mark.parametrize("act,renorm,shared", [("swiglu", True, 0), ("relu2", False, 0), ("swiglu", True, 1),
+                                                ("gelu_tanh", True, 0)])
 def test_layer_dense_ffn_invariant(act, renorm, shared):
     rng = np.random.default_rng(11)
     T, H, E, k, I = 9, 64, 6, 3, 24
-    N1 = 2 * I if act == "swiglu" else I
+    N1 = 2 * I if act != "relu2" else I
     x = _bf16_bits(torch.from_numpy(rng.standard_normal((T, H)).astype(np.float32)))
     l = rng.standard_normal((T, E)).astype(np.float32)
     Et = E + shared
