@@ -68,7 +68,10 @@ typedef enum {
  * values are this library's own; the page does not print FlashInfer's enum values. */
 typedef enum {
   MOE_ACT_SWIGLU = 0, /* gated: a_n = silu(gate_n) * up_n, silu(x) = x / (1 + e^-x) */
-  MOE_ACT_RELU2 = 1   /* non-gated: a_n = max(z_n, 0)^2 */
+  MOE_ACT_RELU2 = 1,  /* non-gated: a_n = max(z_n, 0)^2 */
+  MOE_ACT_GELU_TANH = 2 /* gated: a_n = gelu_tanh(gate_n) * up_n, gelu_tanh(x) = 0.5 x (1 +
+                           tanh(sqrt(2/pi) (x + 0.044715 x^3))) ("FlashInfer gated MoE kernel
+                           optimisation for Blackwell", section 2; padded like SWIGLU) */
 } moe_activation_t;
 
 /* Weight / activation number format. */
@@ -209,6 +212,22 @@ moe_status_t moe_forward(const moe_problem_t* problem, const void* hidden,
                          const float* w13_scale, const float* w2_scale, void* out,
                          void* workspace, size_t workspace_bytes, moe_stream_t stream);
 
+/* The routed variant of moe_forward: the caller supplies the expert choice instead of
+ * router logits ("FlashInfer TRTLLM-Gen MoE kernel optimisation: NemotronH support",
+ * section 1, names such a routed form of the fused op), and steps 2-5 run as in
+ * moe_forward.
+ *   topk_ids       device int32 [T, topk]: routed expert ids in [0, E_r), slot order;
+ *                  repeats allowed
+ *   topk_weights   device fp32 [T, topk]: their weights, used as given
+ * With num_shared = 1 the shared slot (id E_r, weight 1) follows the routed slots. An id
+ * outside [0, E_r) is dropped (weight 0) and reported by moe_get_device_status as
+ * MOE_ERR_INVALID_ARG (status word bit 0x20000); the other pairs are unaffected. */
+moe_status_t moe_forward_routed(const moe_problem_t* problem, const void* hidden,
+                                const int32_t* topk_ids, const float* topk_weights,
+                                const void* w13, const void* w2, const float* w13_scale,
+                                const float* w2_scale, void* out, void* workspace,
+                                size_t workspace_bytes, moe_stream_t stream);
+
 /* moe_forward with HOST hidden [T,H] bf16, router_logits [T,E_r] fp32 and out [T,H] bf16
  * (pinned memory gives asynchronous copies; pageable memory works too). The inputs are
  * copied into the workspace staging areas, the forward runs, the output is copied back
@@ -269,8 +288,9 @@ moe_status_t moe_align_noalloc(const moe_problem_t* problem, const int32_t* topk
 
 /* Synchronises `stream`, reads and clears the workspace status word. Returns MOE_OK,
  * MOE_ERR_DEVICE_TIMEOUT if a kernel abandoned a bounded wait since the last query
- * (its outputs are then undefined), or MOE_ERR_CUDA. `*detail` (may be NULL) receives
- * the raw word: bits 0-15 name the wait site. */
+ * (word 0x10000 | site; its outputs are then undefined), MOE_ERR_INVALID_ARG if
+ * moe_forward_routed met an expert id out of range (word 0x20000), or MOE_ERR_CUDA.
+ * `*detail` (may be NULL) receives the raw word. */
 moe_status_t moe_get_device_status(void* workspace, moe_stream_t stream, int32_t* detail);
 
 #ifdef __cplusplus

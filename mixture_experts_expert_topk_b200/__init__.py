@@ -18,7 +18,7 @@ from typing import Dict, Optional, Tuple
 import torch
 
 from . import _capi
-from ._capi import (MOE_ACT_RELU2, MOE_ACT_SWIGLU, MOE_DTYPE_BF16, MOE_DTYPE_FP8_BLOCK128,
+from ._capi import (MOE_ACT_GELU_TANH, MOE_ACT_RELU2, MOE_ACT_SWIGLU, MOE_DTYPE_BF16, MOE_DTYPE_FP8_BLOCK128,
                     MOE_FLAG_PDL, MoeError, Problem, check, lib)
 
 __all__ = [
@@ -29,7 +29,8 @@ __all__ = [
 ]
 
 _ACT = {"swiglu": MOE_ACT_SWIGLU, "silu": MOE_ACT_SWIGLU, "relu2": MOE_ACT_RELU2,
-        MOE_ACT_SWIGLU: MOE_ACT_SWIGLU, MOE_ACT_RELU2: MOE_ACT_RELU2}
+        "gelu_tanh": MOE_ACT_GELU_TANH, "gelu": MOE_ACT_GELU_TANH,
+        MOE_ACT_SWIGLU: MOE_ACT_SWIGLU, MOE_ACT_RELU2: MOE_ACT_RELU2, MOE_ACT_GELU_TANH: MOE_ACT_GELU_TANH}
 
 
 def _act(a) -> int:
@@ -106,7 +107,7 @@ def prepare_weights(prob: Problem, w13: torch.Tensor, w2: torch.Tensor, intermed
     _dev(w2, "w2", dt)
     E = prob.num_routed + prob.num_shared
     I = prob.intermediate
-    N1 = 2 * I if prob.activation == MOE_ACT_SWIGLU else I
+    N1 = I if prob.activation == MOE_ACT_RELU2 else 2 * I
     elt = 1 if fp8 else 2
     n13 = lib().moe_prepared_weights_bytes(ctypes.byref(prob), 0)
     n2 = lib().moe_prepared_weights_bytes(ctypes.byref(prob), 1)
@@ -189,6 +190,42 @@ def moe_forward(hidden: torch.Tensor, router_logits: torch.Tensor, w13: torch.Te
     check(lib().moe_forward(ctypes.byref(prob), _ptr(hidden), _ptr(router_logits), _ptr(w13),
                             _ptr(w2), _ptr(w13_scale), _ptr(w2_scale), _ptr(out),
                             _ptr(workspace), workspace.numel(), _stream(stream)), "moe_forward")
+    return out
+
+
+def moe_forward_routed(hidden: torch.Tensor, topk_ids: torch.Tensor, topk_weights: torch.Tensor,
+                       w13: torch.Tensor, w2: torch.Tensor, num_routed: int, activation_type,
+                       w13_scale: Optional[torch.Tensor] = None, w2_scale: Optional[torch.Tensor] = None,
+                       num_shared: int = 0, *, workspace: Optional[torch.Tensor] = None,
+                       out: Optional[torch.Tensor] = None, pdl: bool = True, stream=None) -> torch.Tensor:
+    """The forward with caller-supplied routing: ``topk_ids`` int32 [T, topk] in
+    [0, num_routed), ``topk_weights`` fp32 [T, topk] (used as given); the rest as
+    :func:`moe_forward`. Out-of-range ids are dropped and reported by
+    :func:`device_status`."""
+    fp8 = w13_scale is not None
+    _dev(hidden, "hidden", torch.bfloat16)
+    _dev(topk_ids, "topk_ids", torch.int32)
+    _dev(topk_weights, "topk_weights", torch.float32)
+    _dev(w13, "w13")
+    _dev(w2, "w2")
+    T, H = hidden.shape
+    topk = topk_ids.shape[1]
+    if topk_ids.shape != (T, topk) or topk_weights.shape != (T, topk):
+        raise ValueError("topk_ids and topk_weights must both be [T, topk]")
+    I = getattr(w2, "moe_intermediate", None)
+    if I is None:
+        if w2.dim() != 3:
+            raise ValueError("w2 must come from prepare_weights (or be [E, H, I] row-major)")
+        I = w2.shape[2]
+    prob = make_problem(T, H, num_routed, topk, I, renormalize=False, activation=activation_type,
+                        num_shared=num_shared, fp8=fp8, pdl=pdl)
+    if workspace is None:
+        workspace = _workspace_for(prob, hidden.device)
+    if out is None:
+        out = torch.empty_like(hidden)
+    check(lib().moe_forward_routed(ctypes.byref(prob), _ptr(hidden), _ptr(topk_ids), _ptr(topk_weights),
+                                   _ptr(w13), _ptr(w2), _ptr(w13_scale), _ptr(w2_scale), _ptr(out),
+                                   _ptr(workspace), workspace.numel(), _stream(stream)), "moe_forward_routed")
     return out
 
 

@@ -64,10 +64,11 @@ moe_status_t make_plan(const moe_problem_t* p, Plan* pl) {
   if (p->num_shared != 0 && p->num_shared != 1) return MOE_ERR_INVALID_ARG;
   if (p->topk > p->num_routed) return MOE_ERR_INVALID_ARG;
   if (p->renormalize != 0 && p->renormalize != 1) return MOE_ERR_INVALID_ARG;
-  if (p->activation != MOE_ACT_SWIGLU && p->activation != MOE_ACT_RELU2) return MOE_ERR_INVALID_ARG;
+  if (p->activation != MOE_ACT_SWIGLU && p->activation != MOE_ACT_RELU2 && p->activation != MOE_ACT_GELU_TANH)
+    return MOE_ERR_INVALID_ARG;
   if (p->wdtype != MOE_DTYPE_BF16 && p->wdtype != MOE_DTYPE_FP8_BLOCK128) return MOE_ERR_INVALID_ARG;
   if (p->flags & ~MOE_FLAG_PDL) return MOE_ERR_INVALID_ARG;
-  q.gated = p->activation == MOE_ACT_SWIGLU;
+  q.gated = p->activation != MOE_ACT_RELU2;
   q.fp8 = p->wdtype == MOE_DTYPE_FP8_BLOCK128;
   // the intermediate size must already be padded (moe_padded_intermediate)
   const int ialign = (q.fp8 || !q.gated) ? 128 : 16;
@@ -410,18 +411,25 @@ Launch launch_of(const moe_problem_t* p, moe_stream_t stream) {
   return l;
 }
 
-moe_status_t forward_device(const Plan& pl, const moe_problem_t* p, const void* hidden, const float* logits,
-                            const void* w13, const void* w2, const float* s13, const float* s2, void* out,
-                            void* ws, moe_stream_t stream, int num_sms) {
-  const Launch l = launch_of(p, stream);
-  moe_status_t st = run_route(pl, logits, ws, l, hidden);
-  if (st == MOE_OK) st = run_align(pl, ws, l);
+// Steps 2-5 (everything after the routing step) on routing already in the workspace.
+moe_status_t forward_after_route(const Plan& pl, const Launch& l, const void* hidden, const void* w13, const void* w2,
+                                 const float* s13, const float* s2, void* out, void* ws, int num_sms) {
+  moe_status_t st = run_align(pl, ws, l);
   if (st == MOE_OK && pl.fp8) st = run_quant_act(pl, hidden, ws, l);
   if (st == MOE_OK) st = run_permute(pl, hidden, ws, l, num_sms);
   if (st == MOE_OK) st = run_gemm1(pl, hidden, w13, s13, ws, l, num_sms);
   if (st == MOE_OK) st = run_gemm2(pl, w2, s2, ws, l, num_sms);
   if (st == MOE_OK) st = run_combine(pl, out, ws, l);
   return st;
+}
+
+moe_status_t forward_device(const Plan& pl, const moe_problem_t* p, const void* hidden, const float* logits,
+                            const void* w13, const void* w2, const float* s13, const float* s2, void* out,
+                            void* ws, moe_stream_t stream, int num_sms) {
+  const Launch l = launch_of(p, stream);
+  const moe_status_t st = run_route(pl, logits, ws, l, hidden);
+  if (st != MOE_OK) return st;
+  return forward_after_route(pl, l, hidden, w13, w2, s13, s2, out, ws, num_sms);
 }
 
 moe_status_t check_weights(const Plan& pl, const void* w13, const void* w2, const float* s13, const float* s2) {
@@ -451,7 +459,7 @@ MOE_API moe_status_t moe_check_problem(const moe_problem_t* problem) {
 
 MOE_API int32_t moe_padded_intermediate(int32_t intermediate, int32_t activation, int32_t wdtype) {
   if (intermediate <= 0 || intermediate > (1 << 20)) return -1;
-  if (activation != MOE_ACT_SWIGLU && activation != MOE_ACT_RELU2) return -1;
+  if (activation != MOE_ACT_SWIGLU && activation != MOE_ACT_RELU2 && activation != MOE_ACT_GELU_TANH) return -1;
   if (wdtype != MOE_DTYPE_BF16 && wdtype != MOE_DTYPE_FP8_BLOCK128) return -1;
   const int a = (wdtype == MOE_DTYPE_FP8_BLOCK128 || activation == MOE_ACT_RELU2) ? 128 : 16;
   return (intermediate + a - 1) / a * a;
@@ -538,6 +546,32 @@ MOE_API moe_status_t moe_forward(const moe_problem_t* problem, const void* hidde
   if (st != MOE_OK || pl.T == 0) return st;
   return forward_device(pl, problem, hidden, router_logits, w13, w2, w13_scale, w2_scale, out, workspace, stream,
                         sms);
+}
+
+MOE_API moe_status_t moe_forward_routed(const moe_problem_t* problem, const void* hidden, const int32_t* topk_ids,
+                                        const float* topk_weights, const void* w13, const void* w2,
+                                        const float* w13_scale, const float* w2_scale, void* out, void* workspace,
+                                        size_t workspace_bytes, moe_stream_t stream) {
+  Plan pl;
+  int sms = 0;
+  moe_status_t st = make_plan(problem, &pl);
+  if (st != MOE_OK || pl.T == 0) return st;  // T == 0: nothing to do, pointers unused
+  if (!aligned16(hidden) || !aligned4(topk_ids) || !aligned4(topk_weights) || !aligned16(out) || hidden == out)
+    return MOE_ERR_INVALID_ARG;
+  st = check_weights(pl, w13, w2, w13_scale, w2_scale);
+  if (st != MOE_OK) return st;
+  st = prologue(problem, workspace, workspace_bytes, &pl, &sms);
+  if (st != MOE_OK || pl.T == 0) return st;
+  const Launch l = launch_of(problem, stream);
+  const auto& L = pl.lay;
+  // the status word and work counters start at zero, as after the routing kernel
+  if (cudaMemsetAsync(ws_ptr<int>(workspace, L.status), 0, 16 * sizeof(int), l.stream) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  st = cuda_status(moe::launch_load_routing(l, topk_ids, topk_weights, pl.T, pl.Er, pl.topk, pl.Es,
+                                            ws_ptr<int>(workspace, L.topk_ids), ws_ptr<float>(workspace, L.topk_w),
+                                            ws_ptr<int>(workspace, L.status)));
+  if (st != MOE_OK) return st;
+  return forward_after_route(pl, l, hidden, w13, w2, w13_scale, w2_scale, out, workspace, sms);
 }
 
 MOE_API moe_status_t moe_forward_host(const moe_problem_t* problem, const void* h_hidden,
@@ -659,5 +693,6 @@ MOE_API moe_status_t moe_get_device_status(void* workspace, moe_stream_t stream,
   if (cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
   if (word != 0 && cudaMemset(workspace, 0, sizeof(word)) != cudaSuccess) return MOE_ERR_CUDA;
   if (detail != nullptr) *detail = word;
-  return word == 0 ? MOE_OK : MOE_ERR_DEVICE_TIMEOUT;
+  if (word == 0) return MOE_OK;
+  return (word & moe::kStatusBadRouting) ? MOE_ERR_INVALID_ARG : MOE_ERR_DEVICE_TIMEOUT;
 }

@@ -332,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // previous store drains.
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
     const uint32_t staging = sStage + (warp - kWarpEpi) * a.staging_bufs * a.staging_bytes;
-    const bool gated = a.activation == 0;
+    const bool gated = a.activation != 1;  // 0 SwiGLU, 2 gelu_tanh; 1 relu2
     // GEMM1: act bf16 rows of 16 (gated) or 32 (relu2) columns per box, no swizzle;
     // GEMM2: y fp32 rows of 32 columns (128 B), 128-byte swizzle
     const int box_cols = a.mode == 0 ? (gated ? 16 : 32) : 32;
@@ -379,7 +379,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < 8; ++i) {
               const float g0 = __uint_as_float(v[4 * i + 0]), u0 = __uint_as_float(v[4 * i + 1]);
               const float g1 = __uint_as_float(v[4 * i + 2]), u1 = __uint_as_float(v[4 * i + 3]);
-              o[i] = pack_bf16x2(silu_f32(g0) * u0, silu_f32(g1) * u1);
+              o[i] = pack_bf16x2(gate_act(g0, a.activation) * u0, gate_act(g1, a.activation) * u1);
             }
             const uint32_t dst = buf + lane * 32;
             asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(o[0]), "r"(o[1]), "r"(o[2]),

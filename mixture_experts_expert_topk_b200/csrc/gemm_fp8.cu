@@ -303,7 +303,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------- promotion + epilogue (warps 6..9) ----------------
     const int q = warp & 3;
     const uint32_t staging = sStage + (warp - kWarpEpi) * 2 * kStagingBuf;
-    const bool gated = a.activation == 0;
+    const bool gated = a.activation != 1;  // 0 SwiGLU, 2 gelu_tanh; 1 relu2
     int nst = 0;
     int np = 0;
     int rslot = 0;
@@ -387,7 +387,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (gated) {
 #pragma unroll
             for (int i = 0; i < 32; ++i)
-              o[i] = pack_bf16x2(silu_f32(acc[4 * i]) * acc[4 * i + 1], silu_f32(acc[4 * i + 2]) * acc[4 * i + 3]);
+              o[i] = pack_bf16x2(gate_act(acc[4 * i], a.activation) * acc[4 * i + 1],
+                                 gate_act(acc[4 * i + 2], a.activation) * acc[4 * i + 3]);
           } else {
 #pragma unroll
             for (int i = 0; i < 32; ++i) {

@@ -12,7 +12,7 @@
 // A TMEM lane is one weight row. GEMM1: the gate and up rows of an intermediate index sit
 // in adjacent lanes (the [gate0, up0, gate1, up1, ...] interleave prepared at load time,
 // "[MoE] SwiGLU fusion into the MoE up-GEMM epilogue", sglang PR 32944, section 3) and are
-// paired with one shuffle before silu(gate)*up (or relu2); the kernel writes only the
+// paired with one shuffle before act(gate)*up (silu or gelu_tanh; or relu2); the kernel writes only the
 // bf16 activation. GEMM2: the epilogue multiplies token column j by topk_w of its pair and
 // writes fp32 y rows (sorted order) for the fixed-order combine.
 //
@@ -329,7 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
     // neighbouring output columns, so each store writes one contiguous piece of an output
     // row (GEMM2: 128 B of fp32; GEMM1: 64 or 32 B of a 128-byte activation chunk row).
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
-    const bool gated = a.activation == 0;
+    const bool gated = a.activation != 1;  // 0 SwiGLU, 2 gelu_tanh; 1 relu2
     const bool odd = (lane & 1) != 0;
     int rslot = 0, it = 0;
     uint32_t rph = 0;
@@ -417,7 +417,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
             const int row = c0 + (odd ? 16 + j : j);
             if (!odd || full)
               *reinterpret_cast<__nv_bfloat16*>(act_grp + row * kChunkBytes + ((((fo >> 3) ^ row) & 7) << 4) +
-                                                (fo & 7) * 2) = __float2bfloat16_rn(silu_f32(g) * u);
+                                                (fo & 7) * 2) = __float2bfloat16_rn(gate_act(g, a.activation) * u);
           }
         }
       }

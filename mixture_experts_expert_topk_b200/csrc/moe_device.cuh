@@ -315,4 +315,12 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // for very negative g) costs no visible accuracy.
 __device__ __forceinline__ float silu_f32(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
+// gelu_tanh(g) = 0.5 g (1 + tanh(sqrt(2/pi) (g + 0.044715 g^3))), with CUDA's tanhf.
+__device__ __forceinline__ float gelu_tanh_f32(float g) {
+  return 0.5f * g * (1.0f + tanhf(0.7978845608028654f * (g + 0.044715f * g * g * g)));
+}
+
+// Gate activation of a gated layer: act 0 = SwiGLU (silu), 2 = gelu_tanh.
+__device__ __forceinline__ float gate_act(float g, int act) { return act == 2 ? gelu_tanh_f32(g) : silu_f32(g); }
+
 }  // namespace moe

@@ -10,6 +10,9 @@ namespace moe {
 constexpr int kMaxExperts = 1024;  // routed + shared
 constexpr int kMaxSlots = 16;      // k' = topk + num_shared
 constexpr int kAlignChunk = 2048;  // pairs per align chunk
+// Status word value (beyond the wait timeouts 0x10000 | site): caller-supplied routing held
+// an expert id outside [0, E_r) (the pair was dropped: id 0, weight 0).
+constexpr int kStatusBadRouting = 0x20000;
 
 // Launch configuration shared by all launchers.
 struct Launch {
@@ -25,6 +28,11 @@ void make_launch_config(cudaLaunchConfig_t* cfg, cudaLaunchAttribute* attr, cons
 cudaError_t launch_route(const Launch& l, const float* logits, int T, int E_routed, int topk,
                          int num_shared, int renormalize, int* topk_ids, float* topk_w,
                          int* status, const void* hidden, int hidden_row_bytes);
+
+// Caller-supplied routing ids/weights [T, topk] into topk_ids/topk_w [T, k'] (route.cu).
+// The caller clears the status words first.
+cudaError_t launch_load_routing(const Launch& l, const int* ids_in, const float* w_in, int T, int E_routed,
+                                int topk, int num_shared, int* topk_ids, float* topk_w, int* status);
 
 // ---- align (align.cu) ----
 // num_blocks[0] = P_pad / block_m. With group_rows > 0 (block_m 16), each expert's rows

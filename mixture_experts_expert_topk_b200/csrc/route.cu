@@ -111,6 +111,37 @@ __global__ void __launch_bounds__(kRouteWarps * 32)
   }
 }
 
+// The routed variant ("FlashInfer TRTLLM-Gen MoE kernel optimisation: NemotronH support",
+// section 1, names a routed form of the fused op that takes the top-k choice): the
+// caller's ids and weights [T, topk] into the workspace's [T, k'] layout, the shared slot
+// (id E_r, weight 1) after them as in route_kernel. An id outside [0, E_r) cannot be
+// routed: the pair becomes expert 0 with weight 0 (contributing nothing) and the status
+// word records kStatusBadRouting.
+__global__ void load_routing_kernel(const int* __restrict__ ids_in, const float* __restrict__ w_in, int T, int E,
+                                    int topk, int num_shared, int* __restrict__ topk_ids, float* __restrict__ topk_w,
+                                    int* __restrict__ status) {
+  griddep_wait();
+  griddep_launch_dependents();
+  const int kk = topk + num_shared;
+  const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= static_cast<long long>(T) * kk) return;
+  const long long t = idx / kk;
+  const int j = static_cast<int>(idx - t * kk);
+  int e = E;
+  float w = 1.0f;
+  if (j < topk) {
+    e = __ldg(ids_in + t * topk + j);
+    w = __ldg(w_in + t * topk + j);
+    if (e < 0 || e >= E) {
+      e = 0;
+      w = 0.0f;
+      atomicCAS(status, 0, kStatusBadRouting);
+    }
+  }
+  topk_ids[idx] = e;
+  topk_w[idx] = w;
+}
+
 template <int VPL>
 cudaError_t launch_vpl(const Launch& l, const float* logits, int T, int E, int topk,
                        int num_shared, int renormalize, int* ids, float* w, int* status,
@@ -124,6 +155,16 @@ cudaError_t launch_vpl(const Launch& l, const float* logits, int T, int E, int t
 }
 
 }  // namespace
+
+cudaError_t launch_load_routing(const Launch& l, const int* ids_in, const float* w_in, int T, int E_routed,
+                                int topk, int num_shared, int* topk_ids, float* topk_w, int* status) {
+  const long long n = static_cast<long long>(T) * (topk + num_shared);
+  cudaLaunchConfig_t cfg;
+  cudaLaunchAttribute attr[1];
+  make_launch_config(&cfg, attr, l, dim3(static_cast<unsigned>((n + 255) / 256)), dim3(256), 0);
+  return cudaLaunchKernelEx(&cfg, load_routing_kernel, ids_in, w_in, T, E_routed, topk, num_shared, topk_ids, topk_w,
+                            status);
+}
 
 cudaError_t launch_route(const Launch& l, const float* logits, int T, int E_routed, int topk,
                          int num_shared, int renormalize, int* topk_ids, float* topk_w,

@@ -46,7 +46,7 @@ class MoeConfig:
 
     @property
     def gated(self) -> bool:
-        return self.activation == "swiglu"
+        return self.activation != "relu2"
 
     @property
     def E_total(self) -> int:

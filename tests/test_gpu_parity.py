@@ -54,6 +54,9 @@ SMALL = {
     # three align chunks (the single-launch align with its grid barrier) and more experts
     # than the align CTA has threads
     "many_experts": _small("many_experts", T=700, H=256, E=300, topk=8, I=128),
+    # the gelu_tanh gated activation, both GEMM paths (with an unaligned intermediate)
+    "gelu_small": _small("gelu_small", T=300, H=256, E=8, topk=2, I=200, activation="gelu_tanh"),
+    "gelu_big": _small("gelu_big", T=600, H=256, E=6, topk=2, I=256, activation="gelu_tanh"),
 }
 
 
@@ -138,7 +141,7 @@ def _check_act(cfg, run, parts, ids, a):
 
 
 @pytest.mark.parametrize("name,bm", [(n, 0) for n in SMALL] +
-                         [(n, 128) for n in ("ragged", "skewed", "pad_gated", "relu2_small")])
+                         [(n, 128) for n in ("ragged", "skewed", "pad_gated", "relu2_small", "gelu_small")])
 def test_layer_parity_small(name, bm):
     # bm 0: the default (bf16: 16-row alignment, weights on the MMA's M); 128: token tiles
     cfg = SMALL[name]
@@ -323,6 +326,7 @@ FP8_SMALL = {
     "fp8_shared_small": _small("fp8_shared_small", T=300, H=384, E=16, topk=3, I=384, num_shared=1, fp8=True),
     "fp8_relu2": _small("fp8_relu2", T=96, H=256, E=6, topk=2, I=256, activation="relu2", renormalize=False,
                         fp8=True),
+    "fp8_gelu": _small("fp8_gelu", T=64, H=256, E=8, topk=2, I=256, activation="gelu_tanh", fp8=True),
 }
 
 
@@ -369,3 +373,75 @@ def test_decode_both_row_tilings(T, bm):
     _check_route_align(cfg, parts, run.inp["logits"])
     ref = oracle_out(cfg, run.inp)
     assert err_beyond_rounding(bf16_to_f64(out), ref) <= BF16_TOL
+
+
+# ---- caller-supplied routing (the routed variant) -------------------------------------
+
+def _routed_call(run, ids, w, cfg):
+    out = torch.empty_like(run.hidden)
+    moe.moe_forward_routed(run.hidden, ids.cuda().contiguous(), w.cuda().contiguous(), run.w13p, run.w2p, cfg.E,
+                           cfg.activation, run.w13_scale, run.w2_scale, num_shared=cfg.num_shared,
+                           workspace=run.ws, out=out)
+    torch.cuda.synchronize()
+    return out
+
+
+@pytest.mark.parametrize("name", ["ragged", "shared_bf16", "tiny"])
+def test_routed_with_own_routing_is_bitwise_the_forward(name):
+    # the routed entry point given the route step's own choice runs the same kernels on
+    # the same routing, so its output is the forward's, bit for bit
+    cfg = SMALL[name]
+    run = GpuRun(cfg)
+    ref = bits(run.forward()).copy()
+    parts = run.parts()
+    ids = torch.from_numpy(parts["topk_ids"][:, :cfg.topk].copy())
+    w = torch.from_numpy(parts["topk_w"][:, :cfg.topk].copy())
+    np.testing.assert_array_equal(bits(_routed_call(run, ids, w, cfg)), ref)
+    assert moe.device_status(run.ws)[0] == 0
+
+
+@pytest.mark.parametrize("name", ["skewed", "shared_bf16", "fp8_tiny"])
+def test_routed_arbitrary_routing_matches_oracle(name):
+    # repeated experts within a token and weights that are not a softmax
+    cfg = SMALL.get(name) or FP8_SMALL[name]
+    run = GpuRun(cfg)
+    g = torch.Generator().manual_seed(21)
+    ids = torch.randint(0, cfg.E, (cfg.T, cfg.topk), generator=g, dtype=torch.int32)
+    ids[::5, 0] = ids[::5, -1]                      # repeats
+    w = torch.rand((cfg.T, cfg.topk), generator=g) * 2.0
+    got = bf16_to_f64(_routed_call(run, ids, w, cfg))
+    routing = O.append_shared_slot(ids.numpy(), w.numpy(), cfg.E, cfg.num_shared)
+    if cfg.fp8:
+        ref = O.moe_forward_fp8(bits(run.inp["hidden"]), None, *O.quantize_weights_fp8(
+            bits(run.inp["w13"]), bits(run.inp["w2"])), topk=cfg.topk, renormalize=False,
+            activation=cfg.activation, num_shared=cfg.num_shared, routing=routing)
+    else:
+        ref = O.moe_forward(bits(run.inp["hidden"]), None, bits(run.inp["w13"]), bits(run.inp["w2"]),
+                            topk=cfg.topk, renormalize=False, activation=cfg.activation,
+                            num_shared=cfg.num_shared, routing=routing)
+    e = err_beyond_rounding(got, ref)
+    assert e <= (FP8_TOL if cfg.fp8 else BF16_TOL), e
+    assert moe.device_status(run.ws)[0] == 0
+
+
+def test_routed_out_of_range_ids_are_dropped_and_reported():
+    cfg = SMALL["ragged"]
+    run = GpuRun(cfg)
+    g = torch.Generator().manual_seed(22)
+    ids = torch.randint(0, cfg.E, (cfg.T, cfg.topk), generator=g, dtype=torch.int32)
+    w = torch.rand((cfg.T, cfg.topk), generator=g)
+    ids[3, 1] = -1
+    ids[10, 0] = cfg.E            # one past the last routed expert
+    got = bf16_to_f64(_routed_call(run, ids, w, cfg))
+    st, word = moe.device_status(run.ws)
+    assert st == 1 and word == 0x20000            # MOE_ERR_INVALID_ARG, bad routing
+    assert moe.device_status(run.ws)[0] == 0      # the query cleared it
+    # the dropped pairs contribute nothing: the oracle with their weights set to zero
+    ids_ok, w_ok = ids.clone(), w.clone()
+    for t, j in ((3, 1), (10, 0)):
+        ids_ok[t, j] = 0
+        w_ok[t, j] = 0.0
+    ref = O.moe_forward(bits(run.inp["hidden"]), None, bits(run.inp["w13"]), bits(run.inp["w2"]),
+                        topk=cfg.topk, renormalize=False, activation=cfg.activation,
+                        routing=O.append_shared_slot(ids_ok.numpy(), w_ok.numpy(), cfg.E, 0))
+    assert err_beyond_rounding(got, ref) <= BF16_TOL
