@@ -485,6 +485,81 @@ def moe_forward_fp8(hidden_bits: np.ndarray, logits: Optional[np.ndarray], w13_q
     return out
 
 
+def quant_per_tensor(x: np.ndarray, scale) -> np.ndarray:
+    """Static per-tensor quantisation to E4M3: q = e4m3(x / scale), the division in
+    fp32 rounded to nearest, saturating at 448. The per-tensor FP8 variant of the
+    fused op (``trtllm_fp8_per_tensor_scale_moe``, [TRTLLM] sections 1 and 2) takes
+    one fp32 scale per tensor: per expert for the weights, one static input scale and
+    one static activation scale for the two GEMM inputs."""
+    x = np.asarray(x, dtype=np.float32)
+    return e4m3_encode((x / np.float32(scale)).astype(np.float32))
+
+
+def quantize_weights_fp8_per_tensor(w13_bits, w2_bits):
+    """Per-expert E4M3 weights for the per-tensor variant: scale = amax / 448 of the
+    expert's matrix in fp32 (1 for an all-zero matrix), codes = quant_per_tensor.
+    Returns (w13 codes, w13 scales [E], w2 codes, w2 scales [E])."""
+    out = []
+    for wb in (w13_bits, w2_bits):
+        w = bf16_bits_to_f32(np.asarray(wb))
+        amax = np.abs(w.reshape(w.shape[0], -1)).max(axis=1)
+        sc = (amax / np.float32(E4M3_MAX)).astype(np.float32)
+        sc = np.where(amax == 0, np.float32(1.0), sc).astype(np.float32)
+        q = np.stack([quant_per_tensor(w[e], sc[e]) for e in range(w.shape[0])])
+        out += [q, sc]
+    return tuple(out)
+
+
+def moe_forward_fp8_per_tensor(hidden_bits: np.ndarray, logits: Optional[np.ndarray], w13_q, w13_s, w2_q, w2_s,
+                               input_scale, activation_scale, *, topk: int, renormalize: bool, activation: str,
+                               num_shared: int = 0, tokens: Optional[Sequence[int]] = None, routing=None):
+    """Per-tensor FP8 layer forward in float64.
+
+    [TRTLLM] section 2 gives the scale algebra of the per-tensor variant: the GEMM1
+    output is dequantised by g1_alphas = w13_scale * input_scale and, after the
+    activation, requantised for GEMM2 by 1 / activation_scale; for a gated layer the
+    two fold into g1_scale_c = g1_alphas / activation_scale, for relu2 (no gate
+    dequantisation term) into 1 / activation_scale. Reading taken (the kernel itself is
+    not printed): the activation acts on the dequantised GEMM1 output, and
+      * x_q = quant_per_tensor(hidden, input_scale);
+      * z = (x_q * input_scale) (W13_q[e] * w13_scale[e])^T, a = activation(z);
+      * a_q = quant_per_tensor(a, activation_scale) (decided in fp32 on a);
+      * y = w_tj * (a_q * activation_scale) (W2_q[e] * w2_scale[e])^T;
+    ``w13_s``/``w2_s`` are float32 [E]; the two static scales are float32 scalars.
+    ``routing`` as in ``moe_forward``.
+    """
+    if routing is not None:
+        ids, w = (np.asarray(routing[0], dtype=np.int32), np.asarray(routing[1], dtype=np.float32))
+        if tokens is not None:
+            tokens = np.asarray(tokens, dtype=np.int64)
+            hidden_bits = np.asarray(hidden_bits)[tokens]
+            ids, w = ids[tokens], w[tokens]
+    else:
+        logits = np.asarray(logits, dtype=np.float32)
+        if tokens is not None:
+            tokens = np.asarray(tokens, dtype=np.int64)
+            hidden_bits = np.asarray(hidden_bits)[tokens]
+            logits = logits[tokens]
+        ids, w = route(logits, topk, renormalize, num_shared)
+    s_in, s_act = np.float32(input_scale), np.float32(activation_scale)
+    x = e4m3_decode(quant_per_tensor(bf16_bits_to_f32(hidden_bits), s_in)) * np.float64(s_in)
+    T, kk = ids.shape
+    H = x.shape[1]
+    I = w2_q.shape[2]
+    y = np.zeros((T, kk, H), dtype=np.float64)
+    for e in np.unique(ids):
+        t_idx, j_idx = np.nonzero(ids == e)
+        W13 = e4m3_decode(np.asarray(w13_q[e])) * np.float64(w13_s[e])
+        W2 = e4m3_decode(np.asarray(w2_q[e])) * np.float64(w2_s[e])
+        a = activation_fn(x[t_idx] @ W13.T, activation, I)
+        ad = e4m3_decode(quant_per_tensor(a, s_act)) * np.float64(s_act)
+        y[t_idx, j_idx] = w[t_idx, j_idx].astype(np.float64)[:, None] * (ad @ W2.T)
+    out = np.zeros((T, H), dtype=np.float64)
+    for j in range(kk):
+        out += y[:, j]
+    return out
+
+
 def quantize_weights_fp8(w13_bits, w2_bits, experts=None):
     """Quantise bf16 master weights per 128x128 block (``quant_blocks_128x128``).
 

@@ -460,6 +460,59 @@ def test_fp8_layer_equals_bf16_layer_on_dequantised_inputs():
     np.testing.assert_allclose(got, want, rtol=1e-9, atol=1e-12)
 
 
+def test_quant_per_tensor_matches_torch_cast():
+    rng = np.random.default_rng(31)
+    x = (rng.standard_normal(20000) * 3).astype(np.float32)
+    scale = np.float32(np.abs(x).max() / 448)
+    want = torch.from_numpy(x / scale).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    np.testing.assert_array_equal(O.quant_per_tensor(x, scale), want)
+    # beyond 448 saturates (the torch cast would give NaN there)
+    assert O.quant_per_tensor(np.array([1000.0, -1000.0], np.float32), 1.0).tolist() == [0x7E, 0xFE]
+
+
+@pytest.mark.parametrize("act", ["swiglu", "relu2", "gelu_tanh"])
+def test_fp8_per_tensor_layer_against_torch_casts(act):
+    # independent restatement with torch float8 casts and a dense per-token loop
+    rng = np.random.default_rng(17)
+    T, H, E, k, I = 6, 256, 3, 2, 128
+    N1 = I if act == "relu2" else 2 * I
+    x = _bf16_bits(torch.from_numpy(rng.standard_normal((T, H)).astype(np.float32)))
+    l = rng.standard_normal((T, E)).astype(np.float32)
+    w13 = _bf16_bits(torch.from_numpy(0.02 * rng.standard_normal((E, N1, H)).astype(np.float32)))
+    w2 = _bf16_bits(torch.from_numpy(0.02 * rng.standard_normal((E, H, I)).astype(np.float32)))
+    q13, s13, q2, s2 = O.quantize_weights_fp8_per_tensor(w13, w2)
+    X = O.bf16_bits_to_f32(x)
+    s_in = np.float32(np.abs(X).max() / 448)
+    s_act = np.float32(0.05)
+    got = O.moe_forward_fp8_per_tensor(x, l, q13, s13, q2, s2, s_in, s_act, topk=k, renormalize=True,
+                                       activation=act)
+
+    def f8(a, s):  # quantise with the torch cast, return the dequantised float64 values
+        q = torch.from_numpy(np.clip(a / s, -448, 448).astype(np.float32)).to(torch.float8_e4m3fn)
+        return q.to(torch.float64).numpy() * np.float64(s)
+
+    W13 = [f8(O.bf16_bits_to_f32(w13[e]), s13[e]) for e in range(E)]
+    W2 = [f8(O.bf16_bits_to_f32(w2[e]), s2[e]) for e in range(E)]
+    Xd = f8(X, s_in)
+    ids, wts = _route_brute(l, k, True)
+    want = np.zeros((T, H))
+    for t in range(T):
+        for j in range(k):
+            e = ids[t, j]
+            z = W13[e] @ Xd[t]
+            if act == "relu2":
+                a = np.maximum(z, 0) ** 2
+            else:
+                g, u = z[:I], z[I:]
+                a = (g / (1 + np.exp(-g)) if act == "swiglu" else
+                     0.5 * g * (1 + np.tanh(np.sqrt(2 / np.pi) * (g + 0.044715 * g ** 3)))) * u
+            want[t] += np.float64(np.float32(wts[t, j])) * (W2[e] @ f8(a.astype(np.float32), s_act))
+    np.testing.assert_allclose(got, want, rtol=1e-9, atol=1e-12)
+    # per-expert weight scales are amax / 448
+    np.testing.assert_array_equal(s13, (np.abs(O.bf16_bits_to_f32(w13).reshape(E, -1)).max(1) / np.float32(448))
+                                  .astype(np.float32))
+
+
 # --------------------------------------------------------------------------
 # planted mistakes: each mutated oracle must fail a pin above
 # --------------------------------------------------------------------------
