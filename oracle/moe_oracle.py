@@ -495,6 +495,17 @@ def quant_per_tensor(x: np.ndarray, scale) -> np.ndarray:
     return e4m3_encode((x / np.float32(scale)).astype(np.float32))
 
 
+def quant_per_tensor_inv(x: np.ndarray, scale) -> np.ndarray:
+    """Static per-tensor quantisation of a GEMM input as the per-tensor variant writes it:
+    [TRTLLM] section 2 scales by the reciprocal, ``* (1.0 / activation_scale)``, so
+    q = e4m3(x * inv) with inv = fp32(1 / scale) and the product rounded to fp32,
+    saturating at 448. Used for the hidden rows (input_scale) and for GEMM1's activation
+    (activation_scale)."""
+    x = np.asarray(x, dtype=np.float32)
+    inv = np.float32(1.0) / np.float32(scale)
+    return e4m3_encode((x * inv).astype(np.float32))
+
+
 def quantize_weights_fp8_per_tensor(w13_bits, w2_bits):
     """Per-expert E4M3 weights for the per-tensor variant: scale = amax / 448 of the
     expert's matrix in fp32 (1 for an all-zero matrix), codes = quant_per_tensor.
@@ -521,9 +532,9 @@ def moe_forward_fp8_per_tensor(hidden_bits: np.ndarray, logits: Optional[np.ndar
     two fold into g1_scale_c = g1_alphas / activation_scale, for relu2 (no gate
     dequantisation term) into 1 / activation_scale. Reading taken (the kernel itself is
     not printed): the activation acts on the dequantised GEMM1 output, and
-      * x_q = quant_per_tensor(hidden, input_scale);
+      * x_q = quant_per_tensor_inv(hidden, input_scale);
       * z = (x_q * input_scale) (W13_q[e] * w13_scale[e])^T, a = activation(z);
-      * a_q = quant_per_tensor(a, activation_scale) (decided in fp32 on a);
+      * a_q = quant_per_tensor_inv(a, activation_scale) (decided in fp32 on a);
       * y = w_tj * (a_q * activation_scale) (W2_q[e] * w2_scale[e])^T;
     ``w13_s``/``w2_s`` are float32 [E]; the two static scales are float32 scalars.
     ``routing`` as in ``moe_forward``.
@@ -542,7 +553,7 @@ def moe_forward_fp8_per_tensor(hidden_bits: np.ndarray, logits: Optional[np.ndar
             logits = logits[tokens]
         ids, w = route(logits, topk, renormalize, num_shared)
     s_in, s_act = np.float32(input_scale), np.float32(activation_scale)
-    x = e4m3_decode(quant_per_tensor(bf16_bits_to_f32(hidden_bits), s_in)) * np.float64(s_in)
+    x = e4m3_decode(quant_per_tensor_inv(bf16_bits_to_f32(hidden_bits), s_in)) * np.float64(s_in)
     T, kk = ids.shape
     H = x.shape[1]
     I = w2_q.shape[2]
@@ -552,7 +563,7 @@ def moe_forward_fp8_per_tensor(hidden_bits: np.ndarray, logits: Optional[np.ndar
         W13 = e4m3_decode(np.asarray(w13_q[e])) * np.float64(w13_s[e])
         W2 = e4m3_decode(np.asarray(w2_q[e])) * np.float64(w2_s[e])
         a = activation_fn(x[t_idx] @ W13.T, activation, I)
-        ad = e4m3_decode(quant_per_tensor(a, s_act)) * np.float64(s_act)
+        ad = e4m3_decode(quant_per_tensor_inv(a, s_act)) * np.float64(s_act)
         y[t_idx, j_idx] = w[t_idx, j_idx].astype(np.float64)[:, None] * (ad @ W2.T)
     out = np.zeros((T, H), dtype=np.float64)
     for j in range(kk):

@@ -468,6 +468,10 @@ def test_quant_per_tensor_matches_torch_cast():
     np.testing.assert_array_equal(O.quant_per_tensor(x, scale), want)
     # beyond 448 saturates (the torch cast would give NaN there)
     assert O.quant_per_tensor(np.array([1000.0, -1000.0], np.float32), 1.0).tolist() == [0x7E, 0xFE]
+    # the reciprocal form for GEMM inputs: the torch cast of x * fp32(1 / scale)
+    inv = np.float32(1.0) / scale
+    want_inv = torch.from_numpy((x * inv).astype(np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    np.testing.assert_array_equal(O.quant_per_tensor_inv(x, scale), want_inv)
 
 
 @pytest.mark.parametrize("act", ["swiglu", "relu2", "gelu_tanh"])
@@ -487,13 +491,19 @@ def test_fp8_per_tensor_layer_against_torch_casts(act):
     got = O.moe_forward_fp8_per_tensor(x, l, q13, s13, q2, s2, s_in, s_act, topk=k, renormalize=True,
                                        activation=act)
 
-    def f8(a, s):  # quantise with the torch cast, return the dequantised float64 values
+    def f8(a, s):  # weights: quantise x / s with the torch cast, dequantise to float64
         q = torch.from_numpy(np.clip(a / s, -448, 448).astype(np.float32)).to(torch.float8_e4m3fn)
+        return q.to(torch.float64).numpy() * np.float64(s)
+
+    def f8i(a, s):  # GEMM inputs: x * fp32(1 / s)
+        inv = np.float32(1.0) / np.float32(s)
+        q = torch.from_numpy(np.clip(a.astype(np.float32) * inv, -448, 448).astype(np.float32)).to(
+            torch.float8_e4m3fn)
         return q.to(torch.float64).numpy() * np.float64(s)
 
     W13 = [f8(O.bf16_bits_to_f32(w13[e]), s13[e]) for e in range(E)]
     W2 = [f8(O.bf16_bits_to_f32(w2[e]), s2[e]) for e in range(E)]
-    Xd = f8(X, s_in)
+    Xd = f8i(X, s_in)
     ids, wts = _route_brute(l, k, True)
     want = np.zeros((T, H))
     for t in range(T):
@@ -506,7 +516,7 @@ def test_fp8_per_tensor_layer_against_torch_casts(act):
                 g, u = z[:I], z[I:]
                 a = (g / (1 + np.exp(-g)) if act == "swiglu" else
                      0.5 * g * (1 + np.tanh(np.sqrt(2 / np.pi) * (g + 0.044715 * g ** 3)))) * u
-            want[t] += np.float64(np.float32(wts[t, j])) * (W2[e] @ f8(a.astype(np.float32), s_act))
+            want[t] += np.float64(np.float32(wts[t, j])) * (W2[e] @ f8i(a.astype(np.float32), s_act))
     np.testing.assert_allclose(got, want, rtol=1e-9, atol=1e-12)
     # per-expert weight scales are amax / 448
     np.testing.assert_array_equal(s13, (np.abs(O.bf16_bits_to_f32(w13).reshape(E, -1)).max(1) / np.float32(448))
