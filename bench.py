@@ -56,7 +56,7 @@ def _peaks():
 
 def _workload_name(cfg: MoeConfig) -> str:
     act = "SwiGLU" if cfg.gated else "relu2"
-    dt = "FP8 e4m3 W8A8 block-128" if cfg.fp8 else "bf16"
+    dt = ("FP8 e4m3 W8A8 per-tensor" if cfg.per_tensor else "FP8 e4m3 W8A8 block-128") if cfg.fp8 else "bf16"
     sh = f"+{cfg.num_shared} shared" if cfg.num_shared else ""
     return (f"{cfg.name}: {dt} {act} MoE layer forward, T={cfg.T} H={cfg.H} E={cfg.E}{sh} "
             f"top-{cfg.topk}{sh} I={cfg.I}")
@@ -178,14 +178,20 @@ def run_ours(cfg: MoeConfig, steps: int, warmup: int, world: int, rank: int, loc
     dev = torch.device("cuda", local)
     inp = make_inputs(cfg, seed=0)
     I_pad = moe.padded_intermediate(cfg.I, cfg.activation, cfg.fp8)
+    s_in = float(inp["hidden"].float().abs().max() / 448) if cfg.per_tensor else 0.0
     prob = moe.make_problem(cfg.T, cfg.H, cfg.E, cfg.topk, I_pad, renormalize=cfg.renormalize,
-                            activation=cfg.activation, num_shared=cfg.num_shared, fp8=cfg.fp8)
+                            activation=cfg.activation, num_shared=cfg.num_shared, fp8=cfg.fp8,
+                            input_scale=s_in, activation_scale=cfg.activation_scale)
+    pt_kw = dict(input_scale=s_in, activation_scale=cfg.activation_scale) if cfg.per_tensor else {}
     hidden = inp["hidden"].to(dev)
     logits = inp["logits"].to(dev)
     s13 = s2 = None
     w13 = inp["w13"].to(dev)
     w2 = inp["w2"].to(dev)
-    if cfg.fp8:
+    if cfg.per_tensor:
+        w13, s13 = moe.quantize_weights_fp8_per_tensor(w13)
+        w2, s2 = moe.quantize_weights_fp8_per_tensor(w2)
+    elif cfg.fp8:
         w13, s13 = moe.quantize_weights_fp8(w13)
         w2, s2 = moe.quantize_weights_fp8(w2)
     w13p, w2p = moe.prepare_weights(prob, w13, w2, cfg.I)
@@ -198,7 +204,7 @@ def run_ours(cfg: MoeConfig, steps: int, warmup: int, world: int, rank: int, loc
 
     def forward():
         moe.moe_forward(hidden, logits, w13p, w2p, cfg.topk, cfg.renormalize, cfg.activation,
-                        s13, s2, num_shared=cfg.num_shared, workspace=ws, out=out)
+                        s13, s2, num_shared=cfg.num_shared, workspace=ws, out=out, **pt_kw)
 
     for _ in range(warmup):
         flush.zero_()
@@ -235,7 +241,7 @@ def run_ours(cfg: MoeConfig, steps: int, warmup: int, world: int, rank: int, loc
 
     # per-kernel breakdown: the same kernels through the per-step entry points, events
     # between the steps on the launching stream
-    names = ["route", "align"] + (["quant_act"] if cfg.fp8 else ["permute"]) + ["gemm1", "gemm2", "combine"]
+    names = ["route", "align"] + (["quant_act"] if cfg.block128 else ["permute"]) + ["gemm1", "gemm2", "combine"]
     per = {n: [] for n in names}
     for _ in range(steps):
         flush.zero_()
@@ -244,7 +250,7 @@ def run_ours(cfg: MoeConfig, steps: int, warmup: int, world: int, rank: int, loc
         k = 0
         moe.stage_route(prob, logits, ws); k += 1; evs[k].record(stream)
         moe.stage_align(prob, ws); k += 1; evs[k].record(stream)
-        if cfg.fp8:
+        if cfg.block128:
             moe.stage_quant_act(prob, hidden, ws); k += 1; evs[k].record(stream)
         else:
             moe.stage_permute(prob, hidden, ws); k += 1; evs[k].record(stream)
@@ -284,7 +290,7 @@ def run_ours(cfg: MoeConfig, steps: int, warmup: int, world: int, rank: int, loc
         "h2d": h_hidden.numel() * 2 + h_logits.numel() * 4, "d2h": h_out.numel() * 2,
         # one kernel per stage, except align (three kernels above one 2048-pair chunk) and
         # FP8 GEMM1 (the GEMM, then the per-row activation quantisation)
-        "launches_per_step": len(names) + (2 if cfg.T * cfg.k_total > 2048 else 0) + (1 if cfg.fp8 else 0),
+        "launches_per_step": len(names) + (2 if cfg.T * cfg.k_total > 2048 else 0) + (1 if cfg.block128 else 0),
     }
 
 
@@ -294,7 +300,7 @@ def _gemm1_traffic(cfg: MoeConfig, g1_bytes: float):
     import hashlib
     src = os.path.join(ROOT, "mixture_experts_expert_topk_b200", "csrc", GEMM1_TRAFFIC["source"])
     sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:12]
-    if cfg.fp8 or GEMM1_TRAFFIC["ratio"] is None or sha != GEMM1_TRAFFIC["source_sha256"]:
+    if cfg.fp8 or GEMM1_TRAFFIC["ratio"] is None or sha != GEMM1_TRAFFIC["source_sha256"]:  # bf16 capture
         return None
     return g1_bytes * GEMM1_TRAFFIC["ratio"]
 
@@ -308,11 +314,19 @@ def cpu_baseline(cfg: MoeConfig, inp, budget_s: float, tokens_hint: int):
 
     hb, lg = bits(inp["hidden"]), inp["logits"].numpy()
     w13b, w2b = bits(inp["w13"]), bits(inp["w2"])
-    fp8w = O.quantize_weights_fp8(w13b, w2b) if cfg.fp8 else None
+    if cfg.per_tensor:
+        fp8w = O.quantize_weights_fp8_per_tensor(w13b, w2b)
+        s_in = np.float32(np.abs(O.bf16_bits_to_f32(hb)).max() / np.float32(448))
+    elif cfg.fp8:
+        fp8w = O.quantize_weights_fp8(w13b, w2b)
     n = max(1, min(cfg.T, tokens_hint))
     tok = np.arange(n)
     t0 = time.perf_counter()
-    if cfg.fp8:
+    if cfg.per_tensor:
+        O.moe_forward_fp8_per_tensor(hb, lg, *fp8w, s_in, cfg.activation_scale, topk=cfg.topk,
+                                     renormalize=cfg.renormalize, activation=cfg.activation,
+                                     num_shared=cfg.num_shared, tokens=tok)
+    elif cfg.fp8:
         O.moe_forward_fp8(hb, lg, *fp8w, topk=cfg.topk, renormalize=cfg.renormalize,
                           activation=cfg.activation, num_shared=cfg.num_shared, tokens=tok)
     else:

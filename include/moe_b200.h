@@ -77,10 +77,14 @@ typedef enum {
 /* Weight / activation number format. */
 typedef enum {
   MOE_DTYPE_BF16 = 0,         /* bf16 weights and activations, fp32 accumulation */
-  MOE_DTYPE_FP8_BLOCK128 = 1  /* e4m3 weights with one fp32 scale per 128x128 block and
+  MOE_DTYPE_FP8_BLOCK128 = 1, /* e4m3 weights with one fp32 scale per 128x128 block and
                                  e4m3 activations with one fp32 scale per 1x128 group
                                  (FP8 W8A8, block_shape [128, 128]; sglang PR 26204
                                  section 1) */
+  MOE_DTYPE_FP8_PER_TENSOR = 2 /* e4m3 weights with one fp32 scale per expert matrix, e4m3
+                                   GEMM inputs with the static problem->input_scale and
+                                   problem->activation_scale (the per-tensor FP8 variant,
+                                   sglang PR 21321 sections 1-2); I and H multiples of 128 */
 } moe_wdtype_t;
 
 /* Bit flags of moe_problem_t.flags. */
@@ -105,6 +109,10 @@ typedef struct {
                            the MMA's M operand and its token rows N) or 128 (128-row token
                            tiles) */
   uint32_t flags;       /* MOE_FLAG_* */
+  float input_scale;      /* MOE_DTYPE_FP8_PER_TENSOR: static scale of the hidden rows,
+                             x_q = e4m3(x / input_scale); finite, > 0 (ignored otherwise) */
+  float activation_scale; /* MOE_DTYPE_FP8_PER_TENSOR: static scale of GEMM1's activation,
+                             a_q = e4m3(a / activation_scale); finite, > 0 (ignored otherwise) */
 } moe_problem_t;
 
 /* Byte offsets of the intermediates inside the caller's workspace (for inspection by
@@ -181,6 +189,15 @@ moe_status_t moe_prepare_weights(const moe_problem_t* problem, int32_t intermedi
                                  const void* w13_in, const void* w2_in, void* w13_out,
                                  void* w2_out, moe_stream_t stream);
 
+/* Per-tensor FP8 quantisation of bf16 weights (MOE_DTYPE_FP8_PER_TENSOR):
+ *   w        device bf16 [num_mats, rows, cols], rows * cols a multiple of 8, num_mats <= 65535;
+ *   codes    device e4m3 [num_mats, rows, cols];
+ *   scales   device fp32 [num_mats]: amax / 448 of each matrix (IEEE division; 1 if amax == 0).
+ * code = e4m3(w / scale), round to nearest even, saturating at 448. */
+moe_status_t moe_quantize_weights_fp8_per_tensor(const void* w, int64_t num_mats, int32_t rows,
+                                                 int32_t cols, void* codes, float* scales,
+                                                 moe_stream_t stream);
+
 /* Bytes of the prepared w13 (which = 0) or w2 (which = 1) for `problem` (host only), or
  * 0 for an invalid problem or `which`. */
 size_t moe_prepared_weights_bytes(const moe_problem_t* problem, int32_t which);
@@ -199,9 +216,9 @@ moe_status_t moe_quantize_weights_fp8(const void* w, int64_t num_mats, int32_t r
  *   hidden         device bf16 [T, H]
  *   router_logits  device fp32 [T, E_r] (finite values; NaN/Inf are not supported)
  *   w13, w2        device, prepared by moe_prepare_weights for this problem's layout
- *   w13_scale      FP8 only (else NULL): device fp32 [E, N1/128, H/128], checkpoint
- *                  (gate-first, un-interleaved) block order
- *   w2_scale       FP8 only (else NULL): device fp32 [E, H/128, I/128]
+ *   w13_scale      FP8 block-128: device fp32 [E, N1/128, H/128], checkpoint (gate-first,
+ *                  un-interleaved) block order; FP8 per-tensor: device fp32 [E]; else NULL
+ *   w2_scale       FP8 block-128: device fp32 [E, H/128, I/128]; per-tensor: [E]; else NULL
  *   out            device bf16 [T, H] (must not alias hidden)
  *   workspace      device, >= moe_workspace_size(problem) bytes, 256-byte aligned; one
  *                  workspace must not be used by two calls in flight at once.

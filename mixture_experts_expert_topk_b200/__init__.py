@@ -19,11 +19,13 @@ import torch
 
 from . import _capi
 from ._capi import (MOE_ACT_GELU_TANH, MOE_ACT_RELU2, MOE_ACT_SWIGLU, MOE_DTYPE_BF16, MOE_DTYPE_FP8_BLOCK128,
+                    MOE_DTYPE_FP8_PER_TENSOR,
                     MOE_FLAG_PDL, MoeError, Problem, check, lib)
 
 __all__ = [
     "MoeError", "Problem", "make_problem", "padded_intermediate", "workspace_layout",
-    "workspace_size", "new_workspace", "prepare_weights", "quantize_weights_fp8", "moe_forward",
+    "workspace_size", "new_workspace", "prepare_weights", "quantize_weights_fp8",
+    "quantize_weights_fp8_per_tensor", "moe_forward",
     "moe_forward_host", "stage_route", "stage_align", "stage_quant_act", "stage_gemm1",
     "stage_gemm2", "stage_combine", "device_status", "read_workspace", "lib", "check",
 ]
@@ -60,18 +62,30 @@ def _dev(t: torch.Tensor, name: str, dtype=None) -> torch.Tensor:
 
 def make_problem(T: int, H: int, num_routed: int, topk: int, intermediate: int, *,
                  renormalize: bool = True, activation="swiglu", num_shared: int = 0,
-                 fp8: bool = False, pdl: bool = True, block_m: int = 0) -> Problem:
-    """Problem description; ``intermediate`` must already be padded."""
+                 fp8=False, pdl: bool = True, block_m: int = 0, input_scale: float = 0.0,
+                 activation_scale: float = 0.0) -> Problem:
+    """Problem description; ``intermediate`` must already be padded. ``fp8``: False (bf16),
+    True or "block128" (e4m3, 128x128 weight blocks, 1x128 activation groups), or
+    "per_tensor" (e4m3, one scale per expert matrix and the static ``input_scale`` /
+    ``activation_scale``)."""
+    if fp8 == "per_tensor":
+        wdtype = MOE_DTYPE_FP8_PER_TENSOR
+    elif fp8 in (True, "block128"):
+        wdtype = MOE_DTYPE_FP8_BLOCK128
+    elif fp8 is False or fp8 is None:
+        wdtype = MOE_DTYPE_BF16
+    else:
+        raise ValueError(f"fp8 must be False, True/'block128' or 'per_tensor', got {fp8!r}")
     return Problem(num_tokens=T, hidden=H, num_routed=num_routed, num_shared=num_shared,
                    intermediate=intermediate, topk=topk, renormalize=int(bool(renormalize)),
-                   activation=_act(activation),
-                   wdtype=MOE_DTYPE_FP8_BLOCK128 if fp8 else MOE_DTYPE_BF16, block_m=block_m,
-                   flags=MOE_FLAG_PDL if pdl else 0)
+                   activation=_act(activation), wdtype=wdtype, block_m=block_m,
+                   flags=MOE_FLAG_PDL if pdl else 0, input_scale=float(input_scale),
+                   activation_scale=float(activation_scale))
 
 
-def padded_intermediate(intermediate: int, activation="swiglu", fp8: bool = False) -> int:
+def padded_intermediate(intermediate: int, activation="swiglu", fp8=False) -> int:
     v = lib().moe_padded_intermediate(intermediate, _act(activation),
-                                      MOE_DTYPE_FP8_BLOCK128 if fp8 else MOE_DTYPE_BF16)
+                                      MOE_DTYPE_FP8_BLOCK128 if fp8 else MOE_DTYPE_BF16)  # both FP8 kinds pad alike
     if v < 0:
         raise ValueError("invalid intermediate size or activation")
     return v
@@ -101,7 +115,7 @@ def prepare_weights(prob: Problem, w13: torch.Tensor, w2: torch.Tensor, intermed
     """Load-time padding + gate/up interleave (bf16, or e4m3 codes as uint8), in the layout
     the problem's GEMMs read: row-major [E, N1, H] / [E, H, I] for 128-row tiles, else the
     tiled layout (1-D tensors; ``.moe_intermediate`` records I for :func:`moe_forward`)."""
-    fp8 = prob.wdtype == MOE_DTYPE_FP8_BLOCK128
+    fp8 = prob.wdtype in (MOE_DTYPE_FP8_BLOCK128, MOE_DTYPE_FP8_PER_TENSOR)
     dt = torch.uint8 if fp8 else torch.bfloat16
     _dev(w13, "w13", dt)
     _dev(w2, "w2", dt)
@@ -126,6 +140,19 @@ def prepare_weights(prob: Problem, w13: torch.Tensor, w2: torch.Tensor, intermed
     return w13p, w2p
 
 
+def quantize_weights_fp8_per_tensor(w: torch.Tensor, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Per-matrix e4m3 quantisation of bf16 [..., rows, cols] weights: (codes uint8, scales
+    fp32 [...]) with scale = amax / 448 per matrix."""
+    _dev(w, "w", torch.bfloat16)
+    rows, cols = w.shape[-2], w.shape[-1]
+    mats = w.numel() // (rows * cols)
+    codes = torch.empty(w.shape, dtype=torch.uint8, device=w.device)
+    scales = torch.empty(tuple(w.shape[:-2]), dtype=torch.float32, device=w.device)
+    check(lib().moe_quantize_weights_fp8_per_tensor(_ptr(w), mats, rows, cols, _ptr(codes), _ptr(scales),
+                                                    _stream(stream)), "moe_quantize_weights_fp8_per_tensor")
+    return codes, scales
+
+
 def quantize_weights_fp8(w: torch.Tensor, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
     """Per-128x128-block e4m3 quantisation of bf16 [..., rows, cols] weights."""
     _dev(w, "w", torch.bfloat16)
@@ -140,7 +167,7 @@ def quantize_weights_fp8(w: torch.Tensor, stream=None) -> Tuple[torch.Tensor, to
 
 
 def _problem_from(hidden, router_logits, w2, topk, renormalize, activation_type, num_shared,
-                  fp8, pdl) -> Problem:
+                  fp8, pdl, input_scale=0.0, activation_scale=0.0) -> Problem:
     T, H = hidden.shape
     E_r = router_logits.shape[1]
     I = getattr(w2, "moe_intermediate", None)
@@ -149,7 +176,8 @@ def _problem_from(hidden, router_logits, w2, topk, renormalize, activation_type,
             raise ValueError("w2 must come from prepare_weights (or be [E, H, I] row-major)")
         I = w2.shape[2]
     return make_problem(T, H, E_r, topk, I, renormalize=renormalize,
-                        activation=activation_type, num_shared=num_shared, fp8=fp8, pdl=pdl)
+                        activation=activation_type, num_shared=num_shared, fp8=fp8, pdl=pdl,
+                        input_scale=input_scale, activation_scale=activation_scale)
 
 
 _WS_CACHE: Dict[tuple, torch.Tensor] = {}
@@ -169,20 +197,24 @@ def moe_forward(hidden: torch.Tensor, router_logits: torch.Tensor, w13: torch.Te
                 w2: torch.Tensor, topk: int, renormalize: bool, activation_type,
                 w13_scale: Optional[torch.Tensor] = None, w2_scale: Optional[torch.Tensor] = None,
                 num_shared: int = 0, *, workspace: Optional[torch.Tensor] = None,
-                out: Optional[torch.Tensor] = None, pdl: bool = True, stream=None) -> torch.Tensor:
+                out: Optional[torch.Tensor] = None, pdl: bool = True, stream=None,
+                input_scale: Optional[float] = None, activation_scale: Optional[float] = None) -> torch.Tensor:
     """Fused MoE layer forward on the current CUDA stream.
 
     ``hidden`` bf16 [T,H]; ``router_logits`` fp32 [T,E_r]; ``w13``/``w2`` prepared by
     :func:`prepare_weights` (bf16, or uint8 e4m3 codes with fp32 block scales
-    ``w13_scale`` [E, N1/128, H/128] and ``w2_scale`` [E, H/128, I/128]). Returns bf16 [T,H].
+    ``w13_scale`` [E, N1/128, H/128] and ``w2_scale`` [E, H/128, I/128]; with
+    ``input_scale`` and ``activation_scale`` given, per-tensor FP8 with ``w13_scale`` and
+    ``w2_scale`` fp32 [E]). Returns bf16 [T,H].
     """
-    fp8 = w13_scale is not None
+    per_tensor = input_scale is not None or activation_scale is not None
+    fp8 = "per_tensor" if per_tensor else w13_scale is not None
     _dev(hidden, "hidden", torch.bfloat16)
     _dev(router_logits, "router_logits", torch.float32)
     _dev(w13, "w13")
     _dev(w2, "w2")
     prob = _problem_from(hidden, router_logits, w2, topk, renormalize, activation_type,
-                         num_shared, fp8, pdl)
+                         num_shared, fp8, pdl, input_scale or 0.0, activation_scale or 0.0)
     if workspace is None:
         workspace = _workspace_for(prob, hidden.device)
     if out is None:
@@ -312,7 +344,12 @@ def read_workspace(prob: Problem, workspace: torch.Tensor) -> Dict[str, torch.Te
         "pair_to_row": view(L["pair_to_row"], P, torch.int32),
         "y": view(L["y"], rows * H, torch.float32).view(rows, H),
     }
-    if L["block_m"] == 16:
+    if prob.wdtype == MOE_DTYPE_FP8_PER_TENSOR:
+        # e4m3 codes in row-group order (128-column chunks per group, swizzled); flat views
+        out["act"] = view(L["act"], rows * I, torch.uint8)
+        out["xs"] = view(L["xs"], rows * H, torch.uint8)
+        out["group_info"] = view(L["group_info"], (rows // 16 + 1) * 2, torch.int32).view(-1, 2)
+    elif L["block_m"] == 16:
         # the swapped-operand GEMMs keep the activation and the permuted hidden rows in
         # row-group order (64-column chunks per group, swizzled); flat views
         act_cols = -(-I // 64) * 64

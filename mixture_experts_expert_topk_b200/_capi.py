@@ -23,6 +23,7 @@ MOE_ERR_DEVICE_TIMEOUT = 5
 MOE_ACT_SWIGLU = 0
 MOE_ACT_RELU2 = 1
 MOE_ACT_GELU_TANH = 2
+MOE_DTYPE_FP8_PER_TENSOR = 2
 MOE_DTYPE_BF16 = 0
 MOE_DTYPE_FP8_BLOCK128 = 1
 MOE_FLAG_PDL = 1
@@ -41,6 +42,8 @@ class Problem(ctypes.Structure):
         ("wdtype", ctypes.c_int32),
         ("block_m", ctypes.c_int32),
         ("flags", ctypes.c_uint32),
+        ("input_scale", ctypes.c_float),
+        ("activation_scale", ctypes.c_float),
     ]
 
 
@@ -76,6 +79,7 @@ SIGNATURES = {
     "moe_prepare_weights": (_I, [_P, _I, _V, _V, _V, _V, _V]),
     "moe_prepared_weights_bytes": (_S, [_P, _I]),
     "moe_quantize_weights_fp8": (_I, [_V, ctypes.c_int64, _I, _I, _V, _V, _V]),
+    "moe_quantize_weights_fp8_per_tensor": (_I, [_V, ctypes.c_int64, _I, _I, _V, _V, _V]),
     "moe_forward": (_I, [_P, _V, _V, _V, _V, _V, _V, _V, _V, _S, _V]),
     "moe_forward_routed": (_I, [_P, _V, _V, _V, _V, _V, _V, _V, _V, _V, _S, _V]),
     "moe_forward_host": (_I, [_P, _V, _V, _V, _V, _V, _V, _V, _V, _S, _V]),

@@ -49,7 +49,8 @@ bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr
 bool aligned4(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 struct Plan {
-  int T, H, Er, Es, E, I, topk, kk, bm, grp, N1, gated, fp8, renorm, act;
+  int T, H, Er, Es, E, I, topk, kk, bm, grp, N1, gated, fp8, pt, q8, renorm, act;
+  float in_scale, act_scale;  // per-tensor FP8 static scales
   long long P;
   int bn1, bn2;
   moe_workspace_layout_t lay;
@@ -66,12 +67,23 @@ moe_status_t make_plan(const moe_problem_t* p, Plan* pl) {
   if (p->renormalize != 0 && p->renormalize != 1) return MOE_ERR_INVALID_ARG;
   if (p->activation != MOE_ACT_SWIGLU && p->activation != MOE_ACT_RELU2 && p->activation != MOE_ACT_GELU_TANH)
     return MOE_ERR_INVALID_ARG;
-  if (p->wdtype != MOE_DTYPE_BF16 && p->wdtype != MOE_DTYPE_FP8_BLOCK128) return MOE_ERR_INVALID_ARG;
+  if (p->wdtype != MOE_DTYPE_BF16 && p->wdtype != MOE_DTYPE_FP8_BLOCK128 && p->wdtype != MOE_DTYPE_FP8_PER_TENSOR)
+    return MOE_ERR_INVALID_ARG;
   if (p->flags & ~MOE_FLAG_PDL) return MOE_ERR_INVALID_ARG;
   q.gated = p->activation != MOE_ACT_RELU2;
   q.fp8 = p->wdtype == MOE_DTYPE_FP8_BLOCK128;
+  q.pt = p->wdtype == MOE_DTYPE_FP8_PER_TENSOR;
+  q.q8 = q.fp8 || q.pt;
+  if (q.pt) {
+    // static scales: finite and positive
+    if (!(p->input_scale > 0.0f && p->input_scale < 3.0e38f) ||
+        !(p->activation_scale > 0.0f && p->activation_scale < 3.0e38f))
+      return MOE_ERR_INVALID_ARG;
+    q.in_scale = p->input_scale;
+    q.act_scale = p->activation_scale;
+  }
   // the intermediate size must already be padded (moe_padded_intermediate)
-  const int ialign = (q.fp8 || !q.gated) ? 128 : 16;
+  const int ialign = (q.q8 || !q.gated) ? 128 : 16;
   if (p->intermediate % ialign != 0) return MOE_ERR_INVALID_ARG;
   if (p->hidden % 128 != 0) return MOE_ERR_UNSUPPORTED;
   if (p->num_routed + p->num_shared > moe::kMaxExperts) return MOE_ERR_UNSUPPORTED;
@@ -94,6 +106,7 @@ moe_status_t make_plan(const moe_problem_t* p, Plan* pl) {
   // operand and row groups of up to 256 token rows as N. FP8, or block_m = 128: 128-row
   // token tiles.
   if (p->block_m == 16 && q.fp8) return MOE_ERR_UNSUPPORTED;
+  if (p->block_m == 128 && q.pt) return MOE_ERR_UNSUPPORTED;
   q.bm = p->block_m != 0 ? p->block_m : (q.fp8 ? 128 : 16);
   q.grp = q.bm == 16 ? kGroupRows : 0;
   q.renorm = p->renormalize;
@@ -129,13 +142,14 @@ moe_status_t make_plan(const moe_problem_t* p, Plan* pl) {
   L.chunk_hist = take(static_cast<size_t>(L.num_chunks) * q.E * 4);
   L.xq = take(q.fp8 ? T * H : 0);
   L.xq_scale = take(q.fp8 ? T * (H / 128) * 4 : 0);
-  // the swapped-operand GEMMs keep the activation in row-group order, 64-column chunks
-  const size_t act_cols = q.bm == 16 ? align_up(I, 64) : I;
-  L.act = take(rows * act_cols * 2);
+  // the swapped-operand GEMMs keep the activation in row-group order, 128-byte chunks (64
+  // bf16 or 128 e4m3 columns)
+  const size_t act_bytes = q.pt ? rows * I : rows * (q.bm == 16 ? align_up(I, 64) : I) * 2;
+  L.act = take(act_bytes);
   L.actq = take(q.fp8 ? rows * I : 0);
   L.act_scale = take(q.fp8 ? rows * (I / 128) * 4 : 0);
   L.y = take(rows * H * 4);
-  L.xs = take(q.bm == 16 ? rows * H * 2 : 0);
+  L.xs = take(q.bm == 16 ? rows * H * (q.pt ? 1 : 2) : 0);
   L.group_info = take(q.bm == 16 ? (rows / 16 + 1) * 8 : 0);
   L.io_hidden = take(T * H * 2);
   L.io_logits = take(T * static_cast<size_t>(q.Er) * 4);
@@ -290,10 +304,14 @@ moe_status_t run_gemm1(const Plan& pl_in, const void* hidden, const void* w13, c
   if (pl.bm == 16) {
     // tiled weights as the MMA's M operand, the token rows in row-group order (run_permute):
     // both operands load with bulk copies
-    moe::SwapOperands o;
+    moe::SwapOperands o{};
     o.w = w13;
     o.x = ws_ptr<void>(ws, L.xs);
-    o.out_chunks = (pl.I + 63) / 64;
+    o.out_chunks = pl.pt ? pl.I / 128 : (pl.I + 63) / 64;
+    o.fp8 = pl.pt;
+    o.w_scale = w13_scale;
+    o.in_scale = pl.in_scale;
+    o.act_scale = pl.act_scale;
     return cuda_status(moe::launch_gemm_swap(l, 0, o, s, b));
   }
   if (!pl.fp8) {
@@ -334,6 +352,10 @@ moe_status_t run_gemm1(const Plan& pl_in, const void* hidden, const void* w13, c
 moe_status_t run_permute(const Plan& pl, const void* hidden, void* ws, const Launch& l, int num_sms) {
   if (pl.bm != 16) return MOE_OK;
   const auto& L = pl.lay;
+  if (pl.pt)
+    return cuda_status(moe::launch_permute_quant_rows(
+        l, hidden, pl.H, ws_ptr<int>(ws, L.sorted_pair_ids), ws_ptr<int>(ws, L.num_blocks) + 1,
+        ws_ptr<int2>(ws, L.group_info), static_cast<int>(pl.P), pl.kk, pl.in_scale, ws_ptr<void>(ws, L.xs), num_sms));
   return cuda_status(moe::launch_permute_rows(l, hidden, pl.H, ws_ptr<int>(ws, L.sorted_pair_ids),
                                               ws_ptr<int>(ws, L.num_blocks) + 1, ws_ptr<int2>(ws, L.group_info),
                                               static_cast<int>(pl.P), pl.kk, ws_ptr<void>(ws, L.xs), num_sms));
@@ -360,10 +382,13 @@ moe_status_t run_gemm2(const Plan& pl_in, const void* w2, const float* w2_scale,
   CUtensorMap ta, tb;
   const uint64_t rows = static_cast<uint64_t>(L.max_rows);
   if (pl.bm == 16) {
-    moe::SwapOperands o;
+    moe::SwapOperands o{};
     o.w = w2;
     o.x = ws_ptr<void>(ws, L.act);
     o.out_chunks = 0;
+    o.fp8 = pl.pt;
+    o.w_scale = w2_scale;
+    o.in_scale = pl.act_scale;
     return cuda_status(moe::launch_gemm_swap(l, 1, o, s, b));
   }
   if (!pl.fp8) {
@@ -434,7 +459,7 @@ moe_status_t forward_device(const Plan& pl, const moe_problem_t* p, const void* 
 
 moe_status_t check_weights(const Plan& pl, const void* w13, const void* w2, const float* s13, const float* s2) {
   if (!aligned16(w13) || !aligned16(w2)) return MOE_ERR_INVALID_ARG;
-  if (pl.fp8 && (!aligned4(s13) || !aligned4(s2))) return MOE_ERR_INVALID_ARG;
+  if (pl.q8 && (!aligned4(s13) || !aligned4(s2))) return MOE_ERR_INVALID_ARG;
   return MOE_OK;
 }
 
@@ -460,8 +485,10 @@ MOE_API moe_status_t moe_check_problem(const moe_problem_t* problem) {
 MOE_API int32_t moe_padded_intermediate(int32_t intermediate, int32_t activation, int32_t wdtype) {
   if (intermediate <= 0 || intermediate > (1 << 20)) return -1;
   if (activation != MOE_ACT_SWIGLU && activation != MOE_ACT_RELU2 && activation != MOE_ACT_GELU_TANH) return -1;
-  if (wdtype != MOE_DTYPE_BF16 && wdtype != MOE_DTYPE_FP8_BLOCK128) return -1;
-  const int a = (wdtype == MOE_DTYPE_FP8_BLOCK128 || activation == MOE_ACT_RELU2) ? 128 : 16;
+  if (wdtype != MOE_DTYPE_BF16 && wdtype != MOE_DTYPE_FP8_BLOCK128 && wdtype != MOE_DTYPE_FP8_PER_TENSOR) return -1;
+  const int a = (wdtype == MOE_DTYPE_FP8_BLOCK128 || wdtype == MOE_DTYPE_FP8_PER_TENSOR || activation == MOE_ACT_RELU2)
+                    ? 128
+                    : 16;
   return (intermediate + a - 1) / a * a;
 }
 
@@ -485,10 +512,10 @@ MOE_API moe_status_t moe_prepare_weights(const moe_problem_t* problem, int32_t i
   moe_status_t st = make_plan(problem, &pl);  // num_tokens plays no part in weight preparation
   if (st != MOE_OK) return st;
   if (moe_padded_intermediate(intermediate_in, pl.act, problem->wdtype) != pl.I) return MOE_ERR_INVALID_ARG;
-  if (pl.fp8 && intermediate_in != pl.I) return MOE_ERR_INVALID_ARG;
+  if (pl.q8 && intermediate_in != pl.I) return MOE_ERR_INVALID_ARG;
   if (!aligned16(w13_in) || !aligned16(w13_out) || w2_in == nullptr || w2_out == nullptr)
     return MOE_ERR_INVALID_ARG;
-  const int elt = pl.fp8 ? 1 : 2;
+  const int elt = pl.q8 ? 1 : 2;
   if ((reinterpret_cast<uintptr_t>(w2_in) | reinterpret_cast<uintptr_t>(w2_out)) & (elt - 1))
     return MOE_ERR_INVALID_ARG;
   int sms = 0;
@@ -496,6 +523,12 @@ MOE_API moe_status_t moe_prepare_weights(const moe_problem_t* problem, int32_t i
   if (st != MOE_OK) return st;
   const Launch l = launch_of(problem, stream);
   cudaError_t e;
+  if (pl.pt) {
+    // e4m3 codes, tiled for the swapped-operand GEMMs
+    e = moe::launch_tile_weights_u8(l, 0, w13_in, w13_out, pl.E, pl.H, pl.I, pl.gated);
+    if (e == cudaSuccess) e = moe::launch_tile_weights_u8(l, 1, w2_in, w2_out, pl.E, pl.H, pl.I, pl.gated);
+    return cuda_status(e);
+  }
   if (pl.bm == 16) {
     // the swapped-operand GEMMs read the weights tiled
     e = moe::launch_tile_weights(l, 0, w13_in, w13_out, pl.E, pl.H, intermediate_in, pl.I, pl.gated);
@@ -510,6 +543,8 @@ MOE_API moe_status_t moe_prepare_weights(const moe_problem_t* problem, int32_t i
 MOE_API size_t moe_prepared_weights_bytes(const moe_problem_t* problem, int32_t which) {
   Plan pl;
   if (make_plan(problem, &pl) != MOE_OK || (which != 0 && which != 1)) return 0;
+  if (pl.pt)
+    return which == 0 ? moe::tiled_weight_bytes_u8(pl.E, pl.N1, pl.H) : moe::tiled_weight_bytes_u8(pl.E, pl.H, pl.I);
   if (pl.bm == 16)
     return which == 0 ? moe::tiled_weight_bytes(pl.E, pl.N1, pl.H) : moe::tiled_weight_bytes(pl.E, pl.H, pl.I);
   const size_t elt = pl.fp8 ? 1 : 2;
@@ -529,6 +564,22 @@ MOE_API moe_status_t moe_quantize_weights_fp8(const void* w, int64_t num_mats, i
   l.stream = reinterpret_cast<cudaStream_t>(stream);
   l.pdl = false;
   return cuda_status(moe::launch_quant_weights(l, w, num_mats, rows, cols, codes, scales));
+}
+
+MOE_API moe_status_t moe_quantize_weights_fp8_per_tensor(const void* w, int64_t num_mats, int32_t rows, int32_t cols,
+                                                         void* codes, float* scales, moe_stream_t stream) {
+  if (num_mats < 0 || num_mats > 65535 || rows <= 0 || cols <= 0) return MOE_ERR_INVALID_ARG;
+  const int64_t elems = static_cast<int64_t>(rows) * cols;
+  if (elems % 8 != 0) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(w) || !aligned16(codes) || !aligned4(scales)) return MOE_ERR_INVALID_ARG;
+  if (num_mats == 0) return MOE_OK;
+  int sms = 0;
+  const moe_status_t st = device_sms(&sms);
+  if (st != MOE_OK) return st;
+  Launch l;
+  l.stream = reinterpret_cast<cudaStream_t>(stream);
+  l.pdl = false;
+  return cuda_status(moe::launch_quant_weights_per_tensor(l, w, num_mats, elems, codes, scales));
 }
 
 MOE_API moe_status_t moe_forward(const moe_problem_t* problem, const void* hidden, const float* router_logits,
@@ -655,7 +706,7 @@ MOE_API moe_status_t moe_stage_gemm1(const moe_problem_t* problem, const void* h
   int sms = 0;
   moe_status_t st = make_plan(problem, &pl);
   if (st != MOE_OK || pl.T == 0) return st;  // T == 0: nothing to do, pointers unused
-  if (!aligned16(hidden) || !aligned16(w13) || (pl.fp8 && !aligned4(w13_scale))) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(hidden) || !aligned16(w13) || (pl.q8 && !aligned4(w13_scale))) return MOE_ERR_INVALID_ARG;
   st = prologue(problem, workspace, workspace_bytes, &pl, &sms);
   if (st != MOE_OK || pl.T == 0) return st;
   return run_gemm1(pl, hidden, w13, w13_scale, workspace, launch_of(problem, stream), sms);
@@ -667,7 +718,7 @@ MOE_API moe_status_t moe_stage_gemm2(const moe_problem_t* problem, const void* w
   int sms = 0;
   moe_status_t st = make_plan(problem, &pl);
   if (st != MOE_OK || pl.T == 0) return st;  // T == 0: nothing to do, pointers unused
-  if (!aligned16(w2) || (pl.fp8 && !aligned4(w2_scale))) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(w2) || (pl.q8 && !aligned4(w2_scale))) return MOE_ERR_INVALID_ARG;
   st = prologue(problem, workspace, workspace_bytes, &pl, &sms);
   if (st != MOE_OK || pl.T == 0) return st;
   return run_gemm2(pl, w2, w2_scale, workspace, launch_of(problem, stream), sms);

@@ -32,12 +32,22 @@
 // One K step of a tile moves kc chunks of W (kc * 16 KB, one copy) and of X (kc * n * 128
 // bytes, one copy), kc = 1..4 chosen from n so that a step holds 48 to 72 KB.
 //
+// Per-tensor FP8 (e4m3 operands, one fp32 scale per tensor): the same tiles and copies
+// with tcgen05.mma kind::f8f6f4 (a 128-byte chunk is 128 elements of K, four K=32 MMAs).
+// GEMM1's epilogue dequantises with w13_scale[e] * input_scale before the activation and
+// writes e4m3(activation * (1 / activation_scale)); GEMM2's multiplies by activation_scale
+// * w2_scale[e] and the routing weight ("FlashInfer TRTLLM-Gen MoE kernel optimisation:
+// NemotronH support", section 2: g1_alphas = w13_scale * input_scale, requantised by
+// 1.0 / activation_scale). The kernel is compiled once per operand type.
+//
 // One persistent CTA per SM, 7 warps:
 //   warp 0      scheduler (tiles from a global atomic counter, published to the other
 //               roles through a shared-memory ring) and W copies;
 //   warp 6      X copies;
 //   warp 1      TMEM allocator and MMA issuer;
 //   warps 2-5   epilogue (TMEM lane quadrant = warp % 4).
+#include <cuda_fp8.h>
+
 #include "moe_device.cuh"
 #include "moe_internal.h"
 
@@ -86,6 +96,9 @@ struct Args {
   const float* topk_w;
   int* tile_counter;       // [2]: next tile, CTAs finished; both 0 between launches
   int* status;
+  const float* w_scale;    // FP8: per-expert weight scales [E]
+  float in_scale;          // FP8 GEMM1: input scale; GEMM2: activation scale (the X scale)
+  float act_inv;           // FP8 GEMM1: 1 / activation scale (requantisation of the output)
 };
 
 // K chunks per step for a group of n rows: steps of 48 to 72 KB.
@@ -148,6 +161,7 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
       : "memory");
 }
 
+template <bool kFp8>
 __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -294,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
         if (!mbar_wait(tempty0 + 8 * acc, ((it >> 1) & 1) ^ 1u, abort_flag, a.status, kSiteTmemEmpty)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * kNMax;
-        const uint32_t idesc = idesc_bf16(kMW, n);
+        const uint32_t idesc = kFp8 ? idesc_e4m3(kMW, n) : idesc_bf16(kMW, n);
         bool ok = true;
         for (int c0 = 0; c0 < a.k_chunks; c0 += kc, ++ks) {
           const int kcs = min(kc, a.k_chunks - c0);
@@ -309,10 +323,17 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
           const uint32_t a_lo = umma_desc_lo(base);
           const uint32_t b_lo = a_lo + static_cast<uint32_t>(kcs) * (kTileW >> 4);
           const uint32_t b_step = static_cast<uint32_t>(n) * (kChunkBytes >> 4);
-          umma_bf16_chunk(d_tmem, a_lo, b_lo, idesc, c0 != 0);
+          if (kFp8) {
+            umma_e4m3_chunk(d_tmem, a_lo, b_lo, idesc, c0 != 0);
 #pragma unroll
-          for (int c = 1; c < 4; ++c)
-            if (c < kcs) umma_bf16_chunk(d_tmem, a_lo + c * (kTileW >> 4), b_lo + c * b_step, idesc, 1u);
+            for (int c = 1; c < 4; ++c)
+              if (c < kcs) umma_e4m3_chunk(d_tmem, a_lo + c * (kTileW >> 4), b_lo + c * b_step, idesc, 1u);
+          } else {
+            umma_bf16_chunk(d_tmem, a_lo, b_lo, idesc, c0 != 0);
+#pragma unroll
+            for (int c = 1; c < 4; ++c)
+              if (c < kcs) umma_bf16_chunk(d_tmem, a_lo + c * (kTileW >> 4), b_lo + c * b_step, idesc, 1u);
+          }
           umma_commit(empty0 + 8 * (ks % kSlots));  // arrives once these MMAs have read the step
         }
         if (!ok) break;
@@ -341,7 +362,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
       const int n = __shfl_sync(0xffffffffu, t.y, 0);
       if (!ok || n == 0) break;
       const int x_row = __shfl_sync(0xffffffffu, t.x, 0);
+      const int expert = __shfl_sync(0xffffffffu, t.z, 0);
       const int mt = __shfl_sync(0xffffffffu, t.w, 0);
+      // FP8: the accumulator's dequantisation scale (GEMM1: before the activation)
+      const float dq = kFp8 ? __ldg(a.w_scale + expert) * a.in_scale : 1.0f;
       // GEMM2: routing weights of the group's tokens (token 32 b + lane in wreg[b]),
       // loaded while the main loop still runs
       float wreg[kNMax / 32];
@@ -358,11 +382,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
       if (!__all_sync(0xffffffffu, got)) break;  // leave warp-uniformly (tcgen05.ld is .aligned)
       tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * kNMax;
-      // GEMM1: this lane's activation feature f lies in K chunk f / 64 of the activation;
-      // byte (f % 64) * 2 of a 128-byte chunk row sits in 16-byte piece ((f % 64) / 8)
-      // ^ (row % 8)
+      // GEMM1: this lane's activation feature f lies in K chunk f / 64 (bf16) or f / 128
+      // (e4m3) of the activation; byte b of a 128-byte chunk row sits in 16-byte piece
+      // (b / 16) ^ (row % 8)
       const int f = gated ? mt * (kMW / 2) + q * 16 + (lane >> 1) : mt * kMW + q * 32 + lane;
-      const int fc = f >> 6, fo = f & 63;
+      const int fc = kFp8 ? f >> 7 : f >> 6;
+      const int fo = kFp8 ? f & 127 : (f & 63) * 2;  // byte offset in the chunk row
       uint8_t* act_grp = static_cast<uint8_t*>(a.out) + static_cast<size_t>(x_row) * a.out_chunks * kChunkBytes +
                          static_cast<size_t>(fc) * n * kChunkBytes;
       for (int c0 = 0; c0 < n; c0 += 32) {
@@ -391,7 +416,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             if (j == 16 && !full) break;
-            const float w = __shfl_sync(0xffffffffu, wl, j);
+            const float w = __shfl_sync(0xffffffffu, wl, j) * dq;
             y[static_cast<size_t>(j) * a.out_cols] = __uint_as_float(v[j]) * w;
           }
         } else if (!gated) {
@@ -399,9 +424,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
           for (int j = 0; j < 32; ++j) {
             if (j == 16 && !full) break;
             const int row = c0 + j;
-            const float z = fmaxf(__uint_as_float(v[j]), 0.f);
-            *reinterpret_cast<__nv_bfloat16*>(act_grp + row * kChunkBytes + ((((fo >> 3) ^ row) & 7) << 4) +
-                                              (fo & 7) * 2) = __float2bfloat16_rn(z * z);
+            const float z = fmaxf(__uint_as_float(v[j]) * dq, 0.f);
+            uint8_t* dst = act_grp + row * kChunkBytes + ((((fo >> 4) ^ row) & 7) << 4) + (fo & 15);
+            if (kFp8)
+              *dst = __nv_cvt_float_to_fp8(z * z * a.act_inv, __NV_SATFINITE, __NV_E4M3);
+            else
+              *reinterpret_cast<__nv_bfloat16*>(dst) = __float2bfloat16_rn(z * z);
           }
         } else {
           // lane pair (2m, 2m+1) = (gate, up) of feature m. The even lane finishes tokens
@@ -409,15 +437,20 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
           // it needs, so every lane evaluates silu on 16 tokens.
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            const float mine_lo = __uint_as_float(v[j]);       // even: gate_j; odd: up_j
-            const float mine_hi = __uint_as_float(v[16 + j]);  // even: gate_{16+j}; odd: up_{16+j}
+            const float mine_lo = __uint_as_float(v[j]) * dq;       // even: gate_j; odd: up_j
+            const float mine_hi = __uint_as_float(v[16 + j]) * dq;  // even: gate_{16+j}; odd: up_{16+j}
             const float other = __shfl_xor_sync(0xffffffffu, odd ? mine_lo : mine_hi, 1);
             const float g = odd ? other : mine_lo;
             const float u = odd ? mine_hi : other;
             const int row = c0 + (odd ? 16 + j : j);
-            if (!odd || full)
-              *reinterpret_cast<__nv_bfloat16*>(act_grp + row * kChunkBytes + ((((fo >> 3) ^ row) & 7) << 4) +
-                                                (fo & 7) * 2) = __float2bfloat16_rn(gate_act(g, a.activation) * u);
+            if (!odd || full) {
+              const float h = gate_act(g, a.activation) * u;
+              uint8_t* dst = act_grp + row * kChunkBytes + ((((fo >> 4) ^ row) & 7) << 4) + (fo & 15);
+              if (kFp8)
+                *dst = __nv_cvt_float_to_fp8(h * a.act_inv, __NV_SATFINITE, __NV_E4M3);
+              else
+                *reinterpret_cast<__nv_bfloat16*>(dst) = __float2bfloat16_rn(h);
+            }
           }
         }
       }
@@ -443,7 +476,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
   }
 }
 
-bool g_attr_set[64] = {};
+bool g_attr_set[2][64] = {};
 
 }  // namespace
 
@@ -453,16 +486,19 @@ cudaError_t launch_gemm_swap(const Launch& l, int mode, const SwapOperands& o, c
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!g_attr_set[dev]) {
-    err = cudaFuncSetAttribute(gemm_swap_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  const int fi = o.fp8 ? 1 : 0;
+  if (!g_attr_set[fi][dev]) {
+    err = cudaFuncSetAttribute(o.fp8 ? gemm_swap_kernel<true> : gemm_swap_kernel<false>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (err != cudaSuccess) return err;
-    g_attr_set[dev] = true;
+    g_attr_set[fi][dev] = true;
   }
   if ((reinterpret_cast<uintptr_t>(o.w) | reinterpret_cast<uintptr_t>(o.x)) & 15u) return cudaErrorInvalidValue;
   Args a;
   a.mode = mode;
   a.m_tiles = (s.N + kMW - 1) / kMW;
-  a.k_chunks = (s.K + 63) / 64;
+  const int chunk_elems = o.fp8 ? 128 : 64;  // elements of K in a 128-byte chunk
+  a.k_chunks = (s.K + chunk_elems - 1) / chunk_elems;
   a.k_total = s.k_total;
   a.num_pairs = s.num_pairs;
   a.activation = s.activation;
@@ -477,10 +513,13 @@ cudaError_t launch_gemm_swap(const Launch& l, int mode, const SwapOperands& o, c
   a.topk_w = b.topk_w;
   a.tile_counter = b.tile_counter;
   a.status = b.status;
+  a.w_scale = o.w_scale;
+  a.in_scale = o.in_scale;
+  a.act_inv = o.act_scale > 0.f ? 1.0f / o.act_scale : 0.f;
   cudaLaunchConfig_t cfg;
   cudaLaunchAttribute attr[1];
   make_launch_config(&cfg, attr, l, dim3(s.num_sms), dim3(kThreads), kSmemBytes);
-  return cudaLaunchKernelEx(&cfg, gemm_swap_kernel, a);
+  return cudaLaunchKernelEx(&cfg, o.fp8 ? gemm_swap_kernel<true> : gemm_swap_kernel<false>, a);
 }
 
 }  // namespace moe

@@ -243,7 +243,8 @@ __device__ __forceinline__ void umma_e4m3(uint32_t d_tmem, uint64_t adesc, uint6
 __device__ __forceinline__ uint32_t umma_desc_lo(uint32_t saddr) { return ((saddr & 0x3FFFFu) >> 4) | (1u << 16); }
 constexpr uint32_t kUmmaDescHi = (1024u >> 4) | (1u << (46 - 32)) | (2u << (61 - 32));
 
-// One 128-byte K chunk of bf16 operands: four K=16 MMAs, each step advancing both
+// One 128-byte K chunk of operands: four MMAs (kind::f16: bf16, K=16; kind::f8f6f4:
+// e4m3, K=32), each step advancing both
 // descriptors by 32 bytes (+2 in the encoded start address). The first MMA accumulates
 // into D when `accumulate` is nonzero, the other three always do. The descriptors are
 // assembled inside the asm block from their low words, so the issuing thread spends a few
@@ -263,6 +264,24 @@ __device__ __forceinline__ void umma_bf16_chunk(uint32_t d_tmem, uint32_t a_lo, 
       "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, q;\n\t"
       "add.u32 al, %1, 6;\n\tadd.u32 bl, %2, 6;\n\tmov.b64 a, {al, %5};\n\tmov.b64 b, {bl, %5};\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, q;\n\t}" ::"r"(d_tmem),
+      "r"(a_lo), "r"(b_lo), "r"(idesc), "r"(accumulate), "n"(kUmmaDescHi)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_e4m3_chunk(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t idesc,
+                                                uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t.reg .b32 al, bl;\n\t.reg .b64 a, b;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.eq.b32 q, %4, %4;\n\t"
+      "mov.b64 a, {%1, %5};\n\tmov.b64 b, {%2, %5};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], a, b, %3, p;\n\t"
+      "add.u32 al, %1, 2;\n\tadd.u32 bl, %2, 2;\n\tmov.b64 a, {al, %5};\n\tmov.b64 b, {bl, %5};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], a, b, %3, q;\n\t"
+      "add.u32 al, %1, 4;\n\tadd.u32 bl, %2, 4;\n\tmov.b64 a, {al, %5};\n\tmov.b64 b, {bl, %5};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], a, b, %3, q;\n\t"
+      "add.u32 al, %1, 6;\n\tadd.u32 bl, %2, 6;\n\tmov.b64 a, {al, %5};\n\tmov.b64 b, {bl, %5};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], a, b, %3, q;\n\t}" ::"r"(d_tmem),
       "r"(a_lo), "r"(b_lo), "r"(idesc), "r"(accumulate), "n"(kUmmaDescHi)
       : "memory");
 }

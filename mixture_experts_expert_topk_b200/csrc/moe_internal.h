@@ -49,6 +49,11 @@ cudaError_t launch_align(const Launch& l, const int* topk_ids, int P, int E, int
 cudaError_t launch_permute_rows(const Launch& l, const void* hidden, int H, const int* sorted_pair_ids,
                                 const int* num_groups, const int2* group_info, int P, int k_total, void* xs,
                                 int num_sms);
+// As launch_permute_rows with every element quantised to e4m3(x * fp32(1 / input_scale)):
+// H bytes per row, 128-byte chunks of 128 elements.
+cudaError_t launch_permute_quant_rows(const Launch& l, const void* hidden, int H, const int* sorted_pair_ids,
+                                      const int* num_groups, const int2* group_info, int P, int k_total,
+                                      float input_scale, void* xs, int num_sms);
 
 // ---- GEMMs (gemm_bf16.cu, gemm_fp8.cu) ----
 struct GemmShape {
@@ -86,6 +91,12 @@ struct SwapOperands {
   const void* w;
   const void* x;
   int out_chunks;
+  // per-tensor FP8 (e4m3 operands): fp8 = 1, w_scale [E]; in_scale = the X operand's scale
+  // (GEMM1: the input scale; GEMM2: the activation scale); act_scale = GEMM1's output
+  // requantisation scale (the activation scale)
+  int fp8;
+  const float* w_scale;
+  float in_scale, act_scale;
 };
 // N tile for a GEMM with N output columns, given an estimate of the number of 128-row
 // tiles and the SM count (0 if no multiple of 32 divides N).
@@ -123,5 +134,14 @@ cudaError_t launch_prepare_w2(const Launch& l, const void* in, void* out, int E,
 size_t tiled_weight_bytes(int E, int rows, int K);
 cudaError_t launch_tile_weights(const Launch& l, int which, const void* in, void* out, int E, int H, int I_in,
                                 int I_pad, int gated);
+// The same for e4m3 codes (1 byte, 128 elements per 128-byte chunk row): tiles of 128 rows x
+// 128 columns; tiled_weight_bytes_u8 gives the size.
+size_t tiled_weight_bytes_u8(int E, int rows, int K);
+cudaError_t launch_tile_weights_u8(const Launch& l, int which, const void* in, void* out, int E, int H, int I,
+                                   int gated);
+// Per-tensor FP8 weight quantisation of num_mats bf16 [rows, cols] matrices: scale = amax
+// / 448 per matrix (1 for all zeros), codes = e4m3(w / scale).
+cudaError_t launch_quant_weights_per_tensor(const Launch& l, const void* w, int64_t num_mats, int64_t mat_elems,
+                                            void* codes, float* scales);
 
 }  // namespace moe

@@ -10,6 +10,8 @@
 // A CTA copies a 32-row slice of a row group; each warp two rows at a time, each lane with
 // sixteen 16-byte loads of the hidden rows in flight (coalesced) before writing them to
 // their chunk rows.
+#include <cuda_fp8.h>
+
 #include "moe_device.cuh"
 #include "moe_internal.h"
 
@@ -71,7 +73,88 @@ __global__ void __launch_bounds__(kThreads)
   }
 }
 
+// Per-tensor FP8: the same row-group order with each element quantised on the way,
+// e4m3(x * inv_scale), inv_scale = fp32(1 / input_scale) (the per-tensor variant scales
+// by the reciprocal: "FlashInfer TRTLLM-Gen MoE kernel optimisation: NemotronH support",
+// section 2), round to nearest, saturating at 448; a chunk is 128 elements (128 bytes).
+// Piece p of a row is elements [16p, 16p + 16); a warp converts two rows at a time, each
+// lane four pieces per row, all loads issued before the conversions.
+constexpr int kQPieces = 4;
+__global__ void __launch_bounds__(kThreads)
+    permute_quant_rows_kernel(const uint4* __restrict__ hidden, int H, const int* __restrict__ sorted_pair_ids,
+                              const int* __restrict__ num_groups, const int2* __restrict__ group_info, int P,
+                              int k_total, float inv_scale, uint8_t* __restrict__ xs) {
+  griddep_wait();
+  griddep_launch_dependents();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int G = *num_groups;
+  const int pieces = H / 16;  // 16 elements: 32 bytes in, 16 bytes out
+  for (int g = blockIdx.x; g < G; g += gridDim.x) {
+    const int2 gi = group_info[g];
+    const int x_row = gi.x, n = gi.y >> 16;
+    uint8_t* base = xs + static_cast<size_t>(x_row) * H;
+    for (int j0 = kRowsPerCta * blockIdx.y + kRowsPerStep * warp; j0 < min(n, kRowsPerCta * (blockIdx.y + 1));
+         j0 += kRowsPerStep * (kThreads / 32)) {
+      const uint4* src[kRowsPerStep];
+#pragma unroll
+      for (int r = 0; r < kRowsPerStep; ++r) {
+        const int pid = j0 + r < n ? sorted_pair_ids[x_row + j0 + r] : P;
+        src[r] = pid < P ? hidden + static_cast<size_t>(pid / k_total) * (H / 8) : nullptr;
+      }
+      for (int p0 = lane; p0 < pieces; p0 += 32 * kQPieces) {
+        uint4 in[kRowsPerStep][kQPieces][2];
+#pragma unroll
+        for (int r = 0; r < kRowsPerStep; ++r)
+#pragma unroll
+          for (int i = 0; i < kQPieces; ++i) {
+            const int p = p0 + 32 * i;
+            const bool ok = src[r] != nullptr && p < pieces;
+            in[r][i][0] = ok ? __ldg(src[r] + 2 * p) : make_uint4(0u, 0u, 0u, 0u);
+            in[r][i][1] = ok ? __ldg(src[r] + 2 * p + 1) : make_uint4(0u, 0u, 0u, 0u);
+          }
+#pragma unroll
+        for (int r = 0; r < kRowsPerStep; ++r) {
+          const int j = j0 + r;
+          if (j >= n) continue;
+#pragma unroll
+          for (int i = 0; i < kQPieces; ++i) {
+            const int p = p0 + 32 * i;
+            if (p >= pieces) continue;
+            const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(in[r][i]);
+            uint32_t o[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const float2 a = __bfloat1622float2(h2[2 * k]);
+              const float2 b = __bfloat1622float2(h2[2 * k + 1]);
+              const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a.x * inv_scale, a.y * inv_scale),
+                                                           __NV_SATFINITE, __NV_E4M3);
+              const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(b.x * inv_scale, b.y * inv_scale),
+                                                           __NV_SATFINITE, __NV_E4M3);
+              o[k] = lo | (hi << 16);
+            }
+            const int c = p >> 3, q = p & 7;
+            *reinterpret_cast<uint4*>(base + static_cast<size_t>(c) * n * 128 + j * 128 + ((q ^ (j & 7)) << 4)) =
+                make_uint4(o[0], o[1], o[2], o[3]);
+          }
+        }
+      }
+    }
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_permute_quant_rows(const Launch& l, const void* hidden, int H, const int* sorted_pair_ids,
+                                      const int* num_groups, const int2* group_info, int P, int k_total,
+                                      float input_scale, void* xs, int num_sms) {
+  if (H % 128 != 0) return cudaErrorInvalidValue;
+  cudaLaunchConfig_t cfg;
+  cudaLaunchAttribute attr[1];
+  make_launch_config(&cfg, attr, l, dim3(2 * num_sms, 256 / kRowsPerCta), dim3(kThreads), 0);
+  const float inv_scale = 1.0f / input_scale;  // IEEE fp32 division on the host
+  return cudaLaunchKernelEx(&cfg, permute_quant_rows_kernel, static_cast<const uint4*>(hidden), H, sorted_pair_ids,
+                            num_groups, group_info, P, k_total, inv_scale, static_cast<uint8_t*>(xs));
+}
 
 cudaError_t launch_permute_rows(const Launch& l, const void* hidden, int H, const int* sorted_pair_ids,
                                 const int* num_groups, const int2* group_info, int P, int k_total, void* xs,

@@ -101,7 +101,55 @@ __global__ void tile_weights_kernel(const uint16_t* __restrict__ in, uint4* __re
   }
 }
 
+// The tiled layout for e4m3 codes: a 128-byte chunk row holds 128 elements, so tile
+// (e, m, c) covers rows [128m, 128m + 128) and columns [128c, 128c + 128). FP8 requires
+// I == I_in (a multiple of 128): only the gate/up interleave of w13 moves rows.
+__global__ void tile_weights_u8_kernel(const uint4* __restrict__ in, uint4* __restrict__ out, long long pieces,
+                                       int which, int rows, int MT, int KC, int K, int I, int gated) {
+  griddep_wait();
+  for (long long o = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; o < pieces;
+       o += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long t = o >> 10;
+    const int rr = static_cast<int>((o >> 3) & 127);
+    const int q = static_cast<int>(o & 7) ^ (rr & 7);
+    const int c = static_cast<int>(t % KC);
+    const long long tm = t / KC;
+    const int m = static_cast<int>(tm % MT);
+    const long long e = tm / MT;
+    const int r = m * 128 + rr;
+    const int k0 = c * 128 + q * 16;
+    long long src = -1;
+    if (r < rows) {
+      if (which == 0 && gated) {
+        const int j = r >> 1, half = r & 1;
+        src = e * 2LL * I + static_cast<long long>(half) * I + j;
+      } else {
+        src = e * static_cast<long long>(rows) + r;
+      }
+    }
+    out[o] = (src >= 0 && k0 < K) ? in[(src * K + k0) / 16] : make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
 }  // namespace
+
+size_t tiled_weight_bytes_u8(int E, int rows, int K) {
+  return static_cast<size_t>(E) * ((rows + 127) / 128) * ((K + 127) / 128) * 16384;
+}
+
+cudaError_t launch_tile_weights_u8(const Launch& l, int which, const void* in, void* out, int E, int H, int I,
+                                   int gated) {
+  const int rows = which == 0 ? (gated ? 2 * I : I) : H;
+  const int K = which == 0 ? H : I;
+  if (K % 16 != 0) return cudaErrorInvalidValue;
+  const int MT = (rows + 127) / 128, KC = (K + 127) / 128;
+  const long long pieces = static_cast<long long>(tiled_weight_bytes_u8(E, rows, K) / 16);
+  cudaLaunchConfig_t cfg;
+  cudaLaunchAttribute attr[1];
+  make_launch_config(&cfg, attr, l, dim3(4096), dim3(256), 0);
+  return cudaLaunchKernelEx(&cfg, tile_weights_u8_kernel, static_cast<const uint4*>(in), static_cast<uint4*>(out),
+                            pieces, which, rows, MT, KC, K, I, gated);
+}
 
 size_t tiled_weight_bytes(int E, int rows, int K) {
   return static_cast<size_t>(E) * ((rows + 127) / 128) * ((K + 63) / 64) * 16384;

@@ -10,6 +10,8 @@
 // precision, so the codes and scales are compared bit for bit.
 #include <cuda_fp8.h>
 
+#include <algorithm>
+
 #include "moe_device.cuh"
 #include "moe_internal.h"
 
@@ -94,7 +96,81 @@ __global__ void __launch_bounds__(256)
   if (threadIdx.x == 0) scale[blk] = s;
 }
 
+// Per-tensor weights ("FlashInfer TRTLLM-Gen MoE kernel optimisation: NemotronH support",
+// section 1: the per-tensor FP8 variant, one fp32 scale per weight tensor). Pass 1: amax
+// of each matrix into amax_bits[mat] (non-negative floats order like their bit patterns,
+// so an integer max is a float max); pass 2: scale = amax / 448 (1 for all zeros) and
+// codes; pass 3: the scales replace the amax bits.
+__global__ void amax_per_matrix_kernel(const uint4* __restrict__ w, long long mat_vecs, int* __restrict__ amax_bits) {
+  griddep_wait();
+  const long long mat = blockIdx.y;
+  float amax = 0.f;
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < mat_vecs;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const uint4 u = w[mat * mat_vecs + i];
+    const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 f = __bfloat1622float2(b[k]);
+      amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if ((threadIdx.x & 31) == 0) atomicMax(amax_bits + mat, __float_as_int(amax));
+}
+
+__device__ __forceinline__ float scale_of(int amax_bits) {
+  const float amax = __int_as_float(amax_bits);
+  return amax == 0.f ? 1.f : __fdiv_rn(amax, 448.f);
+}
+
+__global__ void quant_per_matrix_kernel(const uint4* __restrict__ w, long long mat_vecs, const int* __restrict__ amax_bits,
+                                        uint2* __restrict__ q) {
+  const long long mat = blockIdx.y;
+  const float s = scale_of(amax_bits[mat]);
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < mat_vecs;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const uint4 u = w[mat * mat_vecs + i];
+    const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&u);
+    float v[8];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 f = __bfloat1622float2(b[k]);
+      v[2 * k] = f.x;
+      v[2 * k + 1] = f.y;
+    }
+    uint2 o;
+    o.x = e4m3x4(__fdiv_rn(v[0], s), __fdiv_rn(v[1], s), __fdiv_rn(v[2], s), __fdiv_rn(v[3], s));
+    o.y = e4m3x4(__fdiv_rn(v[4], s), __fdiv_rn(v[5], s), __fdiv_rn(v[6], s), __fdiv_rn(v[7], s));
+    q[mat * mat_vecs + i] = o;
+  }
+}
+
+__global__ void scales_from_amax_kernel(int* __restrict__ amax_bits, long long num_mats) {
+  const long long m = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (m < num_mats) amax_bits[m] = __float_as_int(scale_of(amax_bits[m]));
+}
+
 }  // namespace
+
+cudaError_t launch_quant_weights_per_tensor(const Launch& l, const void* w, int64_t num_mats, int64_t mat_elems,
+                                            void* codes, float* scales) {
+  if (mat_elems % 8 != 0 || num_mats <= 0 || num_mats > 65535) return cudaErrorInvalidValue;
+  const long long vecs = mat_elems / 8;
+  int* bits = reinterpret_cast<int*>(scales);
+  cudaError_t err = cudaMemsetAsync(bits, 0, static_cast<size_t>(num_mats) * sizeof(int), l.stream);
+  if (err != cudaSuccess) return err;
+  const unsigned bx = static_cast<unsigned>(std::min<long long>((vecs + 255) / 256, 1024));
+  amax_per_matrix_kernel<<<dim3(bx, static_cast<unsigned>(num_mats)), 256, 0, l.stream>>>(
+      static_cast<const uint4*>(w), vecs, bits);
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  quant_per_matrix_kernel<<<dim3(bx, static_cast<unsigned>(num_mats)), 256, 0, l.stream>>>(
+      static_cast<const uint4*>(w), vecs, bits, static_cast<uint2*>(codes));
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  scales_from_amax_kernel<<<static_cast<unsigned>((num_mats + 255) / 256), 256, 0, l.stream>>>(bits, num_mats);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_quant_act(const Launch& l, const void* x, int T, int H, void* q, float* scale) {
   const int G = H / 128;

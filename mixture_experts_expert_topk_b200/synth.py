@@ -36,13 +36,25 @@ class MoeConfig:
     topk: int              # routed experts per token
     I: int                 # intermediate size (unpadded)
     renormalize: bool
-    activation: str        # "swiglu" | "relu2"
+    activation: str        # "swiglu" | "relu2" | "gelu_tanh"
     num_shared: int = 0    # fused shared-expert slots appended after the routed experts
-    fp8: bool = False      # weights/activations quantised to e4m3 with 128-wide block scales
+    # False: bf16. True: e4m3 with 128-wide block scales. "per_tensor": e4m3 with one scale
+    # per expert matrix and static input / activation scales (activation_scale below; the
+    # input scale is the hidden rows' amax / 448)
+    fp8: object = False
+    activation_scale: float = 0.03
     hidden_std: float = 1.0
     weight_std: float = 0.02
     logit_bias_std: float = 0.0   # per-expert bias added to the logits (skewed load)
     block_m: int = 128
+
+    @property
+    def per_tensor(self) -> bool:
+        return self.fp8 == "per_tensor"
+
+    @property
+    def block128(self) -> bool:
+        return self.fp8 is True
 
     @property
     def gated(self) -> bool:
@@ -80,6 +92,9 @@ CONFIGS: Dict[str, MoeConfig] = {
                        activation="relu2"),
     "fp8_shared": MoeConfig("fp8_shared", T=8192, H=2048, E=512, topk=10, I=512,
                             renormalize=True, activation="swiglu", num_shared=1, fp8=True),
+    # the same shape with per-tensor FP8 scales
+    "fp8pt_shared": MoeConfig("fp8pt_shared", T=8192, H=2048, E=512, topk=10, I=512,
+                              renormalize=True, activation="swiglu", num_shared=1, fp8="per_tensor"),
 }
 
 

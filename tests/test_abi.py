@@ -49,7 +49,8 @@ def test_check_problem_accepts_the_workloads(L):
     from mixture_experts_expert_topk_b200.synth import CONFIGS
     for cfg in CONFIGS.values():
         p = moe.make_problem(cfg.T, cfg.H, cfg.E, cfg.topk, cfg.I, renormalize=cfg.renormalize,
-                             activation=cfg.activation, num_shared=cfg.num_shared, fp8=cfg.fp8)
+                             activation=cfg.activation, num_shared=cfg.num_shared, fp8=cfg.fp8,
+                             input_scale=0.01, activation_scale=cfg.activation_scale)
         assert L.moe_check_problem(ctypes.byref(p)) == 0, cfg.name
 
 
@@ -84,6 +85,9 @@ def test_padded_intermediate_follows_page_rule(L):
         assert L.moe_padded_intermediate(int(i_in), act, 0) == int(i_pad)
     assert L.moe_padded_intermediate(500, _capi.MOE_ACT_SWIGLU, 1) == 512   # FP8: 128
     assert L.moe_padded_intermediate(0, 0, 0) == -1
+    assert L.moe_padded_intermediate(200, _capi.MOE_ACT_SWIGLU, _capi.MOE_DTYPE_FP8_PER_TENSOR) == 256
+    assert L.moe_padded_intermediate(200, _capi.MOE_ACT_GELU_TANH, 0) == 208
+    assert L.moe_padded_intermediate(200, 0, 3) == -1
     assert L.moe_padded_intermediate(16, 7, 0) == -1
 
 
@@ -91,17 +95,20 @@ def test_workspace_layout(L):
     from mixture_experts_expert_topk_b200.synth import CONFIGS
     for cfg in CONFIGS.values():
         p = moe.make_problem(cfg.T, cfg.H, cfg.E, cfg.topk, cfg.I, renormalize=cfg.renormalize,
-                             activation=cfg.activation, num_shared=cfg.num_shared, fp8=cfg.fp8)
+                             activation=cfg.activation, num_shared=cfg.num_shared, fp8=cfg.fp8,
+                             input_scale=0.01, activation_scale=cfg.activation_scale)
         lay = moe.workspace_layout(p)
         P = cfg.T * cfg.k_total
         E = cfg.E_total
         assert lay["status"] == 0
         bm = lay["block_m"]
-        # bf16 aligns each expert to 16 rows (token rows on the MMA's N), FP8 to 128-row tiles
-        assert bm == (128 if cfg.fp8 else 16)
+        # bf16 and per-tensor FP8 align each expert to 16 rows (token rows on the MMA's N),
+        # block-128 FP8 to 128-row tiles
+        assert bm == (128 if cfg.block128 else 16)
         # the permuted hidden rows (row-group order) exist for the 16-row alignment
         xs_bytes = lay["group_info"] - lay["xs"]
-        assert xs_bytes == (-(-lay["max_rows"] * cfg.H * 2 // 1024) * 1024 if not cfg.fp8 else 0)
+        elt = 1 if cfg.per_tensor else 2
+        assert xs_bytes == (-(-lay["max_rows"] * cfg.H * elt // 1024) * 1024 if not cfg.block128 else 0)
         assert lay["max_rows"] == -(-(P + min(E, P) * (bm - 1)) // bm) * bm
         assert lay["num_chunks"] == -(-P // 2048)
         offs = sorted(v for k, v in lay.items() if k not in ("total_bytes", "max_rows", "num_chunks", "block_m"))
@@ -166,3 +173,26 @@ def test_python_layer_fails_loudly_without_a_gpu_tensor():
     with pytest.raises(ValueError):
         moe.moe_forward(torch.zeros(4, 256, dtype=torch.bfloat16), torch.zeros(4, 8),
                         torch.zeros(1), torch.zeros(1), 2, True, "swiglu")
+
+
+def test_per_tensor_fp8_problem_rules(L):
+    ok = moe.make_problem(64, 256, 8, 2, 256, fp8="per_tensor", input_scale=0.01, activation_scale=0.05)
+    assert L.moe_check_problem(ctypes.byref(ok)) == 0
+    lay = moe.workspace_layout(ok)
+    assert lay["block_m"] == 16
+    # e4m3 tiles of 128 x 128: w13 [8, 512, 256] and w2 [8, 256, 256]
+    assert L.moe_prepared_weights_bytes(ctypes.byref(ok), 0) == 8 * 4 * 2 * 16384
+    assert L.moe_prepared_weights_bytes(ctypes.byref(ok), 1) == 8 * 2 * 2 * 16384
+    # the activation (e4m3, rows x I) and permuted rows (rows x H) are one byte per element
+    assert lay["y"] - lay["act"] >= lay["max_rows"] * 256
+    for bad in (dict(input_scale=0.0), dict(activation_scale=-1.0), dict(input_scale=float("nan")),
+                dict(activation_scale=float("inf"))):
+        kw = dict(input_scale=0.01, activation_scale=0.05)
+        kw.update(bad)
+        p = moe.make_problem(64, 256, 8, 2, 256, fp8="per_tensor", **kw)
+        assert L.moe_check_problem(ctypes.byref(p)) == 1, bad
+    p = moe.make_problem(64, 256, 8, 2, 256, fp8="per_tensor", input_scale=0.01, activation_scale=0.05,
+                         block_m=128)
+    assert L.moe_check_problem(ctypes.byref(p)) == 2          # 128-row tiles: not for per-tensor
+    p = moe.make_problem(64, 256, 8, 2, 200, fp8="per_tensor", input_scale=0.01, activation_scale=0.05)
+    assert L.moe_check_problem(ctypes.byref(p)) == 1          # I must be padded to 128

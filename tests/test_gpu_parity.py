@@ -445,3 +445,90 @@ def test_routed_out_of_range_ids_are_dropped_and_reported():
                         topk=cfg.topk, renormalize=False, activation=cfg.activation,
                         routing=O.append_shared_slot(ids_ok.numpy(), w_ok.numpy(), cfg.E, 0))
     assert err_beyond_rounding(got, ref) <= BF16_TOL
+
+
+# ---- per-tensor FP8 -------------------------------------------------------------------
+
+PT_SMALL = {
+    "pt_swiglu": _small("pt_swiglu", T=300, H=256, E=8, topk=2, I=256),
+    "pt_relu2": _small("pt_relu2", T=200, H=384, E=6, topk=3, I=384, activation="relu2", renormalize=False),
+    "pt_gelu_shared": _small("pt_gelu_shared", T=130, H=256, E=12, topk=3, I=256, num_shared=1,
+                             activation="gelu_tanh"),
+    # groups of more than 128 rows (one K chunk per step) and three align chunks
+    "pt_big_groups": _small("pt_big_groups", T=1500, H=256, E=4, topk=2, I=128),
+    "pt_decode": _small("pt_decode", T=4, H=512, E=32, topk=4, I=256),
+}
+
+
+def _untile_u8(flat, group_info, num_groups, rows, kchunks):
+    """Row-major [rows, 128 * kchunks] bytes from row-group order with 128-byte chunks of
+    e4m3 codes (row j's 16-byte piece q stored at position q ^ (j % 8))."""
+    flat = np.asarray(flat).reshape(-1)
+    out = np.zeros((rows, 128 * kchunks), dtype=np.uint8)
+    for g in range(num_groups):
+        x_row, meta = int(group_info[g][0]), int(group_info[g][1])
+        n = meta >> 16
+        grp = flat[x_row * 128 * kchunks:(x_row + n) * 128 * kchunks].reshape(kchunks, n, 8, 16)
+        j = np.arange(n)
+        phys = np.arange(8)[None, :] ^ (j[:, None] & 7)
+        out[x_row:x_row + n] = grp[:, j[:, None], phys, :].transpose(1, 0, 2, 3).reshape(n, 128 * kchunks)
+    return out
+
+
+@pytest.mark.parametrize("name", list(PT_SMALL))
+def test_fp8_per_tensor_layer_parity(name):
+    cfg = PT_SMALL[name]
+    inp = make_inputs(cfg, 0)
+    dev = torch.device("cuda:0")
+    hidden, logits = inp["hidden"].to(dev), inp["logits"].to(dev)
+    w13, w2 = inp["w13"].to(dev), inp["w2"].to(dev)
+    # device quantiser, bit-exact against the oracle's
+    q13, s13 = moe.quantize_weights_fp8_per_tensor(w13)
+    q2, s2 = moe.quantize_weights_fp8_per_tensor(w2)
+    o13, os13, o2, os2 = O.quantize_weights_fp8_per_tensor(bits(inp["w13"]), bits(inp["w2"]))
+    np.testing.assert_array_equal(q13.cpu().numpy(), o13)
+    np.testing.assert_array_equal(q2.cpu().numpy(), o2)
+    np.testing.assert_array_equal(s13.cpu().numpy(), os13)
+    np.testing.assert_array_equal(s2.cpu().numpy(), os2)
+    # static scales: the hidden amax, and an activation calibration from the bf16 oracle's
+    # GEMM1 output on these inputs (values beyond it saturate, in the kernel and the oracle)
+    s_in = float(np.float32(np.abs(bf16_to_f64(inp["hidden"])).max() / 448))
+    x = bf16_to_f64(inp["hidden"])
+    W13 = bf16_to_f64(inp["w13"])
+    ids0, _ = O.route(inp["logits"].numpy(), cfg.topk, cfg.renormalize, cfg.num_shared)
+    amax = max(float(np.abs(O.activation_fn(x[np.nonzero(ids0 == e)[0]] @ W13[e].T, cfg.activation, cfg.I)).max())
+               for e in np.unique(ids0))
+    s_act = float(np.float32(amax / 448 * 0.8))
+    prob = moe.make_problem(cfg.T, cfg.H, cfg.E, cfg.topk, cfg.I, renormalize=cfg.renormalize,
+                            activation=cfg.activation, num_shared=cfg.num_shared, fp8="per_tensor",
+                            input_scale=s_in, activation_scale=s_act)
+    w13p, w2p = moe.prepare_weights(prob, q13, q2, cfg.I)
+    ws = moe.new_workspace(prob)
+    out = moe.moe_forward(hidden, logits, w13p, w2p, cfg.topk, cfg.renormalize, cfg.activation, s13, s2,
+                          num_shared=cfg.num_shared, workspace=ws, input_scale=s_in, activation_scale=s_act)
+    torch.cuda.synchronize()
+    assert moe.device_status(ws)[0] == 0
+    parts = {k: v.cpu().numpy() for k, v in moe.read_workspace(prob, ws).items()}
+    # routing and permutation, bit for bit
+    ids_o, w_o = O.route(inp["logits"].numpy(), cfg.topk, cfg.renormalize, cfg.num_shared)
+    np.testing.assert_array_equal(parts["topk_ids"], ids_o)
+    al = O.align(ids_o, cfg.E_total, 16)
+    P_pad = int(al["P_pad"])
+    np.testing.assert_array_equal(parts["sorted_pair_ids"][:P_pad], al["sorted_pair_ids"])
+    # the permuted, quantised hidden rows: e4m3(hidden * fp32(1 / input_scale)), bit for bit
+    ng = int(parts["num_blocks"][1])
+    xs = _untile_u8(parts["xs"], parts["group_info"], ng, P_pad, cfg.H // 128)
+    pids = al["sorted_pair_ids"][:P_pad]
+    real = pids < cfg.T * cfg.k_total
+    xq = O.quant_per_tensor_inv(O.bf16_bits_to_f32(bits(inp["hidden"])), s_in)
+    np.testing.assert_array_equal(xs[real], xq[pids[real] // cfg.k_total])
+    assert np.all(xs[~real] == 0)
+    # the layer
+    ref = O.moe_forward_fp8_per_tensor(bits(inp["hidden"]), inp["logits"].numpy(), o13, os13, o2, os2, s_in, s_act,
+                                       topk=cfg.topk, renormalize=cfg.renormalize, activation=cfg.activation,
+                                       num_shared=cfg.num_shared)
+    got = bf16_to_f64(out)
+    assert np.all(np.isfinite(got))
+    e = err_beyond_rounding(got, ref)
+    print(f"{name}: beyond-rounding {e:.4f}, raw {max_err_over_rms(got, ref):.4f}")
+    assert e <= FP8_TOL, e
