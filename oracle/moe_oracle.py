@@ -589,6 +589,113 @@ def quantize_weights_fp8(w13_bits, w2_bits, experts=None):
     return w13_q, w13_s, w2_q, w2_s
 
 
+# --------------------------------------------------------------------------
+# MXFP8: E4M3 values sharing one power-of-two scale per block of 32
+# --------------------------------------------------------------------------
+
+MX_BLOCK = 32        # values per scale ([TRTLLM] section 2, ``_align_mxfp8_moe_weights``)
+E4M3_EMAX = 8        # exponent of the largest power of two E4M3 holds (2^8 = 256 <= 448)
+
+
+def quant_mx(x: np.ndarray):
+    """MXFP8 quantisation along the last axis (the GEMM's reduction dimension).
+
+    [TRTLLM] section 2 (``_align_mxfp8_moe_weights``) fixes the block: one scale per 32
+    consecutive values of K (the scale tensors' last dimension is K / 32) and pads the
+    scales with the weights. The pages print no conversion rule; reading taken: the OCP
+    Microscaling Formats (MX) v1.0 conversion for MXFP8 E4M3, i.e. per block
+      shared exponent  s = floor(log2(amax)) - 8  (8 = E4M3's largest exponent),
+                       clamped to [-127, 127]; an all-zero block takes -127;
+      scale            2^s, stored as the E8M0 byte s + 127;
+      elements         e4m3(x * 2^-s), round to nearest even, saturating at 448.
+    The product x * 2^-s is exact (a power-of-two scaling of an fp32 value), so the codes
+    are decided exactly; the block's largest value lands in [256, 512).
+    Returns (codes uint8 [..., K], scale bytes uint8 [..., K / 32]).
+    """
+    x = np.asarray(x, dtype=np.float32)
+    K = x.shape[-1]
+    assert K % MX_BLOCK == 0
+    b = x.reshape(x.shape[:-1] + (K // MX_BLOCK, MX_BLOCK)).astype(np.float64)
+    amax = np.abs(b).max(axis=-1)
+    _, ex = np.frexp(amax)                                  # amax = m * 2^ex, m in [0.5, 1)
+    s = np.where(amax > 0, ex.astype(np.int64) - 1 - E4M3_EMAX, -127)
+    s = np.clip(s, -127, 127)
+    scaled = (b * np.ldexp(1.0, (-s)[..., None].astype(np.int32))).astype(np.float32)
+    codes = e4m3_encode(scaled).reshape(x.shape)
+    return codes, (s + 127).astype(np.uint8)
+
+
+def dequant_mx(codes: np.ndarray, scale_bytes: np.ndarray) -> np.ndarray:
+    """codes * 2^(byte - 127) per block of 32 along the last axis, in float64."""
+    s = np.repeat(scale_bytes.astype(np.int64) - 127, MX_BLOCK, axis=-1)
+    return e4m3_decode(codes) * np.ldexp(1.0, s.astype(np.int32))
+
+
+def quantize_weights_mxfp8(w13_bits, w2_bits, experts=None):
+    """MXFP8 weights (``quant_mx`` along each matrix's K: H for w13, I for w2).
+
+    Returns (w13 codes [E, N1, H], w13 scale bytes [E, N1, H/32], w2 codes [E, H, I],
+    w2 scale bytes [E, H, I/32]) in the checkpoint layout. ``experts`` limits the work to
+    the listed experts (the others stay zero).
+    """
+    out = []
+    for wb in (w13_bits, w2_bits):
+        wb = np.asarray(wb)
+        E, R, C = wb.shape
+        q = np.zeros((E, R, C), dtype=np.uint8)
+        sc = np.zeros((E, R, C // MX_BLOCK), dtype=np.uint8)
+        for e in (range(E) if experts is None else experts):
+            q[e], sc[e] = quant_mx(bf16_bits_to_f32(wb[e]))
+        out += [q, sc]
+    return tuple(out)
+
+
+def moe_forward_mxfp8(hidden_bits: np.ndarray, logits: Optional[np.ndarray], w13_q, w13_sc, w2_q, w2_sc, *,
+                      topk: int, renormalize: bool, activation: str, num_shared: int = 0,
+                      tokens: Optional[Sequence[int]] = None, routing=None):
+    """MXFP8 W8A8 layer forward in float64.
+
+    [TRTLLM] section 2 adds MXFP8 MoE weights with per-32 scales beside the FP8 ones.
+    Reading taken for what the pages leave open: both GEMM inputs are MXFP8 (the
+    block-scaled MMA takes one scale per 32 values of K on each operand), so
+      * the bf16 hidden rows are quantised per token (``quant_mx``) before GEMM1;
+      * GEMM1's activation is stored in bf16 (as in the bf16 and 128x128 FP8 paths) and
+        quantised per pair row the same way before GEMM2;
+      * every product uses the exactly dequantised values in float64.
+    ``w13_q``/``w2_q`` uint8 codes, ``w13_sc`` [E, N1, H/32] and ``w2_sc`` [E, H, I/32]
+    uint8 E8M0 scale bytes. ``routing`` as in ``moe_forward``.
+    """
+    if routing is not None:
+        ids, w = (np.asarray(routing[0], dtype=np.int32), np.asarray(routing[1], dtype=np.float32))
+        if tokens is not None:
+            tokens = np.asarray(tokens, dtype=np.int64)
+            hidden_bits = np.asarray(hidden_bits)[tokens]
+            ids, w = ids[tokens], w[tokens]
+    else:
+        logits = np.asarray(logits, dtype=np.float32)
+        if tokens is not None:
+            tokens = np.asarray(tokens, dtype=np.int64)
+            hidden_bits = np.asarray(hidden_bits)[tokens]
+            logits = logits[tokens]
+        ids, w = route(logits, topk, renormalize, num_shared)
+    x = dequant_mx(*quant_mx(bf16_bits_to_f32(hidden_bits)))
+    T, kk = ids.shape
+    H = x.shape[1]
+    I = w2_q.shape[2]
+    y = np.zeros((T, kk, H), dtype=np.float64)
+    for e in np.unique(ids):
+        t_idx, j_idx = np.nonzero(ids == e)
+        W13 = dequant_mx(np.asarray(w13_q[e]), np.asarray(w13_sc[e]))
+        W2 = dequant_mx(np.asarray(w2_q[e]), np.asarray(w2_sc[e]))
+        a = activation_fn(x[t_idx] @ W13.T, activation, I)
+        ad = dequant_mx(*quant_mx(round_to_bf16(a)))
+        y[t_idx, j_idx] = w[t_idx, j_idx].astype(np.float64)[:, None] * (ad @ W2.T)
+    out = np.zeros((T, H), dtype=np.float64)
+    for j in range(kk):
+        out += y[:, j]
+    return out
+
+
 def rms(x: np.ndarray) -> float:
     x = np.asarray(x, dtype=np.float64)
     return math.sqrt(float(np.mean(x * x))) if x.size else 0.0

@@ -524,6 +524,109 @@ def test_fp8_per_tensor_layer_against_torch_casts(act):
 
 
 # --------------------------------------------------------------------------
+# MXFP8 (OCP MX v1.0 conversion, block 32, E8M0 scales)
+# --------------------------------------------------------------------------
+
+
+def test_quant_mx_golden_points():
+    # hand-derived: all ones -> floor(log2 1) - 8 = -8 (byte 119), 1 * 2^8 = 256 -> 0x78
+    q, s = O.quant_mx(np.ones(32, np.float32))
+    assert s.tolist() == [119] and np.all(q == 0x78)
+    # amax 3 -> s = 1 - 8 = -7 (byte 120); 3 * 128 = 384 = 1.5 * 2^8 -> 0x7C;
+    # -0.375 * 128 = -48 = -1.5 * 2^5 -> sign | exponent field 12 | mantissa 4 = 0xE4
+    x = np.zeros(32, np.float32)
+    x[0], x[31] = 3.0, -0.375
+    q, s = O.quant_mx(x)
+    assert s.tolist() == [120] and q[0] == 0x7C and q[31] == 0xE4 and np.all(q[1:31] == 0)
+    # 255/128 -> s = -8, scaled 510 saturates to 448 (0x7E)
+    q, s = O.quant_mx(np.full(32, 255.0 / 128.0, np.float32))
+    assert s.tolist() == [119] and np.all(q == 0x7E)
+    # all-zero block: byte 0, codes 0
+    q, s = O.quant_mx(np.zeros(32, np.float32))
+    assert s.tolist() == [0] and np.all(q == 0)
+    # exponent clamps: amax 2^-130 wants s = -138 -> -127 (byte 0), 2^-130 * 2^127 = 2^-3 -> 0x20;
+    # amax 2^120 -> s = 112 (byte 239) -> 2^8 -> 0x78
+    q, s = O.quant_mx(np.array([2.0 ** -130] + [0.0] * 31 + [2.0 ** 120] + [0.0] * 31, np.float32))
+    assert s.tolist() == [0, 239] and q[0] == 0x20 and q[32] == 0x78
+
+
+def test_quant_mx_against_math_frexp_and_torch_cast():
+    rng = np.random.default_rng(41)
+    x = (rng.standard_normal((6, 256)) * np.exp2(rng.integers(-12, 12, (6, 1)))).astype(np.float32)
+    x[2, 64:96] = 0.0
+    x[3, 5] = 1e30                               # one huge value dominates its block
+    q, s = O.quant_mx(x)
+    assert q.shape == x.shape and s.shape == (6, 8) and s.dtype == np.uint8
+    for r in range(6):
+        for b in range(8):
+            blk = x[r, 32 * b:32 * b + 32].astype(np.float64)
+            amax = float(np.abs(blk).max())
+            e = (math.frexp(amax)[1] - 1 - 8) if amax > 0 else -127
+            e = max(-127, min(127, e))
+            assert int(s[r, b]) == e + 127
+            scaled = torch.from_numpy(np.clip(blk * 2.0 ** -e, -448, 448).astype(np.float32))
+            want = scaled.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+            np.testing.assert_array_equal(q[r, 32 * b:32 * b + 32], want)
+            if amax > 0:                          # the block maximum lands in [256, 512)
+                assert 256.0 <= amax * 2.0 ** -e < 512.0
+    # dequantisation: exact for E4M3 values times a power of two, else within half a step
+    d = O.dequant_mx(q, s)
+    step = np.repeat(np.ldexp(1.0, s.astype(np.int32) - 127), 32, 1)
+    sat = np.abs(x) * np.repeat(np.ldexp(1.0, 127 - s.astype(np.int32)), 32, 1) > 448
+    assert np.all(np.abs(d - x)[~sat] <= (np.abs(x) * 2.0 ** -4 + step * 2.0 ** -10)[~sat])
+    # a block of E4M3 values whose largest is 448 keeps scale 2^0 (times any power of two)
+    codes = np.concatenate([rng.integers(0, 0x7E, (3, 31)), np.full((3, 1), 0x7E)], 1).astype(np.uint8)
+    codes[1] |= 0x80
+    v = (O.e4m3_decode(codes) * np.ldexp(1.0, np.array([-5, 0, 7]))[:, None]).reshape(1, 96)
+    q2, s2 = O.quant_mx(v.astype(np.float32))
+    assert s2.tolist() == [[122, 127, 134]]
+    np.testing.assert_array_equal(O.dequant_mx(q2, s2), v)
+
+
+@pytest.mark.parametrize("act", ["swiglu", "relu2"])
+def test_mxfp8_layer_against_torch_casts(act):
+    # independent restatement: math.frexp exponents, torch float8 casts, a dense per-token loop
+    rng = np.random.default_rng(43)
+    T, H, E, k, I = 5, 128, 3, 2, 64
+    N1 = I if act == "relu2" else 2 * I
+    x = _bf16_bits(torch.from_numpy(rng.standard_normal((T, H)).astype(np.float32)))
+    l = rng.standard_normal((T, E)).astype(np.float32)
+    w13 = _bf16_bits(torch.from_numpy(0.02 * rng.standard_normal((E, N1, H)).astype(np.float32)))
+    w2 = _bf16_bits(torch.from_numpy(0.02 * rng.standard_normal((E, H, I)).astype(np.float32)))
+    q13, s13, q2, s2 = O.quantize_weights_mxfp8(w13, w2)
+    got = O.moe_forward_mxfp8(x, l, q13, s13, q2, s2, topk=k, renormalize=True, activation=act)
+
+    def mx(a):  # quantise + dequantise rows of a (float32) in blocks of 32
+        a = np.asarray(a, np.float32)
+        out = np.zeros(a.shape)
+        for idx in np.ndindex(a.shape[:-1]):
+            for b in range(a.shape[-1] // 32):
+                blk = a[idx][32 * b:32 * b + 32].astype(np.float64)
+                amax = float(np.abs(blk).max())
+                e = max(-127, min(127, (math.frexp(amax)[1] - 9) if amax > 0 else -127))
+                c = torch.from_numpy(np.clip(blk * 2.0 ** -e, -448, 448).astype(np.float32)).to(torch.float8_e4m3fn)
+                out[idx][32 * b:32 * b + 32] = c.to(torch.float64).numpy() * 2.0 ** e
+        return out
+
+    W13 = [mx(O.bf16_bits_to_f32(w13[e])) for e in range(E)]
+    W2 = [mx(O.bf16_bits_to_f32(w2[e])) for e in range(E)]
+    Xd = mx(O.bf16_bits_to_f32(x))
+    ids, wts = _route_brute(l, k, True)
+    want = np.zeros((T, H))
+    for t in range(T):
+        for j in range(k):
+            e = ids[t, j]
+            z = W13[e] @ Xd[t]
+            a = np.maximum(z, 0) ** 2 if act == "relu2" else z[:I] / (1 + np.exp(-z[:I])) * z[I:]
+            a16 = torch.from_numpy(a.astype(np.float32)).to(torch.bfloat16).to(torch.float32).numpy()
+            want[t] += np.float64(np.float32(wts[t, j])) * (W2[e] @ mx(a16[None])[0])
+    np.testing.assert_allclose(got, want, rtol=1e-9, atol=1e-12)
+    # the MX layer stays near the bf16 layer (three E4M3 roundings of about 4% RMS each)
+    ref = O.moe_forward(x, l, w13, w2, topk=k, renormalize=True, activation=act)
+    assert O.rms(got - ref) < 0.15 * O.rms(ref)
+
+
+# --------------------------------------------------------------------------
 # planted mistakes: each mutated oracle must fail a pin above
 # --------------------------------------------------------------------------
 
