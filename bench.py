@@ -42,7 +42,7 @@ L2_FLUSH_BYTES = 512 << 20
 # (dram__bytes_read.sum + dram__bytes_write.sum of the GEMM1 launch on the 64-expert
 # prefill case), valid only for the kernel source it was taken on (sha256 prefix of the
 # file below); None until such a capture exists for that source.
-GEMM1_TRAFFIC = {"source": "gemm_swap.cu", "source_sha256": "13e7861c9da1", "ratio": 308.78 / 281.02}
+GEMM1_TRAFFIC = {"source": "gemm_swap.cu", "source_sha256": "063971d6a1a3", "ratio": 308.49 / 281.02}
 
 
 def _peaks():
@@ -56,7 +56,8 @@ def _peaks():
 
 def _workload_name(cfg: MoeConfig) -> str:
     act = "SwiGLU" if cfg.gated else "relu2"
-    dt = ("FP8 e4m3 W8A8 per-tensor" if cfg.per_tensor else "FP8 e4m3 W8A8 block-128") if cfg.fp8 else "bf16"
+    dt = ("MXFP8 e4m3 W8A8 (E8M0 scale per 32)" if cfg.mx else
+          ("FP8 e4m3 W8A8 per-tensor" if cfg.per_tensor else "FP8 e4m3 W8A8 block-128")) if cfg.fp8 else "bf16"
     sh = f"+{cfg.num_shared} shared" if cfg.num_shared else ""
     return (f"{cfg.name}: {dt} {act} MoE layer forward, T={cfg.T} H={cfg.H} E={cfg.E}{sh} "
             f"top-{cfg.topk}{sh} I={cfg.I}")
@@ -188,13 +189,21 @@ def run_ours(cfg: MoeConfig, steps: int, warmup: int, world: int, rank: int, loc
     s13 = s2 = None
     w13 = inp["w13"].to(dev)
     w2 = inp["w2"].to(dev)
-    if cfg.per_tensor:
+    if cfg.mx:
+        w13, s13 = moe.quantize_weights_mxfp8(w13)
+        w2, s2 = moe.quantize_weights_mxfp8(w2)
+    elif cfg.per_tensor:
         w13, s13 = moe.quantize_weights_fp8_per_tensor(w13)
         w2, s2 = moe.quantize_weights_fp8_per_tensor(w2)
     elif cfg.fp8:
         w13, s13 = moe.quantize_weights_fp8(w13)
         w2, s2 = moe.quantize_weights_fp8(w2)
-    w13p, w2p = moe.prepare_weights(prob, w13, w2, cfg.I)
+    if cfg.mx:
+        # the E8M0 scales travel inside the prepared weights; the forward takes none
+        w13p, w2p = moe.prepare_weights(prob, w13, w2, cfg.I, w13_scale=s13, w2_scale=s2)
+        s13 = s2 = None
+    else:
+        w13p, w2p = moe.prepare_weights(prob, w13, w2, cfg.I)
     del w13, w2
     ws = moe.new_workspace(prob, dev)
     out = torch.empty_like(hidden)
@@ -289,8 +298,9 @@ def run_ours(cfg: MoeConfig, steps: int, warmup: int, world: int, rank: int, loc
         "e2e_total_ms": e2e_total, "ids": ids, "inp": inp,
         "h2d": h_hidden.numel() * 2 + h_logits.numel() * 4, "d2h": h_out.numel() * 2,
         # one kernel per stage, except align (three kernels above one 2048-pair chunk) and
-        # FP8 GEMM1 (the GEMM, then the per-row activation quantisation)
-        "launches_per_step": len(names) + (2 if cfg.T * cfg.k_total > 2048 else 0) + (1 if cfg.block128 else 0),
+        # block-128 FP8 and MXFP8 GEMM1 (the GEMM, then the activation quantisation)
+        "launches_per_step": len(names) + (2 if cfg.T * cfg.k_total > 2048 else 0) +
+                             (1 if cfg.block128 or cfg.mx else 0),
     }
 
 
@@ -314,15 +324,22 @@ def cpu_baseline(cfg: MoeConfig, inp, budget_s: float, tokens_hint: int):
 
     hb, lg = bits(inp["hidden"]), inp["logits"].numpy()
     w13b, w2b = bits(inp["w13"]), bits(inp["w2"])
-    if cfg.per_tensor:
+    n = max(1, min(cfg.T, tokens_hint))
+    tok = np.arange(n)
+    if cfg.mx:
+        # quantise only the experts the sampled tokens use (the others do not enter the sample)
+        ids, _ = O.route(lg[tok], cfg.topk, cfg.renormalize, cfg.num_shared)
+        fp8w = O.quantize_weights_mxfp8(w13b, w2b, experts=sorted(set(int(e) for e in ids.reshape(-1))))
+    elif cfg.per_tensor:
         fp8w = O.quantize_weights_fp8_per_tensor(w13b, w2b)
         s_in = np.float32(np.abs(O.bf16_bits_to_f32(hb)).max() / np.float32(448))
     elif cfg.fp8:
         fp8w = O.quantize_weights_fp8(w13b, w2b)
-    n = max(1, min(cfg.T, tokens_hint))
-    tok = np.arange(n)
     t0 = time.perf_counter()
-    if cfg.per_tensor:
+    if cfg.mx:
+        O.moe_forward_mxfp8(hb, lg, *fp8w, topk=cfg.topk, renormalize=cfg.renormalize,
+                            activation=cfg.activation, num_shared=cfg.num_shared, tokens=tok)
+    elif cfg.per_tensor:
         O.moe_forward_fp8_per_tensor(hb, lg, *fp8w, s_in, cfg.activation_scale, topk=cfg.topk,
                                      renormalize=cfg.renormalize, activation=cfg.activation,
                                      num_shared=cfg.num_shared, tokens=tok)
@@ -367,7 +384,7 @@ def main():
     metric = "fused MoE layer forward throughput (TFLOP/s; us/call in ms_per_step)"
     base = {"metric": metric, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "fp8_e4m3" if cfg.fp8 else "bf16", "data": "synthetic"}
+            "vs_baseline": None, "dtype": ("mxfp8_e4m3" if cfg.mx else "fp8_e4m3") if cfg.fp8 else "bf16", "data": "synthetic"}
 
     if args.impl == "reference":
         if rank != 0:
@@ -402,6 +419,8 @@ def main():
     hbm_peak, tc_peak, peak_kind = _peaks()
     elt = 1 if cfg.fp8 else 2
     n_touched, w13_bytes, w2_bytes = touched_expert_bytes(r["ids"], cfg, elt)
+    if cfg.mx:  # one E8M0 byte per 32 weights
+        w13_bytes, w2_bytes = w13_bytes * 33 // 32, w2_bytes * 33 // 32
     P = cfg.T * cfg.k_total
     # GEMM1 algorithmic bytes per launch: touched w13, hidden rows read once, act written
     g1_bytes = w13_bytes + cfg.T * cfg.H * elt + P * cfg.I * elt

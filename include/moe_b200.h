@@ -81,10 +81,19 @@ typedef enum {
                                  e4m3 activations with one fp32 scale per 1x128 group
                                  (FP8 W8A8, block_shape [128, 128]; sglang PR 26204
                                  section 1) */
-  MOE_DTYPE_FP8_PER_TENSOR = 2 /* e4m3 weights with one fp32 scale per expert matrix, e4m3
+  MOE_DTYPE_FP8_PER_TENSOR = 2, /* e4m3 weights with one fp32 scale per expert matrix, e4m3
                                    GEMM inputs with the static problem->input_scale and
                                    problem->activation_scale (the per-tensor FP8 variant,
                                    sglang PR 21321 sections 1-2); I and H multiples of 128 */
+  MOE_DTYPE_MXFP8 = 3           /* MXFP8: e4m3 weights and GEMM inputs, each with one E8M0
+                                   (power-of-two) scale per 32 values of K (the MXFP8 weights
+                                   of sglang PR 21321 section 2), applied by the tensor core's
+                                   block-scaled MMA. Conversion (weights, hidden rows and
+                                   GEMM1's bf16 activation): OCP Microscaling v1.0, shared
+                                   exponent floor(log2(amax)) - 8 clamped to [-127, 127]
+                                   (-127 for an all-zero block), byte = exponent + 127, codes
+                                   e4m3(x * 2^-exponent) round to nearest even, saturating.
+                                   I and H multiples of 128. */
 } moe_wdtype_t;
 
 /* Bit flags of moe_problem_t.flags. */
@@ -104,10 +113,10 @@ typedef struct {
   int32_t renormalize;  /* 0/1: divide the selected softmax weights by their sum */
   int32_t activation;   /* moe_activation_t */
   int32_t wdtype;       /* moe_wdtype_t */
-  int32_t block_m;      /* row alignment of each expert's segment: 0 = default (16 for
-                           BF16, 128 for FP8), 16 (BF16 only: the expert's weight rows are
-                           the MMA's M operand and its token rows N) or 128 (128-row token
-                           tiles) */
+  int32_t block_m;      /* row alignment of each expert's segment: 0 = default (128 for
+                           FP8 block-128, 16 otherwise), 16 (all but FP8 block-128: the
+                           expert's weight rows are the MMA's M operand and its token rows
+                           N) or 128 (BF16 and FP8 block-128: 128-row token tiles) */
   uint32_t flags;       /* MOE_FLAG_* */
   float input_scale;      /* MOE_DTYPE_FP8_PER_TENSOR: static scale of the hidden rows,
                              x_q = e4m3(x / input_scale); finite, > 0 (ignored otherwise) */
@@ -138,6 +147,8 @@ typedef struct {
   size_t y;               /* fp32 [max_rows, H]: weighted GEMM2 rows in sorted order */
   size_t xs;              /* bf16 [max_rows, H]: hidden rows in sorted order (block_m 16,
                              more than 1024 pairs; size 0 otherwise) */
+  size_t xs_scale;        /* MXFP8: E8M0 scale bytes of xs: per row group, 1024 bytes per
+                             128 columns at ((first row / 16) * H/128 + chunk) * 1024 */
   size_t group_info;      /* int32 pairs [max_rows/16 + 1]: row groups {first row, expert |
                              rows << 16} of the GEMMs (block_m 16); the count is the second
                              int32 of the num_blocks region */
@@ -198,6 +209,33 @@ moe_status_t moe_quantize_weights_fp8_per_tensor(const void* w, int64_t num_mats
                                                  int32_t cols, void* codes, float* scales,
                                                  moe_stream_t stream);
 
+/* MXFP8 quantisation of bf16 weights (MOE_DTYPE_MXFP8), along each row:
+ *   w        device bf16 [num_mats, rows, cols], cols a multiple of 32;
+ *   codes    device e4m3 [num_mats, rows, cols];
+ *   scales   device uint8 [num_mats, rows, cols/32]: E8M0 bytes (exponent + 127).
+ * Per block of 32 values of a row: the OCP Microscaling v1.0 conversion (see
+ * MOE_DTYPE_MXFP8). Asynchronous on `stream`. */
+moe_status_t moe_quantize_weights_mxfp8(const void* w, int64_t num_mats, int32_t rows, int32_t cols,
+                                        void* codes, void* scales, moe_stream_t stream);
+
+/* Load-time preparation of MXFP8 weights (problem->wdtype == MOE_DTYPE_MXFP8, default
+ * block_m 16):
+ *   w13_codes [E, N1, H] e4m3 and w13_scales [E, N1, H/32] E8M0 bytes, checkpoint order
+ *             (gate rows then up rows for a gated activation);
+ *   w2_codes  [E, H, I] and w2_scales [E, H, I/32]; I = problem->intermediate (a multiple
+ *             of 128: the weights come already padded, as for FP8).
+ * Each output (moe_prepared_weights_bytes(problem, 0 / 1) bytes, 16-byte aligned) holds the
+ * codes tiled as for per-tensor FP8 (tile (e, m, c): rows [128m, 128m+128), columns
+ * [128c, 128c+128), 16384 bytes at ((e*MT + m)*KC + c) * 16384, gated rows interleaved
+ * [gate0, up0, ...], 16-byte pieces of row r at position q ^ (r % 8)), followed by the
+ * scales: a 512-byte block per tile at the same tile index, byte 16 l + 4 j + k = scale of
+ * tile row 32 j + l for K block 4 c + k (zero past the matrix). moe_forward takes the
+ * prepared buffers and NULL scale pointers. Asynchronous on `stream`. */
+moe_status_t moe_prepare_weights_mxfp8(const moe_problem_t* problem, const void* w13_codes,
+                                       const void* w13_scales, const void* w2_codes,
+                                       const void* w2_scales, void* w13_out, void* w2_out,
+                                       moe_stream_t stream);
+
 /* Bytes of the prepared w13 (which = 0) or w2 (which = 1) for `problem` (host only), or
  * 0 for an invalid problem or `which`. */
 size_t moe_prepared_weights_bytes(const moe_problem_t* problem, int32_t which);
@@ -219,6 +257,7 @@ moe_status_t moe_quantize_weights_fp8(const void* w, int64_t num_mats, int32_t r
  *   w13_scale      FP8 block-128: device fp32 [E, N1/128, H/128], checkpoint (gate-first,
  *                  un-interleaved) block order; FP8 per-tensor: device fp32 [E]; else NULL
  *   w2_scale       FP8 block-128: device fp32 [E, H/128, I/128]; per-tensor: [E]; else NULL
+ *                  (MXFP8: both NULL, the scales are part of the prepared weights)
  *   out            device bf16 [T, H] (must not alias hidden)
  *   workspace      device, >= moe_workspace_size(problem) bytes, 256-byte aligned; one
  *                  workspace must not be used by two calls in flight at once.

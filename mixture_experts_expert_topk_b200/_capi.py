@@ -24,6 +24,7 @@ MOE_ACT_SWIGLU = 0
 MOE_ACT_RELU2 = 1
 MOE_ACT_GELU_TANH = 2
 MOE_DTYPE_FP8_PER_TENSOR = 2
+MOE_DTYPE_MXFP8 = 3
 MOE_DTYPE_BF16 = 0
 MOE_DTYPE_FP8_BLOCK128 = 1
 MOE_FLAG_PDL = 1
@@ -51,7 +52,7 @@ class Layout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in (
         "total_bytes", "status", "num_blocks", "topk_ids", "topk_w", "sorted_pair_ids",
         "expert_offsets", "block_expert", "pair_to_row", "chunk_hist", "xq", "xq_scale", "act",
-        "actq", "act_scale", "y", "xs", "group_info", "io_hidden", "io_logits", "io_out")] + [
+        "actq", "act_scale", "y", "xs", "xs_scale", "group_info", "io_hidden", "io_logits", "io_out")] + [
         ("max_rows", ctypes.c_int64),
         ("num_chunks", ctypes.c_int32),
         ("block_m", ctypes.c_int32),
@@ -80,6 +81,8 @@ SIGNATURES = {
     "moe_prepared_weights_bytes": (_S, [_P, _I]),
     "moe_quantize_weights_fp8": (_I, [_V, ctypes.c_int64, _I, _I, _V, _V, _V]),
     "moe_quantize_weights_fp8_per_tensor": (_I, [_V, ctypes.c_int64, _I, _I, _V, _V, _V]),
+    "moe_quantize_weights_mxfp8": (_I, [_V, ctypes.c_int64, _I, _I, _V, _V, _V]),
+    "moe_prepare_weights_mxfp8": (_I, [_P, _V, _V, _V, _V, _V, _V, _V]),
     "moe_forward": (_I, [_P, _V, _V, _V, _V, _V, _V, _V, _V, _S, _V]),
     "moe_forward_routed": (_I, [_P, _V, _V, _V, _V, _V, _V, _V, _V, _V, _S, _V]),
     "moe_forward_host": (_I, [_P, _V, _V, _V, _V, _V, _V, _V, _V, _S, _V]),

@@ -49,7 +49,7 @@ bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr
 bool aligned4(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 struct Plan {
-  int T, H, Er, Es, E, I, topk, kk, bm, grp, N1, gated, fp8, pt, q8, renorm, act;
+  int T, H, Er, Es, E, I, topk, kk, bm, grp, N1, gated, fp8, pt, mx, q8, renorm, act;
   float in_scale, act_scale;  // per-tensor FP8 static scales
   long long P;
   int bn1, bn2;
@@ -67,13 +67,15 @@ moe_status_t make_plan(const moe_problem_t* p, Plan* pl) {
   if (p->renormalize != 0 && p->renormalize != 1) return MOE_ERR_INVALID_ARG;
   if (p->activation != MOE_ACT_SWIGLU && p->activation != MOE_ACT_RELU2 && p->activation != MOE_ACT_GELU_TANH)
     return MOE_ERR_INVALID_ARG;
-  if (p->wdtype != MOE_DTYPE_BF16 && p->wdtype != MOE_DTYPE_FP8_BLOCK128 && p->wdtype != MOE_DTYPE_FP8_PER_TENSOR)
+  if (p->wdtype != MOE_DTYPE_BF16 && p->wdtype != MOE_DTYPE_FP8_BLOCK128 && p->wdtype != MOE_DTYPE_FP8_PER_TENSOR &&
+      p->wdtype != MOE_DTYPE_MXFP8)
     return MOE_ERR_INVALID_ARG;
   if (p->flags & ~MOE_FLAG_PDL) return MOE_ERR_INVALID_ARG;
   q.gated = p->activation != MOE_ACT_RELU2;
   q.fp8 = p->wdtype == MOE_DTYPE_FP8_BLOCK128;
   q.pt = p->wdtype == MOE_DTYPE_FP8_PER_TENSOR;
-  q.q8 = q.fp8 || q.pt;
+  q.mx = p->wdtype == MOE_DTYPE_MXFP8;
+  q.q8 = q.fp8 || q.pt || q.mx;  // 8-bit weights: I must come padded to 128
   if (q.pt) {
     // static scales: finite and positive
     if (!(p->input_scale > 0.0f && p->input_scale < 3.0e38f) ||
@@ -106,9 +108,9 @@ moe_status_t make_plan(const moe_problem_t* p, Plan* pl) {
   // operand and row groups of up to 256 token rows as N. FP8, or block_m = 128: 128-row
   // token tiles.
   if (p->block_m == 16 && q.fp8) return MOE_ERR_UNSUPPORTED;
-  if (p->block_m == 128 && q.pt) return MOE_ERR_UNSUPPORTED;
+  if (p->block_m == 128 && (q.pt || q.mx)) return MOE_ERR_UNSUPPORTED;
   q.bm = p->block_m != 0 ? p->block_m : (q.fp8 ? 128 : 16);
-  q.grp = q.bm == 16 ? kGroupRows : 0;
+  q.grp = q.bm == 16 ? (q.mx ? moe::kMxGroupRows : kGroupRows) : 0;
   q.renorm = p->renormalize;
   q.act = p->activation;
   q.P = static_cast<long long>(q.T) * q.kk;
@@ -146,10 +148,13 @@ moe_status_t make_plan(const moe_problem_t* p, Plan* pl) {
   // bf16 or 128 e4m3 columns)
   const size_t act_bytes = q.pt ? rows * I : rows * (q.bm == 16 ? align_up(I, 64) : I) * 2;
   L.act = take(act_bytes);
-  L.actq = take(q.fp8 ? rows * I : 0);
-  L.act_scale = take(q.fp8 ? rows * (I / 128) * 4 : 0);
+  // MXFP8: the activation's codes (128-column chunks) and scales: 1024 bytes per 16 rows per
+  // 128 columns (a group's scale blocks sit at its first row / 16)
+  L.actq = take(q.fp8 || q.mx ? rows * I : 0);
+  L.act_scale = take(q.fp8 ? rows * (I / 128) * 4 : (q.mx ? rows / 16 * (I / 128) * 1024 : 0));
   L.y = take(rows * H * 4);
-  L.xs = take(q.bm == 16 ? rows * H * (q.pt ? 1 : 2) : 0);
+  L.xs = take(q.bm == 16 ? rows * H * (q.pt || q.mx ? 1 : 2) : 0);
+  L.xs_scale = take(q.mx ? rows / 16 * (H / 128) * 1024 : 0);
   L.group_info = take(q.bm == 16 ? (rows / 16 + 1) * 8 : 0);
   L.io_hidden = take(T * H * 2);
   L.io_logits = take(T * static_cast<size_t>(q.Er) * 4);
@@ -312,6 +317,18 @@ moe_status_t run_gemm1(const Plan& pl_in, const void* hidden, const void* w13, c
     o.w_scale = w13_scale;
     o.in_scale = pl.in_scale;
     o.act_scale = pl.act_scale;
+    if (pl.mx) {
+      // the weight scales follow the tiled codes; GEMM1 writes the bf16 activation, which is
+      // then quantised for GEMM2
+      o.mx = 1;
+      o.w_sf = static_cast<const uint8_t*>(w13) + moe::tiled_weight_bytes_u8(pl.E, pl.N1, pl.H);
+      o.x_sf = ws_ptr<void>(ws, L.xs_scale);
+      moe_status_t st = cuda_status(moe::launch_gemm_swap(l, 0, o, s, b));
+      if (st != MOE_OK) return st;
+      return cuda_status(moe::launch_act_quant_mx(l, ws_ptr<void>(ws, L.act), pl.I, ws_ptr<int>(ws, L.num_blocks) + 1,
+                                                  ws_ptr<int2>(ws, L.group_info), ws_ptr<void>(ws, L.actq),
+                                                  ws_ptr<void>(ws, L.act_scale), num_sms));
+    }
     return cuda_status(moe::launch_gemm_swap(l, 0, o, s, b));
   }
   if (!pl.fp8) {
@@ -352,6 +369,11 @@ moe_status_t run_gemm1(const Plan& pl_in, const void* hidden, const void* w13, c
 moe_status_t run_permute(const Plan& pl, const void* hidden, void* ws, const Launch& l, int num_sms) {
   if (pl.bm != 16) return MOE_OK;
   const auto& L = pl.lay;
+  if (pl.mx)
+    return cuda_status(moe::launch_permute_mx_rows(
+        l, hidden, pl.H, ws_ptr<int>(ws, L.sorted_pair_ids), ws_ptr<int>(ws, L.num_blocks) + 1,
+        ws_ptr<int2>(ws, L.group_info), static_cast<int>(pl.P), pl.kk, ws_ptr<void>(ws, L.xs),
+        ws_ptr<void>(ws, L.xs_scale), num_sms));
   if (pl.pt)
     return cuda_status(moe::launch_permute_quant_rows(
         l, hidden, pl.H, ws_ptr<int>(ws, L.sorted_pair_ids), ws_ptr<int>(ws, L.num_blocks) + 1,
@@ -389,6 +411,12 @@ moe_status_t run_gemm2(const Plan& pl_in, const void* w2, const float* w2_scale,
     o.fp8 = pl.pt;
     o.w_scale = w2_scale;
     o.in_scale = pl.act_scale;
+    if (pl.mx) {
+      o.mx = 1;
+      o.x = ws_ptr<void>(ws, L.actq);
+      o.w_sf = static_cast<const uint8_t*>(w2) + moe::tiled_weight_bytes_u8(pl.E, pl.H, pl.I);
+      o.x_sf = ws_ptr<void>(ws, L.act_scale);
+    }
     return cuda_status(moe::launch_gemm_swap(l, 1, o, s, b));
   }
   if (!pl.fp8) {
@@ -457,9 +485,16 @@ moe_status_t forward_device(const Plan& pl, const moe_problem_t* p, const void* 
   return forward_after_route(pl, l, hidden, w13, w2, s13, s2, out, ws, num_sms);
 }
 
+// A weight-scale pointer as the problem's format wants it: fp32 (4-byte aligned) for the
+// FP8 formats, NULL for bf16 (ignored) and for MXFP8 (its scales are in the prepared weights).
+bool scale_ok(const Plan& pl, const float* s) {
+  if (pl.mx) return s == nullptr;
+  return !pl.q8 || aligned4(s);
+}
+
 moe_status_t check_weights(const Plan& pl, const void* w13, const void* w2, const float* s13, const float* s2) {
   if (!aligned16(w13) || !aligned16(w2)) return MOE_ERR_INVALID_ARG;
-  if (pl.q8 && (!aligned4(s13) || !aligned4(s2))) return MOE_ERR_INVALID_ARG;
+  if (!scale_ok(pl, s13) || !scale_ok(pl, s2)) return MOE_ERR_INVALID_ARG;
   return MOE_OK;
 }
 
@@ -485,10 +520,10 @@ MOE_API moe_status_t moe_check_problem(const moe_problem_t* problem) {
 MOE_API int32_t moe_padded_intermediate(int32_t intermediate, int32_t activation, int32_t wdtype) {
   if (intermediate <= 0 || intermediate > (1 << 20)) return -1;
   if (activation != MOE_ACT_SWIGLU && activation != MOE_ACT_RELU2 && activation != MOE_ACT_GELU_TANH) return -1;
-  if (wdtype != MOE_DTYPE_BF16 && wdtype != MOE_DTYPE_FP8_BLOCK128 && wdtype != MOE_DTYPE_FP8_PER_TENSOR) return -1;
-  const int a = (wdtype == MOE_DTYPE_FP8_BLOCK128 || wdtype == MOE_DTYPE_FP8_PER_TENSOR || activation == MOE_ACT_RELU2)
-                    ? 128
-                    : 16;
+  if (wdtype != MOE_DTYPE_BF16 && wdtype != MOE_DTYPE_FP8_BLOCK128 && wdtype != MOE_DTYPE_FP8_PER_TENSOR &&
+      wdtype != MOE_DTYPE_MXFP8)
+    return -1;
+  const int a = (wdtype != MOE_DTYPE_BF16 || activation == MOE_ACT_RELU2) ? 128 : 16;
   return (intermediate + a - 1) / a * a;
 }
 
@@ -511,6 +546,7 @@ MOE_API moe_status_t moe_prepare_weights(const moe_problem_t* problem, int32_t i
   Plan pl;
   moe_status_t st = make_plan(problem, &pl);  // num_tokens plays no part in weight preparation
   if (st != MOE_OK) return st;
+  if (pl.mx) return MOE_ERR_INVALID_ARG;  // MXFP8 weights carry scales: moe_prepare_weights_mxfp8
   if (moe_padded_intermediate(intermediate_in, pl.act, problem->wdtype) != pl.I) return MOE_ERR_INVALID_ARG;
   if (pl.q8 && intermediate_in != pl.I) return MOE_ERR_INVALID_ARG;
   if (!aligned16(w13_in) || !aligned16(w13_out) || w2_in == nullptr || w2_out == nullptr)
@@ -543,12 +579,56 @@ MOE_API moe_status_t moe_prepare_weights(const moe_problem_t* problem, int32_t i
 MOE_API size_t moe_prepared_weights_bytes(const moe_problem_t* problem, int32_t which) {
   Plan pl;
   if (make_plan(problem, &pl) != MOE_OK || (which != 0 && which != 1)) return 0;
+  if (pl.mx)
+    return which == 0 ? moe::tiled_weight_bytes_u8(pl.E, pl.N1, pl.H) + moe::tiled_scale_bytes_mx(pl.E, pl.N1, pl.H)
+                      : moe::tiled_weight_bytes_u8(pl.E, pl.H, pl.I) + moe::tiled_scale_bytes_mx(pl.E, pl.H, pl.I);
   if (pl.pt)
     return which == 0 ? moe::tiled_weight_bytes_u8(pl.E, pl.N1, pl.H) : moe::tiled_weight_bytes_u8(pl.E, pl.H, pl.I);
   if (pl.bm == 16)
     return which == 0 ? moe::tiled_weight_bytes(pl.E, pl.N1, pl.H) : moe::tiled_weight_bytes(pl.E, pl.H, pl.I);
   const size_t elt = pl.fp8 ? 1 : 2;
   return which == 0 ? static_cast<size_t>(pl.E) * pl.N1 * pl.H * elt : static_cast<size_t>(pl.E) * pl.H * pl.I * elt;
+}
+
+MOE_API moe_status_t moe_prepare_weights_mxfp8(const moe_problem_t* problem, const void* w13_codes,
+                                               const void* w13_scales, const void* w2_codes, const void* w2_scales,
+                                               void* w13_out, void* w2_out, moe_stream_t stream) {
+  Plan pl;
+  moe_status_t st = make_plan(problem, &pl);  // num_tokens plays no part in weight preparation
+  if (st != MOE_OK) return st;
+  if (!pl.mx) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(w13_codes) || !aligned16(w2_codes) || !aligned16(w13_out) || !aligned16(w2_out) ||
+      w13_scales == nullptr || w2_scales == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  int sms = 0;
+  st = device_sms(&sms);
+  if (st != MOE_OK) return st;
+  const Launch l = launch_of(problem, stream);
+  uint8_t* o13 = static_cast<uint8_t*>(w13_out);
+  uint8_t* o2 = static_cast<uint8_t*>(w2_out);
+  cudaError_t e = moe::launch_tile_weights_u8(l, 0, w13_codes, o13, pl.E, pl.H, pl.I, pl.gated);
+  if (e == cudaSuccess) e = moe::launch_tile_weights_u8(l, 1, w2_codes, o2, pl.E, pl.H, pl.I, pl.gated);
+  if (e == cudaSuccess)
+    e = moe::launch_tile_scales_mx(l, 0, w13_scales, o13 + moe::tiled_weight_bytes_u8(pl.E, pl.N1, pl.H), pl.E, pl.H,
+                                   pl.I, pl.gated);
+  if (e == cudaSuccess)
+    e = moe::launch_tile_scales_mx(l, 1, w2_scales, o2 + moe::tiled_weight_bytes_u8(pl.E, pl.H, pl.I), pl.E, pl.H,
+                                   pl.I, pl.gated);
+  return cuda_status(e);
+}
+
+MOE_API moe_status_t moe_quantize_weights_mxfp8(const void* w, int64_t num_mats, int32_t rows, int32_t cols,
+                                                void* codes, void* scales, moe_stream_t stream) {
+  if (num_mats < 0 || rows <= 0 || cols <= 0 || cols % 32 != 0) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(w) || !aligned16(codes) || scales == nullptr) return MOE_ERR_INVALID_ARG;
+  if (num_mats == 0) return MOE_OK;
+  int sms = 0;
+  moe_status_t st = device_sms(&sms);
+  if (st != MOE_OK) return st;
+  Launch l;
+  l.stream = reinterpret_cast<cudaStream_t>(stream);
+  l.pdl = false;
+  return cuda_status(moe::launch_quant_weights_mx(l, w, num_mats * rows, cols, codes, scales));
 }
 
 MOE_API moe_status_t moe_quantize_weights_fp8(const void* w, int64_t num_mats, int32_t rows, int32_t cols,
@@ -706,7 +786,7 @@ MOE_API moe_status_t moe_stage_gemm1(const moe_problem_t* problem, const void* h
   int sms = 0;
   moe_status_t st = make_plan(problem, &pl);
   if (st != MOE_OK || pl.T == 0) return st;  // T == 0: nothing to do, pointers unused
-  if (!aligned16(hidden) || !aligned16(w13) || (pl.q8 && !aligned4(w13_scale))) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(hidden) || !aligned16(w13) || !scale_ok(pl, w13_scale)) return MOE_ERR_INVALID_ARG;
   st = prologue(problem, workspace, workspace_bytes, &pl, &sms);
   if (st != MOE_OK || pl.T == 0) return st;
   return run_gemm1(pl, hidden, w13, w13_scale, workspace, launch_of(problem, stream), sms);
@@ -718,7 +798,7 @@ MOE_API moe_status_t moe_stage_gemm2(const moe_problem_t* problem, const void* w
   int sms = 0;
   moe_status_t st = make_plan(problem, &pl);
   if (st != MOE_OK || pl.T == 0) return st;  // T == 0: nothing to do, pointers unused
-  if (!aligned16(w2) || (pl.q8 && !aligned4(w2_scale))) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(w2) || !scale_ok(pl, w2_scale)) return MOE_ERR_INVALID_ARG;
   st = prologue(problem, workspace, workspace_bytes, &pl, &sms);
   if (st != MOE_OK || pl.T == 0) return st;
   return run_gemm2(pl, w2, w2_scale, workspace, launch_of(problem, stream), sms);

@@ -40,6 +40,15 @@
 // NemotronH support", section 2: g1_alphas = w13_scale * input_scale, requantised by
 // 1.0 / activation_scale). The kernel is compiled once per operand type.
 //
+// MXFP8 (e4m3 operands, one E8M0 power-of-two scale per 32 values of K on both operands,
+// the block size of the MXFP8 weights of the same page, section 2): tcgen05.mma
+// kind::mxf8f6f4.block_scale applies the scales inside the MMA. Each K step also carries
+// the scale bytes (512 per W chunk, 1024 per X chunk) in the ring; the MMA thread copies
+// them to TMEM with tcgen05.cp (row r's scale for K block k in lane r % 32, column r / 32,
+// byte k) and MMA k of a chunk selects byte k. Row groups have at most 192 rows so that
+// the two accumulators leave 128 TMEM columns for four scale buffers. GEMM1's epilogue
+// writes the bf16 activation, which a separate pass quantises for GEMM2.
+//
 // One persistent CTA per SM, 7 warps:
 //   warp 0      scheduler (tiles from a global atomic counter, published to the other
 //               roles through a shared-memory ring) and W copies;
@@ -64,6 +73,15 @@ constexpr int kTileRing = 4;
 constexpr int kRingReaders = 6;  // MMA, 4 epilogue warps, X producer
 constexpr int kSmemCap = 232448;
 constexpr uint32_t kTmemCols = 2 * kNMax;
+// MXFP8: scale bytes per chunk in the ring, TMEM columns of the accumulators and of the
+// scale buffers (a step of kcs chunks needs 4 kcs columns for W and 4 or 8 per chunk for X)
+constexpr int kSfW = 512;
+constexpr int kSfX = 1024;
+constexpr int kMxAccCols = kMxGroupRows;
+constexpr int kSfBufs = 4;
+constexpr int kSfBufCols = 32;
+constexpr int kSfCol0 = 2 * kMxAccCols;
+static_assert(kSfCol0 + kSfBufs * kSfBufCols <= static_cast<int>(kTmemCols), "TMEM columns");
 
 // Operand ring: a K step takes kc * (16 KB + n * 128) contiguous bytes (W chunks, then X
 // chunks); a step that would cross the end of the ring starts again at its beginning.
@@ -77,7 +95,7 @@ static_assert(kSmemBytes <= kSmemCap, "shared memory");
 
 enum : int {
   kSiteEmpty = 1, kSiteFull = 2, kSiteTmemEmpty = 3, kSiteTmemFull = 4, kSiteTileFull = 5, kSiteTileEmpty = 6,
-  kSiteEmptyX = 7
+  kSiteEmptyX = 7, kSiteSfFree = 8
 };
 
 struct Args {
@@ -99,12 +117,24 @@ struct Args {
   const float* w_scale;    // FP8: per-expert weight scales [E]
   float in_scale;          // FP8 GEMM1: input scale; GEMM2: activation scale (the X scale)
   float act_inv;           // FP8 GEMM1: 1 / activation scale (requantisation of the output)
+  const uint8_t* w_sf;     // MXFP8: tiled weight scales, 512 bytes per (expert, 128-row block, K chunk)
+  const uint8_t* x_sf;     // MXFP8: X scales, 1024 bytes per (16 rows of the group's first row, K chunk)
 };
 
 // K chunks per step for a group of n rows: steps of 48 to 72 KB.
 __host__ __device__ constexpr int chunks_per_step(int n) {
   return n <= 32 ? 4 : (n <= 64 ? 3 : (n <= 128 ? 2 : 1));
 }
+// Ring bytes of one K step of kcs chunks for a group of n rows. MXFP8 steps add the scale
+// blocks of W and X and round up to the 1024-byte period of the swizzle.
+template <bool kMx>
+__device__ __forceinline__ uint32_t step_bytes(int kcs, int n) {
+  const uint32_t b = static_cast<uint32_t>(kcs) * (kTileW + n * kChunkBytes);
+  return kMx ? (b + static_cast<uint32_t>(kcs) * (kSfW + kSfX) + 1023u) & ~1023u : b;
+}
+static_assert(4 * (kTileW + 32 * kChunkBytes + kSfW + kSfX) <= kRingBytes / 2 &&
+                  kTileW + kMxGroupRows * kChunkBytes + kSfW + kSfX <= kRingBytes / 2,
+              "at least two MXFP8 steps fit the ring");
 static_assert(4 * (kTileW + 32 * kChunkBytes) <= kRingBytes / 2 && 2 * (kTileW + 128 * kChunkBytes) <= kRingBytes / 2 &&
                   kTileW + kNMax * kChunkBytes <= kRingBytes / 2,
               "at least two steps fit the ring");
@@ -161,8 +191,12 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
       : "memory");
 }
 
-template <bool kFp8>
+// kKind: 0 bf16, 1 per-tensor e4m3, 2 MXFP8.
+template <int kKind>
 __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
+  constexpr bool kFp8 = kKind == 1;  // scales applied in the epilogue
+  constexpr bool kMx = kKind == 2;   // scales applied by the MMA
+  constexpr int kAccCols = kMx ? kMxAccCols : kNMax;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -252,15 +286,20 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
         const uint8_t* wsrc = a.w + (static_cast<size_t>(e) * a.m_tiles + mt) * a.k_chunks * kTileW;
         for (int c0 = 0; c0 < a.k_chunks; c0 += kc, ++ks) {
           const int kcs = min(kc, a.k_chunks - c0);
-          const uint32_t off = ring_alloc(pos, head, static_cast<uint32_t>(kcs) * (kTileW + n * kChunkBytes));
+          const uint32_t off = ring_alloc(pos, head, step_bytes<kMx>(kcs, n));
           if (!ring_reserve(head, freed, ks, oldest, step_end_w, empty0, abort_flag, a.status, kSiteEmpty)) {
             ok = false;
             break;
           }
           const uint32_t full = full0 + 8 * (ks % kSlots);
           const uint32_t bytes = static_cast<uint32_t>(kcs) * kTileW;
-          mbar_arrive_expect_tx(full, bytes);
+          const uint32_t sf_bytes = kMx ? static_cast<uint32_t>(kcs) * kSfW : 0u;
+          mbar_arrive_expect_tx(full, bytes + sf_bytes);
           bulk_load(s0 + off, wsrc + static_cast<size_t>(c0) * kTileW, bytes, full, pol);
+          if constexpr (kMx)
+            bulk_load(s0 + off + static_cast<uint32_t>(kcs) * (kTileW + n * kChunkBytes),
+                      a.w_sf + ((static_cast<size_t>(e) * a.m_tiles + mt) * a.k_chunks + c0) * kSfW, sf_bytes, full,
+                      pol);
         }
         tile = next;
       }
@@ -281,15 +320,19 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
         const uint8_t* xsrc = a.x + static_cast<size_t>(x_row) * x_row_bytes;
         for (int c0 = 0; c0 < a.k_chunks; c0 += kc, ++ks) {
           const int kcs = min(kc, a.k_chunks - c0);
-          const uint32_t off = ring_alloc(pos, head, static_cast<uint32_t>(kcs) * (kTileW + n * kChunkBytes));
+          const uint32_t off = ring_alloc(pos, head, step_bytes<kMx>(kcs, n));
           if (!ring_reserve(head, freed, ks, oldest, step_end_x, empty0, abort_flag, a.status, kSiteEmptyX)) {
             ok = false;
             break;
           }
           const uint32_t full = full0 + 8 * (ks % kSlots);
           const uint32_t bytes = static_cast<uint32_t>(kcs * n) * kChunkBytes;
-          mbar_arrive_expect_tx(full, bytes);
+          const uint32_t sf_bytes = kMx ? static_cast<uint32_t>(kcs) * kSfX : 0u;
+          mbar_arrive_expect_tx(full, bytes + sf_bytes);
           bulk_load(s0 + off + kcs * kTileW, xsrc + static_cast<size_t>(c0) * n * kChunkBytes, bytes, full, pol);
+          if constexpr (kMx)
+            bulk_load(s0 + off + static_cast<uint32_t>(kcs) * (kTileW + n * kChunkBytes + kSfW),
+                      a.x_sf + (static_cast<size_t>(x_row >> 4) * a.k_chunks + c0) * kSfX, sf_bytes, full, pol);
         }
       }
     }
@@ -307,12 +350,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
         const int acc = it & 1;
         if (!mbar_wait(tempty0 + 8 * acc, ((it >> 1) & 1) ^ 1u, abort_flag, a.status, kSiteTmemEmpty)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + acc * kNMax;
-        const uint32_t idesc = kFp8 ? idesc_e4m3(kMW, n) : idesc_bf16(kMW, n);
+        const uint32_t d_tmem = tmem_base + acc * kAccCols;
+        const uint32_t idesc = kMx ? idesc_mx(kMW, n) : (kFp8 ? idesc_e4m3(kMW, n) : idesc_bf16(kMW, n));
         bool ok = true;
         for (int c0 = 0; c0 < a.k_chunks; c0 += kc, ++ks) {
           const int kcs = min(kc, a.k_chunks - c0);
-          const uint32_t base = s0 + ring_alloc(pos, head, static_cast<uint32_t>(kcs) * (kTileW + n * kChunkBytes));
+          const uint32_t base = s0 + ring_alloc(pos, head, step_bytes<kMx>(kcs, n));
           if (!mbar_wait(full0 + 8 * (ks % kSlots), (ks / kSlots) & 1u, abort_flag, a.status, kSiteFull)) {
             ok = false;
             break;
@@ -323,7 +366,31 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
           const uint32_t a_lo = umma_desc_lo(base);
           const uint32_t b_lo = a_lo + static_cast<uint32_t>(kcs) * (kTileW >> 4);
           const uint32_t b_step = static_cast<uint32_t>(n) * (kChunkBytes >> 4);
-          if (kFp8) {
+          if constexpr (kMx) {
+            // the scale buffer of this step was last read by the MMAs of step ks - kSfBufs
+            if (ks >= static_cast<uint32_t>(kSfBufs) &&
+                !mbar_wait(empty0 + 8 * ((ks - kSfBufs) % kSlots), ((ks - kSfBufs) / kSlots) & 1u, abort_flag,
+                           a.status, kSiteSfFree)) {
+              ok = false;
+              break;
+            }
+            const uint32_t sf_s = base + static_cast<uint32_t>(kcs) * (kTileW + n * kChunkBytes);
+            const uint32_t sf_t = tmem_base + kSfCol0 + (ks % kSfBufs) * kSfBufCols;
+            const int nb = n > 128 ? 2 : 1;  // 128-row scale blocks of X
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              if (c < kcs) {
+                tmem_cp_sf(sf_t + 4 * c, sf_s + c * kSfW);
+                tmem_cp_sf(sf_t + 4 * kcs + 4 * nb * c, sf_s + kcs * kSfW + c * kSfX);
+                if (nb == 2) tmem_cp_sf(sf_t + 4 * kcs + 4 * nb * c + 4, sf_s + kcs * kSfW + c * kSfX + 512);
+              }
+            }
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+              if (c < kcs)
+                umma_mx_chunk(d_tmem, a_lo + c * (kTileW >> 4), b_lo + c * b_step, idesc, sf_t + 4 * c,
+                              sf_t + 4 * kcs + 4 * nb * c, (c0 != 0 || c != 0) ? 1u : 0u);
+          } else if (kFp8) {
             umma_e4m3_chunk(d_tmem, a_lo, b_lo, idesc, c0 != 0);
 #pragma unroll
             for (int c = 1; c < 4; ++c)
@@ -381,7 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
       const bool got = mbar_wait(tfull0 + 8 * acc, (it >> 1) & 1, abort_flag, a.status, kSiteTmemFull);
       if (!__all_sync(0xffffffffu, got)) break;  // leave warp-uniformly (tcgen05.ld is .aligned)
       tc_fence_after();
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * kNMax;
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * kAccCols;
       // GEMM1: this lane's activation feature f lies in K chunk f / 64 (bf16) or f / 128
       // (e4m3) of the activation; byte b of a 128-byte chunk row sits in 16-byte piece
       // (b / 16) ^ (row % 8)
@@ -476,7 +543,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
   }
 }
 
-bool g_attr_set[2][64] = {};
+bool g_attr_set[3][64] = {};
 
 }  // namespace
 
@@ -486,18 +553,22 @@ cudaError_t launch_gemm_swap(const Launch& l, int mode, const SwapOperands& o, c
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  const int fi = o.fp8 ? 1 : 0;
-  if (!g_attr_set[fi][dev]) {
-    err = cudaFuncSetAttribute(o.fp8 ? gemm_swap_kernel<true> : gemm_swap_kernel<false>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  const int kind = o.mx ? 2 : (o.fp8 ? 1 : 0);
+  void (*const kernel)(const Args) =
+      kind == 2 ? gemm_swap_kernel<2> : (kind == 1 ? gemm_swap_kernel<1> : gemm_swap_kernel<0>);
+  if (!g_attr_set[kind][dev]) {
+    err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (err != cudaSuccess) return err;
-    g_attr_set[fi][dev] = true;
+    g_attr_set[kind][dev] = true;
   }
   if ((reinterpret_cast<uintptr_t>(o.w) | reinterpret_cast<uintptr_t>(o.x)) & 15u) return cudaErrorInvalidValue;
+  if (kind == 2 && (o.w_sf == nullptr || o.x_sf == nullptr ||
+                    ((reinterpret_cast<uintptr_t>(o.w_sf) | reinterpret_cast<uintptr_t>(o.x_sf)) & 15u)))
+    return cudaErrorInvalidValue;
   Args a;
   a.mode = mode;
   a.m_tiles = (s.N + kMW - 1) / kMW;
-  const int chunk_elems = o.fp8 ? 128 : 64;  // elements of K in a 128-byte chunk
+  const int chunk_elems = kind != 0 ? 128 : 64;  // elements of K in a 128-byte chunk
   a.k_chunks = (s.K + chunk_elems - 1) / chunk_elems;
   a.k_total = s.k_total;
   a.num_pairs = s.num_pairs;
@@ -516,10 +587,12 @@ cudaError_t launch_gemm_swap(const Launch& l, int mode, const SwapOperands& o, c
   a.w_scale = o.w_scale;
   a.in_scale = o.in_scale;
   a.act_inv = o.act_scale > 0.f ? 1.0f / o.act_scale : 0.f;
+  a.w_sf = static_cast<const uint8_t*>(o.w_sf);
+  a.x_sf = static_cast<const uint8_t*>(o.x_sf);
   cudaLaunchConfig_t cfg;
   cudaLaunchAttribute attr[1];
   make_launch_config(&cfg, attr, l, dim3(s.num_sms), dim3(kThreads), kSmemBytes);
-  return cudaLaunchKernelEx(&cfg, o.fp8 ? gemm_swap_kernel<true> : gemm_swap_kernel<false>, a);
+  return cudaLaunchKernelEx(&cfg, kernel, a);
 }
 
 }  // namespace moe

@@ -5,6 +5,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -341,5 +342,78 @@ __device__ __forceinline__ float gelu_tanh_f32(float g) {
 
 // Gate activation of a gated layer: act 0 = SwiGLU (silu), 2 = gelu_tanh.
 __device__ __forceinline__ float gate_act(float g, int act) { return act == 2 ? gelu_tanh_f32(g) : silu_f32(g); }
+
+// ---- MXFP8 (OCP Microscaling v1.0: E4M3 values, one E8M0 power-of-two scale per 32) ----
+
+// Shared exponent of a block whose largest magnitude is amax: floor(log2(amax)) - 8 (8 is
+// the exponent of E4M3's largest power of two), clamped to [-127, 127]; -127 for an
+// all-zero block. The scale byte is the exponent + 127.
+__device__ __forceinline__ int mx_exponent(float amax) {
+  if (!(amax > 0.f)) return -127;
+  return max(-127, min(127, ilogbf(amax) - 8));
+}
+// 2^-e as an fp32 (e in [-127, 119] for finite bf16 or fp32 inputs: always a normal number),
+// so that x * mx_inv(e) is exact unless the product falls below the normal range.
+__device__ __forceinline__ float mx_inv(int e) { return __int_as_float((127 - min(e, 126)) << 23); }
+// Four values scaled by inv, to E4M3 (round to nearest even, saturating), packed low first.
+__device__ __forceinline__ uint32_t mx_e4m3x4(float a, float b, float c, float d, float inv) {
+  const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a * inv, b * inv), __NV_SATFINITE, __NV_E4M3);
+  const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(c * inv, d * inv), __NV_SATFINITE, __NV_E4M3);
+  return lo | (hi << 16);
+}
+
+// Instruction descriptor for kind::mxf8f6f4.block_scale with e4m3 A/B (both K-major), fp32
+// D and E8M0 scales. The scale-factor byte of A (bits 29-30) and B (bits 4-5) selects which
+// byte of the scale columns this MMA reads: the K block within a 128-element chunk.
+__host__ __device__ constexpr uint32_t idesc_mx(int M, int N) {
+  return (0u << 7)                                   // A format: e4m3
+         | (0u << 10)                                // B format: e4m3
+         | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8
+         | (1u << 23)                                // scale format: E8M0
+         | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
+}
+
+// Shared-memory descriptor of a 32-row x 16-byte block (no swizzle, K-major, rows 16
+// bytes apart: core matrices of 8 rows 128 bytes apart) for tcgen05.cp.
+__device__ __forceinline__ uint64_t sf_block_desc(uint32_t saddr) {
+  uint64_t d = static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>(128 >> 4) << 16;  // leading byte offset (one core matrix wide: unused)
+  d |= static_cast<uint64_t>(128 >> 4) << 32;  // stride byte offset: next 8 rows
+  d |= static_cast<uint64_t>(1) << 46;         // descriptor version
+  return d;
+}
+
+// Copy a 32 x 16-byte block of scale bytes to TMEM columns [col, col + 4) of lanes 0-31,
+// replicated to the four lane quadrants: byte 16 l + 4 j + k lands in lane l (+ 32 q),
+// column col + j, byte k. With row r's scales at l = r % 32, j = r / 32 and byte k = its
+// K block, this is where a block-scaled MMA of M (or N) <= 128 rows reads them.
+__device__ __forceinline__ void tmem_cp_sf(uint32_t taddr, uint32_t saddr) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sf_block_desc(saddr))
+               : "memory");
+}
+
+// One 128-byte K chunk of e4m3 operands with block scales: four MMAs of K = 32; MMA k reads
+// scale byte k of the A columns at sfa and the B columns at sfb. The first accumulates into
+// D when `accumulate` is nonzero, the others always do.
+__device__ __forceinline__ void umma_mx_chunk(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t idesc,
+                                              uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t.reg .b32 al, bl, id;\n\t.reg .b64 a, b;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.eq.b32 q, %4, %4;\n\t"
+      "mov.b64 a, {%1, %5};\n\tmov.b64 b, {%2, %5};\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], a, b, %3, [%6], [%7], p;\n\t"
+      "add.u32 al, %1, 2;\n\tadd.u32 bl, %2, 2;\n\tmov.b64 a, {al, %5};\n\tmov.b64 b, {bl, %5};\n\t"
+      "or.b32 id, %3, 0x20000010;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], a, b, id, [%6], [%7], q;\n\t"
+      "add.u32 al, %1, 4;\n\tadd.u32 bl, %2, 4;\n\tmov.b64 a, {al, %5};\n\tmov.b64 b, {bl, %5};\n\t"
+      "or.b32 id, %3, 0x40000020;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], a, b, id, [%6], [%7], q;\n\t"
+      "add.u32 al, %1, 6;\n\tadd.u32 bl, %2, 6;\n\tmov.b64 a, {al, %5};\n\tmov.b64 b, {bl, %5};\n\t"
+      "or.b32 id, %3, 0x60000030;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], a, b, id, [%6], [%7], q;\n\t}" ::"r"(d_tmem),
+      "r"(a_lo), "r"(b_lo), "r"(idesc), "r"(accumulate), "n"(kUmmaDescHi), "r"(sfa), "r"(sfb)
+      : "memory");
+}
 
 }  // namespace moe

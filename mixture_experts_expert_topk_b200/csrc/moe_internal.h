@@ -97,7 +97,16 @@ struct SwapOperands {
   int fp8;
   const float* w_scale;
   float in_scale, act_scale;
+  // MXFP8 (e4m3 operands with E8M0 scales per 32 values of K, applied by the MMA): mx = 1;
+  // w_sf = the tiled weight scales (512 bytes per 128-row x 128-column tile), x_sf = the X
+  // operand's scales (1024 bytes per 128-column chunk per 16 rows of the group's first row)
+  int mx;
+  const void* w_sf;
+  const void* x_sf;
 };
+// Row groups of the MXFP8 swapped-operand GEMMs: at most this many rows, so that two
+// accumulators leave a quarter of TMEM for the block scales.
+constexpr int kMxGroupRows = 192;
 // N tile for a GEMM with N output columns, given an estimate of the number of 128-row
 // tiles and the SM count (0 if no multiple of 32 divides N).
 int pick_bn(int N, long long est_row_tiles, int num_sms);
@@ -115,6 +124,25 @@ cudaError_t launch_gemm1_fp8(const Launch& l, const void* xq, const CUtensorMap&
                              const CUtensorMap& tm_act_store, const GemmShape& s, const GemmBuffers& b);
 cudaError_t launch_gemm2_fp8(const Launch& l, const CUtensorMap& tm_actq, const CUtensorMap& tm_w2,
                              const CUtensorMap& tm_y_store, const GemmShape& s, const GemmBuffers& b);
+
+// ---- MXFP8 (quant.cu, permute.cu, prepare.cu) ----
+// Codes and E8M0 scale bytes of rows of bf16 values, one scale per 32 columns.
+cudaError_t launch_quant_weights_mx(const Launch& l, const void* w, long long rows, int cols, void* codes,
+                                    void* scales);
+// Hidden rows in row-group order as MXFP8 codes (128-column chunks, like the per-tensor
+// layout) plus their scales: for the group starting at sorted row x_row, chunk c, a
+// 1024-byte block at ((x_row / 16) * H/128 + c) * 1024 holding two 512-byte blocks of 128
+// rows each (byte 16 l + 4 j + k: row 32 j + l, K block 4 c + k).
+cudaError_t launch_permute_mx_rows(const Launch& l, const void* hidden, int H, const int* sorted_pair_ids,
+                                   const int* num_groups, const int2* group_info, int P, int k_total, void* xs,
+                                   void* xs_sf, int num_sms);
+// GEMM1's bf16 activation (row-group order, 64-column chunks) to MXFP8 codes (128-column
+// chunks) and scales in the layout above, for GEMM2.
+cudaError_t launch_act_quant_mx(const Launch& l, const void* act, int I, const int* num_groups,
+                                const int2* group_info, void* actq, void* act_sf, int num_sms);
+size_t tiled_scale_bytes_mx(int E, int rows, int K);
+cudaError_t launch_tile_scales_mx(const Launch& l, int which, const void* in, void* out, int E, int H, int I,
+                                  int gated);
 
 // ---- elementwise (combine.cu, quant.cu, prepare.cu) ----
 cudaError_t launch_combine(const Launch& l, const void* y, const int* pair_to_row, int T, int k_total, int H,

@@ -142,6 +142,126 @@ __global__ void __launch_bounds__(kThreads)
   }
 }
 
+// MXFP8: the same row-group order, each row quantised per 32 columns (OCP Microscaling
+// v1.0: E8M0 exponent floor(log2(amax)) - 8, e4m3 codes of x * 2^-exponent, saturating),
+// with the scale bytes laid out for the block-scaled MMA: the group starting at x_row owns
+// the 1024-byte block ((x_row / 16) * H/128 + c) * 1024 of column chunk c, whose byte
+// 512 h + 16 l + 4 j + k is the scale of group row 128 h + 32 j + l for K block 4 c + k.
+// Lanes 2m and 2m+1 hold the two 16-column pieces of one 32-column block and exchange
+// their maxima with one shuffle; every lane runs every iteration so the shuffles are
+// warp-wide.
+__global__ void __launch_bounds__(kThreads)
+    permute_mx_rows_kernel(const uint4* __restrict__ hidden, int H, const int* __restrict__ sorted_pair_ids,
+                           const int* __restrict__ num_groups, const int2* __restrict__ group_info, int P,
+                           int k_total, uint8_t* __restrict__ xs, uint8_t* __restrict__ xs_sf) {
+  griddep_wait();
+  griddep_launch_dependents();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int G = *num_groups;
+  const int pieces = H / 16, KC = H / 128;
+  for (int g = blockIdx.x; g < G; g += gridDim.x) {
+    const int2 gi = group_info[g];
+    const int x_row = gi.x, n = gi.y >> 16;
+    uint8_t* base = xs + static_cast<size_t>(x_row) * H;
+    uint8_t* sf = xs_sf + static_cast<size_t>(x_row >> 4) * KC * 1024;
+    for (int j0 = kRowsPerCta * blockIdx.y + kRowsPerStep * warp; j0 < min(n, kRowsPerCta * (blockIdx.y + 1));
+         j0 += kRowsPerStep * (kThreads / 32)) {
+      const uint4* src[kRowsPerStep];
+#pragma unroll
+      for (int r = 0; r < kRowsPerStep; ++r) {
+        const int pid = j0 + r < n ? sorted_pair_ids[x_row + j0 + r] : P;
+        src[r] = pid < P ? hidden + static_cast<size_t>(pid / k_total) * (H / 8) : nullptr;
+      }
+      for (int p0 = 0; p0 < pieces; p0 += 32 * kQPieces) {
+        uint4 in[kRowsPerStep][kQPieces][2];
+#pragma unroll
+        for (int r = 0; r < kRowsPerStep; ++r)
+#pragma unroll
+          for (int i = 0; i < kQPieces; ++i) {
+            const int p = p0 + lane + 32 * i;
+            const bool ok = src[r] != nullptr && p < pieces;
+            in[r][i][0] = ok ? __ldg(src[r] + 2 * p) : make_uint4(0u, 0u, 0u, 0u);
+            in[r][i][1] = ok ? __ldg(src[r] + 2 * p + 1) : make_uint4(0u, 0u, 0u, 0u);
+          }
+#pragma unroll
+        for (int r = 0; r < kRowsPerStep; ++r) {
+          const int j = j0 + r;  // warp-uniform
+#pragma unroll
+          for (int i = 0; i < kQPieces; ++i) {
+            const int p = p0 + lane + 32 * i;  // p and p ^ 1 are both inside the row or both past it
+            const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(in[r][i]);
+            float v[16];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const float2 f = __bfloat1622float2(h2[k]);
+              v[2 * k] = f.x;
+              v[2 * k + 1] = f.y;
+            }
+            float amax = 0.f;
+#pragma unroll
+            for (int k = 0; k < 16; ++k) amax = fmaxf(amax, fabsf(v[k]));
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+            const int e = mx_exponent(amax);
+            const float inv = mx_inv(e);
+            if (p < pieces && j < n) {
+              const int c = p >> 3, q = p & 7;
+              *reinterpret_cast<uint4*>(base + static_cast<size_t>(c) * n * 128 + j * 128 + ((q ^ (j & 7)) << 4)) =
+                  make_uint4(mx_e4m3x4(v[0], v[1], v[2], v[3], inv), mx_e4m3x4(v[4], v[5], v[6], v[7], inv),
+                             mx_e4m3x4(v[8], v[9], v[10], v[11], inv), mx_e4m3x4(v[12], v[13], v[14], v[15], inv));
+              if ((lane & 1) == 0) {
+                const int b = p >> 1;  // 32-column block
+                sf[static_cast<size_t>(b >> 2) * 1024 + (j >> 7) * 512 + (j & 31) * 16 + ((j >> 5) & 3) * 4 + (b & 3)] =
+                    static_cast<uint8_t>(e + 127);
+              }
+            }
+          }
+        }
+      }
+    }
+  }
+}
+
+// GEMM1's bf16 activation (row-group order, 64-column chunks of 128-byte rows) to MXFP8
+// codes (128-column chunks) and scales, in the layout of permute_mx_rows_kernel, for
+// GEMM2. A warp converts one 128-column chunk of one row: lane l takes columns 4l..4l+3
+// (8 bytes of bf16 chunk 2c + l/16), eight lanes form a 32-column block.
+__global__ void __launch_bounds__(kThreads)
+    act_quant_mx_kernel(const uint8_t* __restrict__ act, int I, const int* __restrict__ num_groups,
+                        const int2* __restrict__ group_info, uint8_t* __restrict__ actq,
+                        uint8_t* __restrict__ act_sf) {
+  griddep_wait();
+  griddep_launch_dependents();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int G = *num_groups;
+  const int KCb = I / 64, KCq = I / 128;
+  const int warps = gridDim.y * (kThreads / 32);
+  for (int g = blockIdx.x; g < G; g += gridDim.x) {
+    const int2 gi = group_info[g];
+    const int x_row = gi.x, n = gi.y >> 16;
+    const uint8_t* in = act + static_cast<size_t>(x_row) * KCb * 128;
+    uint8_t* out = actq + static_cast<size_t>(x_row) * KCq * 128;
+    uint8_t* sf = act_sf + static_cast<size_t>(x_row >> 4) * KCq * 1024;
+    for (int it = blockIdx.y * (kThreads / 32) + warp; it < n * KCq; it += warps) {
+      const int j = it / KCq, c = it - (it / KCq) * KCq;
+      const int ib = 8 * (lane & 15);  // byte of the bf16 chunk row
+      const uint2 raw = *reinterpret_cast<const uint2*>(in + static_cast<size_t>(2 * c + (lane >> 4)) * n * 128 +
+                                                        j * 128 + ((((ib >> 4) ^ j) & 7) << 4) + (ib & 15));
+      const float2 f01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.x));
+      const float2 f23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.y));
+      float amax = fmaxf(fmaxf(fabsf(f01.x), fabsf(f01.y)), fmaxf(fabsf(f23.x), fabsf(f23.y)));
+#pragma unroll
+      for (int o = 1; o < 8; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+      const int e = mx_exponent(amax);
+      const int ob = 4 * lane;  // byte of the e4m3 chunk row
+      *reinterpret_cast<uint32_t*>(out + static_cast<size_t>(c) * n * 128 + j * 128 + ((((ob >> 4) ^ j) & 7) << 4) +
+                                   (ob & 15)) = mx_e4m3x4(f01.x, f01.y, f23.x, f23.y, mx_inv(e));
+      if ((lane & 7) == 0)
+        sf[static_cast<size_t>(c) * 1024 + (j >> 7) * 512 + (j & 31) * 16 + ((j >> 5) & 3) * 4 + (lane >> 3)] =
+            static_cast<uint8_t>(e + 127);
+    }
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_permute_quant_rows(const Launch& l, const void* hidden, int H, const int* sorted_pair_ids,
@@ -165,6 +285,29 @@ cudaError_t launch_permute_rows(const Launch& l, const void* hidden, int H, cons
   make_launch_config(&cfg, attr, l, dim3(2 * num_sms, 256 / kRowsPerCta), dim3(kThreads), 0);
   return cudaLaunchKernelEx(&cfg, permute_rows_kernel, static_cast<const uint4*>(hidden), H / 8, sorted_pair_ids,
                             num_groups, group_info, P, k_total, static_cast<uint8_t*>(xs));
+}
+
+cudaError_t launch_permute_mx_rows(const Launch& l, const void* hidden, int H, const int* sorted_pair_ids,
+                                   const int* num_groups, const int2* group_info, int P, int k_total, void* xs,
+                                   void* xs_sf, int num_sms) {
+  if (H % 128 != 0) return cudaErrorInvalidValue;
+  cudaLaunchConfig_t cfg;
+  cudaLaunchAttribute attr[1];
+  make_launch_config(&cfg, attr, l, dim3(2 * num_sms, (kMxGroupRows + kRowsPerCta - 1) / kRowsPerCta),
+                     dim3(kThreads), 0);
+  return cudaLaunchKernelEx(&cfg, permute_mx_rows_kernel, static_cast<const uint4*>(hidden), H, sorted_pair_ids,
+                            num_groups, group_info, P, k_total, static_cast<uint8_t*>(xs),
+                            static_cast<uint8_t*>(xs_sf));
+}
+
+cudaError_t launch_act_quant_mx(const Launch& l, const void* act, int I, const int* num_groups,
+                                const int2* group_info, void* actq, void* act_sf, int num_sms) {
+  if (I % 128 != 0) return cudaErrorInvalidValue;
+  cudaLaunchConfig_t cfg;
+  cudaLaunchAttribute attr[1];
+  make_launch_config(&cfg, attr, l, dim3(2 * num_sms, 2), dim3(kThreads), 0);
+  return cudaLaunchKernelEx(&cfg, act_quant_mx_kernel, static_cast<const uint8_t*>(act), I, num_groups,
+                            group_info, static_cast<uint8_t*>(actq), static_cast<uint8_t*>(act_sf));
 }
 
 }  // namespace moe

@@ -131,6 +131,38 @@ __global__ void tile_weights_u8_kernel(const uint4* __restrict__ in, uint4* __re
   }
 }
 
+// MXFP8 weight scales beside the tiled codes: tile (e, m, c) (128 rows, 128 columns of K)
+// has a 512-byte block whose byte 16 l + 4 j + k is the E8M0 scale of tile row 32 j + l for
+// K block 4 c + k, the order in which tcgen05.cp (32 lanes x 16 bytes, replicated to the
+// four lane quadrants) leaves row r's scale for K block k in TMEM lane r % 32, column
+// r / 32, byte k: where the block-scaled MMA reads it. Rows follow the code tiles (gate
+// and up interleaved for w13 of a gated layer); rows or K blocks past the matrix take 0.
+__global__ void tile_scales_mx_kernel(const uint8_t* __restrict__ in, uint8_t* __restrict__ out, long long bytes,
+                                      int which, int rows, int MT, int KC, int KB, int I, int gated) {
+  griddep_wait();
+  for (long long o = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; o < bytes;
+       o += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long t = o >> 9;
+    const int b = static_cast<int>(o & 511);
+    const int l = b >> 4, j = (b >> 2) & 3, k = b & 3;
+    const int c = static_cast<int>(t % KC);
+    const long long tm = t / KC;
+    const int m = static_cast<int>(tm % MT);
+    const long long e = tm / MT;
+    const int r = m * 128 + 32 * j + l;
+    const int kb = 4 * c + k;
+    long long src = -1;
+    if (r < rows) {
+      if (which == 0 && gated) {
+        src = e * 2LL * I + static_cast<long long>(r & 1) * I + (r >> 1);
+      } else {
+        src = e * static_cast<long long>(rows) + r;
+      }
+    }
+    out[o] = (src >= 0 && kb < KB) ? in[src * KB + kb] : static_cast<uint8_t>(0);
+  }
+}
+
 }  // namespace
 
 size_t tiled_weight_bytes_u8(int E, int rows, int K) {
@@ -192,6 +224,24 @@ cudaError_t launch_prepare_w2(const Launch& l, const void* in, void* out, int E,
                               static_cast<uint16_t*>(out), rows, I_in, I_pad);
   return cudaLaunchKernelEx(&cfg, prepare_w2_kernel<uint8_t>, static_cast<const uint8_t*>(in),
                             static_cast<uint8_t*>(out), rows, I_in, I_pad);
+}
+
+size_t tiled_scale_bytes_mx(int E, int rows, int K) {
+  return static_cast<size_t>(E) * ((rows + 127) / 128) * ((K + 127) / 128) * 512;
+}
+
+cudaError_t launch_tile_scales_mx(const Launch& l, int which, const void* in, void* out, int E, int H, int I,
+                                  int gated) {
+  const int rows = which == 0 ? (gated ? 2 * I : I) : H;
+  const int K = which == 0 ? H : I;
+  if (K % 32 != 0) return cudaErrorInvalidValue;
+  const int MT = (rows + 127) / 128, KC = (K + 127) / 128;
+  const long long bytes = static_cast<long long>(tiled_scale_bytes_mx(E, rows, K));
+  cudaLaunchConfig_t cfg;
+  cudaLaunchAttribute attr[1];
+  make_launch_config(&cfg, attr, l, dim3(2048), dim3(256), 0);
+  return cudaLaunchKernelEx(&cfg, tile_scales_mx_kernel, static_cast<const uint8_t*>(in),
+                            static_cast<uint8_t*>(out), bytes, which, rows, MT, KC, K / 32, I, gated);
 }
 
 }  // namespace moe

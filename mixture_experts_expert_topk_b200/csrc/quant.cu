@@ -152,6 +152,42 @@ __global__ void scales_from_amax_kernel(int* __restrict__ amax_bits, long long n
   if (m < num_mats) amax_bits[m] = __float_as_int(scale_of(amax_bits[m]));
 }
 
+// MXFP8 weights (OCP Microscaling v1.0, block 32 along the row): one thread per block,
+// 64 bytes of bf16 in, 32 code bytes and one E8M0 scale byte out. The MXFP8 weight
+// scales of "FlashInfer TRTLLM-Gen MoE kernel optimisation: NemotronH support" (section 2,
+// the MXFP8 alignment helper) hold one scale per 32 values of K.
+__global__ void __launch_bounds__(256)
+    quant_mx_rows_kernel(const uint4* __restrict__ w, long long blocks, uint4* __restrict__ codes,
+                         uint8_t* __restrict__ scales) {
+  griddep_wait();
+  for (long long b = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; b < blocks;
+       b += static_cast<long long>(gridDim.x) * blockDim.x) {
+    float v[32];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint4 raw = w[b * 4 + i];
+      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float2 f = __bfloat1622float2(h[k]);
+        v[8 * i + 2 * k] = f.x;
+        v[8 * i + 2 * k + 1] = f.y;
+      }
+    }
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    const int e = mx_exponent(amax);
+    const float inv = mx_inv(e);
+    uint32_t c[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) c[i] = mx_e4m3x4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3], inv);
+    codes[b * 2] = make_uint4(c[0], c[1], c[2], c[3]);
+    codes[b * 2 + 1] = make_uint4(c[4], c[5], c[6], c[7]);
+    scales[b] = static_cast<uint8_t>(e + 127);
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_quant_weights_per_tensor(const Launch& l, const void* w, int64_t num_mats, int64_t mat_elems,
@@ -201,6 +237,19 @@ cudaError_t launch_quant_weights(const Launch& l, const void* w, int64_t num_mat
   make_launch_config(&cfg, attr, l, dim3(static_cast<unsigned>(blocks)), dim3(256), 0);
   return cudaLaunchKernelEx(&cfg, quant_weights_kernel, static_cast<const uint4*>(w), rows, cols,
                             static_cast<uint2*>(q), scale);
+}
+
+cudaError_t launch_quant_weights_mx(const Launch& l, const void* w, long long rows, int cols, void* codes,
+                                    void* scales) {
+  if (cols % 32 != 0 || rows < 0) return cudaErrorInvalidValue;
+  const long long blocks = rows * (cols / 32);
+  if (blocks == 0) return cudaSuccess;
+  cudaLaunchConfig_t cfg;
+  cudaLaunchAttribute attr[1];
+  make_launch_config(&cfg, attr, l, dim3(static_cast<unsigned>(std::min<long long>((blocks + 255) / 256, 8192))),
+                     dim3(256), 0);
+  return cudaLaunchKernelEx(&cfg, quant_mx_rows_kernel, static_cast<const uint4*>(w), blocks,
+                            static_cast<uint4*>(codes), static_cast<uint8_t*>(scales));
 }
 
 }  // namespace moe

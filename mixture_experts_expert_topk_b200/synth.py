@@ -40,7 +40,8 @@ class MoeConfig:
     num_shared: int = 0    # fused shared-expert slots appended after the routed experts
     # False: bf16. True: e4m3 with 128-wide block scales. "per_tensor": e4m3 with one scale
     # per expert matrix and static input / activation scales (activation_scale below; the
-    # input scale is the hidden rows' amax / 448)
+    # input scale is the hidden rows' amax / 448). "mxfp8": e4m3 with a power-of-two scale
+    # per 32 values of K on both GEMM inputs
     fp8: object = False
     activation_scale: float = 0.03
     hidden_std: float = 1.0
@@ -55,6 +56,10 @@ class MoeConfig:
     @property
     def block128(self) -> bool:
         return self.fp8 is True
+
+    @property
+    def mx(self) -> bool:
+        return self.fp8 == "mxfp8"
 
     @property
     def gated(self) -> bool:
@@ -98,11 +103,17 @@ CONFIGS: Dict[str, MoeConfig] = {
 }
 
 
+# The prefill shape with MXFP8 weights and GEMM inputs.
+CONFIGS["mxfp8_prefill"] = MoeConfig("mxfp8_prefill", T=4096, H=2048, E=256, topk=8, I=512, renormalize=True,
+                                     activation="swiglu", logit_bias_std=0.5, fp8="mxfp8")
+
+
 # A smaller case of the prefill workload for profiler captures: the same shapes per
 # expert (H, I, top-8, about 128 pairs per expert) with 64 experts, so the weights
 # (400 MB) still exceed L2 but a capture holds well under a gigabyte.
 CONFIGS["prefill_e64"] = MoeConfig("prefill_e64", T=1024, H=2048, E=64, topk=8, I=512,
                                    renormalize=True, activation="swiglu", logit_bias_std=0.5)
+CONFIGS["mxfp8_e64"] = CONFIGS["prefill_e64"].replace(name="mxfp8_e64", fp8="mxfp8")
 
 
 def decode_config(T: int) -> MoeConfig:

@@ -87,7 +87,8 @@ def test_padded_intermediate_follows_page_rule(L):
     assert L.moe_padded_intermediate(0, 0, 0) == -1
     assert L.moe_padded_intermediate(200, _capi.MOE_ACT_SWIGLU, _capi.MOE_DTYPE_FP8_PER_TENSOR) == 256
     assert L.moe_padded_intermediate(200, _capi.MOE_ACT_GELU_TANH, 0) == 208
-    assert L.moe_padded_intermediate(200, 0, 3) == -1
+    assert L.moe_padded_intermediate(200, 0, _capi.MOE_DTYPE_MXFP8) == 256   # MXFP8: 128
+    assert L.moe_padded_intermediate(200, 0, 4) == -1
     assert L.moe_padded_intermediate(16, 7, 0) == -1
 
 
@@ -106,8 +107,8 @@ def test_workspace_layout(L):
         # block-128 FP8 to 128-row tiles
         assert bm == (128 if cfg.block128 else 16)
         # the permuted hidden rows (row-group order) exist for the 16-row alignment
-        xs_bytes = lay["group_info"] - lay["xs"]
-        elt = 1 if cfg.per_tensor else 2
+        xs_bytes = lay["xs_scale"] - lay["xs"]
+        elt = 1 if (cfg.per_tensor or cfg.mx) else 2
         assert xs_bytes == (-(-lay["max_rows"] * cfg.H * elt // 1024) * 1024 if not cfg.block128 else 0)
         assert lay["max_rows"] == -(-(P + min(E, P) * (bm - 1)) // bm) * bm
         assert lay["num_chunks"] == -(-P // 2048)
@@ -196,3 +197,34 @@ def test_per_tensor_fp8_problem_rules(L):
     assert L.moe_check_problem(ctypes.byref(p)) == 2          # 128-row tiles: not for per-tensor
     p = moe.make_problem(64, 256, 8, 2, 200, fp8="per_tensor", input_scale=0.01, activation_scale=0.05)
     assert L.moe_check_problem(ctypes.byref(p)) == 1          # I must be padded to 128
+
+
+def test_mxfp8_problem_rules(L):
+    ok = moe.make_problem(64, 256, 8, 2, 256, fp8="mxfp8")
+    assert L.moe_check_problem(ctypes.byref(ok)) == 0
+    lay = moe.workspace_layout(ok)
+    assert lay["block_m"] == 16
+    # e4m3 tiles of 128 x 128 plus one 512-byte scale block per tile: w13 [8, 512, 256], w2 [8, 256, 256]
+    assert L.moe_prepared_weights_bytes(ctypes.byref(ok), 0) == 8 * 4 * 2 * (16384 + 512)
+    assert L.moe_prepared_weights_bytes(ctypes.byref(ok), 1) == 8 * 2 * 2 * (16384 + 512)
+    # scale blocks of the permuted hidden rows and of the activation: 1024 bytes per 16 rows
+    # per 128 columns
+    assert lay["group_info"] - lay["xs_scale"] >= lay["max_rows"] // 16 * 2 * 1024
+    assert lay["y"] - lay["act_scale"] >= lay["max_rows"] // 16 * 2 * 1024
+    assert lay["act_scale"] - lay["actq"] >= lay["max_rows"] * 256
+    p = moe.make_problem(64, 256, 8, 2, 256, fp8="mxfp8", block_m=128)
+    assert L.moe_check_problem(ctypes.byref(p)) == 2          # 128-row tiles: not for MXFP8
+    p = moe.make_problem(64, 256, 8, 2, 200, fp8="mxfp8")
+    assert L.moe_check_problem(ctypes.byref(p)) == 1          # I must be padded to 128
+    fake = ctypes.c_void_p(1 << 20)
+    s = ctypes.c_void_p(0)
+    n = moe.workspace_size(ok)
+    # the scales travel inside the prepared weights: scale pointers must be NULL
+    assert L.moe_forward(ctypes.byref(ok), fake, fake, fake, fake, fake, None, ctypes.c_void_p(3 << 20),
+                         ctypes.c_void_p(4 << 20), n, s) == 1
+    # the generic preparation refuses MXFP8; the MXFP8 one refuses other formats and missing scales
+    assert L.moe_prepare_weights(ctypes.byref(ok), 256, fake, fake, fake, fake, s) == 1
+    assert L.moe_prepare_weights_mxfp8(ctypes.byref(_prob()), fake, fake, fake, fake, fake, fake, s) == 1
+    assert L.moe_prepare_weights_mxfp8(ctypes.byref(ok), fake, None, fake, fake, fake, fake, s) == 1
+    assert L.moe_quantize_weights_mxfp8(fake, 1, 4, 48, fake, fake, s) == 1   # 32-column blocks
+    assert L.moe_quantize_weights_mxfp8(fake, 0, 4, 64, fake, fake, s) == 0

@@ -532,3 +532,139 @@ def test_fp8_per_tensor_layer_parity(name):
     e = err_beyond_rounding(got, ref)
     print(f"{name}: beyond-rounding {e:.4f}, raw {max_err_over_rms(got, ref):.4f}")
     assert e <= FP8_TOL, e
+
+
+# ---- MXFP8 ------------------------------------------------------------------------------
+
+MX_SMALL = {
+    "mx_swiglu": _small("mx_swiglu", T=300, H=256, E=8, topk=2, I=256, fp8="mxfp8"),
+    "mx_relu2": _small("mx_relu2", T=200, H=384, E=6, topk=3, I=384, activation="relu2", renormalize=False,
+                       fp8="mxfp8"),
+    "mx_gelu_shared": _small("mx_gelu_shared", T=130, H=256, E=12, topk=3, I=256, num_shared=1,
+                             activation="gelu_tanh", fp8="mxfp8"),
+    # row groups of 129-192 rows (two 128-row scale blocks per chunk, one K chunk per step)
+    # and three align chunks
+    "mx_big_groups": _small("mx_big_groups", T=1500, H=256, E=4, topk=2, I=128, fp8="mxfp8"),
+    "mx_decode": _small("mx_decode", T=4, H=512, E=32, topk=4, I=256, fp8="mxfp8"),
+}
+
+
+def _mx_group_scales(sf_flat, group_info, num_groups, rows, kchunks):
+    """[rows, 4 * kchunks] scale bytes from the row-group scale blocks: the group at x_row
+    owns the 1024-byte block ((x_row / 16) * kchunks + c) * 1024 of chunk c, whose byte
+    512 h + 16 l + 4 j + k is the scale of group row 128 h + 32 j + l for K block 4 c + k."""
+    flat = np.asarray(sf_flat).reshape(-1)
+    out = np.zeros((rows, 4 * kchunks), dtype=np.uint8)
+    for g in range(num_groups):
+        x_row, meta = int(group_info[g][0]), int(group_info[g][1])
+        n = meta >> 16
+        for r in range(n):
+            for c in range(kchunks):
+                base = ((x_row // 16) * kchunks + c) * 1024 + (r // 128) * 512 + (r % 32) * 16 + ((r // 32) % 4) * 4
+                out[x_row + r, 4 * c:4 * c + 4] = flat[base:base + 4]
+    return out
+
+
+def _mx_weight_scales(flat, E, rows, K, gated):
+    """The tiled weight scale blocks back to the checkpoint layout [E, rows, K/32] (gated w13
+    rows un-interleaved)."""
+    MT, KC = -(-rows // 128), -(-K // 128)
+    t = np.asarray(flat).reshape(E, MT, KC, 32, 4, 4)            # [e, m, c, l, j, k]
+    s = t.transpose(0, 1, 4, 3, 2, 5).reshape(E, MT * 128, KC * 4)  # row 128 m + 32 j + l, block 4 c + k
+    s = s[:, :rows, :K // 32]
+    if gated:
+        I = rows // 2
+        s = np.concatenate([s[:, 0::2], s[:, 1::2]], axis=1)      # [gate0, up0, ...] -> gate rows, up rows
+        assert s.shape[1] == 2 * I
+    return s
+
+
+@pytest.mark.parametrize("name", list(MX_SMALL))
+def test_mxfp8_layer_parity(name):
+    cfg = MX_SMALL[name]
+    inp = make_inputs(cfg, 0)
+    dev = torch.device("cuda:0")
+    hidden, logits = inp["hidden"].to(dev), inp["logits"].to(dev)
+    # device quantiser, bit-exact against the oracle's (OCP MX conversion decided in fp32)
+    q13, s13 = moe.quantize_weights_mxfp8(inp["w13"].to(dev))
+    q2, s2 = moe.quantize_weights_mxfp8(inp["w2"].to(dev))
+    o13, os13, o2, os2 = O.quantize_weights_mxfp8(bits(inp["w13"]), bits(inp["w2"]))
+    np.testing.assert_array_equal(q13.cpu().numpy(), o13)
+    np.testing.assert_array_equal(s13.cpu().numpy(), os13)
+    np.testing.assert_array_equal(q2.cpu().numpy(), o2)
+    np.testing.assert_array_equal(s2.cpu().numpy(), os2)
+    prob = moe.make_problem(cfg.T, cfg.H, cfg.E, cfg.topk, cfg.I, renormalize=cfg.renormalize,
+                            activation=cfg.activation, num_shared=cfg.num_shared, fp8="mxfp8")
+    w13p, w2p = moe.prepare_weights(prob, q13, q2, cfg.I, w13_scale=s13, w2_scale=s2)
+    # prepared layout: the codes as the per-tensor tiles, then one scale block per tile
+    E, N1 = cfg.E_total, cfg.N1
+    c13 = 16384 * E * (-(-N1 // 128)) * (cfg.H // 128)
+    c2 = 16384 * E * (cfg.H // 128) * (cfg.I // 128)
+    np.testing.assert_array_equal(_mx_weight_scales(w13p[c13:].cpu().numpy(), E, N1, cfg.H, cfg.gated), os13)
+    np.testing.assert_array_equal(_mx_weight_scales(w2p[c2:].cpu().numpy(), E, cfg.H, cfg.I, False), os2)
+    ws = moe.new_workspace(prob)
+    out = moe.moe_forward(hidden, logits, w13p, w2p, cfg.topk, cfg.renormalize, cfg.activation,
+                          num_shared=cfg.num_shared, workspace=ws)
+    torch.cuda.synchronize()
+    assert moe.device_status(ws)[0] == 0
+    raw = moe.read_workspace(prob, ws)
+    act_bits = raw.pop("act").view(torch.int16).cpu().numpy().view(np.uint16)
+    parts = {k: v.cpu().numpy() for k, v in raw.items()}
+    ids_o, _ = O.route(inp["logits"].numpy(), cfg.topk, cfg.renormalize, cfg.num_shared)
+    np.testing.assert_array_equal(parts["topk_ids"], ids_o)
+    al = O.align(ids_o, cfg.E_total, 16)
+    P_pad = int(al["P_pad"])
+    np.testing.assert_array_equal(parts["sorted_pair_ids"][:P_pad], al["sorted_pair_ids"])
+    ng = int(parts["num_blocks"][1])
+    gi = parts["group_info"]
+    assert max(int(gi[g][1]) >> 16 for g in range(ng)) <= 192
+    # the permuted hidden rows: MXFP8 codes and scale bytes, bit for bit
+    pids = al["sorted_pair_ids"][:P_pad]
+    real = pids < cfg.T * cfg.k_total
+    xq, xsc = O.quant_mx(O.bf16_bits_to_f32(bits(inp["hidden"])))
+    xs = _untile_u8(parts["xs"], gi, ng, P_pad, cfg.H // 128)
+    np.testing.assert_array_equal(xs[real], xq[pids[real] // cfg.k_total])
+    assert np.all(xs[~real] == 0)
+    xss = _mx_group_scales(parts["xs_scale"], gi, ng, P_pad, cfg.H // 128)
+    np.testing.assert_array_equal(xss[real], xsc[pids[real] // cfg.k_total])
+    assert np.all(xss[~real] == 0)
+    # GEMM2's input: the kernel's own bf16 activation quantised per 32, bit for bit
+    act = untile_groups(act_bits, gi, ng, P_pad, -(-cfg.I // 64))[:, :cfg.I]
+    aq, asc = O.quant_mx(O.bf16_bits_to_f32(act))
+    np.testing.assert_array_equal(_untile_u8(parts["actq"], gi, ng, P_pad, cfg.I // 128), aq)
+    np.testing.assert_array_equal(_mx_group_scales(parts["act_scale"], gi, ng, P_pad, cfg.I // 128), asc)
+    # the layer
+    ref = O.moe_forward_mxfp8(bits(inp["hidden"]), inp["logits"].numpy(), o13, os13, o2, os2, topk=cfg.topk,
+                              renormalize=cfg.renormalize, activation=cfg.activation, num_shared=cfg.num_shared)
+    got = bf16_to_f64(out)
+    assert np.all(np.isfinite(got))
+    e = err_beyond_rounding(got, ref)
+    print(f"{name}: beyond-rounding {e:.4f}, raw {max_err_over_rms(got, ref):.4f}")
+    assert e <= FP8_TOL, e
+
+
+def test_mxfp8_full_size_sampled_tokens():
+    """The MXFP8 prefill workload at full size against the oracle on sampled tokens."""
+    cfg = CONFIGS["mxfp8_prefill"]
+    inp = make_inputs(cfg, 0)
+    dev = torch.device("cuda:0")
+    q13, s13 = moe.quantize_weights_mxfp8(inp["w13"].to(dev))
+    q2, s2 = moe.quantize_weights_mxfp8(inp["w2"].to(dev))
+    prob = moe.make_problem(cfg.T, cfg.H, cfg.E, cfg.topk, cfg.I, renormalize=cfg.renormalize,
+                            activation=cfg.activation, fp8="mxfp8")
+    w13p, w2p = moe.prepare_weights(prob, q13, q2, cfg.I, w13_scale=s13, w2_scale=s2)
+    ws = moe.new_workspace(prob)
+    out = moe.moe_forward(inp["hidden"].to(dev), inp["logits"].to(dev), w13p, w2p, cfg.topk, cfg.renormalize,
+                          cfg.activation, workspace=ws)
+    torch.cuda.synchronize()
+    assert moe.device_status(ws)[0] == 0
+    tokens = np.random.default_rng(5).choice(cfg.T, 24, replace=False)
+    ids, _ = O.route(inp["logits"].numpy()[tokens], cfg.topk, cfg.renormalize)
+    experts = sorted(set(int(e) for e in ids.reshape(-1)))
+    o13, os13, o2, os2 = O.quantize_weights_mxfp8(bits(inp["w13"]), bits(inp["w2"]), experts=experts)
+    ref = O.moe_forward_mxfp8(bits(inp["hidden"]), inp["logits"].numpy(), o13, os13, o2, os2, topk=cfg.topk,
+                              renormalize=cfg.renormalize, activation=cfg.activation, tokens=tokens)
+    got = bf16_to_f64(out.cpu()[torch.from_numpy(tokens)])
+    e = err_beyond_rounding(got, ref)
+    print(f"mxfp8_prefill: beyond-rounding {e:.4f} on {len(tokens)} tokens")
+    assert e <= FP8_TOL, e
