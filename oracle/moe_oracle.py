@@ -696,6 +696,139 @@ def moe_forward_mxfp8(hidden_bits: np.ndarray, logits: Optional[np.ndarray], w13
     return out
 
 
+# --------------------------------------------------------------------------
+# NVFP4: E2M1 values, an E4M3 scale per 16, an fp32 scale per tensor
+# --------------------------------------------------------------------------
+
+NVFP4_BLOCK = 16
+E2M1_MAX = 6.0
+
+
+def e2m1_encode(x: np.ndarray) -> np.ndarray:
+    """Encode float32 values as FP4 E2M1 codes (uint8 0..15).
+
+    Format: 1 sign bit (bit 3), 2 exponent bits with bias 1, 1 mantissa bit; magnitudes
+    0, 0.5 (exponent field 0: subnormal), 1, 1.5, 2, 3, 4, 6. Round to nearest, ties to the
+    even code (the one whose mantissa bit is 0); magnitudes beyond 6 saturate to 6. The sign
+    of zero is kept. Finite inputs only.
+    """
+    x = np.asarray(x, dtype=np.float32)
+    a = np.abs(x).astype(np.float64)
+    _, ex = np.frexp(a)
+    e = np.maximum(ex.astype(np.int64) - 1, 0)        # exponent of a, subnormal range below 1
+    quantum = np.ldexp(1.0, (e - 1).astype(np.int32))  # spacing: 0.5 below 2, then 1, then 2
+    r = np.minimum(np.rint(a / quantum) * quantum, E2M1_MAX)
+    # r -> code: 0 -> 0, 0.5 -> 1, then 2 codes per power of two
+    _, ex2 = np.frexp(r)
+    e2 = ex2.astype(np.int64) - 1
+    code = np.where(r == 0, 0, np.where(r == 0.5, 1, 2 * (e2 + 1) + (r / np.ldexp(1.0, e2.astype(np.int32)) > 1)))
+    return (code.astype(np.uint8) | (np.signbit(x).astype(np.uint8) << 3)).astype(np.uint8)
+
+
+def e2m1_decode(codes: np.ndarray) -> np.ndarray:
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    mag = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])[c & 7]
+    return np.where(c & 8, -mag, mag)
+
+
+def nvfp4_global_scale(amax) -> np.float32:
+    """Per-tensor decode scale: amax / (6 * 448), so that every block scale fits E4M3; 1 for
+    an all-zero tensor. fp32."""
+    amax = np.float32(amax)
+    return np.float32(1.0) if amax == 0 else np.float32(amax / np.float32(E2M1_MAX * E4M3_MAX))
+
+
+def quant_nvfp4(x: np.ndarray, global_scale):
+    """NVFP4 quantisation along the last axis with the tensor's fp32 decode scale g.
+
+    The pages name NVFP4 weights ("FlashInfer gated MoE kernel optimisation for
+    Blackwell", section 4; the NVFP4 results of [TRTLLM]) without printing the format.
+    Reading taken: NVIDIA's published NVFP4 — E2M1 values, one E4M3 scale per 16 consecutive
+    values of K and one fp32 scale per tensor — with, per block, in fp32:
+      block scale  s = e4m3(amax / 6 / g)            (round to nearest even, saturating);
+      elements     q = e2m1(x / (decode(s) * g))     (0 when the block scale decodes to 0);
+      value        decode(q) * decode(s) * g.
+    Returns (codes uint8 [..., K] holding one E2M1 code each, scale codes uint8 [..., K/16]).
+    """
+    x = np.asarray(x, dtype=np.float32)
+    K = x.shape[-1]
+    assert K % NVFP4_BLOCK == 0
+    g = np.float32(global_scale)
+    b = x.reshape(x.shape[:-1] + (K // NVFP4_BLOCK, NVFP4_BLOCK))
+    amax = np.abs(b).max(axis=-1).astype(np.float32)
+    s_code = e4m3_encode((amax / np.float32(E2M1_MAX) / g).astype(np.float32))
+    denom = (e4m3_decode(s_code).astype(np.float32) * g).astype(np.float32)
+    safe = np.where(denom > 0, denom, np.float32(1.0)).astype(np.float32)
+    scaled = np.where(denom[..., None] > 0, (b / safe[..., None]).astype(np.float32), np.float32(0.0))
+    codes = e2m1_encode(scaled.astype(np.float32)).reshape(x.shape)
+    return codes, s_code
+
+
+def dequant_nvfp4(codes: np.ndarray, scale_codes: np.ndarray, global_scale) -> np.ndarray:
+    s = np.repeat(e4m3_decode(scale_codes), NVFP4_BLOCK, axis=-1)
+    return e2m1_decode(codes) * s * np.float64(np.float32(global_scale))
+
+
+def quantize_weights_nvfp4(w13_bits, w2_bits, experts=None):
+    """NVFP4 weights: per expert matrix a global scale from its amax, then ``quant_nvfp4``
+    along K. Returns (w13 codes, w13 block scales, w13 global scales [E], the same for w2)."""
+    out = []
+    for wb in (w13_bits, w2_bits):
+        wb = np.asarray(wb)
+        E, R, C = wb.shape
+        q = np.zeros((E, R, C), dtype=np.uint8)
+        sc = np.zeros((E, R, C // NVFP4_BLOCK), dtype=np.uint8)
+        gs = np.ones(E, dtype=np.float32)
+        for e in (range(E) if experts is None else experts):
+            w = bf16_bits_to_f32(wb[e])
+            gs[e] = nvfp4_global_scale(np.abs(w).max())
+            q[e], sc[e] = quant_nvfp4(w, gs[e])
+        out += [q, sc, gs]
+    return tuple(out)
+
+
+def moe_forward_nvfp4(hidden_bits: np.ndarray, logits: Optional[np.ndarray], w13_q, w13_sc, w13_g, w2_q, w2_sc,
+                      w2_g, input_scale, activation_scale, *, topk: int, renormalize: bool, activation: str,
+                      num_shared: int = 0, tokens: Optional[Sequence[int]] = None, routing=None):
+    """NVFP4 W4A4 layer forward in float64.
+
+    Reading taken (see ``quant_nvfp4``): the weights carry their own global scales; the two
+    GEMM inputs are quantised with the static per-tensor global scales ``input_scale`` (the
+    hidden rows) and ``activation_scale`` (GEMM1's activation, stored in bf16 first), the
+    static input / activation scales of the per-tensor algebra of [TRTLLM] section 2, and
+    dynamic E4M3 block scales per 16. Products use the exactly dequantised values.
+    """
+    if routing is not None:
+        ids, w = (np.asarray(routing[0], dtype=np.int32), np.asarray(routing[1], dtype=np.float32))
+        if tokens is not None:
+            tokens = np.asarray(tokens, dtype=np.int64)
+            hidden_bits = np.asarray(hidden_bits)[tokens]
+            ids, w = ids[tokens], w[tokens]
+    else:
+        logits = np.asarray(logits, dtype=np.float32)
+        if tokens is not None:
+            tokens = np.asarray(tokens, dtype=np.int64)
+            hidden_bits = np.asarray(hidden_bits)[tokens]
+            logits = logits[tokens]
+        ids, w = route(logits, topk, renormalize, num_shared)
+    x = dequant_nvfp4(*quant_nvfp4(bf16_bits_to_f32(hidden_bits), input_scale), input_scale)
+    T, kk = ids.shape
+    H = x.shape[1]
+    I = w2_q.shape[2]
+    y = np.zeros((T, kk, H), dtype=np.float64)
+    for e in np.unique(ids):
+        t_idx, j_idx = np.nonzero(ids == e)
+        W13 = dequant_nvfp4(np.asarray(w13_q[e]), np.asarray(w13_sc[e]), w13_g[e])
+        W2 = dequant_nvfp4(np.asarray(w2_q[e]), np.asarray(w2_sc[e]), w2_g[e])
+        a = activation_fn(x[t_idx] @ W13.T, activation, I)
+        ad = dequant_nvfp4(*quant_nvfp4(round_to_bf16(a), activation_scale), activation_scale)
+        y[t_idx, j_idx] = w[t_idx, j_idx].astype(np.float64)[:, None] * (ad @ W2.T)
+    out = np.zeros((T, H), dtype=np.float64)
+    for j in range(kk):
+        out += y[:, j]
+    return out
+
+
 def rms(x: np.ndarray) -> float:
     x = np.asarray(x, dtype=np.float64)
     return math.sqrt(float(np.mean(x * x))) if x.size else 0.0

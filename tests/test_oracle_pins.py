@@ -627,6 +627,113 @@ def test_mxfp8_layer_against_torch_casts(act):
 
 
 # --------------------------------------------------------------------------
+# NVFP4 (E2M1 values, E4M3 scale per 16, fp32 scale per tensor)
+# --------------------------------------------------------------------------
+
+# the E2M1 grid (sign bit 3, exponent bias 1, one mantissa bit): code -> value
+E2M1_TABLE = {0: 0.0, 1: 0.5, 2: 1.0, 3: 1.5, 4: 2.0, 5: 3.0, 6: 4.0, 7: 6.0}
+
+
+def _e2m1_brute(v: float) -> int:
+    """Nearest grid magnitude by exhaustive search; on a tie the code with mantissa bit 0."""
+    a = min(abs(v), 6.0)
+    best = min(E2M1_TABLE, key=lambda c: (abs(a - E2M1_TABLE[c]), c & 1))
+    return best | (8 if math.copysign(1.0, v) < 0 else 0)
+
+
+def test_e2m1_decode_table_and_brute_force_encode():
+    np.testing.assert_array_equal(O.e2m1_decode(np.arange(16, dtype=np.uint8)),
+                                  [0, .5, 1, 1.5, 2, 3, 4, 6, -0.0, -.5, -1, -1.5, -2, -3, -4, -6])
+    # every tie point, every grid point, values around them and beyond the range
+    pts = sorted(set(E2M1_TABLE.values()))
+    mids = [(a + b) / 2 for a, b in zip(pts, pts[1:])]
+    vals = pts + mids + [m + d for m in mids for d in (-1e-3, 1e-3)] + [6.5, 7.0, 100.0, 1e-30]
+    vals = np.array(vals + [-v for v in vals] + [-0.0], dtype=np.float32)
+    rng = np.random.default_rng(47)
+    vals = np.concatenate([vals, (rng.standard_normal(4000) * 3).astype(np.float32)])
+    got = O.e2m1_encode(vals)
+    want = np.array([_e2m1_brute(float(v)) for v in vals], dtype=np.uint8)
+    np.testing.assert_array_equal(got, want)
+    # hand-picked ties: 0.25 -> 0, 0.75 -> 1.0, 1.25 -> 1.0, 1.75 -> 2, 2.5 -> 2, 3.5 -> 4, 5 -> 4
+    t = O.e2m1_encode(np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0], np.float32))
+    assert t.tolist() == [0, 2, 2, 4, 4, 6, 6]
+
+
+def test_quant_nvfp4_definition():
+    rng = np.random.default_rng(53)
+    x = (rng.standard_normal((4, 64)) * np.exp2(rng.integers(-6, 6, (4, 1)))).astype(np.float32)
+    x[1, 16:32] = 0.0
+    g = O.nvfp4_global_scale(np.abs(x).max())
+    assert g == np.float32(np.float32(np.abs(x).max()) / np.float32(2688.0))
+    q, s = O.quant_nvfp4(x, g)
+    assert q.shape == x.shape and s.shape == (4, 4)
+    for r in range(4):
+        for b in range(4):
+            blk = x[r, 16 * b:16 * b + 16]
+            amax = np.float32(np.abs(blk).max())
+            sc = torch.tensor([float(np.float32(np.float32(amax / np.float32(6.0)) / g))]).to(torch.float8_e4m3fn)
+            assert int(s[r, b]) == int(sc.view(torch.uint8).item())
+            den = np.float32(np.float32(sc.to(torch.float32).item()) * g)
+            want = [(_e2m1_brute(float(np.float32(v / den))) if den > 0 else 0) for v in blk]
+            assert q[r, 16 * b:16 * b + 16].tolist() == want
+    assert np.all(q[1, 16:32] == 0) and s[1, 1] == 0
+    # dequantisation stays within half an E2M1 step of the scaled value plus the block-scale error
+    d = O.dequant_nvfp4(q, s, g)
+    assert np.all(np.abs(d - x) <= 0.25 * np.abs(x) + np.repeat(O.e4m3_decode(s), 16, 1) * g * 0.26 + 1e-30)
+    # the tensor's largest value keeps its block at E2M1's top: code 6.0 (7) when 6 * s * g reaches it
+    i = np.unravel_index(np.argmax(np.abs(x)), x.shape)
+    assert (q[i] & 7) in (6, 7)
+
+
+@pytest.mark.parametrize("act", ["swiglu", "relu2"])
+def test_nvfp4_layer_against_dense_restatement(act):
+    rng = np.random.default_rng(59)
+    T, H, E, k, I = 5, 128, 3, 2, 64
+    N1 = I if act == "relu2" else 2 * I
+    x = _bf16_bits(torch.from_numpy(rng.standard_normal((T, H)).astype(np.float32)))
+    l = rng.standard_normal((T, E)).astype(np.float32)
+    w13 = _bf16_bits(torch.from_numpy(0.02 * rng.standard_normal((E, N1, H)).astype(np.float32)))
+    w2 = _bf16_bits(torch.from_numpy(0.02 * rng.standard_normal((E, H, I)).astype(np.float32)))
+    q13, s13, g13, q2, s2, g2 = O.quantize_weights_nvfp4(w13, w2)
+    g_in, g_act = np.float32(0.002), np.float32(0.0004)
+    got = O.moe_forward_nvfp4(x, l, q13, s13, g13, q2, s2, g2, g_in, g_act, topk=k, renormalize=True,
+                              activation=act)
+
+    def fp4(a, g):  # per row, per 16: torch E4M3 block scale, brute-force E2M1 values
+        a = np.asarray(a, np.float32)
+        out = np.zeros(a.shape)
+        for idx in np.ndindex(a.shape[:-1]):
+            row = a[idx]
+            for b in range(row.shape[0] // 16):
+                blk = row[16 * b:16 * b + 16]
+                sc = torch.tensor([float(np.float32(np.float32(np.abs(blk).max() / np.float32(6)) / g))]).to(
+                    torch.float8_e4m3fn).to(torch.float32).item()
+                den = np.float32(np.float32(sc) * g)
+                for i, v in enumerate(blk):
+                    c = _e2m1_brute(float(np.float32(v / den))) if den > 0 else 0
+                    # the value is exact: code * block scale * global scale, in float64
+                    out[idx][16 * b + i] = (-1 if c & 8 else 1) * E2M1_TABLE[c & 7] * sc * float(g)
+        return out
+
+    W13 = [fp4(O.bf16_bits_to_f32(w13[e]), g13[e]) for e in range(E)]
+    W2 = [fp4(O.bf16_bits_to_f32(w2[e]), g2[e]) for e in range(E)]
+    Xd = fp4(O.bf16_bits_to_f32(x), g_in)
+    ids, wts = _route_brute(l, k, True)
+    want = np.zeros((T, H))
+    for t in range(T):
+        for j in range(k):
+            e = ids[t, j]
+            z = W13[e] @ Xd[t]
+            a = np.maximum(z, 0) ** 2 if act == "relu2" else z[:I] / (1 + np.exp(-z[:I])) * z[I:]
+            a16 = torch.from_numpy(a.astype(np.float32)).to(torch.bfloat16).to(torch.float32).numpy()
+            want[t] += np.float64(np.float32(wts[t, j])) * (W2[e] @ fp4(a16[None], g_act)[0])
+    np.testing.assert_allclose(got, want, rtol=1e-9, atol=1e-12)
+    # per-expert global scales: amax / (6 * 448)
+    np.testing.assert_array_equal(g13, (np.abs(O.bf16_bits_to_f32(w13).reshape(E, -1)).max(1) / np.float32(2688))
+                                  .astype(np.float32))
+
+
+# --------------------------------------------------------------------------
 # planted mistakes: each mutated oracle must fail a pin above
 # --------------------------------------------------------------------------
 
