@@ -342,6 +342,46 @@ moe_status_t moe_align_noalloc(const moe_problem_t* problem, const int32_t* topk
                                int32_t* block_expert, int32_t* pair_to_row, int32_t* num_blocks,
                                moe_stream_t stream);
 
+/* Expert parallelism over `world` ranks (one process per GPU): rank r owns the routed
+ * experts [r*E_r/world, (r+1)*E_r/world) (E_r a multiple of world) and a copy of the shared
+ * expert, which serves its own rank's tokens. ("W4A8 grouped GEMM optimisation for GLM-5.2
+ * MoE on H200", sglang PR 38220, introduction, tunes for EP-8 layouts; the contiguous split and
+ * the replicated shared expert are this library's reading.) A forward is: route this rank's T tokens
+ * (moe_stage_route), moe_ep_dispatch, an all-to-all of the send segments, the routed forward
+ * on the received rows (moe_forward_routed with topk 1 and the rank's E_r/world routed experts
+ * plus the shared copy as local experts 0..E_r/world), the reverse all-to-all of the weighted
+ * output rows, and moe_ep_combine. `problem` describes the layer on this rank's tokens.
+ *
+ * Bytes of the dispatch workspace (0 for an invalid problem or world) and the largest
+ * number of send rows (-1 if invalid): round_up(T*k' + min(T*k', world)*15, 16). Host only. */
+size_t moe_ep_workspace_size(const moe_problem_t* problem, int32_t world);
+int64_t moe_ep_max_send_rows(const moe_problem_t* problem, int32_t world);
+
+/* Dispatch: this rank's (token, slot) pairs sorted stably by owner rank, each owner's
+ * segment padded to a multiple of 16 rows.
+ *   topk_ids, topk_weights  device int32 / fp32 [T, k']: the route step's output (the shared
+ *                           slot, id E_r, included)
+ *   send_rows     device bf16 [max_send_rows, H]: row i = hidden row of the i-th sorted pair
+ *   send_expert   device int32 [max_send_rows]: the pair's expert id on its owner (id mod
+ *                 E_r/world; E_r/world for the shared slot)
+ *   send_weight   device fp32 [max_send_rows]: its routing weight
+ *   send_offsets  device int32 [world+1]: the owner-r segment is rows [offsets[r], offsets[r+1])
+ *   pair_to_send_row device int32 [T*k']: send row of pair t*k' + j
+ * Padding rows are zero rows with expert 0 and weight 0. workspace: device,
+ * moe_ep_workspace_size bytes, 256-byte aligned. T == 0 writes zero offsets. */
+moe_status_t moe_ep_dispatch(const moe_problem_t* problem, int32_t world, int32_t rank, const void* hidden,
+                             const int32_t* topk_ids, const float* topk_weights, void* send_rows,
+                             int32_t* send_expert, float* send_weight, int32_t* send_offsets,
+                             int32_t* pair_to_send_row, void* workspace, size_t workspace_bytes,
+                             moe_stream_t stream);
+
+/* Combine: out[t] = sum over j = 0..k'-1 of returned_rows[pair_to_send_row[t*k' + j]], in slot
+ * order in fp32, rounded once to bf16.
+ *   returned_rows  device bf16 [max_send_rows, H]: the owners' weighted outputs, in send order
+ *   out            device bf16 [T, H] */
+moe_status_t moe_ep_combine(const moe_problem_t* problem, int32_t world, const void* returned_rows,
+                            const int32_t* pair_to_send_row, void* out, moe_stream_t stream);
+
 /* Synchronises `stream`, reads and clears the workspace status word. Returns MOE_OK,
  * MOE_ERR_DEVICE_TIMEOUT if a kernel abandoned a bounded wait since the last query
  * (word 0x10000 | site; its outputs are then undefined), MOE_ERR_INVALID_ARG if

@@ -83,6 +83,10 @@ SIGNATURES = {
     "moe_quantize_weights_fp8_per_tensor": (_I, [_V, ctypes.c_int64, _I, _I, _V, _V, _V]),
     "moe_quantize_weights_mxfp8": (_I, [_V, ctypes.c_int64, _I, _I, _V, _V, _V]),
     "moe_prepare_weights_mxfp8": (_I, [_P, _V, _V, _V, _V, _V, _V, _V]),
+    "moe_ep_workspace_size": (_S, [_P, _I]),
+    "moe_ep_max_send_rows": (ctypes.c_int64, [_P, _I]),
+    "moe_ep_dispatch": (_I, [_P, _I, _I, _V, _V, _V, _V, _V, _V, _V, _V, _V, _S, _V]),
+    "moe_ep_combine": (_I, [_P, _I, _V, _V, _V, _V]),
     "moe_forward": (_I, [_P, _V, _V, _V, _V, _V, _V, _V, _V, _S, _V]),
     "moe_forward_routed": (_I, [_P, _V, _V, _V, _V, _V, _V, _V, _V, _V, _S, _V]),
     "moe_forward_host": (_I, [_P, _V, _V, _V, _V, _V, _V, _V, _V, _S, _V]),

@@ -816,6 +816,107 @@ MOE_API moe_status_t moe_stage_combine(const moe_problem_t* problem, void* out, 
   return run_combine(pl, out, workspace, launch_of(problem, stream));
 }
 
+// ---- expert parallelism ----------------------------------------------------------
+
+namespace {
+
+// Workspace of the dispatch sort: this rank's pairs keyed by owner rank (the align kernels
+// with `world` keys and 16-row padding per key).
+struct EpLayout {
+  size_t owner, sorted, block_expert, num_blocks, chunk_hist, total;
+  long long max_rows;
+  int num_chunks;
+};
+
+moe_status_t ep_plan(const moe_problem_t* p, int32_t world, Plan* pl, EpLayout* o) {
+  moe_status_t st = make_plan(p, pl);
+  if (st != MOE_OK) return st;
+  if (world < 1 || world > moe::kMaxExperts || pl->Er % world != 0) return MOE_ERR_INVALID_ARG;
+  const long long P = pl->P;
+  const long long active = P < world ? P : world;
+  o->max_rows = static_cast<long long>(align_up(static_cast<size_t>(P + active * 15), 16));
+  o->num_chunks = static_cast<int>(P == 0 ? 1 : (P + moe::kAlignChunk - 1) / moe::kAlignChunk);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align_up(off + bytes, kAlign);
+    return at;
+  };
+  o->owner = take(static_cast<size_t>(P) * 4);
+  o->sorted = take(static_cast<size_t>(o->max_rows) * 4);
+  o->block_expert = take(static_cast<size_t>(o->max_rows) / 16 * 4 + 4);
+  o->num_blocks = take(256);
+  o->chunk_hist = take(static_cast<size_t>(o->num_chunks) * world * 4);
+  o->total = off;
+  return MOE_OK;
+}
+
+}  // namespace
+
+MOE_API size_t moe_ep_workspace_size(const moe_problem_t* problem, int32_t world) {
+  Plan pl;
+  EpLayout el;
+  return ep_plan(problem, world, &pl, &el) == MOE_OK ? el.total : 0;
+}
+
+MOE_API int64_t moe_ep_max_send_rows(const moe_problem_t* problem, int32_t world) {
+  Plan pl;
+  EpLayout el;
+  return ep_plan(problem, world, &pl, &el) == MOE_OK ? el.max_rows : -1;
+}
+
+MOE_API moe_status_t moe_ep_dispatch(const moe_problem_t* problem, int32_t world, int32_t rank, const void* hidden,
+                                     const int32_t* topk_ids, const float* topk_weights, void* send_rows,
+                                     int32_t* send_expert, float* send_weight, int32_t* send_offsets,
+                                     int32_t* pair_to_send_row, void* workspace, size_t workspace_bytes,
+                                     moe_stream_t stream) {
+  Plan pl;
+  EpLayout el;
+  moe_status_t st = ep_plan(problem, world, &pl, &el);
+  if (st != MOE_OK) return st;
+  if (rank < 0 || rank >= world) return MOE_ERR_INVALID_ARG;
+  if (!aligned4(send_offsets)) return MOE_ERR_INVALID_ARG;
+  if (pl.T == 0) {  // nothing to send: the offsets are all zero
+    return cuda_status(cudaMemsetAsync(send_offsets, 0, (static_cast<size_t>(world) + 1) * 4,
+                                       reinterpret_cast<cudaStream_t>(stream)));
+  }
+  if (!aligned16(hidden) || !aligned4(topk_ids) || !aligned4(topk_weights) || !aligned16(send_rows) ||
+      !aligned4(send_expert) || !aligned4(send_weight) || !aligned4(pair_to_send_row))
+    return MOE_ERR_INVALID_ARG;
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MOE_ERR_INVALID_ARG;
+  if (workspace_bytes < el.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  int sms = 0;
+  st = device_sms(&sms);
+  if (st != MOE_OK) return st;
+  const Launch l = launch_of(problem, stream);
+  const int per_rank = pl.Er / world;
+  int* owner = ws_ptr<int>(workspace, el.owner);
+  int* sorted = ws_ptr<int>(workspace, el.sorted);
+  cudaError_t e = moe::launch_ep_owner(l, topk_ids, pl.P, pl.Er, per_rank, rank, owner);
+  if (e == cudaSuccess)
+    e = moe::launch_align(l, owner, static_cast<int>(pl.P), world, 16, el.num_chunks, ws_ptr<int>(workspace, el.chunk_hist),
+                          sorted, send_offsets, ws_ptr<int>(workspace, el.block_expert), pair_to_send_row,
+                          ws_ptr<int>(workspace, el.num_blocks), 0, nullptr);
+  if (e == cudaSuccess)
+    e = moe::launch_ep_pack(l, hidden, pl.H, sorted, send_offsets, world, static_cast<int>(pl.P), pl.kk, topk_ids,
+                            topk_weights, pl.Er, per_rank, el.max_rows, send_rows, send_expert, send_weight, sms);
+  return cuda_status(e);
+}
+
+MOE_API moe_status_t moe_ep_combine(const moe_problem_t* problem, int32_t world, const void* returned_rows,
+                                    const int32_t* pair_to_send_row, void* out, moe_stream_t stream) {
+  Plan pl;
+  EpLayout el;
+  moe_status_t st = ep_plan(problem, world, &pl, &el);
+  if (st != MOE_OK || pl.T == 0) return st;
+  if (!aligned16(returned_rows) || !aligned4(pair_to_send_row) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+  int sms = 0;
+  st = device_sms(&sms);
+  if (st != MOE_OK) return st;
+  return cuda_status(
+      moe::launch_ep_combine(launch_of(problem, stream), returned_rows, pair_to_send_row, pl.T, pl.kk, pl.H, out));
+}
+
 MOE_API moe_status_t moe_get_device_status(void* workspace, moe_stream_t stream, int32_t* detail) {
   if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MOE_ERR_INVALID_ARG;
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

@@ -144,6 +144,20 @@ size_t tiled_scale_bytes_mx(int E, int rows, int K);
 cudaError_t launch_tile_scales_mx(const Launch& l, int which, const void* in, void* out, int E, int H, int I,
                                   int gated);
 
+// ---- expert parallelism (ep.cu) ----
+// owner[p] = ids[p] / per_rank for a routed id (< E_r), `rank` for the shared slot.
+cudaError_t launch_ep_owner(const Launch& l, const int* ids, long long P, int E_r, int per_rank, int rank,
+                            int* owner);
+// Send rows in the order of sorted_pair_ids (rows < send_offsets[world], at most max_rows):
+// hidden row, owner-local expert id and weight of each pair; zero for padding rows.
+cudaError_t launch_ep_pack(const Launch& l, const void* hidden, int H, const int* sorted_pair_ids,
+                           const int* send_offsets, int world, int P, int k_total, const int* ids, const float* weights,
+                           int E_r, int per_rank, long long max_rows, void* send_rows, int* send_expert,
+                           float* send_weight, int num_sms);
+// out[t] = bf16(sum_j returned[pair_to_row[t k' + j]]) in slot order, fp32 accumulation.
+cudaError_t launch_ep_combine(const Launch& l, const void* returned, const int* pair_to_row, int T, int k_total, int H,
+                              void* out);
+
 // ---- elementwise (combine.cu, quant.cu, prepare.cu) ----
 cudaError_t launch_combine(const Launch& l, const void* y, const int* pair_to_row, int T, int k_total, int H,
                            void* out);
