@@ -224,11 +224,16 @@ def _problem_from(hidden, router_logits, w2, topk, renormalize, activation_type,
 _WS_CACHE: Dict[tuple, torch.Tensor] = {}
 
 
-def _workspace_for(prob: Problem, device) -> torch.Tensor:
-    key = (device, prob.num_tokens, prob.hidden, prob.num_routed, prob.num_shared,
-           prob.intermediate, prob.topk, prob.activation, prob.wdtype, prob.block_m)
+def _workspace_for(prob: Problem, device, stream=None) -> torch.Tensor:
+    """The cached workspace of calls that pass none: one per device, stream and problem
+    shape apart from the token count, grown to the largest token count seen (a workspace
+    sized for more tokens serves fewer), so a caller whose batch size changes from call to
+    call reuses one buffer. Calls on different streams get different workspaces."""
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    key = (str(device), s.cuda_stream, prob.hidden, prob.num_routed, prob.num_shared, prob.intermediate,
+           prob.topk, prob.activation, prob.wdtype, prob.block_m)
     ws = _WS_CACHE.get(key)
-    if ws is None:
+    if ws is None or ws.numel() < workspace_size(prob):
         ws = new_workspace(prob, device)
         _WS_CACHE[key] = ws
     return ws
@@ -260,7 +265,7 @@ def moe_forward(hidden: torch.Tensor, router_logits: torch.Tensor, w13: torch.Te
     prob = _problem_from(hidden, router_logits, w2, topk, renormalize, activation_type,
                          num_shared, fp8, pdl, input_scale or 0.0, activation_scale or 0.0)
     if workspace is None:
-        workspace = _workspace_for(prob, hidden.device)
+        workspace = _workspace_for(prob, hidden.device, stream)
     if out is None:
         out = torch.empty_like(hidden)
     check(lib().moe_forward(ctypes.byref(prob), _ptr(hidden), _ptr(router_logits), _ptr(w13),
@@ -296,7 +301,7 @@ def moe_forward_routed(hidden: torch.Tensor, topk_ids: torch.Tensor, topk_weight
     prob = make_problem(T, H, num_routed, topk, I, renormalize=False, activation=activation_type,
                         num_shared=num_shared, fp8=fp8, pdl=pdl)
     if workspace is None:
-        workspace = _workspace_for(prob, hidden.device)
+        workspace = _workspace_for(prob, hidden.device, stream)
     if out is None:
         out = torch.empty_like(hidden)
     check(lib().moe_forward_routed(ctypes.byref(prob), _ptr(hidden), _ptr(topk_ids), _ptr(topk_weights),
