@@ -650,6 +650,36 @@ def quantize_weights_mxfp8(w13_bits, w2_bits, experts=None):
     return tuple(out)
 
 
+def pad_weights_mxfp8(w13_q, w13_sc, w2_q, w2_sc, I: int, gated: bool, min_alignment: int):
+    """Zero-pad MXFP8 weights and their scales to I_pad = round_up(I, min_alignment).
+
+    [TRTLLM] section 2, ``_align_mxfp8_moe_weights``: the codes are padded like the FP8
+    weights (w13 to up_mult * I_pad rows, w2's last axis to I_pad, zeros after the
+    original values), and the scales with them: w13's scales gain the new rows, w2's scales
+    (one per 32 values of I) grow to I_pad / 32 columns, all zero. As in ``pad_weights``,
+    a gated w13 keeps gate rows [0, I) and up rows [I_pad, I_pad + I), each half padded on
+    its own. Zero codes make the padded rows and columns contribute exact zeros whatever
+    their (zero-byte) scales. Returns (w13_q, w13_sc, w2_q, w2_sc, I_pad); the inputs
+    themselves when I is already aligned.
+    """
+    I_pad = (I + min_alignment - 1) // min_alignment * min_alignment
+    if I_pad == I:
+        return w13_q, w13_sc, w2_q, w2_sc, I
+    assert I_pad % MX_BLOCK == 0 and I % MX_BLOCK == 0
+    E = w13_q.shape[0]
+    halves = 2 if gated else 1
+    out13 = np.zeros((E, halves * I_pad, w13_q.shape[2]), dtype=w13_q.dtype)
+    out13s = np.zeros((E, halves * I_pad, w13_sc.shape[2]), dtype=w13_sc.dtype)
+    for h in range(halves):
+        out13[:, h * I_pad:h * I_pad + I] = w13_q[:, h * I:(h + 1) * I]
+        out13s[:, h * I_pad:h * I_pad + I] = w13_sc[:, h * I:(h + 1) * I]
+    out2 = np.zeros((E, w2_q.shape[1], I_pad), dtype=w2_q.dtype)
+    out2[:, :, :I] = w2_q
+    out2s = np.zeros((E, w2_sc.shape[1], I_pad // MX_BLOCK), dtype=w2_sc.dtype)
+    out2s[:, :, :I // MX_BLOCK] = w2_sc
+    return out13, out13s, out2, out2s, I_pad
+
+
 def moe_forward_mxfp8(hidden_bits: np.ndarray, logits: Optional[np.ndarray], w13_q, w13_sc, w2_q, w2_sc, *,
                       topk: int, renormalize: bool, activation: str, num_shared: int = 0,
                       tokens: Optional[Sequence[int]] = None, routing=None):

@@ -583,6 +583,50 @@ def test_quant_mx_against_math_frexp_and_torch_cast():
     np.testing.assert_array_equal(O.dequant_mx(q2, s2), v)
 
 
+def test_mxfp8_padding_rule_from_page():
+    # the page's rule: I rounded up to min_alignment (16 gated, 128 non-gated), codes and
+    # scales zero-filled after the original values, unchanged when already aligned
+    rng = np.random.default_rng(61)
+    for gated, I, align, I_pad in ((True, 96, 128, 128), (False, 160, 128, 256), (True, 64, 16, 64)):
+        E, H = 2, 64
+        N1 = (2 if gated else 1) * I
+        w13 = rng.integers(1, 255, (E, N1, H)).astype(np.uint8)
+        s13 = rng.integers(100, 140, (E, N1, H // 32)).astype(np.uint8)
+        w2 = rng.integers(1, 255, (E, H, I)).astype(np.uint8)
+        s2 = rng.integers(100, 140, (E, H, I // 32)).astype(np.uint8)
+        p13, ps13, p2, ps2, got = O.pad_weights_mxfp8(w13, s13, w2, s2, I, gated, align)
+        assert got == I_pad
+        if I_pad == I:
+            assert p13 is w13 and ps2 is s2
+            continue
+        assert p13.shape == (E, (2 if gated else 1) * I_pad, H) and ps13.shape == (E, p13.shape[1], H // 32)
+        assert p2.shape == (E, H, I_pad) and ps2.shape == (E, H, I_pad // 32)
+        for h in range(2 if gated else 1):
+            np.testing.assert_array_equal(p13[:, h * I_pad:h * I_pad + I], w13[:, h * I:(h + 1) * I])
+            np.testing.assert_array_equal(ps13[:, h * I_pad:h * I_pad + I], s13[:, h * I:(h + 1) * I])
+            assert np.all(p13[:, h * I_pad + I:(h + 1) * I_pad] == 0) and np.all(ps13[:, h * I_pad + I:(h + 1) * I_pad] == 0)
+        np.testing.assert_array_equal(p2[:, :, :I], w2)
+        np.testing.assert_array_equal(ps2[:, :, :I // 32], s2)
+        assert np.all(p2[:, :, I:] == 0) and np.all(ps2[:, :, I // 32:] == 0)
+
+
+def test_mxfp8_padding_leaves_layer_unchanged():
+    rng = np.random.default_rng(67)
+    for act, I in (("swiglu", 96), ("relu2", 160)):
+        gated = act == "swiglu"
+        T, H, E, k = 5, 128, 3, 2
+        x = _bf16_bits(torch.from_numpy(rng.standard_normal((T, H)).astype(np.float32)))
+        l = rng.standard_normal((T, E)).astype(np.float32)
+        w13 = _bf16_bits(torch.from_numpy(0.05 * rng.standard_normal((E, (2 if gated else 1) * I, H)).astype(np.float32)))
+        w2 = _bf16_bits(torch.from_numpy(0.05 * rng.standard_normal((E, H, I)).astype(np.float32)))
+        q = O.quantize_weights_mxfp8(w13, w2)
+        padded = O.pad_weights_mxfp8(*q, I, gated, 128)
+        a = O.moe_forward_mxfp8(x, l, *q, topk=k, renormalize=True, activation=act)
+        b = O.moe_forward_mxfp8(x, l, *padded[:4], topk=k, renormalize=True, activation=act)
+        # the padded activation columns are exact zeros, and an all-zero 32-block quantises to zero
+        np.testing.assert_allclose(b, a, rtol=1e-12, atol=1e-12)
+
+
 @pytest.mark.parametrize("act", ["swiglu", "relu2"])
 def test_mxfp8_layer_against_torch_casts(act):
     # independent restatement: math.frexp exponents, torch float8 casts, a dense per-token loop
