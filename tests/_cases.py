@@ -23,7 +23,7 @@ def cpu_inputs(cfg: MoeConfig, seed: int = 0) -> Dict[str, torch.Tensor]:
     return make_inputs(cfg, seed)
 
 
-class GpuRun:
+class GpuForward:
     """One forward of ``cfg`` on cuda:0 with every intermediate kept in the workspace."""
 
     def __init__(self, cfg: MoeConfig, seed: int = 0, inputs: Optional[dict] = None, pdl: bool = True,
@@ -119,7 +119,7 @@ def err_beyond_rounding(got: np.ndarray, ref: np.ndarray) -> float:
     return float(np.max(np.abs(got - ref) - half_ulp_bf16(ref)) / r)
 
 
-__all__ = ["CONFIGS", "GpuRun", "bits", "cpu_inputs", "oracle_out", "bf16_to_f64", "max_err_over_rms",
+__all__ = ["CONFIGS", "GpuForward", "bits", "cpu_inputs", "oracle_out", "bf16_to_f64", "max_err_over_rms",
            "half_ulp_bf16", "err_beyond_rounding"]
 
 

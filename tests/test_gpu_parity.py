@@ -18,7 +18,7 @@ import mixture_experts_expert_topk_b200 as moe
 from mixture_experts_expert_topk_b200.synth import CONFIGS, MoeConfig, make_inputs
 from oracle import moe_oracle as O
 
-from _cases import (GpuRun, bf16_to_f64, bits, cpu_inputs, err_beyond_rounding, max_err_over_rms, oracle_out,
+from _cases import (GpuForward, bf16_to_f64, bits, cpu_inputs, err_beyond_rounding, max_err_over_rms, oracle_out,
                     untile_groups, untile_weights)
 
 pytestmark = pytest.mark.gpu
@@ -145,7 +145,7 @@ def _check_act(cfg, run, parts, ids, a):
 def test_layer_parity_small(name, bm):
     # bm 0: the default (bf16: 16-row alignment, weights on the MMA's M); 128: token tiles
     cfg = SMALL[name]
-    run = GpuRun(cfg, block_m=bm)
+    run = GpuForward(cfg, block_m=bm)
     out = run.forward()
     parts = run.parts()
     ids, a = _check_route_align(cfg, parts, run.inp["logits"])
@@ -162,17 +162,17 @@ def test_layer_parity_small(name, bm):
 
 def test_forward_is_bitwise_deterministic_and_pdl_invariant():
     cfg = SMALL["ragged"]
-    run = GpuRun(cfg)
+    run = GpuForward(cfg)
     a = bits(run.forward()).copy()
     b = bits(run.forward()).copy()
     np.testing.assert_array_equal(a, b)
-    run2 = GpuRun(cfg, pdl=False)
+    run2 = GpuForward(cfg, pdl=False)
     np.testing.assert_array_equal(bits(run2.forward()), a)
 
 
 def test_stage_entry_points_match_forward():
     cfg = SMALL["ragged"]
-    run = GpuRun(cfg)
+    run = GpuForward(cfg)
     ref = bits(run.forward()).copy()
     ws = moe.new_workspace(run.prob)
     out = torch.empty_like(run.hidden)
@@ -191,7 +191,7 @@ def test_tied_logits_pick_lowest_indices():
     inp = make_inputs(cfg, 3)
     inp["logits"][:] = 0.5
     inp["logits"][5, 9] = 0.5   # still tied
-    run = GpuRun(cfg, inputs=inp)
+    run = GpuForward(cfg, inputs=inp)
     run.forward()
     parts = run.parts()
     assert (parts["topk_ids"] == np.arange(4)).all()
@@ -205,7 +205,7 @@ def test_all_tokens_one_expert_and_empty_experts(T):
     cfg = _small("one_expert", T=T, H=256, E=8, topk=1, I=256)
     inp = make_inputs(cfg, 4)
     inp["logits"][:, 5] += 100.0   # every token picks expert 5; 7 experts empty
-    run = GpuRun(cfg, inputs=inp)
+    run = GpuForward(cfg, inputs=inp)
     run.forward()
     parts = run.parts()
     ids, a = _check_route_align(cfg, parts, inp["logits"])
@@ -279,7 +279,7 @@ def test_fp8_quantizers_bit_exact():
 # ---- the workloads at full size ------------------------------------------------------
 
 def _full_size(cfg, n_sample=48, seed=0):
-    run = GpuRun(cfg, seed)
+    run = GpuForward(cfg, seed)
     out = run.forward()
     parts = run.parts()
     ids, a = _check_route_align(cfg, parts, run.inp["logits"])
@@ -310,7 +310,7 @@ def test_workload_full_size(name, n_sample):
 @pytest.mark.parametrize("T", [1, 4, 16, 64])
 def test_decode_full(T):
     cfg = CONFIGS[f"decode_T{T}"]
-    run = GpuRun(cfg)
+    run = GpuForward(cfg)
     out = run.forward()
     parts = run.parts()
     _check_route_align(cfg, parts, run.inp["logits"])
@@ -333,7 +333,7 @@ FP8_SMALL = {
 @pytest.mark.parametrize("name", list(FP8_SMALL))
 def test_fp8_layer_parity_small(name):
     cfg = FP8_SMALL[name]
-    run = GpuRun(cfg)
+    run = GpuForward(cfg)
     out = run.forward()
     parts = run.parts()
     ids, a = _check_route_align(cfg, parts, run.inp["logits"])
@@ -366,7 +366,7 @@ def test_decode_both_row_tilings(T, bm):
     # the same decode batch through 16-row token blocks (weights as the MMA's M operand)
     # and through 128-row tiles must both match the oracle
     cfg = CONFIGS[f"decode_T{T}"]
-    run = GpuRun(cfg, block_m=bm)
+    run = GpuForward(cfg, block_m=bm)
     out = run.forward()
     parts = run.parts()
     assert parts["block_m"] == bm
@@ -391,7 +391,7 @@ def test_routed_with_own_routing_is_bitwise_the_forward(name):
     # the routed entry point given the route step's own choice runs the same kernels on
     # the same routing, so its output is the forward's, bit for bit
     cfg = SMALL[name]
-    run = GpuRun(cfg)
+    run = GpuForward(cfg)
     ref = bits(run.forward()).copy()
     parts = run.parts()
     ids = torch.from_numpy(parts["topk_ids"][:, :cfg.topk].copy())
@@ -404,7 +404,7 @@ def test_routed_with_own_routing_is_bitwise_the_forward(name):
 def test_routed_arbitrary_routing_matches_oracle(name):
     # repeated experts within a token and weights that are not a softmax
     cfg = SMALL.get(name) or FP8_SMALL[name]
-    run = GpuRun(cfg)
+    run = GpuForward(cfg)
     g = torch.Generator().manual_seed(21)
     ids = torch.randint(0, cfg.E, (cfg.T, cfg.topk), generator=g, dtype=torch.int32)
     ids[::5, 0] = ids[::5, -1]                      # repeats
@@ -426,7 +426,7 @@ def test_routed_arbitrary_routing_matches_oracle(name):
 
 def test_routed_out_of_range_ids_are_dropped_and_reported():
     cfg = SMALL["ragged"]
-    run = GpuRun(cfg)
+    run = GpuForward(cfg)
     g = torch.Generator().manual_seed(22)
     ids = torch.randint(0, cfg.E, (cfg.T, cfg.topk), generator=g, dtype=torch.int32)
     w = torch.rand((cfg.T, cfg.topk), generator=g)
