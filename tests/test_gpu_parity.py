@@ -582,7 +582,22 @@ def _mx_weight_scales(flat, E, rows, K, gated):
 @pytest.mark.parametrize("name", list(MX_SMALL))
 def test_mxfp8_layer_parity(name):
     cfg = MX_SMALL[name]
+    _mx_parity(cfg, make_inputs(cfg, 0), name)
+
+
+def test_mxfp8_zero_blocks_and_rows():
+    """All-zero 32-column blocks (scale byte 0, codes 0) and all-zero hidden rows."""
+    cfg = MX_SMALL["mx_swiglu"]
     inp = make_inputs(cfg, 0)
+    h = inp["hidden"].clone()
+    h[::7] = 0                       # whole rows
+    h[1::5, 32:96] = 0               # two 32-column blocks of other rows
+    h[2::9, 224:256] = 0             # the last block
+    inp["hidden"] = h
+    _mx_parity(cfg, inp, "mx_zero_blocks")
+
+
+def _mx_parity(cfg, inp, name):
     dev = torch.device("cuda:0")
     hidden, logits = inp["hidden"].to(dev), inp["logits"].to(dev)
     # device quantiser, bit-exact against the oracle's (OCP MX conversion decided in fp32)
