@@ -426,6 +426,12 @@ def main():
     g1_bytes = w13_bytes + cfg.T * cfg.H * elt + P * cfg.I * elt
     g1_ms = r["kernel_ms"]["gemm1"]
     g1_gbs = g1_bytes / (g1_ms / 1e3) / 1e9
+    g1_flops = 2.0 * P * cfg.H * cfg.N1
+    g1_tflops = g1_flops / (g1_ms / 1e3) / 1e12
+    # the binding roof of GEMM1: tensor cores when its arithmetic intensity exceeds the
+    # ridge of the measured peaks (a contraction in 8-bit types takes twice the bf16 peak)
+    tc_dtype_peak = tc_peak * (2.0 if cfg.fp8 else 1.0)
+    tensor_bound = g1_flops / g1_bytes > tc_dtype_peak * 1e12 / (hbm_peak * 1e9)
     minimal_bytes = w13_bytes + w2_bytes + cfg.T * cfg.H * 2 * 2 + cfg.T * cfg.E * 4
     layer_gbs = minimal_bytes / (ms_per_step / 1e3) / 1e9
     line = dict(base)
@@ -440,11 +446,18 @@ def main():
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": r["h2d"],
                 "d2h_bytes_per_step": r["d2h"]},
         "gpu_launches": r["launches_per_step"] * args.steps,
-        "roofline": {"bound": "hbm", "kernel": "gemm1 (grouped up-GEMM + activation)",
-                     "achieved": g1_gbs, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": g1_gbs / hbm_peak, "traffic": _gemm1_traffic(cfg, g1_bytes),
-                     "peak_source": f"{peak_kind} hbm_gbs",
-                     "algorithmic_bytes_per_launch": g1_bytes, "avg_launch_ms": g1_ms},
+        "roofline": ({"bound": "tensor", "kernel": "gemm1 (grouped up-GEMM + activation)",
+                      "achieved": g1_tflops, "peak": tc_dtype_peak, "unit": "TFLOP/s",
+                      "frac": g1_tflops / tc_dtype_peak, "traffic": _gemm1_traffic(cfg, g1_bytes),
+                      "peak_source": f"{peak_kind} bf16_tflops" + (" x 2 (8-bit)" if cfg.fp8 else ""),
+                      "algorithmic_flops_per_launch": g1_flops, "algorithmic_bytes_per_launch": g1_bytes,
+                      "avg_launch_ms": g1_ms} if tensor_bound else
+                     {"bound": "hbm", "kernel": "gemm1 (grouped up-GEMM + activation)",
+                      "achieved": g1_gbs, "peak": hbm_peak, "unit": "GB/s",
+                      "frac": g1_gbs / hbm_peak, "traffic": _gemm1_traffic(cfg, g1_bytes),
+                      "peak_source": f"{peak_kind} hbm_gbs",
+                      "algorithmic_bytes_per_launch": g1_bytes, "avg_launch_ms": g1_ms,
+                      "gemm1_tflops": g1_tflops}),
         "layer_hbm": {"minimal_bytes": minimal_bytes, "achieved_gbs": layer_gbs,
                       "frac": layer_gbs / hbm_peak, "touched_experts": n_touched},
         "tensor_frac": value / tc_peak,

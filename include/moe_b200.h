@@ -69,9 +69,14 @@ typedef enum {
 typedef enum {
   MOE_ACT_SWIGLU = 0, /* gated: a_n = silu(gate_n) * up_n, silu(x) = x / (1 + e^-x) */
   MOE_ACT_RELU2 = 1,  /* non-gated: a_n = max(z_n, 0)^2 */
-  MOE_ACT_GELU_TANH = 2 /* gated: a_n = gelu_tanh(gate_n) * up_n, gelu_tanh(x) = 0.5 x (1 +
-                           tanh(sqrt(2/pi) (x + 0.044715 x^3))) ("FlashInfer gated MoE kernel
-                           optimisation for Blackwell", section 2; padded like SWIGLU) */
+  MOE_ACT_GELU_TANH = 2, /* gated: a_n = gelu_tanh(gate_n) * up_n, gelu_tanh(x) = 0.5 x (1 +
+                            tanh(sqrt(2/pi) (x + 0.044715 x^3))) ("FlashInfer gated MoE kernel
+                            optimisation for Blackwell", section 2; padded like SWIGLU) */
+  MOE_ACT_SWIGLUOAI = 3  /* gated, "swigluoai_uninterleave" of the same page, section 2: the
+                            SwiGLU variant published with OpenAI's gpt-oss models, on gate and
+                            up halves that are not interleaved (the w13 checkpoint layout of
+                            SWIGLU): g = min(gate_n, 7), u = clamp(up_n, -7, 7),
+                            a_n = g / (1 + e^(-1.702 g)) * (u + 1); padded like SWIGLU */
 } moe_activation_t;
 
 /* Weight / activation number format. */
@@ -322,13 +327,22 @@ moe_status_t moe_stage_combine(const moe_problem_t* problem, void* out, void* wo
  * (an engine plugin that is handed only its input and output tensors, code running under
  * stream capture, or a path where an allocation could synchronise the device). The pages
  * have no counterpart of this entry point; it runs the same kernels as moe_stage_align.
- *   topk_ids        device int32 [T, k'] expert ids (e.g. from moe_stage_route), each in
- *                   [0, E); read only
- *   sorted_pair_ids device int32 [max_rows]   } outputs, laid out exactly as the
- *   expert_offsets  device int32 [E+1]        } workspace fields of the same names
- *   block_expert    device int32 [max_rows/128] } (moe_workspace_layout gives max_rows)
- *   pair_to_row     device int32 [T*k']       }
- *   num_blocks      device int32 [1]          }
+ * Sizes below use max_rows and block_m from moe_workspace_layout(problem) (block_m is 16
+ * for the BF16 default, 128 for FP8 block-128 or an explicit problem->block_m of 128):
+ *   topk_ids        device int32 [T, k'] expert ids (e.g. from moe_stage_route); read only.
+ *                   An id outside [0, E) is skipped: its pair is not placed in any segment
+ *                   and its pair_to_row entry is -1 (nothing outside the buffers below is
+ *                   written).
+ *   sorted_pair_ids device int32 [max_rows]: pair ids sorted by expert, sentinel T*k' in
+ *                   the padding (entries past P_pad = num_blocks[0]*block_m are not written)
+ *   expert_offsets  device int32 [E+1]
+ *   block_expert    device int32 [max_rows/block_m]: expert of each block_m-row tile
+ *                   (entries past num_blocks[0] are not written)
+ *   pair_to_row     device int32 [T*k']
+ *   num_blocks      device int32 [1]: P_pad / block_m
+ * These are the workspace fields of the same names. The row groups that moe_stage_align
+ * also writes for block_m 16 (group_info and the second num_blocks entry) are not
+ * produced, so these outputs do not drive the block_m-16 GEMM stages by themselves.
  * Its scratch is a fixed array of 262144 int32 (1 MiB) in device memory owned by the
  * library: every GPU that loads the library holds it until the process exits. A problem
  * needing more (ceil(T*k'/2048) * E > 262144) returns MOE_ERR_UNSUPPORTED. The first call
@@ -388,6 +402,20 @@ moe_status_t moe_ep_combine(const moe_problem_t* problem, int32_t world, const v
  * moe_forward_routed met an expert id out of range (word 0x20000), or MOE_ERR_CUDA.
  * `*detail` (may be NULL) receives the raw word. */
 moe_status_t moe_get_device_status(void* workspace, moe_stream_t stream, int32_t* detail);
+
+/* Test of the device-side timeout path (failure detection without a GPU fault). Every
+ * wait inside this library's kernels is bounded: when its limit passes, the kernel records
+ * 0x10000 | site in the workspace status word and returns, and moe_get_device_status then
+ * reports MOE_ERR_DEVICE_TIMEOUT. This call launches one small kernel that waits, through
+ * that same bounded wait, on an mbarrier expecting one arrival:
+ *   workspace  device, 256-byte aligned; only its status word (offset 0) is written
+ *   limit_us   the wait's limit, 1 .. 1000000 microseconds
+ *   arrive     1: the kernel arrives first, so the wait completes and the status word is
+ *              untouched; 0: nothing arrives, the wait gives up after limit_us and the
+ *              status word becomes 0x1007F (site 0x7F)
+ * Asynchronous on `stream`; MOE_ERR_INVALID_ARG for a bad pointer or limit. */
+moe_status_t moe_selftest_bounded_wait(void* workspace, uint32_t limit_us, int32_t arrive,
+                                       moe_stream_t stream);
 
 #ifdef __cplusplus
 }

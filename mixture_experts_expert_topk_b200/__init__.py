@@ -18,7 +18,7 @@ from typing import Dict, Optional, Tuple
 import torch
 
 from . import _capi
-from ._capi import (MOE_ACT_GELU_TANH, MOE_ACT_RELU2, MOE_ACT_SWIGLU, MOE_DTYPE_BF16, MOE_DTYPE_FP8_BLOCK128,
+from ._capi import (MOE_ACT_GELU_TANH, MOE_ACT_RELU2, MOE_ACT_SWIGLU, MOE_ACT_SWIGLUOAI, MOE_DTYPE_BF16, MOE_DTYPE_FP8_BLOCK128,
                     MOE_DTYPE_FP8_PER_TENSOR, MOE_DTYPE_MXFP8,
                     MOE_FLAG_PDL, MoeError, Problem, check, lib)
 
@@ -32,7 +32,9 @@ __all__ = [
 
 _ACT = {"swiglu": MOE_ACT_SWIGLU, "silu": MOE_ACT_SWIGLU, "relu2": MOE_ACT_RELU2,
         "gelu_tanh": MOE_ACT_GELU_TANH, "gelu": MOE_ACT_GELU_TANH,
-        MOE_ACT_SWIGLU: MOE_ACT_SWIGLU, MOE_ACT_RELU2: MOE_ACT_RELU2, MOE_ACT_GELU_TANH: MOE_ACT_GELU_TANH}
+        "swigluoai": MOE_ACT_SWIGLUOAI, "swigluoai_uninterleave": MOE_ACT_SWIGLUOAI,
+        MOE_ACT_SWIGLU: MOE_ACT_SWIGLU, MOE_ACT_RELU2: MOE_ACT_RELU2, MOE_ACT_GELU_TANH: MOE_ACT_GELU_TANH,
+        MOE_ACT_SWIGLUOAI: MOE_ACT_SWIGLUOAI}
 
 
 def _act(a) -> int:

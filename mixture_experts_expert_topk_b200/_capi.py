@@ -23,6 +23,7 @@ MOE_ERR_DEVICE_TIMEOUT = 5
 MOE_ACT_SWIGLU = 0
 MOE_ACT_RELU2 = 1
 MOE_ACT_GELU_TANH = 2
+MOE_ACT_SWIGLUOAI = 3
 MOE_DTYPE_FP8_PER_TENSOR = 2
 MOE_DTYPE_MXFP8 = 3
 MOE_DTYPE_BF16 = 0
@@ -99,6 +100,7 @@ SIGNATURES = {
     "moe_stage_combine": (_I, [_P, _V, _V, _S, _V]),
     "moe_get_device_status": (_I, [_V, _V, ctypes.POINTER(_I)]),
     "moe_align_noalloc": (_I, [_P, _V, _V, _V, _V, _V, _V, _V]),
+    "moe_selftest_bounded_wait": (_I, [_V, ctypes.c_uint32, _I, _V]),
 }
 
 _lib = None

@@ -39,12 +39,17 @@ constexpr int kScanSmemInts = 40960;             // 160 KB of chunk-histogram st
 
 static_assert(kPairsPerWarp % 32 == 0, "warp slices are whole 32-pair steps");
 
-// Load this warp's pair ids (p = base + 32 i + lane); -1 marks pairs past the end.
-__device__ __forceinline__ void load_ids(const int* ids, int base, int end, int lane, int (&e)[kIdsPerLane]) {
+// Load this warp's pair ids (p = base + 32 i + lane); -1 marks pairs past the end and
+// kBadId a pair whose expert id lies outside [0, E): such a pair is neither counted nor
+// placed, and its pair_to_row entry becomes -1.
+constexpr int kBadId = -2;
+__device__ __forceinline__ void load_ids(const int* ids, int base, int end, int E, int lane,
+                                         int (&e)[kIdsPerLane]) {
 #pragma unroll
   for (int i = 0; i < kIdsPerLane; ++i) {
     const int p = base + 32 * i + lane;
-    e[i] = p < end ? ids[p] : -1;
+    const int id = p < end ? ids[p] : -1;
+    e[i] = p >= end ? -1 : (static_cast<unsigned>(id) < static_cast<unsigned>(E) ? id : kBadId);
   }
 }
 
@@ -70,6 +75,8 @@ __device__ __forceinline__ void warp_place(const int (&e)[kIdsPerLane], int base
       const int pos = next[e[i]] + __popc(peers & lt);
       sorted_pair_ids[pos] = p;
       pair_to_row[p] = pos;
+    } else if (e[i] == kBadId) {
+      pair_to_row[base + 32 * i + lane] = -1;
     }
     __syncwarp();
     if (e[i] >= 0 && lane == 31 - __clz(peers)) next[e[i]] += __popc(peers);
@@ -145,7 +152,10 @@ __global__ void __launch_bounds__(kWarps * 32)
   __syncthreads();
   const int base = blockIdx.x * kAlignChunk;
   const int end = min(base + kAlignChunk, P);
-  for (int p = base + threadIdx.x; p < end; p += blockDim.x) atomicAdd(&hist[ids[p]], 1);
+  for (int p = base + threadIdx.x; p < end; p += blockDim.x) {
+    const int id = ids[p];
+    if (static_cast<unsigned>(id) < static_cast<unsigned>(E)) atomicAdd(&hist[id], 1);
+  }
   __syncthreads();
   int* out = chunk_hist + static_cast<size_t>(blockIdx.x) * E;
   for (int e = threadIdx.x; e < E; e += blockDim.x) out[e] = hist[e];
@@ -210,7 +220,7 @@ __global__ void __launch_bounds__(kWarps * 32)
   for (int i = threadIdx.x; i < kWarps * E; i += blockDim.x) cnt[i / E][i % E] = 0;
   const int base = blockIdx.x * kAlignChunk + warp * kPairsPerWarp;
   int e[kIdsPerLane];
-  load_ids(ids, base, P, lane, e);
+  load_ids(ids, base, P, E, lane, e);
   __syncthreads();
   warp_count(e, lane, cnt[warp]);
   __syncthreads();
@@ -242,7 +252,7 @@ __global__ void __launch_bounds__(kWarps * 32)
   for (int i = threadIdx.x; i < kWarps * E; i += blockDim.x) cnt[i / E][i % E] = 0;
   const int base = warp * kPairsPerWarp;
   int e[kIdsPerLane];
-  load_ids(ids, base, P, lane, e);
+  load_ids(ids, base, P, E, lane, e);
   __syncthreads();
   warp_count(e, lane, cnt[warp]);
   __syncthreads();

@@ -65,7 +65,8 @@ moe_status_t make_plan(const moe_problem_t* p, Plan* pl) {
   if (p->num_shared != 0 && p->num_shared != 1) return MOE_ERR_INVALID_ARG;
   if (p->topk > p->num_routed) return MOE_ERR_INVALID_ARG;
   if (p->renormalize != 0 && p->renormalize != 1) return MOE_ERR_INVALID_ARG;
-  if (p->activation != MOE_ACT_SWIGLU && p->activation != MOE_ACT_RELU2 && p->activation != MOE_ACT_GELU_TANH)
+  if (p->activation != MOE_ACT_SWIGLU && p->activation != MOE_ACT_RELU2 && p->activation != MOE_ACT_GELU_TANH &&
+      p->activation != MOE_ACT_SWIGLUOAI)
     return MOE_ERR_INVALID_ARG;
   if (p->wdtype != MOE_DTYPE_BF16 && p->wdtype != MOE_DTYPE_FP8_BLOCK128 && p->wdtype != MOE_DTYPE_FP8_PER_TENSOR &&
       p->wdtype != MOE_DTYPE_MXFP8)
@@ -519,7 +520,9 @@ MOE_API moe_status_t moe_check_problem(const moe_problem_t* problem) {
 
 MOE_API int32_t moe_padded_intermediate(int32_t intermediate, int32_t activation, int32_t wdtype) {
   if (intermediate <= 0 || intermediate > (1 << 20)) return -1;
-  if (activation != MOE_ACT_SWIGLU && activation != MOE_ACT_RELU2 && activation != MOE_ACT_GELU_TANH) return -1;
+  if (activation != MOE_ACT_SWIGLU && activation != MOE_ACT_RELU2 && activation != MOE_ACT_GELU_TANH &&
+      activation != MOE_ACT_SWIGLUOAI)
+    return -1;
   if (wdtype != MOE_DTYPE_BF16 && wdtype != MOE_DTYPE_FP8_BLOCK128 && wdtype != MOE_DTYPE_FP8_PER_TENSOR &&
       wdtype != MOE_DTYPE_MXFP8)
     return -1;

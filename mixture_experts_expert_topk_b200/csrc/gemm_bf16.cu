@@ -218,6 +218,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t pol_a = policy_evict_last();
       int rslot = 0, sa = 0;
       uint32_t rph = 0, pha = 0;
+      uint32_t fills = 0;
       bool ok = true;
       while (ok) {
         const int tile = ring_take(ringfull0, ringempty0, ring, rslot, rph, abort_flag, a.status);
@@ -230,12 +231,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           mbar_arrive_expect_tx(fullA0 + 8 * sa, kStageA);
           tma_load_2d(sA + sa * kStageA, &tmA, fullA0 + 8 * sa, kb * 64, mb * kBM, pol_a);
+          ++fills;
           if (++sa == SA) {
             sa = 0;
             pha ^= 1u;
           }
         }
       }
+      drain_fills(fullA0, SA, fills);  // no A copy may land after the CTA exits
     }
   } else if (warp == kWarpSched) {
     // ---------------- tile scheduler + B producer ----------------
@@ -246,6 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t b_bytes = static_cast<uint32_t>(a.BN) * kBKBytes;
       int wslot = 0, sb = 0;
       uint32_t wph = 0, phb = 0;
+      uint32_t fills = 0;
       int tile = atomicAdd(a.tile_counter, 1);
       while (true) {
         if (!mbar_wait(ringempty0 + 8 * wslot, wph ^ 1u, abort_flag, a.status, kSiteTileEmpty)) break;
@@ -269,6 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           mbar_arrive_expect_tx(fullB0 + 8 * sb, b_bytes);
           tma_load_2d(sB + sb * kStageB, &tmB, fullB0 + 8 * sb, kb * 64, brow, pol_b);
+          ++fills;
           if (++sb == SB) {
             sb = 0;
             phb ^= 1u;
@@ -277,6 +282,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         tile = next;
       }
+      drain_fills(fullB0, SB, fills);  // no B copy may land after the CTA exits
     }
   } else if (warp == kWarpMma) {
     // ---------------- MMA issuer ----------------
@@ -332,7 +338,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // previous store drains.
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
     const uint32_t staging = sStage + (warp - kWarpEpi) * a.staging_bufs * a.staging_bytes;
-    const bool gated = a.activation != 1;  // 0 SwiGLU, 2 gelu_tanh; 1 relu2
+    const bool gated = a.activation != 1;  // 0 SwiGLU, 2 gelu_tanh, 3 swigluoai; 1 relu2
     // GEMM1: act bf16 rows of 16 (gated) or 32 (relu2) columns per box, no swizzle;
     // GEMM2: y fp32 rows of 32 columns (128 B), 128-byte swizzle
     const int box_cols = a.mode == 0 ? (gated ? 16 : 32) : 32;
@@ -379,7 +385,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < 8; ++i) {
               const float g0 = __uint_as_float(v[4 * i + 0]), u0 = __uint_as_float(v[4 * i + 1]);
               const float g1 = __uint_as_float(v[4 * i + 2]), u1 = __uint_as_float(v[4 * i + 3]);
-              o[i] = pack_bf16x2(gate_act(g0, a.activation) * u0, gate_act(g1, a.activation) * u1);
+              o[i] = pack_bf16x2(gated_act(g0, u0, a.activation), gated_act(g1, u1, a.activation));
             }
             const uint32_t dst = buf + lane * 32;
             asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(o[0]), "r"(o[1]), "r"(o[2]),

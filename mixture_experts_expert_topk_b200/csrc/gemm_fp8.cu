@@ -199,6 +199,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t pol_a = policy_evict_last();
       int rslot = 0, sa = 0;
       uint32_t rph = 0, pha = 0;
+      uint32_t fills = 0;
       bool ok = true;
       while (ok) {
         const int tile = ring_take(ringfull0, ringempty0, ring, rslot, rph, abort_flag, a.status);
@@ -211,12 +212,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           mbar_arrive_expect_tx(fullA0 + 8 * sa, kStageA);
           tma_load_2d(sA + sa * kStageA, &tmA, fullA0 + 8 * sa, kb * kBKBytes, mb * kBM, pol_a);
+          ++fills;
           if (++sa == kStagesA) {
             sa = 0;
             pha ^= 1u;
           }
         }
       }
+      drain_fills(fullA0, kStagesA, fills);  // no A copy may land after the CTA exits
     }
   } else if (warp == kWarpSched) {
     // ---------------- tile scheduler + B producer ----------------
@@ -224,6 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t pol_b = gather_a ? policy_evict_first() : policy_evict_last();
       int wslot = 0, sb = 0;
       uint32_t wph = 0, phb = 0;
+      uint32_t fills = 0;
       int tile = atomicAdd(a.tile_counter, 1);
       while (true) {
         if (!mbar_wait(ringempty0 + 8 * wslot, wph ^ 1u, abort_flag, a.status, kSiteTileEmpty)) break;
@@ -247,6 +251,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           mbar_arrive_expect_tx(fullB0 + 8 * sb, kStageB);
           tma_load_2d(sB + sb * kStageB, &tmB, fullB0 + 8 * sb, kb * kBKBytes, brow, pol_b);
+          ++fills;
           if (++sb == kStagesB) {
             sb = 0;
             phb ^= 1u;
@@ -255,6 +260,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         tile = next;
       }
+      drain_fills(fullB0, kStagesB, fills);  // no B copy may land after the CTA exits
     }
   } else if (warp == kWarpMma) {
     // ---------------- MMA issuer: one partial per K block ----------------
@@ -303,7 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------- promotion + epilogue (warps 6..9) ----------------
     const int q = warp & 3;
     const uint32_t staging = sStage + (warp - kWarpEpi) * 2 * kStagingBuf;
-    const bool gated = a.activation != 1;  // 0 SwiGLU, 2 gelu_tanh; 1 relu2
+    const bool gated = a.activation != 1;  // 0 SwiGLU, 2 gelu_tanh, 3 swigluoai; 1 relu2
     int nst = 0;
     int np = 0;
     int rslot = 0;
@@ -387,8 +393,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (gated) {
 #pragma unroll
             for (int i = 0; i < 32; ++i)
-              o[i] = pack_bf16x2(gate_act(acc[4 * i], a.activation) * acc[4 * i + 1],
-                                 gate_act(acc[4 * i + 2], a.activation) * acc[4 * i + 3]);
+              o[i] = pack_bf16x2(gated_act(acc[4 * i], acc[4 * i + 1], a.activation),
+                                 gated_act(acc[4 * i + 2], acc[4 * i + 3], a.activation));
           } else {
 #pragma unroll
             for (int i = 0; i < 32; ++i) {

@@ -12,7 +12,8 @@
 // A TMEM lane is one weight row. GEMM1: the gate and up rows of an intermediate index sit
 // in adjacent lanes (the [gate0, up0, gate1, up1, ...] interleave prepared at load time,
 // "[MoE] SwiGLU fusion into the MoE up-GEMM epilogue", sglang PR 32944, section 3) and are
-// paired with one shuffle before act(gate)*up (silu or gelu_tanh; or relu2); the kernel writes only the
+// paired with one shuffle before the gated activation (silu(gate)*up, gelu_tanh(gate)*up or
+// swigluoai; or relu2 without a gate); the kernel writes only the
 // bf16 activation. GEMM2: the epilogue multiplies token column j by topk_w of its pair and
 // writes fp32 y rows (sorted order) for the fixed-order combine.
 //
@@ -95,7 +96,7 @@ static_assert(kSmemBytes <= kSmemCap, "shared memory");
 
 enum : int {
   kSiteEmpty = 1, kSiteFull = 2, kSiteTmemEmpty = 3, kSiteTmemFull = 4, kSiteTileFull = 5, kSiteTileEmpty = 6,
-  kSiteEmptyX = 7, kSiteSfFree = 8
+  kSiteEmptyX = 7, kSiteSfFree = 8, kSiteFullX = 9
 };
 
 struct Args {
@@ -209,7 +210,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
   const uint32_t rfull0 = tempty0 + 16;
   const uint32_t rempty0 = rfull0 + 8 * kTileRing;
   const uint32_t drain_bar = rempty0 + 8 * kTileRing;
-  uint64_t* step_end_w = bars + 2 * kSlots + 4 + 2 * kTileRing + 1;           // [kSlots]
+  const uint32_t fullx0 = drain_bar + 8;                                      // [kSlots]
+  uint64_t* step_end_w = bars + 3 * kSlots + 4 + 2 * kTileRing + 1;           // [kSlots]
   uint64_t* step_end_x = step_end_w + kSlots;                                 // [kSlots]
   volatile int* ring = reinterpret_cast<volatile int*>(step_end_x + kSlots);  // [kTileRing][4]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(const_cast<int*>(ring) + 4 * kTileRing);
@@ -220,7 +222,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kSlots; ++s) {
-      mbar_init(full0 + 8 * s, 2);  // the W and the X expect-tx arrivals
+      mbar_init(full0 + 8 * s, 1);   // the W copies of a step
+      mbar_init(fullx0 + 8 * s, 1);  // the X copies of a step
       mbar_init(empty0 + 8 * s, 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -303,6 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
         }
         tile = next;
       }
+      drain_fills(full0, kSlots, ks);  // no W copy may land after the CTA exits
     }
   } else if (warp == kWarpX) {
     // ---------------- X producer ----------------
@@ -325,7 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
             ok = false;
             break;
           }
-          const uint32_t full = full0 + 8 * (ks % kSlots);
+          const uint32_t full = fullx0 + 8 * (ks % kSlots);
           const uint32_t bytes = static_cast<uint32_t>(kcs * n) * kChunkBytes;
           const uint32_t sf_bytes = kMx ? static_cast<uint32_t>(kcs) * kSfX : 0u;
           mbar_arrive_expect_tx(full, bytes + sf_bytes);
@@ -335,6 +339,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
                       a.x_sf + (static_cast<size_t>(x_row >> 4) * a.k_chunks + c0) * kSfX, sf_bytes, full, pol);
         }
       }
+      drain_fills(fullx0, kSlots, ks);  // no X copy may land after the CTA exits
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
@@ -356,7 +361,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
         for (int c0 = 0; c0 < a.k_chunks; c0 += kc, ++ks) {
           const int kcs = min(kc, a.k_chunks - c0);
           const uint32_t base = s0 + ring_alloc(pos, head, step_bytes<kMx>(kcs, n));
-          if (!mbar_wait(full0 + 8 * (ks % kSlots), (ks / kSlots) & 1u, abort_flag, a.status, kSiteFull)) {
+          if (!mbar_wait(full0 + 8 * (ks % kSlots), (ks / kSlots) & 1u, abort_flag, a.status, kSiteFull) ||
+              !mbar_wait(fullx0 + 8 * (ks % kSlots), (ks / kSlots) & 1u, abort_flag, a.status, kSiteFullX)) {
             ok = false;
             break;
           }
@@ -417,7 +423,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
     // neighbouring output columns, so each store writes one contiguous piece of an output
     // row (GEMM2: 128 B of fp32; GEMM1: 64 or 32 B of a 128-byte activation chunk row).
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
-    const bool gated = a.activation != 1;  // 0 SwiGLU, 2 gelu_tanh; 1 relu2
+    const bool gated = a.activation != 1;  // 0 SwiGLU, 2 gelu_tanh, 3 swigluoai; 1 relu2
     const bool odd = (lane & 1) != 0;
     int rslot = 0, it = 0;
     uint32_t rph = 0;
@@ -511,7 +517,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
             const float u = odd ? mine_hi : other;
             const int row = c0 + (odd ? 16 + j : j);
             if (!odd || full) {
-              const float h = gate_act(g, a.activation) * u;
+              const float h = gated_act(g, u, a.activation);
               uint8_t* dst = act_grp + row * kChunkBytes + ((((fo >> 4) ^ row) & 7) << 4) + (fo & 15);
               if (kFp8)
                 *dst = __nv_cvt_float_to_fp8(h * a.act_inv, __NV_SATFINITE, __NV_E4M3);

@@ -66,23 +66,27 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Wait for the phase of parity `parity` of barrier `bar` to complete. Gives up when
-// another thread of the CTA has raised `*abort` or after kWaitTimeoutNs; a timeout
-// raises `*abort` and records `kStatusTimeout | site` in the device status word.
-// Returns true when the phase completed.
-static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort,
-                                            int* status, int site) {
+// another thread of the CTA has raised `*abort` or after `limit_ns`; a timeout raises
+// `*abort` and records `kStatusTimeout | site` in the device status word. Returns true
+// when the phase completed.
+static __device__ __noinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort,
+                                                      int* status, int site, unsigned long long limit_ns) {
   const unsigned long long t0 = globaltimer_ns();
   for (uint32_t i = 0;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 31u) == 31u) {
       if (*abort) return false;
-      if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         *abort = 1;
         atomicCAS(status, 0, kStatusTimeout | site);
         return false;
       }
     }
   }
+}
+static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort,
+                                                   int* status, int site) {
+  return mbar_wait_bounded(bar, parity, abort, status, site, kWaitTimeoutNs);
 }
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
                                           int* status, int site) {
@@ -96,6 +100,17 @@ static __device__ __noinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parit
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 31u) == 31u && globaltimer_ns() - t0 > kWaitTimeoutNs) return false;
   }
+}
+
+// Before a producer thread leaves (normally or after an abort): wait, bounded, until the
+// copies it issued into a ring of `stages` full barriers (one arrival each, from this
+// thread only, stage s at full0 + 8 s) have landed, so that no copy writes shared memory
+// after the CTA exits. `fills` counts the stages this thread filled, in order from
+// stage 0; fill i used stage i % stages with phase parity (i / stages) & 1. On the
+// normal path every fill was consumed long ago and each wait returns at once.
+__device__ __forceinline__ void drain_fills(uint32_t full0, uint32_t stages, uint32_t fills) {
+  const uint32_t first = fills > stages ? fills - stages : 0u;
+  for (uint32_t i = first; i < fills; ++i) mbar_wait_drain(full0 + 8 * (i % stages), (i / stages) & 1u);
 }
 
 // ---- TMA -----------------------------------------------------------------------------
@@ -342,6 +357,21 @@ __device__ __forceinline__ float gelu_tanh_f32(float g) {
 
 // Gate activation of a gated layer: act 0 = SwiGLU (silu), 2 = gelu_tanh.
 __device__ __forceinline__ float gate_act(float g, int act) { return act == 2 ? gelu_tanh_f32(g) : silu_f32(g); }
+
+// The SwiGLU variant published with OpenAI's gpt-oss models (alpha 1.702, limit 7): the gate
+// clamped from above and the up value to [-7, 7], then g sigmoid(1.702 g) (u + 1). The
+// division is the fast one, as in silu_f32 (a very negative g gives 0).
+__device__ __forceinline__ float swigluoai_f32(float g, float u) {
+  const float gc = fminf(g, 7.0f);
+  const float uc = fminf(fmaxf(u, -7.0f), 7.0f);
+  return __fdividef(gc, 1.0f + __expf(-1.702f * gc)) * (uc + 1.0f);
+}
+
+// Activation of a gated layer from its gate and up values: act 0 = SwiGLU, 2 = gelu_tanh
+// (act(gate) * up), 3 = swigluoai.
+__device__ __forceinline__ float gated_act(float g, float u, int act) {
+  return act == 3 ? swigluoai_f32(g, u) : gate_act(g, act) * u;
+}
 
 // ---- MXFP8 (OCP Microscaling v1.0: E4M3 values, one E8M0 power-of-two scale per 32) ----
 

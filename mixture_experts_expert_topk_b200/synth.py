@@ -36,7 +36,7 @@ class MoeConfig:
     topk: int              # routed experts per token
     I: int                 # intermediate size (unpadded)
     renormalize: bool
-    activation: str        # "swiglu" | "relu2" | "gelu_tanh"
+    activation: str        # "swiglu" | "relu2" | "gelu_tanh" | "swigluoai"
     num_shared: int = 0    # fused shared-expert slots appended after the routed experts
     # False: bf16. True: e4m3 with 128-wide block scales. "per_tensor": e4m3 with one scale
     # per expert matrix and static input / activation scales (activation_scale below; the
@@ -114,6 +114,15 @@ CONFIGS["mxfp8_prefill"] = MoeConfig("mxfp8_prefill", T=4096, H=2048, E=256, top
 CONFIGS["prefill_e64"] = MoeConfig("prefill_e64", T=1024, H=2048, E=64, topk=8, I=512,
                                    renormalize=True, activation="swiglu", logit_bias_std=0.5)
 CONFIGS["mxfp8_e64"] = CONFIGS["prefill_e64"].replace(name="mxfp8_e64", fp8="mxfp8")
+CONFIGS["fp8_e64"] = CONFIGS["prefill_e64"].replace(name="fp8_e64", fp8=True)
+
+
+# A compute-bound case of the prefill kernels: the prefill shapes (H=2048, I=512, SwiGLU,
+# top-8) with 8 experts and 16384 tokens, so every expert receives 16384 rows (about 16k
+# tokens per expert, far above the ~250 flop/byte ridge) and the grouped GEMMs are bound
+# by the tensor cores rather than by the weight stream.
+CONFIGS["compute_diag"] = MoeConfig("compute_diag", T=16384, H=2048, E=8, topk=8, I=512, renormalize=True,
+                                    activation="swiglu")
 
 
 def decode_config(T: int) -> MoeConfig:

@@ -13,7 +13,7 @@ The layer (one forward call) computes, for every token t with hidden row x_t:
   2. align:   stable sort of the (token, slot) pairs by expert, each expert's
               segment padded to the GEMM row tile ``block_m``;
   3. GEMM1:   z = W13[e] x_t, then a gated activation act(gate)*up (SwiGLU: silu;
-              gelu_tanh) or relu2 max(z,0)^2;
+              gelu_tanh), swigluoai(gate, up), or relu2 max(z,0)^2;
   4. GEMM2:   y = w_tj * (W2[e] a);
   5. combine: out_t = sum_j y_tj in slot order j = 0..k'-1.
 
@@ -342,7 +342,23 @@ def gelu_tanh(x: np.ndarray) -> np.ndarray:
     return 0.5 * x * (1.0 + np.tanh(math.sqrt(2.0 / math.pi) * (x + 0.044715 * x * x * x)))
 
 
-GATED_ACTIVATIONS = ("swiglu", "gelu_tanh")
+SWIGLUOAI_ALPHA = 1.702   # sigmoid slope of the gpt-oss SwiGLU
+SWIGLUOAI_LIMIT = 7.0     # its clamp on the gate (from above) and on the up value
+
+
+def swigluoai(gate: np.ndarray, up: np.ndarray) -> np.ndarray:
+    """``swigluoai_uninterleave``, a SwiGLU variant among the gated activations of [GATED]
+    section 2, which reuses the standard formula without printing it. Reading taken: the
+    SwiGLU published with OpenAI's gpt-oss models, on gate and up halves that are not
+    interleaved (the gate-first checkpoint layout of SwiGLU here):
+      g = min(gate, 7),  u = clamp(up, -7, 7),  a = g * sigmoid(1.702 g) * (u + 1)."""
+    g = np.minimum(gate, SWIGLUOAI_LIMIT)
+    u = np.clip(up, -SWIGLUOAI_LIMIT, SWIGLUOAI_LIMIT)
+    with np.errstate(over="ignore"):
+        return g / (1.0 + np.exp(-SWIGLUOAI_ALPHA * g)) * (u + 1.0)
+
+
+GATED_ACTIVATIONS = ("swiglu", "gelu_tanh", "swigluoai")
 
 
 def is_gated(activation: str) -> bool:
@@ -354,9 +370,12 @@ def activation_fn(z: np.ndarray, activation: str, I: int) -> np.ndarray:
 
     Gated: a = act(z[:, :I]) * z[:, I:2I] with act = silu for SwiGLU ([SWIGLU]
     section 1, ``silu(gate) * up``) or gelu_tanh ([GATED] section 2; [GATED]
-    section 1: activation(gate) * up).
+    section 1: activation(gate) * up); swigluoai(z[:, :I], z[:, I:2I]) ([GATED]
+    section 2).
     relu2: a = relu2(z) over the I columns.
     """
+    if activation == "swigluoai":
+        return swigluoai(z[:, :I], z[:, I:2 * I])
     if is_gated(activation):
         act = silu if activation == "swiglu" else gelu_tanh
         return act(z[:, :I]) * z[:, I:2 * I]

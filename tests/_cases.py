@@ -152,3 +152,124 @@ def untile_weights(flat_bits: np.ndarray, E: int, rows: int, K: int) -> np.ndarr
     phys = np.arange(8)[None, :] ^ (r[:, None] & 7)
     u = t[:, :, :, r[:, None], phys, :]                          # [E, MT, KC, 128, 8, 8]
     return u.transpose(0, 1, 3, 2, 4, 5).reshape(E, MT * 128, KC * 64)
+
+
+def cover_tokens(ids: np.ndarray, num_routed: int, extra: int = 0, seed: int = 0) -> np.ndarray:
+    """A token sample in which every routed expert that receives any pair appears at
+    least once: tokens taken greedily (most still-uncovered routed experts first, lowest
+    index on ties), plus ``extra`` more drawn at random. Ids >= num_routed (the shared
+    slot) count as covered. Returns sorted token indices."""
+    clipped = np.minimum(np.asarray(ids), num_routed)
+    covered = np.ones(num_routed + 1, dtype=bool)
+    covered[np.unique(clipped[clipped < num_routed])] = False
+    chosen = []
+    while not covered.all():
+        t = int(np.argmax((~covered[clipped]).sum(axis=1)))
+        chosen.append(t)
+        covered[clipped[t]] = True
+    rest = np.setdiff1d(np.arange(clipped.shape[0]), chosen)
+    if extra > 0 and rest.size:
+        chosen += list(np.random.default_rng(seed).choice(rest, size=min(extra, rest.size), replace=False))
+    return np.sort(np.asarray(chosen, dtype=np.int64))
+
+
+def per_expert_threaded(fn, experts, workers: int = 8) -> dict:
+    """{e: fn(e)} for every listed expert, evaluated on a thread pool (the oracle's
+    NumPy routines release the interpreter lock inside their array operations)."""
+    from concurrent.futures import ThreadPoolExecutor
+    experts = [int(e) for e in experts]
+    with ThreadPoolExecutor(max_workers=workers) as ex:
+        return dict(zip(experts, ex.map(fn, experts)))
+
+
+def oracle_fp8_block_weights(w13_bits, w2_bits, experts):
+    """O.quantize_weights_fp8 for the listed experts (others zero), expert by expert on
+    a thread pool."""
+    E = w13_bits.shape[0]
+    w13_q = np.zeros(w13_bits.shape, dtype=np.uint8)
+    w2_q = np.zeros(w2_bits.shape, dtype=np.uint8)
+    w13_s = np.zeros((E, w13_bits.shape[1] // 128, w13_bits.shape[2] // 128), dtype=np.float32)
+    w2_s = np.zeros((E, w2_bits.shape[1] // 128, w2_bits.shape[2] // 128), dtype=np.float32)
+
+    def one(e):
+        return (O.quant_blocks_128x128(O.bf16_bits_to_f32(np.asarray(w13_bits[e]))),
+                O.quant_blocks_128x128(O.bf16_bits_to_f32(np.asarray(w2_bits[e]))))
+
+    for e, ((q13, s13), (q2, s2)) in per_expert_threaded(one, experts).items():
+        w13_q[e], w13_s[e], w2_q[e], w2_s[e] = q13, s13, q2, s2
+    return w13_q, w13_s, w2_q, w2_s
+
+
+def oracle_mxfp8_weights(w13_bits, w2_bits, experts):
+    """O.quantize_weights_mxfp8 for the listed experts (others zero), on a thread pool."""
+    E, N1, H = w13_bits.shape
+    I = w2_bits.shape[2]
+    out = [np.zeros((E, N1, H), np.uint8), np.zeros((E, N1, H // 32), np.uint8),
+           np.zeros((E, H, I), np.uint8), np.zeros((E, H, I // 32), np.uint8)]
+
+    def one(e):
+        return (O.quant_mx(O.bf16_bits_to_f32(np.asarray(w13_bits[e]))),
+                O.quant_mx(O.bf16_bits_to_f32(np.asarray(w2_bits[e]))))
+
+    for e, ((q13, s13), (q2, s2)) in per_expert_threaded(one, experts).items():
+        out[0][e], out[1][e], out[2][e], out[3][e] = q13, s13, q2, s2
+    return tuple(out)
+
+
+def sampled_pairs(ids: np.ndarray, tokens: np.ndarray):
+    """(token, slot, expert) of every pair of the sampled tokens."""
+    t = np.repeat(np.asarray(tokens, dtype=np.int64), ids.shape[1])
+    j = np.tile(np.arange(ids.shape[1]), len(tokens))
+    return t, j, ids[t, j]
+
+
+def check_act_pairs(ref_fn, got_rows: np.ndarray, ids: np.ndarray, tokens: np.ndarray, pair_to_row: np.ndarray,
+                    bound_fn) -> float:
+    """GEMM1's stored activation of every pair of the sampled tokens against the oracle's.
+    ref_fn(e, token_indices) -> reference activation rows [n, I] (float64); got_rows[r] is
+    the kernel's activation of sorted row r (float64, [rows, I]); bound_fn(ref, got) ->
+    True where the element is within its bound. Returns the number of elements checked."""
+    kk = ids.shape[1]
+    t, j, e = sampled_pairs(ids, tokens)
+    n = 0
+    for ex in np.unique(e):
+        sel = e == ex
+        ref = ref_fn(int(ex), t[sel])
+        got = got_rows[pair_to_row[t[sel] * kk + j[sel]], :ref.shape[1]]
+        ok = bound_fn(ref, got)
+        if not np.all(ok):
+            bad = np.argwhere(~ok)[0]
+            raise AssertionError(f"activation of expert {ex}, pair {bad}: got {got[tuple(bad)]}, ref {ref[tuple(bad)]}")
+        n += ref.size
+    return n
+
+
+def bf16_act_bound(ref: np.ndarray, got: np.ndarray) -> np.ndarray:
+    """A bf16-stored activation: its rounding (2^-8 relative, with room for fp32
+    accumulation order) plus 1e-3 of the RMS of the checked rows."""
+    return np.abs(got - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-3 * O.rms(ref) + 1e-30
+
+
+def act_rows_f64(parts: Dict[str, np.ndarray], I_pad: int) -> np.ndarray:
+    """GEMM1's bf16 activation as float64 [rows, I_pad] in sorted row order, from the
+    row-group layout (block_m 16) or the row-major one (block_m 128)."""
+    if parts["block_m"] == 16:
+        rows = parts["sorted_pair_ids"].shape[0]
+        b = untile_groups(parts["act"], parts["group_info"], int(parts["num_blocks"][1]), rows, -(-I_pad // 64))
+        return bf16_to_f64(b[:, :I_pad])
+    return bf16_to_f64(parts["act"])
+
+
+def untile_u8(flat, group_info, num_groups, rows, kchunks):
+    """Row-major [rows, 128 * kchunks] bytes from row-group order with 128-byte chunks of
+    e4m3 codes (row j's 16-byte piece q stored at position q ^ (j % 8))."""
+    flat = np.asarray(flat).reshape(-1)
+    out = np.zeros((rows, 128 * kchunks), dtype=np.uint8)
+    for g in range(num_groups):
+        x_row, meta = int(group_info[g][0]), int(group_info[g][1])
+        n = meta >> 16
+        grp = flat[x_row * 128 * kchunks:(x_row + n) * 128 * kchunks].reshape(kchunks, n, 8, 16)
+        j = np.arange(n)
+        phys = np.arange(8)[None, :] ^ (j[:, None] & 7)
+        out[x_row:x_row + n] = grp[:, j[:, None], phys, :].transpose(1, 0, 2, 3).reshape(n, 128 * kchunks)
+    return out

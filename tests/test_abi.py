@@ -87,6 +87,8 @@ def test_padded_intermediate_follows_page_rule(L):
     assert L.moe_padded_intermediate(0, 0, 0) == -1
     assert L.moe_padded_intermediate(200, _capi.MOE_ACT_SWIGLU, _capi.MOE_DTYPE_FP8_PER_TENSOR) == 256
     assert L.moe_padded_intermediate(200, _capi.MOE_ACT_GELU_TANH, 0) == 208
+    assert L.moe_padded_intermediate(200, _capi.MOE_ACT_SWIGLUOAI, 0) == 208   # gated: 16
+    assert L.moe_padded_intermediate(200, 4, 0) == -1                          # no such activation
     assert L.moe_padded_intermediate(200, 0, _capi.MOE_DTYPE_MXFP8) == 256   # MXFP8: 128
     assert L.moe_padded_intermediate(200, 0, 4) == -1
     assert L.moe_padded_intermediate(16, 7, 0) == -1

@@ -18,8 +18,9 @@ import mixture_experts_expert_topk_b200 as moe
 from mixture_experts_expert_topk_b200.synth import CONFIGS, MoeConfig, make_inputs
 from oracle import moe_oracle as O
 
-from _cases import (GpuForward, bf16_to_f64, bits, cpu_inputs, err_beyond_rounding, max_err_over_rms, oracle_out,
-                    untile_groups, untile_weights)
+from _cases import (GpuForward, act_rows_f64, bf16_act_bound, bf16_to_f64, bits, check_act_pairs, cover_tokens,
+                    cpu_inputs, err_beyond_rounding, max_err_over_rms, oracle_fp8_block_weights, oracle_mxfp8_weights,
+                    oracle_out, untile_groups, untile_u8, untile_weights)
 
 pytestmark = pytest.mark.gpu
 
@@ -57,6 +58,10 @@ SMALL = {
     # the gelu_tanh gated activation, both GEMM paths (with an unaligned intermediate)
     "gelu_small": _small("gelu_small", T=300, H=256, E=8, topk=2, I=200, activation="gelu_tanh"),
     "gelu_big": _small("gelu_big", T=600, H=256, E=6, topk=2, I=256, activation="gelu_tanh"),
+    # swigluoai; weights large enough (z ~ N(0, 8^2)) that both of its clamps are active
+    "oai_small": _small("oai_small", T=300, H=256, E=8, topk=2, I=200, activation="swigluoai", weight_std=0.5),
+    "oai_big": _small("oai_big", T=600, H=256, E=6, topk=2, I=256, activation="swigluoai", weight_std=0.5,
+                      num_shared=1),
 }
 
 
@@ -141,7 +146,8 @@ def _check_act(cfg, run, parts, ids, a):
 
 
 @pytest.mark.parametrize("name,bm", [(n, 0) for n in SMALL] +
-                         [(n, 128) for n in ("ragged", "skewed", "pad_gated", "relu2_small", "gelu_small")])
+                         [(n, 128) for n in ("ragged", "skewed", "pad_gated", "relu2_small", "gelu_small",
+                                             "oai_small")])
 def test_layer_parity_small(name, bm):
     # bm 0: the default (bf16: 16-row alignment, weights on the MMA's M); 128: token tiles
     cfg = SMALL[name]
@@ -297,10 +303,9 @@ def _full_size(cfg, n_sample=48, seed=0):
     return err_beyond_rounding(got, ref), run
 
 
-@pytest.mark.parametrize("name,n_sample", [("prefill", 4096), ("relu2", 512), ("fp8_shared", 8)])
+@pytest.mark.parametrize("name,n_sample", [("prefill", 4096), ("relu2", 512)])
 def test_workload_full_size(name, n_sample):
-    # prefill: every token; relu2 (541 GFLOP in float64): a quarter of the tokens;
-    # FP8 with the shared slot: 8 tokens (the oracle quantises each expert they touch)
+    # prefill: every token; relu2 (541 GFLOP in float64): a quarter of the tokens
     cfg = CONFIGS[name]
     e, run = _full_size(cfg, n_sample=n_sample)
     assert e <= (FP8_TOL if cfg.fp8 else BF16_TOL), e
@@ -327,6 +332,7 @@ FP8_SMALL = {
     "fp8_relu2": _small("fp8_relu2", T=96, H=256, E=6, topk=2, I=256, activation="relu2", renormalize=False,
                         fp8=True),
     "fp8_gelu": _small("fp8_gelu", T=64, H=256, E=8, topk=2, I=256, activation="gelu_tanh", fp8=True),
+    "fp8_oai": _small("fp8_oai", T=200, H=256, E=8, topk=2, I=256, activation="swigluoai", fp8=True, weight_std=0.5),
 }
 
 
@@ -352,6 +358,13 @@ def test_fp8_layer_parity_small(name):
     fp8w = O.quantize_weights_fp8(bits(run.inp["w13"]), bits(run.inp["w2"]))
     np.testing.assert_array_equal(run.w13_q.cpu().numpy(), fp8w[0])
     np.testing.assert_array_equal(run.w13_scale.cpu().numpy(), fp8w[1])
+    # GEMM1's bf16 activation element by element against the oracle's activation of the
+    # same quantised operands (before its 1x128 re-quantisation)
+    xd = O.dequant_groups_1x128(qx, sx)
+    check_act_pairs(
+        lambda e, t: O.activation_fn(xd[t] @ O.dequant_blocks_128x128(fp8w[0][e], fp8w[1][e]).T, cfg.activation,
+                                     cfg.I),
+        act_rows_f64(parts, run.I_pad), ids, np.arange(cfg.T), a["pair_to_row"], bf16_act_bound)
     ref = oracle_out(cfg, run.inp, fp8_weights=fp8w)
     got = bf16_to_f64(out)
     assert np.all(np.isfinite(got))
@@ -457,22 +470,8 @@ PT_SMALL = {
     # groups of more than 128 rows (one K chunk per step) and three align chunks
     "pt_big_groups": _small("pt_big_groups", T=1500, H=256, E=4, topk=2, I=128),
     "pt_decode": _small("pt_decode", T=4, H=512, E=32, topk=4, I=256),
+    "pt_oai": _small("pt_oai", T=200, H=256, E=8, topk=2, I=256, activation="swigluoai", weight_std=0.5),
 }
-
-
-def _untile_u8(flat, group_info, num_groups, rows, kchunks):
-    """Row-major [rows, 128 * kchunks] bytes from row-group order with 128-byte chunks of
-    e4m3 codes (row j's 16-byte piece q stored at position q ^ (j % 8))."""
-    flat = np.asarray(flat).reshape(-1)
-    out = np.zeros((rows, 128 * kchunks), dtype=np.uint8)
-    for g in range(num_groups):
-        x_row, meta = int(group_info[g][0]), int(group_info[g][1])
-        n = meta >> 16
-        grp = flat[x_row * 128 * kchunks:(x_row + n) * 128 * kchunks].reshape(kchunks, n, 8, 16)
-        j = np.arange(n)
-        phys = np.arange(8)[None, :] ^ (j[:, None] & 7)
-        out[x_row:x_row + n] = grp[:, j[:, None], phys, :].transpose(1, 0, 2, 3).reshape(n, 128 * kchunks)
-    return out
 
 
 @pytest.mark.parametrize("name", list(PT_SMALL))
@@ -517,7 +516,7 @@ def test_fp8_per_tensor_layer_parity(name):
     np.testing.assert_array_equal(parts["sorted_pair_ids"][:P_pad], al["sorted_pair_ids"])
     # the permuted, quantised hidden rows: e4m3(hidden * fp32(1 / input_scale)), bit for bit
     ng = int(parts["num_blocks"][1])
-    xs = _untile_u8(parts["xs"], parts["group_info"], ng, P_pad, cfg.H // 128)
+    xs = untile_u8(parts["xs"], parts["group_info"], ng, P_pad, cfg.H // 128)
     pids = al["sorted_pair_ids"][:P_pad]
     real = pids < cfg.T * cfg.k_total
     xq = O.quant_per_tensor_inv(O.bf16_bits_to_f32(bits(inp["hidden"])), s_in)
@@ -546,6 +545,8 @@ MX_SMALL = {
     # and three align chunks
     "mx_big_groups": _small("mx_big_groups", T=1500, H=256, E=4, topk=2, I=128, fp8="mxfp8"),
     "mx_decode": _small("mx_decode", T=4, H=512, E=32, topk=4, I=256, fp8="mxfp8"),
+    "mx_oai": _small("mx_oai", T=200, H=256, E=8, topk=2, I=256, activation="swigluoai", fp8="mxfp8",
+                     weight_std=0.5),
 }
 
 
@@ -637,7 +638,7 @@ def _mx_parity(cfg, inp, name):
     pids = al["sorted_pair_ids"][:P_pad]
     real = pids < cfg.T * cfg.k_total
     xq, xsc = O.quant_mx(O.bf16_bits_to_f32(bits(inp["hidden"])))
-    xs = _untile_u8(parts["xs"], gi, ng, P_pad, cfg.H // 128)
+    xs = untile_u8(parts["xs"], gi, ng, P_pad, cfg.H // 128)
     np.testing.assert_array_equal(xs[real], xq[pids[real] // cfg.k_total])
     assert np.all(xs[~real] == 0)
     xss = _mx_group_scales(parts["xs_scale"], gi, ng, P_pad, cfg.H // 128)
@@ -646,7 +647,7 @@ def _mx_parity(cfg, inp, name):
     # GEMM2's input: the kernel's own bf16 activation quantised per 32, bit for bit
     act = untile_groups(act_bits, gi, ng, P_pad, -(-cfg.I // 64))[:, :cfg.I]
     aq, asc = O.quant_mx(O.bf16_bits_to_f32(act))
-    np.testing.assert_array_equal(_untile_u8(parts["actq"], gi, ng, P_pad, cfg.I // 128), aq)
+    np.testing.assert_array_equal(untile_u8(parts["actq"], gi, ng, P_pad, cfg.I // 128), aq)
     np.testing.assert_array_equal(_mx_group_scales(parts["act_scale"], gi, ng, P_pad, cfg.I // 128), asc)
     # the layer
     ref = O.moe_forward_mxfp8(bits(inp["hidden"]), inp["logits"].numpy(), o13, os13, o2, os2, topk=cfg.topk,
@@ -658,8 +659,10 @@ def _mx_parity(cfg, inp, name):
     assert e <= FP8_TOL, e
 
 
-def test_mxfp8_full_size_sampled_tokens():
-    """The MXFP8 prefill workload at full size against the oracle on sampled tokens."""
+def test_mxfp8_full_size_every_expert():
+    """The MXFP8 prefill workload at full size: routing and align over all tokens, the
+    layer output and GEMM1's stored activation on a token sample that covers every
+    routed expert."""
     cfg = CONFIGS["mxfp8_prefill"]
     inp = make_inputs(cfg, 0)
     dev = torch.device("cuda:0")
@@ -668,18 +671,142 @@ def test_mxfp8_full_size_sampled_tokens():
     prob = moe.make_problem(cfg.T, cfg.H, cfg.E, cfg.topk, cfg.I, renormalize=cfg.renormalize,
                             activation=cfg.activation, fp8="mxfp8")
     w13p, w2p = moe.prepare_weights(prob, q13, q2, cfg.I, w13_scale=s13, w2_scale=s2)
+    del q13, q2, s13, s2
     ws = moe.new_workspace(prob)
     out = moe.moe_forward(inp["hidden"].to(dev), inp["logits"].to(dev), w13p, w2p, cfg.topk, cfg.renormalize,
                           cfg.activation, workspace=ws)
     torch.cuda.synchronize()
     assert moe.device_status(ws)[0] == 0
-    tokens = np.random.default_rng(5).choice(cfg.T, 24, replace=False)
-    ids, _ = O.route(inp["logits"].numpy()[tokens], cfg.topk, cfg.renormalize)
-    experts = sorted(set(int(e) for e in ids.reshape(-1)))
-    o13, os13, o2, os2 = O.quantize_weights_mxfp8(bits(inp["w13"]), bits(inp["w2"]), experts=experts)
+    raw = moe.read_workspace(prob, ws)
+    act_bits = raw.pop("act").view(torch.int16).cpu().numpy().view(np.uint16)
+    parts = {k: v.cpu().numpy() for k, v in raw.items()}
+    ids, _ = O.route(inp["logits"].numpy(), cfg.topk, cfg.renormalize)
+    np.testing.assert_array_equal(parts["topk_ids"], ids)
+    al = O.align(ids, cfg.E_total, 16)
+    P_pad = int(al["P_pad"])
+    np.testing.assert_array_equal(parts["sorted_pair_ids"][:P_pad], al["sorted_pair_ids"])
+    np.testing.assert_array_equal(parts["pair_to_row"], al["pair_to_row"])
+    tokens = cover_tokens(ids, cfg.E, extra=16)
+    experts = np.unique(ids[tokens])
+    assert len(experts) == len(np.unique(ids))
+    o13, os13, o2, os2 = oracle_mxfp8_weights(bits(inp["w13"]), bits(inp["w2"]), experts)
+    # GEMM1's bf16 activation of every sampled pair against the oracle's (same MXFP8 inputs)
+    gi, ng = parts["group_info"], int(parts["num_blocks"][1])
+    act = bf16_to_f64(untile_groups(act_bits, gi, ng, P_pad, -(-cfg.I // 64))[:, :cfg.I])
+    x = O.dequant_mx(*O.quant_mx(O.bf16_bits_to_f32(bits(inp["hidden"]))))
+    n = check_act_pairs(lambda e, t: O.activation_fn(x[t] @ O.dequant_mx(o13[e], os13[e]).T, cfg.activation, cfg.I),
+                        act, ids, tokens, al["pair_to_row"], bf16_act_bound)
     ref = O.moe_forward_mxfp8(bits(inp["hidden"]), inp["logits"].numpy(), o13, os13, o2, os2, topk=cfg.topk,
                               renormalize=cfg.renormalize, activation=cfg.activation, tokens=tokens)
     got = bf16_to_f64(out.cpu()[torch.from_numpy(tokens)])
     e = err_beyond_rounding(got, ref)
-    print(f"mxfp8_prefill: beyond-rounding {e:.4f} on {len(tokens)} tokens")
+    print(f"mxfp8_prefill: {len(tokens)} tokens over {len(experts)} experts, {n} activation values; "
+          f"beyond-rounding {e:.4f}, raw {max_err_over_rms(got, ref):.4f}")
+    assert e <= FP8_TOL, e
+
+
+def test_fp8_block128_full_size_every_expert():
+    """FP8 block-128 with the fused shared slot at full size (T=8192, 512+1 experts,
+    top-10+1): routing and align over all tokens; the quantised hidden rows bit for bit;
+    GEMM1's stored activation and the layer output on a token sample that covers every
+    routed expert."""
+    cfg = CONFIGS["fp8_shared"]
+    run = GpuForward(cfg)
+    out = run.forward()
+    parts = run.parts()
+    ids, a = _check_route_align(cfg, parts, run.inp["logits"])
+    hid32 = O.bf16_bits_to_f32(bits(run.inp["hidden"]))
+    qx, sx = O.quant_groups_1x128(hid32)
+    np.testing.assert_array_equal(parts["xq"], qx)
+    np.testing.assert_array_equal(parts["xq_scale"], sx)
+    tokens = cover_tokens(ids, cfg.E, extra=16)
+    experts = np.unique(ids[tokens])
+    assert len(experts) == cfg.E_total
+    fp8w = oracle_fp8_block_weights(bits(run.inp["w13"]), bits(run.inp["w2"]), experts)
+    xd = O.dequant_groups_1x128(qx, sx)
+    act = act_rows_f64(parts, run.I_pad)
+    n = check_act_pairs(
+        lambda e, t: O.activation_fn(xd[t] @ O.dequant_blocks_128x128(fp8w[0][e], fp8w[1][e]).T, cfg.activation,
+                                     cfg.I),
+        act, ids, tokens, a["pair_to_row"], bf16_act_bound)
+    ref = oracle_out(cfg, run.inp, tokens=tokens, fp8_weights=fp8w)
+    got = bf16_to_f64(out)[tokens]
+    assert np.all(np.isfinite(bf16_to_f64(out)))
+    e = err_beyond_rounding(got, ref)
+    print(f"fp8_shared: {len(tokens)} tokens over {len(experts)} experts, {n} activation values; "
+          f"beyond-rounding {e:.4f}, raw {max_err_over_rms(got, ref):.4f}")
+    assert e <= FP8_TOL, e
+    assert moe.device_status(run.ws)[0] == 0
+
+
+def _e4m3_within_one_step(ref_scaled: np.ndarray, got_codes: np.ndarray) -> np.ndarray:
+    """True where the code is the e4m3 rounding of ref_scaled (saturated at 448) or the
+    neighbouring value: fp32 accumulation against float64 may flip a rounding decision."""
+    r = np.clip(ref_scaled, -448.0, 448.0)
+    step = np.ldexp(1.0, np.maximum(np.floor(np.log2(np.maximum(np.abs(r), 2.0 ** -9))), -6).astype(np.int64) - 3)
+    return np.abs(O.e4m3_decode(got_codes) - r) <= step * (1 + 1e-9)
+
+
+def test_fp8_per_tensor_full_size_every_expert():
+    """Per-tensor FP8 with the fused shared slot at its full benchmarked shape (T=8192,
+    512+1 experts, top-10+1), with the static scales calibrated as the benchmark does
+    (input scale = amax(hidden) / 448, activation scale 0.03): weights, routing, align
+    and the quantised permuted hidden rows bit for bit; GEMM1's e4m3 activation codes
+    within one step of the oracle's and the layer output on a token sample that covers
+    every routed expert."""
+    cfg = CONFIGS["fp8pt_shared"]
+    inp = make_inputs(cfg, 0)
+    dev = torch.device("cuda:0")
+    s_in = float(inp["hidden"].float().abs().max() / 448)
+    s_act = cfg.activation_scale
+    q13, s13 = moe.quantize_weights_fp8_per_tensor(inp["w13"].to(dev))
+    q2, s2 = moe.quantize_weights_fp8_per_tensor(inp["w2"].to(dev))
+    o13, os13, o2, os2 = O.quantize_weights_fp8_per_tensor(bits(inp["w13"]), bits(inp["w2"]))
+    np.testing.assert_array_equal(s13.cpu().numpy(), os13)
+    np.testing.assert_array_equal(s2.cpu().numpy(), os2)
+    np.testing.assert_array_equal(q13.cpu().numpy(), o13)
+    np.testing.assert_array_equal(q2.cpu().numpy(), o2)
+    prob = moe.make_problem(cfg.T, cfg.H, cfg.E, cfg.topk, cfg.I, renormalize=cfg.renormalize,
+                            activation=cfg.activation, num_shared=cfg.num_shared, fp8="per_tensor",
+                            input_scale=s_in, activation_scale=s_act)
+    w13p, w2p = moe.prepare_weights(prob, q13, q2, cfg.I)
+    del q13, q2
+    ws = moe.new_workspace(prob)
+    out = moe.moe_forward(inp["hidden"].to(dev), inp["logits"].to(dev), w13p, w2p, cfg.topk, cfg.renormalize,
+                          cfg.activation, s13, s2, num_shared=cfg.num_shared, workspace=ws, input_scale=s_in,
+                          activation_scale=s_act)
+    torch.cuda.synchronize()
+    assert moe.device_status(ws)[0] == 0
+    parts = {k: v.cpu().numpy() for k, v in moe.read_workspace(prob, ws).items()}
+    ids, w = O.route(inp["logits"].numpy(), cfg.topk, cfg.renormalize, cfg.num_shared)
+    np.testing.assert_array_equal(parts["topk_ids"], ids)
+    np.testing.assert_allclose(parts["topk_w"], w, rtol=1e-5, atol=1e-7)
+    al = O.align(ids, cfg.E_total, 16)
+    P_pad = int(al["P_pad"])
+    np.testing.assert_array_equal(parts["sorted_pair_ids"][:P_pad], al["sorted_pair_ids"])
+    np.testing.assert_array_equal(parts["pair_to_row"], al["pair_to_row"])
+    gi, ng = parts["group_info"], int(parts["num_blocks"][1])
+    pids = al["sorted_pair_ids"][:P_pad]
+    real = pids < cfg.T * cfg.k_total
+    xq = O.quant_per_tensor_inv(O.bf16_bits_to_f32(bits(inp["hidden"])), s_in)
+    xs = untile_u8(parts["xs"], gi, ng, P_pad, cfg.H // 128)
+    np.testing.assert_array_equal(xs[real], xq[pids[real] // cfg.k_total])
+    assert np.all(xs[~real] == 0)
+    tokens = cover_tokens(ids, cfg.E, extra=16)
+    assert len(np.unique(ids[tokens])) == cfg.E_total
+    # GEMM1's e4m3 activation codes: the oracle's activation / activation_scale, one step
+    x = O.e4m3_decode(xq) * np.float64(np.float32(s_in))
+    codes = untile_u8(parts["act"], gi, ng, P_pad, cfg.I // 128)
+    inv = np.float64(np.float32(1.0) / np.float32(s_act))
+    n = check_act_pairs(
+        lambda e, t: O.activation_fn(x[t] @ (O.e4m3_decode(o13[e]) * np.float64(os13[e])).T, cfg.activation,
+                                     cfg.I) * inv,
+        codes, ids, tokens, al["pair_to_row"], lambda ref, got: _e4m3_within_one_step(ref, got.astype(np.uint8)))
+    ref = O.moe_forward_fp8_per_tensor(bits(inp["hidden"]), inp["logits"].numpy(), o13, os13, o2, os2, s_in, s_act,
+                                       topk=cfg.topk, renormalize=cfg.renormalize, activation=cfg.activation,
+                                       num_shared=cfg.num_shared, tokens=tokens)
+    got = bf16_to_f64(out.cpu()[torch.from_numpy(tokens)])
+    e = err_beyond_rounding(got, ref)
+    print(f"fp8pt_shared: {len(tokens)} tokens, {n} activation codes; beyond-rounding {e:.4f}, "
+          f"raw {max_err_over_rms(got, ref):.4f}")
     assert e <= FP8_TOL, e

@@ -183,6 +183,40 @@ def test_gelu_tanh_against_torch_and_limits():
     assert O.is_gated("gelu_tanh") and O.is_gated("swiglu") and not O.is_gated("relu2")
 
 
+def _swigluoai_decimal(g: float, u: float) -> float:
+    """The gpt-oss SwiGLU at one point in 40-digit decimal arithmetic (independent of
+    NumPy): g clamped to <= 7, u to [-7, 7], g / (1 + e^(-1.702 g)) * (u + 1)."""
+    from decimal import Decimal, getcontext
+    getcontext().prec = 40
+    gd = min(Decimal(repr(g)), Decimal(7))
+    ud = max(min(Decimal(repr(u)), Decimal(7)), Decimal(-7))
+    return float(gd / (1 + (-Decimal("1.702") * gd).exp()) * (ud + 1))
+
+
+def test_swigluoai_closed_forms():
+    pts = [(0.0, 5.0), (1.0, 0.0), (2.0, -1.0), (10.0, 10.0), (-3.0, 2.0), (7.0, -9.0), (-20.0, 0.5),
+           (6.5, -6.5), (7.5, 3.0), (-0.25, 100.0)]
+    for g, u in pts:
+        got = float(O.swigluoai(np.array([g]), np.array([u]))[0])
+        assert got == pytest.approx(_swigluoai_decimal(g, u), rel=1e-14, abs=1e-300), (g, u)
+    # special cases: a zero gate or an up value of -1 gives exactly 0; beyond the limits the
+    # value no longer depends on the input (the clamps)
+    assert float(O.swigluoai(np.array([0.0]), np.array([3.0]))[0]) == 0.0
+    assert float(O.swigluoai(np.array([4.0]), np.array([-1.0]))[0]) == 0.0
+    a = O.swigluoai(np.array([7.0, 9.0, 100.0]), np.array([7.0, 8.0, 1e6]))
+    assert a[0] == a[1] == a[2]
+    assert float(O.swigluoai(np.array([-1000.0]), np.array([1.0]))[0]) == 0.0   # no NaN at overflow
+    # inside the limits it is silu(1.702 g) / 1.702 * (u + 1), through the separately pinned silu
+    rng = np.random.default_rng(8)
+    g = rng.uniform(-7, 7, 500)
+    u = rng.uniform(-7, 7, 500)
+    np.testing.assert_allclose(O.swigluoai(g, u), O.silu(1.702 * g) / 1.702 * (u + 1.0), rtol=1e-12, atol=1e-15)
+    # the gated form takes the gate-first (un-interleaved) halves
+    z = rng.standard_normal((5, 8)) * 4
+    np.testing.assert_array_equal(O.activation_fn(z, "swigluoai", 4), O.swigluoai(z[:, :4], z[:, 4:8]))
+    assert O.is_gated("swigluoai")
+
+
 def test_routed_variant_equals_logit_routing():
     # the forward with caller-supplied routing, given route()'s routed choice, is the
     # logit-routed forward; append_shared_slot adds the shared slot exactly as route()
@@ -234,10 +268,11 @@ def test_interleave_order_from_page():
 
 
 def test_padding_leaves_layer_unchanged():
-    # zero-padding the intermediate size adds exact zeros: silu(0)*0 = relu2(0) = 0
+    # zero-padding the intermediate size adds exact zeros: silu(0)*0 = relu2(0) =
+    # swigluoai(0, 0) = 0
     rng = np.random.default_rng(5)
-    for act, I in (("swiglu", 40), ("relu2", 100)):
-        gated = act == "swiglu"
+    for act, I in (("swiglu", 40), ("relu2", 100), ("swigluoai", 40)):
+        gated = act != "relu2"
         T, H, E, k = 6, 128, 3, 2
         x = _bf16_bits(torch.from_numpy(rng.standard_normal((T, H)).astype(np.float32)))
         l = rng.standard_normal((T, E)).astype(np.float32)
@@ -277,6 +312,9 @@ def _dense_layer(x, logits, w13, w2, topk, renorm, act, num_shared=0):
     elif act == "gelu_tanh":
         g0 = z[:, :, :I]
         a = 0.5 * g0 * (1.0 + np.tanh(np.sqrt(2.0 / np.pi) * (g0 + 0.044715 * g0 ** 3))) * z[:, :, I:]
+    elif act == "swigluoai":
+        g0 = np.minimum(z[:, :, :I], 7.0)
+        a = g0 * (1.0 / (1.0 + np.exp(-1.702 * g0))) * (np.clip(z[:, :, I:], -7.0, 7.0) + 1.0)
     else:
         a = np.maximum(z, 0.0) ** 2
     ffn = np.einsum("tei,ehi->teh", a, w2)
@@ -284,7 +322,7 @@ def _dense_layer(x, logits, w13, w2, topk, renorm, act, num_shared=0):
 
 
 @pytest.mark.parametrize("act,renorm,shared", [("swiglu", True, 0), ("relu2", False, 0), ("swiglu", True, 1),
-                                                ("gelu_tanh", True, 0)])
+                                                ("gelu_tanh", True, 0), ("swigluoai", True, 0)])
 def test_layer_dense_ffn_invariant(act, renorm, shared):
     rng = np.random.default_rng(11)
     T, H, E, k, I = 9, 64, 6, 3, 24
