@@ -250,7 +250,7 @@ def run_ours(cfg: MoeConfig, steps: int, warmup: int, world: int, rank: int, loc
 
     # per-kernel breakdown: the same kernels through the per-step entry points, events
     # between the steps on the launching stream
-    names = ["route", "align"] + (["quant_act"] if cfg.block128 else ["permute"]) + ["gemm1", "gemm2", "combine"]
+    names = ["route", "align", "permute", "gemm1", "gemm2", "combine"]
     per = {n: [] for n in names}
     for _ in range(steps):
         flush.zero_()
@@ -259,10 +259,7 @@ def run_ours(cfg: MoeConfig, steps: int, warmup: int, world: int, rank: int, loc
         k = 0
         moe.stage_route(prob, logits, ws); k += 1; evs[k].record(stream)
         moe.stage_align(prob, ws); k += 1; evs[k].record(stream)
-        if cfg.block128:
-            moe.stage_quant_act(prob, hidden, ws); k += 1; evs[k].record(stream)
-        else:
-            moe.stage_permute(prob, hidden, ws); k += 1; evs[k].record(stream)
+        moe.stage_permute(prob, hidden, ws); k += 1; evs[k].record(stream)
         moe.stage_gemm1(prob, hidden, w13p, ws, s13); k += 1; evs[k].record(stream)
         moe.stage_gemm2(prob, w2p, ws, s2); k += 1; evs[k].record(stream)
         moe.stage_combine(prob, out, ws); k += 1; evs[k].record(stream)
@@ -298,7 +295,8 @@ def run_ours(cfg: MoeConfig, steps: int, warmup: int, world: int, rank: int, loc
         "e2e_total_ms": e2e_total, "ids": ids, "inp": inp,
         "h2d": h_hidden.numel() * 2 + h_logits.numel() * 4, "d2h": h_out.numel() * 2,
         # one kernel per stage, except align (three kernels above one 2048-pair chunk) and
-        # block-128 FP8 and MXFP8 GEMM1 (the GEMM, then the activation quantisation)
+        # the 8-bit formats' GEMM1 with a separate activation quantisation (block-128 FP8 and
+        # MXFP8: the GEMM, then the quantisation)
         "launches_per_step": len(names) + (2 if cfg.T * cfg.k_total > 2048 else 0) +
                              (1 if cfg.block128 or cfg.mx else 0),
     }

@@ -118,10 +118,9 @@ typedef struct {
   int32_t renormalize;  /* 0/1: divide the selected softmax weights by their sum */
   int32_t activation;   /* moe_activation_t */
   int32_t wdtype;       /* moe_wdtype_t */
-  int32_t block_m;      /* row alignment of each expert's segment: 0 = default (128 for
-                           FP8 block-128, 16 otherwise), 16 (all but FP8 block-128: the
+  int32_t block_m;      /* row alignment of each expert's segment: 0 = default (16), 16 (the
                            expert's weight rows are the MMA's M operand and its token rows
-                           N) or 128 (BF16 and FP8 block-128: 128-row token tiles) */
+                           N) or 128 (BF16 and FP8 block-128 only: 128-row token tiles) */
   uint32_t flags;       /* MOE_FLAG_* */
   float input_scale;      /* MOE_DTYPE_FP8_PER_TENSOR: static scale of the hidden rows,
                              x_q = e4m3(x / input_scale); finite, > 0 (ignored otherwise) */
@@ -144,14 +143,20 @@ typedef struct {
   size_t block_expert;    /* int32 [max_rows/block_m]: expert of each row tile */
   size_t pair_to_row;     /* int32 [T*k']: sorted row of each pair */
   size_t chunk_hist;      /* int32 [num_chunks, E]: align scratch */
-  size_t xq;              /* FP8: e4m3 [T, H] quantised hidden */
-  size_t xq_scale;        /* FP8: fp32 [T, H/128] */
-  size_t act;             /* GEMM1 output: bf16 [max_rows, I] */
-  size_t actq;            /* FP8: the activation quantised per 1x128 group, e4m3 [max_rows, I] */
-  size_t act_scale;       /* FP8: fp32 [max_rows, I/128] */
+  size_t xq;              /* FP8 block-128, block_m 128: e4m3 [T, H] quantised hidden */
+  size_t xq_scale;        /* FP8 block-128, block_m 128: fp32 [T, H/128] */
+  size_t act;             /* GEMM1 output: bf16 [max_rows, I] (block_m 128) or bf16 in
+                             row-group order (block_m 16; per-tensor FP8: e4m3 codes) */
+  size_t actq;            /* FP8 block-128: the activation quantised per 1x128 group, e4m3
+                             [max_rows, I] (block_m 128) or codes and fp32 scales in the
+                             layout of xs (block_m 16); MXFP8: e4m3 codes in row-group order */
+  size_t act_scale;       /* FP8 block-128, block_m 128: fp32 [max_rows, I/128]; MXFP8: E8M0
+                             scale blocks */
   size_t y;               /* fp32 [max_rows, H]: weighted GEMM2 rows in sorted order */
-  size_t xs;              /* bf16 [max_rows, H]: hidden rows in sorted order (block_m 16,
-                             more than 1024 pairs; size 0 otherwise) */
+  size_t xs;              /* block_m 16: the hidden rows of every row group in row-group order
+                             (bf16; e4m3 codes for the 8-bit formats; FP8 block-128: each K
+                             step's e4m3 codes followed by its rows' fp32 1x128 scales, 132
+                             bytes per row per 128 columns); size 0 otherwise */
   size_t xs_scale;        /* MXFP8: E8M0 scale bytes of xs: per row group, 1024 bytes per
                              128 columns at ((first row / 16) * H/128 + chunk) * 1024 */
   size_t group_info;      /* int32 pairs [max_rows/16 + 1]: row groups {first row, expert |
@@ -190,12 +195,13 @@ size_t moe_workspace_size(const moe_problem_t* problem);
  * problem->intermediate = moe_padded_intermediate(intermediate_in, ...), SWIGLU rows
  * interleaved [gate0, up0, gate1, up1, ...] and rows of padded indices zero; and w2
  * [E, H, I] with columns >= intermediate_in zero. They are stored
- *   - block_m 128 (FP8, or BF16 with block_m = 128): row-major as above;
- *   - block_m 16 (the BF16 default): tiled for the GEMMs that take the weights as the
- *     MMA's M operand: tile (e, m, c) of rows [128m, 128m+128) and columns [64c, 64c+64)
- *     at byte ((e*MT + m)*KC + c) * 16384, MT = ceil(rows/128), KC = ceil(cols/64); each
- *     tile row is 128 contiguous bytes whose 16-byte piece q sits at position q ^ (r % 8);
- *     rows and columns past the matrix are zero.
+ *   - block_m 128 (FP8 block-128 or BF16 with block_m = 128): row-major as above;
+ *   - block_m 16 (the default): tiled for the GEMMs that take the weights as the MMA's M
+ *     operand: tile (e, m, c) of rows [128m, 128m+128) and the 128 bytes of columns of
+ *     chunk c (64 bf16 or 128 e4m3 columns) at byte ((e*MT + m)*KC + c) * 16384, MT =
+ *     ceil(rows/128), KC = the number of such chunks; each tile row is 128 contiguous
+ *     bytes whose 16-byte piece q sits at position q ^ (r % 8); rows and columns past the
+ *     matrix are zero.
  *   w13_out, w2_out  device, moe_prepared_weights_bytes(problem, 0 / 1) bytes each,
  *                    16-byte aligned, not overlapping the inputs.
  * Elements are bf16 (2 bytes) or e4m3 codes (1 byte) per problem->wdtype. For FP8 the
@@ -299,20 +305,22 @@ moe_status_t moe_forward_host(const moe_problem_t* problem, const void* h_hidden
                               const float* w13_scale, const float* w2_scale, void* h_out,
                               void* workspace, size_t workspace_bytes, moe_stream_t stream);
 
-/* The steps as separate calls on the same workspace: route, align, quant_act (FP8),
- * permute (block_m 16), gemm1, gemm2, combine; moe_forward runs exactly these, in this
- * order. They exist so tests can check each intermediate and tools can time each kernel;
+/* The steps as separate calls on the same workspace: route, align, quant_act (FP8
+ * block-128 with block_m 128), permute (block_m 16), gemm1, gemm2, combine; moe_forward
+ * runs exactly these, in this order. They exist so tests can check each intermediate and tools can time each kernel;
  * each requires the previous steps to have been enqueued. */
 moe_status_t moe_stage_route(const moe_problem_t* problem, const float* router_logits,
                              void* workspace, size_t workspace_bytes, moe_stream_t stream);
 moe_status_t moe_stage_align(const moe_problem_t* problem, void* workspace,
                              size_t workspace_bytes, moe_stream_t stream);
-/* FP8 only: quantise hidden per token per 128 columns into the workspace (xq, xq_scale). */
+/* FP8 block-128 only (else MOE_ERR_INVALID_ARG): with block_m 128, quantise hidden per
+ * token per 128 columns into the workspace (xq, xq_scale); with block_m 16 the permute
+ * step quantises the rows instead and this call does nothing (MOE_OK). */
 moe_status_t moe_stage_quant_act(const moe_problem_t* problem, const void* hidden,
                                  void* workspace, size_t workspace_bytes, moe_stream_t stream);
-/* block_m 16 (the BF16 default): copy the token rows of every row group into the
- * workspace in the order GEMM1 reads them (xs); hidden device bf16 [T, H]. Other
- * problems: nothing to do, MOE_OK. */
+/* block_m 16 (the default): copy the token rows of every row group into the workspace in
+ * the order GEMM1 reads them (xs), quantised on the way for the 8-bit formats; hidden
+ * device bf16 [T, H]. block_m 128: nothing to do, MOE_OK. */
 moe_status_t moe_stage_permute(const moe_problem_t* problem, const void* hidden, void* workspace,
                                size_t workspace_bytes, moe_stream_t stream);
 moe_status_t moe_stage_gemm1(const moe_problem_t* problem, const void* hidden, const void* w13,

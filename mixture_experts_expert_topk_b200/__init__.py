@@ -405,6 +405,15 @@ def read_workspace(prob: Problem, workspace: torch.Tensor) -> Dict[str, torch.Te
         out["actq"] = view(L["actq"], rows * I, torch.uint8)
         out["act_scale"] = view(L["act_scale"], rows // 16 * (I // 128) * 1024, torch.uint8)
         out["group_info"] = view(L["group_info"], (rows // 16 + 1) * 2, torch.int32).view(-1, 2)
+    elif fp8 and L["block_m"] == 16:
+        # FP8 block-128 on the swapped-operand GEMMs: the bf16 activation (64-column
+        # chunks), and the quantised hidden rows and activation with each K step's fp32 row
+        # scales behind its codes (132 bytes per row per 128 columns); flat views
+        act_cols = -(-I // 64) * 64
+        out["act"] = view(L["act"], rows * act_cols, torch.bfloat16)
+        out["xs"] = view(L["xs"], rows * (H // 128) * 132, torch.uint8)
+        out["actq"] = view(L["actq"], rows * (I // 128) * 132, torch.uint8)
+        out["group_info"] = view(L["group_info"], (rows // 16 + 1) * 2, torch.int32).view(-1, 2)
     elif prob.wdtype == MOE_DTYPE_FP8_PER_TENSOR:
         # e4m3 codes in row-group order (128-column chunks per group, swizzled); flat views
         out["act"] = view(L["act"], rows * I, torch.uint8)
@@ -419,7 +428,7 @@ def read_workspace(prob: Problem, workspace: torch.Tensor) -> Dict[str, torch.Te
         out["group_info"] = view(L["group_info"], (rows // 16 + 1) * 2, torch.int32).view(-1, 2)
     else:
         out["act"] = view(L["act"], rows * I, torch.bfloat16).view(rows, I)
-    if fp8:
+    if fp8 and L["block_m"] == 128:
         out["xq"] = view(L["xq"], T * H, torch.uint8).view(T, H)
         out["xq_scale"] = view(L["xq_scale"], T * (H // 128), torch.float32).view(T, H // 128)
         out["actq"] = view(L["actq"], rows * I, torch.uint8).view(rows, I)

@@ -105,13 +105,12 @@ moe_status_t make_plan(const moe_problem_t* p, Plan* pl) {
   q.topk = p->topk;
   q.kk = q.topk + q.Es;
   q.N1 = q.gated ? 2 * q.I : q.I;
-  // Row alignment. bf16 (default): 16-row blocks, the expert's weights as the MMA's M
-  // operand and row groups of up to 256 token rows as N. FP8, or block_m = 128: 128-row
-  // token tiles.
-  if (p->block_m == 16 && q.fp8) return MOE_ERR_UNSUPPORTED;
+  // Row alignment. Default: 16-row blocks, the expert's weights as the MMA's M operand and
+  // row groups of token rows as N (up to 256 rows; 192 for MXFP8, 128 for FP8 block-128).
+  // block_m = 128 (BF16 and FP8 block-128 only): 128-row token tiles.
   if (p->block_m == 128 && (q.pt || q.mx)) return MOE_ERR_UNSUPPORTED;
-  q.bm = p->block_m != 0 ? p->block_m : (q.fp8 ? 128 : 16);
-  q.grp = q.bm == 16 ? (q.mx ? moe::kMxGroupRows : kGroupRows) : 0;
+  q.bm = p->block_m != 0 ? p->block_m : 16;
+  q.grp = q.bm == 16 ? (q.mx ? moe::kMxGroupRows : (q.fp8 ? moe::kB128GroupRows : kGroupRows)) : 0;
   q.renorm = p->renormalize;
   q.act = p->activation;
   q.P = static_cast<long long>(q.T) * q.kk;
@@ -143,18 +142,23 @@ moe_status_t make_plan(const moe_problem_t* p, Plan* pl) {
   L.block_expert = take(rows / q.bm * 4 + 4);
   L.pair_to_row = take(P * 4);
   L.chunk_hist = take(static_cast<size_t>(L.num_chunks) * q.E * 4);
-  L.xq = take(q.fp8 ? T * H : 0);
-  L.xq_scale = take(q.fp8 ? T * (H / 128) * 4 : 0);
+  const bool fp8_tiles = q.fp8 && q.bm == 128;  // FP8 block-128 with 128-row token tiles
+  const bool b128 = q.fp8 && q.bm == 16;        // FP8 block-128 on the swapped-operand GEMMs
+  L.xq = take(fp8_tiles ? T * H : 0);
+  L.xq_scale = take(fp8_tiles ? T * (H / 128) * 4 : 0);
   // the swapped-operand GEMMs keep the activation in row-group order, 128-byte chunks (64
   // bf16 or 128 e4m3 columns)
   const size_t act_bytes = q.pt ? rows * I : rows * (q.bm == 16 ? align_up(I, 64) : I) * 2;
   L.act = take(act_bytes);
-  // MXFP8: the activation's codes (128-column chunks) and scales: 1024 bytes per 16 rows per
-  // 128 columns (a group's scale blocks sit at its first row / 16)
-  L.actq = take(q.fp8 || q.mx ? rows * I : 0);
-  L.act_scale = take(q.fp8 ? rows * (I / 128) * 4 : (q.mx ? rows / 16 * (I / 128) * 1024 : 0));
+  // the activation quantised for GEMM2: FP8 block-128 with token tiles: e4m3 [rows, I] and
+  // fp32 [rows, I/128]; on the swapped-operand GEMMs: codes and scales together (132 bytes
+  // per row per 128 columns); MXFP8: codes (128-column chunks) and scales, 1024 bytes per 16
+  // rows per 128 columns (a group's scale blocks sit at its first row / 16)
+  L.actq = take(fp8_tiles || q.mx ? rows * I : (b128 ? rows * (I / 128) * moe::kB128RowBytesPerChunk : 0));
+  L.act_scale = take(fp8_tiles ? rows * (I / 128) * 4 : (q.mx ? rows / 16 * (I / 128) * 1024 : 0));
   L.y = take(rows * H * 4);
-  L.xs = take(q.bm == 16 ? rows * H * (q.pt || q.mx ? 1 : 2) : 0);
+  L.xs = take(q.bm == 16 ? (b128 ? rows * (H / 128) * moe::kB128RowBytesPerChunk : rows * H * (q.pt || q.mx ? 1 : 2))
+                         : 0);
   L.xs_scale = take(q.mx ? rows / 16 * (H / 128) * 1024 : 0);
   L.group_info = take(q.bm == 16 ? (rows / 16 + 1) * 8 : 0);
   L.io_hidden = take(T * H * 2);
@@ -246,7 +250,8 @@ moe_status_t run_route(const Plan& pl, const float* logits, void* ws, const Laun
   // the route kernel also resets the device status word: it starts every forward
   return cuda_status(moe::launch_route(l, logits, pl.T, pl.Er, pl.topk, pl.Es, pl.renorm,
                                        ws_ptr<int>(ws, L.topk_ids), ws_ptr<float>(ws, L.topk_w),
-                                       ws_ptr<int>(ws, L.status), pl.fp8 ? nullptr : hidden, pl.H * 2));
+                                       ws_ptr<int>(ws, L.status), (pl.fp8 && pl.bm == 128) ? nullptr : hidden,
+                                       pl.H * 2));
 }
 
 moe_status_t run_align(const Plan& pl, void* ws, const Launch& l) {
@@ -318,6 +323,15 @@ moe_status_t run_gemm1(const Plan& pl_in, const void* hidden, const void* w13, c
     o.w_scale = w13_scale;
     o.in_scale = pl.in_scale;
     o.act_scale = pl.act_scale;
+    if (pl.fp8) {
+      // FP8 block-128: GEMM1 writes the bf16 activation, then quantised per 1x128 for GEMM2
+      o.b128 = 1;
+      o.up_block = pl.gated ? pl.I / 128 : 0;
+      moe_status_t st = cuda_status(moe::launch_gemm_swap(l, 0, o, s, b));
+      if (st != MOE_OK) return st;
+      return cuda_status(moe::launch_act_quant_b128(l, ws_ptr<void>(ws, L.act), pl.I, ws_ptr<int>(ws, L.num_blocks) + 1,
+                                                    ws_ptr<int2>(ws, L.group_info), ws_ptr<void>(ws, L.actq), num_sms));
+    }
     if (pl.mx) {
       // the weight scales follow the tiled codes; GEMM1 writes the bf16 activation, which is
       // then quantised for GEMM2
@@ -370,6 +384,10 @@ moe_status_t run_gemm1(const Plan& pl_in, const void* hidden, const void* w13, c
 moe_status_t run_permute(const Plan& pl, const void* hidden, void* ws, const Launch& l, int num_sms) {
   if (pl.bm != 16) return MOE_OK;
   const auto& L = pl.lay;
+  if (pl.fp8)
+    return cuda_status(moe::launch_permute_b128_rows(l, hidden, pl.H, ws_ptr<int>(ws, L.sorted_pair_ids),
+                                                     ws_ptr<int>(ws, L.num_blocks) + 1, ws_ptr<int2>(ws, L.group_info),
+                                                     static_cast<int>(pl.P), pl.kk, ws_ptr<void>(ws, L.xs), num_sms));
   if (pl.mx)
     return cuda_status(moe::launch_permute_mx_rows(
         l, hidden, pl.H, ws_ptr<int>(ws, L.sorted_pair_ids), ws_ptr<int>(ws, L.num_blocks) + 1,
@@ -412,6 +430,10 @@ moe_status_t run_gemm2(const Plan& pl_in, const void* w2, const float* w2_scale,
     o.fp8 = pl.pt;
     o.w_scale = w2_scale;
     o.in_scale = pl.act_scale;
+    if (pl.fp8) {
+      o.b128 = 1;
+      o.x = ws_ptr<void>(ws, L.actq);
+    }
     if (pl.mx) {
       o.mx = 1;
       o.x = ws_ptr<void>(ws, L.actq);
@@ -469,7 +491,7 @@ Launch launch_of(const moe_problem_t* p, moe_stream_t stream) {
 moe_status_t forward_after_route(const Plan& pl, const Launch& l, const void* hidden, const void* w13, const void* w2,
                                  const float* s13, const float* s2, void* out, void* ws, int num_sms) {
   moe_status_t st = run_align(pl, ws, l);
-  if (st == MOE_OK && pl.fp8) st = run_quant_act(pl, hidden, ws, l);
+  if (st == MOE_OK && pl.fp8 && pl.bm == 128) st = run_quant_act(pl, hidden, ws, l);
   if (st == MOE_OK) st = run_permute(pl, hidden, ws, l, num_sms);
   if (st == MOE_OK) st = run_gemm1(pl, hidden, w13, s13, ws, l, num_sms);
   if (st == MOE_OK) st = run_gemm2(pl, w2, s2, ws, l, num_sms);
@@ -562,7 +584,7 @@ MOE_API moe_status_t moe_prepare_weights(const moe_problem_t* problem, int32_t i
   if (st != MOE_OK) return st;
   const Launch l = launch_of(problem, stream);
   cudaError_t e;
-  if (pl.pt) {
+  if (pl.pt || (pl.fp8 && pl.bm == 16)) {
     // e4m3 codes, tiled for the swapped-operand GEMMs
     e = moe::launch_tile_weights_u8(l, 0, w13_in, w13_out, pl.E, pl.H, pl.I, pl.gated);
     if (e == cudaSuccess) e = moe::launch_tile_weights_u8(l, 1, w2_in, w2_out, pl.E, pl.H, pl.I, pl.gated);
@@ -585,7 +607,7 @@ MOE_API size_t moe_prepared_weights_bytes(const moe_problem_t* problem, int32_t 
   if (pl.mx)
     return which == 0 ? moe::tiled_weight_bytes_u8(pl.E, pl.N1, pl.H) + moe::tiled_scale_bytes_mx(pl.E, pl.N1, pl.H)
                       : moe::tiled_weight_bytes_u8(pl.E, pl.H, pl.I) + moe::tiled_scale_bytes_mx(pl.E, pl.H, pl.I);
-  if (pl.pt)
+  if (pl.pt || (pl.fp8 && pl.bm == 16))
     return which == 0 ? moe::tiled_weight_bytes_u8(pl.E, pl.N1, pl.H) : moe::tiled_weight_bytes_u8(pl.E, pl.H, pl.I);
   if (pl.bm == 16)
     return which == 0 ? moe::tiled_weight_bytes(pl.E, pl.N1, pl.H) : moe::tiled_weight_bytes(pl.E, pl.H, pl.I);
@@ -766,7 +788,7 @@ MOE_API moe_status_t moe_stage_quant_act(const moe_problem_t* problem, const voi
   if (st != MOE_OK || pl.T == 0) return st;  // T == 0: nothing to do, pointers unused
   if (!pl.fp8 || !aligned16(hidden)) return MOE_ERR_INVALID_ARG;
   st = prologue(problem, workspace, workspace_bytes, &pl, &sms);
-  if (st != MOE_OK || pl.T == 0) return st;
+  if (st != MOE_OK || pl.T == 0 || pl.bm != 128) return st;  // block_m 16: quantised by the permute step
   return run_quant_act(pl, hidden, workspace, launch_of(problem, stream));
 }
 

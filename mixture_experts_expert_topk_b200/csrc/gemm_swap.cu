@@ -50,6 +50,21 @@
 // the two accumulators leave 128 TMEM columns for four scale buffers. GEMM1's epilogue
 // writes the bf16 activation, which a separate pass quantises for GEMM2.
 //
+// FP8 E4M3 W8A8 with 128x128 weight blocks and 1x128 activation groups ("Qwen3-Next FP8
+// MoE optimisation: shared-expert fusion for H200", sglang PR 26204, section 1): the same
+// tiles with kind::f8f6f4, but the scales are arbitrary fp32 (amax / 448), which the tensor
+// core's power-of-two block scaling cannot carry. Every 128-element K chunk is therefore
+// its own partial product in TMEM (four 128-column buffers, so the MMAs run up to four
+// chunks ahead), and the epilogue warps promote it in registers:
+// acc[j] += partial[j] * s_w(row block, chunk) * s_x(token j, chunk). A 128-row weight tile
+// is exactly one scale block row (gated: its even lanes are gate rows, its odd lanes up
+// rows, two block rows of the checkpoint layout), so s_w is one value per lane per chunk;
+// s_x varies along N, so each K step of X carries, right behind its codes, the fp32 scales
+// of its rows (chunk-major), which the epilogue reads from shared memory as broadcasts.
+// The epilogue, not the MMA, then releases the step's ring space. Row groups have at most
+// 128 rows (kB128GroupRows) so the accumulator fits the epilogue threads' registers.
+// GEMM1 writes the bf16 activation, which a separate pass quantises per 1x128 for GEMM2.
+//
 // One persistent CTA per SM, 7 warps:
 //   warp 0      scheduler (tiles from a global atomic counter, published to the other
 //               roles through a shared-memory ring) and W copies;
@@ -83,6 +98,10 @@ constexpr int kSfBufs = 4;
 constexpr int kSfBufCols = 32;
 constexpr int kSfCol0 = 2 * kMxAccCols;
 static_assert(kSfCol0 + kSfBufs * kSfBufCols <= static_cast<int>(kTmemCols), "TMEM columns");
+// FP8 block-128: partial-product buffers in TMEM (one per K chunk in flight)
+constexpr int kPartBufs = 4;
+constexpr int kPartCols = kB128GroupRows;
+static_assert(kPartBufs * kPartCols <= static_cast<int>(kTmemCols), "TMEM columns");
 
 // Operand ring: a K step takes kc * (16 KB + n * 128) contiguous bytes (W chunks, then X
 // chunks); a step that would cross the end of the ring starts again at its beginning.
@@ -91,12 +110,14 @@ constexpr int kRingBytes = 225 * 1024;
 constexpr int kSlots = 16;  // barrier pairs: at most this many K steps in flight
 constexpr int kBarOff = kRingBytes;
 constexpr int kBarBytes = 1024;  // barriers, step ends, tile ring, TMEM address, abort flag
+static_assert((3 * kSlots + 4 + 2 * kTileRing + 1 + 2 * 4) * 8 + 2 * kSlots * 8 + 16 * kTileRing + 8 <= kBarBytes,
+              "barrier region");
 constexpr int kSmemBytes = kBarOff + kBarBytes + 1024;
 static_assert(kSmemBytes <= kSmemCap, "shared memory");
 
 enum : int {
   kSiteEmpty = 1, kSiteFull = 2, kSiteTmemEmpty = 3, kSiteTmemFull = 4, kSiteTileFull = 5, kSiteTileEmpty = 6,
-  kSiteEmptyX = 7, kSiteSfFree = 8, kSiteFullX = 9
+  kSiteEmptyX = 7, kSiteSfFree = 8, kSiteFullX = 9, kSitePartEmpty = 10, kSitePartFull = 11
 };
 
 struct Args {
@@ -120,18 +141,21 @@ struct Args {
   float act_inv;           // FP8 GEMM1: 1 / activation scale (requantisation of the output)
   const uint8_t* w_sf;     // MXFP8: tiled weight scales, 512 bytes per (expert, 128-row block, K chunk)
   const uint8_t* x_sf;     // MXFP8: X scales, 1024 bytes per (16 rows of the group's first row, K chunk)
+  // FP8 block-128: w_scale is fp32 [E, ws_rows, k_chunks] (checkpoint block layout); gated
+  // GEMM1 tiles take the gate block row mt / 2 and the up block row up_block + mt / 2
+  int ws_rows;             // 128-row scale blocks per expert
+  int up_block;            // gated GEMM1: I / 128; 0 otherwise
 };
 
-// K chunks per step for a group of n rows: steps of 48 to 72 KB.
-__host__ __device__ constexpr int chunks_per_step(int n) {
-  return n <= 32 ? 4 : (n <= 64 ? 3 : (n <= 128 ? 2 : 1));
-}
 // Ring bytes of one K step of kcs chunks for a group of n rows. MXFP8 steps add the scale
-// blocks of W and X and round up to the 1024-byte period of the swizzle.
-template <bool kMx>
+// blocks of W and X, FP8 block-128 steps the fp32 scales of the X rows (4 bytes per row
+// per chunk); both round up to the 1024-byte period of the swizzle.
+template <int kKind>
 __device__ __forceinline__ uint32_t step_bytes(int kcs, int n) {
   const uint32_t b = static_cast<uint32_t>(kcs) * (kTileW + n * kChunkBytes);
-  return kMx ? (b + static_cast<uint32_t>(kcs) * (kSfW + kSfX) + 1023u) & ~1023u : b;
+  if (kKind == 2) return (b + static_cast<uint32_t>(kcs) * (kSfW + kSfX) + 1023u) & ~1023u;
+  if (kKind == 3) return (b + static_cast<uint32_t>(kcs * n) * 4u + 1023u) & ~1023u;
+  return b;
 }
 static_assert(4 * (kTileW + 32 * kChunkBytes + kSfW + kSfX) <= kRingBytes / 2 &&
                   kTileW + kMxGroupRows * kChunkBytes + kSfW + kSfX <= kRingBytes / 2,
@@ -139,6 +163,9 @@ static_assert(4 * (kTileW + 32 * kChunkBytes + kSfW + kSfX) <= kRingBytes / 2 &&
 static_assert(4 * (kTileW + 32 * kChunkBytes) <= kRingBytes / 2 && 2 * (kTileW + 128 * kChunkBytes) <= kRingBytes / 2 &&
                   kTileW + kNMax * kChunkBytes <= kRingBytes / 2,
               "at least two steps fit the ring");
+static_assert(4 * (kTileW + 32 * (kChunkBytes + 4)) + 1024 <= kRingBytes / 2 &&
+                  2 * (kTileW + kB128GroupRows * (kChunkBytes + 4)) + 1024 <= kRingBytes / 2,
+              "at least two FP8 block-128 steps fit the ring");
 
 // Byte offset in the ring of the next step of `bytes`. pos: offset of the next free byte;
 // head: running count of the bytes used, skipped ring tails included.
@@ -192,11 +219,13 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
       : "memory");
 }
 
-// kKind: 0 bf16, 1 per-tensor e4m3, 2 MXFP8.
+// kKind: 0 bf16, 1 per-tensor e4m3, 2 MXFP8, 3 FP8 block-128.
 template <int kKind>
 __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
   constexpr bool kFp8 = kKind == 1;  // scales applied in the epilogue
   constexpr bool kMx = kKind == 2;   // scales applied by the MMA
+  constexpr bool kB128 = kKind == 3; // a partial per K chunk, promoted in the epilogue
+  constexpr bool kE4m3 = kFp8 || kB128;
   constexpr int kAccCols = kMx ? kMxAccCols : kNMax;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -211,7 +240,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
   const uint32_t rempty0 = rfull0 + 8 * kTileRing;
   const uint32_t drain_bar = rempty0 + 8 * kTileRing;
   const uint32_t fullx0 = drain_bar + 8;                                      // [kSlots]
-  uint64_t* step_end_w = bars + 3 * kSlots + 4 + 2 * kTileRing + 1;           // [kSlots]
+  const uint32_t pfull0 = fullx0 + 8 * kSlots;                                // [kPartBufs]
+  const uint32_t pempty0 = pfull0 + 8 * kPartBufs;                            // [kPartBufs]
+  uint64_t* step_end_w = bars + 3 * kSlots + 4 + 2 * kTileRing + 1 + 2 * kPartBufs;  // [kSlots]
   uint64_t* step_end_x = step_end_w + kSlots;                                 // [kSlots]
   volatile int* ring = reinterpret_cast<volatile int*>(step_end_x + kSlots);  // [kTileRing][4]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(const_cast<int*>(ring) + 4 * kTileRing);
@@ -224,7 +255,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
     for (int s = 0; s < kSlots; ++s) {
       mbar_init(full0 + 8 * s, 1);   // the W copies of a step
       mbar_init(fullx0 + 8 * s, 1);  // the X copies of a step
-      mbar_init(empty0 + 8 * s, 1);
+      // released by the MMAs' commit; FP8 block-128: by the four epilogue warps, which
+      // read the step's X scales after its MMAs
+      mbar_init(empty0 + 8 * s, kB128 ? 4 : 1);
+    }
+    for (int b = 0; b < kPartBufs; ++b) {
+      mbar_init(pfull0 + 8 * b, 1);
+      mbar_init(pempty0 + 8 * b, 128);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull0 + 8 * b, 1);
@@ -251,7 +288,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
   griddep_wait();
   griddep_launch_dependents();
 
-  const size_t x_row_bytes = static_cast<size_t>(a.k_chunks) * kChunkBytes;
+  // bytes of X per row: a 128-byte chunk row per K chunk (FP8 block-128: and its fp32 scale)
+  const size_t x_row_bytes = static_cast<size_t>(a.k_chunks) * (kB128 ? kB128RowBytesPerChunk : kChunkBytes);
 
   if (warp == 0) {
     // ---------------- scheduler + W producer ----------------
@@ -289,7 +327,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
         const uint8_t* wsrc = a.w + (static_cast<size_t>(e) * a.m_tiles + mt) * a.k_chunks * kTileW;
         for (int c0 = 0; c0 < a.k_chunks; c0 += kc, ++ks) {
           const int kcs = min(kc, a.k_chunks - c0);
-          const uint32_t off = ring_alloc(pos, head, step_bytes<kMx>(kcs, n));
+          const uint32_t off = ring_alloc(pos, head, step_bytes<kKind>(kcs, n));
           if (!ring_reserve(head, freed, ks, oldest, step_end_w, empty0, abort_flag, a.status, kSiteEmpty)) {
             ok = false;
             break;
@@ -324,16 +362,18 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
         const uint8_t* xsrc = a.x + static_cast<size_t>(x_row) * x_row_bytes;
         for (int c0 = 0; c0 < a.k_chunks; c0 += kc, ++ks) {
           const int kcs = min(kc, a.k_chunks - c0);
-          const uint32_t off = ring_alloc(pos, head, step_bytes<kMx>(kcs, n));
+          const uint32_t off = ring_alloc(pos, head, step_bytes<kKind>(kcs, n));
           if (!ring_reserve(head, freed, ks, oldest, step_end_x, empty0, abort_flag, a.status, kSiteEmptyX)) {
             ok = false;
             break;
           }
           const uint32_t full = fullx0 + 8 * (ks % kSlots);
-          const uint32_t bytes = static_cast<uint32_t>(kcs * n) * kChunkBytes;
+          // FP8 block-128: the step's codes and then its rows' scales, contiguous in X
+          const uint32_t bytes = static_cast<uint32_t>(kcs * n) * (kB128 ? kB128RowBytesPerChunk : kChunkBytes);
           const uint32_t sf_bytes = kMx ? static_cast<uint32_t>(kcs) * kSfX : 0u;
           mbar_arrive_expect_tx(full, bytes + sf_bytes);
-          bulk_load(s0 + off + kcs * kTileW, xsrc + static_cast<size_t>(c0) * n * kChunkBytes, bytes, full, pol);
+          bulk_load(s0 + off + kcs * kTileW, xsrc + static_cast<size_t>(c0) * n * (kB128 ? kB128RowBytesPerChunk : kChunkBytes),
+                    bytes, full, pol);
           if constexpr (kMx)
             bulk_load(s0 + off + static_cast<uint32_t>(kcs) * (kTileW + n * kChunkBytes + kSfW),
                       a.x_sf + (static_cast<size_t>(x_row >> 4) * a.k_chunks + c0) * kSfX, sf_bytes, full, pol);
@@ -345,7 +385,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       int rslot = 0, it = 0;
-      uint32_t rph = 0, ks = 0, pos = 0;
+      uint32_t rph = 0, ks = 0, pos = 0, pc = 0;  // pc: FP8 block-128 partials issued
       uint64_t head = 0;  // the producers' ring allocation, replayed
       while (true) {
         int4 t;
@@ -353,14 +393,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
         const int n = t.y;
         const int kc = chunks_per_step(n);
         const int acc = it & 1;
-        if (!mbar_wait(tempty0 + 8 * acc, ((it >> 1) & 1) ^ 1u, abort_flag, a.status, kSiteTmemEmpty)) break;
+        if (!kB128 && !mbar_wait(tempty0 + 8 * acc, ((it >> 1) & 1) ^ 1u, abort_flag, a.status, kSiteTmemEmpty)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * kAccCols;
-        const uint32_t idesc = kMx ? idesc_mx(kMW, n) : (kFp8 ? idesc_e4m3(kMW, n) : idesc_bf16(kMW, n));
+        const uint32_t idesc = kMx ? idesc_mx(kMW, n) : (kE4m3 ? idesc_e4m3(kMW, n) : idesc_bf16(kMW, n));
         bool ok = true;
         for (int c0 = 0; c0 < a.k_chunks; c0 += kc, ++ks) {
           const int kcs = min(kc, a.k_chunks - c0);
-          const uint32_t base = s0 + ring_alloc(pos, head, step_bytes<kMx>(kcs, n));
+          const uint32_t base = s0 + ring_alloc(pos, head, step_bytes<kKind>(kcs, n));
           if (!mbar_wait(full0 + 8 * (ks % kSlots), (ks / kSlots) & 1u, abort_flag, a.status, kSiteFull) ||
               !mbar_wait(fullx0 + 8 * (ks % kSlots), (ks / kSlots) & 1u, abort_flag, a.status, kSiteFullX)) {
             ok = false;
@@ -396,6 +436,20 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
               if (c < kcs)
                 umma_mx_chunk(d_tmem, a_lo + c * (kTileW >> 4), b_lo + c * b_step, idesc, sf_t + 4 * c,
                               sf_t + 4 * kcs + 4 * nb * c, (c0 != 0 || c != 0) ? 1u : 0u);
+          } else if (kB128) {
+            // one fresh partial per K chunk, into the next free buffer
+            for (int c = 0; c < kcs; ++c, ++pc) {
+              const uint32_t pb = pc % kPartBufs;
+              if (!mbar_wait(pempty0 + 8 * pb, ((pc / kPartBufs) & 1u) ^ 1u, abort_flag, a.status, kSitePartEmpty)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              umma_e4m3_chunk(tmem_base + pb * kPartCols, a_lo + c * (kTileW >> 4), b_lo + c * b_step, idesc, 0u);
+              umma_commit(pfull0 + 8 * pb);
+            }
+            if (!ok) break;
+            continue;  // the epilogue releases the step's ring space
           } else if (kFp8) {
             umma_e4m3_chunk(d_tmem, a_lo, b_lo, idesc, c0 != 0);
 #pragma unroll
@@ -410,7 +464,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
           umma_commit(empty0 + 8 * (ks % kSlots));  // arrives once these MMAs have read the step
         }
         if (!ok) break;
-        umma_commit(tfull0 + 8 * acc);
+        if (!kB128) umma_commit(tfull0 + 8 * acc);
         ++it;
       }
       // all MMAs of this thread complete before TMEM is released
@@ -419,14 +473,16 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
     }
   } else {
     // ---------------- epilogue (warps 2..5): lane = weight row ----------------
-    // 32 token columns per TMEM load. For a given token the warp's 32 lanes hold
-    // neighbouring output columns, so each store writes one contiguous piece of an output
-    // row (GEMM2: 128 B of fp32; GEMM1: 64 or 32 B of a 128-byte activation chunk row).
+    // 32 token columns at a time. For a given token the warp's 32 lanes hold neighbouring
+    // output columns, so each store writes one contiguous piece of an output row (GEMM2:
+    // 128 B of fp32; GEMM1: 64 or 32 B of a 128-byte activation chunk row).
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
     const bool gated = a.activation != 1;  // 0 SwiGLU, 2 gelu_tanh, 3 swigluoai; 1 relu2
     const bool odd = (lane & 1) != 0;
     int rslot = 0, it = 0;
     uint32_t rph = 0;
+    uint32_t ks = 0, pos = 0, pc = 0;  // FP8 block-128: the ring allocation replayed, partials consumed
+    uint64_t head = 0;
     while (true) {
       int4 t = make_int4(0, 0, 0, 0);
       int ok = 0;
@@ -437,7 +493,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
       const int x_row = __shfl_sync(0xffffffffu, t.x, 0);
       const int expert = __shfl_sync(0xffffffffu, t.z, 0);
       const int mt = __shfl_sync(0xffffffffu, t.w, 0);
-      // FP8: the accumulator's dequantisation scale (GEMM1: before the activation)
+      // FP8 per-tensor: the accumulator's dequantisation scale (GEMM1: before the activation)
       const float dq = kFp8 ? __ldg(a.w_scale + expert) * a.in_scale : 1.0f;
       // GEMM2: routing weights of the group's tokens (token 32 b + lane in wreg[b]),
       // loaded while the main loop still runs
@@ -450,11 +506,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
           if (pid < a.num_pairs) wreg[b] = a.topk_w[pid];
         }
       }
-      const int acc = it & 1;
-      const bool got = mbar_wait(tfull0 + 8 * acc, (it >> 1) & 1, abort_flag, a.status, kSiteTmemFull);
-      if (!__all_sync(0xffffffffu, got)) break;  // leave warp-uniformly (tcgen05.ld is .aligned)
-      tc_fence_after();
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * kAccCols;
       // GEMM1: this lane's activation feature f lies in K chunk f / 64 (bf16) or f / 128
       // (e4m3) of the activation; byte b of a 128-byte chunk row sits in 16-byte piece
       // (b / 16) ^ (row % 8)
@@ -463,26 +514,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
       const int fo = kFp8 ? f & 127 : (f & 63) * 2;  // byte offset in the chunk row
       uint8_t* act_grp = static_cast<uint8_t*>(a.out) + static_cast<size_t>(x_row) * a.out_chunks * kChunkBytes +
                          static_cast<size_t>(fc) * n * kChunkBytes;
-      for (int c0 = 0; c0 < n; c0 += 32) {
-        const bool full = n - c0 >= 32;  // else 16 columns remain
-        float wl = wreg[0];              // GEMM2: routing weight of token column c0 + lane
+
+      // Output of token columns c0 .. c0 + 31 (c0 .. c0 + 15 unless `full`) of this lane's
+      // weight row, from v[j] = accumulator of column c0 + j.
+      auto store_block = [&](const uint32_t(&v)[32], int c0, bool full) {
+        float wl = wreg[0];  // GEMM2: routing weight of token column c0 + lane
 #pragma unroll
         for (int b = 1; b < kNMax / 32; ++b)
           if (c0 == 32 * b) wl = wreg[b];
-        uint32_t v[32];
-        if (full) {
-          tmem_ld32(taddr + c0, v);
-        } else {
-          uint32_t(&v16)[16] = *reinterpret_cast<uint32_t(*)[16]>(&v[0]);
-          tmem_ld16(taddr + c0, v16);
-#pragma unroll
-          for (int j = 16; j < 32; ++j) v[j] = 0u;
-        }
-        tmem_wait_ld();
-        if (c0 + 32 >= n) {
-          tc_fence_before();
-          mbar_arrive(tempty0 + 8 * acc);  // the accumulator is in registers now
-        }
         if (a.mode != 0) {
           const int col = mt * kMW + q * 32 + lane;
           float* y = static_cast<float*>(a.out) + static_cast<size_t>(x_row + c0) * a.out_cols + col;
@@ -507,7 +546,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
         } else {
           // lane pair (2m, 2m+1) = (gate, up) of feature m. The even lane finishes tokens
           // 0..15 of the batch, the odd lane tokens 16..31: each passes the other the half
-          // it needs, so every lane evaluates silu on 16 tokens.
+          // it needs, so every lane evaluates the activation on 16 tokens.
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const float mine_lo = __uint_as_float(v[j]) * dq;       // even: gate_j; odd: up_j
@@ -525,6 +564,110 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
                 *reinterpret_cast<__nv_bfloat16*>(dst) = __float2bfloat16_rn(h);
             }
           }
+        }
+      };
+
+      if constexpr (kB128) {
+        // promote each K chunk's partial: acc[j] += partial[j] * s_w * s_x[j]
+        const int kc = chunks_per_step(n);
+        // the tile's weight scales, lane k holding K chunk k (k_chunks <= 32): gated GEMM1's
+        // even lanes are gate rows (block row mt / 2), its odd lanes up rows
+        const float* sw_e = a.w_scale + static_cast<size_t>(expert) * a.ws_rows * a.k_chunks;
+        const int rb_even = a.up_block > 0 ? mt >> 1 : mt;
+        const int rb_odd = a.up_block > 0 ? a.up_block + (mt >> 1) : mt;
+        const float swl_even = lane < a.k_chunks ? __ldg(sw_e + static_cast<size_t>(rb_even) * a.k_chunks + lane) : 0.f;
+        const float swl_odd = lane < a.k_chunks ? __ldg(sw_e + static_cast<size_t>(rb_odd) * a.k_chunks + lane) : 0.f;
+        float acc[kB128GroupRows];
+#pragma unroll
+        for (int i = 0; i < kB128GroupRows; ++i) acc[i] = 0.f;
+        bool good = true;
+        for (int c0 = 0; c0 < a.k_chunks && good; c0 += kc, ++ks) {
+          const int kcs = min(kc, a.k_chunks - c0);
+          // the X scales of this step: [chunk][row] fp32 right behind its codes
+          const uint32_t sf = s0 + ring_alloc(pos, head, step_bytes<kKind>(kcs, n)) +
+                              static_cast<uint32_t>(kcs) * (kTileW + n * kChunkBytes);
+          for (int c = 0; c < kcs; ++c, ++pc) {
+            const uint32_t pb = pc % kPartBufs;
+            const bool got = mbar_wait(pfull0 + 8 * pb, (pc / kPartBufs) & 1u, abort_flag, a.status, kSitePartFull);
+            if (!__all_sync(0xffffffffu, got)) {  // leave warp-uniformly (tcgen05.ld is .aligned)
+              good = false;
+              break;
+            }
+            tc_fence_after();
+            const float sw_e_k = __shfl_sync(0xffffffffu, swl_even, c0 + c);
+            const float sw_o_k = __shfl_sync(0xffffffffu, swl_odd, c0 + c);
+            const float sw = odd ? sw_o_k : sw_e_k;
+            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + pb * kPartCols;
+            const uint32_t sfc = sf + static_cast<uint32_t>(c * n) * 4u;
+#pragma unroll
+            for (int cb = 0; cb < kB128GroupRows / 32; ++cb) {
+              if (cb * 32 < n) {
+                const bool full = n - cb * 32 >= 32;
+                uint32_t v[32];
+                if (full) {
+                  tmem_ld32(taddr + cb * 32, v);
+                } else {
+                  uint32_t(&v16)[16] = *reinterpret_cast<uint32_t(*)[16]>(&v[0]);
+                  tmem_ld16(taddr + cb * 32, v16);
+#pragma unroll
+                  for (int j = 16; j < 32; ++j) v[j] = 0u;
+                }
+                tmem_wait_ld();
+#pragma unroll
+                for (int j4 = 0; j4 < 8; ++j4) {
+                  if (j4 == 4 && !full) break;
+                  float4 sx;  // the same four scales for every lane: a shared-memory broadcast
+                  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                               : "=f"(sx.x), "=f"(sx.y), "=f"(sx.z), "=f"(sx.w)
+                               : "r"(sfc + static_cast<uint32_t>(cb * 32 + 4 * j4) * 4u));
+                  const int j = cb * 32 + 4 * j4;
+                  acc[j + 0] = fmaf(__uint_as_float(v[4 * j4 + 0]), sx.x * sw, acc[j + 0]);
+                  acc[j + 1] = fmaf(__uint_as_float(v[4 * j4 + 1]), sx.y * sw, acc[j + 1]);
+                  acc[j + 2] = fmaf(__uint_as_float(v[4 * j4 + 2]), sx.z * sw, acc[j + 2]);
+                  acc[j + 3] = fmaf(__uint_as_float(v[4 * j4 + 3]), sx.w * sw, acc[j + 3]);
+                }
+              }
+            }
+            tc_fence_before();
+            mbar_arrive(pempty0 + 8 * pb);  // the partial is in registers now
+          }
+          if (!good) break;
+          __syncwarp();  // every lane has read the step's scales
+          if (lane == 0) mbar_arrive(empty0 + 8 * (ks % kSlots));
+        }
+        if (!__all_sync(0xffffffffu, good)) break;
+#pragma unroll
+        for (int cb = 0; cb < kB128GroupRows / 32; ++cb) {
+          if (cb * 32 < n) {
+            uint32_t v[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(acc[cb * 32 + j]);
+            store_block(v, cb * 32, n - cb * 32 >= 32);
+          }
+        }
+      } else {
+        const int acc = it & 1;
+        const bool got = mbar_wait(tfull0 + 8 * acc, (it >> 1) & 1, abort_flag, a.status, kSiteTmemFull);
+        if (!__all_sync(0xffffffffu, got)) break;  // leave warp-uniformly (tcgen05.ld is .aligned)
+        tc_fence_after();
+        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * kAccCols;
+        for (int c0 = 0; c0 < n; c0 += 32) {
+          const bool full = n - c0 >= 32;  // else 16 columns remain
+          uint32_t v[32];
+          if (full) {
+            tmem_ld32(taddr + c0, v);
+          } else {
+            uint32_t(&v16)[16] = *reinterpret_cast<uint32_t(*)[16]>(&v[0]);
+            tmem_ld16(taddr + c0, v16);
+#pragma unroll
+            for (int j = 16; j < 32; ++j) v[j] = 0u;
+          }
+          tmem_wait_ld();
+          if (c0 + 32 >= n) {
+            tc_fence_before();
+            mbar_arrive(tempty0 + 8 * acc);  // the accumulator is in registers now
+          }
+          store_block(v, c0, full);
         }
       }
       ++it;
@@ -549,7 +692,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
   }
 }
 
-bool g_attr_set[3][64] = {};
+bool g_attr_set[4][64] = {};
 
 }  // namespace
 
@@ -559,9 +702,10 @@ cudaError_t launch_gemm_swap(const Launch& l, int mode, const SwapOperands& o, c
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  const int kind = o.mx ? 2 : (o.fp8 ? 1 : 0);
+  const int kind = o.b128 ? 3 : (o.mx ? 2 : (o.fp8 ? 1 : 0));
   void (*const kernel)(const Args) =
-      kind == 2 ? gemm_swap_kernel<2> : (kind == 1 ? gemm_swap_kernel<1> : gemm_swap_kernel<0>);
+      kind == 3 ? gemm_swap_kernel<3>
+                : (kind == 2 ? gemm_swap_kernel<2> : (kind == 1 ? gemm_swap_kernel<1> : gemm_swap_kernel<0>));
   if (!g_attr_set[kind][dev]) {
     err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (err != cudaSuccess) return err;
@@ -570,6 +714,10 @@ cudaError_t launch_gemm_swap(const Launch& l, int mode, const SwapOperands& o, c
   if ((reinterpret_cast<uintptr_t>(o.w) | reinterpret_cast<uintptr_t>(o.x)) & 15u) return cudaErrorInvalidValue;
   if (kind == 2 && (o.w_sf == nullptr || o.x_sf == nullptr ||
                     ((reinterpret_cast<uintptr_t>(o.w_sf) | reinterpret_cast<uintptr_t>(o.x_sf)) & 15u)))
+    return cudaErrorInvalidValue;
+  // FP8 block-128: K and the weight rows whole 128-blocks, the K chunks' weight scales held
+  // one per lane of a warp
+  if (kind == 3 && (o.w_scale == nullptr || s.K % 128 != 0 || s.N % 128 != 0 || s.K / 128 > 32))
     return cudaErrorInvalidValue;
   Args a;
   a.mode = mode;
@@ -595,6 +743,8 @@ cudaError_t launch_gemm_swap(const Launch& l, int mode, const SwapOperands& o, c
   a.act_inv = o.act_scale > 0.f ? 1.0f / o.act_scale : 0.f;
   a.w_sf = static_cast<const uint8_t*>(o.w_sf);
   a.x_sf = static_cast<const uint8_t*>(o.x_sf);
+  a.ws_rows = s.N / 128;
+  a.up_block = o.up_block;
   cudaLaunchConfig_t cfg;
   cudaLaunchAttribute attr[1];
   make_launch_config(&cfg, attr, l, dim3(s.num_sms), dim3(kThreads), kSmemBytes);

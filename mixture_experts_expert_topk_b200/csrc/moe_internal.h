@@ -54,6 +54,17 @@ cudaError_t launch_permute_rows(const Launch& l, const void* hidden, int H, cons
 cudaError_t launch_permute_quant_rows(const Launch& l, const void* hidden, int H, const int* sorted_pair_ids,
                                       const int* num_groups, const int2* group_info, int P, int k_total,
                                       float input_scale, void* xs, int num_sms);
+// FP8 block-128: the token rows of every row group quantised per 1x128 group (scale =
+// amax / 448, 1 for an all-zero group; code = e4m3(x / scale), IEEE fp32 divisions, round to
+// nearest even, saturating), in the X layout above with KC = H / 128. Padding rows are zero
+// codes with scale 1.
+cudaError_t launch_permute_b128_rows(const Launch& l, const void* hidden, int H, const int* sorted_pair_ids,
+                                     const int* num_groups, const int2* group_info, int P, int k_total, void* xs,
+                                     int num_sms);
+// FP8 block-128: GEMM1's bf16 activation (row-group order, 64-column chunks) quantised per
+// 1x128 group the same way into the X layout above with KC = I / 128, for GEMM2.
+cudaError_t launch_act_quant_b128(const Launch& l, const void* act, int I, const int* num_groups,
+                                  const int2* group_info, void* actq, int num_sms);
 
 // ---- GEMMs (gemm_bf16.cu, gemm_fp8.cu) ----
 struct GemmShape {
@@ -103,10 +114,32 @@ struct SwapOperands {
   int mx;
   const void* w_sf;
   const void* x_sf;
+  // FP8 block-128 (e4m3 operands, fp32 scales per 128x128 weight block and per 1x128 group
+  // of X, promoted in the epilogue): b128 = 1; w_scale [E, rows/128, K/128] in the
+  // checkpoint block layout; gated GEMM1 sets up_block = I / 128 (the up half's first block
+  // row). X is in row-group order with each K step's codes followed by the fp32 scales of
+  // its rows (launch_permute_b128_rows, launch_act_quant_b128).
+  int b128;
+  int up_block;
 };
 // Row groups of the MXFP8 swapped-operand GEMMs: at most this many rows, so that two
 // accumulators leave a quarter of TMEM for the block scales.
 constexpr int kMxGroupRows = 192;
+// Row groups of the FP8 block-128 swapped-operand GEMMs: at most this many rows, so that a
+// group's fp32 accumulator fits the epilogue threads' registers.
+constexpr int kB128GroupRows = 128;
+// K chunks (128-byte chunk rows) per K step of the swapped-operand GEMMs for a row group
+// of n rows: steps of 48 to 72 KB of operands.
+__host__ __device__ constexpr int chunks_per_step(int n) {
+  return n <= 32 ? 4 : (n <= 64 ? 3 : (n <= 128 ? 2 : 1));
+}
+// FP8 block-128 X layout (row-group order with each K step's fp32 row scales behind its
+// codes): the group of n rows at sorted row x_row owns bytes [x_row * KC * 132, (x_row + n)
+// * KC * 132); its step of chunks [c0, c0 + kcs), kcs = min(chunks_per_step(n), KC - c0),
+// starts at c0 * n * 132 and holds kcs chunks of n rows x 128 bytes of e4m3 codes (row j
+// of chunk c at (c - c0) * n * 128 + j * 128, its 16-byte pieces swizzled by j % 8), then
+// the fp32 scales of chunk c, row j at kcs * n * 128 + ((c - c0) * n + j) * 4.
+constexpr int kB128RowBytesPerChunk = 132;
 // N tile for a GEMM with N output columns, given an estimate of the number of 128-row
 // tiles and the SM count (0 if no multiple of 32 divides N).
 int pick_bn(int N, long long est_row_tiles, int num_sms);

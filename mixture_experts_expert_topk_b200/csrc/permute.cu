@@ -262,7 +262,135 @@ __global__ void __launch_bounds__(kThreads)
   }
 }
 
+// Byte offsets, inside a row group of n rows and KC chunks, of row j's codes in chunk c
+// (unswizzled start of the 128-byte chunk row) and of its fp32 scale: the FP8 block-128
+// X layout (moe_internal.h).
+__device__ __forceinline__ void b128_offsets(int n, int KC, int c, int j, size_t& code, size_t& scale) {
+  const int kc = chunks_per_step(n);
+  const int c0 = c - c % kc;
+  const int kcs = min(kc, KC - c0);
+  const size_t step = static_cast<size_t>(c0) * n * kB128RowBytesPerChunk;
+  code = step + static_cast<size_t>(c - c0) * n * 128 + static_cast<size_t>(j) * 128;
+  scale = step + static_cast<size_t>(kcs) * n * 128 + (static_cast<size_t>(c - c0) * n + j) * 4;
+}
+
+// One 1x128 group held as four values per lane: scale = amax / 448 (1 for all zeros) and
+// the lane's four codes e4m3(x / scale), IEEE divisions. Every lane takes part.
+__device__ __forceinline__ uint32_t quant_group_1x128(float x0, float x1, float x2, float x3, float& s) {
+  float amax = fmaxf(fmaxf(fabsf(x0), fabsf(x1)), fmaxf(fabsf(x2), fabsf(x3)));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  s = amax == 0.f ? 1.f : __fdiv_rn(amax, 448.f);
+  const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(__fdiv_rn(x0, s), __fdiv_rn(x1, s)), __NV_SATFINITE,
+                                               __NV_E4M3);
+  const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(__fdiv_rn(x2, s), __fdiv_rn(x3, s)), __NV_SATFINITE,
+                                               __NV_E4M3);
+  return lo | (hi << 16);
+}
+
+// FP8 block-128: a warp quantises one row of a group, lane l taking columns 4l..4l+3 of
+// every 128-column chunk (all of the row's loads issued first).
+constexpr int kB128MaxChunks = 32;  // H <= 4096
+__global__ void __launch_bounds__(kThreads)
+    permute_b128_rows_kernel(const uint2* __restrict__ hidden, int H, const int* __restrict__ sorted_pair_ids,
+                             const int* __restrict__ num_groups, const int2* __restrict__ group_info, int P,
+                             int k_total, uint8_t* __restrict__ xs) {
+  griddep_wait();
+  griddep_launch_dependents();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int G = *num_groups;
+  const int KC = H / 128;
+  for (int g = blockIdx.x; g < G; g += gridDim.x) {
+    const int2 gi = group_info[g];
+    const int x_row = gi.x, n = gi.y >> 16;
+    uint8_t* base = xs + static_cast<size_t>(x_row) * KC * kB128RowBytesPerChunk;
+    for (int j = blockIdx.y * (kThreads / 32) + warp; j < n; j += gridDim.y * (kThreads / 32)) {
+      const int pid = sorted_pair_ids[x_row + j];
+      const uint2* src = pid < P ? hidden + static_cast<size_t>(pid / k_total) * (H / 4) : nullptr;
+      uint2 in[kB128MaxChunks];
+#pragma unroll
+      for (int c = 0; c < kB128MaxChunks; ++c)
+        in[c] = (c < KC && src != nullptr) ? __ldg(src + c * 32 + lane) : make_uint2(0u, 0u);
+#pragma unroll
+      for (int c = 0; c < kB128MaxChunks; ++c) {
+        if (c >= KC) break;
+        const float2 f01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&in[c].x));
+        const float2 f23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&in[c].y));
+        float sc;
+        const uint32_t codes = quant_group_1x128(f01.x, f01.y, f23.x, f23.y, sc);
+        size_t co, so;
+        b128_offsets(n, KC, c, j, co, so);
+        const int ob = 4 * lane;
+        *reinterpret_cast<uint32_t*>(base + co + ((((ob >> 4) ^ j) & 7) << 4) + (ob & 15)) = codes;
+        if (lane == 0) *reinterpret_cast<float*>(base + so) = sc;
+      }
+    }
+  }
+}
+
+// FP8 block-128: GEMM1's bf16 activation (64-column chunks of 128-byte rows, row-group
+// order) quantised per 1x128 group into the X layout; a warp takes one row, lane l columns
+// 4l..4l+3 of each 128-column chunk (8 bytes of bf16 chunk 2c + l / 16).
+__global__ void __launch_bounds__(kThreads)
+    act_quant_b128_kernel(const uint8_t* __restrict__ act, int I, const int* __restrict__ num_groups,
+                          const int2* __restrict__ group_info, uint8_t* __restrict__ actq) {
+  griddep_wait();
+  griddep_launch_dependents();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int G = *num_groups;
+  const int KCb = I / 64, KC = I / 128;
+  for (int g = blockIdx.x; g < G; g += gridDim.x) {
+    const int2 gi = group_info[g];
+    const int x_row = gi.x, n = gi.y >> 16;
+    const uint8_t* in = act + static_cast<size_t>(x_row) * KCb * 128;
+    uint8_t* base = actq + static_cast<size_t>(x_row) * KC * kB128RowBytesPerChunk;
+    for (int j = blockIdx.y * (kThreads / 32) + warp; j < n; j += gridDim.y * (kThreads / 32)) {
+      const int ib = 8 * (lane & 15);  // byte of the bf16 chunk row
+      uint2 raw[kB128MaxChunks];
+#pragma unroll
+      for (int c = 0; c < kB128MaxChunks; ++c)
+        raw[c] = c < KC ? *reinterpret_cast<const uint2*>(in + static_cast<size_t>(2 * c + (lane >> 4)) * n * 128 +
+                                                            j * 128 + ((((ib >> 4) ^ j) & 7) << 4) + (ib & 15))
+                        : make_uint2(0u, 0u);
+#pragma unroll
+      for (int c = 0; c < kB128MaxChunks; ++c) {
+        if (c >= KC) break;
+        const float2 f01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw[c].x));
+        const float2 f23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw[c].y));
+        float sc;
+        const uint32_t codes = quant_group_1x128(f01.x, f01.y, f23.x, f23.y, sc);
+        size_t co, so;
+        b128_offsets(n, KC, c, j, co, so);
+        const int ob = 4 * lane;
+        *reinterpret_cast<uint32_t*>(base + co + ((((ob >> 4) ^ j) & 7) << 4) + (ob & 15)) = codes;
+        if (lane == 0) *reinterpret_cast<float*>(base + so) = sc;
+      }
+    }
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_permute_b128_rows(const Launch& l, const void* hidden, int H, const int* sorted_pair_ids,
+                                     const int* num_groups, const int2* group_info, int P, int k_total, void* xs,
+                                     int num_sms) {
+  if (H % 128 != 0 || H / 128 > kB128MaxChunks) return cudaErrorInvalidValue;
+  cudaLaunchConfig_t cfg;
+  cudaLaunchAttribute attr[1];
+  make_launch_config(&cfg, attr, l, dim3(2 * num_sms, kB128GroupRows / (kThreads / 32)), dim3(kThreads), 0);
+  return cudaLaunchKernelEx(&cfg, permute_b128_rows_kernel, static_cast<const uint2*>(hidden), H, sorted_pair_ids,
+                            num_groups, group_info, P, k_total, static_cast<uint8_t*>(xs));
+}
+
+cudaError_t launch_act_quant_b128(const Launch& l, const void* act, int I, const int* num_groups,
+                                  const int2* group_info, void* actq, int num_sms) {
+  if (I % 128 != 0 || I / 128 > kB128MaxChunks) return cudaErrorInvalidValue;
+  cudaLaunchConfig_t cfg;
+  cudaLaunchAttribute attr[1];
+  make_launch_config(&cfg, attr, l, dim3(2 * num_sms, kB128GroupRows / (kThreads / 32)), dim3(kThreads), 0);
+  return cudaLaunchKernelEx(&cfg, act_quant_b128_kernel, static_cast<const uint8_t*>(act), I, num_groups,
+                            group_info, static_cast<uint8_t*>(actq));
+}
 
 cudaError_t launch_permute_quant_rows(const Launch& l, const void* hidden, int H, const int* sorted_pair_ids,
                                       const int* num_groups, const int2* group_info, int P, int k_total,

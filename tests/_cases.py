@@ -273,3 +273,31 @@ def untile_u8(flat, group_info, num_groups, rows, kchunks):
         phys = np.arange(8)[None, :] ^ (j[:, None] & 7)
         out[x_row:x_row + n] = grp[:, j[:, None], phys, :].transpose(1, 0, 2, 3).reshape(n, 128 * kchunks)
     return out
+
+
+def untile_b128(flat, group_info, num_groups, rows, kchunks):
+    """(codes uint8 [rows, 128 * kchunks], scales float32 [rows, kchunks]) from the FP8
+    block-128 X layout of the swapped-operand GEMMs: the group of n rows at x_row owns
+    bytes from x_row * kchunks * 132; its K step of chunks [c0, c0 + kcs) (kcs chunks per
+    step as the GEMM takes them for n rows: 4 up to 32 rows, 3 up to 64, 2 up to 128)
+    starts at c0 * n * 132 with kcs chunks of n swizzled 128-byte code rows, then the
+    step's fp32 scales, chunk-major. Rows outside every group stay zero."""
+    flat = np.asarray(flat).reshape(-1)
+    codes = np.zeros((rows, 128 * kchunks), dtype=np.uint8)
+    scales = np.zeros((rows, kchunks), dtype=np.float32)
+    for g in range(num_groups):
+        x_row, meta = int(group_info[g][0]), int(group_info[g][1])
+        n = meta >> 16
+        kc = 4 if n <= 32 else (3 if n <= 64 else (2 if n <= 128 else 1))
+        base = x_row * kchunks * 132
+        j = np.arange(n)
+        phys = np.arange(8)[None, :] ^ (j[:, None] & 7)
+        for c0 in range(0, kchunks, kc):
+            kcs = min(kc, kchunks - c0)
+            step = base + c0 * n * 132
+            cod = flat[step:step + kcs * n * 128].reshape(kcs, n, 8, 16)
+            codes[x_row:x_row + n, 128 * c0:128 * (c0 + kcs)] = \
+                cod[:, j[:, None], phys, :].transpose(1, 0, 2, 3).reshape(n, 128 * kcs)
+            sc = flat[step + kcs * n * 128:step + kcs * n * 132].copy().view(np.float32).reshape(kcs, n)
+            scales[x_row:x_row + n, c0:c0 + kcs] = sc.T
+    return codes, scales

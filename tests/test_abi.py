@@ -59,7 +59,9 @@ def test_check_problem_accepts_the_workloads(L):
     (dict(topk=9), 1), (dict(topk=0), 1), (dict(intermediate=500), 1),
     (dict(intermediate=512, activation="relu2"), 0), (dict(intermediate=528, activation="relu2"), 1),
     (dict(num_routed=1100, topk=2), 2), (dict(num_routed=32, topk=17), 2),
-    (dict(block_m=64), 2), (dict(intermediate=528, fp8=True), 1), (dict(block_m=16, fp8=True), 2),
+    (dict(block_m=64), 2), (dict(intermediate=528, fp8=True), 1), (dict(block_m=16, fp8=True), 0),
+    (dict(block_m=128, fp8="mxfp8"), 2), (dict(block_m=128, fp8="per_tensor", input_scale=0.1, activation_scale=0.1), 2),
+    (dict(H=4224, fp8=True), 2),
 ])
 def test_check_problem_rejects(L, kw, status):
     p = _prob(**kw)
@@ -105,13 +107,13 @@ def test_workspace_layout(L):
         E = cfg.E_total
         assert lay["status"] == 0
         bm = lay["block_m"]
-        # bf16 and per-tensor FP8 align each expert to 16 rows (token rows on the MMA's N),
-        # block-128 FP8 to 128-row tiles
-        assert bm == (128 if cfg.block128 else 16)
-        # the permuted hidden rows (row-group order) exist for the 16-row alignment
+        # every format aligns each expert to 16 rows by default (token rows on the MMA's N)
+        assert bm == 16
+        # the permuted hidden rows (row-group order): bf16, e4m3 codes, or (FP8 block-128)
+        # e4m3 codes with a 4-byte scale per row per 128 columns
         xs_bytes = lay["xs_scale"] - lay["xs"]
-        elt = 1 if (cfg.per_tensor or cfg.mx) else 2
-        assert xs_bytes == (-(-lay["max_rows"] * cfg.H * elt // 1024) * 1024 if not cfg.block128 else 0)
+        row_bytes = cfg.H * 132 // 128 if cfg.block128 else cfg.H * (1 if (cfg.per_tensor or cfg.mx) else 2)
+        assert xs_bytes == -(-lay["max_rows"] * row_bytes // 1024) * 1024
         assert lay["max_rows"] == -(-(P + min(E, P) * (bm - 1)) // bm) * bm
         assert lay["num_chunks"] == -(-P // 2048)
         offs = sorted(v for k, v in lay.items() if k not in ("total_bytes", "max_rows", "num_chunks", "block_m"))

@@ -20,7 +20,7 @@ from oracle import moe_oracle as O
 
 from _cases import (GpuForward, act_rows_f64, bf16_act_bound, bf16_to_f64, bits, check_act_pairs, cover_tokens,
                     cpu_inputs, err_beyond_rounding, max_err_over_rms, oracle_fp8_block_weights, oracle_mxfp8_weights,
-                    oracle_out, untile_groups, untile_u8, untile_weights)
+                    oracle_out, untile_b128, untile_groups, untile_u8, untile_weights)
 
 pytestmark = pytest.mark.gpu
 
@@ -84,10 +84,10 @@ def _check_route_align(cfg, parts, logits, bm=None):
 
 def _check_groups(cfg, parts, a):
     """Row groups of the swapped-operand GEMMs: each expert's padded segment cut into
-    ceil(rows / 256) groups of whole 16-row blocks, sizes as even as possible, larger
-    first; and the permuted hidden rows."""
+    ceil(rows / G) groups of whole 16-row blocks, sizes as even as possible, larger first
+    (G = 256; 128 for FP8 block-128); and, for bf16, the permuted hidden rows."""
     P = cfg.T * cfg.k_total
-    G = 256
+    G = 128 if cfg.block128 else 256
     off = a["expert_offsets"]
     expect = []
     for e in range(cfg.E_total):
@@ -105,6 +105,8 @@ def _check_groups(cfg, parts, a):
         assert row == off[e + 1]
     assert int(parts["num_blocks"][1]) == len(expect)
     np.testing.assert_array_equal(parts["group_info"][:len(expect)], np.array(expect, dtype=np.int32).reshape(-1, 2))
+    if cfg.fp8:
+        return
     # the permuted hidden rows, in row-group order
     rows = int(a["P_pad"])
     xs = untile_groups(parts["xs"], parts["group_info"], len(expect), rows, cfg.H // 64)
@@ -264,7 +266,7 @@ def test_fp8_quantizers_bit_exact():
     x = torch.randn((37, 512), generator=g).to(torch.bfloat16)
     x[3, 128:256] = 0
     x[5, :5] = 1000.0
-    prob = moe.make_problem(37, 512, 8, 2, 512, fp8=True)
+    prob = moe.make_problem(37, 512, 8, 2, 512, fp8=True, block_m=128)   # the token-tile path quantises [T, H]
     ws = moe.new_workspace(prob)
     moe.stage_quant_act(prob, x.cuda(), ws)
     torch.cuda.synchronize()
@@ -336,25 +338,53 @@ FP8_SMALL = {
 }
 
 
-@pytest.mark.parametrize("name", list(FP8_SMALL))
-def test_fp8_layer_parity_small(name):
+def _check_b128_operands(cfg, parts, a, hidden_bits):
+    """FP8 block-128 on the swapped-operand GEMMs: the permuted hidden rows and GEMM2's
+    input (GEMM1's own bf16 activation) quantised per 1x128, codes and scales bit for bit
+    against the oracle's quantiser; padding rows are zero codes with scale 1."""
+    kk = cfg.k_total
+    P = cfg.T * kk
+    P_pad = int(a["P_pad"])
+    gi, ng = parts["group_info"], int(parts["num_blocks"][1])
+    pids = a["sorted_pair_ids"][:P_pad]
+    real = pids < P
+    qx, sx = O.quant_groups_1x128(O.bf16_bits_to_f32(hidden_bits))
+    xs_c, xs_s = untile_b128(parts["xs"], gi, ng, P_pad, cfg.H // 128)
+    np.testing.assert_array_equal(xs_c[real], qx[pids[real] // kk])
+    np.testing.assert_array_equal(xs_s[real], sx[pids[real] // kk])
+    assert np.all(xs_c[~real] == 0) and np.all(xs_s[~real] == 1.0)
+    act_bits = untile_groups(parts["act"], gi, ng, P_pad, -(-cfg.I // 64))[:, :cfg.I]
+    qa, sa = O.quant_groups_1x128(O.bf16_bits_to_f32(act_bits[real]))
+    aq_c, aq_s = untile_b128(parts["actq"], gi, ng, P_pad, cfg.I // 128)
+    np.testing.assert_array_equal(aq_c[real], qa)
+    np.testing.assert_array_equal(aq_s[real], sa)
+    return qx, sx
+
+
+@pytest.mark.parametrize("name,bm", [(n, 0) for n in FP8_SMALL] +
+                         [(n, 128) for n in ("fp8_tiny", "fp8_shared_small", "fp8_relu2", "fp8_oai")])
+def test_fp8_layer_parity_small(name, bm):
+    # bm 0: the default (16-row alignment, weights on the MMA's M, per-chunk partials
+    # promoted in the epilogue); 128: 128-row token tiles
     cfg = FP8_SMALL[name]
-    run = GpuForward(cfg)
+    run = GpuForward(cfg, block_m=bm)
     out = run.forward()
     parts = run.parts()
     ids, a = _check_route_align(cfg, parts, run.inp["logits"])
-    # the GPU quantises its own bf16 activation per 1x128 group: codes and scales must be
-    # what the oracle's quantiser gives for those same bf16 values
-    P_pad = int(a["P_pad"])
-    rows = np.nonzero(a["sorted_pair_ids"] < cfg.T * cfg.k_total)[0]
-    act32 = O.bf16_bits_to_f32(parts["act"][rows])
-    q, sc = O.quant_groups_1x128(act32)
-    np.testing.assert_array_equal(parts["actq"][rows], q)
-    np.testing.assert_array_equal(parts["act_scale"][rows], sc)
-    # the hidden quantisation too
-    qx, sx = O.quant_groups_1x128(O.bf16_bits_to_f32(bits(run.inp["hidden"])))
-    np.testing.assert_array_equal(parts["xq"], qx)
-    np.testing.assert_array_equal(parts["xq_scale"], sx)
+    if parts["block_m"] == 16:
+        qx, sx = _check_b128_operands(cfg, parts, a, bits(run.inp["hidden"]))
+    else:
+        # the GPU quantises its own bf16 activation per 1x128 group: codes and scales must be
+        # what the oracle's quantiser gives for those same bf16 values
+        rows = np.nonzero(a["sorted_pair_ids"] < cfg.T * cfg.k_total)[0]
+        act32 = O.bf16_bits_to_f32(parts["act"][rows])
+        q, sc = O.quant_groups_1x128(act32)
+        np.testing.assert_array_equal(parts["actq"][rows], q)
+        np.testing.assert_array_equal(parts["act_scale"][rows], sc)
+        # the hidden quantisation too
+        qx, sx = O.quant_groups_1x128(O.bf16_bits_to_f32(bits(run.inp["hidden"])))
+        np.testing.assert_array_equal(parts["xq"], qx)
+        np.testing.assert_array_equal(parts["xq_scale"], sx)
     fp8w = O.quantize_weights_fp8(bits(run.inp["w13"]), bits(run.inp["w2"]))
     np.testing.assert_array_equal(run.w13_q.cpu().numpy(), fp8w[0])
     np.testing.assert_array_equal(run.w13_scale.cpu().numpy(), fp8w[1])
@@ -369,7 +399,7 @@ def test_fp8_layer_parity_small(name):
     got = bf16_to_f64(out)
     assert np.all(np.isfinite(got))
     e = err_beyond_rounding(got, ref)
-    print(f"{name}: beyond-rounding {e:.4f}, raw {max_err_over_rms(got, ref):.4f}")
+    print(f"{name}/bm{parts['block_m']}: beyond-rounding {e:.4f}, raw {max_err_over_rms(got, ref):.4f}")
     assert e <= FP8_TOL, e
     assert moe.device_status(run.ws)[0] == 0
 
@@ -715,10 +745,8 @@ def test_fp8_block128_full_size_every_expert():
     out = run.forward()
     parts = run.parts()
     ids, a = _check_route_align(cfg, parts, run.inp["logits"])
-    hid32 = O.bf16_bits_to_f32(bits(run.inp["hidden"]))
-    qx, sx = O.quant_groups_1x128(hid32)
-    np.testing.assert_array_equal(parts["xq"], qx)
-    np.testing.assert_array_equal(parts["xq_scale"], sx)
+    assert parts["block_m"] == 16
+    qx, sx = _check_b128_operands(cfg, parts, a, bits(run.inp["hidden"]))
     tokens = cover_tokens(ids, cfg.E, extra=16)
     experts = np.unique(ids[tokens])
     assert len(experts) == cfg.E_total
