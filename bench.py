@@ -250,7 +250,7 @@ def run_ours(cfg: MoeConfig, steps: int, warmup: int, world: int, rank: int, loc
 
     # per-kernel breakdown: the same kernels through the per-step entry points, events
     # between the steps on the launching stream
-    names = ["route", "align", "permute", "gemm1", "gemm2", "combine"]
+    names = ["route", "align"] + (["quant_act"] if cfg.block128 else []) + ["permute", "gemm1", "gemm2", "combine"]
     per = {n: [] for n in names}
     for _ in range(steps):
         flush.zero_()
@@ -259,6 +259,8 @@ def run_ours(cfg: MoeConfig, steps: int, warmup: int, world: int, rank: int, loc
         k = 0
         moe.stage_route(prob, logits, ws); k += 1; evs[k].record(stream)
         moe.stage_align(prob, ws); k += 1; evs[k].record(stream)
+        if cfg.block128:
+            moe.stage_quant_act(prob, hidden, ws); k += 1; evs[k].record(stream)
         moe.stage_permute(prob, hidden, ws); k += 1; evs[k].record(stream)
         moe.stage_gemm1(prob, hidden, w13p, ws, s13); k += 1; evs[k].record(stream)
         moe.stage_gemm2(prob, w2p, ws, s2); k += 1; evs[k].record(stream)

@@ -143,8 +143,8 @@ typedef struct {
   size_t block_expert;    /* int32 [max_rows/block_m]: expert of each row tile */
   size_t pair_to_row;     /* int32 [T*k']: sorted row of each pair */
   size_t chunk_hist;      /* int32 [num_chunks, E]: align scratch */
-  size_t xq;              /* FP8 block-128, block_m 128: e4m3 [T, H] quantised hidden */
-  size_t xq_scale;        /* FP8 block-128, block_m 128: fp32 [T, H/128] */
+  size_t xq;              /* FP8 block-128: e4m3 [T, H] quantised hidden */
+  size_t xq_scale;        /* FP8 block-128: fp32 [T, H/128] */
   size_t act;             /* GEMM1 output: bf16 [max_rows, I] (block_m 128) or bf16 in
                              row-group order (block_m 16; per-tensor FP8: e4m3 codes) */
   size_t actq;            /* FP8 block-128: the activation quantised per 1x128 group, e4m3
@@ -152,7 +152,9 @@ typedef struct {
                              layout of xs (block_m 16); MXFP8: e4m3 codes in row-group order */
   size_t act_scale;       /* FP8 block-128, block_m 128: fp32 [max_rows, I/128]; MXFP8: E8M0
                              scale blocks */
-  size_t y;               /* fp32 [max_rows, H]: weighted GEMM2 rows in sorted order */
+  size_t y;               /* weighted GEMM2 rows in sorted order: block_m 128: fp32 [max_rows,
+                             H]; block_m 16: fp16 [max_rows, H] followed by int8 [max_rows,
+                             H/32], row r's columns [32b, 32b+32) scaled by 2^(int8 [r, b]) */
   size_t xs;              /* block_m 16: the hidden rows of every row group in row-group order
                              (bf16; e4m3 codes for the 8-bit formats; FP8 block-128: each K
                              step's e4m3 codes followed by its rows' fp32 1x128 scales, 132
@@ -306,21 +308,21 @@ moe_status_t moe_forward_host(const moe_problem_t* problem, const void* h_hidden
                               void* workspace, size_t workspace_bytes, moe_stream_t stream);
 
 /* The steps as separate calls on the same workspace: route, align, quant_act (FP8
- * block-128 with block_m 128), permute (block_m 16), gemm1, gemm2, combine; moe_forward
- * runs exactly these, in this order. They exist so tests can check each intermediate and tools can time each kernel;
+ * block-128), permute (block_m 16), gemm1, gemm2, combine; moe_forward runs exactly these,
+ * in this order. They exist so tests can check each intermediate and tools can time each kernel;
  * each requires the previous steps to have been enqueued. */
 moe_status_t moe_stage_route(const moe_problem_t* problem, const float* router_logits,
                              void* workspace, size_t workspace_bytes, moe_stream_t stream);
 moe_status_t moe_stage_align(const moe_problem_t* problem, void* workspace,
                              size_t workspace_bytes, moe_stream_t stream);
-/* FP8 block-128 only (else MOE_ERR_INVALID_ARG): with block_m 128, quantise hidden per
- * token per 128 columns into the workspace (xq, xq_scale); with block_m 16 the permute
- * step quantises the rows instead and this call does nothing (MOE_OK). */
+/* FP8 block-128 only (else MOE_ERR_INVALID_ARG): quantise hidden per token per 128 columns
+ * into the workspace (xq, xq_scale). */
 moe_status_t moe_stage_quant_act(const moe_problem_t* problem, const void* hidden,
                                  void* workspace, size_t workspace_bytes, moe_stream_t stream);
 /* block_m 16 (the default): copy the token rows of every row group into the workspace in
- * the order GEMM1 reads them (xs), quantised on the way for the 8-bit formats; hidden
- * device bf16 [T, H]. block_m 128: nothing to do, MOE_OK. */
+ * the order GEMM1 reads them (xs), quantised on the way for per-tensor FP8 and MXFP8 (FP8
+ * block-128 copies the codes and scales of the quant_act step); hidden device bf16 [T, H].
+ * block_m 128: nothing to do, MOE_OK. */
 moe_status_t moe_stage_permute(const moe_problem_t* problem, const void* hidden, void* workspace,
                                size_t workspace_bytes, moe_stream_t stream);
 moe_status_t moe_stage_gemm1(const moe_problem_t* problem, const void* hidden, const void* w13,

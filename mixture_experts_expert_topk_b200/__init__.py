@@ -393,8 +393,14 @@ def read_workspace(prob: Problem, workspace: torch.Tensor) -> Dict[str, torch.Te
         "expert_offsets": view(L["expert_offsets"], E + 1, torch.int32),
         "block_expert": view(L["block_expert"], rows // L["block_m"], torch.int32),
         "pair_to_row": view(L["pair_to_row"], P, torch.int32),
-        "y": view(L["y"], rows * H, torch.float32).view(rows, H),
     }
+    if L["block_m"] == 16:
+        # weighted GEMM2 rows as fp16 with a power-of-two exponent per 32 columns:
+        # y = y16 * 2^y_exp
+        out["y16"] = view(L["y"], rows * H, torch.float16).view(rows, H)
+        out["y_exp"] = view(L["y"] + rows * H * 2, rows * (H // 32), torch.int8).view(rows, H // 32)
+    else:
+        out["y"] = view(L["y"], rows * H, torch.float32).view(rows, H)
     if prob.wdtype == MOE_DTYPE_MXFP8:
         # bf16 activation (64-column chunks), e4m3 codes of the hidden rows and of the
         # activation (128-column chunks), all in row-group order; the scale blocks raw
@@ -428,9 +434,10 @@ def read_workspace(prob: Problem, workspace: torch.Tensor) -> Dict[str, torch.Te
         out["group_info"] = view(L["group_info"], (rows // 16 + 1) * 2, torch.int32).view(-1, 2)
     else:
         out["act"] = view(L["act"], rows * I, torch.bfloat16).view(rows, I)
-    if fp8 and L["block_m"] == 128:
+    if fp8:
         out["xq"] = view(L["xq"], T * H, torch.uint8).view(T, H)
         out["xq_scale"] = view(L["xq_scale"], T * (H // 128), torch.float32).view(T, H // 128)
+    if fp8 and L["block_m"] == 128:
         out["actq"] = view(L["actq"], rows * I, torch.uint8).view(rows, I)
         out["act_scale"] = view(L["act_scale"], rows * (I // 128), torch.float32).view(rows, I // 128)
     return out

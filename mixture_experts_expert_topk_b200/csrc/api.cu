@@ -144,8 +144,8 @@ moe_status_t make_plan(const moe_problem_t* p, Plan* pl) {
   L.chunk_hist = take(static_cast<size_t>(L.num_chunks) * q.E * 4);
   const bool fp8_tiles = q.fp8 && q.bm == 128;  // FP8 block-128 with 128-row token tiles
   const bool b128 = q.fp8 && q.bm == 16;        // FP8 block-128 on the swapped-operand GEMMs
-  L.xq = take(fp8_tiles ? T * H : 0);
-  L.xq_scale = take(fp8_tiles ? T * (H / 128) * 4 : 0);
+  L.xq = take(q.fp8 ? T * H : 0);
+  L.xq_scale = take(q.fp8 ? T * (H / 128) * 4 : 0);
   // the swapped-operand GEMMs keep the activation in row-group order, 128-byte chunks (64
   // bf16 or 128 e4m3 columns)
   const size_t act_bytes = q.pt ? rows * I : rows * (q.bm == 16 ? align_up(I, 64) : I) * 2;
@@ -250,7 +250,7 @@ moe_status_t run_route(const Plan& pl, const float* logits, void* ws, const Laun
   // the route kernel also resets the device status word: it starts every forward
   return cuda_status(moe::launch_route(l, logits, pl.T, pl.Er, pl.topk, pl.Es, pl.renorm,
                                        ws_ptr<int>(ws, L.topk_ids), ws_ptr<float>(ws, L.topk_w),
-                                       ws_ptr<int>(ws, L.status), (pl.fp8 && pl.bm == 128) ? nullptr : hidden,
+                                       ws_ptr<int>(ws, L.status), pl.fp8 ? nullptr : hidden,
                                        pl.H * 2));
 }
 
@@ -284,6 +284,14 @@ GemmBuffers common_buffers(const Plan& pl, void* ws) {
   return b;
 }
 
+
+// The swapped-operand GEMMs (block_m 16) store y as fp16 [max_rows, H] followed by its
+// int8 exponents [max_rows, H/32] (y = y16 * 2^exp); the 128-row token-tile GEMMs store
+// fp32 [max_rows, H] (no exponents).
+int8_t* y_exp_ptr(const Plan& pl, void* ws) {
+  if (pl.bm != 16) return nullptr;
+  return ws_ptr<int8_t>(ws, pl.lay.y + static_cast<size_t>(pl.lay.max_rows) * pl.H * 2);
+}
 
 // Lower bound on the number of 128-row tiles align produces: every expert that receives
 // a pair gets at least one, and there are at least ceil(P / 128).
@@ -385,9 +393,10 @@ moe_status_t run_permute(const Plan& pl, const void* hidden, void* ws, const Lau
   if (pl.bm != 16) return MOE_OK;
   const auto& L = pl.lay;
   if (pl.fp8)
-    return cuda_status(moe::launch_permute_b128_rows(l, hidden, pl.H, ws_ptr<int>(ws, L.sorted_pair_ids),
-                                                     ws_ptr<int>(ws, L.num_blocks) + 1, ws_ptr<int2>(ws, L.group_info),
-                                                     static_cast<int>(pl.P), pl.kk, ws_ptr<void>(ws, L.xs), num_sms));
+    return cuda_status(moe::launch_permute_b128_rows(
+        l, ws_ptr<void>(ws, L.xq), ws_ptr<float>(ws, L.xq_scale), pl.H, ws_ptr<int>(ws, L.sorted_pair_ids),
+        ws_ptr<int>(ws, L.num_blocks) + 1, ws_ptr<int2>(ws, L.group_info), static_cast<int>(pl.P), pl.kk,
+        ws_ptr<void>(ws, L.xs), num_sms));
   if (pl.mx)
     return cuda_status(moe::launch_permute_mx_rows(
         l, hidden, pl.H, ws_ptr<int>(ws, L.sorted_pair_ids), ws_ptr<int>(ws, L.num_blocks) + 1,
@@ -419,6 +428,7 @@ moe_status_t run_gemm2(const Plan& pl_in, const void* w2, const float* w2_scale,
   s.num_sms = num_sms;
   GemmBuffers b = common_buffers(pl, ws);
   b.out = ws_ptr<void>(ws, L.y);
+  b.out_exp = y_exp_ptr(pl, ws);
   b.tile_counter = ws_ptr<int>(ws, L.status) + 6;
   CUtensorMap ta, tb;
   const uint64_t rows = static_cast<uint64_t>(L.max_rows);
@@ -466,8 +476,8 @@ moe_status_t run_gemm2(const Plan& pl_in, const void* w2, const float* w2_scale,
 }
 
 moe_status_t run_combine(const Plan& pl, void* out, void* ws, const Launch& l) {
-  return cuda_status(moe::launch_combine(l, ws_ptr<void>(ws, pl.lay.y), ws_ptr<int>(ws, pl.lay.pair_to_row), pl.T,
-                                         pl.kk, pl.H, out));
+  return cuda_status(moe::launch_combine(l, ws_ptr<void>(ws, pl.lay.y), y_exp_ptr(pl, ws),
+                                         ws_ptr<int>(ws, pl.lay.pair_to_row), pl.T, pl.kk, pl.H, out));
 }
 
 // Common preamble of the entry points that launch: plan, workspace, device.
@@ -491,7 +501,7 @@ Launch launch_of(const moe_problem_t* p, moe_stream_t stream) {
 moe_status_t forward_after_route(const Plan& pl, const Launch& l, const void* hidden, const void* w13, const void* w2,
                                  const float* s13, const float* s2, void* out, void* ws, int num_sms) {
   moe_status_t st = run_align(pl, ws, l);
-  if (st == MOE_OK && pl.fp8 && pl.bm == 128) st = run_quant_act(pl, hidden, ws, l);
+  if (st == MOE_OK && pl.fp8) st = run_quant_act(pl, hidden, ws, l);
   if (st == MOE_OK) st = run_permute(pl, hidden, ws, l, num_sms);
   if (st == MOE_OK) st = run_gemm1(pl, hidden, w13, s13, ws, l, num_sms);
   if (st == MOE_OK) st = run_gemm2(pl, w2, s2, ws, l, num_sms);
@@ -788,7 +798,7 @@ MOE_API moe_status_t moe_stage_quant_act(const moe_problem_t* problem, const voi
   if (st != MOE_OK || pl.T == 0) return st;  // T == 0: nothing to do, pointers unused
   if (!pl.fp8 || !aligned16(hidden)) return MOE_ERR_INVALID_ARG;
   st = prologue(problem, workspace, workspace_bytes, &pl, &sms);
-  if (st != MOE_OK || pl.T == 0 || pl.bm != 128) return st;  // block_m 16: quantised by the permute step
+  if (st != MOE_OK || pl.T == 0) return st;
   return run_quant_act(pl, hidden, workspace, launch_of(problem, stream));
 }
 

@@ -1,15 +1,20 @@
 // Step 5 of the layer: deterministic combine back to token order.
 //
-// out[t, h] = sum_{j=0}^{k'-1} y[pair_to_row[t*k' + j], h], where y (fp32, sorted row
-// order) already carries the routing weight (GEMM2 epilogue). The sum runs in slot order
+// out[t, h] = sum_{j=0}^{k'-1} y[pair_to_row[t*k' + j], h], where y (sorted row order)
+// already carries the routing weight (GEMM2 epilogue). The sum runs in slot order
 // j = 0, 1, ..., k'-1 in fp32 and is rounded once to bf16, so the result does not depend
-// on scheduling. The output is bf16
-// of the hidden shape ("FlashInfer TRTLLM-Gen MoE kernel optimisation: NemotronH
-// support", sglang PR 21321, section 1: the fused op returns a bf16 tensor shaped like
-// hidden_states).
+// on scheduling. The output is bf16 of the hidden shape ("FlashInfer TRTLLM-Gen MoE kernel
+// optimisation: NemotronH support", sglang PR 21321, section 1: the fused op returns a
+// bf16 tensor shaped like hidden_states).
 //
-// HBM-bound: each thread owns 8 consecutive columns of one token, reads k' x 32 bytes
-// and writes 16.
+// y comes in one of two formats: fp32 (the 128-row token-tile GEMMs), or fp16 with one
+// power-of-two exponent per 32 columns of a row (the swapped-operand GEMMs: y = y16 *
+// 2^exp, exact in fp32), which halves the bytes of this HBM-bound pass.
+//
+// Each thread owns 8 consecutive columns of one token and reads k' x 32 (fp32) or k' x 17
+// (fp16 + exponent) bytes, writing 16.
+#include <cuda_fp16.h>
+
 #include "moe_device.cuh"
 #include "moe_internal.h"
 
@@ -19,8 +24,8 @@ namespace {
 constexpr int kCombineThreads = 256;
 
 __global__ void __launch_bounds__(kCombineThreads)
-    combine_kernel(const float4* __restrict__ y, const int* __restrict__ pair_to_row, int T, int k_total, int H8,
-                   uint4* __restrict__ out) {
+    combine_f32_kernel(const float4* __restrict__ y, const int* __restrict__ pair_to_row, int T, int k_total, int H8,
+                       uint4* __restrict__ out) {
   griddep_wait();
   griddep_launch_dependents();
   const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -47,17 +52,57 @@ __global__ void __launch_bounds__(kCombineThreads)
   out[idx] = o;
 }
 
+__global__ void __launch_bounds__(kCombineThreads)
+    combine_f16_kernel(const uint4* __restrict__ y, const int8_t* __restrict__ y_exp, const int* __restrict__ pair_to_row,
+                       int T, int k_total, int H8, uint4* __restrict__ out) {
+  griddep_wait();
+  griddep_launch_dependents();
+  const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= static_cast<long long>(T) * H8) return;
+  const long long t = idx / H8;
+  const int c = static_cast<int>(idx - t * H8);
+  float acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+  const int* rows = pair_to_row + t * k_total;
+  const int H32 = H8 >> 2;  // exponents per row
+  for (int j = 0; j < k_total; ++j) {
+    const long long r = __ldg(rows + j);
+    const uint4 v = __ldcs(y + r * H8 + c);  // columns 8c..8c+7, read once: streaming
+    const int s = __ldg(y_exp + r * H32 + (c >> 2));
+    const float scale = __int_as_float((127 + s) << 23);  // 2^s, s in [-100, 113]
+    const __half2* h = reinterpret_cast<const __half2*>(&v);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __half22float2(h[i]);
+      acc[2 * i] += f.x * scale;
+      acc[2 * i + 1] += f.y * scale;
+    }
+  }
+  uint4 o;
+  o.x = pack_bf16x2(acc[0], acc[1]);
+  o.y = pack_bf16x2(acc[2], acc[3]);
+  o.z = pack_bf16x2(acc[4], acc[5]);
+  o.w = pack_bf16x2(acc[6], acc[7]);
+  out[idx] = o;
+}
+
 }  // namespace
 
-cudaError_t launch_combine(const Launch& l, const void* y, const int* pair_to_row, int T, int k_total, int H,
-                           void* out) {
+cudaError_t launch_combine(const Launch& l, const void* y, const int8_t* y_exp, const int* pair_to_row, int T,
+                           int k_total, int H, void* out) {
   const int H8 = H / 8;
   const long long n = static_cast<long long>(T) * H8;
   cudaLaunchConfig_t cfg;
   cudaLaunchAttribute attr[1];
   make_launch_config(&cfg, attr, l, dim3(static_cast<unsigned>((n + kCombineThreads - 1) / kCombineThreads)),
                      dim3(kCombineThreads), 0);
-  return cudaLaunchKernelEx(&cfg, combine_kernel, static_cast<const float4*>(y), pair_to_row, T, k_total, H8,
+  if (y_exp != nullptr) {
+    if (H % 32 != 0) return cudaErrorInvalidValue;
+    return cudaLaunchKernelEx(&cfg, combine_f16_kernel, static_cast<const uint4*>(y), y_exp, pair_to_row, T, k_total,
+                              H8, static_cast<uint4*>(out));
+  }
+  return cudaLaunchKernelEx(&cfg, combine_f32_kernel, static_cast<const float4*>(y), pair_to_row, T, k_total, H8,
                             static_cast<uint4*>(out));
 }
 

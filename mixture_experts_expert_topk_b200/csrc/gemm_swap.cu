@@ -59,10 +59,12 @@
 // acc[j] += partial[j] * s_w(row block, chunk) * s_x(token j, chunk). A 128-row weight tile
 // is exactly one scale block row (gated: its even lanes are gate rows, its odd lanes up
 // rows, two block rows of the checkpoint layout), so s_w is one value per lane per chunk;
-// s_x varies along N, so each K step of X carries, right behind its codes, the fp32 scales
-// of its rows (chunk-major), which the epilogue reads from shared memory as broadcasts.
-// The epilogue, not the MMA, then releases the step's ring space. Row groups have at most
-// 128 rows (kB128GroupRows) so the accumulator fits the epilogue threads' registers.
+// s_x varies along N: each K step of X stores, right behind its codes, the fp32 scales of
+// its rows (chunk-major), and the X producer copies them into a small ring of their own
+// (8 slots of 1 KB) that the epilogue reads as shared-memory broadcasts and frees after
+// the step's last chunk; the operand ring is released by the MMAs as in the other kinds.
+// Row groups have at most 128 rows (kB128GroupRows) so the accumulator fits the epilogue
+// threads' registers.
 // GEMM1 writes the bf16 activation, which a separate pass quantises per 1x128 for GEMM2.
 //
 // One persistent CTA per SM, 7 warps:
@@ -71,6 +73,7 @@
 //   warp 6      X copies;
 //   warp 1      TMEM allocator and MMA issuer;
 //   warps 2-5   epilogue (TMEM lane quadrant = warp % 4).
+#include <cuda_fp16.h>
 #include <cuda_fp8.h>
 
 #include "moe_device.cuh"
@@ -107,17 +110,25 @@ static_assert(kPartBufs * kPartCols <= static_cast<int>(kTmemCols), "TMEM column
 // chunks); a step that would cross the end of the ring starts again at its beginning.
 // Offsets stay multiples of 1024 bytes, the period of the 128-byte swizzle.
 constexpr int kRingBytes = 225 * 1024;
+// FP8 block-128: a shorter operand ring, then kSxSlots slots of the X scale ring
+constexpr int kSxSlots = 8;
+constexpr int kSxSlotBytes = 1024;  // a step's scales: kcs * n * 4 <= 4 * 32 * 4 = 3 * 64 * 4 < 2 * 128 * 4 + 1
+constexpr int kRingBytesB128 = kRingBytes - kSxSlots * kSxSlotBytes - 1024;
+static_assert(4 * 32 * 4 <= kSxSlotBytes && 3 * 64 * 4 <= kSxSlotBytes && 2 * kB128GroupRows * 4 <= kSxSlotBytes,
+              "a step's X scales fit a slot");
+template <int kKind>
+__host__ __device__ constexpr int ring_bytes() { return kKind == 3 ? kRingBytesB128 : kRingBytes; }
 constexpr int kSlots = 16;  // barrier pairs: at most this many K steps in flight
 constexpr int kBarOff = kRingBytes;
 constexpr int kBarBytes = 1024;  // barriers, step ends, tile ring, TMEM address, abort flag
-static_assert((3 * kSlots + 4 + 2 * kTileRing + 1 + 2 * 4) * 8 + 2 * kSlots * 8 + 16 * kTileRing + 8 <= kBarBytes,
+static_assert((3 * kSlots + 4 + 2 * kTileRing + 1 + 2 * 4 + 8) * 8 + 2 * kSlots * 8 + 16 * kTileRing + 8 <= kBarBytes,
               "barrier region");
 constexpr int kSmemBytes = kBarOff + kBarBytes + 1024;
 static_assert(kSmemBytes <= kSmemCap, "shared memory");
 
 enum : int {
   kSiteEmpty = 1, kSiteFull = 2, kSiteTmemEmpty = 3, kSiteTmemFull = 4, kSiteTileFull = 5, kSiteTileEmpty = 6,
-  kSiteEmptyX = 7, kSiteSfFree = 8, kSiteFullX = 9, kSitePartEmpty = 10, kSitePartFull = 11
+  kSiteEmptyX = 7, kSiteSfFree = 8, kSiteFullX = 9, kSitePartEmpty = 10, kSitePartFull = 11, kSiteSxFree = 12
 };
 
 struct Args {
@@ -145,16 +156,15 @@ struct Args {
   // GEMM1 tiles take the gate block row mt / 2 and the up block row up_block + mt / 2
   int ws_rows;             // 128-row scale blocks per expert
   int up_block;            // gated GEMM1: I / 128; 0 otherwise
+  int8_t* y_exp;           // GEMM2: the power-of-two exponent of each 32 columns of y
 };
 
 // Ring bytes of one K step of kcs chunks for a group of n rows. MXFP8 steps add the scale
-// blocks of W and X, FP8 block-128 steps the fp32 scales of the X rows (4 bytes per row
-// per chunk); both round up to the 1024-byte period of the swizzle.
+// blocks of W and X and round up to the 1024-byte period of the swizzle.
 template <int kKind>
 __device__ __forceinline__ uint32_t step_bytes(int kcs, int n) {
   const uint32_t b = static_cast<uint32_t>(kcs) * (kTileW + n * kChunkBytes);
   if (kKind == 2) return (b + static_cast<uint32_t>(kcs) * (kSfW + kSfX) + 1023u) & ~1023u;
-  if (kKind == 3) return (b + static_cast<uint32_t>(kcs * n) * 4u + 1023u) & ~1023u;
   return b;
 }
 static_assert(4 * (kTileW + 32 * kChunkBytes + kSfW + kSfX) <= kRingBytes / 2 &&
@@ -163,15 +173,16 @@ static_assert(4 * (kTileW + 32 * kChunkBytes + kSfW + kSfX) <= kRingBytes / 2 &&
 static_assert(4 * (kTileW + 32 * kChunkBytes) <= kRingBytes / 2 && 2 * (kTileW + 128 * kChunkBytes) <= kRingBytes / 2 &&
                   kTileW + kNMax * kChunkBytes <= kRingBytes / 2,
               "at least two steps fit the ring");
-static_assert(4 * (kTileW + 32 * (kChunkBytes + 4)) + 1024 <= kRingBytes / 2 &&
-                  2 * (kTileW + kB128GroupRows * (kChunkBytes + 4)) + 1024 <= kRingBytes / 2,
+static_assert(4 * (kTileW + 32 * kChunkBytes) <= kRingBytesB128 / 2 &&
+                  2 * (kTileW + kB128GroupRows * kChunkBytes) <= kRingBytesB128 / 2,
               "at least two FP8 block-128 steps fit the ring");
 
 // Byte offset in the ring of the next step of `bytes`. pos: offset of the next free byte;
 // head: running count of the bytes used, skipped ring tails included.
+template <int kBytes>
 __device__ __forceinline__ uint32_t ring_alloc(uint32_t& pos, uint64_t& head, uint32_t bytes) {
-  if (pos + bytes > static_cast<uint32_t>(kRingBytes)) {
-    head += kRingBytes - pos;
+  if (pos + bytes > static_cast<uint32_t>(kBytes)) {
+    head += kBytes - pos;
     pos = 0;
   }
   const uint32_t off = pos;
@@ -183,10 +194,11 @@ __device__ __forceinline__ uint32_t ring_alloc(uint32_t& pos, uint64_t& head, ui
 // Waits, oldest step first, until the step just allocated (its end is `head`, its index
 // ks) fits the ring and has a free slot. Each producer keeps its own copy of this state;
 // both allocate the same sequence of steps.
+template <int kBytes>
 __device__ __forceinline__ bool ring_reserve(uint64_t head, uint64_t& freed, uint32_t ks, uint32_t& oldest,
                                              uint64_t* step_end, uint32_t empty0, volatile int* abort, int* status,
                                              int site) {
-  while (head - freed > static_cast<uint64_t>(kRingBytes) || ks - oldest >= static_cast<uint32_t>(kSlots)) {
+  while (head - freed > static_cast<uint64_t>(kBytes) || ks - oldest >= static_cast<uint32_t>(kSlots)) {
     if (!mbar_wait(empty0 + 8 * (oldest % kSlots), (oldest / kSlots) & 1u, abort, status, site)) return false;
     freed = step_end[oldest % kSlots];
     ++oldest;
@@ -242,7 +254,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
   const uint32_t fullx0 = drain_bar + 8;                                      // [kSlots]
   const uint32_t pfull0 = fullx0 + 8 * kSlots;                                // [kPartBufs]
   const uint32_t pempty0 = pfull0 + 8 * kPartBufs;                            // [kPartBufs]
-  uint64_t* step_end_w = bars + 3 * kSlots + 4 + 2 * kTileRing + 1 + 2 * kPartBufs;  // [kSlots]
+  const uint32_t sxfree0 = pempty0 + 8 * kPartBufs;                           // [kSxSlots]
+  const uint32_t sx0 = s0 + kRingBytesB128;                                   // FP8 block-128 X scale ring
+  uint64_t* step_end_w = bars + 3 * kSlots + 4 + 2 * kTileRing + 1 + 2 * kPartBufs + kSxSlots;  // [kSlots]
   uint64_t* step_end_x = step_end_w + kSlots;                                 // [kSlots]
   volatile int* ring = reinterpret_cast<volatile int*>(step_end_x + kSlots);  // [kTileRing][4]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(const_cast<int*>(ring) + 4 * kTileRing);
@@ -255,14 +269,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
     for (int s = 0; s < kSlots; ++s) {
       mbar_init(full0 + 8 * s, 1);   // the W copies of a step
       mbar_init(fullx0 + 8 * s, 1);  // the X copies of a step
-      // released by the MMAs' commit; FP8 block-128: by the four epilogue warps, which
-      // read the step's X scales after its MMAs
-      mbar_init(empty0 + 8 * s, kB128 ? 4 : 1);
+      mbar_init(empty0 + 8 * s, 1);  // released by the MMAs' commit
     }
     for (int b = 0; b < kPartBufs; ++b) {
       mbar_init(pfull0 + 8 * b, 1);
       mbar_init(pempty0 + 8 * b, 128);
     }
+    for (int b = 0; b < kSxSlots; ++b) mbar_init(sxfree0 + 8 * b, 4);  // the four epilogue warps
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull0 + 8 * b, 1);
       mbar_init(tempty0 + 8 * b, 128);
@@ -327,8 +340,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
         const uint8_t* wsrc = a.w + (static_cast<size_t>(e) * a.m_tiles + mt) * a.k_chunks * kTileW;
         for (int c0 = 0; c0 < a.k_chunks; c0 += kc, ++ks) {
           const int kcs = min(kc, a.k_chunks - c0);
-          const uint32_t off = ring_alloc(pos, head, step_bytes<kKind>(kcs, n));
-          if (!ring_reserve(head, freed, ks, oldest, step_end_w, empty0, abort_flag, a.status, kSiteEmpty)) {
+          const uint32_t off = ring_alloc<ring_bytes<kKind>()>(pos, head, step_bytes<kKind>(kcs, n));
+          if (!ring_reserve<ring_bytes<kKind>()>(head, freed, ks, oldest, step_end_w, empty0, abort_flag, a.status, kSiteEmpty)) {
             ok = false;
             break;
           }
@@ -362,18 +375,25 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
         const uint8_t* xsrc = a.x + static_cast<size_t>(x_row) * x_row_bytes;
         for (int c0 = 0; c0 < a.k_chunks; c0 += kc, ++ks) {
           const int kcs = min(kc, a.k_chunks - c0);
-          const uint32_t off = ring_alloc(pos, head, step_bytes<kKind>(kcs, n));
-          if (!ring_reserve(head, freed, ks, oldest, step_end_x, empty0, abort_flag, a.status, kSiteEmptyX)) {
+          const uint32_t off = ring_alloc<ring_bytes<kKind>()>(pos, head, step_bytes<kKind>(kcs, n));
+          if (!ring_reserve<ring_bytes<kKind>()>(head, freed, ks, oldest, step_end_x, empty0, abort_flag, a.status, kSiteEmptyX)) {
             ok = false;
             break;
           }
           const uint32_t full = fullx0 + 8 * (ks % kSlots);
-          // FP8 block-128: the step's codes and then its rows' scales, contiguous in X
-          const uint32_t bytes = static_cast<uint32_t>(kcs * n) * (kB128 ? kB128RowBytesPerChunk : kChunkBytes);
-          const uint32_t sf_bytes = kMx ? static_cast<uint32_t>(kcs) * kSfX : 0u;
+          const uint32_t bytes = static_cast<uint32_t>(kcs * n) * kChunkBytes;
+          // MXFP8: the scale blocks; FP8 block-128: the rows' scales, stored right behind
+          // the step's codes, into a slot of the X scale ring once the epilogue freed it
+          const uint32_t sf_bytes = kMx ? static_cast<uint32_t>(kcs) * kSfX : (kB128 ? static_cast<uint32_t>(kcs * n) * 4u : 0u);
+          if (kB128 && !mbar_wait(sxfree0 + 8 * (ks % kSxSlots), ((ks / kSxSlots) & 1u) ^ 1u, abort_flag, a.status,
+                                  kSiteSxFree)) {
+            ok = false;
+            break;
+          }
           mbar_arrive_expect_tx(full, bytes + sf_bytes);
-          bulk_load(s0 + off + kcs * kTileW, xsrc + static_cast<size_t>(c0) * n * (kB128 ? kB128RowBytesPerChunk : kChunkBytes),
-                    bytes, full, pol);
+          const uint8_t* step_src = xsrc + static_cast<size_t>(c0) * n * (kB128 ? kB128RowBytesPerChunk : kChunkBytes);
+          bulk_load(s0 + off + kcs * kTileW, step_src, bytes, full, pol);
+          if constexpr (kB128) bulk_load(sx0 + (ks % kSxSlots) * kSxSlotBytes, step_src + bytes, sf_bytes, full, pol);
           if constexpr (kMx)
             bulk_load(s0 + off + static_cast<uint32_t>(kcs) * (kTileW + n * kChunkBytes + kSfW),
                       a.x_sf + (static_cast<size_t>(x_row >> 4) * a.k_chunks + c0) * kSfX, sf_bytes, full, pol);
@@ -400,7 +420,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
         bool ok = true;
         for (int c0 = 0; c0 < a.k_chunks; c0 += kc, ++ks) {
           const int kcs = min(kc, a.k_chunks - c0);
-          const uint32_t base = s0 + ring_alloc(pos, head, step_bytes<kKind>(kcs, n));
+          const uint32_t base = s0 + ring_alloc<ring_bytes<kKind>()>(pos, head, step_bytes<kKind>(kcs, n));
           if (!mbar_wait(full0 + 8 * (ks % kSlots), (ks / kSlots) & 1u, abort_flag, a.status, kSiteFull) ||
               !mbar_wait(fullx0 + 8 * (ks % kSlots), (ks / kSlots) & 1u, abort_flag, a.status, kSiteFullX)) {
             ok = false;
@@ -449,7 +469,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
               umma_commit(pfull0 + 8 * pb);
             }
             if (!ok) break;
-            continue;  // the epilogue releases the step's ring space
           } else if (kFp8) {
             umma_e4m3_chunk(d_tmem, a_lo, b_lo, idesc, c0 != 0);
 #pragma unroll
@@ -481,8 +500,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
     const bool odd = (lane & 1) != 0;
     int rslot = 0, it = 0;
     uint32_t rph = 0;
-    uint32_t ks = 0, pos = 0, pc = 0;  // FP8 block-128: the ring allocation replayed, partials consumed
-    uint64_t head = 0;
+    uint32_t ks = 0, pc = 0;  // FP8 block-128: K steps and partials consumed
     while (true) {
       int4 t = make_int4(0, 0, 0, 0);
       int ok = 0;
@@ -523,13 +541,21 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
         for (int b = 1; b < kNMax / 32; ++b)
           if (c0 == 32 * b) wl = wreg[b];
         if (a.mode != 0) {
+          // y = acc * routing weight, stored as fp16 scaled by a power of two per 32 columns
+          // (this warp's columns of one token row): 2^-s brings the block's largest
+          // magnitude into [2^14, 2^15), so no value overflows fp16 and each keeps 11
+          // significant bits; s (at least -100) goes to y_exp.
           const int col = mt * kMW + q * 32 + lane;
-          float* y = static_cast<float*>(a.out) + static_cast<size_t>(x_row + c0) * a.out_cols + col;
+          __half* y = static_cast<__half*>(a.out) + static_cast<size_t>(x_row + c0) * a.out_cols + col;
+          int8_t* ye = a.y_exp + static_cast<size_t>(x_row + c0) * (a.out_cols >> 5) + (col >> 5);
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             if (j == 16 && !full) break;
-            const float w = __shfl_sync(0xffffffffu, wl, j) * dq;
-            y[static_cast<size_t>(j) * a.out_cols] = __uint_as_float(v[j]) * w;
+            const float val = __uint_as_float(v[j]) * (__shfl_sync(0xffffffffu, wl, j) * dq);
+            const uint32_t amax = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(val)));
+            const int s = amax == 0u ? 0 : max(static_cast<int>(amax >> 23) - 127 - 14, -100);
+            y[static_cast<size_t>(j) * a.out_cols] = __float2half_rn(val * __int_as_float((127 - s) << 23));
+            if (lane == 0) ye[static_cast<size_t>(j) * (a.out_cols >> 5)] = static_cast<int8_t>(s);
           }
         } else if (!gated) {
 #pragma unroll
@@ -583,9 +609,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
         bool good = true;
         for (int c0 = 0; c0 < a.k_chunks && good; c0 += kc, ++ks) {
           const int kcs = min(kc, a.k_chunks - c0);
-          // the X scales of this step: [chunk][row] fp32 right behind its codes
-          const uint32_t sf = s0 + ring_alloc(pos, head, step_bytes<kKind>(kcs, n)) +
-                              static_cast<uint32_t>(kcs) * (kTileW + n * kChunkBytes);
+          // the X scales of this step, [chunk][row] fp32, in its slot of the X scale ring (the
+          // full barrier the partials' MMAs waited on also covered this copy)
+          const uint32_t sf = sx0 + (ks % kSxSlots) * kSxSlotBytes;
           for (int c = 0; c < kcs; ++c, ++pc) {
             const uint32_t pb = pc % kPartBufs;
             const bool got = mbar_wait(pfull0 + 8 * pb, (pc / kPartBufs) & 1u, abort_flag, a.status, kSitePartFull);
@@ -633,7 +659,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
           }
           if (!good) break;
           __syncwarp();  // every lane has read the step's scales
-          if (lane == 0) mbar_arrive(empty0 + 8 * (ks % kSlots));
+          if (lane == 0) mbar_arrive(sxfree0 + 8 * (ks % kSxSlots));
         }
         if (!__all_sync(0xffffffffu, good)) break;
 #pragma unroll
@@ -745,6 +771,8 @@ cudaError_t launch_gemm_swap(const Launch& l, int mode, const SwapOperands& o, c
   a.x_sf = static_cast<const uint8_t*>(o.x_sf);
   a.ws_rows = s.N / 128;
   a.up_block = o.up_block;
+  a.y_exp = b.out_exp;
+  if (mode == 1 && (a.y_exp == nullptr || s.out_cols % 32 != 0)) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg;
   cudaLaunchAttribute attr[1];
   make_launch_config(&cfg, attr, l, dim3(s.num_sms), dim3(kThreads), kSmemBytes);

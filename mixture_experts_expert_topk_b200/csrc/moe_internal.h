@@ -54,13 +54,12 @@ cudaError_t launch_permute_rows(const Launch& l, const void* hidden, int H, cons
 cudaError_t launch_permute_quant_rows(const Launch& l, const void* hidden, int H, const int* sorted_pair_ids,
                                       const int* num_groups, const int2* group_info, int P, int k_total,
                                       float input_scale, void* xs, int num_sms);
-// FP8 block-128: the token rows of every row group quantised per 1x128 group (scale =
-// amax / 448, 1 for an all-zero group; code = e4m3(x / scale), IEEE fp32 divisions, round to
-// nearest even, saturating), in the X layout above with KC = H / 128. Padding rows are zero
-// codes with scale 1.
-cudaError_t launch_permute_b128_rows(const Launch& l, const void* hidden, int H, const int* sorted_pair_ids,
-                                     const int* num_groups, const int2* group_info, int P, int k_total, void* xs,
-                                     int num_sms);
+// FP8 block-128: the token rows of every row group, quantised per 1x128 group once per token
+// by launch_quant_act (xq e4m3 [T, H], xq_scale fp32 [T, H/128]), copied into the X layout
+// above with KC = H / 128. Padding rows are zero codes with scale 1.
+cudaError_t launch_permute_b128_rows(const Launch& l, const void* xq, const float* xq_scale, int H,
+                                     const int* sorted_pair_ids, const int* num_groups, const int2* group_info, int P,
+                                     int k_total, void* xs, int num_sms);
 // FP8 block-128: GEMM1's bf16 activation (row-group order, 64-column chunks) quantised per
 // 1x128 group the same way into the X layout above with KC = I / 128, for GEMM2.
 cudaError_t launch_act_quant_b128(const Launch& l, const void* act, int I, const int* num_groups,
@@ -95,6 +94,9 @@ struct GemmBuffers {
   int* status;
   const int* num_groups;    // row groups (gemm_swap)
   const int2* group_info;
+  // GEMM2 of the swapped-operand GEMMs: y as fp16 [rows, H] (out) with one power-of-two
+  // exponent per 32 columns of each row here, int8 [rows, H/32]: y = y16 * 2^exp
+  int8_t* out_exp;
 };
 // Operands of the swapped-operand GEMM: tiled weights, X in row-group order, and (GEMM1)
 // the number of 64-column chunks of the activation it writes in row-group order.
@@ -192,8 +194,9 @@ cudaError_t launch_ep_combine(const Launch& l, const void* returned, const int* 
                               void* out);
 
 // ---- elementwise (combine.cu, quant.cu, prepare.cu) ----
-cudaError_t launch_combine(const Launch& l, const void* y, const int* pair_to_row, int T, int k_total, int H,
-                           void* out);
+// y: fp32 [rows, H] (y_exp == nullptr), or fp16 [rows, H] scaled by 2^y_exp[row][col / 32].
+cudaError_t launch_combine(const Launch& l, const void* y, const int8_t* y_exp, const int* pair_to_row, int T,
+                           int k_total, int H, void* out);
 cudaError_t launch_quant_act(const Launch& l, const void* x, int T, int H, void* q, float* scale);
 // As launch_quant_act over the first num_blocks[0] * block_m of max_rows rows.
 cudaError_t launch_quant_rows(const Launch& l, const void* x, int max_rows, int cols, const int* num_blocks,

@@ -288,49 +288,59 @@ __device__ __forceinline__ uint32_t quant_group_1x128(float x0, float x1, float 
   return lo | (hi << 16);
 }
 
-// FP8 block-128: a warp quantises one row of a group, lane l taking columns 4l..4l+3 of
-// every 128-column chunk (all of the row's loads issued first).
-constexpr int kB128MaxChunks = 32;  // H <= 4096
+// FP8 block-128: the token rows, already quantised once per token (quant_act_kernel: e4m3
+// codes [T, H] and fp32 1x128 scales [T, H/128]), copied into the X layout of their row
+// groups. A warp copies one row: lane l moves 16-byte pieces l, l + 32, ... of the row's
+// codes (all loads first) and lanes 0..KC-1 its scales. Padding rows get zero codes and
+// scale 1 (an all-zero group).
+constexpr int kB128Pieces = 4;  // 16-byte pieces per lane per pass (a 2 KB row in one pass)
 __global__ void __launch_bounds__(kThreads)
-    permute_b128_rows_kernel(const uint2* __restrict__ hidden, int H, const int* __restrict__ sorted_pair_ids,
-                             const int* __restrict__ num_groups, const int2* __restrict__ group_info, int P,
-                             int k_total, uint8_t* __restrict__ xs) {
+    permute_b128_rows_kernel(const uint4* __restrict__ xq, const float* __restrict__ xq_scale, int H,
+                             const int* __restrict__ sorted_pair_ids, const int* __restrict__ num_groups,
+                             const int2* __restrict__ group_info, int P, int k_total, uint8_t* __restrict__ xs) {
   griddep_wait();
   griddep_launch_dependents();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int G = *num_groups;
-  const int KC = H / 128;
+  const int KC = H / 128, pieces = H / 16;
   for (int g = blockIdx.x; g < G; g += gridDim.x) {
     const int2 gi = group_info[g];
     const int x_row = gi.x, n = gi.y >> 16;
     uint8_t* base = xs + static_cast<size_t>(x_row) * KC * kB128RowBytesPerChunk;
     for (int j = blockIdx.y * (kThreads / 32) + warp; j < n; j += gridDim.y * (kThreads / 32)) {
       const int pid = sorted_pair_ids[x_row + j];
-      const uint2* src = pid < P ? hidden + static_cast<size_t>(pid / k_total) * (H / 4) : nullptr;
-      uint2 in[kB128MaxChunks];
+      const long long tok = pid < P ? pid / k_total : -1;
+      for (int p0 = 0; p0 < pieces; p0 += 32 * kB128Pieces) {
+        uint4 v[kB128Pieces];
 #pragma unroll
-      for (int c = 0; c < kB128MaxChunks; ++c)
-        in[c] = (c < KC && src != nullptr) ? __ldg(src + c * 32 + lane) : make_uint2(0u, 0u);
+        for (int i = 0; i < kB128Pieces; ++i) {
+          const int p = p0 + lane + 32 * i;
+          v[i] = (tok >= 0 && p < pieces) ? __ldg(xq + tok * pieces + p) : make_uint4(0u, 0u, 0u, 0u);
+        }
 #pragma unroll
-      for (int c = 0; c < kB128MaxChunks; ++c) {
-        if (c >= KC) break;
-        const float2 f01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&in[c].x));
-        const float2 f23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&in[c].y));
-        float sc;
-        const uint32_t codes = quant_group_1x128(f01.x, f01.y, f23.x, f23.y, sc);
+        for (int i = 0; i < kB128Pieces; ++i) {
+          const int p = p0 + lane + 32 * i;
+          if (p < pieces) {
+            size_t co, so;
+            b128_offsets(n, KC, p >> 3, j, co, so);
+            *reinterpret_cast<uint4*>(base + co + ((((p & 7) ^ j) & 7) << 4)) = v[i];
+          }
+        }
+      }
+      for (int c = lane; c < KC; c += 32) {
         size_t co, so;
         b128_offsets(n, KC, c, j, co, so);
-        const int ob = 4 * lane;
-        *reinterpret_cast<uint32_t*>(base + co + ((((ob >> 4) ^ j) & 7) << 4) + (ob & 15)) = codes;
-        if (lane == 0) *reinterpret_cast<float*>(base + so) = sc;
+        *reinterpret_cast<float*>(base + so) = tok >= 0 ? __ldg(xq_scale + tok * KC + c) : 1.0f;
       }
     }
   }
 }
 
 // FP8 block-128: GEMM1's bf16 activation (64-column chunks of 128-byte rows, row-group
-// order) quantised per 1x128 group into the X layout; a warp takes one row, lane l columns
-// 4l..4l+3 of each 128-column chunk (8 bytes of bf16 chunk 2c + l / 16).
+// order) quantised per 1x128 group into the X layout; a warp takes one row, four chunks at
+// a time (their loads first), lane l columns 4l..4l+3 of each 128-column chunk (8 bytes of
+// bf16 chunk 2c + l / 16).
+constexpr int kActChunksPerPass = 4;
 __global__ void __launch_bounds__(kThreads)
     act_quant_b128_kernel(const uint8_t* __restrict__ act, int I, const int* __restrict__ num_groups,
                           const int2* __restrict__ group_info, uint8_t* __restrict__ actq) {
@@ -346,24 +356,29 @@ __global__ void __launch_bounds__(kThreads)
     uint8_t* base = actq + static_cast<size_t>(x_row) * KC * kB128RowBytesPerChunk;
     for (int j = blockIdx.y * (kThreads / 32) + warp; j < n; j += gridDim.y * (kThreads / 32)) {
       const int ib = 8 * (lane & 15);  // byte of the bf16 chunk row
-      uint2 raw[kB128MaxChunks];
+      for (int c0 = 0; c0 < KC; c0 += kActChunksPerPass) {
+        uint2 raw[kActChunksPerPass];
 #pragma unroll
-      for (int c = 0; c < kB128MaxChunks; ++c)
-        raw[c] = c < KC ? *reinterpret_cast<const uint2*>(in + static_cast<size_t>(2 * c + (lane >> 4)) * n * 128 +
+        for (int i = 0; i < kActChunksPerPass; ++i) {
+          const int c = c0 + i;
+          raw[i] = c < KC ? *reinterpret_cast<const uint2*>(in + static_cast<size_t>(2 * c + (lane >> 4)) * n * 128 +
                                                             j * 128 + ((((ib >> 4) ^ j) & 7) << 4) + (ib & 15))
-                        : make_uint2(0u, 0u);
+                          : make_uint2(0u, 0u);
+        }
 #pragma unroll
-      for (int c = 0; c < kB128MaxChunks; ++c) {
-        if (c >= KC) break;
-        const float2 f01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw[c].x));
-        const float2 f23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw[c].y));
-        float sc;
-        const uint32_t codes = quant_group_1x128(f01.x, f01.y, f23.x, f23.y, sc);
-        size_t co, so;
-        b128_offsets(n, KC, c, j, co, so);
-        const int ob = 4 * lane;
-        *reinterpret_cast<uint32_t*>(base + co + ((((ob >> 4) ^ j) & 7) << 4) + (ob & 15)) = codes;
-        if (lane == 0) *reinterpret_cast<float*>(base + so) = sc;
+        for (int i = 0; i < kActChunksPerPass; ++i) {
+          const int c = c0 + i;
+          if (c >= KC) break;  // warp-uniform
+          const float2 f01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw[i].x));
+          const float2 f23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw[i].y));
+          float sc;
+          const uint32_t codes = quant_group_1x128(f01.x, f01.y, f23.x, f23.y, sc);
+          size_t co, so;
+          b128_offsets(n, KC, c, j, co, so);
+          const int ob = 4 * lane;
+          *reinterpret_cast<uint32_t*>(base + co + ((((ob >> 4) ^ j) & 7) << 4) + (ob & 15)) = codes;
+          if (lane == 0) *reinterpret_cast<float*>(base + so) = sc;
+        }
       }
     }
   }
@@ -371,20 +386,20 @@ __global__ void __launch_bounds__(kThreads)
 
 }  // namespace
 
-cudaError_t launch_permute_b128_rows(const Launch& l, const void* hidden, int H, const int* sorted_pair_ids,
-                                     const int* num_groups, const int2* group_info, int P, int k_total, void* xs,
-                                     int num_sms) {
-  if (H % 128 != 0 || H / 128 > kB128MaxChunks) return cudaErrorInvalidValue;
+cudaError_t launch_permute_b128_rows(const Launch& l, const void* xq, const float* xq_scale, int H,
+                                     const int* sorted_pair_ids, const int* num_groups, const int2* group_info, int P,
+                                     int k_total, void* xs, int num_sms) {
+  if (H % 128 != 0) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg;
   cudaLaunchAttribute attr[1];
   make_launch_config(&cfg, attr, l, dim3(2 * num_sms, kB128GroupRows / (kThreads / 32)), dim3(kThreads), 0);
-  return cudaLaunchKernelEx(&cfg, permute_b128_rows_kernel, static_cast<const uint2*>(hidden), H, sorted_pair_ids,
-                            num_groups, group_info, P, k_total, static_cast<uint8_t*>(xs));
+  return cudaLaunchKernelEx(&cfg, permute_b128_rows_kernel, static_cast<const uint4*>(xq), xq_scale, H,
+                            sorted_pair_ids, num_groups, group_info, P, k_total, static_cast<uint8_t*>(xs));
 }
 
 cudaError_t launch_act_quant_b128(const Launch& l, const void* act, int I, const int* num_groups,
                                   const int2* group_info, void* actq, int num_sms) {
-  if (I % 128 != 0 || I / 128 > kB128MaxChunks) return cudaErrorInvalidValue;
+  if (I % 128 != 0) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg;
   cudaLaunchAttribute attr[1];
   make_launch_config(&cfg, attr, l, dim3(2 * num_sms, kB128GroupRows / (kThreads / 32)), dim3(kThreads), 0);

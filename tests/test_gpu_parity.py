@@ -349,6 +349,8 @@ def _check_b128_operands(cfg, parts, a, hidden_bits):
     pids = a["sorted_pair_ids"][:P_pad]
     real = pids < P
     qx, sx = O.quant_groups_1x128(O.bf16_bits_to_f32(hidden_bits))
+    np.testing.assert_array_equal(parts["xq"], qx)          # once per token
+    np.testing.assert_array_equal(parts["xq_scale"], sx)
     xs_c, xs_s = untile_b128(parts["xs"], gi, ng, P_pad, cfg.H // 128)
     np.testing.assert_array_equal(xs_c[real], qx[pids[real] // kk])
     np.testing.assert_array_equal(xs_s[real], sx[pids[real] // kk])
