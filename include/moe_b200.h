@@ -152,9 +152,11 @@ typedef struct {
                              layout of xs (block_m 16); MXFP8: e4m3 codes in row-group order */
   size_t act_scale;       /* FP8 block-128, block_m 128: fp32 [max_rows, I/128]; MXFP8: E8M0
                              scale blocks */
-  size_t y;               /* weighted GEMM2 rows in sorted order: block_m 128: fp32 [max_rows,
-                             H]; block_m 16: fp16 [max_rows, H] followed by int8 [max_rows,
-                             H/32], row r's columns [32b, 32b+32) scaled by 2^(int8 [r, b]) */
+  size_t y;               /* GEMM2 rows in sorted order: block_m 128: fp32 [max_rows, H], times
+                             the routing weight; block_m 16: fp16 [max_rows, H] followed by
+                             int8 [max_rows, H/32], row r's columns [32b, 32b+32) scaled by
+                             2^(int8 [r, b]), without the routing weight (the combine applies
+                             it) */
   size_t xs;              /* block_m 16: the hidden rows of every row group in row-group order
                              (bf16; e4m3 codes for the 8-bit formats; FP8 block-128: each K
                              step's e4m3 codes followed by its rows' fp32 1x128 scales, 132

@@ -285,9 +285,9 @@ GemmBuffers common_buffers(const Plan& pl, void* ws) {
 }
 
 
-// The swapped-operand GEMMs (block_m 16) store y as fp16 [max_rows, H] followed by its
-// int8 exponents [max_rows, H/32] (y = y16 * 2^exp); the 128-row token-tile GEMMs store
-// fp32 [max_rows, H] (no exponents).
+// The swapped-operand GEMMs (block_m 16) store unweighted y as fp16 [max_rows, H] followed
+// by its int8 exponents [max_rows, H/32] (y = y16 * 2^exp; the combine applies the routing
+// weight); the 128-row token-tile GEMMs store weighted fp32 [max_rows, H] (no exponents).
 int8_t* y_exp_ptr(const Plan& pl, void* ws) {
   if (pl.bm != 16) return nullptr;
   return ws_ptr<int8_t>(ws, pl.lay.y + static_cast<size_t>(pl.lay.max_rows) * pl.H * 2);
@@ -477,7 +477,8 @@ moe_status_t run_gemm2(const Plan& pl_in, const void* w2, const float* w2_scale,
 
 moe_status_t run_combine(const Plan& pl, void* out, void* ws, const Launch& l) {
   return cuda_status(moe::launch_combine(l, ws_ptr<void>(ws, pl.lay.y), y_exp_ptr(pl, ws),
-                                         ws_ptr<int>(ws, pl.lay.pair_to_row), pl.T, pl.kk, pl.H, out));
+                                         ws_ptr<float>(ws, pl.lay.topk_w), ws_ptr<int>(ws, pl.lay.pair_to_row), pl.T,
+                                         pl.kk, pl.H, out));
 }
 
 // Common preamble of the entry points that launch: plan, workspace, device.

@@ -7,9 +7,11 @@
 // optimisation: NemotronH support", sglang PR 21321, section 1: the fused op returns a
 // bf16 tensor shaped like hidden_states).
 //
-// y comes in one of two formats: fp32 (the 128-row token-tile GEMMs), or fp16 with one
-// power-of-two exponent per 32 columns of a row (the swapped-operand GEMMs: y = y16 *
-// 2^exp, exact in fp32), which halves the bytes of this HBM-bound pass.
+// y comes in one of two formats: fp32 rows already weighted (the 128-row token-tile GEMMs),
+// or unweighted fp16 rows with one power-of-two exponent per 32 columns of each row (the
+// swapped-operand GEMMs), for which the combine applies the routing weight:
+// out[t] = sum_j w_tj * y16_j * 2^exp_j, each product exact in fp32 but the one by w. The
+// fp16 form halves the bytes of this HBM-bound pass.
 //
 // Each thread owns 8 consecutive columns of one token and reads k' x 32 (fp32) or k' x 17
 // (fp16 + exponent) bytes, writing 16.
@@ -53,8 +55,8 @@ __global__ void __launch_bounds__(kCombineThreads)
 }
 
 __global__ void __launch_bounds__(kCombineThreads)
-    combine_f16_kernel(const uint4* __restrict__ y, const int8_t* __restrict__ y_exp, const int* __restrict__ pair_to_row,
-                       int T, int k_total, int H8, uint4* __restrict__ out) {
+    combine_f16_kernel(const uint4* __restrict__ y, const int8_t* __restrict__ y_exp, const float* __restrict__ topk_w,
+                       const int* __restrict__ pair_to_row, int T, int k_total, int H8, uint4* __restrict__ out) {
   griddep_wait();
   griddep_launch_dependents();
   const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -65,12 +67,13 @@ __global__ void __launch_bounds__(kCombineThreads)
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i] = 0.f;
   const int* rows = pair_to_row + t * k_total;
+  const float* w = topk_w + t * k_total;
   const int H32 = H8 >> 2;  // exponents per row
   for (int j = 0; j < k_total; ++j) {
     const long long r = __ldg(rows + j);
     const uint4 v = __ldcs(y + r * H8 + c);  // columns 8c..8c+7, read once: streaming
     const int s = __ldg(y_exp + r * H32 + (c >> 2));
-    const float scale = __int_as_float((127 + s) << 23);  // 2^s, s in [-100, 113]
+    const float scale = __ldg(w + j) * __int_as_float((127 + s) << 23);  // w * 2^s, s in [-100, 113]
     const __half2* h = reinterpret_cast<const __half2*>(&v);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -89,8 +92,8 @@ __global__ void __launch_bounds__(kCombineThreads)
 
 }  // namespace
 
-cudaError_t launch_combine(const Launch& l, const void* y, const int8_t* y_exp, const int* pair_to_row, int T,
-                           int k_total, int H, void* out) {
+cudaError_t launch_combine(const Launch& l, const void* y, const int8_t* y_exp, const float* topk_w,
+                           const int* pair_to_row, int T, int k_total, int H, void* out) {
   const int H8 = H / 8;
   const long long n = static_cast<long long>(T) * H8;
   cudaLaunchConfig_t cfg;
@@ -98,9 +101,9 @@ cudaError_t launch_combine(const Launch& l, const void* y, const int8_t* y_exp, 
   make_launch_config(&cfg, attr, l, dim3(static_cast<unsigned>((n + kCombineThreads - 1) / kCombineThreads)),
                      dim3(kCombineThreads), 0);
   if (y_exp != nullptr) {
-    if (H % 32 != 0) return cudaErrorInvalidValue;
-    return cudaLaunchKernelEx(&cfg, combine_f16_kernel, static_cast<const uint4*>(y), y_exp, pair_to_row, T, k_total,
-                              H8, static_cast<uint4*>(out));
+    if (H % 32 != 0 || topk_w == nullptr) return cudaErrorInvalidValue;
+    return cudaLaunchKernelEx(&cfg, combine_f16_kernel, static_cast<const uint4*>(y), y_exp, topk_w, pair_to_row, T,
+                              k_total, H8, static_cast<uint4*>(out));
   }
   return cudaLaunchKernelEx(&cfg, combine_f32_kernel, static_cast<const float4*>(y), pair_to_row, T, k_total, H8,
                             static_cast<uint4*>(out));

@@ -88,8 +88,12 @@ constexpr int kTileW = kMW * kChunkBytes;  // 16 KB: one W chunk
 constexpr int kNMax = 256;                 // rows of a row group at most (MMA N)
 constexpr int kThreads = 224;
 constexpr int kWarpX = 6;
+// FP8 block-128 adds four epilogue warps (7..10): two per TMEM lane quadrant, each
+// promoting 64 of a tile's token columns
+template <int kKind>
+__host__ __device__ constexpr int threads_for() { return kKind == 3 ? 352 : kThreads; }
 constexpr int kTileRing = 4;
-constexpr int kRingReaders = 6;  // MMA, 4 epilogue warps, X producer
+constexpr int kRingReaders = 6;  // MMA, 4 epilogue warps, X producer (FP8 block-128: 8 epilogue warps)
 constexpr int kSmemCap = 232448;
 constexpr uint32_t kTmemCols = 2 * kNMax;
 // MXFP8: scale bytes per chunk in the ring, TMEM columns of the accumulators and of the
@@ -233,7 +237,7 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
 
 // kKind: 0 bf16, 1 per-tensor e4m3, 2 MXFP8, 3 FP8 block-128.
 template <int kKind>
-__global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
+__global__ void __launch_bounds__(threads_for<kKind>(), 1) gemm_swap_kernel(const Args a) {
   constexpr bool kFp8 = kKind == 1;  // scales applied in the epilogue
   constexpr bool kMx = kKind == 2;   // scales applied by the MMA
   constexpr bool kB128 = kKind == 3; // a partial per K chunk, promoted in the epilogue
@@ -273,16 +277,16 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
     }
     for (int b = 0; b < kPartBufs; ++b) {
       mbar_init(pfull0 + 8 * b, 1);
-      mbar_init(pempty0 + 8 * b, 128);
+      mbar_init(pempty0 + 8 * b, 256);  // every thread of the eight epilogue warps
     }
-    for (int b = 0; b < kSxSlots; ++b) mbar_init(sxfree0 + 8 * b, 4);  // the four epilogue warps
+    for (int b = 0; b < kSxSlots; ++b) mbar_init(sxfree0 + 8 * b, 8);  // the eight epilogue warps
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull0 + 8 * b, 1);
       mbar_init(tempty0 + 8 * b, 128);
     }
     for (int s = 0; s < kTileRing; ++s) {
       mbar_init(rfull0 + 8 * s, 1);
-      mbar_init(rempty0 + 8 * s, kRingReaders);
+      mbar_init(rempty0 + 8 * s, kB128 ? kRingReaders + 4 : kRingReaders);
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -491,11 +495,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
       mbar_wait_drain(drain_bar, 0);
     }
   } else {
-    // ---------------- epilogue (warps 2..5): lane = weight row ----------------
+    // ---------------- epilogue (warps 2..5; FP8 block-128 also 7..10): lane = weight row ----
     // 32 token columns at a time. For a given token the warp's 32 lanes hold neighbouring
     // output columns, so each store writes one contiguous piece of an output row (GEMM2:
-    // 128 B of fp32; GEMM1: 64 or 32 B of a 128-byte activation chunk row).
+    // 64 B of fp16; GEMM1: 64 or 32 B of a 128-byte activation chunk row).
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    const int half = kB128 && warp > kWarpX ? 1 : 0;  // FP8 block-128: token columns [64 half, 64 half + 64)
     const bool gated = a.activation != 1;  // 0 SwiGLU, 2 gelu_tanh, 3 swigluoai; 1 relu2
     const bool odd = (lane & 1) != 0;
     int rslot = 0, it = 0;
@@ -513,17 +518,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
       const int mt = __shfl_sync(0xffffffffu, t.w, 0);
       // FP8 per-tensor: the accumulator's dequantisation scale (GEMM1: before the activation)
       const float dq = kFp8 ? __ldg(a.w_scale + expert) * a.in_scale : 1.0f;
-      // GEMM2: routing weights of the group's tokens (token 32 b + lane in wreg[b]),
-      // loaded while the main loop still runs
-      float wreg[kNMax / 32];
-#pragma unroll
-      for (int b = 0; b < kNMax / 32; ++b) {
-        wreg[b] = 0.f;
-        if (a.mode != 0 && 32 * b + lane < n) {
-          const int pid = a.sorted_pair_ids[x_row + 32 * b + lane];
-          if (pid < a.num_pairs) wreg[b] = a.topk_w[pid];
-        }
-      }
       // GEMM1: this lane's activation feature f lies in K chunk f / 64 (bf16) or f / 128
       // (e4m3) of the activation; byte b of a 128-byte chunk row sits in 16-byte piece
       // (b / 16) ^ (row % 8)
@@ -536,27 +530,28 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
       // Output of token columns c0 .. c0 + 31 (c0 .. c0 + 15 unless `full`) of this lane's
       // weight row, from v[j] = accumulator of column c0 + j.
       auto store_block = [&](const uint32_t(&v)[32], int c0, bool full) {
-        float wl = wreg[0];  // GEMM2: routing weight of token column c0 + lane
-#pragma unroll
-        for (int b = 1; b < kNMax / 32; ++b)
-          if (c0 == 32 * b) wl = wreg[b];
         if (a.mode != 0) {
-          // y = acc * routing weight, stored as fp16 scaled by a power of two per 32 columns
-          // (this warp's columns of one token row): 2^-s brings the block's largest
-          // magnitude into [2^14, 2^15), so no value overflows fp16 and each keeps 11
-          // significant bits; s (at least -100) goes to y_exp.
+          // GEMM2: y = acc * dq (the routing weight is applied by the combine), stored as fp16
+          // scaled by a power of two shared by this block of 32 tokens x 32 columns (the
+          // warp's lanes): 2^-s brings the block's largest magnitude into [2^14, 2^15), so no
+          // value overflows fp16, and every value within 2^-28 of that maximum keeps 11
+          // significant bits. s (at least -100) is stored for each of the block's token rows.
+          float m = 0.f;
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (j < 16 || full) m = fmaxf(m, fabsf(__uint_as_float(v[j])));
+          const uint32_t amax = __reduce_max_sync(0xffffffffu, __float_as_uint(m * dq));
+          const int s = amax == 0u ? 0 : max(static_cast<int>(amax >> 23) - 127 - 14, -100);
+          const float f = dq * __int_as_float((127 - s) << 23);
           const int col = mt * kMW + q * 32 + lane;
           __half* y = static_cast<__half*>(a.out) + static_cast<size_t>(x_row + c0) * a.out_cols + col;
-          int8_t* ye = a.y_exp + static_cast<size_t>(x_row + c0) * (a.out_cols >> 5) + (col >> 5);
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             if (j == 16 && !full) break;
-            const float val = __uint_as_float(v[j]) * (__shfl_sync(0xffffffffu, wl, j) * dq);
-            const uint32_t amax = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(val)));
-            const int s = amax == 0u ? 0 : max(static_cast<int>(amax >> 23) - 127 - 14, -100);
-            y[static_cast<size_t>(j) * a.out_cols] = __float2half_rn(val * __int_as_float((127 - s) << 23));
-            if (lane == 0) ye[static_cast<size_t>(j) * (a.out_cols >> 5)] = static_cast<int8_t>(s);
+            y[static_cast<size_t>(j) * a.out_cols] = __float2half_rn(__uint_as_float(v[j]) * f);
           }
+          if (lane < 16 || full)
+            a.y_exp[static_cast<size_t>(x_row + c0 + lane) * (a.out_cols >> 5) + (col >> 5)] = static_cast<int8_t>(s);
         } else if (!gated) {
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
@@ -603,9 +598,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
         const int rb_odd = a.up_block > 0 ? a.up_block + (mt >> 1) : mt;
         const float swl_even = lane < a.k_chunks ? __ldg(sw_e + static_cast<size_t>(rb_even) * a.k_chunks + lane) : 0.f;
         const float swl_odd = lane < a.k_chunks ? __ldg(sw_e + static_cast<size_t>(rb_odd) * a.k_chunks + lane) : 0.f;
-        float acc[kB128GroupRows];
+        // this warp's token columns [64 half, 64 half + 64): blocks cb = 2 half, 2 half + 1
+        const int nb0 = n - 64 * half;              // columns left from this warp's first
+        const bool has0 = nb0 > 0, full0 = nb0 >= 32;
+        const bool has1 = nb0 > 32, full1 = nb0 >= 64;
+        float acc[64];
 #pragma unroll
-        for (int i = 0; i < kB128GroupRows; ++i) acc[i] = 0.f;
+        for (int i = 0; i < 64; ++i) acc[i] = 0.f;
         bool good = true;
         for (int c0 = 0; c0 < a.k_chunks && good; c0 += kc, ++ks) {
           const int kcs = min(kc, a.k_chunks - c0);
@@ -623,35 +622,34 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
             const float sw_e_k = __shfl_sync(0xffffffffu, swl_even, c0 + c);
             const float sw_o_k = __shfl_sync(0xffffffffu, swl_odd, c0 + c);
             const float sw = odd ? sw_o_k : sw_e_k;
-            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + pb * kPartCols;
-            const uint32_t sfc = sf + static_cast<uint32_t>(c * n) * 4u;
+            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + pb * kPartCols + 64 * half;
+            const uint32_t sfc = sf + static_cast<uint32_t>(c * n + 64 * half) * 4u;
+            // both 32-column loads in flight before one wait
+            uint32_t v[64];
+            if (full0) {
+              tmem_ld32(taddr, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+            } else if (has0) {
+              tmem_ld16(taddr, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
+            }
+            if (full1) {
+              tmem_ld32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+            } else if (has1) {
+              tmem_ld16(taddr + 32, *reinterpret_cast<uint32_t(*)[16]>(&v[32]));
+            }
+            tmem_wait_ld();
 #pragma unroll
-            for (int cb = 0; cb < kB128GroupRows / 32; ++cb) {
-              if (cb * 32 < n) {
-                const bool full = n - cb * 32 >= 32;
-                uint32_t v[32];
-                if (full) {
-                  tmem_ld32(taddr + cb * 32, v);
-                } else {
-                  uint32_t(&v16)[16] = *reinterpret_cast<uint32_t(*)[16]>(&v[0]);
-                  tmem_ld16(taddr + cb * 32, v16);
-#pragma unroll
-                  for (int j = 16; j < 32; ++j) v[j] = 0u;
-                }
-                tmem_wait_ld();
-#pragma unroll
-                for (int j4 = 0; j4 < 8; ++j4) {
-                  if (j4 == 4 && !full) break;
-                  float4 sx;  // the same four scales for every lane: a shared-memory broadcast
-                  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
-                               : "=f"(sx.x), "=f"(sx.y), "=f"(sx.z), "=f"(sx.w)
-                               : "r"(sfc + static_cast<uint32_t>(cb * 32 + 4 * j4) * 4u));
-                  const int j = cb * 32 + 4 * j4;
-                  acc[j + 0] = fmaf(__uint_as_float(v[4 * j4 + 0]), sx.x * sw, acc[j + 0]);
-                  acc[j + 1] = fmaf(__uint_as_float(v[4 * j4 + 1]), sx.y * sw, acc[j + 1]);
-                  acc[j + 2] = fmaf(__uint_as_float(v[4 * j4 + 2]), sx.z * sw, acc[j + 2]);
-                  acc[j + 3] = fmaf(__uint_as_float(v[4 * j4 + 3]), sx.w * sw, acc[j + 3]);
-                }
+            for (int j4 = 0; j4 < 16; ++j4) {
+              // columns 4 j4 .. 4 j4 + 3 of this warp's 64; past n they are skipped
+              if (4 * j4 < nb0) {
+                float4 sx;  // the same four scales for every lane: a shared-memory broadcast
+                asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                             : "=f"(sx.x), "=f"(sx.y), "=f"(sx.z), "=f"(sx.w)
+                             : "r"(sfc + static_cast<uint32_t>(4 * j4) * 4u));
+                const int j = 4 * j4;
+                acc[j + 0] = fmaf(__uint_as_float(v[j + 0]), sx.x * sw, acc[j + 0]);
+                acc[j + 1] = fmaf(__uint_as_float(v[j + 1]), sx.y * sw, acc[j + 1]);
+                acc[j + 2] = fmaf(__uint_as_float(v[j + 2]), sx.z * sw, acc[j + 2]);
+                acc[j + 3] = fmaf(__uint_as_float(v[j + 3]), sx.w * sw, acc[j + 3]);
               }
             }
             tc_fence_before();
@@ -663,14 +661,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_swap_kernel(const Args a) {
         }
         if (!__all_sync(0xffffffffu, good)) break;
 #pragma unroll
-        for (int cb = 0; cb < kB128GroupRows / 32; ++cb) {
-          if (cb * 32 < n) {
-            uint32_t v[32];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(acc[cb * 32 + j]);
-            store_block(v, cb * 32, n - cb * 32 >= 32);
-          }
-        }
+        for (int b = 0; b < 2; ++b)
+          if (32 * b < nb0)
+            store_block(*reinterpret_cast<const uint32_t(*)[32]>(&acc[32 * b]), 64 * half + 32 * b,
+                        nb0 - 32 * b >= 32);
       } else {
         const int acc = it & 1;
         const bool got = mbar_wait(tfull0 + 8 * acc, (it >> 1) & 1, abort_flag, a.status, kSiteTmemFull);
@@ -775,7 +769,7 @@ cudaError_t launch_gemm_swap(const Launch& l, int mode, const SwapOperands& o, c
   if (mode == 1 && (a.y_exp == nullptr || s.out_cols % 32 != 0)) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg;
   cudaLaunchAttribute attr[1];
-  make_launch_config(&cfg, attr, l, dim3(s.num_sms), dim3(kThreads), kSmemBytes);
+  make_launch_config(&cfg, attr, l, dim3(s.num_sms), dim3(kind == 3 ? threads_for<3>() : kThreads), kSmemBytes);
   return cudaLaunchKernelEx(&cfg, kernel, a);
 }
 

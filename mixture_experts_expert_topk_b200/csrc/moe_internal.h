@@ -94,8 +94,8 @@ struct GemmBuffers {
   int* status;
   const int* num_groups;    // row groups (gemm_swap)
   const int2* group_info;
-  // GEMM2 of the swapped-operand GEMMs: y as fp16 [rows, H] (out) with one power-of-two
-  // exponent per 32 columns of each row here, int8 [rows, H/32]: y = y16 * 2^exp
+  // GEMM2 of the swapped-operand GEMMs: unweighted y as fp16 [rows, H] (out) with one
+  // power-of-two exponent per 32 columns of each row here, int8 [rows, H/32]: y = y16 * 2^exp
   int8_t* out_exp;
 };
 // Operands of the swapped-operand GEMM: tiled weights, X in row-group order, and (GEMM1)
@@ -194,9 +194,10 @@ cudaError_t launch_ep_combine(const Launch& l, const void* returned, const int* 
                               void* out);
 
 // ---- elementwise (combine.cu, quant.cu, prepare.cu) ----
-// y: fp32 [rows, H] (y_exp == nullptr), or fp16 [rows, H] scaled by 2^y_exp[row][col / 32].
-cudaError_t launch_combine(const Launch& l, const void* y, const int8_t* y_exp, const int* pair_to_row, int T,
-                           int k_total, int H, void* out);
+// y: fp32 [rows, H] already weighted (y_exp == nullptr), or unweighted fp16 [rows, H] scaled by
+// 2^y_exp[row][col / 32], weighted here by topk_w [T, k'].
+cudaError_t launch_combine(const Launch& l, const void* y, const int8_t* y_exp, const float* topk_w,
+                           const int* pair_to_row, int T, int k_total, int H, void* out);
 cudaError_t launch_quant_act(const Launch& l, const void* x, int T, int H, void* q, float* scale);
 // As launch_quant_act over the first num_blocks[0] * block_m of max_rows rows.
 cudaError_t launch_quant_rows(const Launch& l, const void* x, int max_rows, int cols, const int* num_blocks,
