@@ -56,8 +56,9 @@ def _peaks():
 
 def _workload_name(cfg: MoeConfig) -> str:
     act = "SwiGLU" if cfg.gated else "relu2"
-    dt = ("MXFP8 e4m3 W8A8 (E8M0 scale per 32)" if cfg.mx else
-          ("FP8 e4m3 W8A8 per-tensor" if cfg.per_tensor else "FP8 e4m3 W8A8 block-128")) if cfg.fp8 else "bf16"
+    dt = ("NVFP4 E2M1 W4A4 (E4M3 scale per 16, fp32 per tensor)" if cfg.nv else
+          ("MXFP8 e4m3 W8A8 (E8M0 scale per 32)" if cfg.mx else
+           ("FP8 e4m3 W8A8 per-tensor" if cfg.per_tensor else "FP8 e4m3 W8A8 block-128"))) if cfg.fp8 else "bf16"
     sh = f"+{cfg.num_shared} shared" if cfg.num_shared else ""
     return (f"{cfg.name}: {dt} {act} MoE layer forward, T={cfg.T} H={cfg.H} E={cfg.E}{sh} "
             f"top-{cfg.topk}{sh} I={cfg.I}")
@@ -179,17 +180,23 @@ def run_ours(cfg: MoeConfig, steps: int, warmup: int, world: int, rank: int, loc
     dev = torch.device("cuda", local)
     inp = make_inputs(cfg, seed=0)
     I_pad = moe.padded_intermediate(cfg.I, cfg.activation, cfg.fp8)
-    s_in = float(inp["hidden"].float().abs().max() / 448) if cfg.per_tensor else 0.0
+    # static input scale: the hidden rows' amax / 448 (per-tensor FP8) or / (6 * 448) (NVFP4)
+    s_in = (float(inp["hidden"].float().abs().max() / 448) if cfg.per_tensor else
+            (float(inp["hidden"].float().abs().max() / 2688) if cfg.nv else 0.0))
     prob = moe.make_problem(cfg.T, cfg.H, cfg.E, cfg.topk, I_pad, renormalize=cfg.renormalize,
                             activation=cfg.activation, num_shared=cfg.num_shared, fp8=cfg.fp8,
                             input_scale=s_in, activation_scale=cfg.activation_scale)
-    pt_kw = dict(input_scale=s_in, activation_scale=cfg.activation_scale) if cfg.per_tensor else {}
+    pt_kw = dict(input_scale=s_in, activation_scale=cfg.activation_scale) if (cfg.per_tensor or cfg.nv) else {}
     hidden = inp["hidden"].to(dev)
     logits = inp["logits"].to(dev)
     s13 = s2 = None
     w13 = inp["w13"].to(dev)
     w2 = inp["w2"].to(dev)
-    if cfg.mx:
+    g13 = g2 = None
+    if cfg.nv:
+        w13, s13, g13 = moe.quantize_weights_nvfp4(w13)
+        w2, s2, g2 = moe.quantize_weights_nvfp4(w2)
+    elif cfg.mx:
         w13, s13 = moe.quantize_weights_mxfp8(w13)
         w2, s2 = moe.quantize_weights_mxfp8(w2)
     elif cfg.per_tensor:
@@ -198,10 +205,11 @@ def run_ours(cfg: MoeConfig, steps: int, warmup: int, world: int, rank: int, loc
     elif cfg.fp8:
         w13, s13 = moe.quantize_weights_fp8(w13)
         w2, s2 = moe.quantize_weights_fp8(w2)
-    if cfg.mx:
-        # the E8M0 scales travel inside the prepared weights; the forward takes none
+    if cfg.mx or cfg.nv:
+        # the block scales travel inside the prepared weights; the forward takes none
+        # (MXFP8) or the weights' tensor scales (NVFP4)
         w13p, w2p = moe.prepare_weights(prob, w13, w2, cfg.I, w13_scale=s13, w2_scale=s2)
-        s13 = s2 = None
+        s13, s2 = g13, g2
     else:
         w13p, w2p = moe.prepare_weights(prob, w13, w2, cfg.I)
     del w13, w2
@@ -326,17 +334,26 @@ def cpu_baseline(cfg: MoeConfig, inp, budget_s: float, tokens_hint: int):
     w13b, w2b = bits(inp["w13"]), bits(inp["w2"])
     n = max(1, min(cfg.T, tokens_hint))
     tok = np.arange(n)
-    if cfg.mx:
+    if cfg.mx or cfg.nv:
         # quantise only the experts the sampled tokens use (the others do not enter the sample)
         ids, _ = O.route(lg[tok], cfg.topk, cfg.renormalize, cfg.num_shared)
-        fp8w = O.quantize_weights_mxfp8(w13b, w2b, experts=sorted(set(int(e) for e in ids.reshape(-1))))
+        used = sorted(set(int(e) for e in ids.reshape(-1)))
+        if cfg.nv:
+            fp8w = O.quantize_weights_nvfp4(w13b, w2b, experts=used)
+            s_in = np.float32(np.abs(O.bf16_bits_to_f32(hb)).max() / np.float32(2688))
+        else:
+            fp8w = O.quantize_weights_mxfp8(w13b, w2b, experts=used)
     elif cfg.per_tensor:
         fp8w = O.quantize_weights_fp8_per_tensor(w13b, w2b)
         s_in = np.float32(np.abs(O.bf16_bits_to_f32(hb)).max() / np.float32(448))
     elif cfg.fp8:
         fp8w = O.quantize_weights_fp8(w13b, w2b)
     t0 = time.perf_counter()
-    if cfg.mx:
+    if cfg.nv:
+        O.moe_forward_nvfp4(hb, lg, *fp8w, s_in, np.float32(cfg.activation_scale), topk=cfg.topk,
+                            renormalize=cfg.renormalize, activation=cfg.activation, num_shared=cfg.num_shared,
+                            tokens=tok)
+    elif cfg.mx:
         O.moe_forward_mxfp8(hb, lg, *fp8w, topk=cfg.topk, renormalize=cfg.renormalize,
                             activation=cfg.activation, num_shared=cfg.num_shared, tokens=tok)
     elif cfg.per_tensor:
@@ -384,7 +401,9 @@ def main():
     metric = "fused MoE layer forward throughput (TFLOP/s; us/call in ms_per_step)"
     base = {"metric": metric, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": ("mxfp8_e4m3" if cfg.mx else "fp8_e4m3") if cfg.fp8 else "bf16", "data": "synthetic"}
+            "vs_baseline": None,
+            "dtype": ("nvfp4_e2m1" if cfg.nv else ("mxfp8_e4m3" if cfg.mx else "fp8_e4m3")) if cfg.fp8 else "bf16",
+            "data": "synthetic"}
 
     if args.impl == "reference":
         if rank != 0:
@@ -421,9 +440,13 @@ def main():
     n_touched, w13_bytes, w2_bytes = touched_expert_bytes(r["ids"], cfg, elt)
     if cfg.mx:  # one E8M0 byte per 32 weights
         w13_bytes, w2_bytes = w13_bytes * 33 // 32, w2_bytes * 33 // 32
+    if cfg.nv:  # half a byte per weight plus one E4M3 byte per 16
+        w13_bytes, w2_bytes = w13_bytes * 9 // 16, w2_bytes * 9 // 16
     P = cfg.T * cfg.k_total
     # GEMM1 algorithmic bytes per launch: touched w13, hidden rows read once, act written
-    g1_bytes = w13_bytes + cfg.T * cfg.H * elt + P * cfg.I * elt
+    act_elt = 2 if (cfg.mx or cfg.nv or cfg.block128) else elt  # GEMM1 writes bf16 before re-quantising
+    x_elt = 0.5625 if cfg.nv else elt                            # the GEMM1 input rows read once
+    g1_bytes = w13_bytes + cfg.T * cfg.H * x_elt + P * cfg.I * act_elt
     g1_ms = r["kernel_ms"]["gemm1"]
     g1_gbs = g1_bytes / (g1_ms / 1e3) / 1e9
     g1_flops = 2.0 * P * cfg.H * cfg.N1

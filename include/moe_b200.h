@@ -90,7 +90,7 @@ typedef enum {
                                    GEMM inputs with the static problem->input_scale and
                                    problem->activation_scale (the per-tensor FP8 variant,
                                    sglang PR 21321 sections 1-2); I and H multiples of 128 */
-  MOE_DTYPE_MXFP8 = 3           /* MXFP8: e4m3 weights and GEMM inputs, each with one E8M0
+  MOE_DTYPE_MXFP8 = 3,          /* MXFP8: e4m3 weights and GEMM inputs, each with one E8M0
                                    (power-of-two) scale per 32 values of K (the MXFP8 weights
                                    of sglang PR 21321 section 2), applied by the tensor core's
                                    block-scaled MMA. Conversion (weights, hidden rows and
@@ -99,6 +99,18 @@ typedef enum {
                                    (-127 for an all-zero block), byte = exponent + 127, codes
                                    e4m3(x * 2^-exponent) round to nearest even, saturating.
                                    I and H multiples of 128. */
+  MOE_DTYPE_NVFP4 = 4           /* NVFP4 W4A4 ("FlashInfer gated MoE kernel optimisation for
+                                   Blackwell", section 4, names NVFP4 weights; the format is
+                                   NVIDIA's): E2M1 values packed two per byte (lower K index in
+                                   the low nibble), one E4M3 scale per 16 values of K and one
+                                   fp32 scale g per tensor, value = e2m1 * e4m3 * g, with block
+                                   scale e4m3(amax / 6 / g) and codes e2m1(x / (scale * g)), round
+                                   to nearest even, saturating. The weights carry g per expert
+                                   matrix (moe_quantize_weights_nvfp4: amax / (6 * 448)); the GEMM
+                                   inputs use the static problem->input_scale (hidden rows) and
+                                   problem->activation_scale (GEMM1's activation) as their g, with
+                                   block scales per 16 values. The block-scaled MMA applies the
+                                   block scales. I and H multiples of 256. */
 } moe_wdtype_t;
 
 /* Bit flags of moe_problem_t.flags. */
@@ -112,8 +124,9 @@ typedef struct {
   int32_t num_shared;   /* 0 or 1: shared-expert slots; slot id E_r, weight 1, after the
                            routed slots (sglang PR 26204 section 2). Experts in the
                            weights: E = E_r + num_shared <= 1024. */
-  int32_t intermediate; /* I after padding (moe_padded_intermediate): multiple of 16 for
-                           SWIGLU, of 128 for RELU2 and for FP8 */
+  int32_t intermediate; /* I after padding (moe_padded_intermediate): multiple of 16 for the
+                           gated activations, of 128 for RELU2 and the 8-bit formats, of 256
+                           for NVFP4 */
   int32_t topk;         /* 1 <= topk <= E_r; topk + num_shared <= 16 */
   int32_t renormalize;  /* 0/1: divide the selected softmax weights by their sum */
   int32_t activation;   /* moe_activation_t */
@@ -123,9 +136,11 @@ typedef struct {
                            N) or 128 (BF16 and FP8 block-128 only: 128-row token tiles) */
   uint32_t flags;       /* MOE_FLAG_* */
   float input_scale;      /* MOE_DTYPE_FP8_PER_TENSOR: static scale of the hidden rows,
-                             x_q = e4m3(x / input_scale); finite, > 0 (ignored otherwise) */
+                             x_q = e4m3(x / input_scale); MOE_DTYPE_NVFP4: the hidden rows'
+                             tensor scale g; finite, > 0 (ignored otherwise) */
   float activation_scale; /* MOE_DTYPE_FP8_PER_TENSOR: static scale of GEMM1's activation,
-                             a_q = e4m3(a / activation_scale); finite, > 0 (ignored otherwise) */
+                             a_q = e4m3(a / activation_scale); MOE_DTYPE_NVFP4: the
+                             activation's tensor scale g; finite, > 0 (ignored otherwise) */
 } moe_problem_t;
 
 /* Byte offsets of the intermediates inside the caller's workspace (for inspection by
@@ -251,6 +266,34 @@ moe_status_t moe_prepare_weights_mxfp8(const moe_problem_t* problem, const void*
                                        const void* w2_scales, void* w13_out, void* w2_out,
                                        moe_stream_t stream);
 
+/* NVFP4 quantisation of bf16 weights (MOE_DTYPE_NVFP4), along each row:
+ *   w              device bf16 [num_mats, rows, cols], cols a multiple of 16, num_mats <= 65535;
+ *   codes          device uint8 [num_mats, rows, cols/2]: E2M1 pairs, lower column in the low nibble;
+ *   scales         device uint8 [num_mats, rows, cols/16]: E4M3 block scales;
+ *   global_scales  device fp32 [num_mats]: g = amax / (6 * 448) of each matrix (1 if all zero).
+ * Per block of 16 values: scale = e4m3(amax / 6 / g), codes = e2m1(x / (scale * g)) (IEEE
+ * divisions; round to nearest even, saturating). Asynchronous on `stream`. */
+moe_status_t moe_quantize_weights_nvfp4(const void* w, int64_t num_mats, int32_t rows, int32_t cols,
+                                        void* codes, void* scales, float* global_scales,
+                                        moe_stream_t stream);
+
+/* Load-time preparation of NVFP4 weights (problem->wdtype == MOE_DTYPE_NVFP4):
+ *   w13_codes [E, N1, H/2] and w13_scales [E, N1, H/16] (checkpoint order: gate rows then up
+ *             rows for a gated activation), w2_codes [E, H, I/2] and w2_scales [E, H, I/16],
+ *             as moe_quantize_weights_nvfp4 writes them; I = problem->intermediate (a multiple
+ *             of 256: the weights come padded).
+ * Each output (moe_prepared_weights_bytes(problem, 0 / 1) bytes, 16-byte aligned) holds the
+ * codes tiled as 128 rows x 128 bytes (256 values of K) per tile at ((e*MT + m)*KC + c) *
+ * 16384 (gated rows interleaved [gate0, up0, ...], 16-byte pieces of row r at position
+ * q ^ (r % 8)), followed by the scales: a 2048-byte block per tile at the same tile index,
+ * byte 512 mm + 16 l + 4 j + k = scale of tile row 32 j + l for block 16 c + 4 mm + k (zero
+ * past the matrix). moe_forward takes the prepared buffers with w13_scale / w2_scale = the
+ * global scales [E]. Asynchronous on `stream`. */
+moe_status_t moe_prepare_weights_nvfp4(const moe_problem_t* problem, const void* w13_codes,
+                                       const void* w13_scales, const void* w2_codes,
+                                       const void* w2_scales, void* w13_out, void* w2_out,
+                                       moe_stream_t stream);
+
 /* Bytes of the prepared w13 (which = 0) or w2 (which = 1) for `problem` (host only), or
  * 0 for an invalid problem or `which`. */
 size_t moe_prepared_weights_bytes(const moe_problem_t* problem, int32_t which);
@@ -270,9 +313,10 @@ moe_status_t moe_quantize_weights_fp8(const void* w, int64_t num_mats, int32_t r
  *   router_logits  device fp32 [T, E_r] (finite values; NaN/Inf are not supported)
  *   w13, w2        device, prepared by moe_prepare_weights for this problem's layout
  *   w13_scale      FP8 block-128: device fp32 [E, N1/128, H/128], checkpoint (gate-first,
- *                  un-interleaved) block order; FP8 per-tensor: device fp32 [E]; else NULL
- *   w2_scale       FP8 block-128: device fp32 [E, H/128, I/128]; per-tensor: [E]; else NULL
- *                  (MXFP8: both NULL, the scales are part of the prepared weights)
+ *                  un-interleaved) block order; FP8 per-tensor and NVFP4: device fp32 [E]
+ *                  (NVFP4: the global scales); else NULL
+ *   w2_scale       FP8 block-128: device fp32 [E, H/128, I/128]; per-tensor, NVFP4: [E]; else
+ *                  NULL (MXFP8: both NULL, the scales are part of the prepared weights)
  *   out            device bf16 [T, H] (must not alias hidden)
  *   workspace      device, >= moe_workspace_size(problem) bytes, 256-byte aligned; one
  *                  workspace must not be used by two calls in flight at once.
@@ -310,15 +354,16 @@ moe_status_t moe_forward_host(const moe_problem_t* problem, const void* h_hidden
                               void* workspace, size_t workspace_bytes, moe_stream_t stream);
 
 /* The steps as separate calls on the same workspace: route, align, quant_act (FP8
- * block-128), permute (block_m 16), gemm1, gemm2, combine; moe_forward runs exactly these,
- * in this order. They exist so tests can check each intermediate and tools can time each kernel;
+ * block-128, NVFP4), permute (block_m 16), gemm1, gemm2, combine; moe_forward runs exactly
+ * these, in this order. They exist so tests can check each intermediate and tools can time each kernel;
  * each requires the previous steps to have been enqueued. */
 moe_status_t moe_stage_route(const moe_problem_t* problem, const float* router_logits,
                              void* workspace, size_t workspace_bytes, moe_stream_t stream);
 moe_status_t moe_stage_align(const moe_problem_t* problem, void* workspace,
                              size_t workspace_bytes, moe_stream_t stream);
-/* FP8 block-128 only (else MOE_ERR_INVALID_ARG): quantise hidden per token per 128 columns
- * into the workspace (xq, xq_scale). */
+/* FP8 block-128 and NVFP4 only (else MOE_ERR_INVALID_ARG): quantise hidden once per token
+ * into the workspace (xq, xq_scale): per 128 columns (FP8 block-128) or to NVFP4 with the
+ * input scale (NVFP4). */
 moe_status_t moe_stage_quant_act(const moe_problem_t* problem, const void* hidden,
                                  void* workspace, size_t workspace_bytes, moe_stream_t stream);
 /* block_m 16 (the default): copy the token rows of every row group into the workspace in

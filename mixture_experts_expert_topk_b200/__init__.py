@@ -19,13 +19,13 @@ import torch
 
 from . import _capi
 from ._capi import (MOE_ACT_GELU_TANH, MOE_ACT_RELU2, MOE_ACT_SWIGLU, MOE_ACT_SWIGLUOAI, MOE_DTYPE_BF16, MOE_DTYPE_FP8_BLOCK128,
-                    MOE_DTYPE_FP8_PER_TENSOR, MOE_DTYPE_MXFP8,
+                    MOE_DTYPE_FP8_PER_TENSOR, MOE_DTYPE_MXFP8, MOE_DTYPE_NVFP4,
                     MOE_FLAG_PDL, MoeError, Problem, check, lib)
 
 __all__ = [
     "MoeError", "Problem", "make_problem", "padded_intermediate", "workspace_layout",
     "workspace_size", "new_workspace", "prepare_weights", "quantize_weights_fp8",
-    "quantize_weights_fp8_per_tensor", "quantize_weights_mxfp8", "moe_forward",
+    "quantize_weights_fp8_per_tensor", "quantize_weights_mxfp8", "quantize_weights_nvfp4", "moe_forward",
     "moe_forward_host", "stage_route", "stage_align", "stage_quant_act", "stage_gemm1",
     "stage_gemm2", "stage_combine", "device_status", "read_workspace", "lib", "check",
 ]
@@ -70,17 +70,21 @@ def make_problem(T: int, H: int, num_routed: int, topk: int, intermediate: int, 
     True or "block128" (e4m3, 128x128 weight blocks, 1x128 activation groups), or
     "per_tensor" (e4m3, one scale per expert matrix and the static ``input_scale`` /
     ``activation_scale``), or "mxfp8" (e4m3 with an E8M0 scale per 32 values of K on both
-    GEMM inputs)."""
+    GEMM inputs), or "nvfp4" (E2M1 with an E4M3 scale per 16 values of K, tensor scales:
+    per expert matrix for the weights, ``input_scale`` / ``activation_scale`` for the GEMM
+    inputs)."""
     if fp8 == "per_tensor":
         wdtype = MOE_DTYPE_FP8_PER_TENSOR
     elif fp8 == "mxfp8":
         wdtype = MOE_DTYPE_MXFP8
+    elif fp8 == "nvfp4":
+        wdtype = MOE_DTYPE_NVFP4
     elif fp8 in (True, "block128"):
         wdtype = MOE_DTYPE_FP8_BLOCK128
     elif fp8 is False or fp8 is None:
         wdtype = MOE_DTYPE_BF16
     else:
-        raise ValueError(f"fp8 must be False, True/'block128', 'per_tensor' or 'mxfp8', got {fp8!r}")
+        raise ValueError(f"fp8 must be False, True/'block128', 'per_tensor', 'mxfp8' or 'nvfp4', got {fp8!r}")
     return Problem(num_tokens=T, hidden=H, num_routed=num_routed, num_shared=num_shared,
                    intermediate=intermediate, topk=topk, renormalize=int(bool(renormalize)),
                    activation=_act(activation), wdtype=wdtype, block_m=block_m,
@@ -89,8 +93,8 @@ def make_problem(T: int, H: int, num_routed: int, topk: int, intermediate: int, 
 
 
 def padded_intermediate(intermediate: int, activation="swiglu", fp8=False) -> int:
-    v = lib().moe_padded_intermediate(intermediate, _act(activation),
-                                      MOE_DTYPE_FP8_BLOCK128 if fp8 else MOE_DTYPE_BF16)  # every 8-bit format pads to 128
+    wd = MOE_DTYPE_NVFP4 if fp8 == "nvfp4" else (MOE_DTYPE_FP8_BLOCK128 if fp8 else MOE_DTYPE_BF16)
+    v = lib().moe_padded_intermediate(intermediate, _act(activation), wd)  # every 8-bit format pads to 128
     if v < 0:
         raise ValueError("invalid intermediate size or activation")
     return v
@@ -125,6 +129,8 @@ def prepare_weights(prob: Problem, w13: torch.Tensor, w2: torch.Tensor, intermed
     ``w2_scale`` [E, H, I/32]; the prepared tensors then carry them (``.moe_mxfp8``)."""
     if prob.wdtype == MOE_DTYPE_MXFP8:
         return _prepare_weights_mxfp8(prob, w13, w2, w13_scale, w2_scale, stream)
+    if prob.wdtype == MOE_DTYPE_NVFP4:
+        return _prepare_weights_nvfp4(prob, w13, w2, w13_scale, w2_scale, stream)
     fp8 = prob.wdtype in (MOE_DTYPE_FP8_BLOCK128, MOE_DTYPE_FP8_PER_TENSOR)
     dt = torch.uint8 if fp8 else torch.bfloat16
     _dev(w13, "w13", dt)
@@ -168,6 +174,41 @@ def _prepare_weights_mxfp8(prob, w13, w2, w13_scale, w2_scale, stream):
         t.moe_intermediate = prob.intermediate
         t.moe_mxfp8 = True
     return w13p, w2p
+
+
+def _prepare_weights_nvfp4(prob, w13, w2, w13_scale, w2_scale, stream):
+    for t, n in ((w13, "w13"), (w2, "w2"), (w13_scale, "w13_scale"), (w2_scale, "w2_scale")):
+        if t is None:
+            raise ValueError(f"NVFP4 preparation needs {n} (packed codes and E4M3 block scales)")
+        _dev(t, n, torch.uint8)
+    n13 = lib().moe_prepared_weights_bytes(ctypes.byref(prob), 0)
+    n2 = lib().moe_prepared_weights_bytes(ctypes.byref(prob), 1)
+    if n13 == 0 or n2 == 0:
+        check(lib().moe_check_problem(ctypes.byref(prob)), "moe_prepared_weights_bytes")
+    w13p = torch.empty(n13, dtype=torch.uint8, device=w13.device)
+    w2p = torch.empty(n2, dtype=torch.uint8, device=w2.device)
+    check(lib().moe_prepare_weights_nvfp4(ctypes.byref(prob), _ptr(w13), _ptr(w13_scale), _ptr(w2),
+                                          _ptr(w2_scale), _ptr(w13p), _ptr(w2p), _stream(stream)),
+          "moe_prepare_weights_nvfp4")
+    for t in (w13p, w2p):
+        t.moe_intermediate = prob.intermediate
+        t.moe_nvfp4 = True
+    return w13p, w2p
+
+
+def quantize_weights_nvfp4(w: torch.Tensor, stream=None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """NVFP4 quantisation of bf16 [..., rows, cols] weights along each row: (packed E2M1
+    codes uint8 [..., rows, cols/2], E4M3 block scales uint8 [..., rows, cols/16], tensor
+    scales fp32 [...] = amax / (6 * 448) per matrix)."""
+    _dev(w, "w", torch.bfloat16)
+    rows, cols = w.shape[-2], w.shape[-1]
+    mats = w.numel() // (rows * cols)
+    codes = torch.empty(tuple(w.shape[:-1]) + (cols // 2,), dtype=torch.uint8, device=w.device)
+    scales = torch.empty(tuple(w.shape[:-1]) + (cols // 16,), dtype=torch.uint8, device=w.device)
+    g = torch.empty(tuple(w.shape[:-2]), dtype=torch.float32, device=w.device)
+    check(lib().moe_quantize_weights_nvfp4(_ptr(w), mats, rows, cols, _ptr(codes), _ptr(scales), _ptr(g),
+                                           _stream(stream)), "moe_quantize_weights_nvfp4")
+    return codes, scales, g
 
 
 def quantize_weights_mxfp8(w: torch.Tensor, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
@@ -258,6 +299,8 @@ def moe_forward(hidden: torch.Tensor, router_logits: torch.Tensor, w13: torch.Te
     per_tensor = input_scale is not None or activation_scale is not None
     if getattr(w13, "moe_mxfp8", False):
         fp8 = "mxfp8"  # scales inside the prepared weights
+    elif getattr(w13, "moe_nvfp4", False):
+        fp8 = "nvfp4"  # block scales inside the prepared weights; w13_scale / w2_scale: tensor scales
     else:
         fp8 = "per_tensor" if per_tensor else w13_scale is not None
     _dev(hidden, "hidden", torch.bfloat16)
@@ -285,7 +328,8 @@ def moe_forward_routed(hidden: torch.Tensor, topk_ids: torch.Tensor, topk_weight
     [0, num_routed), ``topk_weights`` fp32 [T, topk] (used as given); the rest as
     :func:`moe_forward`. Out-of-range ids are dropped and reported by
     :func:`device_status`."""
-    fp8 = "mxfp8" if getattr(w13, "moe_mxfp8", False) else w13_scale is not None
+    fp8 = ("mxfp8" if getattr(w13, "moe_mxfp8", False) else
+           ("nvfp4" if getattr(w13, "moe_nvfp4", False) else w13_scale is not None))
     _dev(hidden, "hidden", torch.bfloat16)
     _dev(topk_ids, "topk_ids", torch.int32)
     _dev(topk_weights, "topk_weights", torch.float32)
@@ -419,6 +463,19 @@ def read_workspace(prob: Problem, workspace: torch.Tensor) -> Dict[str, torch.Te
         out["act"] = view(L["act"], rows * act_cols, torch.bfloat16)
         out["xs"] = view(L["xs"], rows * (H // 128) * 132, torch.uint8)
         out["actq"] = view(L["actq"], rows * (I // 128) * 132, torch.uint8)
+        out["group_info"] = view(L["group_info"], (rows // 16 + 1) * 2, torch.int32).view(-1, 2)
+    elif prob.wdtype == MOE_DTYPE_NVFP4:
+        # bf16 activation (64-column chunks); packed E2M1 codes of the hidden rows and of the
+        # activation (128-byte chunks of 256 values) in row-group order; the scale blocks raw;
+        # the per-token quantised hidden rows
+        act_cols = -(-I // 64) * 64
+        out["act"] = view(L["act"], rows * act_cols, torch.bfloat16)
+        out["xq"] = view(L["xq"], T * H // 2, torch.uint8).view(T, H // 2)
+        out["xq_scale"] = view(L["xq_scale"], T * H // 16, torch.uint8).view(T, H // 16)
+        out["xs"] = view(L["xs"], rows * H // 2, torch.uint8)
+        out["xs_scale"] = view(L["xs_scale"], rows // 16 * (H // 256) * 2048, torch.uint8)
+        out["actq"] = view(L["actq"], rows * I // 2, torch.uint8)
+        out["act_scale"] = view(L["act_scale"], rows // 16 * (I // 256) * 2048, torch.uint8)
         out["group_info"] = view(L["group_info"], (rows // 16 + 1) * 2, torch.int32).view(-1, 2)
     elif prob.wdtype == MOE_DTYPE_FP8_PER_TENSOR:
         # e4m3 codes in row-group order (128-column chunks per group, swizzled); flat views

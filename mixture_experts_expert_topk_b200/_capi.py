@@ -26,6 +26,7 @@ MOE_ACT_GELU_TANH = 2
 MOE_ACT_SWIGLUOAI = 3
 MOE_DTYPE_FP8_PER_TENSOR = 2
 MOE_DTYPE_MXFP8 = 3
+MOE_DTYPE_NVFP4 = 4
 MOE_DTYPE_BF16 = 0
 MOE_DTYPE_FP8_BLOCK128 = 1
 MOE_FLAG_PDL = 1
@@ -84,6 +85,8 @@ SIGNATURES = {
     "moe_quantize_weights_fp8_per_tensor": (_I, [_V, ctypes.c_int64, _I, _I, _V, _V, _V]),
     "moe_quantize_weights_mxfp8": (_I, [_V, ctypes.c_int64, _I, _I, _V, _V, _V]),
     "moe_prepare_weights_mxfp8": (_I, [_P, _V, _V, _V, _V, _V, _V, _V]),
+    "moe_quantize_weights_nvfp4": (_I, [_V, ctypes.c_int64, _I, _I, _V, _V, _V, _V]),
+    "moe_prepare_weights_nvfp4": (_I, [_P, _V, _V, _V, _V, _V, _V, _V]),
     "moe_ep_workspace_size": (_S, [_P, _I]),
     "moe_ep_max_send_rows": (ctypes.c_int64, [_P, _I]),
     "moe_ep_dispatch": (_I, [_P, _I, _I, _V, _V, _V, _V, _V, _V, _V, _V, _V, _S, _V]),

@@ -49,8 +49,8 @@ bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr
 bool aligned4(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 struct Plan {
-  int T, H, Er, Es, E, I, topk, kk, bm, grp, N1, gated, fp8, pt, mx, q8, renorm, act;
-  float in_scale, act_scale;  // per-tensor FP8 static scales
+  int T, H, Er, Es, E, I, topk, kk, bm, grp, N1, gated, fp8, pt, mx, nv, q8, renorm, act;
+  float in_scale, act_scale;  // static scales of the GEMM inputs (per-tensor FP8, NVFP4)
   long long P;
   int bn1, bn2;
   moe_workspace_layout_t lay;
@@ -69,15 +69,16 @@ moe_status_t make_plan(const moe_problem_t* p, Plan* pl) {
       p->activation != MOE_ACT_SWIGLUOAI)
     return MOE_ERR_INVALID_ARG;
   if (p->wdtype != MOE_DTYPE_BF16 && p->wdtype != MOE_DTYPE_FP8_BLOCK128 && p->wdtype != MOE_DTYPE_FP8_PER_TENSOR &&
-      p->wdtype != MOE_DTYPE_MXFP8)
+      p->wdtype != MOE_DTYPE_MXFP8 && p->wdtype != MOE_DTYPE_NVFP4)
     return MOE_ERR_INVALID_ARG;
   if (p->flags & ~MOE_FLAG_PDL) return MOE_ERR_INVALID_ARG;
   q.gated = p->activation != MOE_ACT_RELU2;
   q.fp8 = p->wdtype == MOE_DTYPE_FP8_BLOCK128;
   q.pt = p->wdtype == MOE_DTYPE_FP8_PER_TENSOR;
   q.mx = p->wdtype == MOE_DTYPE_MXFP8;
-  q.q8 = q.fp8 || q.pt || q.mx;  // 8-bit weights: I must come padded to 128
-  if (q.pt) {
+  q.nv = p->wdtype == MOE_DTYPE_NVFP4;
+  q.q8 = q.fp8 || q.pt || q.mx || q.nv;  // quantised weights: I must come padded (128; NVFP4 256)
+  if (q.pt || q.nv) {
     // static scales: finite and positive
     if (!(p->input_scale > 0.0f && p->input_scale < 3.0e38f) ||
         !(p->activation_scale > 0.0f && p->activation_scale < 3.0e38f))
@@ -86,9 +87,9 @@ moe_status_t make_plan(const moe_problem_t* p, Plan* pl) {
     q.act_scale = p->activation_scale;
   }
   // the intermediate size must already be padded (moe_padded_intermediate)
-  const int ialign = (q.q8 || !q.gated) ? 128 : 16;
+  const int ialign = q.nv ? 256 : ((q.q8 || !q.gated) ? 128 : 16);
   if (p->intermediate % ialign != 0) return MOE_ERR_INVALID_ARG;
-  if (p->hidden % 128 != 0) return MOE_ERR_UNSUPPORTED;
+  if (p->hidden % (q.nv ? 256 : 128) != 0) return MOE_ERR_UNSUPPORTED;
   if (p->num_routed + p->num_shared > moe::kMaxExperts) return MOE_ERR_UNSUPPORTED;
   if (p->topk + p->num_shared > moe::kMaxSlots) return MOE_ERR_UNSUPPORTED;
   if (p->block_m != 0 && p->block_m != 16 && p->block_m != 128) return MOE_ERR_UNSUPPORTED;
@@ -108,9 +109,11 @@ moe_status_t make_plan(const moe_problem_t* p, Plan* pl) {
   // Row alignment. Default: 16-row blocks, the expert's weights as the MMA's M operand and
   // row groups of token rows as N (up to 256 rows; 192 for MXFP8, 128 for FP8 block-128).
   // block_m = 128 (BF16 and FP8 block-128 only): 128-row token tiles.
-  if (p->block_m == 128 && (q.pt || q.mx)) return MOE_ERR_UNSUPPORTED;
+  if (p->block_m == 128 && (q.pt || q.mx || q.nv)) return MOE_ERR_UNSUPPORTED;
   q.bm = p->block_m != 0 ? p->block_m : 16;
-  q.grp = q.bm == 16 ? (q.mx ? moe::kMxGroupRows : (q.fp8 ? moe::kB128GroupRows : kGroupRows)) : 0;
+  q.grp = q.bm == 16 ? (q.mx ? moe::kMxGroupRows
+                             : (q.fp8 ? moe::kB128GroupRows : (q.nv ? moe::kNvGroupRows : kGroupRows)))
+                     : 0;
   q.renorm = p->renormalize;
   q.act = p->activation;
   q.P = static_cast<long long>(q.T) * q.kk;
@@ -144,8 +147,10 @@ moe_status_t make_plan(const moe_problem_t* p, Plan* pl) {
   L.chunk_hist = take(static_cast<size_t>(L.num_chunks) * q.E * 4);
   const bool fp8_tiles = q.fp8 && q.bm == 128;  // FP8 block-128 with 128-row token tiles
   const bool b128 = q.fp8 && q.bm == 16;        // FP8 block-128 on the swapped-operand GEMMs
-  L.xq = take(q.fp8 ? T * H : 0);
-  L.xq_scale = take(q.fp8 ? T * (H / 128) * 4 : 0);
+  // the hidden rows quantised once per token: FP8 block-128 e4m3 [T, H] + fp32 [T, H/128];
+  // NVFP4 packed E2M1 [T, H/2] + E4M3 [T, H/16]
+  L.xq = take(q.fp8 ? T * H : (q.nv ? T * H / 2 : 0));
+  L.xq_scale = take(q.fp8 ? T * (H / 128) * 4 : (q.nv ? T * H / 16 : 0));
   // the swapped-operand GEMMs keep the activation in row-group order, 128-byte chunks (64
   // bf16 or 128 e4m3 columns)
   const size_t act_bytes = q.pt ? rows * I : rows * (q.bm == 16 ? align_up(I, 64) : I) * 2;
@@ -154,12 +159,18 @@ moe_status_t make_plan(const moe_problem_t* p, Plan* pl) {
   // fp32 [rows, I/128]; on the swapped-operand GEMMs: codes and scales together (132 bytes
   // per row per 128 columns); MXFP8: codes (128-column chunks) and scales, 1024 bytes per 16
   // rows per 128 columns (a group's scale blocks sit at its first row / 16)
-  L.actq = take(fp8_tiles || q.mx ? rows * I : (b128 ? rows * (I / 128) * moe::kB128RowBytesPerChunk : 0));
-  L.act_scale = take(fp8_tiles ? rows * (I / 128) * 4 : (q.mx ? rows / 16 * (I / 128) * 1024 : 0));
+  // NVFP4: packed codes (256-value chunks) and scale blocks, 2048 bytes per 16 rows per 256
+  // columns (a group's blocks sit at its first row / 16)
+  L.actq = take(fp8_tiles || q.mx ? rows * I
+                                  : (b128 ? rows * (I / 128) * moe::kB128RowBytesPerChunk : (q.nv ? rows * I / 2 : 0)));
+  L.act_scale = take(fp8_tiles ? rows * (I / 128) * 4
+                               : (q.mx ? rows / 16 * (I / 128) * 1024
+                                       : (q.nv ? rows / 16 * (I / 256) * moe::kNvChunkScaleBytes : 0)));
   L.y = take(rows * H * 4);
-  L.xs = take(q.bm == 16 ? (b128 ? rows * (H / 128) * moe::kB128RowBytesPerChunk : rows * H * (q.pt || q.mx ? 1 : 2))
+  L.xs = take(q.bm == 16 ? (b128 ? rows * (H / 128) * moe::kB128RowBytesPerChunk
+                                : (q.nv ? rows * H / 2 : rows * H * (q.pt || q.mx ? 1 : 2)))
                          : 0);
-  L.xs_scale = take(q.mx ? rows / 16 * (H / 128) * 1024 : 0);
+  L.xs_scale = take(q.mx ? rows / 16 * (H / 128) * 1024 : (q.nv ? rows / 16 * (H / 256) * moe::kNvChunkScaleBytes : 0));
   L.group_info = take(q.bm == 16 ? (rows / 16 + 1) * 8 : 0);
   L.io_hidden = take(T * H * 2);
   L.io_logits = take(T * static_cast<size_t>(q.Er) * 4);
@@ -266,6 +277,9 @@ moe_status_t run_align(const Plan& pl, void* ws, const Launch& l) {
 
 moe_status_t run_quant_act(const Plan& pl, const void* hidden, void* ws, const Launch& l) {
   const auto& L = pl.lay;
+  if (pl.nv)
+    return cuda_status(moe::launch_quant_rows_nvfp4(l, hidden, pl.T, pl.H, pl.in_scale, ws_ptr<void>(ws, L.xq),
+                                                    ws_ptr<void>(ws, L.xq_scale)));
   return cuda_status(moe::launch_quant_act(l, hidden, pl.T, pl.H, ws_ptr<void>(ws, L.xq),
                                            ws_ptr<float>(ws, L.xq_scale)));
 }
@@ -331,6 +345,18 @@ moe_status_t run_gemm1(const Plan& pl_in, const void* hidden, const void* w13, c
     o.w_scale = w13_scale;
     o.in_scale = pl.in_scale;
     o.act_scale = pl.act_scale;
+    if (pl.nv) {
+      // NVFP4: the codes and then the scale blocks in the prepared weights; GEMM1 writes the
+      // bf16 activation, quantised with the activation scale for GEMM2
+      o.nv = 1;
+      o.w_sf = static_cast<const uint8_t*>(w13) + moe::tiled_weight_bytes_u8(pl.E, pl.N1, pl.H / 2);
+      o.x_sf = ws_ptr<void>(ws, L.xs_scale);
+      moe_status_t st = cuda_status(moe::launch_gemm_swap(l, 0, o, s, b));
+      if (st != MOE_OK) return st;
+      return cuda_status(moe::launch_act_quant_nvfp4(l, ws_ptr<void>(ws, L.act), pl.I, pl.act_scale,
+                                                     ws_ptr<int>(ws, L.num_blocks) + 1, ws_ptr<int2>(ws, L.group_info),
+                                                     ws_ptr<void>(ws, L.actq), ws_ptr<void>(ws, L.act_scale), num_sms));
+    }
     if (pl.fp8) {
       // FP8 block-128: GEMM1 writes the bf16 activation, then quantised per 1x128 for GEMM2
       o.b128 = 1;
@@ -397,6 +423,11 @@ moe_status_t run_permute(const Plan& pl, const void* hidden, void* ws, const Lau
         l, ws_ptr<void>(ws, L.xq), ws_ptr<float>(ws, L.xq_scale), pl.H, ws_ptr<int>(ws, L.sorted_pair_ids),
         ws_ptr<int>(ws, L.num_blocks) + 1, ws_ptr<int2>(ws, L.group_info), static_cast<int>(pl.P), pl.kk,
         ws_ptr<void>(ws, L.xs), num_sms));
+  if (pl.nv)
+    return cuda_status(moe::launch_permute_nvfp4_rows(
+        l, ws_ptr<void>(ws, L.xq), ws_ptr<void>(ws, L.xq_scale), pl.H, ws_ptr<int>(ws, L.sorted_pair_ids),
+        ws_ptr<int>(ws, L.num_blocks) + 1, ws_ptr<int2>(ws, L.group_info), static_cast<int>(pl.P), pl.kk,
+        ws_ptr<void>(ws, L.xs), ws_ptr<void>(ws, L.xs_scale), num_sms));
   if (pl.mx)
     return cuda_status(moe::launch_permute_mx_rows(
         l, hidden, pl.H, ws_ptr<int>(ws, L.sorted_pair_ids), ws_ptr<int>(ws, L.num_blocks) + 1,
@@ -443,6 +474,12 @@ moe_status_t run_gemm2(const Plan& pl_in, const void* w2, const float* w2_scale,
     if (pl.fp8) {
       o.b128 = 1;
       o.x = ws_ptr<void>(ws, L.actq);
+    }
+    if (pl.nv) {
+      o.nv = 1;
+      o.x = ws_ptr<void>(ws, L.actq);
+      o.w_sf = static_cast<const uint8_t*>(w2) + moe::tiled_weight_bytes_u8(pl.E, pl.H, pl.I / 2);
+      o.x_sf = ws_ptr<void>(ws, L.act_scale);
     }
     if (pl.mx) {
       o.mx = 1;
@@ -502,7 +539,7 @@ Launch launch_of(const moe_problem_t* p, moe_stream_t stream) {
 moe_status_t forward_after_route(const Plan& pl, const Launch& l, const void* hidden, const void* w13, const void* w2,
                                  const float* s13, const float* s2, void* out, void* ws, int num_sms) {
   moe_status_t st = run_align(pl, ws, l);
-  if (st == MOE_OK && pl.fp8) st = run_quant_act(pl, hidden, ws, l);
+  if (st == MOE_OK && (pl.fp8 || pl.nv)) st = run_quant_act(pl, hidden, ws, l);
   if (st == MOE_OK) st = run_permute(pl, hidden, ws, l, num_sms);
   if (st == MOE_OK) st = run_gemm1(pl, hidden, w13, s13, ws, l, num_sms);
   if (st == MOE_OK) st = run_gemm2(pl, w2, s2, ws, l, num_sms);
@@ -557,9 +594,9 @@ MOE_API int32_t moe_padded_intermediate(int32_t intermediate, int32_t activation
       activation != MOE_ACT_SWIGLUOAI)
     return -1;
   if (wdtype != MOE_DTYPE_BF16 && wdtype != MOE_DTYPE_FP8_BLOCK128 && wdtype != MOE_DTYPE_FP8_PER_TENSOR &&
-      wdtype != MOE_DTYPE_MXFP8)
+      wdtype != MOE_DTYPE_MXFP8 && wdtype != MOE_DTYPE_NVFP4)
     return -1;
-  const int a = (wdtype != MOE_DTYPE_BF16 || activation == MOE_ACT_RELU2) ? 128 : 16;
+  const int a = wdtype == MOE_DTYPE_NVFP4 ? 256 : ((wdtype != MOE_DTYPE_BF16 || activation == MOE_ACT_RELU2) ? 128 : 16);
   return (intermediate + a - 1) / a * a;
 }
 
@@ -582,7 +619,7 @@ MOE_API moe_status_t moe_prepare_weights(const moe_problem_t* problem, int32_t i
   Plan pl;
   moe_status_t st = make_plan(problem, &pl);  // num_tokens plays no part in weight preparation
   if (st != MOE_OK) return st;
-  if (pl.mx) return MOE_ERR_INVALID_ARG;  // MXFP8 weights carry scales: moe_prepare_weights_mxfp8
+  if (pl.mx || pl.nv) return MOE_ERR_INVALID_ARG;  // block-scaled weights: moe_prepare_weights_mxfp8 / _nvfp4
   if (moe_padded_intermediate(intermediate_in, pl.act, problem->wdtype) != pl.I) return MOE_ERR_INVALID_ARG;
   if (pl.q8 && intermediate_in != pl.I) return MOE_ERR_INVALID_ARG;
   if (!aligned16(w13_in) || !aligned16(w13_out) || w2_in == nullptr || w2_out == nullptr)
@@ -618,6 +655,10 @@ MOE_API size_t moe_prepared_weights_bytes(const moe_problem_t* problem, int32_t 
   if (pl.mx)
     return which == 0 ? moe::tiled_weight_bytes_u8(pl.E, pl.N1, pl.H) + moe::tiled_scale_bytes_mx(pl.E, pl.N1, pl.H)
                       : moe::tiled_weight_bytes_u8(pl.E, pl.H, pl.I) + moe::tiled_scale_bytes_mx(pl.E, pl.H, pl.I);
+  if (pl.nv)
+    return which == 0
+               ? moe::tiled_weight_bytes_u8(pl.E, pl.N1, pl.H / 2) + moe::tiled_scale_bytes_nvfp4(pl.E, pl.N1, pl.H)
+               : moe::tiled_weight_bytes_u8(pl.E, pl.H, pl.I / 2) + moe::tiled_scale_bytes_nvfp4(pl.E, pl.H, pl.I);
   if (pl.pt || (pl.fp8 && pl.bm == 16))
     return which == 0 ? moe::tiled_weight_bytes_u8(pl.E, pl.N1, pl.H) : moe::tiled_weight_bytes_u8(pl.E, pl.H, pl.I);
   if (pl.bm == 16)
@@ -651,6 +692,48 @@ MOE_API moe_status_t moe_prepare_weights_mxfp8(const moe_problem_t* problem, con
     e = moe::launch_tile_scales_mx(l, 1, w2_scales, o2 + moe::tiled_weight_bytes_u8(pl.E, pl.H, pl.I), pl.E, pl.H,
                                    pl.I, pl.gated);
   return cuda_status(e);
+}
+
+MOE_API moe_status_t moe_prepare_weights_nvfp4(const moe_problem_t* problem, const void* w13_codes,
+                                               const void* w13_scales, const void* w2_codes, const void* w2_scales,
+                                               void* w13_out, void* w2_out, moe_stream_t stream) {
+  Plan pl;
+  moe_status_t st = make_plan(problem, &pl);  // num_tokens plays no part in weight preparation
+  if (st != MOE_OK) return st;
+  if (!pl.nv) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(w13_codes) || !aligned16(w2_codes) || !aligned16(w13_out) || !aligned16(w2_out) ||
+      w13_scales == nullptr || w2_scales == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  int sms = 0;
+  st = device_sms(&sms);
+  if (st != MOE_OK) return st;
+  const Launch l = launch_of(problem, stream);
+  uint8_t* o13 = static_cast<uint8_t*>(w13_out);
+  uint8_t* o2 = static_cast<uint8_t*>(w2_out);
+  cudaError_t e = moe::launch_tile_weights_u8(l, 0, w13_codes, o13, pl.E, pl.H, pl.I, pl.gated, 2);
+  if (e == cudaSuccess) e = moe::launch_tile_weights_u8(l, 1, w2_codes, o2, pl.E, pl.H, pl.I, pl.gated, 2);
+  if (e == cudaSuccess)
+    e = moe::launch_tile_scales_nvfp4(l, 0, w13_scales, o13 + moe::tiled_weight_bytes_u8(pl.E, pl.N1, pl.H / 2), pl.E,
+                                      pl.H, pl.I, pl.gated);
+  if (e == cudaSuccess)
+    e = moe::launch_tile_scales_nvfp4(l, 1, w2_scales, o2 + moe::tiled_weight_bytes_u8(pl.E, pl.H, pl.I / 2), pl.E,
+                                      pl.H, pl.I, pl.gated);
+  return cuda_status(e);
+}
+
+MOE_API moe_status_t moe_quantize_weights_nvfp4(const void* w, int64_t num_mats, int32_t rows, int32_t cols,
+                                                void* codes, void* scales, float* global_scales, moe_stream_t stream) {
+  if (num_mats < 0 || num_mats > 65535 || rows <= 0 || cols <= 0 || cols % 16 != 0) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(w) || !aligned16(codes) || scales == nullptr || !aligned4(global_scales)) return MOE_ERR_INVALID_ARG;
+  if (num_mats == 0) return MOE_OK;
+  int sms = 0;
+  moe_status_t st = device_sms(&sms);
+  if (st != MOE_OK) return st;
+  Launch l;
+  l.stream = reinterpret_cast<cudaStream_t>(stream);
+  l.pdl = false;
+  return cuda_status(moe::launch_quant_weights_nvfp4(l, w, num_mats, static_cast<int64_t>(rows) * cols, codes, scales,
+                                                     global_scales));
 }
 
 MOE_API moe_status_t moe_quantize_weights_mxfp8(const void* w, int64_t num_mats, int32_t rows, int32_t cols,
@@ -797,7 +880,7 @@ MOE_API moe_status_t moe_stage_quant_act(const moe_problem_t* problem, const voi
   int sms = 0;
   moe_status_t st = make_plan(problem, &pl);
   if (st != MOE_OK || pl.T == 0) return st;  // T == 0: nothing to do, pointers unused
-  if (!pl.fp8 || !aligned16(hidden)) return MOE_ERR_INVALID_ARG;
+  if (!(pl.fp8 || pl.nv) || !aligned16(hidden)) return MOE_ERR_INVALID_ARG;
   st = prologue(problem, workspace, workspace_bytes, &pl, &sms);
   if (st != MOE_OK || pl.T == 0) return st;
   return run_quant_act(pl, hidden, workspace, launch_of(problem, stream));

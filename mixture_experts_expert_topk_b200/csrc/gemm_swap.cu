@@ -67,6 +67,16 @@
 // threads' registers.
 // GEMM1 writes the bf16 activation, which a separate pass quantises per 1x128 for GEMM2.
 //
+// NVFP4 (packed E2M1 operands, one E4M3 scale per 16 values of K on both operands, an fp32
+// scale per tensor; NVIDIA's NVFP4, named by "FlashInfer gated MoE kernel optimisation for
+// Blackwell", section 4): tcgen05.mma kind::mxf4nvf4.block_scale.scale_vec::4X applies the
+// block scales inside the MMA. A 128-byte chunk row holds 256 values: four MMAs of K = 64,
+// each reading four TMEM scale columns per operand (row r's four block scales in lane
+// r % 32, column r / 32, one byte per block). Each K step (at most two chunks) carries the
+// W and X scale blocks (2 KB per chunk each) after its codes; the MMA thread copies them to
+// TMEM with tcgen05.cp. The epilogue multiplies by the two tensor scales (the expert's
+// weight scale and the static input / activation scale). Row groups have at most 128 rows.
+//
 // One persistent CTA per SM, 7 warps:
 //   warp 0      scheduler (tiles from a global atomic counter, published to the other
 //               roles through a shared-memory ring) and W copies;
@@ -105,6 +115,10 @@ constexpr int kSfBufs = 4;
 constexpr int kSfBufCols = 32;
 constexpr int kSfCol0 = 2 * kMxAccCols;
 static_assert(kSfCol0 + kSfBufs * kSfBufCols <= static_cast<int>(kTmemCols), "TMEM columns");
+// NVFP4: the same four scale buffers, 64 columns each (two chunks of 16 W and 16 X columns)
+constexpr int kNvSfCol0 = 2 * kNvGroupRows;
+constexpr int kNvSfBufCols = 64;
+static_assert(kNvSfCol0 + kSfBufs * kNvSfBufCols <= static_cast<int>(kTmemCols), "TMEM columns");
 // FP8 block-128: partial-product buffers in TMEM (one per K chunk in flight)
 constexpr int kPartBufs = 4;
 constexpr int kPartCols = kB128GroupRows;
@@ -169,7 +183,13 @@ template <int kKind>
 __device__ __forceinline__ uint32_t step_bytes(int kcs, int n) {
   const uint32_t b = static_cast<uint32_t>(kcs) * (kTileW + n * kChunkBytes);
   if (kKind == 2) return (b + static_cast<uint32_t>(kcs) * (kSfW + kSfX) + 1023u) & ~1023u;
+  if (kKind == 4) return b + static_cast<uint32_t>(kcs) * 2u * kNvChunkScaleBytes;
   return b;
+}
+// K chunks per step: NVFP4 steps take at most two (their scale buffers hold two chunks)
+template <int kKind>
+__device__ __forceinline__ int step_chunks(int n) {
+  return kKind == 4 ? min(chunks_per_step(n), 2) : chunks_per_step(n);
 }
 static_assert(4 * (kTileW + 32 * kChunkBytes + kSfW + kSfX) <= kRingBytes / 2 &&
                   kTileW + kMxGroupRows * kChunkBytes + kSfW + kSfX <= kRingBytes / 2,
@@ -235,14 +255,15 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
       : "memory");
 }
 
-// kKind: 0 bf16, 1 per-tensor e4m3, 2 MXFP8, 3 FP8 block-128.
+// kKind: 0 bf16, 1 per-tensor e4m3, 2 MXFP8, 3 FP8 block-128, 4 NVFP4.
 template <int kKind>
 __global__ void __launch_bounds__(threads_for<kKind>(), 1) gemm_swap_kernel(const Args a) {
   constexpr bool kFp8 = kKind == 1;  // scales applied in the epilogue
   constexpr bool kMx = kKind == 2;   // scales applied by the MMA
   constexpr bool kB128 = kKind == 3; // a partial per K chunk, promoted in the epilogue
   constexpr bool kE4m3 = kFp8 || kB128;
-  constexpr int kAccCols = kMx ? kMxAccCols : kNMax;
+  constexpr bool kNv = kKind == 4;   // block scales applied by the MMA, tensor scales in the epilogue
+  constexpr int kAccCols = kMx ? kMxAccCols : (kNv ? kNvGroupRows : kNMax);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -340,7 +361,7 @@ __global__ void __launch_bounds__(threads_for<kKind>(), 1) gemm_swap_kernel(cons
         }
         if (n == 0) break;
         const int next = atomicAdd(a.tile_counter, 1);  // its latency overlaps the loads
-        const int kc = chunks_per_step(n);
+        const int kc = step_chunks<kKind>(n);
         const uint8_t* wsrc = a.w + (static_cast<size_t>(e) * a.m_tiles + mt) * a.k_chunks * kTileW;
         for (int c0 = 0; c0 < a.k_chunks; c0 += kc, ++ks) {
           const int kcs = min(kc, a.k_chunks - c0);
@@ -351,12 +372,13 @@ __global__ void __launch_bounds__(threads_for<kKind>(), 1) gemm_swap_kernel(cons
           }
           const uint32_t full = full0 + 8 * (ks % kSlots);
           const uint32_t bytes = static_cast<uint32_t>(kcs) * kTileW;
-          const uint32_t sf_bytes = kMx ? static_cast<uint32_t>(kcs) * kSfW : 0u;
+          constexpr uint32_t kWsf = kMx ? kSfW : (kNv ? kNvChunkScaleBytes : 0u);  // W scale bytes per chunk
+          const uint32_t sf_bytes = static_cast<uint32_t>(kcs) * kWsf;
           mbar_arrive_expect_tx(full, bytes + sf_bytes);
           bulk_load(s0 + off, wsrc + static_cast<size_t>(c0) * kTileW, bytes, full, pol);
-          if constexpr (kMx)
+          if constexpr (kMx || kNv)
             bulk_load(s0 + off + static_cast<uint32_t>(kcs) * (kTileW + n * kChunkBytes),
-                      a.w_sf + ((static_cast<size_t>(e) * a.m_tiles + mt) * a.k_chunks + c0) * kSfW, sf_bytes, full,
+                      a.w_sf + ((static_cast<size_t>(e) * a.m_tiles + mt) * a.k_chunks + c0) * kWsf, sf_bytes, full,
                       pol);
         }
         tile = next;
@@ -375,7 +397,7 @@ __global__ void __launch_bounds__(threads_for<kKind>(), 1) gemm_swap_kernel(cons
         int4 t;
         if (!ring_read(rfull0, rempty0, ring, rslot, rph, abort_flag, a.status, t) || t.y == 0) break;
         const int x_row = t.x, n = t.y;
-        const int kc = chunks_per_step(n);
+        const int kc = step_chunks<kKind>(n);
         const uint8_t* xsrc = a.x + static_cast<size_t>(x_row) * x_row_bytes;
         for (int c0 = 0; c0 < a.k_chunks; c0 += kc, ++ks) {
           const int kcs = min(kc, a.k_chunks - c0);
@@ -388,7 +410,9 @@ __global__ void __launch_bounds__(threads_for<kKind>(), 1) gemm_swap_kernel(cons
           const uint32_t bytes = static_cast<uint32_t>(kcs * n) * kChunkBytes;
           // MXFP8: the scale blocks; FP8 block-128: the rows' scales, stored right behind
           // the step's codes, into a slot of the X scale ring once the epilogue freed it
-          const uint32_t sf_bytes = kMx ? static_cast<uint32_t>(kcs) * kSfX : (kB128 ? static_cast<uint32_t>(kcs * n) * 4u : 0u);
+          const uint32_t sf_bytes = kMx ? static_cast<uint32_t>(kcs) * kSfX
+                                        : (kNv ? static_cast<uint32_t>(kcs) * kNvChunkScaleBytes
+                                               : (kB128 ? static_cast<uint32_t>(kcs * n) * 4u : 0u));
           if (kB128 && !mbar_wait(sxfree0 + 8 * (ks % kSxSlots), ((ks / kSxSlots) & 1u) ^ 1u, abort_flag, a.status,
                                   kSiteSxFree)) {
             ok = false;
@@ -401,6 +425,10 @@ __global__ void __launch_bounds__(threads_for<kKind>(), 1) gemm_swap_kernel(cons
           if constexpr (kMx)
             bulk_load(s0 + off + static_cast<uint32_t>(kcs) * (kTileW + n * kChunkBytes + kSfW),
                       a.x_sf + (static_cast<size_t>(x_row >> 4) * a.k_chunks + c0) * kSfX, sf_bytes, full, pol);
+          if constexpr (kNv)
+            bulk_load(s0 + off + static_cast<uint32_t>(kcs) * (kTileW + n * kChunkBytes + kNvChunkScaleBytes),
+                      a.x_sf + (static_cast<size_t>(x_row >> 4) * a.k_chunks + c0) * kNvChunkScaleBytes, sf_bytes,
+                      full, pol);
         }
       }
       drain_fills(fullx0, kSlots, ks);  // no X copy may land after the CTA exits
@@ -415,12 +443,13 @@ __global__ void __launch_bounds__(threads_for<kKind>(), 1) gemm_swap_kernel(cons
         int4 t;
         if (!ring_read(rfull0, rempty0, ring, rslot, rph, abort_flag, a.status, t) || t.y == 0) break;
         const int n = t.y;
-        const int kc = chunks_per_step(n);
+        const int kc = step_chunks<kKind>(n);
         const int acc = it & 1;
         if (!kB128 && !mbar_wait(tempty0 + 8 * acc, ((it >> 1) & 1) ^ 1u, abort_flag, a.status, kSiteTmemEmpty)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * kAccCols;
-        const uint32_t idesc = kMx ? idesc_mx(kMW, n) : (kE4m3 ? idesc_e4m3(kMW, n) : idesc_bf16(kMW, n));
+        const uint32_t idesc =
+            kMx ? idesc_mx(kMW, n) : (kNv ? idesc_nvf4(kMW, n) : (kE4m3 ? idesc_e4m3(kMW, n) : idesc_bf16(kMW, n)));
         bool ok = true;
         for (int c0 = 0; c0 < a.k_chunks; c0 += kc, ++ks) {
           const int kcs = min(kc, a.k_chunks - c0);
@@ -460,6 +489,32 @@ __global__ void __launch_bounds__(threads_for<kKind>(), 1) gemm_swap_kernel(cons
               if (c < kcs)
                 umma_mx_chunk(d_tmem, a_lo + c * (kTileW >> 4), b_lo + c * b_step, idesc, sf_t + 4 * c,
                               sf_t + 4 * kcs + 4 * nb * c, (c0 != 0 || c != 0) ? 1u : 0u);
+          } else if (kNv) {
+            // the scale buffer of this step was last read by the MMAs of step ks - kSfBufs
+            if (ks >= static_cast<uint32_t>(kSfBufs) &&
+                !mbar_wait(empty0 + 8 * ((ks - kSfBufs) % kSlots), ((ks - kSfBufs) / kSlots) & 1u, abort_flag,
+                           a.status, kSiteSfFree)) {
+              ok = false;
+              break;
+            }
+            const uint32_t sf_s = base + static_cast<uint32_t>(kcs) * (kTileW + n * kChunkBytes);
+            const uint32_t sf_t = tmem_base + kNvSfCol0 + (ks % kSfBufs) * kNvSfBufCols;
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              if (c < kcs) {
+#pragma unroll
+                for (int mm = 0; mm < 4; ++mm) {
+                  tmem_cp_sf(sf_t + 16 * c + 4 * mm, sf_s + c * kNvChunkScaleBytes + mm * 512);
+                  tmem_cp_sf(sf_t + 32 + 16 * c + 4 * mm,
+                             sf_s + (kcs + c) * kNvChunkScaleBytes + mm * 512);
+                }
+              }
+            }
+#pragma unroll
+            for (int c = 0; c < 2; ++c)
+              if (c < kcs)
+                umma_nvf4_chunk(d_tmem, a_lo + c * (kTileW >> 4), b_lo + c * b_step, idesc, sf_t + 16 * c,
+                                sf_t + 32 + 16 * c, (c0 != 0 || c != 0) ? 1u : 0u);
           } else if (kB128) {
             // one fresh partial per K chunk, into the next free buffer
             for (int c = 0; c < kcs; ++c, ++pc) {
@@ -516,8 +571,9 @@ __global__ void __launch_bounds__(threads_for<kKind>(), 1) gemm_swap_kernel(cons
       const int x_row = __shfl_sync(0xffffffffu, t.x, 0);
       const int expert = __shfl_sync(0xffffffffu, t.z, 0);
       const int mt = __shfl_sync(0xffffffffu, t.w, 0);
-      // FP8 per-tensor: the accumulator's dequantisation scale (GEMM1: before the activation)
-      const float dq = kFp8 ? __ldg(a.w_scale + expert) * a.in_scale : 1.0f;
+      // FP8 per-tensor, NVFP4: the accumulator's dequantisation scale (the weight's and the
+      // X operand's tensor scales; GEMM1: before the activation)
+      const float dq = (kFp8 || kNv) ? __ldg(a.w_scale + expert) * a.in_scale : 1.0f;
       // GEMM1: this lane's activation feature f lies in K chunk f / 64 (bf16) or f / 128
       // (e4m3) of the activation; byte b of a 128-byte chunk row sits in 16-byte piece
       // (b / 16) ^ (row % 8)
@@ -590,7 +646,7 @@ __global__ void __launch_bounds__(threads_for<kKind>(), 1) gemm_swap_kernel(cons
 
       if constexpr (kB128) {
         // promote each K chunk's partial: acc[j] += partial[j] * s_w * s_x[j]
-        const int kc = chunks_per_step(n);
+        const int kc = step_chunks<kKind>(n);
         // the tile's weight scales, lane k holding K chunk k (k_chunks <= 32): gated GEMM1's
         // even lanes are gate rows (block row mt / 2), its odd lanes up rows
         const float* sw_e = a.w_scale + static_cast<size_t>(expert) * a.ws_rows * a.k_chunks;
@@ -712,7 +768,7 @@ __global__ void __launch_bounds__(threads_for<kKind>(), 1) gemm_swap_kernel(cons
   }
 }
 
-bool g_attr_set[4][64] = {};
+bool g_attr_set[5][64] = {};
 
 }  // namespace
 
@@ -722,17 +778,18 @@ cudaError_t launch_gemm_swap(const Launch& l, int mode, const SwapOperands& o, c
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  const int kind = o.b128 ? 3 : (o.mx ? 2 : (o.fp8 ? 1 : 0));
+  const int kind = o.nv ? 4 : (o.b128 ? 3 : (o.mx ? 2 : (o.fp8 ? 1 : 0)));
   void (*const kernel)(const Args) =
-      kind == 3 ? gemm_swap_kernel<3>
-                : (kind == 2 ? gemm_swap_kernel<2> : (kind == 1 ? gemm_swap_kernel<1> : gemm_swap_kernel<0>));
+      kind == 4 ? gemm_swap_kernel<4>
+                : (kind == 3 ? gemm_swap_kernel<3>
+                             : (kind == 2 ? gemm_swap_kernel<2> : (kind == 1 ? gemm_swap_kernel<1> : gemm_swap_kernel<0>)));
   if (!g_attr_set[kind][dev]) {
     err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (err != cudaSuccess) return err;
     g_attr_set[kind][dev] = true;
   }
   if ((reinterpret_cast<uintptr_t>(o.w) | reinterpret_cast<uintptr_t>(o.x)) & 15u) return cudaErrorInvalidValue;
-  if (kind == 2 && (o.w_sf == nullptr || o.x_sf == nullptr ||
+  if ((kind == 2 || kind == 4) && (o.w_sf == nullptr || o.x_sf == nullptr ||
                     ((reinterpret_cast<uintptr_t>(o.w_sf) | reinterpret_cast<uintptr_t>(o.x_sf)) & 15u)))
     return cudaErrorInvalidValue;
   // FP8 block-128: K and the weight rows whole 128-blocks, the K chunks' weight scales held
@@ -742,7 +799,8 @@ cudaError_t launch_gemm_swap(const Launch& l, int mode, const SwapOperands& o, c
   Args a;
   a.mode = mode;
   a.m_tiles = (s.N + kMW - 1) / kMW;
-  const int chunk_elems = kind != 0 ? 128 : 64;  // elements of K in a 128-byte chunk
+  if (kind == 4 && (o.w_scale == nullptr || s.K % 256 != 0)) return cudaErrorInvalidValue;
+  const int chunk_elems = kind == 4 ? 256 : (kind != 0 ? 128 : 64);  // elements of K in a 128-byte chunk
   a.k_chunks = (s.K + chunk_elems - 1) / chunk_elems;
   a.k_total = s.k_total;
   a.num_pairs = s.num_pairs;

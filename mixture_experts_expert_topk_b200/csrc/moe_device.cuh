@@ -5,6 +5,8 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp4.h>
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -442,6 +444,74 @@ __device__ __forceinline__ void umma_mx_chunk(uint32_t d_tmem, uint32_t a_lo, ui
       "add.u32 al, %1, 6;\n\tadd.u32 bl, %2, 6;\n\tmov.b64 a, {al, %5};\n\tmov.b64 b, {bl, %5};\n\t"
       "or.b32 id, %3, 0x60000030;\n\t"
       "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], a, b, id, [%6], [%7], q;\n\t}" ::"r"(d_tmem),
+      "r"(a_lo), "r"(b_lo), "r"(idesc), "r"(accumulate), "n"(kUmmaDescHi), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
+// ---- NVFP4 (E2M1 values, one E4M3 scale per 16 values, one fp32 scale per tensor) ----
+
+// Per-tensor decode scale from the tensor's largest magnitude: amax / (6 * 448), so that
+// every block scale fits E4M3 (IEEE division); 1 for an all-zero tensor.
+__device__ __forceinline__ float nvfp4_tensor_scale(float amax) { return amax == 0.f ? 1.f : __fdiv_rn(amax, 2688.f); }
+// E4M3 code of the block scale of 16 values with largest magnitude amax under the tensor
+// scale g: e4m3(amax / 6 / g), two IEEE divisions, round to nearest even, saturating.
+__device__ __forceinline__ uint8_t nvfp4_block_scale(float amax, float g) {
+  return __nv_cvt_float_to_fp8(__fdiv_rn(__fdiv_rn(amax, 6.0f), g), __NV_SATFINITE, __NV_E4M3);
+}
+__device__ __forceinline__ float e4m3_value(uint8_t code) {
+  return __half2float(__half(__nv_cvt_fp8_to_halfraw(code, __NV_E4M3)));
+}
+// Two values a, b (K order) divided by d (IEEE) to E2M1, round to nearest even, saturating,
+// packed into one byte with a in the low nibble; both 0 when d is not positive.
+__device__ __forceinline__ uint32_t nvfp4_pair(float a, float b, float d) {
+  if (!(d > 0.f)) return 0u;
+  return __nv_cvt_float2_to_fp4x2(make_float2(__fdiv_rn(a, d), __fdiv_rn(b, d)), __NV_E2M1, cudaRoundNearest);
+}
+// Sixteen values (one block) to NVFP4 under tensor scale g: the block's E4M3 scale code and
+// its eight code bytes packed as two words (value 2i in the low nibble of byte i).
+__device__ __forceinline__ uint8_t nvfp4_block(const float (&v)[16], float g, uint2& packed) {
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  const uint8_t s = nvfp4_block_scale(amax, g);
+  const float d = e4m3_value(s) * g;
+  uint32_t w[2] = {0u, 0u};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) w[i >> 2] |= nvfp4_pair(v[2 * i], v[2 * i + 1], d) << (8 * (i & 3));
+  packed = make_uint2(w[0], w[1]);
+  return s;
+}
+
+// Instruction descriptor for kind::mxf4nvf4.block_scale with E2M1 A/B (both K-major), fp32
+// D and UE4M3 scales (one per 16 values, scale_vec::4X: the scale-factor byte selectors are
+// 0, each MMA reads all four bytes of its scale columns).
+__host__ __device__ constexpr uint32_t idesc_nvf4(int M, int N) {
+  return (1u << 7)                                   // A format: E2M1
+         | (1u << 10)                                // B format: E2M1
+         | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8
+         | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16; bit 23 clear: UE4M3 scales
+}
+
+// One 128-byte K chunk of packed E2M1 operands (256 values): four MMAs of K = 64, MMA m
+// reading the four scale columns sfa + 4 m (A) and sfb + 4 m (B). The first accumulates
+// into D when `accumulate` is nonzero, the others always do.
+__device__ __forceinline__ void umma_nvf4_chunk(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t idesc,
+                                                uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t.reg .b32 al, bl, sa, sb;\n\t.reg .b64 a, b;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.eq.b32 q, %4, %4;\n\t"
+      "mov.b64 a, {%1, %5};\n\tmov.b64 b, {%2, %5};\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], a, b, %3, [%6], [%7], p;\n\t"
+      "add.u32 al, %1, 2;\n\tadd.u32 bl, %2, 2;\n\tmov.b64 a, {al, %5};\n\tmov.b64 b, {bl, %5};\n\t"
+      "add.u32 sa, %6, 4;\n\tadd.u32 sb, %7, 4;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], a, b, %3, [sa], [sb], q;\n\t"
+      "add.u32 al, %1, 4;\n\tadd.u32 bl, %2, 4;\n\tmov.b64 a, {al, %5};\n\tmov.b64 b, {bl, %5};\n\t"
+      "add.u32 sa, %6, 8;\n\tadd.u32 sb, %7, 8;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], a, b, %3, [sa], [sb], q;\n\t"
+      "add.u32 al, %1, 6;\n\tadd.u32 bl, %2, 6;\n\tmov.b64 a, {al, %5};\n\tmov.b64 b, {bl, %5};\n\t"
+      "add.u32 sa, %6, 12;\n\tadd.u32 sb, %7, 12;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], a, b, %3, [sa], [sb], q;\n\t}" ::"r"(d_tmem),
       "r"(a_lo), "r"(b_lo), "r"(idesc), "r"(accumulate), "n"(kUmmaDescHi), "r"(sfa), "r"(sfb)
       : "memory");
 }

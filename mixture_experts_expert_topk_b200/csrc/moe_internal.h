@@ -123,6 +123,10 @@ struct SwapOperands {
   // its rows (launch_permute_b128_rows, launch_act_quant_b128).
   int b128;
   int up_block;
+  // NVFP4 (packed E2M1 operands, E4M3 scales per 16 values of K applied by the MMA): nv = 1;
+  // w_sf / x_sf = the tiled weight scales / the X scale blocks (kNvChunkScaleBytes per 128-row
+  // block per chunk); w_scale [E] and in_scale the tensor scales (dequantised in the epilogue)
+  int nv;
 };
 // Row groups of the MXFP8 swapped-operand GEMMs: at most this many rows, so that two
 // accumulators leave a quarter of TMEM for the block scales.
@@ -176,6 +180,41 @@ cudaError_t launch_permute_mx_rows(const Launch& l, const void* hidden, int H, c
 cudaError_t launch_act_quant_mx(const Launch& l, const void* act, int I, const int* num_groups,
                                 const int2* group_info, void* actq, void* act_sf, int num_sms);
 size_t tiled_scale_bytes_mx(int E, int rows, int K);
+
+// ---- NVFP4 (quant.cu, permute.cu, prepare.cu) ----
+// Row groups of the NVFP4 swapped-operand GEMMs: at most this many rows (two accumulators
+// leave half of TMEM for four buffers of block scales).
+constexpr int kNvGroupRows = 128;
+// Bytes of one K chunk's block scales for 128 rows: four 512-byte blocks, one per MMA of
+// K = 64 (a 128-byte chunk row holds 256 E2M1 values, sixteen 16-value blocks): byte
+// 512 m + 16 l + 4 j + k of a chunk's blocks is the scale of row 32 j + l for block 4 m + k.
+constexpr int kNvChunkScaleBytes = 2048;
+// NVFP4 weights: per matrix g = amax / (6 * 448) (1 if all zero) into global_scales[m],
+// then per block of 16 values of a row: scale e4m3(amax / 6 / g) and E2M1 codes of
+// x / (scale * g), two per byte (lower K index in the low nibble). w bf16 [num_mats,
+// mat_elems]; codes [num_mats, mat_elems / 2]; scales [num_mats, mat_elems / 16].
+cudaError_t launch_quant_weights_nvfp4(const Launch& l, const void* w, int64_t num_mats, int64_t mat_elems,
+                                       void* codes, void* scales, float* global_scales);
+// The same for rows of bf16 values with a fixed tensor scale g (the hidden rows: the input
+// scale; GEMM1's activation: the activation scale).
+cudaError_t launch_quant_rows_nvfp4(const Launch& l, const void* x, long long rows, int cols, float g, void* codes,
+                                    void* scales);
+// The token rows of every row group (quantised per token by launch_quant_rows_nvfp4: codes
+// [T, H/2], scales [T, H/16]) in row-group order: codes in 128-byte chunk rows (256 values)
+// as the per-tensor FP8 layout, scales in kNvChunkScaleBytes blocks at ((x_row / 16) *
+// (H / 256) + c) * kNvChunkScaleBytes for the group starting at sorted row x_row.
+cudaError_t launch_permute_nvfp4_rows(const Launch& l, const void* xq, const void* xq_scale, int H,
+                                      const int* sorted_pair_ids, const int* num_groups, const int2* group_info, int P,
+                                      int k_total, void* xs, void* xs_sf, int num_sms);
+// GEMM1's bf16 activation (row-group order, 64-column chunks) to NVFP4 under tensor scale g,
+// in the layout of launch_permute_nvfp4_rows with H = I, for GEMM2.
+cudaError_t launch_act_quant_nvfp4(const Launch& l, const void* act, int I, float g, const int* num_groups,
+                                   const int2* group_info, void* actq, void* act_sf, int num_sms);
+// Tiled NVFP4 weight scales beside the tiled codes: per (expert, 128-row block, 256-value
+// chunk) one kNvChunkScaleBytes block (rows interleaved like the codes for gated w13).
+size_t tiled_scale_bytes_nvfp4(int E, int rows, int K);
+cudaError_t launch_tile_scales_nvfp4(const Launch& l, int which, const void* in, void* out, int E, int H, int I,
+                                     int gated);
 cudaError_t launch_tile_scales_mx(const Launch& l, int which, const void* in, void* out, int E, int H, int I,
                                   int gated);
 
@@ -214,10 +253,11 @@ size_t tiled_weight_bytes(int E, int rows, int K);
 cudaError_t launch_tile_weights(const Launch& l, int which, const void* in, void* out, int E, int H, int I_in,
                                 int I_pad, int gated);
 // The same for e4m3 codes (1 byte, 128 elements per 128-byte chunk row): tiles of 128 rows x
-// 128 columns; tiled_weight_bytes_u8 gives the size.
+// 128 bytes; tiled_weight_bytes_u8 gives the size (rows, K bytes). k_div = 2 tiles packed
+// E2M1 codes (two values per byte: 256 values per chunk row, K bytes = K / 2).
 size_t tiled_weight_bytes_u8(int E, int rows, int K);
 cudaError_t launch_tile_weights_u8(const Launch& l, int which, const void* in, void* out, int E, int H, int I,
-                                   int gated);
+                                   int gated, int k_div = 1);
 // Per-tensor FP8 weight quantisation of num_mats bf16 [rows, cols] matrices: scale = amax
 // / 448 per matrix (1 for all zeros), codes = e4m3(w / scale).
 cudaError_t launch_quant_weights_per_tensor(const Launch& l, const void* w, int64_t num_mats, int64_t mat_elems,

@@ -384,7 +384,129 @@ __global__ void __launch_bounds__(kThreads)
   }
 }
 
+// NVFP4: the token rows, quantised once per token (codes [T, H/2], scales [T, H/16]),
+// copied into their row groups: codes as 128-byte chunk rows (256 values, swizzled like the
+// other 8-bit layouts), scales into the group's 2048-byte block per chunk (byte 512 mm +
+// 16 (j % 32) + 4 (j / 32) + k: group row j, 16-value block 16 c + 4 mm + k). A warp copies
+// one row; lane l moves 16-byte code pieces l, l + 32, ... and the row's scale bytes 4l..4l+3
+// (blocks 4l..4l+3: one MMA's four). Padding rows are zero codes and zero scales.
+__global__ void __launch_bounds__(kThreads)
+    permute_nvfp4_rows_kernel(const uint4* __restrict__ xq, const uint8_t* __restrict__ xq_scale, int H,
+                              const int* __restrict__ sorted_pair_ids, const int* __restrict__ num_groups,
+                              const int2* __restrict__ group_info, int P, int k_total, uint8_t* __restrict__ xs,
+                              uint8_t* __restrict__ xs_sf) {
+  griddep_wait();
+  griddep_launch_dependents();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int G = *num_groups;
+  const int KC = H / 256, pieces = H / 32, sbytes = H / 16;
+  for (int g = blockIdx.x; g < G; g += gridDim.x) {
+    const int2 gi = group_info[g];
+    const int x_row = gi.x, n = gi.y >> 16;
+    uint8_t* base = xs + static_cast<size_t>(x_row) * KC * 128;
+    uint8_t* sfb = xs_sf + static_cast<size_t>(x_row >> 4) * KC * kNvChunkScaleBytes;
+    for (int j = blockIdx.y * (kThreads / 32) + warp; j < n; j += gridDim.y * (kThreads / 32)) {
+      const int pid = sorted_pair_ids[x_row + j];
+      const long long tok = pid < P ? pid / k_total : -1;
+      for (int p0 = 0; p0 < pieces; p0 += 32 * kB128Pieces) {
+        uint4 v[kB128Pieces];
+#pragma unroll
+        for (int i = 0; i < kB128Pieces; ++i) {
+          const int p = p0 + lane + 32 * i;
+          v[i] = (tok >= 0 && p < pieces) ? __ldg(xq + tok * pieces + p) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int i = 0; i < kB128Pieces; ++i) {
+          const int p = p0 + lane + 32 * i;
+          if (p < pieces)
+            *reinterpret_cast<uint4*>(base + static_cast<size_t>(p >> 3) * n * 128 + j * 128 +
+                                      ((((p & 7) ^ j) & 7) << 4)) = v[i];
+        }
+      }
+      for (int b0 = 4 * lane; b0 < sbytes; b0 += 128) {
+        const uint32_t w = tok >= 0 ? __ldg(reinterpret_cast<const uint32_t*>(xq_scale + tok * sbytes + b0)) : 0u;
+        const int c = b0 >> 4, mm = (b0 >> 2) & 3;
+        *reinterpret_cast<uint32_t*>(sfb + static_cast<size_t>(c) * kNvChunkScaleBytes + mm * 512 + 16 * (j & 31) +
+                                     4 * (j >> 5)) = w;
+      }
+    }
+  }
+}
+
+// NVFP4: GEMM1's bf16 activation (64-column chunks of 128-byte rows, row-group order)
+// quantised with tensor scale g into the layout of permute_nvfp4_rows_kernel. A warp takes
+// one (row, 256-column chunk): lane l converts columns 8l..8l+7 (16 bytes of bf16 chunk
+// 4c + l / 8); lanes 2b and 2b+1 share 16-value block b and exchange their maxima.
+__global__ void __launch_bounds__(kThreads)
+    act_quant_nvfp4_kernel(const uint8_t* __restrict__ act, int I, float g, const int* __restrict__ num_groups,
+                           const int2* __restrict__ group_info, uint8_t* __restrict__ actq, uint8_t* __restrict__ act_sf) {
+  griddep_wait();
+  griddep_launch_dependents();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int G = *num_groups;
+  const int KCb = I / 64, KC = I / 256;
+  const int warps = gridDim.y * (kThreads / 32);
+  for (int gr = blockIdx.x; gr < G; gr += gridDim.x) {
+    const int2 gi = group_info[gr];
+    const int x_row = gi.x, n = gi.y >> 16;
+    const uint8_t* in = act + static_cast<size_t>(x_row) * KCb * 128;
+    uint8_t* out = actq + static_cast<size_t>(x_row) * KC * 128;
+    uint8_t* sf = act_sf + static_cast<size_t>(x_row >> 4) * KC * kNvChunkScaleBytes;
+    for (int it = blockIdx.y * (kThreads / 32) + warp; it < n * KC; it += warps) {
+      const int j = it / KC, c = it - (it / KC) * KC;
+      const int ib = 16 * (lane & 7);  // byte of the bf16 chunk row
+      const uint4 raw = *reinterpret_cast<const uint4*>(in + static_cast<size_t>(4 * c + (lane >> 3)) * n * 128 +
+                                                        j * 128 + ((((ib >> 4) ^ j) & 7) << 4));
+      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+      float v[8];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float2 f = __bfloat1622float2(h[k]);
+        v[2 * k] = f.x;
+        v[2 * k + 1] = f.y;
+      }
+      float amax = 0.f;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) amax = fmaxf(amax, fabsf(v[k]));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+      const uint8_t s = nvfp4_block_scale(amax, g);
+      const float d = e4m3_value(s) * g;
+      const uint32_t codes = nvfp4_pair(v[0], v[1], d) | (nvfp4_pair(v[2], v[3], d) << 8) |
+                             (nvfp4_pair(v[4], v[5], d) << 16) | (nvfp4_pair(v[6], v[7], d) << 24);
+      const int ob = 4 * lane;  // byte of the code chunk row
+      *reinterpret_cast<uint32_t*>(out + static_cast<size_t>(c) * n * 128 + j * 128 + ((((ob >> 4) ^ j) & 7) << 4) +
+                                   (ob & 15)) = codes;
+      if ((lane & 1) == 0) {
+        const int b = lane >> 1;
+        sf[static_cast<size_t>(c) * kNvChunkScaleBytes + (b >> 2) * 512 + 16 * (j & 31) + 4 * (j >> 5) + (b & 3)] = s;
+      }
+    }
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_permute_nvfp4_rows(const Launch& l, const void* xq, const void* xq_scale, int H,
+                                      const int* sorted_pair_ids, const int* num_groups, const int2* group_info, int P,
+                                      int k_total, void* xs, void* xs_sf, int num_sms) {
+  if (H % 256 != 0) return cudaErrorInvalidValue;
+  cudaLaunchConfig_t cfg;
+  cudaLaunchAttribute attr[1];
+  make_launch_config(&cfg, attr, l, dim3(2 * num_sms, kNvGroupRows / (kThreads / 32)), dim3(kThreads), 0);
+  return cudaLaunchKernelEx(&cfg, permute_nvfp4_rows_kernel, static_cast<const uint4*>(xq),
+                            static_cast<const uint8_t*>(xq_scale), H, sorted_pair_ids, num_groups, group_info, P,
+                            k_total, static_cast<uint8_t*>(xs), static_cast<uint8_t*>(xs_sf));
+}
+
+cudaError_t launch_act_quant_nvfp4(const Launch& l, const void* act, int I, float g, const int* num_groups,
+                                   const int2* group_info, void* actq, void* act_sf, int num_sms) {
+  if (I % 256 != 0) return cudaErrorInvalidValue;
+  cudaLaunchConfig_t cfg;
+  cudaLaunchAttribute attr[1];
+  make_launch_config(&cfg, attr, l, dim3(2 * num_sms, 4), dim3(kThreads), 0);
+  return cudaLaunchKernelEx(&cfg, act_quant_nvfp4_kernel, static_cast<const uint8_t*>(act), I, g, num_groups,
+                            group_info, static_cast<uint8_t*>(actq), static_cast<uint8_t*>(act_sf));
+}
 
 cudaError_t launch_permute_b128_rows(const Launch& l, const void* xq, const float* xq_scale, int H,
                                      const int* sorted_pair_ids, const int* num_groups, const int2* group_info, int P,

@@ -163,16 +163,68 @@ __global__ void tile_scales_mx_kernel(const uint8_t* __restrict__ in, uint8_t* _
   }
 }
 
+// NVFP4 weight scales beside the tiled codes: tile (e, m, c) (128 rows, 256 values of K in
+// one 128-byte chunk row) has a 2048-byte block of four 512-byte blocks, one per MMA of
+// K = 64: byte 512 mm + 16 l + 4 j + k is the E4M3 scale of tile row 32 j + l for the
+// 16-value block 16 c + 4 mm + k. tcgen05.cp (32 lanes x 16 bytes, replicated to the four
+// lane quadrants) leaves MMA mm's scales of row r in TMEM lane r % 32, column r / 32 of its
+// four columns, byte k = the row's block k of that MMA's 64 values: where the block-scaled
+// MMA with scale_vec::4X reads them. Rows follow the code tiles (gate and up interleaved for
+// w13 of a gated layer); rows or blocks past the matrix take 0.
+__global__ void tile_scales_nvfp4_kernel(const uint8_t* __restrict__ in, uint8_t* __restrict__ out, long long bytes,
+                                         int which, int rows, int MT, int KC, int KB, int I, int gated) {
+  griddep_wait();
+  for (long long o = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; o < bytes;
+       o += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long t = o >> 11;
+    const int b = static_cast<int>(o & 2047);
+    const int mm = b >> 9, l = (b >> 4) & 31, j = (b >> 2) & 3, k = b & 3;
+    const int c = static_cast<int>(t % KC);
+    const long long tm = t / KC;
+    const int m = static_cast<int>(tm % MT);
+    const long long e = tm / MT;
+    const int r = m * 128 + 32 * j + l;
+    const int kb = 16 * c + 4 * mm + k;
+    long long src = -1;
+    if (r < rows) {
+      if (which == 0 && gated) {
+        src = e * 2LL * I + static_cast<long long>(r & 1) * I + (r >> 1);
+      } else {
+        src = e * static_cast<long long>(rows) + r;
+      }
+    }
+    out[o] = (src >= 0 && kb < KB) ? in[src * KB + kb] : static_cast<uint8_t>(0);
+  }
+}
+
 }  // namespace
+
+size_t tiled_scale_bytes_nvfp4(int E, int rows, int K) {
+  return static_cast<size_t>(E) * ((rows + 127) / 128) * ((K + 255) / 256) * kNvChunkScaleBytes;
+}
+
+cudaError_t launch_tile_scales_nvfp4(const Launch& l, int which, const void* in, void* out, int E, int H, int I,
+                                     int gated) {
+  const int rows = which == 0 ? (gated ? 2 * I : I) : H;
+  const int K = which == 0 ? H : I;
+  if (K % 16 != 0) return cudaErrorInvalidValue;
+  const int MT = (rows + 127) / 128, KC = (K + 255) / 256;
+  const long long bytes = static_cast<long long>(tiled_scale_bytes_nvfp4(E, rows, K));
+  cudaLaunchConfig_t cfg;
+  cudaLaunchAttribute attr[1];
+  make_launch_config(&cfg, attr, l, dim3(4096), dim3(256), 0);
+  return cudaLaunchKernelEx(&cfg, tile_scales_nvfp4_kernel, static_cast<const uint8_t*>(in),
+                            static_cast<uint8_t*>(out), bytes, which, rows, MT, KC, K / 16, I, gated);
+}
 
 size_t tiled_weight_bytes_u8(int E, int rows, int K) {
   return static_cast<size_t>(E) * ((rows + 127) / 128) * ((K + 127) / 128) * 16384;
 }
 
 cudaError_t launch_tile_weights_u8(const Launch& l, int which, const void* in, void* out, int E, int H, int I,
-                                   int gated) {
+                                   int gated, int k_div) {
   const int rows = which == 0 ? (gated ? 2 * I : I) : H;
-  const int K = which == 0 ? H : I;
+  const int K = (which == 0 ? H : I) / k_div;  // bytes per row: packed E2M1 holds two values per byte
   if (K % 16 != 0) return cudaErrorInvalidValue;
   const int MT = (rows + 127) / 128, KC = (K + 127) / 128;
   const long long pieces = static_cast<long long>(tiled_weight_bytes_u8(E, rows, K) / 16);

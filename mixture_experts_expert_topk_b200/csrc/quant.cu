@@ -188,7 +188,79 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// NVFP4 ("FlashInfer gated MoE kernel optimisation for Blackwell", section 4, names NVFP4
+// weights; the format is NVIDIA's: E2M1 values, an E4M3 scale per 16 values, an fp32 scale
+// per tensor). One thread per block of 16 values along a row: 32 bytes of bf16 in, 8 code
+// bytes (two values per byte, the lower K index in the low nibble) and one scale byte out.
+// The tensor scale is g_static, or (amax_bits != nullptr) amax / (6 * 448) of the block's
+// matrix, from pass 1 of the per-tensor path (amax_per_matrix_kernel).
+__global__ void __launch_bounds__(256)
+    quant_nvfp4_rows_kernel(const uint4* __restrict__ w, long long blocks, long long blocks_per_mat,
+                            const int* __restrict__ amax_bits, float g_static, uint2* __restrict__ codes,
+                            uint8_t* __restrict__ scales) {
+  griddep_wait();
+  griddep_launch_dependents();
+  for (long long b = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; b < blocks;
+       b += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const float g = amax_bits != nullptr ? nvfp4_tensor_scale(__int_as_float(amax_bits[b / blocks_per_mat])) : g_static;
+    float v[16];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const uint4 raw = w[b * 2 + i];
+      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float2 f = __bfloat1622float2(h[k]);
+        v[8 * i + 2 * k] = f.x;
+        v[8 * i + 2 * k + 1] = f.y;
+      }
+    }
+    uint2 packed;
+    scales[b] = nvfp4_block(v, g, packed);
+    codes[b] = packed;
+  }
+}
+
+__global__ void nvfp4_scales_from_amax_kernel(int* __restrict__ amax_bits, long long num_mats) {
+  const long long m = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (m < num_mats) amax_bits[m] = __float_as_int(nvfp4_tensor_scale(__int_as_float(amax_bits[m])));
+}
+
 }  // namespace
+
+cudaError_t launch_quant_weights_nvfp4(const Launch& l, const void* w, int64_t num_mats, int64_t mat_elems,
+                                       void* codes, void* scales, float* global_scales) {
+  if (mat_elems % 16 != 0 || num_mats <= 0 || num_mats > 65535) return cudaErrorInvalidValue;
+  const long long vecs = mat_elems / 8;
+  int* bits = reinterpret_cast<int*>(global_scales);
+  cudaError_t err = cudaMemsetAsync(bits, 0, static_cast<size_t>(num_mats) * sizeof(int), l.stream);
+  if (err != cudaSuccess) return err;
+  const unsigned bx = static_cast<unsigned>(std::min<long long>((vecs + 255) / 256, 1024));
+  amax_per_matrix_kernel<<<dim3(bx, static_cast<unsigned>(num_mats)), 256, 0, l.stream>>>(
+      static_cast<const uint4*>(w), vecs, bits);
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  const long long blocks = num_mats * (mat_elems / 16);
+  quant_nvfp4_rows_kernel<<<static_cast<unsigned>(std::min<long long>((blocks + 255) / 256, 8192)), 256, 0,
+                            l.stream>>>(static_cast<const uint4*>(w), blocks, mat_elems / 16, bits, 1.0f,
+                                        static_cast<uint2*>(codes), static_cast<uint8_t*>(scales));
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  nvfp4_scales_from_amax_kernel<<<static_cast<unsigned>((num_mats + 255) / 256), 256, 0, l.stream>>>(bits, num_mats);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_rows_nvfp4(const Launch& l, const void* x, long long rows, int cols, float g, void* codes,
+                                    void* scales) {
+  if (cols % 16 != 0 || rows < 0) return cudaErrorInvalidValue;
+  const long long blocks = rows * (cols / 16);
+  if (blocks == 0) return cudaSuccess;
+  cudaLaunchConfig_t cfg;
+  cudaLaunchAttribute attr[1];
+  make_launch_config(&cfg, attr, l, dim3(static_cast<unsigned>(std::min<long long>((blocks + 255) / 256, 8192))),
+                     dim3(256), 0);
+  return cudaLaunchKernelEx(&cfg, quant_nvfp4_rows_kernel, static_cast<const uint4*>(x), blocks, blocks,
+                            static_cast<const int*>(nullptr), g, static_cast<uint2*>(codes),
+                            static_cast<uint8_t*>(scales));
+}
 
 cudaError_t launch_quant_weights_per_tensor(const Launch& l, const void* w, int64_t num_mats, int64_t mat_elems,
                                             void* codes, float* scales) {

@@ -41,7 +41,9 @@ class MoeConfig:
     # False: bf16. True: e4m3 with 128-wide block scales. "per_tensor": e4m3 with one scale
     # per expert matrix and static input / activation scales (activation_scale below; the
     # input scale is the hidden rows' amax / 448). "mxfp8": e4m3 with a power-of-two scale
-    # per 32 values of K on both GEMM inputs
+    # per 32 values of K on both GEMM inputs. "nvfp4": E2M1 with an E4M3 scale per 16 values
+    # of K and tensor scales (the input's: the hidden rows' amax / (6 * 448); the
+    # activation's: activation_scale below)
     fp8: object = False
     activation_scale: float = 0.03
     hidden_std: float = 1.0
@@ -60,6 +62,10 @@ class MoeConfig:
     @property
     def mx(self) -> bool:
         return self.fp8 == "mxfp8"
+
+    @property
+    def nv(self) -> bool:
+        return self.fp8 == "nvfp4"
 
     @property
     def gated(self) -> bool:
@@ -115,6 +121,14 @@ CONFIGS["prefill_e64"] = MoeConfig("prefill_e64", T=1024, H=2048, E=64, topk=8, 
                                    renormalize=True, activation="swiglu", logit_bias_std=0.5)
 CONFIGS["mxfp8_e64"] = CONFIGS["prefill_e64"].replace(name="mxfp8_e64", fp8="mxfp8")
 CONFIGS["fp8_e64"] = CONFIGS["prefill_e64"].replace(name="fp8_e64", fp8=True)
+
+
+# The prefill shape with NVFP4 weights and GEMM inputs (W4A4). The activation's tensor scale
+# is 12 / (6 * 448): GEMM1's activation on this workload stays below about 10 in magnitude
+# (the float64 activation over an eighth of the tokens peaks at 10.06), so no block scale
+# saturates.
+CONFIGS["nvfp4_prefill"] = CONFIGS["prefill"].replace(name="nvfp4_prefill", fp8="nvfp4", activation_scale=12.0 / 2688)
+CONFIGS["nvfp4_e64"] = CONFIGS["prefill_e64"].replace(name="nvfp4_e64", fp8="nvfp4", activation_scale=12.0 / 2688)
 
 
 # A compute-bound case of the prefill kernels: the prefill shapes (H=2048, I=512, SwiGLU,

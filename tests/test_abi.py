@@ -92,7 +92,8 @@ def test_padded_intermediate_follows_page_rule(L):
     assert L.moe_padded_intermediate(200, _capi.MOE_ACT_SWIGLUOAI, 0) == 208   # gated: 16
     assert L.moe_padded_intermediate(200, 4, 0) == -1                          # no such activation
     assert L.moe_padded_intermediate(200, 0, _capi.MOE_DTYPE_MXFP8) == 256   # MXFP8: 128
-    assert L.moe_padded_intermediate(200, 0, 4) == -1
+    assert L.moe_padded_intermediate(200, 0, _capi.MOE_DTYPE_NVFP4) == 256   # NVFP4: 256-value chunks
+    assert L.moe_padded_intermediate(200, 0, 5) == -1
     assert L.moe_padded_intermediate(16, 7, 0) == -1
 
 
@@ -112,7 +113,8 @@ def test_workspace_layout(L):
         # the permuted hidden rows (row-group order): bf16, e4m3 codes, or (FP8 block-128)
         # e4m3 codes with a 4-byte scale per row per 128 columns
         xs_bytes = lay["xs_scale"] - lay["xs"]
-        row_bytes = cfg.H * 132 // 128 if cfg.block128 else cfg.H * (1 if (cfg.per_tensor or cfg.mx) else 2)
+        row_bytes = (cfg.H * 132 // 128 if cfg.block128 else
+                     (cfg.H // 2 if cfg.nv else cfg.H * (1 if (cfg.per_tensor or cfg.mx) else 2)))
         assert xs_bytes == -(-lay["max_rows"] * row_bytes // 1024) * 1024
         assert lay["max_rows"] == -(-(P + min(E, P) * (bm - 1)) // bm) * bm
         assert lay["num_chunks"] == -(-P // 2048)
