@@ -143,7 +143,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull0 + 8 * b, 1);
-      mbar_init(tempty0 + 8 * b, 128);
+      mbar_init(tempty0 + 8 * b, 4);  // one arrival per epilogue warp
     }
     // tile-ring readers: the A warps (4 gathering, or the one TMA warp), MMA, 4 epilogue warps
     const uint32_t readers = (gather_a ? kNumAWarps : 1) + 1 + 4;
@@ -424,7 +424,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(tempty0 + 8 * acc);
+      __syncwarp();  // every lane's loads of the accumulator are complete
+      if (lane == 0) mbar_arrive(tempty0 + 8 * acc);
       ++it;
     }
     if (lane == 0) bulk_wait_group<0>();  // stores complete before the CTA retires

@@ -126,7 +126,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(pfull0 + 8 * b, 1);
-      mbar_init(pempty0 + 8 * b, 128);
+      mbar_init(pempty0 + 8 * b, 4);  // one arrival per epilogue warp
     }
     const uint32_t readers = (gather_a ? kNumAWarps : 1) + 1 + 4;
     for (int s = 0; s < kTileRing; ++s) {
@@ -375,7 +375,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         tc_fence_before();
-        mbar_arrive(pempty0 + 8 * pb);
+        __syncwarp();  // every lane's loads of the partial are complete
+        if (lane == 0) mbar_arrive(pempty0 + 8 * pb);
       }
       if (!ok) break;
       const bool any_valid = __ballot_sync(0xffffffffu, valid) != 0u;

@@ -298,12 +298,12 @@ __global__ void __launch_bounds__(threads_for<kKind>(), 1) gemm_swap_kernel(cons
     }
     for (int b = 0; b < kPartBufs; ++b) {
       mbar_init(pfull0 + 8 * b, 1);
-      mbar_init(pempty0 + 8 * b, 256);  // every thread of the eight epilogue warps
+      mbar_init(pempty0 + 8 * b, 8);  // one arrival per epilogue warp
     }
     for (int b = 0; b < kSxSlots; ++b) mbar_init(sxfree0 + 8 * b, 8);  // the eight epilogue warps
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull0 + 8 * b, 1);
-      mbar_init(tempty0 + 8 * b, 128);
+      mbar_init(tempty0 + 8 * b, 4);  // one arrival per epilogue warp
     }
     for (int s = 0; s < kTileRing; ++s) {
       mbar_init(rfull0 + 8 * s, 1);
@@ -709,7 +709,8 @@ __global__ void __launch_bounds__(threads_for<kKind>(), 1) gemm_swap_kernel(cons
               }
             }
             tc_fence_before();
-            mbar_arrive(pempty0 + 8 * pb);  // the partial is in registers now
+            __syncwarp();  // every lane's loads of the partial are complete
+            if (lane == 0) mbar_arrive(pempty0 + 8 * pb);  // the partial is in registers now
           }
           if (!good) break;
           __syncwarp();  // every lane has read the step's scales
@@ -741,7 +742,8 @@ __global__ void __launch_bounds__(threads_for<kKind>(), 1) gemm_swap_kernel(cons
           tmem_wait_ld();
           if (c0 + 32 >= n) {
             tc_fence_before();
-            mbar_arrive(tempty0 + 8 * acc);  // the accumulator is in registers now
+            __syncwarp();  // every lane's loads of the accumulator are complete
+            if (lane == 0) mbar_arrive(tempty0 + 8 * acc);  // the accumulator is in registers now
           }
           store_block(v, c0, full);
         }
