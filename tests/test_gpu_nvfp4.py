@@ -88,8 +88,8 @@ def group_scales(flat, group_info, num_groups, rows, KC) -> np.ndarray:
 
 
 def deinterleave(rows_tiled: np.ndarray, I: int) -> np.ndarray:
-    """Interleaved [gate0, up0, gate1, up1, ...] rows -> gate rows then up rows."""
-    return np.concatenate([rows_tiled[:, 0:2 * I:2], rows_tiled[:, 1:2 * I:2]], axis=1)
+    """Interleaved [gate0, up0, gate1, up1, ...] rows ([2I, cols]) -> gate rows then up rows."""
+    return np.concatenate([rows_tiled[0:2 * I:2], rows_tiled[1:2 * I:2]], axis=0)
 
 
 def _act_scale(cfg, inp, s_in) -> float:
