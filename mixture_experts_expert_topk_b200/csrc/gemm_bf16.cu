@@ -250,7 +250,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       int wslot = 0, sb = 0;
       uint32_t wph = 0, phb = 0;
       uint32_t fills = 0;
-      int tile = atomicAdd(a.tile_counter, 1);
+      // the first tile is the CTA index; later ones come from the counter, after the grid's first tiles
+      int tile = static_cast<int>(blockIdx.x);
       while (true) {
         if (!mbar_wait(ringempty0 + 8 * wslot, wph ^ 1u, abort_flag, a.status, kSiteTileEmpty)) break;
         const bool done = tile >= num_tiles;
@@ -261,7 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           wph ^= 1u;
         }
         if (done) break;
-        const int next = atomicAdd(a.tile_counter, 1);  // its latency overlaps this tile's loads
+        const int next = static_cast<int>(gridDim.x) + atomicAdd(a.tile_counter, 1);  // its latency overlaps this tile's loads
         const int mb = tile / a.n_tiles;
         const int nt = tile - mb * a.n_tiles;
         const int brow = a.block_expert[mb] * a.w_rows_per_expert + nt * a.BN;

@@ -337,7 +337,8 @@ __global__ void __launch_bounds__(threads_for<kKind>(), 1) gemm_swap_kernel(cons
       int wslot = 0;
       uint32_t wph = 0, pos = 0, ks = 0, oldest = 0;
       uint64_t head = 0, freed = 0;
-      int tile = atomicAdd(a.tile_counter, 1);
+      // the first tile is the CTA index; later ones come from the counter, after the grid's first tiles
+      int tile = static_cast<int>(blockIdx.x);
       bool ok = true;
       while (ok) {
         if (!mbar_wait(rempty0 + 8 * wslot, wph ^ 1u, abort_flag, a.status, kSiteTileEmpty)) break;
@@ -360,7 +361,7 @@ __global__ void __launch_bounds__(threads_for<kKind>(), 1) gemm_swap_kernel(cons
           wph ^= 1u;
         }
         if (n == 0) break;
-        const int next = atomicAdd(a.tile_counter, 1);  // its latency overlaps the loads
+        const int next = static_cast<int>(gridDim.x) + atomicAdd(a.tile_counter, 1);  // its latency overlaps the loads
         const int kc = step_chunks<kKind>(n);
         const uint8_t* wsrc = a.w + (static_cast<size_t>(e) * a.m_tiles + mt) * a.k_chunks * kTileW;
         for (int c0 = 0; c0 < a.k_chunks; c0 += kc, ++ks) {
