@@ -113,15 +113,18 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_sums, int* 
 }
 
 // Padded segments of experts [0, E): sentinel rows after each expert's pairs and the
-// expert id of each row tile. One warp per expert, lanes striding over its rows, so the
-// stores are coalesced. seg_off/seg_cnt/seg_pad are shared-memory arrays.
+// expert id of each row tile. One thread per expert (at most block_m - 1 sentinels and
+// padded / block_m tile ids each), so no warp walks the experts one after another; most
+// experts of a small batch have no rows at all. seg_off/seg_cnt/seg_pad are shared-memory
+// arrays; off and pad are multiples of block_m.
 __device__ __forceinline__ void write_segments(int E, const int* seg_off, const int* seg_cnt, const int* seg_pad,
                                                int block_m, int P, int* sorted_pair_ids, int* block_expert) {
-  const int lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
-  for (int e = threadIdx.x >> 5; e < E; e += nwarps) {
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
     const int off = seg_off[e], cnt = seg_cnt[e], pad = seg_pad[e];
-    for (int r = off + cnt + lane; r < off + pad; r += 32) sorted_pair_ids[r] = P;
-    for (int b = off / block_m + lane; b < (off + pad) / block_m; b += 32) block_expert[b] = e;
+    if (pad == 0) continue;
+    for (int r = off + cnt; r < off + pad; ++r) sorted_pair_ids[r] = P;
+    const int b0 = off / block_m, b1 = (off + pad) / block_m;
+    for (int b = b0; b < b1; ++b) block_expert[b] = e;
   }
 }
 
@@ -217,7 +220,9 @@ __global__ void __launch_bounds__(kWarps * 32)
   griddep_wait();
   griddep_launch_dependents();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int i = threadIdx.x; i < kWarps * E; i += blockDim.x) cnt[i / E][i % E] = 0;
+  for (int x = threadIdx.x; x < E; x += blockDim.x)
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) cnt[w][x] = 0;
   const int base = blockIdx.x * kAlignChunk + warp * kPairsPerWarp;
   int e[kIdsPerLane];
   load_ids(ids, base, P, E, lane, e);
@@ -249,7 +254,9 @@ __global__ void __launch_bounds__(kWarps * 32)
   griddep_wait();
   griddep_launch_dependents();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int i = threadIdx.x; i < kWarps * E; i += blockDim.x) cnt[i / E][i % E] = 0;
+  for (int x = threadIdx.x; x < E; x += blockDim.x)
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) cnt[w][x] = 0;
   const int base = warp * kPairsPerWarp;
   int e[kIdsPerLane];
   load_ids(ids, base, P, E, lane, e);

@@ -98,12 +98,14 @@ constexpr int kTileW = kMW * kChunkBytes;  // 16 KB: one W chunk
 constexpr int kNMax = 256;                 // rows of a row group at most (MMA N)
 constexpr int kThreads = 224;
 constexpr int kWarpX = 6;
-// FP8 block-128 adds four epilogue warps (7..10): two per TMEM lane quadrant, each
-// promoting 64 of a tile's token columns
+// FP8 block-128 adds twelve epilogue warps (7..18): four per TMEM lane quadrant in all, each
+// promoting 32 of a tile's token columns (warps 2..5 columns 0..31, warps 3 + 4 p .. 6 + 4 p
+// columns 32 p .. 32 p + 31 for p = 1, 2, 3)
+constexpr int kB128EpiWarps = 16;
 template <int kKind>
-__host__ __device__ constexpr int threads_for() { return kKind == 3 ? 352 : kThreads; }
+__host__ __device__ constexpr int threads_for() { return kKind == 3 ? kThreads + 32 * (kB128EpiWarps - 4) : kThreads; }
 constexpr int kTileRing = 4;
-constexpr int kRingReaders = 6;  // MMA, 4 epilogue warps, X producer (FP8 block-128: 8 epilogue warps)
+constexpr int kRingReaders = 6;  // MMA, 4 epilogue warps, X producer (FP8 block-128: 16 epilogue warps)
 constexpr int kSmemCap = 232448;
 constexpr uint32_t kTmemCols = 2 * kNMax;
 // MXFP8: scale bytes per chunk in the ring, TMEM columns of the accumulators and of the
@@ -298,16 +300,16 @@ __global__ void __launch_bounds__(threads_for<kKind>(), 1) gemm_swap_kernel(cons
     }
     for (int b = 0; b < kPartBufs; ++b) {
       mbar_init(pfull0 + 8 * b, 1);
-      mbar_init(pempty0 + 8 * b, 8);  // one arrival per epilogue warp
+      mbar_init(pempty0 + 8 * b, kB128EpiWarps);  // one arrival per epilogue warp
     }
-    for (int b = 0; b < kSxSlots; ++b) mbar_init(sxfree0 + 8 * b, 8);  // the eight epilogue warps
+    for (int b = 0; b < kSxSlots; ++b) mbar_init(sxfree0 + 8 * b, kB128EpiWarps);  // every epilogue warp
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull0 + 8 * b, 1);
       mbar_init(tempty0 + 8 * b, 4);  // one arrival per epilogue warp
     }
     for (int s = 0; s < kTileRing; ++s) {
       mbar_init(rfull0 + 8 * s, 1);
-      mbar_init(rempty0 + 8 * s, kB128 ? kRingReaders + 4 : kRingReaders);
+      mbar_init(rempty0 + 8 * s, kB128 ? kRingReaders + kB128EpiWarps - 4 : kRingReaders);
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -556,7 +558,8 @@ __global__ void __launch_bounds__(threads_for<kKind>(), 1) gemm_swap_kernel(cons
     // output columns, so each store writes one contiguous piece of an output row (GEMM2:
     // 64 B of fp16; GEMM1: 64 or 32 B of a 128-byte activation chunk row).
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
-    const int half = kB128 && warp > kWarpX ? 1 : 0;  // FP8 block-128: token columns [64 half, 64 half + 64)
+    // FP8 block-128: this warp's token columns [32 part, 32 part + 32)
+    const int part = kB128 && warp > kWarpX ? 1 + (warp - kWarpX - 1) / 4 : 0;
     const bool gated = a.activation != 1;  // 0 SwiGLU, 2 gelu_tanh, 3 swigluoai; 1 relu2
     const bool odd = (lane & 1) != 0;
     int rslot = 0, it = 0;
@@ -655,19 +658,18 @@ __global__ void __launch_bounds__(threads_for<kKind>(), 1) gemm_swap_kernel(cons
         const int rb_odd = a.up_block > 0 ? a.up_block + (mt >> 1) : mt;
         const float swl_even = lane < a.k_chunks ? __ldg(sw_e + static_cast<size_t>(rb_even) * a.k_chunks + lane) : 0.f;
         const float swl_odd = lane < a.k_chunks ? __ldg(sw_e + static_cast<size_t>(rb_odd) * a.k_chunks + lane) : 0.f;
-        // this warp's token columns [64 half, 64 half + 64): blocks cb = 2 half, 2 half + 1
-        const int nb0 = n - 64 * half;              // columns left from this warp's first
-        const bool has0 = nb0 > 0, full0 = nb0 >= 32;
-        const bool has1 = nb0 > 32, full1 = nb0 >= 64;
-        float acc[64];
+        // this warp's token columns [32 part, 32 part + 32)
+        const int nb = n - 32 * part;  // columns left from this warp's first
+        const bool has = nb > 0, full = nb >= 32;
+        float2 acc[16];
 #pragma unroll
-        for (int i = 0; i < 64; ++i) acc[i] = 0.f;
+        for (int i = 0; i < 16; ++i) acc[i] = make_float2(0.f, 0.f);
         bool good = true;
         for (int c0 = 0; c0 < a.k_chunks && good; c0 += kc, ++ks) {
           const int kcs = min(kc, a.k_chunks - c0);
           // the X scales of this step, [chunk][row] fp32, in its slot of the X scale ring (the
           // full barrier the partials' MMAs waited on also covered this copy)
-          const uint32_t sf = sx0 + (ks % kSxSlots) * kSxSlotBytes;
+          const uint32_t sf = (ks % kSxSlots) * kSxSlotBytes + kRingBytesB128;
           for (int c = 0; c < kcs; ++c, ++pc) {
             const uint32_t pb = pc % kPartBufs;
             const bool got = mbar_wait(pfull0 + 8 * pb, (pc / kPartBufs) & 1u, abort_flag, a.status, kSitePartFull);
@@ -676,37 +678,31 @@ __global__ void __launch_bounds__(threads_for<kKind>(), 1) gemm_swap_kernel(cons
               break;
             }
             tc_fence_after();
+            // lane k holds chunk k's weight scales (even and odd rows)
             const float sw_e_k = __shfl_sync(0xffffffffu, swl_even, c0 + c);
             const float sw_o_k = __shfl_sync(0xffffffffu, swl_odd, c0 + c);
             const float sw = odd ? sw_o_k : sw_e_k;
-            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + pb * kPartCols + 64 * half;
-            const uint32_t sfc = sf + static_cast<uint32_t>(c * n + 64 * half) * 4u;
-            // both 32-column loads in flight before one wait
-            uint32_t v[64];
-            if (full0) {
-              tmem_ld32(taddr, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-            } else if (has0) {
-              tmem_ld16(taddr, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
-            }
-            if (full1) {
-              tmem_ld32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
-            } else if (has1) {
-              tmem_ld16(taddr + 32, *reinterpret_cast<uint32_t(*)[16]>(&v[32]));
-            }
-            tmem_wait_ld();
+            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + pb * kPartCols + 32 * part;
+            // the partial in two halves of 16 columns (fewer live registers than one load of 32)
+            const float4* sx4 = reinterpret_cast<const float4*>(smem + sf + static_cast<uint32_t>(c * n + 32 * part) * 4u);
+            const float2 sw2 = make_float2(sw, sw);
 #pragma unroll
-            for (int j4 = 0; j4 < 16; ++j4) {
-              // columns 4 j4 .. 4 j4 + 3 of this warp's 64; past n they are skipped
-              if (4 * j4 < nb0) {
-                float4 sx;  // the same four scales for every lane: a shared-memory broadcast
-                asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
-                             : "=f"(sx.x), "=f"(sx.y), "=f"(sx.z), "=f"(sx.w)
-                             : "r"(sfc + static_cast<uint32_t>(4 * j4) * 4u));
-                const int j = 4 * j4;
-                acc[j + 0] = fmaf(__uint_as_float(v[j + 0]), sx.x * sw, acc[j + 0]);
-                acc[j + 1] = fmaf(__uint_as_float(v[j + 1]), sx.y * sw, acc[j + 1]);
-                acc[j + 2] = fmaf(__uint_as_float(v[j + 2]), sx.z * sw, acc[j + 2]);
-                acc[j + 3] = fmaf(__uint_as_float(v[j + 3]), sx.w * sw, acc[j + 3]);
+            for (int h = 0; h < 2; ++h) {
+              if (16 * h < nb) {  // warp-uniform
+                uint32_t v[16];
+                tmem_ld16(taddr + 16 * h, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j4 = 0; j4 < 4; ++j4) {
+                  // columns 16 h + 4 j4 .. + 3 of this warp's 32: acc pairs 8 h + 2 j4, + 1; the
+                  // same scales for every lane (shared-memory broadcasts)
+                  const int j = 4 * j4, a2 = 8 * h + 2 * j4;
+                  const float4 sx = sx4[4 * h + j4];
+                  acc[a2] = __ffma2_rn(make_float2(__uint_as_float(v[j]), __uint_as_float(v[j + 1])),
+                                       __fmul2_rn(make_float2(sx.x, sx.y), sw2), acc[a2]);
+                  acc[a2 + 1] = __ffma2_rn(make_float2(__uint_as_float(v[j + 2]), __uint_as_float(v[j + 3])),
+                                           __fmul2_rn(make_float2(sx.z, sx.w), sw2), acc[a2 + 1]);
+                }
               }
             }
             tc_fence_before();
@@ -718,11 +714,7 @@ __global__ void __launch_bounds__(threads_for<kKind>(), 1) gemm_swap_kernel(cons
           if (lane == 0) mbar_arrive(sxfree0 + 8 * (ks % kSxSlots));
         }
         if (!__all_sync(0xffffffffu, good)) break;
-#pragma unroll
-        for (int b = 0; b < 2; ++b)
-          if (32 * b < nb0)
-            store_block(*reinterpret_cast<const uint32_t(*)[32]>(&acc[32 * b]), 64 * half + 32 * b,
-                        nb0 - 32 * b >= 32);
+        if (has) store_block(*reinterpret_cast<const uint32_t(*)[32]>(&acc[0]), 32 * part, full);
       } else {
         const int acc = it & 1;
         const bool got = mbar_wait(tfull0 + 8 * acc, (it >> 1) & 1, abort_flag, a.status, kSiteTmemFull);

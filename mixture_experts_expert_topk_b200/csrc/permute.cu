@@ -73,6 +73,7 @@ __global__ void __launch_bounds__(kThreads)
   }
 }
 
+
 // Per-tensor FP8: the same row-group order with each element quantised on the way,
 // e4m3(x * inv_scale), inv_scale = fp32(1 / input_scale) (the per-tensor variant scales
 // by the reciprocal: "FlashInfer TRTLLM-Gen MoE kernel optimisation: NemotronH support",
@@ -223,8 +224,10 @@ __global__ void __launch_bounds__(kThreads)
 
 // GEMM1's bf16 activation (row-group order, 64-column chunks of 128-byte rows) to MXFP8
 // codes (128-column chunks) and scales, in the layout of permute_mx_rows_kernel, for
-// GEMM2. A warp converts one 128-column chunk of one row: lane l takes columns 4l..4l+3
-// (8 bytes of bf16 chunk 2c + l/16), eight lanes form a 32-column block.
+// GEMM2. A warp converts one row, four 128-column chunks at a time (their loads first):
+// lane l takes columns 4l..4l+3 of each (8 bytes of bf16 chunk 2c + l/16), eight lanes form
+// a 32-column block.
+constexpr int kActChunksPerPass = 4;
 __global__ void __launch_bounds__(kThreads)
     act_quant_mx_kernel(const uint8_t* __restrict__ act, int I, const int* __restrict__ num_groups,
                         const int2* __restrict__ group_info, uint8_t* __restrict__ actq,
@@ -234,30 +237,42 @@ __global__ void __launch_bounds__(kThreads)
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int G = *num_groups;
   const int KCb = I / 64, KCq = I / 128;
-  const int warps = gridDim.y * (kThreads / 32);
+  const int ib = 8 * (lane & 15);  // byte of the bf16 chunk row
+  const int ob = 4 * lane;         // byte of the e4m3 chunk row
   for (int g = blockIdx.x; g < G; g += gridDim.x) {
     const int2 gi = group_info[g];
     const int x_row = gi.x, n = gi.y >> 16;
     const uint8_t* in = act + static_cast<size_t>(x_row) * KCb * 128;
     uint8_t* out = actq + static_cast<size_t>(x_row) * KCq * 128;
     uint8_t* sf = act_sf + static_cast<size_t>(x_row >> 4) * KCq * 1024;
-    for (int it = blockIdx.y * (kThreads / 32) + warp; it < n * KCq; it += warps) {
-      const int j = it / KCq, c = it - (it / KCq) * KCq;
-      const int ib = 8 * (lane & 15);  // byte of the bf16 chunk row
-      const uint2 raw = *reinterpret_cast<const uint2*>(in + static_cast<size_t>(2 * c + (lane >> 4)) * n * 128 +
-                                                        j * 128 + ((((ib >> 4) ^ j) & 7) << 4) + (ib & 15));
-      const float2 f01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.x));
-      const float2 f23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.y));
-      float amax = fmaxf(fmaxf(fabsf(f01.x), fabsf(f01.y)), fmaxf(fabsf(f23.x), fabsf(f23.y)));
+    for (int j = blockIdx.y * (kThreads / 32) + warp; j < n; j += gridDim.y * (kThreads / 32)) {
+      for (int c0 = 0; c0 < KCq; c0 += kActChunksPerPass) {
+        uint2 raw[kActChunksPerPass];
 #pragma unroll
-      for (int o = 1; o < 8; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-      const int e = mx_exponent(amax);
-      const int ob = 4 * lane;  // byte of the e4m3 chunk row
-      *reinterpret_cast<uint32_t*>(out + static_cast<size_t>(c) * n * 128 + j * 128 + ((((ob >> 4) ^ j) & 7) << 4) +
-                                   (ob & 15)) = mx_e4m3x4(f01.x, f01.y, f23.x, f23.y, mx_inv(e));
-      if ((lane & 7) == 0)
-        sf[static_cast<size_t>(c) * 1024 + (j >> 7) * 512 + (j & 31) * 16 + ((j >> 5) & 3) * 4 + (lane >> 3)] =
-            static_cast<uint8_t>(e + 127);
+        for (int i = 0; i < kActChunksPerPass; ++i) {
+          const int c = c0 + i;
+          raw[i] = c < KCq ? *reinterpret_cast<const uint2*>(in + static_cast<size_t>(2 * c + (lane >> 4)) * n * 128 +
+                                                             j * 128 + ((((ib >> 4) ^ j) & 7) << 4) + (ib & 15))
+                           : make_uint2(0u, 0u);
+        }
+#pragma unroll
+        for (int i = 0; i < kActChunksPerPass; ++i) {
+          const int c = c0 + i;
+          if (c >= KCq) break;  // warp-uniform
+          const float2 f01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw[i].x));
+          const float2 f23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw[i].y));
+          float amax = fmaxf(fmaxf(fabsf(f01.x), fabsf(f01.y)), fmaxf(fabsf(f23.x), fabsf(f23.y)));
+#pragma unroll
+          for (int o = 1; o < 8; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+          const int e = mx_exponent(amax);
+          *reinterpret_cast<uint32_t*>(out + static_cast<size_t>(c) * n * 128 + j * 128 +
+                                       ((((ob >> 4) ^ j) & 7) << 4) + (ob & 15)) =
+              mx_e4m3x4(f01.x, f01.y, f23.x, f23.y, mx_inv(e));
+          if ((lane & 7) == 0)
+            sf[static_cast<size_t>(c) * 1024 + (j >> 7) * 512 + (j & 31) * 16 + ((j >> 5) & 3) * 4 + (lane >> 3)] =
+                static_cast<uint8_t>(e + 127);
+        }
+      }
     }
   }
 }
@@ -340,7 +355,6 @@ __global__ void __launch_bounds__(kThreads)
 // order) quantised per 1x128 group into the X layout; a warp takes one row, four chunks at
 // a time (their loads first), lane l columns 4l..4l+3 of each 128-column chunk (8 bytes of
 // bf16 chunk 2c + l / 16).
-constexpr int kActChunksPerPass = 4;
 __global__ void __launch_bounds__(kThreads)
     act_quant_b128_kernel(const uint8_t* __restrict__ act, int I, const int* __restrict__ num_groups,
                           const int2* __restrict__ group_info, uint8_t* __restrict__ actq) {
@@ -435,8 +449,9 @@ __global__ void __launch_bounds__(kThreads)
 
 // NVFP4: GEMM1's bf16 activation (64-column chunks of 128-byte rows, row-group order)
 // quantised with tensor scale g into the layout of permute_nvfp4_rows_kernel. A warp takes
-// one (row, 256-column chunk): lane l converts columns 8l..8l+7 (16 bytes of bf16 chunk
-// 4c + l / 8); lanes 2b and 2b+1 share 16-value block b and exchange their maxima.
+// one row, four 256-column chunks at a time (their loads first): lane l converts columns
+// 8l..8l+7 of each (16 bytes of bf16 chunk 4c + l / 8); lanes 2b and 2b+1 share 16-value
+// block b and exchange their maxima.
 __global__ void __launch_bounds__(kThreads)
     act_quant_nvfp4_kernel(const uint8_t* __restrict__ act, int I, float g, const int* __restrict__ num_groups,
                            const int2* __restrict__ group_info, uint8_t* __restrict__ actq, uint8_t* __restrict__ act_sf) {
@@ -445,40 +460,52 @@ __global__ void __launch_bounds__(kThreads)
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int G = *num_groups;
   const int KCb = I / 64, KC = I / 256;
-  const int warps = gridDim.y * (kThreads / 32);
+  const int ib = 16 * (lane & 7);  // byte of the bf16 chunk row
+  const int ob = 4 * lane;         // byte of the code chunk row
   for (int gr = blockIdx.x; gr < G; gr += gridDim.x) {
     const int2 gi = group_info[gr];
     const int x_row = gi.x, n = gi.y >> 16;
     const uint8_t* in = act + static_cast<size_t>(x_row) * KCb * 128;
     uint8_t* out = actq + static_cast<size_t>(x_row) * KC * 128;
     uint8_t* sf = act_sf + static_cast<size_t>(x_row >> 4) * KC * kNvChunkScaleBytes;
-    for (int it = blockIdx.y * (kThreads / 32) + warp; it < n * KC; it += warps) {
-      const int j = it / KC, c = it - (it / KC) * KC;
-      const int ib = 16 * (lane & 7);  // byte of the bf16 chunk row
-      const uint4 raw = *reinterpret_cast<const uint4*>(in + static_cast<size_t>(4 * c + (lane >> 3)) * n * 128 +
-                                                        j * 128 + ((((ib >> 4) ^ j) & 7) << 4));
-      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
-      float v[8];
+    for (int j = blockIdx.y * (kThreads / 32) + warp; j < n; j += gridDim.y * (kThreads / 32)) {
+      for (int c0 = 0; c0 < KC; c0 += kActChunksPerPass) {
+        uint4 raw[kActChunksPerPass];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float2 f = __bfloat1622float2(h[k]);
-        v[2 * k] = f.x;
-        v[2 * k + 1] = f.y;
-      }
-      float amax = 0.f;
+        for (int i = 0; i < kActChunksPerPass; ++i) {
+          const int c = c0 + i;
+          raw[i] = c < KC ? *reinterpret_cast<const uint4*>(in + static_cast<size_t>(4 * c + (lane >> 3)) * n * 128 +
+                                                            j * 128 + ((((ib >> 4) ^ j) & 7) << 4))
+                          : make_uint4(0u, 0u, 0u, 0u);
+        }
 #pragma unroll
-      for (int k = 0; k < 8; ++k) amax = fmaxf(amax, fabsf(v[k]));
-      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-      const uint8_t s = nvfp4_block_scale(amax, g);
-      const float d = e4m3_value(s) * g;
-      const uint32_t codes = nvfp4_pair(v[0], v[1], d) | (nvfp4_pair(v[2], v[3], d) << 8) |
-                             (nvfp4_pair(v[4], v[5], d) << 16) | (nvfp4_pair(v[6], v[7], d) << 24);
-      const int ob = 4 * lane;  // byte of the code chunk row
-      *reinterpret_cast<uint32_t*>(out + static_cast<size_t>(c) * n * 128 + j * 128 + ((((ob >> 4) ^ j) & 7) << 4) +
-                                   (ob & 15)) = codes;
-      if ((lane & 1) == 0) {
-        const int b = lane >> 1;
-        sf[static_cast<size_t>(c) * kNvChunkScaleBytes + (b >> 2) * 512 + 16 * (j & 31) + 4 * (j >> 5) + (b & 3)] = s;
+        for (int i = 0; i < kActChunksPerPass; ++i) {
+          const int c = c0 + i;
+          if (c >= KC) break;  // warp-uniform
+          const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw[i]);
+          float v[8];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float2 f = __bfloat1622float2(h[k]);
+            v[2 * k] = f.x;
+            v[2 * k + 1] = f.y;
+          }
+          float amax = 0.f;
+#pragma unroll
+          for (int k = 0; k < 8; ++k) amax = fmaxf(amax, fabsf(v[k]));
+          amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+          const uint8_t s = nvfp4_block_scale(amax, g);
+          const float d = e4m3_value(s) * g;
+          const uint32_t codes = nvfp4_pair(v[0], v[1], d) | (nvfp4_pair(v[2], v[3], d) << 8) |
+                                 (nvfp4_pair(v[4], v[5], d) << 16) | (nvfp4_pair(v[6], v[7], d) << 24);
+          *reinterpret_cast<uint32_t*>(out + static_cast<size_t>(c) * n * 128 + j * 128 +
+                                       ((((ob >> 4) ^ j) & 7) << 4) + (ob & 15)) = codes;
+          if ((lane & 1) == 0) {
+            const int b = lane >> 1;
+            sf[static_cast<size_t>(c) * kNvChunkScaleBytes + (b >> 2) * 512 + 16 * (j & 31) + 4 * (j >> 5) + (b & 3)] =
+                s;
+          }
+        }
       }
     }
   }
@@ -503,7 +530,7 @@ cudaError_t launch_act_quant_nvfp4(const Launch& l, const void* act, int I, floa
   if (I % 256 != 0) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg;
   cudaLaunchAttribute attr[1];
-  make_launch_config(&cfg, attr, l, dim3(2 * num_sms, 4), dim3(kThreads), 0);
+  make_launch_config(&cfg, attr, l, dim3(2 * num_sms, kNvGroupRows / (kThreads / 32)), dim3(kThreads), 0);
   return cudaLaunchKernelEx(&cfg, act_quant_nvfp4_kernel, static_cast<const uint8_t*>(act), I, g, num_groups,
                             group_info, static_cast<uint8_t*>(actq), static_cast<uint8_t*>(act_sf));
 }
@@ -570,7 +597,7 @@ cudaError_t launch_act_quant_mx(const Launch& l, const void* act, int I, const i
   if (I % 128 != 0) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg;
   cudaLaunchAttribute attr[1];
-  make_launch_config(&cfg, attr, l, dim3(2 * num_sms, 2), dim3(kThreads), 0);
+  make_launch_config(&cfg, attr, l, dim3(2 * num_sms, kMxGroupRows / (kThreads / 32)), dim3(kThreads), 0);
   return cudaLaunchKernelEx(&cfg, act_quant_mx_kernel, static_cast<const uint8_t*>(act), I, num_groups,
                             group_info, static_cast<uint8_t*>(actq), static_cast<uint8_t*>(act_sf));
 }
