@@ -27,6 +27,7 @@
 
 #include "moe_device.cuh"
 #include "moe_internal.h"
+#include "route_device.cuh"
 
 namespace moe {
 namespace {
@@ -48,7 +49,7 @@ __device__ __forceinline__ void load_ids(const int* ids, int base, int end, int 
 #pragma unroll
   for (int i = 0; i < kIdsPerLane; ++i) {
     const int p = base + 32 * i + lane;
-    const int id = p < end ? ids[p] : -1;
+    const int id = p < end ? __ldcg(ids + p) : -1;  // L2: the ids may come from this CTA
     e[i] = p >= end ? -1 : (static_cast<unsigned>(id) < static_cast<unsigned>(E) ? id : kBadId);
   }
 }
@@ -242,17 +243,21 @@ __global__ void __launch_bounds__(kWarps * 32)
   warp_place(e, base, lane, cnt[warp], sorted_pair_ids, pair_to_row);
 }
 
-// All of align for P <= kAlignChunk in one CTA of kWarps warps.
-__global__ void __launch_bounds__(kWarps * 32)
-    align_single_kernel(const int* __restrict__ ids, int P, int E, int block_m, int* __restrict__ sorted_pair_ids,
-                        int* __restrict__ expert_offsets, int* __restrict__ block_expert,
-                        int* __restrict__ pair_to_row, int* __restrict__ num_blocks, int group_rows,
-                        int2* __restrict__ group_info) {
-  __shared__ int cnt[kWarps][kMaxExperts];
-  __shared__ int warp_sums[32];
-  __shared__ int seg_off[kMaxExperts], seg_cnt[kMaxExperts], seg_pad[kMaxExperts];
-  griddep_wait();
-  griddep_launch_dependents();
+// All of align for P <= kAlignChunk by one CTA of kWarps warps (every thread calls it).
+struct AlignSingleSmem {
+  int cnt[kWarps][kMaxExperts];
+  int warp_sums[32];
+  int seg_off[kMaxExperts], seg_cnt[kMaxExperts], seg_pad[kMaxExperts];
+};
+__device__ __forceinline__ void align_single_cta(AlignSingleSmem& sm, const int* ids, int P, int E, int block_m,
+                                                 int* sorted_pair_ids, int* expert_offsets, int* block_expert,
+                                                 int* pair_to_row, int* num_blocks, int group_rows,
+                                                 int2* group_info) {
+  auto& cnt = sm.cnt;
+  int* warp_sums = sm.warp_sums;
+  int* seg_off = sm.seg_off;
+  int* seg_cnt = sm.seg_cnt;
+  int* seg_pad = sm.seg_pad;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int x = threadIdx.x; x < E; x += blockDim.x)
 #pragma unroll
@@ -301,6 +306,59 @@ __global__ void __launch_bounds__(kWarps * 32)
   warp_place(e, base, lane, cnt[warp], sorted_pair_ids, pair_to_row);
 }
 
+__global__ void __launch_bounds__(kWarps * 32)
+    align_single_kernel(const int* __restrict__ ids, int P, int E, int block_m, int* __restrict__ sorted_pair_ids,
+                        int* __restrict__ expert_offsets, int* __restrict__ block_expert,
+                        int* __restrict__ pair_to_row, int* __restrict__ num_blocks, int group_rows,
+                        int2* __restrict__ group_info) {
+  __shared__ AlignSingleSmem sm;
+  griddep_wait();
+  griddep_launch_dependents();
+  align_single_cta(sm, ids, P, E, block_m, sorted_pair_ids, expert_offsets, block_expert, pair_to_row, num_blocks,
+                   group_rows, group_info);
+}
+
+// Routing and align of a small batch (T <= kWarps * kRouteAlignTokensPerWarp tokens, one
+// align chunk) in one CTA, one kernel boundary fewer: each warp routes its tokens
+// (route_token, as the routing kernel), the CTA synchronises, then aligns the pairs it just
+// wrote (read back through L2). Like the routing kernel it starts the forward: it clears the
+// status word and the GEMMs' work counters, and prefetches the token rows into L2.
+template <int VPL>
+__global__ void __launch_bounds__(kWarps * 32)
+    route_align_kernel(const float* __restrict__ logits, int T, int E_r, int topk, int num_shared, int renormalize,
+                       int* topk_ids, float* topk_w, int* status, const uint8_t* __restrict__ hidden,
+                       int hidden_row_bytes, int E, int block_m, int* sorted_pair_ids, int* expert_offsets,
+                       int* block_expert, int* pair_to_row, int* num_blocks, int group_rows, int2* group_info) {
+  __shared__ AlignSingleSmem sm;
+  griddep_wait();
+  griddep_launch_dependents();
+  if (threadIdx.x < 8) status[threadIdx.x] = 0;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int t = warp; t < T; t += kWarps) {
+    if (hidden != nullptr && lane == 0)
+      prefetch_l2_bulk(hidden + static_cast<size_t>(t) * hidden_row_bytes, static_cast<uint32_t>(hidden_row_bytes));
+    route_token<VPL>(logits, t, E_r, topk, num_shared, renormalize, lane, topk_ids, topk_w);
+  }
+  __syncthreads();  // every token's slots are written (global memory, visible to the CTA)
+  align_single_cta(sm, topk_ids, T * (topk + num_shared), E, block_m, sorted_pair_ids, expert_offsets, block_expert,
+                   pair_to_row, num_blocks, group_rows, group_info);
+}
+
+template <int VPL>
+cudaError_t launch_route_align_vpl(const Launch& l, const float* logits, int T, int E_r, int topk, int num_shared,
+                                   int renormalize, int* topk_ids, float* topk_w, int* status, const void* hidden,
+                                   int hidden_row_bytes, int E, int block_m, int* sorted_pair_ids,
+                                   int* expert_offsets, int* block_expert, int* pair_to_row, int* num_blocks,
+                                   int group_rows, int2* group_info) {
+  cudaLaunchConfig_t cfg;
+  cudaLaunchAttribute attr[1];
+  make_launch_config(&cfg, attr, l, dim3(1), dim3(kWarps * 32), 0);
+  return cudaLaunchKernelEx(&cfg, route_align_kernel<VPL>, logits, T, E_r, topk, num_shared, renormalize, topk_ids,
+                            topk_w, status, static_cast<const uint8_t*>(hidden), hidden_row_bytes, E, block_m,
+                            sorted_pair_ids, expert_offsets, block_expert, pair_to_row, num_blocks, group_rows,
+                            group_info);
+}
+
 bool g_scan_attr[64] = {};
 
 }  // namespace
@@ -336,6 +394,28 @@ cudaError_t launch_align(const Launch& l, const int* topk_ids, int P, int E, int
   make_launch_config(&cfg, attr, l, dim3(num_chunks), dim3(kWarps * 32), 0);
   return cudaLaunchKernelEx(&cfg, align_scatter_kernel, (const int*)topk_ids, P, E, (const int*)chunk_hist,
                             (const int*)expert_offsets, sorted_pair_ids, pair_to_row);
+}
+
+cudaError_t launch_route_align(const Launch& l, const float* logits, int T, int E_routed, int topk, int num_shared,
+                               int renormalize, int* topk_ids, float* topk_w, int* status, const void* hidden,
+                               int hidden_row_bytes, int E, int block_m, int* sorted_pair_ids, int* expert_offsets,
+                               int* block_expert, int* pair_to_row, int* num_blocks, int group_rows,
+                               int2* group_info) {
+  if (T > kWarps * kRouteAlignTokensPerWarp || T * (topk + num_shared) > kAlignChunk || E > kMaxExperts ||
+      (group_rows != 0 && (block_m != 16 || group_rows % 16 != 0 || group_rows > 256)))
+    return cudaErrorInvalidValue;
+  const int vpl = (E_routed + 31) / 32;
+#define MOE_RA(V)                                                                                              \
+  return launch_route_align_vpl<V>(l, logits, T, E_routed, topk, num_shared, renormalize, topk_ids, topk_w, status, \
+                                   hidden, hidden_row_bytes, E, block_m, sorted_pair_ids, expert_offsets,         \
+                                   block_expert, pair_to_row, num_blocks, group_rows, group_info)
+  if (vpl <= 1) MOE_RA(1);
+  if (vpl <= 2) MOE_RA(2);
+  if (vpl <= 4) MOE_RA(4);
+  if (vpl <= 8) MOE_RA(8);
+  if (vpl <= 16) MOE_RA(16);
+  MOE_RA(32);
+#undef MOE_RA
 }
 
 }  // namespace moe

@@ -265,6 +265,16 @@ moe_status_t run_route(const Plan& pl, const float* logits, void* ws, const Laun
                                        pl.H * 2));
 }
 
+// Routing and align of a small batch in one kernel (the same results as run_route, run_align).
+moe_status_t run_route_align(const Plan& pl, const float* logits, void* ws, const Launch& l, const void* hidden) {
+  const auto& L = pl.lay;
+  return cuda_status(moe::launch_route_align(
+      l, logits, pl.T, pl.Er, pl.topk, pl.Es, pl.renorm, ws_ptr<int>(ws, L.topk_ids), ws_ptr<float>(ws, L.topk_w),
+      ws_ptr<int>(ws, L.status), pl.fp8 ? nullptr : hidden, pl.H * 2, pl.E, pl.bm, ws_ptr<int>(ws, L.sorted_pair_ids),
+      ws_ptr<int>(ws, L.expert_offsets), ws_ptr<int>(ws, L.block_expert), ws_ptr<int>(ws, L.pair_to_row),
+      ws_ptr<int>(ws, L.num_blocks), pl.grp, pl.grp != 0 ? ws_ptr<int2>(ws, L.group_info) : nullptr));
+}
+
 moe_status_t run_align(const Plan& pl, void* ws, const Launch& l) {
   const auto& L = pl.lay;
   return cuda_status(moe::launch_align(l, ws_ptr<int>(ws, L.topk_ids), static_cast<int>(pl.P), pl.E, pl.bm,
@@ -535,10 +545,12 @@ Launch launch_of(const moe_problem_t* p, moe_stream_t stream) {
   return l;
 }
 
-// Steps 2-5 (everything after the routing step) on routing already in the workspace.
+// Steps 2-5 (everything after the routing step) on routing already in the workspace; with
+// `aligned` the align step has run too.
 moe_status_t forward_after_route(const Plan& pl, const Launch& l, const void* hidden, const void* w13, const void* w2,
-                                 const float* s13, const float* s2, void* out, void* ws, int num_sms) {
-  moe_status_t st = run_align(pl, ws, l);
+                                 const float* s13, const float* s2, void* out, void* ws, int num_sms,
+                                 bool aligned = false) {
+  moe_status_t st = aligned ? MOE_OK : run_align(pl, ws, l);
   if (st == MOE_OK && (pl.fp8 || pl.nv)) st = run_quant_act(pl, hidden, ws, l);
   if (st == MOE_OK) st = run_permute(pl, hidden, ws, l, num_sms);
   if (st == MOE_OK) st = run_gemm1(pl, hidden, w13, s13, ws, l, num_sms);
@@ -551,9 +563,11 @@ moe_status_t forward_device(const Plan& pl, const moe_problem_t* p, const void* 
                             const void* w13, const void* w2, const float* s13, const float* s2, void* out,
                             void* ws, moe_stream_t stream, int num_sms) {
   const Launch l = launch_of(p, stream);
-  const moe_status_t st = run_route(pl, logits, ws, l, hidden);
+  // a small batch (one align chunk, at most 16 tokens): routing and align in one kernel
+  const bool fused = pl.T <= 8 * moe::kRouteAlignTokensPerWarp && pl.lay.num_chunks == 1;
+  const moe_status_t st = fused ? run_route_align(pl, logits, ws, l, hidden) : run_route(pl, logits, ws, l, hidden);
   if (st != MOE_OK) return st;
-  return forward_after_route(pl, l, hidden, w13, w2, s13, s2, out, ws, num_sms);
+  return forward_after_route(pl, l, hidden, w13, w2, s13, s2, out, ws, num_sms, fused);
 }
 
 // A weight-scale pointer as the problem's format wants it: fp32 (4-byte aligned) for the

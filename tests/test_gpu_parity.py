@@ -420,6 +420,40 @@ def test_decode_both_row_tilings(T, bm):
     assert err_beyond_rounding(bf16_to_f64(out), ref) <= BF16_TOL
 
 
+FUSED_ROUTE_ALIGN = {
+    "tiny": CONFIGS["tiny"],
+    "decode_T1": CONFIGS["decode_T1"],
+    "decode_T16": CONFIGS["decode_T16"],
+    "shared_t12": _small("shared_t12", T=12, H=256, E=12, topk=3, I=256, num_shared=1),
+}
+
+
+@pytest.mark.parametrize("name", sorted(FUSED_ROUTE_ALIGN))
+def test_fused_route_align_matches_the_separate_steps(name):
+    # batches of at most 16 tokens route and align in one kernel inside the forward; its
+    # routing, permutation, offsets and row groups must be those of the separate route and
+    # align steps, bit for bit
+    cfg = FUSED_ROUTE_ALIGN[name]
+    assert cfg.T <= 16
+    run = GpuForward(cfg)
+    run.forward()
+    keys = ["topk_ids", "topk_w", "sorted_pair_ids", "expert_offsets", "pair_to_row", "num_blocks", "group_info"]
+    fused = {k: v.clone() for k, v in moe.read_workspace(run.prob, run.ws).items() if k in keys}
+    run.ws.zero_()
+    moe.stage_route(run.prob, run.logits, run.ws)
+    moe.stage_align(run.prob, run.ws)
+    torch.cuda.synchronize()
+    staged = moe.read_workspace(run.prob, run.ws)
+    # only the written prefixes: the padded rows and the row groups that align produced
+    rows = int(staged["expert_offsets"][-1])
+    groups = int(staged["num_blocks"][1])
+    assert int(fused["expert_offsets"][-1]) == rows and int(fused["num_blocks"][1]) == groups
+    fused["sorted_pair_ids"], staged["sorted_pair_ids"] = fused["sorted_pair_ids"][:rows], staged["sorted_pair_ids"][:rows]
+    fused["group_info"], staged["group_info"] = fused["group_info"][:groups], staged["group_info"][:groups]
+    for k in keys:
+        assert torch.equal(fused[k].cpu(), staged[k].cpu()), k
+
+
 # ---- caller-supplied routing (the routed variant) -------------------------------------
 
 def _routed_call(run, ids, w, cfg):
