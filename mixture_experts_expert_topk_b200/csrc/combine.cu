@@ -1,9 +1,8 @@
 // Step 5 of the layer: deterministic combine back to token order.
 //
-// out[t, h] = sum_{j=0}^{k'-1} y[pair_to_row[t*k' + j], h], where y (sorted row order)
-// already carries the routing weight (GEMM2 epilogue). The sum runs in slot order
-// j = 0, 1, ..., k'-1 in fp32 and is rounded once to bf16, so the result does not depend
-// on scheduling. The output is bf16 of the hidden shape ("FlashInfer TRTLLM-Gen MoE kernel
+// out[t, h] = sum_{j=0}^{k'-1} w_tj * y[pair_to_row[t*k' + j], h], y in sorted row order
+// (GEMM2's output). The sum runs in slot order j = 0, 1, ..., k'-1 in fp32 and is rounded
+// once to bf16, so the result does not depend on scheduling. The output is bf16 of the hidden shape ("FlashInfer TRTLLM-Gen MoE kernel
 // optimisation: NemotronH support", sglang PR 21321, section 1: the fused op returns a
 // bf16 tensor shaped like hidden_states).
 //

@@ -188,14 +188,20 @@ __device__ __forceinline__ uint32_t step_bytes(int kcs, int n) {
   if (kKind == 4) return b + static_cast<uint32_t>(kcs) * 2u * kNvChunkScaleBytes;
   return b;
 }
-// K chunks per step: NVFP4 steps take at most two (their scale buffers hold two chunks)
+// K chunks per step: NVFP4 steps take at most two (their scale buffers hold two chunks);
+// per-tensor FP8 and MXFP8 groups of more than 128 rows take two (one 16 KB weight copy per
+// step measured slower for these kinds, while bf16 keeps one: its GEMMs ran slower with
+// two, from the fewer steps in flight)
 template <int kKind>
 __device__ __forceinline__ int step_chunks(int n) {
-  return kKind == 4 ? min(chunks_per_step(n), 2) : chunks_per_step(n);
+  if (kKind == 4) return min(chunks_per_step(n), 2);
+  if ((kKind == 1 || kKind == 2) && n > 128) return 2;
+  return chunks_per_step(n);
 }
 static_assert(4 * (kTileW + 32 * kChunkBytes + kSfW + kSfX) <= kRingBytes / 2 &&
-                  kTileW + kMxGroupRows * kChunkBytes + kSfW + kSfX <= kRingBytes / 2,
+                  2 * (kTileW + kMxGroupRows * kChunkBytes + kSfW + kSfX) + 1023 <= kRingBytes / 2,
               "at least two MXFP8 steps fit the ring");
+static_assert(2 * (kTileW + kNMax * kChunkBytes) <= kRingBytes / 2, "at least two per-tensor FP8 steps fit the ring");
 static_assert(4 * (kTileW + 32 * kChunkBytes) <= kRingBytes / 2 && 2 * (kTileW + 128 * kChunkBytes) <= kRingBytes / 2 &&
                   kTileW + kNMax * kChunkBytes <= kRingBytes / 2,
               "at least two steps fit the ring");
