@@ -322,13 +322,17 @@ __global__ void __launch_bounds__(kWarps * 32)
 // align chunk) in one CTA, one kernel boundary fewer: each warp routes its tokens
 // (route_token, as the routing kernel), the CTA synchronises, then aligns the pairs it just
 // wrote (read back through L2). Like the routing kernel it starts the forward: it clears the
-// status word and the GEMMs' work counters, and prefetches the token rows into L2.
+// status word and the GEMMs' work counters, and prefetches the token rows into L2. With xs
+// (bf16, at most kFusedPermutePairs pairs) it also copies each pair's token row into its
+// row group (the permute step's layout; padding rows are not written), a warp per pair: the
+// group is found by binary search over the row groups just written.
 template <int VPL>
 __global__ void __launch_bounds__(kWarps * 32)
     route_align_kernel(const float* __restrict__ logits, int T, int E_r, int topk, int num_shared, int renormalize,
                        int* topk_ids, float* topk_w, int* status, const uint8_t* __restrict__ hidden,
                        int hidden_row_bytes, int E, int block_m, int* sorted_pair_ids, int* expert_offsets,
-                       int* block_expert, int* pair_to_row, int* num_blocks, int group_rows, int2* group_info) {
+                       int* block_expert, int* pair_to_row, int* num_blocks, int group_rows, int2* group_info,
+                       uint8_t* xs) {
   __shared__ AlignSingleSmem sm;
   griddep_wait();
   griddep_launch_dependents();
@@ -340,8 +344,31 @@ __global__ void __launch_bounds__(kWarps * 32)
     route_token<VPL>(logits, t, E_r, topk, num_shared, renormalize, lane, topk_ids, topk_w);
   }
   __syncthreads();  // every token's slots are written (global memory, visible to the CTA)
-  align_single_cta(sm, topk_ids, T * (topk + num_shared), E, block_m, sorted_pair_ids, expert_offsets, block_expert,
-                   pair_to_row, num_blocks, group_rows, group_info);
+  const int P = T * (topk + num_shared);
+  align_single_cta(sm, topk_ids, P, E, block_m, sorted_pair_ids, expert_offsets, block_expert, pair_to_row,
+                   num_blocks, group_rows, group_info);
+  if (xs == nullptr) return;
+  __syncthreads();  // pair_to_row, the row groups and their count are written
+  const int G = __ldcg(num_blocks + 1);
+  const int pieces = hidden_row_bytes >> 4;  // 16-byte pieces of a row: 8 per 128-byte chunk
+  for (int p = warp; p < P; p += kWarps) {
+    const int pos = __ldcg(pair_to_row + p);
+    if (pos < 0) continue;  // an unroutable id (warp-uniform)
+    int lo = 0, hi = G - 1;  // the last group starting at or before pos
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (__ldcg(&group_info[mid].x) <= pos) lo = mid; else hi = mid - 1;
+    }
+    const int2 gi = __ldcg(group_info + lo);
+    const int n = gi.y >> 16, j = pos - gi.x;
+    const uint4* src = reinterpret_cast<const uint4*>(hidden + static_cast<size_t>(p / (topk + num_shared)) * hidden_row_bytes);
+    uint8_t* base = xs + static_cast<size_t>(gi.x) * hidden_row_bytes;
+    for (int q = lane; q < pieces; q += 32) {
+      const int c = q >> 3;
+      *reinterpret_cast<uint4*>(base + static_cast<size_t>(c) * n * 128 + j * 128 + (((q & 7) ^ (j & 7)) << 4)) =
+          __ldg(src + q);
+    }
+  }
 }
 
 template <int VPL>
@@ -349,14 +376,14 @@ cudaError_t launch_route_align_vpl(const Launch& l, const float* logits, int T, 
                                    int renormalize, int* topk_ids, float* topk_w, int* status, const void* hidden,
                                    int hidden_row_bytes, int E, int block_m, int* sorted_pair_ids,
                                    int* expert_offsets, int* block_expert, int* pair_to_row, int* num_blocks,
-                                   int group_rows, int2* group_info) {
+                                   int group_rows, int2* group_info, void* xs) {
   cudaLaunchConfig_t cfg;
   cudaLaunchAttribute attr[1];
   make_launch_config(&cfg, attr, l, dim3(1), dim3(kWarps * 32), 0);
   return cudaLaunchKernelEx(&cfg, route_align_kernel<VPL>, logits, T, E_r, topk, num_shared, renormalize, topk_ids,
                             topk_w, status, static_cast<const uint8_t*>(hidden), hidden_row_bytes, E, block_m,
                             sorted_pair_ids, expert_offsets, block_expert, pair_to_row, num_blocks, group_rows,
-                            group_info);
+                            group_info, static_cast<uint8_t*>(xs));
 }
 
 bool g_scan_attr[64] = {};
@@ -400,15 +427,18 @@ cudaError_t launch_route_align(const Launch& l, const float* logits, int T, int 
                                int renormalize, int* topk_ids, float* topk_w, int* status, const void* hidden,
                                int hidden_row_bytes, int E, int block_m, int* sorted_pair_ids, int* expert_offsets,
                                int* block_expert, int* pair_to_row, int* num_blocks, int group_rows,
-                               int2* group_info) {
+                               int2* group_info, void* xs) {
   if (T > kWarps * kRouteAlignTokensPerWarp || T * (topk + num_shared) > kAlignChunk || E > kMaxExperts ||
       (group_rows != 0 && (block_m != 16 || group_rows % 16 != 0 || group_rows > 256)))
+    return cudaErrorInvalidValue;
+  if (xs != nullptr && (group_rows == 0 || hidden == nullptr || T * (topk + num_shared) > kFusedPermutePairs ||
+                        hidden_row_bytes % 128 != 0))
     return cudaErrorInvalidValue;
   const int vpl = (E_routed + 31) / 32;
 #define MOE_RA(V)                                                                                              \
   return launch_route_align_vpl<V>(l, logits, T, E_routed, topk, num_shared, renormalize, topk_ids, topk_w, status, \
                                    hidden, hidden_row_bytes, E, block_m, sorted_pair_ids, expert_offsets,         \
-                                   block_expert, pair_to_row, num_blocks, group_rows, group_info)
+                                   block_expert, pair_to_row, num_blocks, group_rows, group_info, xs)
   if (vpl <= 1) MOE_RA(1);
   if (vpl <= 2) MOE_RA(2);
   if (vpl <= 4) MOE_RA(4);

@@ -265,14 +265,17 @@ moe_status_t run_route(const Plan& pl, const float* logits, void* ws, const Laun
                                        pl.H * 2));
 }
 
-// Routing and align of a small batch in one kernel (the same results as run_route, run_align).
-moe_status_t run_route_align(const Plan& pl, const float* logits, void* ws, const Launch& l, const void* hidden) {
+// Routing and align of a small batch in one kernel (the same results as run_route, run_align);
+// with `permute` also the bf16 permute step (the same xs as run_permute).
+moe_status_t run_route_align(const Plan& pl, const float* logits, void* ws, const Launch& l, const void* hidden,
+                             bool permute) {
   const auto& L = pl.lay;
   return cuda_status(moe::launch_route_align(
       l, logits, pl.T, pl.Er, pl.topk, pl.Es, pl.renorm, ws_ptr<int>(ws, L.topk_ids), ws_ptr<float>(ws, L.topk_w),
       ws_ptr<int>(ws, L.status), pl.fp8 ? nullptr : hidden, pl.H * 2, pl.E, pl.bm, ws_ptr<int>(ws, L.sorted_pair_ids),
       ws_ptr<int>(ws, L.expert_offsets), ws_ptr<int>(ws, L.block_expert), ws_ptr<int>(ws, L.pair_to_row),
-      ws_ptr<int>(ws, L.num_blocks), pl.grp, pl.grp != 0 ? ws_ptr<int2>(ws, L.group_info) : nullptr));
+      ws_ptr<int>(ws, L.num_blocks), pl.grp, pl.grp != 0 ? ws_ptr<int2>(ws, L.group_info) : nullptr,
+      permute ? ws_ptr<void>(ws, L.xs) : nullptr));
 }
 
 moe_status_t run_align(const Plan& pl, void* ws, const Launch& l) {
@@ -326,7 +329,8 @@ long long est_row_tiles(const Plan& pl) {
 }
 
 moe_status_t run_gemm1(const Plan& pl_in, const void* hidden, const void* w13, const float* w13_scale, void* ws,
-                       const Launch& l, int num_sms) {
+                       const Launch& l, int num_sms,
+                       bool w_early = true) {
   Plan pl = pl_in;
   if (!pl.fp8) pl.bn1 = moe::pick_bn(pl.N1, est_row_tiles(pl), num_sms);
   const auto& L = pl.lay;
@@ -349,6 +353,9 @@ moe_status_t run_gemm1(const Plan& pl_in, const void* hidden, const void* w13, c
     // both operands load with bulk copies
     moe::SwapOperands o{};
     o.w = w13;
+    // the kernel before GEMM1 (the permute) does not write the row groups, unless the
+    // permute ran inside the routing + align kernel
+    o.w_early = w_early ? 1 : 0;
     o.x = ws_ptr<void>(ws, L.xs);
     o.out_chunks = pl.pt ? pl.I / 128 : (pl.I + 63) / 64;
     o.fp8 = pl.pt;
@@ -476,6 +483,7 @@ moe_status_t run_gemm2(const Plan& pl_in, const void* w2, const float* w2_scale,
   if (pl.bm == 16) {
     moe::SwapOperands o{};
     o.w = w2;
+    o.w_early = 1;  // the kernel before GEMM2 (GEMM1 or the activation quantiser) writes no row groups
     o.x = ws_ptr<void>(ws, L.act);
     o.out_chunks = 0;
     o.fp8 = pl.pt;
@@ -546,14 +554,14 @@ Launch launch_of(const moe_problem_t* p, moe_stream_t stream) {
 }
 
 // Steps 2-5 (everything after the routing step) on routing already in the workspace; with
-// `aligned` the align step has run too.
+// `aligned` the align step has run too, with `permuted` also the permute step.
 moe_status_t forward_after_route(const Plan& pl, const Launch& l, const void* hidden, const void* w13, const void* w2,
                                  const float* s13, const float* s2, void* out, void* ws, int num_sms,
-                                 bool aligned = false) {
+                                 bool aligned = false, bool permuted = false) {
   moe_status_t st = aligned ? MOE_OK : run_align(pl, ws, l);
   if (st == MOE_OK && (pl.fp8 || pl.nv)) st = run_quant_act(pl, hidden, ws, l);
-  if (st == MOE_OK) st = run_permute(pl, hidden, ws, l, num_sms);
-  if (st == MOE_OK) st = run_gemm1(pl, hidden, w13, s13, ws, l, num_sms);
+  if (st == MOE_OK && !permuted) st = run_permute(pl, hidden, ws, l, num_sms);
+  if (st == MOE_OK) st = run_gemm1(pl, hidden, w13, s13, ws, l, num_sms, !permuted);
   if (st == MOE_OK) st = run_gemm2(pl, w2, s2, ws, l, num_sms);
   if (st == MOE_OK) st = run_combine(pl, out, ws, l);
   return st;
@@ -563,11 +571,15 @@ moe_status_t forward_device(const Plan& pl, const moe_problem_t* p, const void* 
                             const void* w13, const void* w2, const float* s13, const float* s2, void* out,
                             void* ws, moe_stream_t stream, int num_sms) {
   const Launch l = launch_of(p, stream);
-  // a small batch (one align chunk, at most 16 tokens): routing and align in one kernel
+  // a small batch (one align chunk, at most 16 tokens): routing and align in one kernel, and
+  // for bf16 row groups of at most kFusedPermutePairs pairs the permute too
   const bool fused = pl.T <= 8 * moe::kRouteAlignTokensPerWarp && pl.lay.num_chunks == 1;
-  const moe_status_t st = fused ? run_route_align(pl, logits, ws, l, hidden) : run_route(pl, logits, ws, l, hidden);
+  const bool bf16 = !(pl.fp8 || pl.pt || pl.mx || pl.nv);
+  const bool permute = fused && bf16 && pl.bm == 16 && pl.P <= moe::kFusedPermutePairs;
+  const moe_status_t st =
+      fused ? run_route_align(pl, logits, ws, l, hidden, permute) : run_route(pl, logits, ws, l, hidden);
   if (st != MOE_OK) return st;
-  return forward_after_route(pl, l, hidden, w13, w2, s13, s2, out, ws, num_sms, fused);
+  return forward_after_route(pl, l, hidden, w13, w2, s13, s2, out, ws, num_sms, fused, permute);
 }
 
 // A weight-scale pointer as the problem's format wants it: fp32 (4-byte aligned) for the

@@ -177,6 +177,7 @@ struct Args {
   int ws_rows;             // 128-row scale blocks per expert
   int up_block;            // gated GEMM1: I / 128; 0 otherwise
   int8_t* y_exp;           // GEMM2: the power-of-two exponent of each 32 columns of y
+  int w_early;             // 1: the previous kernel does not write the row groups (see below)
 };
 
 // Ring bytes of one K step of kcs chunks for a group of n rows. MXFP8 steps add the scale
@@ -330,9 +331,15 @@ __global__ void __launch_bounds__(threads_for<kKind>(), 1) gemm_swap_kernel(cons
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  // everything above overlaps the previous kernel; inputs are read only after this
-  griddep_wait();
-  griddep_launch_dependents();
+  // Everything above overlaps the previous kernel. With w_early the scheduler + W producer
+  // (warp 0) starts right away: it reads only the weights, align's row groups and the work
+  // counter, which the launcher vouches were complete before the previous kernel (itself
+  // behind its own wait) could launch this one, so the first weight copies overlap that
+  // kernel's tail. Every other role waits for the previous kernel's output (X) first.
+  if (warp != 0 || !a.w_early) {
+    griddep_wait();
+    griddep_launch_dependents();
+  }
 
   // bytes of X per row: a 128-byte chunk row per K chunk (FP8 block-128: and its fp32 scale)
   const size_t x_row_bytes = static_cast<size_t>(a.k_chunks) * (kB128 ? kB128RowBytesPerChunk : kChunkBytes);
@@ -581,6 +588,14 @@ __global__ void __launch_bounds__(threads_for<kKind>(), 1) gemm_swap_kernel(cons
       const int x_row = __shfl_sync(0xffffffffu, t.x, 0);
       const int expert = __shfl_sync(0xffffffffu, t.z, 0);
       const int mt = __shfl_sync(0xffffffffu, t.w, 0);
+      // GEMM1: a group's padding rows (pair id P) are a suffix of fewer than 16 rows (an
+      // expert's segment is its pairs, then sentinels up to a multiple of 16), so its real
+      // rows are n minus the sentinels among its last 16
+      int n_real = n;
+      if (a.mode == 0) {
+        const bool sentinel = lane < 16 && __ldg(a.sorted_pair_ids + x_row + n - 16 + lane) >= a.num_pairs;
+        n_real = n - __popc(__ballot_sync(0xffffffffu, sentinel));
+      }
       // FP8 per-tensor, NVFP4: the accumulator's dequantisation scale (the weight's and the
       // X operand's tensor scales; GEMM1: before the activation)
       const float dq = (kFp8 || kNv) ? __ldg(a.w_scale + expert) * a.in_scale : 1.0f;
@@ -618,37 +633,41 @@ __global__ void __launch_bounds__(threads_for<kKind>(), 1) gemm_swap_kernel(cons
           }
           if (lane < 16 || full)
             a.y_exp[static_cast<size_t>(x_row + c0 + lane) * (a.out_cols >> 5) + (col >> 5)] = static_cast<int8_t>(s);
-        } else if (!gated) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            if (j == 16 && !full) break;
-            const int row = c0 + j;
-            const float z = fmaxf(__uint_as_float(v[j]) * dq, 0.f);
-            uint8_t* dst = act_grp + row * kChunkBytes + ((((fo >> 4) ^ row) & 7) << 4) + (fo & 15);
-            if (kFp8)
-              *dst = __nv_cvt_float_to_fp8(z * z * a.act_inv, __NV_SATFINITE, __NV_E4M3);
-            else
-              *reinterpret_cast<__nv_bfloat16*>(dst) = __float2bfloat16_rn(z * z);
-          }
         } else {
-          // lane pair (2m, 2m+1) = (gate, up) of feature m. The even lane finishes tokens
-          // 0..15 of the batch, the odd lane tokens 16..31: each passes the other the half
-          // it needs, so every lane evaluates the activation on 16 tokens.
+          // GEMM1: a group's padding rows store zeros whatever X held there (the permute does
+          // not write them), so GEMM2 sees zero rows
+          if (!gated) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const float mine_lo = __uint_as_float(v[j]) * dq;       // even: gate_j; odd: up_j
-            const float mine_hi = __uint_as_float(v[16 + j]) * dq;  // even: gate_{16+j}; odd: up_{16+j}
-            const float other = __shfl_xor_sync(0xffffffffu, odd ? mine_lo : mine_hi, 1);
-            const float g = odd ? other : mine_lo;
-            const float u = odd ? mine_hi : other;
-            const int row = c0 + (odd ? 16 + j : j);
-            if (!odd || full) {
-              const float h = gated_act(g, u, a.activation);
+            for (int j = 0; j < 32; ++j) {
+              if (j == 16 && !full) break;
+              const int row = c0 + j;
+              const float z = row >= n_real ? 0.f : fmaxf(__uint_as_float(v[j]) * dq, 0.f);
               uint8_t* dst = act_grp + row * kChunkBytes + ((((fo >> 4) ^ row) & 7) << 4) + (fo & 15);
               if (kFp8)
-                *dst = __nv_cvt_float_to_fp8(h * a.act_inv, __NV_SATFINITE, __NV_E4M3);
+                *dst = __nv_cvt_float_to_fp8(z * z * a.act_inv, __NV_SATFINITE, __NV_E4M3);
               else
-                *reinterpret_cast<__nv_bfloat16*>(dst) = __float2bfloat16_rn(h);
+                *reinterpret_cast<__nv_bfloat16*>(dst) = __float2bfloat16_rn(z * z);
+            }
+          } else {
+            // lane pair (2m, 2m+1) = (gate, up) of feature m. The even lane finishes tokens
+            // 0..15 of the batch, the odd lane tokens 16..31: each passes the other the half
+            // it needs, so every lane evaluates the activation on 16 tokens.
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const float mine_lo = __uint_as_float(v[j]) * dq;       // even: gate_j; odd: up_j
+              const float mine_hi = __uint_as_float(v[16 + j]) * dq;  // even: gate_{16+j}; odd: up_{16+j}
+              const float other = __shfl_xor_sync(0xffffffffu, odd ? mine_lo : mine_hi, 1);
+              const float g = odd ? other : mine_lo;
+              const float u = odd ? mine_hi : other;
+              const int row = c0 + (odd ? 16 + j : j);
+              if (!odd || full) {
+                const float h = row >= n_real ? 0.f : gated_act(g, u, a.activation);
+                uint8_t* dst = act_grp + row * kChunkBytes + ((((fo >> 4) ^ row) & 7) << 4) + (fo & 15);
+                if (kFp8)
+                  *dst = __nv_cvt_float_to_fp8(h * a.act_inv, __NV_SATFINITE, __NV_E4M3);
+                else
+                  *reinterpret_cast<__nv_bfloat16*>(dst) = __float2bfloat16_rn(h);
+              }
             }
           }
         }
@@ -826,6 +845,7 @@ cudaError_t launch_gemm_swap(const Launch& l, int mode, const SwapOperands& o, c
   a.up_block = o.up_block;
   a.y_exp = b.out_exp;
   if (mode == 1 && (a.y_exp == nullptr || s.out_cols % 32 != 0)) return cudaErrorInvalidValue;
+  a.w_early = o.w_early;
   cudaLaunchConfig_t cfg;
   cudaLaunchAttribute attr[1];
   make_launch_config(&cfg, attr, l, dim3(s.num_sms), dim3(kind == 3 ? threads_for<3>() : kThreads), kSmemBytes);

@@ -11,6 +11,7 @@ constexpr int kMaxExperts = 1024;  // routed + shared
 constexpr int kMaxSlots = 16;      // k' = topk + num_shared
 constexpr int kAlignChunk = 2048;  // pairs per align chunk
 constexpr int kRouteAlignTokensPerWarp = 2;  // fused routing + align: tokens per warp (8 warps)
+constexpr int kFusedPermutePairs = 64;       // fused routing + align also permutes (bf16) up to this many pairs
 // Status word value (beyond the wait timeouts 0x10000 | site): caller-supplied routing held
 // an expert id outside [0, E_r) (the pair was dropped: id 0, weight 0).
 constexpr int kStatusBadRouting = 0x20000;
@@ -45,12 +46,14 @@ cudaError_t launch_align(const Launch& l, const int* topk_ids, int P, int E, int
                          int* expert_offsets, int* block_expert, int* pair_to_row,
                          int* num_blocks, int group_rows, int2* group_info);
 // Routing (as launch_route) and align (as launch_align with one chunk) of a batch of at most
-// 8 * kRouteAlignTokensPerWarp tokens and kAlignChunk pairs in one single-CTA kernel.
+// 8 * kRouteAlignTokensPerWarp tokens and kAlignChunk pairs in one single-CTA kernel; with xs
+// (bf16 hidden rows of hidden_row_bytes, row groups, at most kFusedPermutePairs pairs) also
+// the permute step into xs.
 cudaError_t launch_route_align(const Launch& l, const float* logits, int T, int E_routed, int topk, int num_shared,
                                int renormalize, int* topk_ids, float* topk_w, int* status, const void* hidden,
                                int hidden_row_bytes, int E, int block_m, int* sorted_pair_ids, int* expert_offsets,
                                int* block_expert, int* pair_to_row, int* num_blocks, int group_rows,
-                               int2* group_info);
+                               int2* group_info, void* xs);
 // The token rows of every row group in the row-group order of the swapped-operand GEMM
 // (gemm_swap.cu): row j of the group starting at x_row is hidden[sorted_pair_ids[x_row +
 // j] / k_total] (zero for padding), H / 64 chunks of 128 bytes, swizzled.
@@ -135,6 +138,10 @@ struct SwapOperands {
   // w_sf / x_sf = the tiled weight scales / the X scale blocks (kNvChunkScaleBytes per 128-row
   // block per chunk); w_scale [E] and in_scale the tensor scales (dequantised in the epilogue)
   int nv;
+  // 1: the kernel launched before this GEMM does not write the row groups (they were complete
+  // before it could launch this one), so the weight stream may start before the dependency
+  // wait; 0: everything waits
+  int w_early;
 };
 // Row groups of the MXFP8 swapped-operand GEMMs: at most this many rows, so that two
 // accumulators leave a quarter of TMEM for the block scales.

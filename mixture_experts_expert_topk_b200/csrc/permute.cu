@@ -1,7 +1,9 @@
 // GEMM1's token rows in the row-group order of the swapped-operand GEMM (gemm_swap.cu).
 //
 // For each row group (x_row, n) of align's output, row j of the group is the hidden row of
-// its pair's token, hidden[sorted_pair_ids[x_row + j] / k'], or zero for a padding row.
+// its pair's token, hidden[sorted_pair_ids[x_row + j] / k']; padding rows are not written
+// (GEMM1 stores zeros for them whatever they hold, since an MMA output column depends only on
+// its own X column).
 // The group occupies bytes [x_row * H * 2, (x_row + n) * H * 2) of xs; 64-column chunk c of
 // it is n rows of 128 bytes at offset c * n * 128, the 16-byte piece q of row j stored at
 // position q ^ (j % 8) (the 128-byte swizzle the MMA reads). The GEMM then loads each K
@@ -57,7 +59,7 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
         for (int r = 0; r < kRowsPerStep; ++r) {
           const int j = j0 + r;
-          if (j >= n) continue;
+          if (j >= n || src[r] == nullptr) continue;  // padding rows are not written
 #pragma unroll
           for (int i = 0; i < kPiecesPerLane; ++i) {
             const int p = p0 + 32 * i;
@@ -116,7 +118,7 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
         for (int r = 0; r < kRowsPerStep; ++r) {
           const int j = j0 + r;
-          if (j >= n) continue;
+          if (j >= n || src[r] == nullptr) continue;  // padding rows are not written
 #pragma unroll
           for (int i = 0; i < kQPieces; ++i) {
             const int p = p0 + 32 * i;
@@ -204,7 +206,7 @@ __global__ void __launch_bounds__(kThreads)
             amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
             const int e = mx_exponent(amax);
             const float inv = mx_inv(e);
-            if (p < pieces && j < n) {
+            if (p < pieces && j < n && src[r] != nullptr) {  // padding rows are not written
               const int c = p >> 3, q = p & 7;
               *reinterpret_cast<uint4*>(base + static_cast<size_t>(c) * n * 128 + j * 128 + ((q ^ (j & 7)) << 4)) =
                   make_uint4(mx_e4m3x4(v[0], v[1], v[2], v[3], inv), mx_e4m3x4(v[4], v[5], v[6], v[7], inv),
@@ -306,8 +308,8 @@ __device__ __forceinline__ uint32_t quant_group_1x128(float x0, float x1, float 
 // FP8 block-128: the token rows, already quantised once per token (quant_act_kernel: e4m3
 // codes [T, H] and fp32 1x128 scales [T, H/128]), copied into the X layout of their row
 // groups. A warp copies one row: lane l moves 16-byte pieces l, l + 32, ... of the row's
-// codes (all loads first) and lanes 0..KC-1 its scales. Padding rows get zero codes and
-// scale 1 (an all-zero group).
+// codes (all loads first) and lanes 0..KC-1 its scales. Padding rows are not written (GEMM1
+// stores zeros for them whatever they hold).
 constexpr int kB128Pieces = 4;  // 16-byte pieces per lane per pass (a 2 KB row in one pass)
 __global__ void __launch_bounds__(kThreads)
     permute_b128_rows_kernel(const uint4* __restrict__ xq, const float* __restrict__ xq_scale, int H,
@@ -324,13 +326,14 @@ __global__ void __launch_bounds__(kThreads)
     uint8_t* base = xs + static_cast<size_t>(x_row) * KC * kB128RowBytesPerChunk;
     for (int j = blockIdx.y * (kThreads / 32) + warp; j < n; j += gridDim.y * (kThreads / 32)) {
       const int pid = sorted_pair_ids[x_row + j];
-      const long long tok = pid < P ? pid / k_total : -1;
+      if (pid >= P) continue;  // a padding row (warp-uniform)
+      const long long tok = pid / k_total;
       for (int p0 = 0; p0 < pieces; p0 += 32 * kB128Pieces) {
         uint4 v[kB128Pieces];
 #pragma unroll
         for (int i = 0; i < kB128Pieces; ++i) {
           const int p = p0 + lane + 32 * i;
-          v[i] = (tok >= 0 && p < pieces) ? __ldg(xq + tok * pieces + p) : make_uint4(0u, 0u, 0u, 0u);
+          v[i] = p < pieces ? __ldg(xq + tok * pieces + p) : make_uint4(0u, 0u, 0u, 0u);
         }
 #pragma unroll
         for (int i = 0; i < kB128Pieces; ++i) {
@@ -345,7 +348,7 @@ __global__ void __launch_bounds__(kThreads)
       for (int c = lane; c < KC; c += 32) {
         size_t co, so;
         b128_offsets(n, KC, c, j, co, so);
-        *reinterpret_cast<float*>(base + so) = tok >= 0 ? __ldg(xq_scale + tok * KC + c) : 1.0f;
+        *reinterpret_cast<float*>(base + so) = __ldg(xq_scale + tok * KC + c);
       }
     }
   }
@@ -403,7 +406,8 @@ __global__ void __launch_bounds__(kThreads)
 // other 8-bit layouts), scales into the group's 2048-byte block per chunk (byte 512 mm +
 // 16 (j % 32) + 4 (j / 32) + k: group row j, 16-value block 16 c + 4 mm + k). A warp copies
 // one row; lane l moves 16-byte code pieces l, l + 32, ... and the row's scale bytes 4l..4l+3
-// (blocks 4l..4l+3: one MMA's four). Padding rows are zero codes and zero scales.
+// (blocks 4l..4l+3: one MMA's four). Padding rows are not written (GEMM1 stores zeros for
+// them whatever they hold).
 __global__ void __launch_bounds__(kThreads)
     permute_nvfp4_rows_kernel(const uint4* __restrict__ xq, const uint8_t* __restrict__ xq_scale, int H,
                               const int* __restrict__ sorted_pair_ids, const int* __restrict__ num_groups,
@@ -421,13 +425,14 @@ __global__ void __launch_bounds__(kThreads)
     uint8_t* sfb = xs_sf + static_cast<size_t>(x_row >> 4) * KC * kNvChunkScaleBytes;
     for (int j = blockIdx.y * (kThreads / 32) + warp; j < n; j += gridDim.y * (kThreads / 32)) {
       const int pid = sorted_pair_ids[x_row + j];
-      const long long tok = pid < P ? pid / k_total : -1;
+      if (pid >= P) continue;  // a padding row (warp-uniform)
+      const long long tok = pid / k_total;
       for (int p0 = 0; p0 < pieces; p0 += 32 * kB128Pieces) {
         uint4 v[kB128Pieces];
 #pragma unroll
         for (int i = 0; i < kB128Pieces; ++i) {
           const int p = p0 + lane + 32 * i;
-          v[i] = (tok >= 0 && p < pieces) ? __ldg(xq + tok * pieces + p) : make_uint4(0u, 0u, 0u, 0u);
+          v[i] = p < pieces ? __ldg(xq + tok * pieces + p) : make_uint4(0u, 0u, 0u, 0u);
         }
 #pragma unroll
         for (int i = 0; i < kB128Pieces; ++i) {
@@ -438,7 +443,7 @@ __global__ void __launch_bounds__(kThreads)
         }
       }
       for (int b0 = 4 * lane; b0 < sbytes; b0 += 128) {
-        const uint32_t w = tok >= 0 ? __ldg(reinterpret_cast<const uint32_t*>(xq_scale + tok * sbytes + b0)) : 0u;
+        const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(xq_scale + tok * sbytes + b0));
         const int c = b0 >> 4, mm = (b0 >> 2) & 3;
         *reinterpret_cast<uint32_t*>(sfb + static_cast<size_t>(c) * kNvChunkScaleBytes + mm * 512 + 16 * (j & 31) +
                                      4 * (j >> 5)) = w;

@@ -23,6 +23,14 @@ def cpu_inputs(cfg: MoeConfig, seed: int = 0) -> Dict[str, torch.Tensor]:
     return make_inputs(cfg, seed)
 
 
+def dirty_workspace(prob) -> torch.Tensor:
+    """A workspace whose every byte is 0xFF (NaN as bf16, fp16, fp32, e4m3 and E8M0): the
+    forward must read nothing it has not written (X padding rows are never written)."""
+    ws = moe.new_workspace(prob)
+    ws.fill_(0xFF)
+    return ws
+
+
 class GpuForward:
     """One forward of ``cfg`` on cuda:0 with every intermediate kept in the workspace."""
 
@@ -48,7 +56,7 @@ class GpuForward:
         else:
             self.w13p, self.w2p = moe.prepare_weights(self.prob, w13, w2, cfg.I)
         del w13, w2
-        self.ws = moe.new_workspace(self.prob)
+        self.ws = dirty_workspace(self.prob)
         self.out = torch.empty_like(self.hidden)
 
     def forward(self) -> torch.Tensor:

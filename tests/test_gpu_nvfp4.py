@@ -18,7 +18,8 @@ import mixture_experts_expert_topk_b200 as moe
 from mixture_experts_expert_topk_b200.synth import CONFIGS, MoeConfig, make_inputs
 from oracle import moe_oracle as O
 
-from _cases import (bf16_act_bound, bf16_to_f64, bits, check_act_pairs, cover_tokens, err_beyond_rounding,
+from _cases import (bf16_act_bound, bf16_to_f64, bits, check_act_pairs, cover_tokens, dirty_workspace,
+                    err_beyond_rounding,
                     max_err_over_rms, per_expert_threaded, untile_groups, untile_u8)
 
 pytestmark = pytest.mark.gpu
@@ -117,7 +118,7 @@ def _run(cfg, inp, s_act=None, experts=None, tokens=None):
                             activation=cfg.activation, num_shared=cfg.num_shared, fp8="nvfp4",
                             input_scale=s_in, activation_scale=s_act)
     w13p, w2p = moe.prepare_weights(prob, q13, q2, cfg.I, w13_scale=sc13, w2_scale=sc2)
-    ws = moe.new_workspace(prob)
+    ws = dirty_workspace(prob)
     out = moe.moe_forward(inp["hidden"].to(dev), inp["logits"].to(dev), w13p, w2p, cfg.topk, cfg.renormalize,
                           cfg.activation, g13, g2, num_shared=cfg.num_shared, workspace=ws, input_scale=s_in,
                           activation_scale=s_act)
@@ -153,7 +154,6 @@ def _check(cfg, inp, r, oracle_w, tokens=None):
     KC1 = cfg.H // 256
     xs = untile_u8(parts["xs"], gi, ng, P_pad, KC1)
     np.testing.assert_array_equal(xs[real], pack(hq)[pids[real] // kk])
-    assert np.all(xs[~real] == 0)
     xss = group_scales(parts["xs_scale"], gi, ng, P_pad, KC1)
     np.testing.assert_array_equal(xss[real], hs[pids[real] // kk])
     # GEMM2's input: the kernel's own bf16 activation quantised with the activation scale
