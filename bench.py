@@ -257,7 +257,12 @@ def run_ours(cfg: MoeConfig, steps: int, warmup: int, world: int, rank: int, loc
     clocks = clk.summary()
 
     # per-kernel breakdown: the same kernels through the per-step entry points, events
-    # between the steps on the launching stream
+    # between the steps on the launching stream, launched without programmatic dependent
+    # launch (with it a kernel may start before the previous one ends, across the events), so
+    # each step is timed whole and alone
+    sprob = moe.make_problem(cfg.T, cfg.H, cfg.E, cfg.topk, I_pad, renormalize=cfg.renormalize,
+                             activation=cfg.activation, num_shared=cfg.num_shared, fp8=cfg.fp8,
+                             input_scale=s_in, activation_scale=cfg.activation_scale, pdl=False)
     names = ["route", "align"] + (["quant_act"] if cfg.block128 else []) + ["permute", "gemm1", "gemm2", "combine"]
     per = {n: [] for n in names}
     for _ in range(steps):
@@ -265,14 +270,14 @@ def run_ours(cfg: MoeConfig, steps: int, warmup: int, world: int, rank: int, loc
         evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
         evs[0].record(stream)
         k = 0
-        moe.stage_route(prob, logits, ws); k += 1; evs[k].record(stream)
-        moe.stage_align(prob, ws); k += 1; evs[k].record(stream)
+        moe.stage_route(sprob, logits, ws); k += 1; evs[k].record(stream)
+        moe.stage_align(sprob, ws); k += 1; evs[k].record(stream)
         if cfg.block128:
-            moe.stage_quant_act(prob, hidden, ws); k += 1; evs[k].record(stream)
-        moe.stage_permute(prob, hidden, ws); k += 1; evs[k].record(stream)
-        moe.stage_gemm1(prob, hidden, w13p, ws, s13); k += 1; evs[k].record(stream)
-        moe.stage_gemm2(prob, w2p, ws, s2); k += 1; evs[k].record(stream)
-        moe.stage_combine(prob, out, ws); k += 1; evs[k].record(stream)
+            moe.stage_quant_act(sprob, hidden, ws); k += 1; evs[k].record(stream)
+        moe.stage_permute(sprob, hidden, ws); k += 1; evs[k].record(stream)
+        moe.stage_gemm1(sprob, hidden, w13p, ws, s13); k += 1; evs[k].record(stream)
+        moe.stage_gemm2(sprob, w2p, ws, s2); k += 1; evs[k].record(stream)
+        moe.stage_combine(sprob, out, ws); k += 1; evs[k].record(stream)
         torch.cuda.synchronize(dev)
         for i, n in enumerate(names):
             per[n].append(evs[i].elapsed_time(evs[i + 1]))
