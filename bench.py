@@ -42,7 +42,7 @@ L2_FLUSH_BYTES = 512 << 20
 # (dram__bytes_read.sum + dram__bytes_write.sum of the GEMM1 launch on the 64-expert
 # prefill case), valid only for the kernel source it was taken on (sha256 prefix of the
 # file below); None until such a capture exists for that source.
-GEMM1_TRAFFIC = {"source": "gemm_swap.cu", "source_sha256": "0a5e6afb0085", "ratio": 308.84 / 281.02}
+GEMM1_TRAFFIC = {"source": "gemm_swap.cu", "source_sha256": "1f5867c77b7c", "ratio": 308.59 / 281.02}
 
 
 def _peaks():
@@ -265,6 +265,21 @@ def run_ours(cfg: MoeConfig, steps: int, warmup: int, world: int, rank: int, loc
                              input_scale=s_in, activation_scale=cfg.activation_scale, pdl=False)
     names = ["route", "align"] + (["quant_act"] if cfg.block128 else []) + ["permute", "gemm1", "gemm2", "combine"]
     per = {n: [] for n in names}
+
+    def stages():
+        moe.stage_route(sprob, logits, ws)
+        moe.stage_align(sprob, ws)
+        if cfg.block128:
+            moe.stage_quant_act(sprob, hidden, ws)
+        moe.stage_permute(sprob, hidden, ws)
+        moe.stage_gemm1(sprob, hidden, w13p, ws, s13)
+        moe.stage_gemm2(sprob, w2p, ws, s2)
+        moe.stage_combine(sprob, out, ws)
+
+    # one untimed pass first: small batches' forwards fuse routing, align and permute into
+    # one kernel, so the separate kernels load (lazily) on their first launch here
+    stages()
+    torch.cuda.synchronize(dev)
     for _ in range(steps):
         flush.zero_()
         evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]

@@ -179,8 +179,11 @@ typedef struct {
   size_t xs_scale;        /* MXFP8: E8M0 scale bytes of xs: per row group, 1024 bytes per
                              128 columns at ((first row / 16) * H/128 + chunk) * 1024 */
   size_t group_info;      /* int32 pairs [max_rows/16 + 1]: row groups {first row, expert |
-                             rows << 16} of the GEMMs (block_m 16); the count is the second
-                             int32 of the num_blocks region */
+                             rows << 16 | padding rows << 25} of the GEMMs (block_m 16): rows
+                             a multiple of 16 (at most 256); the padding rows (fewer than 16,
+                             the sentinels of an expert's segment) are the last rows of the
+                             expert's last group; the count is the second int32 of the
+                             num_blocks region */
   size_t io_hidden;       /* staging for moe_forward_host: bf16 [T, H] */
   size_t io_logits;       /* staging for moe_forward_host: fp32 [T, E_r] */
   size_t io_out;          /* staging for moe_forward_host: bf16 [T, H] */

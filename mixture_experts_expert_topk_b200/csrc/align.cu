@@ -133,8 +133,10 @@ __device__ __forceinline__ int num_groups_of(int padded, int group_rows) {
   return group_rows > 0 && padded > 0 ? (padded + group_rows - 1) / group_rows : 0;
 }
 
-// Row groups of expert e's padded segment [off, off + padded), written from index g0.
-__device__ __forceinline__ void write_groups(int e, int off, int padded, int group_rows, int g0, int2* group_info) {
+// Row groups of expert e's padded segment [off, off + padded) holding `count` pairs, written
+// from index g0; the last group carries the segment's padding rows.
+__device__ __forceinline__ void write_groups(int e, int off, int count, int padded, int group_rows, int g0,
+                                             int2* group_info) {
   const int ng = num_groups_of(padded, group_rows);
   if (ng == 0) return;
   const int blocks = padded / 16;
@@ -142,7 +144,7 @@ __device__ __forceinline__ void write_groups(int e, int off, int padded, int gro
   int row = off;
   for (int i = 0; i < ng; ++i) {
     const int rows = 16 * (base + (i < extra ? 1 : 0));
-    group_info[g0 + i] = make_int2(row, e | (rows << 16));
+    group_info[g0 + i] = make_int2(row, group_word(e, rows, i == ng - 1 ? padded - count : 0));
     row += rows;
   }
 }
@@ -203,7 +205,7 @@ __global__ void __launch_bounds__(kScanThreads)
   }
   int gtotal = 0;
   const int g0 = block_exclusive_scan(e < E ? num_groups_of(padded, group_rows) : 0, warp_sums, &gtotal);
-  if (e < E) write_groups(e, off, padded, group_rows, g0, group_info);
+  if (e < E) write_groups(e, off, count, padded, group_rows, g0, group_info);
   if (threadIdx.x == 0) {
     expert_offsets[E] = total;
     num_blocks[0] = total / block_m;
@@ -292,7 +294,7 @@ __device__ __forceinline__ void align_single_cta(AlignSingleSmem& sm, const int*
     }
     int gtotal = 0;
     const int g0 = gcarry + block_exclusive_scan(x < E ? num_groups_of(padded, group_rows) : 0, warp_sums, &gtotal);
-    if (x < E) write_groups(x, off, padded, group_rows, g0, group_info);
+    if (x < E) write_groups(x, off, count, padded, group_rows, g0, group_info);
     carry += total;
     gcarry += gtotal;
   }
@@ -360,7 +362,7 @@ __global__ void __launch_bounds__(kWarps * 32)
       if (__ldcg(&group_info[mid].x) <= pos) lo = mid; else hi = mid - 1;
     }
     const int2 gi = __ldcg(group_info + lo);
-    const int n = gi.y >> 16, j = pos - gi.x;
+    const int n = group_word_rows(gi.y), j = pos - gi.x;
     const uint4* src = reinterpret_cast<const uint4*>(hidden + static_cast<size_t>(p / (topk + num_shared)) * hidden_row_bytes);
     uint8_t* base = xs + static_cast<size_t>(gi.x) * hidden_row_bytes;
     for (int q = lane; q < pieces; q += 32) {

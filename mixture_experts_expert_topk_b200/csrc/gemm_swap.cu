@@ -357,17 +357,18 @@ __global__ void __launch_bounds__(threads_for<kKind>(), 1) gemm_swap_kernel(cons
       bool ok = true;
       while (ok) {
         if (!mbar_wait(rempty0 + 8 * wslot, wph ^ 1u, abort_flag, a.status, kSiteTileEmpty)) break;
-        int x_row = 0, n = 0, e = 0, mt = 0;
+        int x_row = 0, n = 0, e = 0, mt = 0, n_real = 0;
         if (tile < num_tiles) {
           const int g = tile / a.m_tiles;
           mt = tile - g * a.m_tiles;
           const int2 gi = a.group_info[g];
           x_row = gi.x;
-          n = gi.y >> 16;
-          e = gi.y & 0xffff;
+          n = group_word_rows(gi.y);
+          e = group_word_expert(gi.y);
+          n_real = n - group_word_pad(gi.y);  // the group's padding rows are its last
         }
         ring[4 * wslot + 0] = x_row;
-        ring[4 * wslot + 1] = n;  // 0 tells the readers to stop
+        ring[4 * wslot + 1] = n | (n_real << 16);  // the group's real rows beside n; n == 0: stop
         ring[4 * wslot + 2] = e;
         ring[4 * wslot + 3] = mt;
         mbar_arrive(rfull0 + 8 * wslot);  // release: the entry is visible to its readers
@@ -412,7 +413,7 @@ __global__ void __launch_bounds__(threads_for<kKind>(), 1) gemm_swap_kernel(cons
       while (ok) {
         int4 t;
         if (!ring_read(rfull0, rempty0, ring, rslot, rph, abort_flag, a.status, t) || t.y == 0) break;
-        const int x_row = t.x, n = t.y;
+        const int x_row = t.x, n = t.y & 0xffff;
         const int kc = step_chunks<kKind>(n);
         const uint8_t* xsrc = a.x + static_cast<size_t>(x_row) * x_row_bytes;
         for (int c0 = 0; c0 < a.k_chunks; c0 += kc, ++ks) {
@@ -458,7 +459,7 @@ __global__ void __launch_bounds__(threads_for<kKind>(), 1) gemm_swap_kernel(cons
       while (true) {
         int4 t;
         if (!ring_read(rfull0, rempty0, ring, rslot, rph, abort_flag, a.status, t) || t.y == 0) break;
-        const int n = t.y;
+        const int n = t.y & 0xffff;
         const int kc = step_chunks<kKind>(n);
         const int acc = it & 1;
         if (!kB128 && !mbar_wait(tempty0 + 8 * acc, ((it >> 1) & 1) ^ 1u, abort_flag, a.status, kSiteTmemEmpty)) break;
@@ -583,19 +584,12 @@ __global__ void __launch_bounds__(threads_for<kKind>(), 1) gemm_swap_kernel(cons
       int ok = 0;
       if (lane == 0) ok = ring_read(rfull0, rempty0, ring, rslot, rph, abort_flag, a.status, t);
       ok = __shfl_sync(0xffffffffu, ok, 0);
-      const int n = __shfl_sync(0xffffffffu, t.y, 0);
+      const int ny = __shfl_sync(0xffffffffu, t.y, 0);
+      const int n = ny & 0xffff, n_real = ny >> 16;  // GEMM1: the group's rows that are not padding
       if (!ok || n == 0) break;
       const int x_row = __shfl_sync(0xffffffffu, t.x, 0);
       const int expert = __shfl_sync(0xffffffffu, t.z, 0);
       const int mt = __shfl_sync(0xffffffffu, t.w, 0);
-      // GEMM1: a group's padding rows (pair id P) are a suffix of fewer than 16 rows (an
-      // expert's segment is its pairs, then sentinels up to a multiple of 16), so its real
-      // rows are n minus the sentinels among its last 16
-      int n_real = n;
-      if (a.mode == 0) {
-        const bool sentinel = lane < 16 && __ldg(a.sorted_pair_ids + x_row + n - 16 + lane) >= a.num_pairs;
-        n_real = n - __popc(__ballot_sync(0xffffffffu, sentinel));
-      }
       // FP8 per-tensor, NVFP4: the accumulator's dequantisation scale (the weight's and the
       // X operand's tensor scales; GEMM1: before the activation)
       const float dq = (kFp8 || kNv) ? __ldg(a.w_scale + expert) * a.in_scale : 1.0f;
@@ -633,42 +627,54 @@ __global__ void __launch_bounds__(threads_for<kKind>(), 1) gemm_swap_kernel(cons
           }
           if (lane < 16 || full)
             a.y_exp[static_cast<size_t>(x_row + c0 + lane) * (a.out_cols >> 5) + (col >> 5)] = static_cast<int8_t>(s);
-        } else {
-          // GEMM1: a group's padding rows store zeros whatever X held there (the permute does
-          // not write them), so GEMM2 sees zero rows
-          if (!gated) {
+        } else if (!gated) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              if (j == 16 && !full) break;
-              const int row = c0 + j;
-              const float z = row >= n_real ? 0.f : fmaxf(__uint_as_float(v[j]) * dq, 0.f);
+          for (int j = 0; j < 32; ++j) {
+            if (j == 16 && !full) break;
+            const int row = c0 + j;
+            const float z = fmaxf(__uint_as_float(v[j]) * dq, 0.f);
+            uint8_t* dst = act_grp + row * kChunkBytes + ((((fo >> 4) ^ row) & 7) << 4) + (fo & 15);
+            if (kFp8)
+              *dst = __nv_cvt_float_to_fp8(z * z * a.act_inv, __NV_SATFINITE, __NV_E4M3);
+            else
+              *reinterpret_cast<__nv_bfloat16*>(dst) = __float2bfloat16_rn(z * z);
+          }
+        } else {
+          // lane pair (2m, 2m+1) = (gate, up) of feature m. The even lane finishes tokens
+          // 0..15 of the batch, the odd lane tokens 16..31: each passes the other the half
+          // it needs, so every lane evaluates the activation on 16 tokens.
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float mine_lo = __uint_as_float(v[j]) * dq;       // even: gate_j; odd: up_j
+            const float mine_hi = __uint_as_float(v[16 + j]) * dq;  // even: gate_{16+j}; odd: up_{16+j}
+            const float other = __shfl_xor_sync(0xffffffffu, odd ? mine_lo : mine_hi, 1);
+            const float g = odd ? other : mine_lo;
+            const float u = odd ? mine_hi : other;
+            const int row = c0 + (odd ? 16 + j : j);
+            if (!odd || full) {
+              const float h = gated_act(g, u, a.activation);
               uint8_t* dst = act_grp + row * kChunkBytes + ((((fo >> 4) ^ row) & 7) << 4) + (fo & 15);
               if (kFp8)
-                *dst = __nv_cvt_float_to_fp8(z * z * a.act_inv, __NV_SATFINITE, __NV_E4M3);
+                *dst = __nv_cvt_float_to_fp8(h * a.act_inv, __NV_SATFINITE, __NV_E4M3);
               else
-                *reinterpret_cast<__nv_bfloat16*>(dst) = __float2bfloat16_rn(z * z);
+                *reinterpret_cast<__nv_bfloat16*>(dst) = __float2bfloat16_rn(h);
             }
-          } else {
-            // lane pair (2m, 2m+1) = (gate, up) of feature m. The even lane finishes tokens
-            // 0..15 of the batch, the odd lane tokens 16..31: each passes the other the half
-            // it needs, so every lane evaluates the activation on 16 tokens.
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const float mine_lo = __uint_as_float(v[j]) * dq;       // even: gate_j; odd: up_j
-              const float mine_hi = __uint_as_float(v[16 + j]) * dq;  // even: gate_{16+j}; odd: up_{16+j}
-              const float other = __shfl_xor_sync(0xffffffffu, odd ? mine_lo : mine_hi, 1);
-              const float g = odd ? other : mine_lo;
-              const float u = odd ? mine_hi : other;
-              const int row = c0 + (odd ? 16 + j : j);
-              if (!odd || full) {
-                const float h = row >= n_real ? 0.f : gated_act(g, u, a.activation);
-                uint8_t* dst = act_grp + row * kChunkBytes + ((((fo >> 4) ^ row) & 7) << 4) + (fo & 15);
-                if (kFp8)
-                  *dst = __nv_cvt_float_to_fp8(h * a.act_inv, __NV_SATFINITE, __NV_E4M3);
-                else
-                  *reinterpret_cast<__nv_bfloat16*>(dst) = __float2bfloat16_rn(h);
-              }
-            }
+          }
+        }
+        // GEMM1: a group's padding rows (a suffix, from n_real on) hold whatever X held there
+        // (the permute does not write them); zeros over them, so GEMM2 sees zero rows. Only
+        // the block that holds them takes this branch (block-uniform), each thread rewriting
+        // the rows it stored above, in program order.
+        const int c1 = c0 + (full ? 32 : 16);
+        if (a.mode == 0 && c1 > n_real) {
+          const int r0 = gated ? c0 + (odd ? 16 : 0) : c0;
+          const int r1 = gated ? (odd ? (full ? c1 : r0) : min(c1, c0 + 16)) : c1;
+          for (int row = max(r0, n_real); row < r1; ++row) {
+            uint8_t* dst = act_grp + row * kChunkBytes + ((((fo >> 4) ^ row) & 7) << 4) + (fo & 15);
+            if (kFp8)
+              *dst = 0;
+            else
+              *reinterpret_cast<__nv_bfloat16*>(dst) = __float2bfloat16_rn(0.f);
           }
         }
       };

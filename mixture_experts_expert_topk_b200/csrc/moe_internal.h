@@ -10,6 +10,13 @@ namespace moe {
 constexpr int kMaxExperts = 1024;  // routed + shared
 constexpr int kMaxSlots = 16;      // k' = topk + num_shared
 constexpr int kAlignChunk = 2048;  // pairs per align chunk
+// A row group's second int32 (group_info[g].y): expert | rows << 16 | padding rows << 25. rows
+// is a multiple of 16, at most 256; the padding rows (sentinels, fewer than 16) are the
+// group's last rows and only an expert's last group has any.
+__host__ __device__ constexpr int group_word(int e, int rows, int pad) { return e | (rows << 16) | (pad << 25); }
+__host__ __device__ constexpr int group_word_rows(int y) { return (y >> 16) & 0x1ff; }
+__host__ __device__ constexpr int group_word_pad(int y) { return (y >> 25) & 0xf; }
+__host__ __device__ constexpr int group_word_expert(int y) { return y & 0xffff; }
 constexpr int kRouteAlignTokensPerWarp = 2;  // fused routing + align: tokens per warp (8 warps)
 constexpr int kFusedPermutePairs = 64;       // fused routing + align also permutes (bf16) up to this many pairs
 // Status word value (beyond the wait timeouts 0x10000 | site): caller-supplied routing held

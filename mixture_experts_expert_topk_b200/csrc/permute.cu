@@ -36,7 +36,7 @@ __global__ void __launch_bounds__(kThreads)
   // CTA (x, y) copies rows [kRowsPerCta * y, kRowsPerCta * (y + 1)) of groups x, x + gridDim.x, ...
   for (int g = blockIdx.x; g < G; g += gridDim.x) {
     const int2 gi = group_info[g];
-    const int x_row = gi.x, n = gi.y >> 16;
+    const int x_row = gi.x, n = group_word_rows(gi.y);
     uint8_t* base = xs + static_cast<size_t>(x_row) * row_pieces * 16;
     for (int j0 = kRowsPerCta * blockIdx.y + kRowsPerStep * warp; j0 < min(n, kRowsPerCta * (blockIdx.y + 1));
          j0 += kRowsPerStep * (kThreads / 32)) {
@@ -94,7 +94,7 @@ __global__ void __launch_bounds__(kThreads)
   const int pieces = H / 16;  // 16 elements: 32 bytes in, 16 bytes out
   for (int g = blockIdx.x; g < G; g += gridDim.x) {
     const int2 gi = group_info[g];
-    const int x_row = gi.x, n = gi.y >> 16;
+    const int x_row = gi.x, n = group_word_rows(gi.y);
     uint8_t* base = xs + static_cast<size_t>(x_row) * H;
     for (int j0 = kRowsPerCta * blockIdx.y + kRowsPerStep * warp; j0 < min(n, kRowsPerCta * (blockIdx.y + 1));
          j0 += kRowsPerStep * (kThreads / 32)) {
@@ -164,7 +164,7 @@ __global__ void __launch_bounds__(kThreads)
   const int pieces = H / 16, KC = H / 128;
   for (int g = blockIdx.x; g < G; g += gridDim.x) {
     const int2 gi = group_info[g];
-    const int x_row = gi.x, n = gi.y >> 16;
+    const int x_row = gi.x, n = group_word_rows(gi.y);
     uint8_t* base = xs + static_cast<size_t>(x_row) * H;
     uint8_t* sf = xs_sf + static_cast<size_t>(x_row >> 4) * KC * 1024;
     for (int j0 = kRowsPerCta * blockIdx.y + kRowsPerStep * warp; j0 < min(n, kRowsPerCta * (blockIdx.y + 1));
@@ -243,7 +243,7 @@ __global__ void __launch_bounds__(kThreads)
   const int ob = 4 * lane;         // byte of the e4m3 chunk row
   for (int g = blockIdx.x; g < G; g += gridDim.x) {
     const int2 gi = group_info[g];
-    const int x_row = gi.x, n = gi.y >> 16;
+    const int x_row = gi.x, n = group_word_rows(gi.y);
     const uint8_t* in = act + static_cast<size_t>(x_row) * KCb * 128;
     uint8_t* out = actq + static_cast<size_t>(x_row) * KCq * 128;
     uint8_t* sf = act_sf + static_cast<size_t>(x_row >> 4) * KCq * 1024;
@@ -322,7 +322,7 @@ __global__ void __launch_bounds__(kThreads)
   const int KC = H / 128, pieces = H / 16;
   for (int g = blockIdx.x; g < G; g += gridDim.x) {
     const int2 gi = group_info[g];
-    const int x_row = gi.x, n = gi.y >> 16;
+    const int x_row = gi.x, n = group_word_rows(gi.y);
     uint8_t* base = xs + static_cast<size_t>(x_row) * KC * kB128RowBytesPerChunk;
     for (int j = blockIdx.y * (kThreads / 32) + warp; j < n; j += gridDim.y * (kThreads / 32)) {
       const int pid = sorted_pair_ids[x_row + j];
@@ -368,7 +368,7 @@ __global__ void __launch_bounds__(kThreads)
   const int KCb = I / 64, KC = I / 128;
   for (int g = blockIdx.x; g < G; g += gridDim.x) {
     const int2 gi = group_info[g];
-    const int x_row = gi.x, n = gi.y >> 16;
+    const int x_row = gi.x, n = group_word_rows(gi.y);
     const uint8_t* in = act + static_cast<size_t>(x_row) * KCb * 128;
     uint8_t* base = actq + static_cast<size_t>(x_row) * KC * kB128RowBytesPerChunk;
     for (int j = blockIdx.y * (kThreads / 32) + warp; j < n; j += gridDim.y * (kThreads / 32)) {
@@ -420,7 +420,7 @@ __global__ void __launch_bounds__(kThreads)
   const int KC = H / 256, pieces = H / 32, sbytes = H / 16;
   for (int g = blockIdx.x; g < G; g += gridDim.x) {
     const int2 gi = group_info[g];
-    const int x_row = gi.x, n = gi.y >> 16;
+    const int x_row = gi.x, n = group_word_rows(gi.y);
     uint8_t* base = xs + static_cast<size_t>(x_row) * KC * 128;
     uint8_t* sfb = xs_sf + static_cast<size_t>(x_row >> 4) * KC * kNvChunkScaleBytes;
     for (int j = blockIdx.y * (kThreads / 32) + warp; j < n; j += gridDim.y * (kThreads / 32)) {
@@ -469,7 +469,7 @@ __global__ void __launch_bounds__(kThreads)
   const int ob = 4 * lane;         // byte of the code chunk row
   for (int gr = blockIdx.x; gr < G; gr += gridDim.x) {
     const int2 gi = group_info[gr];
-    const int x_row = gi.x, n = gi.y >> 16;
+    const int x_row = gi.x, n = group_word_rows(gi.y);
     const uint8_t* in = act + static_cast<size_t>(x_row) * KCb * 128;
     uint8_t* out = actq + static_cast<size_t>(x_row) * KC * 128;
     uint8_t* sf = act_sf + static_cast<size_t>(x_row >> 4) * KC * kNvChunkScaleBytes;

@@ -141,7 +141,7 @@ def untile_groups(flat_bits: np.ndarray, group_info: np.ndarray, num_groups: int
     out = np.zeros((rows, 64 * kchunks), dtype=flat.dtype)
     for g in range(num_groups):
         x_row, meta = int(group_info[g][0]), int(group_info[g][1])
-        n = meta >> 16
+        n = (meta >> 16) & 0x1FF  # rows (bits 16-24; padding count above)
         base = x_row * 64 * kchunks
         grp = flat[base:base + n * 64 * kchunks].reshape(kchunks, n, 8, 8)
         j = np.arange(n)
@@ -275,7 +275,7 @@ def untile_u8(flat, group_info, num_groups, rows, kchunks):
     out = np.zeros((rows, 128 * kchunks), dtype=np.uint8)
     for g in range(num_groups):
         x_row, meta = int(group_info[g][0]), int(group_info[g][1])
-        n = meta >> 16
+        n = (meta >> 16) & 0x1FF  # rows (bits 16-24; padding count above)
         grp = flat[x_row * 128 * kchunks:(x_row + n) * 128 * kchunks].reshape(kchunks, n, 8, 16)
         j = np.arange(n)
         phys = np.arange(8)[None, :] ^ (j[:, None] & 7)
@@ -295,7 +295,7 @@ def untile_b128(flat, group_info, num_groups, rows, kchunks):
     scales = np.zeros((rows, kchunks), dtype=np.float32)
     for g in range(num_groups):
         x_row, meta = int(group_info[g][0]), int(group_info[g][1])
-        n = meta >> 16
+        n = (meta >> 16) & 0x1FF  # rows (bits 16-24; padding count above)
         kc = 4 if n <= 32 else (3 if n <= 64 else (2 if n <= 128 else 1))
         base = x_row * kchunks * 132
         j = np.arange(n)

@@ -85,7 +85,8 @@ def _check_route_align(cfg, parts, logits, bm=None):
 def _check_groups(cfg, parts, a):
     """Row groups of the swapped-operand GEMMs: each expert's padded segment cut into
     ceil(rows / G) groups of whole 16-row blocks, sizes as even as possible, larger first
-    (G = 256; 128 for FP8 block-128); and, for bf16, the permuted hidden rows."""
+    (G = 256; 128 for FP8 block-128), the word expert | rows << 16 | padding << 25 (the
+    segment's padding rows, all in its last group); and, for bf16, the permuted hidden rows."""
     P = cfg.T * cfg.k_total
     G = 128 if cfg.block128 else 256
     off = a["expert_offsets"]
@@ -94,13 +95,15 @@ def _check_groups(cfg, parts, a):
         seg = int(off[e + 1] - off[e])
         if seg == 0:
             continue
+        count = int(np.sum(a["sorted_pair_ids"][int(off[e]):int(off[e + 1])] < P))
+        assert 0 <= seg - count < 16
         ng = -(-seg // G)
         base, extra = divmod(seg // 16, ng)
         row = int(off[e])
         for i in range(ng):
             n = 16 * (base + (1 if i < extra else 0))
             assert 16 <= n <= G
-            expect.append((row, e | (n << 16)))
+            expect.append((row, e | (n << 16) | ((seg - count if i == ng - 1 else 0) << 25)))
             row += n
         assert row == off[e + 1]
     assert int(parts["num_blocks"][1]) == len(expect)
@@ -639,7 +642,7 @@ def _mx_group_scales(sf_flat, group_info, num_groups, rows, kchunks):
     out = np.zeros((rows, 4 * kchunks), dtype=np.uint8)
     for g in range(num_groups):
         x_row, meta = int(group_info[g][0]), int(group_info[g][1])
-        n = meta >> 16
+        n = (meta >> 16) & 0x1FF
         for r in range(n):
             for c in range(kchunks):
                 base = ((x_row // 16) * kchunks + c) * 1024 + (r // 128) * 512 + (r % 32) * 16 + ((r // 32) % 4) * 4
@@ -714,7 +717,7 @@ def _mx_parity(cfg, inp, name):
     np.testing.assert_array_equal(parts["sorted_pair_ids"][:P_pad], al["sorted_pair_ids"])
     ng = int(parts["num_blocks"][1])
     gi = parts["group_info"]
-    assert max(int(gi[g][1]) >> 16 for g in range(ng)) <= 192
+    assert max((int(gi[g][1]) >> 16) & 0x1FF for g in range(ng)) <= 192
     # the permuted hidden rows: MXFP8 codes and scale bytes, bit for bit
     pids = al["sorted_pair_ids"][:P_pad]
     real = pids < cfg.T * cfg.k_total
