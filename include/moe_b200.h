@@ -175,7 +175,8 @@ typedef struct {
   size_t xs;              /* block_m 16: the hidden rows of every row group in row-group order
                              (bf16; e4m3 codes for the 8-bit formats; FP8 block-128: each K
                              step's e4m3 codes followed by its rows' fp32 1x128 scales, 132
-                             bytes per row per 128 columns); size 0 otherwise */
+                             bytes per row per 128 columns); the padding rows are not written
+                             (GEMM1 stores zero activation rows for them); size 0 otherwise */
   size_t xs_scale;        /* MXFP8: E8M0 scale bytes of xs: per row group, 1024 bytes per
                              128 columns at ((first row / 16) * H/128 + chunk) * 1024 */
   size_t group_info;      /* int32 pairs [max_rows/16 + 1]: row groups {first row, expert |
