@@ -23,6 +23,17 @@ def cpu_inputs(cfg: MoeConfig, seed: int = 0) -> Dict[str, torch.Tensor]:
     return make_inputs(cfg, seed)
 
 
+# Parity figures reported by the GPU tests (one line per configuration), printed again in the
+# session's terminal summary (conftest.py) so that a quiet run still shows them.
+PARITY_REPORT: list = []
+
+
+def report(line: str) -> None:
+    """Print a parity figure and keep it for the session summary."""
+    print(line)
+    PARITY_REPORT.append(line)
+
+
 def dirty_workspace(prob) -> torch.Tensor:
     """A workspace whose every byte is 0xFF (NaN as bf16, fp16, fp32, e4m3 and E8M0): the
     forward must read nothing it has not written (X padding rows are never written)."""

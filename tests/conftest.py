@@ -27,3 +27,13 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    # the parity figures the GPU tests reported (tests/_cases.py: report), one per line
+    mod = sys.modules.get("_cases")
+    lines = getattr(mod, "PARITY_REPORT", None) if mod is not None else None
+    if lines:
+        terminalreporter.section("parity against the oracle: beyond-rounding and raw max|err|/RMS")
+        for line in lines:
+            terminalreporter.write_line(line)

@@ -14,7 +14,7 @@ from mixture_experts_expert_topk_b200 import ep
 from mixture_experts_expert_topk_b200.synth import MoeConfig, make_inputs
 from oracle import moe_oracle as O
 
-from _cases import bits, err_beyond_rounding
+from _cases import bits, err_beyond_rounding, report
 
 pytestmark = pytest.mark.gpu
 
@@ -100,5 +100,5 @@ def test_ep_forward_one_rank_matches_oracle(shared, act):
     ref = O.moe_forward(bits(inp["hidden"]), inp["logits"].numpy(), bits(inp["w13"]), bits(inp["w2"]), topk=cfg.topk,
                         renormalize=cfg.renormalize, activation=act, num_shared=shared)
     e = err_beyond_rounding(out.cpu().float().numpy().astype(np.float64), ref)
-    print(f"ep one rank {act} shared={shared}: beyond-rounding {e:.4f}")
+    report(f"ep one rank {act} shared={shared}: beyond-rounding {e:.4f}")
     assert e <= 2e-2, e

@@ -19,8 +19,8 @@ from mixture_experts_expert_topk_b200.synth import CONFIGS, MoeConfig, make_inpu
 from oracle import moe_oracle as O
 
 from _cases import (bf16_act_bound, bf16_to_f64, bits, check_act_pairs, cover_tokens, dirty_workspace,
-                    err_beyond_rounding,
-                    max_err_over_rms, per_expert_threaded, untile_groups, untile_u8)
+                    err_beyond_rounding, max_err_over_rms, per_expert_threaded, report, untile_groups,
+                    untile_u8)
 
 pytestmark = pytest.mark.gpu
 
@@ -175,7 +175,7 @@ def _check(cfg, inp, r, oracle_w, tokens=None):
     got = bf16_to_f64(r["out"].cpu()[torch.from_numpy(toks)])
     assert np.all(np.isfinite(got))
     e = err_beyond_rounding(got, ref)
-    print(f"{cfg.name}: {len(toks)} tokens, {n_act} activation values; beyond-rounding {e:.4f}, "
+    report(f"{cfg.name}: {len(toks)} tokens, {n_act} activation values; beyond-rounding {e:.4f}, "
           f"raw {max_err_over_rms(got, ref):.4f}")
     assert e <= TOL, e
 

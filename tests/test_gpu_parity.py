@@ -18,9 +18,10 @@ import mixture_experts_expert_topk_b200 as moe
 from mixture_experts_expert_topk_b200.synth import CONFIGS, MoeConfig, make_inputs
 from oracle import moe_oracle as O
 
-from _cases import (GpuForward, act_rows_f64, dirty_workspace, bf16_act_bound, bf16_to_f64, bits, check_act_pairs, cover_tokens,
-                    cpu_inputs, err_beyond_rounding, max_err_over_rms, oracle_fp8_block_weights, oracle_mxfp8_weights,
-                    oracle_out, untile_b128, untile_groups, untile_u8, untile_weights)
+from _cases import (act_rows_f64, bf16_act_bound, bf16_to_f64, bits, check_act_pairs, cover_tokens,
+                    cpu_inputs, dirty_workspace, err_beyond_rounding, GpuForward, max_err_over_rms,
+                    oracle_fp8_block_weights, oracle_mxfp8_weights, oracle_out, report, untile_b128,
+                    untile_groups, untile_u8, untile_weights)
 
 pytestmark = pytest.mark.gpu
 
@@ -168,7 +169,7 @@ def test_layer_parity_small(name, bm):
     got = bf16_to_f64(out)
     assert np.all(np.isfinite(got))
     e = err_beyond_rounding(got, ref)
-    print(f"{name}: beyond-rounding {e:.4f}, raw max|err|/RMS {max_err_over_rms(got, ref):.4f}")
+    report(f"{name}: beyond-rounding {e:.4f}, raw max|err|/RMS {max_err_over_rms(got, ref):.4f}")
     assert e <= BF16_TOL, e
     st, word = moe.device_status(run.ws)
     assert st == 0 and word == 0
@@ -307,7 +308,7 @@ def _full_size(cfg, n_sample=48, seed=0):
     ref = oracle_out(cfg, run.inp, tokens=tokens, fp8_weights=fp8w)
     got = bf16_to_f64(out)[tokens]
     assert np.all(np.isfinite(bf16_to_f64(out)))
-    print(f"{cfg.name}: beyond-rounding {err_beyond_rounding(got, ref):.4f}, raw {max_err_over_rms(got, ref):.4f}")
+    report(f"{cfg.name}: beyond-rounding {err_beyond_rounding(got, ref):.4f}, raw {max_err_over_rms(got, ref):.4f}")
     return err_beyond_rounding(got, ref), run
 
 
@@ -328,7 +329,9 @@ def test_decode_full(T):
     parts = run.parts()
     _check_route_align(cfg, parts, run.inp["logits"])
     ref = oracle_out(cfg, run.inp)
-    assert err_beyond_rounding(bf16_to_f64(out), ref) <= BF16_TOL
+    got = bf16_to_f64(out)
+    report(f"{cfg.name}: beyond-rounding {err_beyond_rounding(got, ref):.4f}, raw {max_err_over_rms(got, ref):.4f}")
+    assert err_beyond_rounding(got, ref) <= BF16_TOL
 
 
 # ---- FP8 E4M3 W8A8 block-128 ---------------------------------------------------------
@@ -408,7 +411,7 @@ def test_fp8_layer_parity_small(name, bm):
     got = bf16_to_f64(out)
     assert np.all(np.isfinite(got))
     e = err_beyond_rounding(got, ref)
-    print(f"{name}/bm{parts['block_m']}: beyond-rounding {e:.4f}, raw {max_err_over_rms(got, ref):.4f}")
+    report(f"{name}/bm{parts['block_m']}: beyond-rounding {e:.4f}, raw {max_err_over_rms(got, ref):.4f}")
     assert e <= FP8_TOL, e
     assert moe.device_status(run.ws)[0] == 0
 
@@ -613,7 +616,7 @@ def test_fp8_per_tensor_layer_parity(name):
     got = bf16_to_f64(out)
     assert np.all(np.isfinite(got))
     e = err_beyond_rounding(got, ref)
-    print(f"{name}: beyond-rounding {e:.4f}, raw {max_err_over_rms(got, ref):.4f}")
+    report(f"{name}: beyond-rounding {e:.4f}, raw {max_err_over_rms(got, ref):.4f}")
     assert e <= FP8_TOL, e
 
 
@@ -737,7 +740,7 @@ def _mx_parity(cfg, inp, name):
     got = bf16_to_f64(out)
     assert np.all(np.isfinite(got))
     e = err_beyond_rounding(got, ref)
-    print(f"{name}: beyond-rounding {e:.4f}, raw {max_err_over_rms(got, ref):.4f}")
+    report(f"{name}: beyond-rounding {e:.4f}, raw {max_err_over_rms(got, ref):.4f}")
     assert e <= FP8_TOL, e
 
 
@@ -782,7 +785,7 @@ def test_mxfp8_full_size_every_expert():
                               renormalize=cfg.renormalize, activation=cfg.activation, tokens=tokens)
     got = bf16_to_f64(out.cpu()[torch.from_numpy(tokens)])
     e = err_beyond_rounding(got, ref)
-    print(f"mxfp8_prefill: {len(tokens)} tokens over {len(experts)} experts, {n} activation values; "
+    report(f"mxfp8_prefill: {len(tokens)} tokens over {len(experts)} experts, {n} activation values; "
           f"beyond-rounding {e:.4f}, raw {max_err_over_rms(got, ref):.4f}")
     assert e <= FP8_TOL, e
 
@@ -813,7 +816,7 @@ def test_fp8_block128_full_size_every_expert():
     got = bf16_to_f64(out)[tokens]
     assert np.all(np.isfinite(bf16_to_f64(out)))
     e = err_beyond_rounding(got, ref)
-    print(f"fp8_shared: {len(tokens)} tokens over {len(experts)} experts, {n} activation values; "
+    report(f"fp8_shared: {len(tokens)} tokens over {len(experts)} experts, {n} activation values; "
           f"beyond-rounding {e:.4f}, raw {max_err_over_rms(got, ref):.4f}")
     assert e <= FP8_TOL, e
     assert moe.device_status(run.ws)[0] == 0
@@ -886,6 +889,6 @@ def test_fp8_per_tensor_full_size_every_expert():
                                        num_shared=cfg.num_shared, tokens=tokens)
     got = bf16_to_f64(out.cpu()[torch.from_numpy(tokens)])
     e = err_beyond_rounding(got, ref)
-    print(f"fp8pt_shared: {len(tokens)} tokens, {n} activation codes; beyond-rounding {e:.4f}, "
+    report(f"fp8pt_shared: {len(tokens)} tokens, {n} activation codes; beyond-rounding {e:.4f}, "
           f"raw {max_err_over_rms(got, ref):.4f}")
     assert e <= FP8_TOL, e
